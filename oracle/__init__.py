@@ -1,0 +1,245 @@
+"""Plain fp64 CPU oracle for the Newton-solved diag-mix sLSTM.
+
+TEST INFRASTRUCTURE ONLY.  The product library never imports, links or calls
+anything here; only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` do.  The arithmetic
+lives in ``slstm_oracle.c`` (fp64, libm, one lane and one step at a time);
+this module compiles it with gcc on first use and marshals numpy arrays.
+
+Pins that tie the oracle to the pages and to mathematics (not to itself) are
+in ``tests/test_oracle_pins.py``.  Every function below is pinned; the oracle
+header in ``slstm_oracle.c`` lists the page sections each one follows.
+
+Layout conversions: the library boundary uses (B, T, 4, d_h) for P and S,
+(4, d_h) for R and bias, (B, 4, d_h) for s0, (B, T, d_h) for dH.  The C code
+works lane-major: one lane is one (b, j) pair.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "slstm_oracle.c")
+_SO = os.path.join(_HERE, "liboracle.so")
+
+FORGET_SIGMOID = 0
+FORGET_EXP = 1
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (no fast-math, IEEE fp64)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        tmp = _SO + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _SO)
+    return _SO
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_SO)
+        D = ctypes.POINTER(ctypes.c_double)
+        I = ctypes.c_int
+        IP = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_step.argtypes = [D, D, D, I, D, D, D]
+        lib.oracle_sequential.argtypes = [I, I, D, D, D, I, D]
+        lib.oracle_sequential_unstabilised.argtypes = [I, I, D, D, D, I, D, D, D]
+        lib.oracle_affine_solve.argtypes = [I, I, D, D, D, I, D]
+        lib.oracle_newton.argtypes = [I, I, D, D, D, I, I, I, ctypes.c_double, D, D, D, IP, IP, IP]
+        lib.oracle_bptt.argtypes = [I, I, D, D, D, D, D, I, D, D, D, D]
+        lib.oracle_gemm.argtypes = [I, I, I, D, I, D, I, D, D]
+        for f in ("oracle_step", "oracle_sequential", "oracle_sequential_unstabilised",
+                  "oracle_affine_solve", "oracle_newton", "oracle_bptt", "oracle_gemm"):
+            getattr(lib, f).restype = None
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _forget_code(forget) -> int:
+    if forget in (FORGET_SIGMOID, "sigmoid"):
+        return FORGET_SIGMOID
+    if forget in (FORGET_EXP, "exp"):
+        return FORGET_EXP
+    raise ValueError(f"unknown forget mode {forget!r}")
+
+
+# ----------------------------------------------------------------------------
+# layout helpers (boundary layout <-> lane-major)
+# ----------------------------------------------------------------------------
+def lanes_from_btgd(P: np.ndarray) -> np.ndarray:
+    """(B, T, 4, d) -> (B*d, T, 4), lane index = b*d + j."""
+    B, T, four, d = P.shape
+    assert four == 4
+    return _f64(np.transpose(P, (0, 3, 1, 2)).reshape(B * d, T, 4))
+
+
+def btgd_from_lanes(X: np.ndarray, B: int, d: int) -> np.ndarray:
+    """(B*d, T, 4) -> (B, T, 4, d)."""
+    T = X.shape[1]
+    return np.ascontiguousarray(np.transpose(X.reshape(B, d, T, 4), (0, 2, 3, 1)))
+
+
+def lanes_from_gd(R: np.ndarray, B: int) -> np.ndarray:
+    """(4, d) per-feature parameters -> (B*d, 4)."""
+    four, d = R.shape
+    return _f64(np.broadcast_to(np.transpose(R)[None], (B, d, 4)).reshape(B * d, 4))
+
+
+def lanes_from_bgd(s0: np.ndarray) -> np.ndarray:
+    """(B, 4, d) -> (B*d, 4)."""
+    B, four, d = s0.shape
+    return _f64(np.transpose(s0, (0, 2, 1)).reshape(B * d, 4))
+
+
+def bgd_from_lanes(X: np.ndarray, B: int, d: int) -> np.ndarray:
+    return np.ascontiguousarray(np.transpose(X.reshape(B, d, 4), (0, 2, 1)))
+
+
+# ----------------------------------------------------------------------------
+# lane-major entry points
+# ----------------------------------------------------------------------------
+def step(sp, p, r, forget="sigmoid"):
+    """One stabilised step; returns (s_t, J (4x4), G (4x4))."""
+    lib = _load()
+    sp, p, r = _f64(sp), _f64(p), _f64(r)
+    out = np.zeros(4)
+    J = np.zeros(16)
+    G = np.zeros(16)
+    lib.oracle_step(_ptr(sp), _ptr(p), _ptr(r), _forget_code(forget), _ptr(out), _ptr(J), _ptr(G))
+    return out, J.reshape(4, 4), G.reshape(4, 4)
+
+
+def sequential(P, R, s0, forget="sigmoid") -> np.ndarray:
+    """P (L,T,4), R (L,4), s0 (L,4) -> S (L,T,4) by stepping through time."""
+    lib = _load()
+    P, R, s0 = _f64(P), _f64(R), _f64(s0)
+    L, T, _ = P.shape
+    S = np.zeros((L, T, 4))
+    lib.oracle_sequential(L, T, _ptr(P), _ptr(R), _ptr(s0), _forget_code(forget), _ptr(S))
+    return S
+
+
+def sequential_unstabilised(P, R, s0, forget="sigmoid"):
+    """Unstabilised recurrence; returns (c_u, n_u, h), each (L, T)."""
+    lib = _load()
+    P, R, s0 = _f64(P), _f64(R), _f64(s0)
+    L, T, _ = P.shape
+    cu, nu, h = np.zeros((L, T)), np.zeros((L, T)), np.zeros((L, T))
+    lib.oracle_sequential_unstabilised(L, T, _ptr(P), _ptr(R), _ptr(s0), _forget_code(forget),
+                                       _ptr(cu), _ptr(nu), _ptr(h))
+    return cu, nu, h
+
+
+def affine_solve(A, b, y0=None, reverse=False) -> np.ndarray:
+    """A (L,T,4,4), b (L,T,4) -> y (L,T,4); see oracle_affine_solve."""
+    lib = _load()
+    A, b = _f64(A), _f64(b)
+    L, T = b.shape[:2]
+    y = np.zeros((L, T, 4))
+    y0p = None
+    if y0 is not None:
+        y0 = _f64(y0)
+        y0p = _ptr(y0)
+    lib.oracle_affine_solve(L, T, _ptr(A), _ptr(b), y0p, 1 if reverse else 0, _ptr(y))
+    return y
+
+
+def newton(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
+    """fp64 Newton; returns (S, stats dict)."""
+    lib = _load()
+    P, R, s0 = _f64(P), _f64(R), _f64(s0)
+    L, T, _ = P.shape
+    S = np.zeros((L, T, 4))
+    hr = np.full(max_iters, np.nan)
+    hs = np.full(max_iters, np.nan)
+    it, conv, div = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    lib.oracle_newton(L, T, _ptr(P), _ptr(R), _ptr(s0), _forget_code(forget), int(max_iters),
+                      1 if fixed else 0, float(tol), _ptr(S), _ptr(hr), _ptr(hs),
+                      ctypes.byref(it), ctypes.byref(conv), ctypes.byref(div))
+    return S, {"iters": it.value, "converged": bool(conv.value), "diverged": bool(div.value),
+               "max_abs_F": hr[: it.value].copy(), "max_scaled_F": hs[: it.value].copy()}
+
+
+def bptt(P, R, s0, S, dH, forget="sigmoid"):
+    """Reverse-time adjoint + cell VJP; returns (dP (L,T,4), dR (L,4), db (L,4), ds0 (L,4))."""
+    lib = _load()
+    P, R, s0, S, dH = _f64(P), _f64(R), _f64(s0), _f64(S), _f64(dH)
+    L, T, _ = P.shape
+    dP = np.zeros((L, T, 4))
+    dR, db, ds0 = np.zeros((L, 4)), np.zeros((L, 4)), np.zeros((L, 4))
+    lib.oracle_bptt(L, T, _ptr(P), _ptr(R), _ptr(s0), _ptr(S), _ptr(dH), _forget_code(forget),
+                    _ptr(dP), _ptr(dR), _ptr(db), _ptr(ds0))
+    return dP, dR, db, ds0
+
+
+def gemm(A, B, ta=False, tb=False, bias=None) -> np.ndarray:
+    """C = op(A) op(B) (+ bias); op(A) is (M,K), op(B) is (K,N)."""
+    lib = _load()
+    A, B = _f64(A), _f64(B)
+    M, K = (A.shape[1], A.shape[0]) if ta else A.shape
+    K2, N = (B.shape[1], B.shape[0]) if tb else B.shape
+    assert K == K2, (A.shape, B.shape, ta, tb)
+    C = np.zeros((M, N))
+    bp = None
+    if bias is not None:
+        bias = _f64(bias)
+        bp = _ptr(bias)
+    lib.oracle_gemm(M, N, K, _ptr(A), int(ta), _ptr(B), int(tb), bp, _ptr(C))
+    return C
+
+
+# ----------------------------------------------------------------------------
+# boundary-layout conveniences (full tensors; small problems only)
+# ----------------------------------------------------------------------------
+def preact(x, Wx, bias) -> np.ndarray:
+    """x (B,T,d_in), Wx (4 d_h, d_in), bias (4, d_h) -> P (B,T,4,d_h)."""
+    B, T, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    P = gemm(np.asarray(x).reshape(B * T, d_in), Wx, tb=True, bias=np.asarray(bias).reshape(-1))
+    return P.reshape(B, T, 4, d_h)
+
+
+def sequential_btgd(P, R, s0, forget="sigmoid") -> np.ndarray:
+    B, T, _, d = P.shape
+    S = sequential(lanes_from_btgd(P), lanes_from_gd(R, B), lanes_from_bgd(s0), forget)
+    return btgd_from_lanes(S, B, d)
+
+
+def newton_btgd(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
+    B, T, _, d = P.shape
+    S, st = newton(lanes_from_btgd(P), lanes_from_gd(R, B), lanes_from_bgd(s0), forget,
+                   max_iters, fixed, tol)
+    return btgd_from_lanes(S, B, d), st
+
+
+def backward_btgd(x, Wx, P, R, s0, S, dH, forget="sigmoid"):
+    """Full gradients of L = sum dH * h: returns dict dx, dWx, dR, db, ds0, dP."""
+    B, T, _, d = P.shape
+    d_in = Wx.shape[1]
+    dHl = _f64(np.transpose(dH, (0, 2, 1)).reshape(B * d, T))
+    dP, dR, db, ds0 = bptt(lanes_from_btgd(P), lanes_from_gd(R, B), lanes_from_bgd(s0),
+                           lanes_from_btgd(S), dHl, forget)
+    dP_b = btgd_from_lanes(dP, B, d)                       # (B,T,4,d)
+    dP2 = dP_b.reshape(B * T, 4 * d)
+    dx = gemm(dP2, Wx).reshape(B, T, d_in)                  # dP W_x
+    dWx = gemm(dP2, np.asarray(x).reshape(B * T, d_in), ta=True)  # dP^T x
+    dR_g = dR.reshape(B, d, 4).sum(axis=0).T.copy()         # (4, d)
+    db_g = db.reshape(B, d, 4).sum(axis=0).T.copy()
+    return {"dx": dx, "dWx": dWx, "dR": dR_g, "db": db_g,
+            "ds0": bgd_from_lanes(ds0, B, d), "dP": dP_b}

@@ -1,0 +1,321 @@
+"""Pins for the fp64 CPU oracle (CPU only).
+
+Each test ties the oracle to something other than itself: a worked example
+derived by hand from the cell equations, closed forms, invariants the pages
+state (stabilised == unstabilised), brute force, finite differences, or a
+library routine.  Sources: "xLSTM - a from-scratch, educational
+reimplementation" (section "Exponential gating + the stabilizer"), "xLSTM:
+Extended Long Short-Term Memory" (summary, section "Method": sLSTM step,
+stabilizer, item 1 "stabilised and unstabilised forms give identical
+outputs"), "sLSTM in this library" (pararnn-torch docs, sections "Cell",
+"Backward"), "pararnn-torch structure" (section "Current surface").
+"""
+import json
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "slstm_two_steps.json")
+
+
+def _ev(s: str) -> float:
+    expr = re.sub(r"ln(\d+)", r"math.log(\1)", s)
+    return float(eval(expr, {"__builtins__": {}, "math": math}))
+
+
+def _rand_lane_inputs(rng, L, T, forget="sigmoid", r_scale=0.5, s0_random=True):
+    P = rng.normal(size=(L, T, 4))
+    P[:, :, 2] += rng.uniform(3, 6, size=(L, 1))       # forget bias as in the workloads
+    R = rng.uniform(-r_scale, r_scale, size=(L, 4))
+    if s0_random:
+        s0 = np.stack([rng.normal(size=L), rng.uniform(0.5, 2.0, size=L),
+                       rng.normal(size=L), rng.uniform(-0.9, 0.9, size=L)], axis=1)
+    else:
+        s0 = np.zeros((L, 4))
+    return P, R, s0
+
+
+# ---------------------------------------------------------------------------
+# worked example by hand
+# ---------------------------------------------------------------------------
+def test_golden_two_steps():
+    g = json.load(open(GOLDEN))
+    R = np.array(g["R"])[None]
+    s0 = np.array(g["s0"])[None]
+    P = np.array([[_ev(v) for v in row] for row in g["P"]])[None]
+    for forget in ("sigmoid", "exp"):
+        S = oracle.sequential(P, R, s0, forget)[0]
+        exp = np.array([[_ev(v) for v in row] for row in g["expected"][forget]])
+        np.testing.assert_allclose(S, exp, rtol=0, atol=1e-14)
+    _, J, _ = oracle.step(np.array([_ev(v) for v in g["expected"]["sigmoid"][0]]), P[0, 1], R[0],
+                          "sigmoid")
+    expJ = np.array([[_ev(v) for v in row] for row in g["expected"]["sigmoid_J_step2"]])
+    np.testing.assert_allclose(J, expJ, rtol=0, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# closed forms and invariants of the forward step
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_stabilised_equals_unstabilised(forget):
+    rng = np.random.default_rng(11)
+    T = 48 if forget == "exp" else 200
+    P, R, s0 = _rand_lane_inputs(rng, 6, T, forget)
+    S = oracle.sequential(P, R, s0, forget)
+    cu, nu, h = oracle.sequential_unstabilised(P, R, s0, forget)
+    np.testing.assert_allclose(S[:, :, 3], h, rtol=0, atol=1e-12 * (1 + np.abs(h)).max())
+    # the stabilised state is the unstabilised one rescaled by exp(-m)
+    np.testing.assert_allclose(S[:, :, 0], cu * np.exp(-S[:, :, 2]), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(S[:, :, 1], nu * np.exp(-S[:, :, 2]), rtol=1e-11, atol=1e-12)
+
+
+def test_first_step_from_zero_state():
+    rng = np.random.default_rng(3)
+    for forget in ("sigmoid", "exp"):
+        for _ in range(50):
+            p = rng.normal(scale=3.0, size=4)
+            r = rng.normal(size=4)
+            m0 = rng.normal(scale=5.0)
+            h0 = rng.normal()
+            s, _, _ = oracle.step(np.array([0.0, 0.0, m0, h0]), p, r, forget)
+            az, ao = p[0] + r[0] * h0, p[3] + r[3] * h0
+            assert abs(s[3] - math.tanh(az) / (1 + math.exp(-ao))) < 1e-14
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_zero_recurrence_closed_form(forget):
+    """R = 0, zero start: h_t = o_t * sum_s w_ts z_s / sum_s w_ts with
+    log w_ts = a_i(s) + sum_{s<u<=t} log f_u (evaluated in log space)."""
+    rng = np.random.default_rng(5)
+    T = 40
+    P, _, _ = _rand_lane_inputs(rng, 3, T, forget)
+    R = np.zeros((3, 4))
+    s0 = np.zeros((3, 4))
+    S = oracle.sequential(P, R, s0, forget)
+    for l in range(3):
+        z = np.tanh(P[l, :, 0])
+        o = 1 / (1 + np.exp(-P[l, :, 3]))
+        lf = P[l, :, 2] if forget == "exp" else -np.logaddexp(0, -P[l, :, 2])
+        cum = np.concatenate([[0.0], np.cumsum(lf)])
+        for t in range(T):
+            lw = P[l, : t + 1, 1] + (cum[t + 1] - cum[1 : t + 2])
+            w = np.exp(lw - lw.max())
+            h = o[t] * (w @ z[: t + 1]) / w.sum()
+            assert abs(S[l, t, 3] - h) < 1e-12
+
+
+def test_stabilised_gates_bounded_and_finite_under_huge_inputs():
+    rng = np.random.default_rng(7)
+    for forget in ("sigmoid", "exp"):
+        P = rng.normal(scale=300.0, size=(4, 64, 4))
+        R = rng.normal(scale=50.0, size=(4, 4))
+        S = oracle.sequential(P, R, np.zeros((4, 4)), forget)
+        assert np.isfinite(S).all()
+        # i', f' in (0, 1] means n_t <= n_{t-1} + 1 and n_t > 0
+        n = S[:, :, 1]
+        assert (n > 0).all()
+        assert (n[:, 1:] <= n[:, :-1] + 1 + 1e-12).all()
+        assert (np.abs(S[:, :, 3]) <= 1 + 1e-12).all()
+
+
+# ---------------------------------------------------------------------------
+# Jacobians
+# ---------------------------------------------------------------------------
+def _fd_jacobian(sp, p, r, forget, eps=1e-6):
+    J = np.zeros((4, 4))
+    for k in range(4):
+        e = np.zeros(4)
+        e[k] = eps
+        fp_, _, _ = oracle.step(sp + e, p, r, forget)
+        fm_, _, _ = oracle.step(sp - e, p, r, forget)
+        J[:, k] = (fp_ - fm_) / (2 * eps)
+    return J
+
+
+def _fd_gate_jacobian(sp, p, r, forget, eps=1e-6):
+    G = np.zeros((4, 4))
+    for k in range(4):
+        e = np.zeros(4)
+        e[k] = eps
+        fp_, _, _ = oracle.step(sp, p + e, r, forget)
+        fm_, _, _ = oracle.step(sp, p - e, r, forget)
+        G[:, k] = (fp_ - fm_) / (2 * eps)
+    return G
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_jacobians_match_finite_differences(forget):
+    rng = np.random.default_rng(17)
+    checked = 0
+    while checked < 60:
+        sp = np.array([rng.normal(), rng.uniform(0.3, 3.0), rng.normal(scale=2), rng.uniform(-1, 1)])
+        p = rng.normal(scale=1.5, size=4)
+        r = rng.uniform(-1, 1, size=4)
+        s, J, G = oracle.step(sp, p, r, forget)
+        # stay away from the tie of the max (non-differentiable there)
+        h0 = sp[3]
+        lf = (p[2] + r[2] * h0) if forget == "exp" else -np.logaddexp(0, -(p[2] + r[2] * h0))
+        if abs(lf + sp[2] - (p[1] + r[1] * h0)) < 1e-3:
+            continue
+        Jfd = _fd_jacobian(sp, p, r, forget)
+        Gfd = _fd_gate_jacobian(sp, p, r, forget)
+        np.testing.assert_allclose(J, Jfd, rtol=1e-6, atol=1e-8)
+        np.testing.assert_allclose(G, Gfd, rtol=1e-6, atol=1e-8)
+        # h_{t-1} enters only through a_t = P_t + r h_{t-1}: J[:, h] = G r
+        np.testing.assert_allclose(J[:, 3], G @ r, rtol=1e-12, atol=1e-14)
+        checked += 1
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_gauge_identity(forget):
+    """Rescaling the unstabilised state leaves h unchanged: with
+    g = (-c, -n, 1, 0), J_t g_{t-1} = beta_t g_t exactly."""
+    rng = np.random.default_rng(23)
+    for _ in range(100):
+        sp = np.array([rng.normal(), rng.uniform(0.3, 3.0), rng.normal(scale=2), rng.uniform(-1, 1)])
+        p = rng.normal(scale=1.5, size=4)
+        r = rng.uniform(-1, 1, size=4)
+        s, J, _ = oracle.step(sp, p, r, forget)
+        beta = J[2, 2]
+        assert beta in (0.0, 1.0)
+        g_prev = np.array([-sp[0], -sp[1], 1.0, 0.0])
+        g_now = np.array([-s[0], -s[1], 1.0, 0.0])
+        np.testing.assert_allclose(J @ g_prev, beta * g_now, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# affine scan
+# ---------------------------------------------------------------------------
+def _tree_compose(maps):
+    """Compose affine maps (A, b), earliest first, by recursive halving."""
+    if len(maps) == 1:
+        return maps[0]
+    mid = len(maps) // 2
+    A1, b1 = _tree_compose(maps[:mid])
+    A2, b2 = _tree_compose(maps[mid:])
+    return A2 @ A1, A2 @ b1 + b2
+
+
+def test_affine_solve_matches_brute_force_and_tree():
+    rng = np.random.default_rng(29)
+    L, T = 3, 37
+    A = rng.normal(scale=0.5, size=(L, T, 4, 4))
+    b = rng.normal(size=(L, T, 4))
+    y0 = rng.normal(size=(L, 4))
+    y = oracle.affine_solve(A, b, y0)
+    yr = oracle.affine_solve(A, b, y0, reverse=True)
+    for l in range(L):
+        # forward: left fold of y -> A y + b
+        v = y0[l].copy()
+        for t in range(T):
+            v = A[l, t] @ v + b[l, t]
+            np.testing.assert_allclose(y[l, t], v, rtol=1e-12, atol=1e-12)
+            At, bt = _tree_compose([(A[l, s], b[l, s]) for s in range(t + 1)])
+            np.testing.assert_allclose(y[l, t], At @ y0[l] + bt, rtol=1e-11, atol=1e-11)
+        # reverse-transposed: y_t = A_t^T y_{t+1} + b_t, y_T = y0
+        v = y0[l].copy()
+        for t in range(T - 1, -1, -1):
+            v = A[l, t].T @ v + b[l, t]
+            np.testing.assert_allclose(yr[l, t], v, rtol=1e-12, atol=1e-12)
+    # missing y0 means zero
+    np.testing.assert_allclose(oracle.affine_solve(A, b), oracle.affine_solve(A, b, np.zeros((L, 4))))
+
+
+# ---------------------------------------------------------------------------
+# Newton
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_newton_prefix_exact_after_k_iterations(forget):
+    """After k Newton iterations the first k steps equal the sequential
+    trajectory (by induction: step t only depends on exact earlier steps),
+    and K = T iterations reproduce the whole trajectory."""
+    rng = np.random.default_rng(31)
+    T = 12
+    P, R, s0 = _rand_lane_inputs(rng, 4, T, forget)
+    Sseq = oracle.sequential(P, R, s0, forget)
+    for k in (1, 2, 5):
+        S, st = oracle.newton(P, R, s0, forget, max_iters=k, fixed=True)
+        assert st["iters"] == k
+        np.testing.assert_allclose(S[:, :k], Sseq[:, :k], rtol=0,
+                                   atol=1e-12 * (1 + np.abs(Sseq).max()))
+    S, st = oracle.newton(P, R, s0, forget, max_iters=T, fixed=True)
+    np.testing.assert_allclose(S, Sseq, rtol=0, atol=1e-12 * (1 + np.abs(Sseq).max()))
+
+
+def test_newton_converges_by_tolerance():
+    rng = np.random.default_rng(37)
+    P, R, s0 = _rand_lane_inputs(rng, 8, 64, "sigmoid", s0_random=False)
+    Sseq = oracle.sequential(P, R, s0, "sigmoid")
+    S, st = oracle.newton(P, R, s0, "sigmoid", max_iters=64, fixed=False, tol=1e-10)
+    assert st["converged"] and not st["diverged"]
+    assert st["iters"] < 64
+    assert st["max_scaled_F"][-1] <= 1e-10
+    # iteration k's recorded residual is the residual of the k-th iterate
+    np.testing.assert_allclose(S, Sseq, rtol=0, atol=1e-9)
+
+
+def test_newton_divergence_flag():
+    P = np.full((1, 8, 4), np.nan)
+    S, st = oracle.newton(P, np.zeros((1, 4)), np.zeros((1, 4)), "sigmoid", max_iters=3)
+    assert st["diverged"] and not st["converged"]
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+def _loss(x, Wx, bias, R, s0, dH, forget):
+    P = oracle.preact(x, Wx, bias)
+    S = oracle.sequential_btgd(P, R, s0, forget)
+    return float((S[:, :, 3, :] * dH).sum())
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_bptt_matches_finite_differences(forget):
+    rng = np.random.default_rng(41)
+    B, T, d_in, d = 2, 10, 3, 2
+    x = rng.normal(size=(B, T, d_in))
+    Wx = rng.normal(size=(4 * d, d_in)) / math.sqrt(d_in)
+    R = rng.uniform(-0.5, 0.5, size=(4, d))
+    bias = np.zeros((4, d))
+    bias[2] = np.linspace(3, 6, d)
+    s0 = np.stack([rng.normal(size=(B, d)), rng.uniform(0.5, 2, size=(B, d)),
+                   rng.normal(size=(B, d)), rng.uniform(-0.5, 0.5, size=(B, d))], axis=1)
+    dH = rng.normal(size=(B, T, d))
+    P = oracle.preact(x, Wx, bias)
+    S = oracle.sequential_btgd(P, R, s0, forget)
+    g = oracle.backward_btgd(x, Wx, P, R, s0, S, dH, forget)
+
+    def check(name, arr, grad):
+        it = np.nditer(arr, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = arr[idx]
+            eps = 1e-6 * max(1.0, abs(old))
+            arr[idx] = old + eps
+            lp = _loss(x, Wx, bias, R, s0, dH, forget)
+            arr[idx] = old - eps
+            lm = _loss(x, Wx, bias, R, s0, dH, forget)
+            arr[idx] = old
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - grad[idx]) <= 1e-6 * (1 + abs(fd)), (name, idx, fd, grad[idx])
+
+    check("x", x, g["dx"])
+    check("Wx", Wx, g["dWx"])
+    check("R", R, g["dR"])
+    check("bias", bias, g["db"])
+    check("s0", s0, g["ds0"])
+
+
+def test_gemm_matches_numpy():
+    rng = np.random.default_rng(43)
+    A = rng.normal(size=(7, 5))
+    Bm = rng.normal(size=(5, 3))
+    bias = rng.normal(size=3)
+    np.testing.assert_allclose(oracle.gemm(A, Bm, bias=bias), A @ Bm + bias, rtol=1e-13)
+    np.testing.assert_allclose(oracle.gemm(A.T.copy(), Bm, ta=True), A @ Bm, rtol=1e-13)
+    np.testing.assert_allclose(oracle.gemm(A, Bm.T.copy(), tb=True), A @ Bm, rtol=1e-13)
