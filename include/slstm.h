@@ -1,0 +1,231 @@
+/*
+ * slstm.h - C ABI of the Newton-solved diag-mix sLSTM library (libslstm.so).
+ *
+ * The library solves the diag-mix sLSTM recurrence of xLSTM in parallel over
+ * the sequence with Newton iterations whose linear solves are associative
+ * scans of 4x4 affine maps, on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (page titles and sections):
+ *   "sLSTM in this library" (pararnn-torch docs): "Cell" (state (B,T,4,d_h)
+ *     = (c,n,m,h), hidden slot 3; mix='diag' with channelwise R of shape
+ *     (4,d_h) and a 4x4 Jacobian per feature), "API notes" (Newton in
+ *     training, sequential stepping in evaluation, W_x is a GEMM, out=
+ *     buffers), "Backward" (one reverse associative scan of J^T, then a packed
+ *     cell VJP for grad R and grad W_x).
+ *   "pararnn-torch structure": "Current surface" (fused kernels prepend h0;
+ *     residual early stop; divergence when max|F| > 1 after K), "Naming"
+ *     (scan_block4 for the (B,T,4,4,d) layout).
+ *   "xLSTM - a from-scratch, educational reimplementation": "Exponential
+ *     gating + the stabilizer" (the stabilised step).
+ *   "xLSTM: Extended Long Short-Term Memory" (summary): "Method", the sLSTM
+ *     step (gate order z, i, f, o; h = o * c / n) and the stabilizer
+ *     m_t = max(log f_t + m_{t-1}, log i_t).
+ *
+ * The cell, per batch row b, feature j and step t (gate order z, i, f, o;
+ * slot order c, n, m, h):
+ *   a_g = P[b,t,g,j] + R[g,j] * h_{t-1}
+ *   z = tanh a_z, o = sigmoid a_o, log i = a_i,
+ *   log f = log sigmoid a_f (SLSTM_FORGET_SIGMOID) or a_f (SLSTM_FORGET_EXP)
+ *   m = max(log f + m_{t-1}, a_i), i' = exp(a_i - m), f' = exp(log f + m_{t-1} - m)
+ *   c = f' c_{t-1} + i' z,  n = f' n_{t-1} + i',  h = o c / n
+ * with (c,n,m,h)_{-1} = s0.
+ *
+ * Conventions shared by every call:
+ *   - Every tensor pointer is DEVICE memory owned by the caller, contiguous
+ *     (row-major in the stated shape) and 16-byte aligned.  Outputs are
+ *     written in full; the library keeps no pointer after the call returns.
+ *   - The library allocates no device memory.  Calls that need scratch take
+ *     a caller-owned workspace (ws, ws_bytes) of at least
+ *     slstm_workspace_size(op, ...) bytes, 256-byte aligned.  Calls that
+ *     share a workspace must not overlap in time (use one stream).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and the call returns without synchronising.
+ *   - Return value: SLSTM_OK, SLSTM_ERR_INVALID_ARG for arguments rejected on
+ *     the host before anything is launched (null or misaligned pointers,
+ *     non-positive or too-large sizes, workspace too small, unknown enum), or
+ *     SLSTM_ERR_CUDA when a launch fails.  Newton outcomes (iterations,
+ *     convergence, divergence, bounded-wait timeouts) are written to the
+ *     device-side stats record and read by the caller after synchronising.
+ *   - No call aborts, traps or throws.
+ *   - Sizes: 1 <= B <= 65535, 1 <= T, 1 <= d_in, d_h, d <= 2^20, B*T < 2^31
+ *     and B * ceil(T/32) * ceil(max(d_in, d_h)/32) < 2^31.
+ */
+#ifndef SLSTM_H
+#define SLSTM_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *slstm_stream_t; /* a cudaStream_t */
+
+typedef enum {
+    SLSTM_OK = 0,
+    SLSTM_ERR_INVALID_ARG = 1,
+    SLSTM_ERR_CUDA = 2,
+    SLSTM_ERR_DIVERGED = 3,    /* stats.error only: max|F| > 1 or non-finite */
+    SLSTM_ERR_TIMEOUT = 4,     /* stats.error only: a bounded wait ran out   */
+    SLSTM_ERR_UNSUPPORTED = 5  /* valid request this build cannot run        */
+} slstm_status;
+
+typedef enum { SLSTM_F32 = 0, SLSTM_BF16 = 1 } slstm_dtype;
+
+typedef enum { SLSTM_FORGET_SIGMOID = 0, SLSTM_FORGET_EXP = 1 } slstm_forget;
+
+/* Operation codes for slstm_workspace_size. */
+typedef enum {
+    SLSTM_OP_PREACT_GEMM = 0,
+    SLSTM_OP_NEWTON_FORWARD = 1,
+    SLSTM_OP_SCAN_BLOCK4 = 2,
+    SLSTM_OP_NEWTON_BACKWARD = 3
+} slstm_op;
+
+#define SLSTM_MAX_ITERS 65536     /* largest accepted max_iters              */
+#define SLSTM_STATS_HISTORY 64    /* residual history kept in the stats record */
+
+/* scan_block4 flags */
+#define SLSTM_SCAN_REVERSE_T 1
+
+/*
+ * Newton solver settings ("pararnn-torch structure", "Current surface":
+ * NewtonConfig(max_iters), residual early stop, fixed-K compile-safe preset).
+ *   max_iters   1..SLSTM_MAX_ITERS: iteration cap (tolerance mode) or the
+ *               exact iteration count (fixed mode).
+ *   fixed_iters 0: stop at the first iteration whose new iterate meets tol;
+ *               1: run exactly max_iters iterations.
+ *   tol         tolerance on the scaled residual max |F| / (1 + |s|), taken
+ *               over every (b, t, slot, j) of the new iterate.
+ *   forget      slstm_forget.
+ *   debug_fault 0 in normal use.  1 makes one tile of the first iteration
+ *               withhold its scan carry, so that its successor's bounded
+ *               wait expires (the run then reports SLSTM_ERR_TIMEOUT in
+ *               stats.error; results are not meaningful).
+ *   wait_limit_us  upper bound of one bounded wait, in microseconds
+ *               (0 = the default of 2 seconds).
+ */
+typedef struct {
+    int max_iters;
+    int fixed_iters;
+    float tol;
+    int forget;
+    int debug_fault;
+    int wait_limit_us;
+} slstm_newton_config;
+
+/*
+ * Newton outcome, in DEVICE memory owned by the caller (zeroing it is not
+ * required; slstm_newton_forward initialises it on the stream).
+ *   iters        Newton iterations performed.
+ *   converged    1 when the last iterate's scaled residual <= tol.
+ *   diverged     1 when not converged and max|F| > 1 or non-finite after the
+ *                last iteration ("NewtonDivergenceError" of the pages).
+ *   error        0, SLSTM_ERR_DIVERGED when diverged, or SLSTM_ERR_TIMEOUT.
+ *   max_abs_F[k % 64], max_scaled_F[k % 64]   residual of the iterate
+ *                produced by iteration k (max over every element), for the
+ *                last min(iters, 64) iterations.  In fixed mode only the final
+ *                iteration evaluates its residual; the others hold -1.
+ */
+typedef struct {
+    int iters;
+    int converged;
+    int diverged;
+    int error;
+    float max_abs_F[SLSTM_STATS_HISTORY];
+    float max_scaled_F[SLSTM_STATS_HISTORY];
+} slstm_newton_stats;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *slstm_status_string(int status);
+
+/*
+ * Bytes of workspace an operation needs for the given sizes (0 when it needs
+ * none).  Unused size arguments may be 0.  Returns 0 for invalid input.
+ */
+size_t slstm_workspace_size(int op, int B, int T, int d_in, int d_h);
+
+/*
+ * Input projection ("sLSTM in this library", "API notes": W_x is a GEMM;
+ * the summary's sLSTM step: W_* x + b_*):
+ *   P[b,t,g,j] = sum_k x[b,t,k] * Wx[g*d_h + j, k] + bias[g,j]
+ *   x     (B, T, d_in)  dtype `dtype` (SLSTM_F32 or SLSTM_BF16)
+ *   Wx    (4*d_h, d_in) same dtype; rows gate-major (z, i, f, o)
+ *   bias  (4, d_h) fp32
+ *   P     (B, T, 4, d_h) fp32 output
+ * bf16 inputs run on the tcgen05 tensor cores with fp32 accumulation; fp32
+ * inputs run an fp32 CUDA-core GEMM.  bf16 requires d_in % 8 == 0.
+ */
+int slstm_preact_gemm(const void *x, const void *Wx, int dtype, const float *bias, float *P,
+                      int B, int T, int d_in, int d_h, void *ws, size_t ws_bytes,
+                      slstm_stream_t stream);
+
+/*
+ * Newton solve of the whole trajectory ("sLSTM in this library", "Cell";
+ * "pararnn-torch structure", "Current surface"):
+ *   guess S = 0 for every step; s0 enters as the step before t = 0;
+ *   each iteration evaluates F_t = S_t - f(S_{t-1}, P_t) and J_t = df/ds_{t-1}
+ *   at the guess, solves delta_t = J_t delta_{t-1} - F_t (delta_{-1} = 0) by a
+ *   blocked associative scan of 4x4 affine maps, and sets S <- S + delta;
+ *   it then evaluates the residual of the new iterate for the stopping test.
+ *   P     (B, T, 4, d_h) fp32
+ *   R     (4, d_h) fp32
+ *   s0    (B, 4, d_h) fp32, or NULL for zeros
+ *   S     (B, T, 4, d_h) fp32 output (the last iterate; h is slot 3)
+ *   cfg   host pointer, read during the call
+ *   stats device pointer to one slstm_newton_stats, written on the stream
+ * The call enqueues max_iters iterations; iterations after convergence (or
+ * after a timeout or non-finite residual) return immediately on the device,
+ * so the call never synchronises with the host.
+ */
+int slstm_newton_forward(const float *P, const float *R, const float *s0, float *S,
+                         const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
+                         int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+/*
+ * Associative scan of 4x4 affine maps ("pararnn-torch structure", "Naming":
+ * scan_block4 for the (B,T,4,4,d) layout; "sLSTM in this library", "Packed
+ * sequences": the Newton inner solve is a scan on the (J, r) monoid):
+ *   flags = 0:                    y_t = A_t y_{t-1} + b_t,   y_{-1} = y0
+ *   flags = SLSTM_SCAN_REVERSE_T: y_t = A_t^T y_{t+1} + b_t, y_T   = y0
+ *   A   (B, T, 4, 4, d) fp32, indexed [b][t][row][col][j]
+ *   b   (B, T, 4, d) fp32
+ *   y0  (B, 4, d) fp32, or NULL for zeros
+ *   y   (B, T, 4, d) fp32 output; may not alias A or b
+ * Composition is in fp32.
+ */
+int scan_block4(const float *A, const float *b, const float *y0, float *y, int B, int T, int d,
+                int flags, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+/*
+ * Sequential stepping ("sLSTM in this library", "API notes": the evaluation
+ * path; T_steps = 1 is one decode step):
+ *   S_t = f(S_{t-1}, P_t) for t = 0 .. T_steps-1, S_{-1} = s0.
+ *   P (B, T_steps, 4, d_h), R (4, d_h), s0 (B, 4, d_h) or NULL, S (B, T_steps, 4, d_h).
+ */
+int slstm_sequential_step(const float *P, const float *R, const float *s0, float *S, int B,
+                          int T_steps, int d_h, int forget, slstm_stream_t stream);
+
+/*
+ * Gradients of L = sum_{b,t,j} dH[b,t,j] * h[b,t,j] at the solution S
+ * ("sLSTM in this library", "Backward": one reverse associative scan of J^T,
+ * then the packed cell VJP):
+ *   lambda_t = e_h dH_t + J_{t+1}^T lambda_{t+1}   (reverse scan, fp32)
+ *   dP_t = G_t^T lambda_t with G_t = ds_t/da_t, a_t = P_t + R h_{t-1}
+ *   dR[g,j] = sum_{b,t} dP[b,t,g,j] h[b,t-1,j]; db[g,j] = sum_{b,t} dP[b,t,g,j]
+ *   ds0 = J_0^T lambda_0;  dx = dP Wx;  dWx = dP^T x
+ *   x (B,T,d_in) and Wx (4*d_h,d_in) in `dtype`; P, S (B,T,4,d_h); R (4,d_h);
+ *   s0 (B,4,d_h) or NULL; dH (B,T,d_h); outputs fp32: dx (B,T,d_in),
+ *   dWx (4*d_h,d_in), dR (4,d_h), db (4,d_h), ds0 (B,4,d_h) (may be NULL).
+ */
+int slstm_newton_backward(const void *x, const void *Wx, int dtype, const float *P,
+                          const float *R, const float *s0, const float *S, const float *dH,
+                          float *dx, float *dWx, float *dR, float *db, float *ds0, int forget,
+                          int B, int T, int d_in, int d_h, void *ws, size_t ws_bytes,
+                          slstm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLSTM_H */

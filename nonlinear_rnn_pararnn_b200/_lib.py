@@ -1,0 +1,89 @@
+"""ctypes loader for libslstm.so (the C ABI declared in include/slstm.h).
+
+Argument marshalling only: no arithmetic of the method happens in Python.
+Importing this module never falls back to anything: if the shared library is
+missing it is built with nvcc, and if that fails the import raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+SLSTM_OK = 0
+SLSTM_ERR_INVALID_ARG = 1
+SLSTM_ERR_CUDA = 2
+SLSTM_ERR_DIVERGED = 3
+SLSTM_ERR_TIMEOUT = 4
+SLSTM_ERR_UNSUPPORTED = 5
+
+SLSTM_F32 = 0
+SLSTM_BF16 = 1
+SLSTM_FORGET_SIGMOID = 0
+SLSTM_FORGET_EXP = 1
+SLSTM_OP_PREACT_GEMM = 0
+SLSTM_OP_NEWTON_FORWARD = 1
+SLSTM_OP_SCAN_BLOCK4 = 2
+SLSTM_OP_NEWTON_BACKWARD = 3
+SLSTM_MAX_ITERS = 65536
+SLSTM_STATS_HISTORY = 64
+SLSTM_SCAN_REVERSE_T = 1
+
+
+class NewtonConfig(ctypes.Structure):
+    _fields_ = [("max_iters", ctypes.c_int), ("fixed_iters", ctypes.c_int), ("tol", ctypes.c_float),
+                ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int)]
+
+
+STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY
+
+_V = ctypes.c_void_p
+_I = ctypes.c_int
+_Z = ctypes.c_size_t
+
+# name -> (restype, argtypes); every function of include/slstm.h
+SIGNATURES = {
+    "slstm_status_string": (ctypes.c_char_p, [_I]),
+    "slstm_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "slstm_preact_gemm": (_I, [_V, _V, _I, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
+    "slstm_newton_forward": (_I, [_V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _V, _Z, _V]),
+    "scan_block4": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
+    "slstm_sequential_step": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
+    "slstm_newton_backward": (_I, [_V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I,
+                                   _V, _Z, _V]),
+}
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def load() -> ctypes.CDLL:
+    """Load libslstm.so (building it first when it is missing or stale)."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError(f"libslstm.so was not built at {path}")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+class SlstmError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = load().slstm_status_string(status).decode()
+        super().__init__(f"{fn} returned {name} ({status})")
+
+
+def check(fn: str, status: int) -> None:
+    if status != SLSTM_OK:
+        raise SlstmError(fn, status)

@@ -1,0 +1,173 @@
+"""Python binding of libslstm: torch tensors in, torch tensors out.
+
+Each function checks shapes, dtypes and devices, allocates outputs and
+workspace with torch (device memory is the one thing torch provides here),
+and calls the C ABI on the current CUDA stream.  Every step of the method
+runs in the library's CUDA kernels; nothing here computes.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import NewtonConfig, check, load
+
+_FORGET = {"sigmoid": _lib.SLSTM_FORGET_SIGMOID, "exp": _lib.SLSTM_FORGET_EXP}
+_DTYPE = {torch.float32: _lib.SLSTM_F32, torch.bfloat16: _lib.SLSTM_BF16}
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype=torch.float32):
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def forget_code(forget) -> int:
+    return _FORGET[forget] if isinstance(forget, str) else int(forget)
+
+
+def workspace_size(op: int, B: int, T: int, d_in: int, d_h: int) -> int:
+    return int(load().slstm_workspace_size(op, B, T, d_in, d_h))
+
+
+def workspace(op: int, B: int, T: int, d_in: int, d_h: int, device=None) -> torch.Tensor:
+    n = workspace_size(op, B, T, d_in, d_h)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def preact_gemm(x: torch.Tensor, Wx: torch.Tensor, bias: torch.Tensor, P: torch.Tensor = None,
+                ws: torch.Tensor = None) -> torch.Tensor:
+    B, T, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    dt = x.dtype
+    _need(x, "x", (B, T, d_in), dt)
+    _need(Wx, "Wx", (4 * d_h, d_in), dt)
+    _need(bias, "bias", (4, d_h))
+    if P is None:
+        P = torch.empty(B, T, 4, d_h, dtype=torch.float32, device=x.device)
+    _need(P, "P", (B, T, 4, d_h))
+    n = workspace_size(_lib.SLSTM_OP_PREACT_GEMM, B, T, d_in, d_h)
+    if n and ws is None:
+        ws = workspace(_lib.SLSTM_OP_PREACT_GEMM, B, T, d_in, d_h, x.device)
+    check("slstm_preact_gemm", load().slstm_preact_gemm(_ptr(x), _ptr(Wx), _DTYPE[dt], _ptr(bias), _ptr(P),
+                                                        B, T, d_in, d_h, _ptr(ws), 0 if ws is None else ws.numel(),
+                                                        _stream()))
+    return P
+
+
+def new_stats(device=None) -> torch.Tensor:
+    return torch.zeros(_lib.STATS_BYTES, dtype=torch.uint8, device=device or "cuda")
+
+
+def read_stats(stats: torch.Tensor) -> dict:
+    """Copy a device stats record to the host and decode it."""
+    raw = stats.detach().to("cpu")
+    ints = raw[:16].view(torch.int32).tolist()
+    fl = raw[16:].view(torch.float32)
+    it = ints[0]
+    m = _lib.SLSTM_STATS_HISTORY
+    ks = list(range(max(0, it - m), it))     # the iterations the ring still holds
+    raw_h, sc_h = fl[:m].tolist(), fl[m:].tolist()
+    return {"iters": it, "converged": bool(ints[1]), "diverged": bool(ints[2]), "error": ints[3],
+            "history_first_iter": ks[0] if ks else 0,
+            "max_abs_F": [raw_h[k % m] for k in ks], "max_scaled_F": [sc_h[k % m] for k in ks]}
+
+
+def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
+                   max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
+                   stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
+                   wait_limit_us: int = 0):
+    """Newton solve; returns (S, stats) with stats a device record (see read_stats)."""
+    B, T, four, d_h = P.shape
+    _need(P, "P", (B, T, 4, d_h))
+    _need(R, "R", (4, d_h))
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    if S is None:
+        S = torch.empty_like(P)
+    _need(S, "S", (B, T, 4, d_h))
+    if stats is None:
+        stats = new_stats(P.device)
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
+    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
+                       int(wait_limit_us))
+    check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
+                                                              ctypes.byref(cfg), _ptr(stats), B, T, d_h,
+                                                              _ptr(ws), ws.numel(), _stream()))
+    return S, stats
+
+
+def scan_block4(A: torch.Tensor, b: torch.Tensor, y0: torch.Tensor = None, reverse: bool = False,
+                y: torch.Tensor = None, ws: torch.Tensor = None) -> torch.Tensor:
+    B, T, four, four2, d = A.shape
+    _need(A, "A", (B, T, 4, 4, d))
+    _need(b, "b", (B, T, 4, d))
+    if y0 is not None:
+        _need(y0, "y0", (B, 4, d))
+    if y is None:
+        y = torch.empty_like(b)
+    _need(y, "y", (B, T, 4, d))
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_SCAN_BLOCK4, B, T, 0, d, A.device)
+    flags = _lib.SLSTM_SCAN_REVERSE_T if reverse else 0
+    check("scan_block4", load().scan_block4(_ptr(A), _ptr(b), _ptr(y0), _ptr(y), B, T, d, flags, _ptr(ws),
+                                            ws.numel(), _stream()))
+    return y
+
+
+def sequential_step(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
+                    S: torch.Tensor = None) -> torch.Tensor:
+    B, T, four, d_h = P.shape
+    _need(P, "P", (B, T, 4, d_h))
+    _need(R, "R", (4, d_h))
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    if S is None:
+        S = torch.empty_like(P)
+    _need(S, "S", (B, T, 4, d_h))
+    check("slstm_sequential_step", load().slstm_sequential_step(_ptr(P), _ptr(R), _ptr(s0), _ptr(S), B, T, d_h,
+                                                                forget_code(forget), _stream()))
+    return S
+
+
+def newton_backward(x, Wx, P, R, s0, S, dH, *, forget="sigmoid", out: dict = None, ws: torch.Tensor = None):
+    """Gradients of sum(dH * h); returns dict dx, dWx, dR, db, ds0."""
+    B, T, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    dt = x.dtype
+    _need(x, "x", (B, T, d_in), dt)
+    _need(Wx, "Wx", (4 * d_h, d_in), dt)
+    _need(P, "P", (B, T, 4, d_h))
+    _need(R, "R", (4, d_h))
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    _need(S, "S", (B, T, 4, d_h))
+    _need(dH, "dH", (B, T, d_h))
+    dev = x.device
+    if out is None:
+        out = {"dx": torch.empty(B, T, d_in, device=dev), "dWx": torch.empty(4 * d_h, d_in, device=dev),
+               "dR": torch.empty(4, d_h, device=dev), "db": torch.empty(4, d_h, device=dev),
+               "ds0": torch.empty(B, 4, d_h, device=dev)}
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_BACKWARD, B, T, d_in, d_h, dev)
+    check("slstm_newton_backward", load().slstm_newton_backward(
+        _ptr(x), _ptr(Wx), _DTYPE[dt], _ptr(P), _ptr(R), _ptr(s0), _ptr(S), _ptr(dH), _ptr(out["dx"]),
+        _ptr(out["dWx"]), _ptr(out["dR"]), _ptr(out["db"]), _ptr(out.get("ds0")), forget_code(forget), B, T,
+        d_in, d_h, _ptr(ws), ws.numel(), _stream()))
+    return out

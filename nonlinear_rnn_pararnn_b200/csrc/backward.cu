@@ -1,0 +1,312 @@
+// Backward pass of the Newton-solved diag-mix sLSTM ("sLSTM in this
+// library", section "Backward": one reverse associative scan of J^T, then a
+// packed cell VJP for the gradients of R and W_x).
+//
+// Fused adjoint + VJP kernel, tiles in reverse time order:
+//   lambda_t = e_h dH_t + J_{t+1}^T lambda_{t+1}   (J recomputed from S_t, P_{t+1})
+//   dP_t     = G_t^T lambda_t,  G_t = d s_t / d a_t (recomputed from S_{t-1}, P_t)
+//   dR      += dP_t * h_{t-1},  db += dP_t   (per-tile partials, reduced after)
+//   ds0      = J_0^T lambda_0
+// then dx = dP W_x and dW_x = dP^T x.
+#include "launchers.h"
+#include "lookback.cuh"
+
+namespace slstm {
+namespace {
+
+constexpr int NW = 8;
+constexpr int L = 4;
+constexpr int TT = NW * L;
+
+struct BwdArgs {
+    const float *P;
+    const float *R;
+    const float *s0;
+    const float *S;
+    const float *dH;
+    float *dP;        // (B, T, 4, d)
+    float *partial;   // [n_tiles][8][32]  dR (4) then db (4)
+    float *ds0;       // (B, 4, d) or null
+    unsigned *ticket;
+    LookbackArgs lb;
+    int T, d, groups_per_row;
+};
+
+template <int FORGET>
+__global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
+{
+    __shared__ float s_agg[NW][20][32];
+    __shared__ float s_carry[NW][4][32];
+    __shared__ float s_part[NW][8][32];
+    __shared__ unsigned s_ticket;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1u);
+    __syncthreads();
+    const unsigned ticket = s_ticket;
+    const int G = a.lb.n_groups;
+    const int chunk = (int)(ticket / (unsigned)G);
+    const int grp = (int)(ticket % (unsigned)G);
+    const int b = grp / a.groups_per_row;
+    const int j = (grp % a.groups_per_row) * 32 + lane;
+    const bool jv = j < a.d;
+    const size_t jj = jv ? (size_t)j : 0;
+    const size_t d = (size_t)a.d;
+    const int T = a.T;
+    const size_t row0 = (size_t)b * T;
+    const int p_seg = chunk * TT + warp * L;  // processing position; t = T-1-p
+
+    float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
+    if (jv) {
+        rz = a.R[jj];
+        ri = a.R[d + jj];
+        rf = a.R[2 * d + jj];
+        ro = a.R[3 * d + jj];
+    }
+    float s0v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.s0 && jv) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s0v[e] = a.s0[((size_t)b * 4 + e) * d + jj];
+    }
+
+    // ---- walk A: fold lambda -> J_{t+1}^T lambda + e_h dH_t, t descending ----
+    Cell Jn[L];  // J_{t+1} for each step of the segment
+    float dh[L];
+    Aff agg;
+    aff_identity(agg);
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+        const int p = p_seg + i;
+        const int t = T - 1 - p;
+        dh[i] = 0.f;
+        cell_identity(Jn[i]);
+        if (p < T && jv) {
+            dh[i] = a.dH[(row0 + t) * d + jj];
+            if (t + 1 < T) {
+                const float *ps = a.S + (row0 + t) * 4 * d + jj;
+                const float *pp = a.P + (row0 + t + 1) * 4 * d + jj;
+                cell_eval<FORGET, true>(ps[0], ps[d], ps[2 * d], ps[3 * d], __ldg(pp), __ldg(pp + d),
+                                        __ldg(pp + 2 * d), __ldg(pp + 3 * d), rz, ri, rf, ro, Jn[i]);
+            } else {
+                // lambda past the end is zero, so the map's matrix is irrelevant
+            }
+        }
+        const float r[4] = {0.f, 0.f, 0.f, dh[i]};
+        fold_jacT(agg, Jn[i], r);
+    }
+    store_aff_smem(s_agg, warp, lane, agg);
+    __syncthreads();
+    if (warp == 0) {
+        const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+        tile_lookback_warp0<NW>(s_agg, s_carry, a.lb, ticket, chunk, zero, false);
+    }
+    __syncthreads();
+
+    // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
+    float lam[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) lam[e] = s_carry[warp][e][lane];
+    float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+        const int p = p_seg + i;
+        const int t = T - 1 - p;
+        if (p < T && jv) {
+            jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
+            lam[3] += dh[i];
+            float prev[4];
+            if (t == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prev[e] = s0v[e];
+            } else {
+                const float *ps = a.S + (row0 + t - 1) * 4 * d + jj;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prev[e] = ps[e * d];
+            }
+            const float *pp = a.P + (row0 + t) * 4 * d + jj;
+            Cell c;
+            CellG g;
+            cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], __ldg(pp), __ldg(pp + d),
+                                          __ldg(pp + 2 * d), __ldg(pp + 3 * d), rz, ri, rf, ro, c, &g);
+            const float dz = fmaf(g.gcz, lam[0], g.ghz * lam[3]);
+            const float di = fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3])));
+            const float df = fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3])));
+            const float dq = g.gho * lam[3];
+            float *pd = a.dP + (row0 + t) * 4 * d + jj;
+            pd[0] = dz;
+            pd[d] = di;
+            pd[2 * d] = df;
+            pd[3 * d] = dq;
+            const float hp = prev[3];
+            dr[0] = fmaf(dz, hp, dr[0]);
+            dr[1] = fmaf(di, hp, dr[1]);
+            dr[2] = fmaf(df, hp, dr[2]);
+            dr[3] = fmaf(dq, hp, dr[3]);
+            dbs[0] += dz;
+            dbs[1] += di;
+            dbs[2] += df;
+            dbs[3] += dq;
+            if (t == 0 && a.ds0) {
+                float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
+                jacT_mul(c, v0, v1, v2, v3);
+                float *q = a.ds0 + (size_t)b * 4 * d + jj;
+                q[0] = v0;
+                q[d] = v1;
+                q[2 * d] = v2;
+                q[3 * d] = v3;
+            }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        s_part[warp][e][lane] = dr[e];
+        s_part[warp][4 + e][lane] = dbs[e];
+    }
+    __syncthreads();
+    {
+        // 256 threads: thread (e, lane) sums entry e over the warps
+        const int e = threadIdx.x >> 5;  // 0..7
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) acc += s_part[w][e][lane];
+        a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
+    }
+}
+
+// dR[g][j] and db[g][j]: sum of the per-tile partials over chunks and batch
+// rows, in a fixed order, accumulated in fp64.
+__global__ void reduce_partials_kernel(const float *__restrict__ partial, float *__restrict__ dR,
+                                       float *__restrict__ db, int B, int n_chunks, int groups_per_row,
+                                       int d)
+{
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // over 8 * d
+    if (idx >= 8 * d) return;
+    const int e = idx / d;
+    const int j = idx % d;
+    const int jb = j / 32, lane = j % 32;
+    const int G = B * groups_per_row;
+    double acc = 0.0;
+    for (int c = 0; c < n_chunks; ++c)
+        for (int b = 0; b < B; ++b) {
+            const size_t ticket = (size_t)c * G + (size_t)b * groups_per_row + jb;
+            acc += partial[(ticket * 8 + e) * 32 + lane];
+        }
+    if (e < 4)
+        dR[(size_t)e * d + j] = (float)acc;
+    else
+        db[(size_t)(e - 4) * d + j] = (float)acc;
+}
+
+struct Layout {
+    size_t ticket, flags, agg, inc, partial, dP, total;
+    int groups_per_row, n_groups, n_chunks, n_tiles;
+};
+
+Layout layout(int B, int T, int d_h)
+{
+    Layout l;
+    l.groups_per_row = (d_h + 31) / 32;
+    l.n_groups = B * l.groups_per_row;
+    l.n_chunks = (T + TT - 1) / TT;
+    l.n_tiles = l.n_groups * l.n_chunks;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return at;
+    };
+    l.ticket = take(256);
+    l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles);
+    l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
+    l.inc = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
+    l.partial = take(sizeof(float) * 8 * 32 * (size_t)l.n_tiles);
+    l.dP = take(sizeof(float) * 4 * (size_t)B * T * d_h);
+    l.total = off;
+    return l;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int T, int d_in, int d_h)
+{
+    (void)d_in;
+    return layout(B, T, d_h).total;
+}
+
+cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *R,
+                            const float *s0, const float *S, const float *dH, float *dx, float *dWx,
+                            float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
+                            int d_h, void *ws, cudaStream_t st)
+{
+    const Layout l = layout(B, T, d_h);
+    char *base = static_cast<char *>(ws);
+    BwdArgs a;
+    a.P = P;
+    a.R = R;
+    a.s0 = s0;
+    a.S = S;
+    a.dH = dH;
+    a.dP = reinterpret_cast<float *>(base + l.dP);
+    a.partial = reinterpret_cast<float *>(base + l.partial);
+    a.ds0 = ds0;
+    a.ticket = reinterpret_cast<unsigned *>(base + l.ticket);
+    a.lb.flags = reinterpret_cast<unsigned *>(base + l.flags);
+    a.lb.agg = reinterpret_cast<float *>(base + l.agg);
+    a.lb.inc = reinterpret_cast<float *>(base + l.inc);
+    a.lb.error = a.ticket + 1;
+    a.lb.epoch = 1;
+    a.lb.wait_ns = 2000000000ull;
+    a.lb.n_groups = l.n_groups;
+    a.T = T;
+    a.d = d_h;
+    a.groups_per_row = l.groups_per_row;
+    cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
+    if (e != cudaSuccess) return e;
+    if (ds0 && !s0) {
+        // ds0 is still defined (the gradient at a zero initial state)
+    }
+    if (forget == SLSTM_FORGET_EXP)
+        adjoint_vjp_kernel<SLSTM_FORGET_EXP><<<l.n_tiles, NW * 32, 0, st>>>(a);
+    else
+        adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID><<<l.n_tiles, NW * 32, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    reduce_partials_kernel<<<(8 * d_h + 255) / 256, 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
+                                                                   l.groups_per_row, d_h);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const long long N4 = 4LL * d_h;
+    // dx[(b,t), k] = sum_{g,j} dP[(b,t), (g,j)] Wx[(g,j), k]
+    GemmDesc gx;
+    gx.M = B * T;
+    gx.N = d_in;
+    gx.K = (int)N4;
+    gx.A = a.dP;
+    gx.a_dtype = SLSTM_F32;
+    gx.sam = N4;
+    gx.sak = 1;
+    gx.B = Wx;
+    gx.b_dtype = dtype;
+    gx.sbk = d_in;
+    gx.sbn = 1;
+    gx.bias = nullptr;
+    gx.C = dx;
+    if ((e = gemm_simt(gx, st)) != cudaSuccess) return e;
+    // dWx[(g,j), k] = sum_{(b,t)} dP[(b,t), (g,j)] x[(b,t), k]
+    GemmDesc gw;
+    gw.M = (int)N4;
+    gw.N = d_in;
+    gw.K = B * T;
+    gw.A = a.dP;
+    gw.a_dtype = SLSTM_F32;
+    gw.sam = 1;
+    gw.sak = N4;
+    gw.B = x;
+    gw.b_dtype = dtype;
+    gw.sbk = d_in;
+    gw.sbn = 1;
+    gw.bias = nullptr;
+    gw.C = dWx;
+    return gemm_simt(gw, st);
+}
+
+}  // namespace slstm

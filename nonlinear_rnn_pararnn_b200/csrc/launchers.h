@@ -1,0 +1,68 @@
+// Internal launchers behind the C ABI in slstm_api.cu.  Arguments have been
+// validated by the caller; every launcher only enqueues work on `st`.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/slstm.h"
+
+namespace slstm {
+
+// Per-iteration counters; iteration k uses slot k & 1 and its finalizer
+// clears the other slot for iteration k + 1.
+struct NewtonSlot {
+    unsigned ticket;
+    unsigned finished;
+    unsigned maxF_raw;     // float bits of a non-negative max
+    unsigned maxF_scaled;
+};
+
+// Device-side control block of one slstm_newton_forward call.
+struct NewtonCtrl {
+    unsigned done;
+    unsigned error;
+    unsigned pad[14];
+    NewtonSlot slot[2];
+};
+
+size_t newton_workspace_bytes(int B, int T, int d);
+cudaError_t newton_forward(const float *P, const float *R, const float *s0, float *S,
+                           const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
+                           int d, void *ws, cudaStream_t st);
+
+size_t scan_workspace_bytes(int B, int T, int d);
+cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, float *y, int B,
+                               int T, int d, bool reverse, void *ws, cudaStream_t st);
+
+cudaError_t sequential_launch(const float *P, const float *R, const float *s0, float *S, int B,
+                              int T, int d, int forget, cudaStream_t st);
+
+size_t backward_workspace_bytes(int B, int T, int d_in, int d_h);
+cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *R,
+                            const float *s0, const float *S, const float *dH, float *dx, float *dWx,
+                            float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
+                            int d_h, void *ws, cudaStream_t st);
+
+// C[M][N] = sum_k A(m,k) B(k,n) (+ bias[n]) with fp32 accumulation.
+// A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn]; element types as
+// `dtype` (SLSTM_F32 / SLSTM_BF16) per operand.
+struct GemmDesc {
+    int M, N, K;
+    const void *A;
+    int a_dtype;
+    long long sam, sak;
+    const void *B;
+    int b_dtype;
+    long long sbk, sbn;
+    const float *bias;  // [N] or null
+    float *C;           // [M][N], row-major
+};
+cudaError_t gemm_simt(const GemmDesc &g, cudaStream_t st);
+
+// Input projection P = x Wx^T + bias on the tcgen05 tensor cores (bf16).
+size_t preact_workspace_bytes(int B, int T, int d_in, int d_h, int dtype);
+cudaError_t preact_launch(const void *x, const void *Wx, int dtype, const float *bias, float *P,
+                          int B, int T, int d_in, int d_h, void *ws, cudaStream_t st);
+
+}  // namespace slstm

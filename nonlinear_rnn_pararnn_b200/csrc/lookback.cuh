@@ -1,0 +1,178 @@
+// Blocked scan of 4x4 affine maps across CTAs with a decoupled look-back.
+//
+// A "tile" is 32 features x (NW warps x L steps).  Inside a tile every warp
+// folds its own L steps serially (one feature per lane); warp 0 then folds
+// the NW warp aggregates, publishes the tile aggregate, looks back over the
+// tiles before it (same feature group, earlier in processing order) until it
+// meets a published inclusive prefix, publishes its own inclusive prefix and
+// hands every warp its incoming carry through shared memory.
+//
+// Tiles take tickets from a global counter in the order CTAs start, and tile
+// (chunk c, group g) has ticket c * n_groups + g, so a tile only ever waits
+// on tiles that started before it: every wait ends.  Waits are bounded in
+// time anyway; on expiry the tile records an error, continues with a zero
+// carry and still publishes, so that no other tile waits on it.
+//
+// Global state per tile (ticket):  flag word, aggregate [20][32] and
+// inclusive prefix [4][32] (feature-contiguous so that a warp moves 128-byte
+// rows).
+#pragma once
+
+#include "common.cuh"
+
+namespace slstm {
+
+struct LookbackArgs {
+    unsigned *flags;   // [n_tiles]
+    float *agg;        // [n_tiles][20][32]
+    float *inc;        // [n_tiles][4][32]
+    unsigned *error;   // set to nonzero when a wait expires
+    unsigned epoch;    // nonzero, unique per launch since the flags were cleared
+    uint64_t wait_ns;  // bound of one wait
+    int n_groups;      // feature groups (tiles per chunk)
+};
+
+// Called by warp 0 only, after every warp wrote its aggregate (in processing
+// order) to s_agg[w][0..19][lane].  Writes the carry entering each warp to
+// s_carry[w][0..3][lane].  `first_carry` is the value entering chunk 0.
+// `withhold` suppresses this tile's publications (fault injection).
+template <int NW>
+SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_carry)[4][32],
+                                      const LookbackArgs &lb, unsigned ticket, int chunk,
+                                      const float first_carry[4], bool withhold)
+{
+    const int lane = threadIdx.x & 31;
+    Aff tile;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) tile.a[e] = s_agg[0][e][lane];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) tile.b[e] = s_agg[0][16 + e][lane];
+    for (int w = 1; w < NW; ++w) {
+        Aff x;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x.a[e] = s_agg[w][e][lane];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x.b[e] = s_agg[w][16 + e][lane];
+        aff_compose(x, tile, tile);
+    }
+
+    float carry[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) carry[e] = first_carry[e];
+
+    if (chunk > 0) {
+        if (!withhold) {
+            float *dst = lb.agg + (size_t)ticket * 20 * 32;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release(lb.flags + ticket, (lb.epoch << 2) | FLAG_AGG);
+        }
+        Aff M;  // composition of the aggregates met so far (latest first)
+        aff_identity(M);
+        int q = chunk - 1;
+        bool expired = false;
+        for (;;) {
+            const unsigned tq = (unsigned)q * (unsigned)lb.n_groups + (ticket % (unsigned)lb.n_groups);
+            unsigned st = 0;
+            if (lane == 0) st = wait_flag(lb.flags + tq, lb.epoch, lb.wait_ns);
+            st = __shfl_sync(0xffffffffu, st, 0);
+            if (st == 0u) {
+                expired = true;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) carry[e] = 0.0f;
+                break;
+            }
+            if (st == FLAG_INC) {
+                float v[4];
+                const float *src = lb.inc + (size_t)tq * 4 * 32;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v[e] = __ldcg(src + e * 32 + lane);
+                aff_apply(M, v, carry);
+                break;
+            }
+            Aff x;
+            const float *src = lb.agg + (size_t)tq * 20 * 32;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+            aff_compose(M, x, M);
+            --q;  // chunk 0 always publishes an inclusive prefix, so q stays >= 0
+        }
+        if (expired && lane == 0) atomicOr(lb.error, 1u);
+    }
+
+    if (!withhold) {
+        float incv[4];
+        aff_apply(tile, carry, incv);
+        float *dst = lb.inc + (size_t)ticket * 4 * 32;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = incv[e];
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release(lb.flags + ticket, (lb.epoch << 2) | FLAG_INC);
+    }
+
+    // carries entering each warp of this tile
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = carry[e];
+    for (int w = 0; w < NW; ++w) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_carry[w][e][lane] = v[e];
+        if (w + 1 < NW) {
+            Aff x;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x.a[e] = s_agg[w][e][lane];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x.b[e] = s_agg[w][16 + e][lane];
+            aff_apply(x, v, v);
+        }
+    }
+}
+
+// Fold one step's map (J, r) into a running aggregate: agg <- (J, r) o agg.
+SLSTM_DEVINL void fold_jac(Aff &agg, const Cell &J, const float r[4])
+{
+#pragma unroll
+    for (int col = 0; col < 4; ++col)
+        jac_mul(J, agg.a[col], agg.a[4 + col], agg.a[8 + col], agg.a[12 + col]);
+    jac_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
+}
+
+// Same with the transposed Jacobian: agg <- (J^T, r) o agg.
+SLSTM_DEVINL void fold_jacT(Aff &agg, const Cell &J, const float r[4])
+{
+#pragma unroll
+    for (int col = 0; col < 4; ++col)
+        jacT_mul(J, agg.a[col], agg.a[4 + col], agg.a[8 + col], agg.a[12 + col]);
+    jacT_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
+}
+
+SLSTM_DEVINL void cell_identity(Cell &J)
+{
+    J.fp = 1.0f;
+    J.jcm = J.jch = J.jnm = J.jnh = 0.0f;
+    J.beta = 1.0f;
+    J.dmh = 0.0f;
+    J.jhc = J.jhn = J.jhm = 0.0f;
+    J.jhh = 1.0f;
+}
+
+SLSTM_DEVINL void store_aff_smem(float (*s_agg)[20][32], int w, int lane, const Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) s_agg[w][e][lane] = x.a[e];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s_agg[w][16 + e][lane] = x.b[e];
+}
+
+}  // namespace slstm

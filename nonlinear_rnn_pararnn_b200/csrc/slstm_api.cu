@@ -1,0 +1,141 @@
+// extern "C" entry points of libslstm.so (declared in include/slstm.h).
+// Host-side validation happens here, before anything is enqueued; the
+// launchers in launchers.h do the work.
+#include <stdint.h>
+
+#include "launchers.h"
+
+using namespace slstm;
+
+namespace {
+
+constexpr long long kIndexLimit = (1LL << 31) - 1;
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned16_or_null(const void *p) { return p == nullptr || aligned16(p); }
+bool aligned256(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// Element offsets are 64-bit everywhere; the limits keep B*T (a GEMM row
+// count), grid sizes and tile tickets inside 32 bits.
+bool sizes_ok(int B, int T, int d_a, int d_b)
+{
+    if (B < 1 || T < 1 || d_a < 1 || d_b < 1) return false;
+    if (B > 65535 || d_a > (1 << 20) || d_b > (1 << 20)) return false;
+    if ((long long)B * T > kIndexLimit) return false;
+    const long long w = (d_a > d_b ? d_a : d_b);
+    const long long tiles = (long long)B * ((T + 31) / 32) * ((w + 31) / 32);
+    return tiles <= kIndexLimit;
+}
+
+bool ws_ok(void *ws, size_t have, size_t need)
+{
+    if (need == 0) return true;
+    return aligned256(ws) && have >= need;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SLSTM_OK : SLSTM_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *slstm_status_string(int status)
+{
+    switch (status) {
+    case SLSTM_OK: return "SLSTM_OK";
+    case SLSTM_ERR_INVALID_ARG: return "SLSTM_ERR_INVALID_ARG";
+    case SLSTM_ERR_CUDA: return "SLSTM_ERR_CUDA";
+    case SLSTM_ERR_DIVERGED: return "SLSTM_ERR_DIVERGED";
+    case SLSTM_ERR_TIMEOUT: return "SLSTM_ERR_TIMEOUT";
+    case SLSTM_ERR_UNSUPPORTED: return "SLSTM_ERR_UNSUPPORTED";
+    default: return "SLSTM_UNKNOWN_STATUS";
+    }
+}
+
+size_t slstm_workspace_size(int op, int B, int T, int d_in, int d_h)
+{
+    switch (op) {
+    case SLSTM_OP_PREACT_GEMM:
+        if (!sizes_ok(B, T, d_in, d_h)) return 0;
+        return preact_workspace_bytes(B, T, d_in, d_h, SLSTM_BF16);
+    case SLSTM_OP_NEWTON_FORWARD:
+        if (!sizes_ok(B, T, d_h, d_h)) return 0;
+        return newton_workspace_bytes(B, T, d_h);
+    case SLSTM_OP_SCAN_BLOCK4:
+        if (!sizes_ok(B, T, d_h, d_h)) return 0;
+        return scan_workspace_bytes(B, T, d_h);
+    case SLSTM_OP_NEWTON_BACKWARD:
+        if (!sizes_ok(B, T, d_in, d_h)) return 0;
+        return backward_workspace_bytes(B, T, d_in, d_h);
+    default: return 0;
+    }
+}
+
+int slstm_preact_gemm(const void *x, const void *Wx, int dtype, const float *bias, float *P, int B,
+                      int T, int d_in, int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (dtype != SLSTM_F32 && dtype != SLSTM_BF16) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_in, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (dtype == SLSTM_BF16 && d_in % 8 != 0) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wx) || !aligned16(bias) || !aligned16(P)) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, preact_workspace_bytes(B, T, d_in, d_h, dtype))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(preact_launch(x, Wx, dtype, bias, P, B, T, d_in, d_h, ws,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_newton_forward(const float *P, const float *R, const float *s0, float *S,
+                         const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
+                         int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (cfg == nullptr) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
+        return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, newton_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(newton_forward(P, R, s0, S, *cfg, stats, B, T, d_h, ws,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int scan_block4(const float *A, const float *b, const float *y0, float *y, int B, int T, int d,
+                int flags, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if ((flags & ~SLSTM_SCAN_REVERSE_T) != 0) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d, d)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(b) || !aligned16_or_null(y0) || !aligned16(y)) return SLSTM_ERR_INVALID_ARG;
+    if (y == A || y == b) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, scan_workspace_bytes(B, T, d))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(scan_block4_launch(A, b, y0, y, B, T, d, (flags & SLSTM_SCAN_REVERSE_T) != 0, ws,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_sequential_step(const float *P, const float *R, const float *s0, float *S, int B,
+                          int T_steps, int d_h, int forget, slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T_steps, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S)) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(sequential_launch(P, R, s0, S, B, T_steps, d_h, forget,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_newton_backward(const void *x, const void *Wx, int dtype, const float *P, const float *R,
+                          const float *s0, const float *S, const float *dH, float *dx, float *dWx,
+                          float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
+                          int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (dtype != SLSTM_F32 && dtype != SLSTM_BF16) return SLSTM_ERR_INVALID_ARG;
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_in, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wx) || !aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) ||
+        !aligned16(S) || !aligned16(dH) || !aligned16(dx) || !aligned16(dWx) || !aligned16(dR) ||
+        !aligned16(db) || !aligned16_or_null(ds0))
+        return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, backward_workspace_bytes(B, T, d_in, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(backward_launch(x, Wx, dtype, P, R, s0, S, dH, dx, dWx, dR, db, ds0, forget, B, T,
+                                       d_in, d_h, ws, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""C-ABI boundary checks that need no GPU: the library builds and loads, it
+exports every function include/slstm.h declares, and host-side validation
+rejects bad arguments before anything is enqueued (these calls never reach
+the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nonlinear_rnn_pararnn_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+FAKE = ctypes.c_void_p(0x10000)          # 16-byte aligned, never dereferenced
+FAKE_MIS = ctypes.c_void_p(0x10004)      # misaligned
+NULL = ctypes.c_void_p(0)
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([A-Za-z_]\w*)\s*\(", text, flags=re.M):
+            if m.group(1) not in ("if", "while", "sizeof", "defined"):
+                names.append(m.group(1))
+    return names
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    assert "slstm_newton_forward" in names and "scan_block4" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    # the binding covers exactly the declared set
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_status_strings():
+    lib = _lib.load()
+    assert lib.slstm_status_string(0) == b"SLSTM_OK"
+    assert lib.slstm_status_string(1) == b"SLSTM_ERR_INVALID_ARG"
+    assert lib.slstm_status_string(4) == b"SLSTM_ERR_TIMEOUT"
+    assert lib.slstm_status_string(99) == b"SLSTM_UNKNOWN_STATUS"
+
+
+def test_workspace_sizes():
+    lib = _lib.load()
+    small = lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD, 2, 64, 8, 8)
+    big = lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD, 4, 65536, 2048, 2048)
+    assert 0 < small < big
+    assert big < 8 * 1024 ** 3
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_SCAN_BLOCK4, 2, 100, 0, 40) > 0
+    bwd = lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_BACKWARD, 2, 64, 8, 8)
+    assert bwd >= 2 * 64 * 4 * 8 * 4  # holds dP
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD, 0, 64, 8, 8) == 0
+    assert lib.slstm_workspace_size(77, 2, 64, 8, 8) == 0
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD, 70000, 64, 8, 8) == 0
+
+
+def _cfg(**kw):
+    base = dict(max_iters=4, fixed_iters=0, tol=1e-5, forget=0, debug_fault=0, wait_limit_us=0)
+    base.update(kw)
+    return _lib.NewtonConfig(**base)
+
+
+def test_newton_forward_rejects_bad_arguments():
+    lib = _lib.load()
+    E = _lib.SLSTM_ERR_INVALID_ARG
+    ws = FAKE
+    big = ctypes.c_size_t(1 << 40)
+
+    def call(P=FAKE, R=FAKE, s0=NULL, S=FAKE, cfg=None, stats=FAKE, B=2, T=64, d=8, w=ws, wb=big):
+        c = cfg if cfg is not None else _cfg()
+        return lib.slstm_newton_forward(P, R, s0, S, ctypes.byref(c), stats, B, T, d, w, wb, NULL)
+
+    assert call(B=0) == E
+    assert call(T=0) == E
+    assert call(d=-1) == E
+    assert call(P=NULL) == E
+    assert call(S=FAKE_MIS) == E
+    assert call(s0=FAKE_MIS) == E
+    assert call(stats=NULL) == E
+    assert call(cfg=_cfg(max_iters=0)) == E
+    assert call(cfg=_cfg(max_iters=65537)) == E
+    assert call(cfg=_cfg(forget=2)) == E
+    assert call(cfg=_cfg(tol=float("nan"))) == E
+    assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
+    assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
+    assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E
+
+
+def test_other_entry_points_reject_bad_arguments():
+    lib = _lib.load()
+    E = _lib.SLSTM_ERR_INVALID_ARG
+    big = ctypes.c_size_t(1 << 40)
+    assert lib.scan_block4(FAKE, FAKE, NULL, FAKE, 2, 100, 0, 0, FAKE, big, NULL) == E
+    assert lib.scan_block4(FAKE, FAKE, NULL, FAKE, 2, 100, 40, 2, FAKE, big, NULL) == E   # unknown flag
+    assert lib.scan_block4(FAKE, FAKE, NULL, FAKE, 2, 100, 40, 0, FAKE, big, NULL) == E   # y aliases A
+    assert lib.slstm_sequential_step(FAKE, FAKE, NULL, FAKE, 2, 0, 8, 0, NULL) == E
+    assert lib.slstm_sequential_step(FAKE, FAKE, NULL, FAKE, 2, 8, 8, 3, NULL) == E
+    assert lib.slstm_preact_gemm(FAKE, FAKE, 7, FAKE, FAKE, 2, 8, 8, 8, FAKE, big, NULL) == E
+    assert lib.slstm_preact_gemm(FAKE, FAKE, _lib.SLSTM_BF16, FAKE, FAKE, 2, 8, 6, 8, FAKE, big, NULL) == E
+    assert lib.slstm_preact_gemm(FAKE_MIS, FAKE, 0, FAKE, FAKE, 2, 8, 8, 8, FAKE, big, NULL) == E
+    args = [FAKE] * 13
+    assert lib.slstm_newton_backward(args[0], args[1], 0, *args[2:12], 0, 2, 0, 8, 8, FAKE, big, NULL) == E
+    assert lib.slstm_newton_backward(args[0], args[1], 5, *args[2:12], 0, 2, 8, 8, 8, FAKE, big, NULL) == E
+
+
+def test_python_binding_validates_before_calling():
+    import torch
+    from nonlinear_rnn_pararnn_b200 import api
+    P = torch.zeros(2, 8, 4, 8)
+    with pytest.raises(ValueError):
+        api.newton_forward(P, torch.zeros(4, 8))     # CPU tensors are refused

@@ -1,0 +1,227 @@
+"""GPU parity: every C-ABI entry point against the fp64 CPU oracle on the same
+seeded inputs, at sizes the oracle finishes in seconds that still span
+several tiles (32 steps x 32 features) and ragged tails in both time and
+features.
+
+Tolerances: max|dh| <= 1e-4 (1 + |h|) for fp32 inputs and <= 5e-3 (1 + |h|)
+for bf16 inputs (the oracle reads the same bf16-rounded values, widened
+exactly).  Gradients: max|dg| <= 1e-4 (1 + max|g|) per tensor for fp32
+inputs; scans: 1e-5 relative to the solution's scale.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nonlinear_rnn_pararnn_b200 import api
+from nonlinear_rnn_pararnn_b200.workloads import WORKLOADS, Workload, as_f64, make_inputs, scaled
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_BF16 = 5e-3
+
+
+def _dev(t):
+    return None if t is None else t.to("cuda").contiguous()
+
+
+def _h_err(S_gpu, S_ref):
+    h = S_ref[:, :, 3, :]
+    return float((np.abs(S_gpu[:, :, 3, :] - h) / (1 + np.abs(h))).max())
+
+
+# ---------------------------------------------------------------------------
+# scan_block4
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,T,d", [(2, 100, 40), (1, 1, 1), (3, 33, 32), (1, 3000, 64)])
+@pytest.mark.parametrize("reverse", [False, True])
+@pytest.mark.parametrize("with_y0", [False, True])
+def test_scan_block4_matches_sequential_solve(B, T, d, reverse, with_y0, cuda_device):
+    g = torch.Generator().manual_seed(1000 + B * T + d)
+    A = (torch.rand(B, T, 4, 4, d, generator=g) * 0.6 - 0.3)
+    b = torch.randn(B, T, 4, d, generator=g)
+    y0 = torch.randn(B, 4, d, generator=g) if with_y0 else None
+    y = api.scan_block4(_dev(A), _dev(b), _dev(y0), reverse=reverse)
+    torch.cuda.synchronize()
+    Al = np.transpose(as_f64(A), (0, 4, 1, 2, 3)).reshape(B * d, T, 4, 4)
+    bl = np.transpose(as_f64(b), (0, 3, 1, 2)).reshape(B * d, T, 4)
+    y0l = None if y0 is None else np.transpose(as_f64(y0), (0, 2, 1)).reshape(B * d, 4)
+    ref = oracle.affine_solve(Al, bl, y0l, reverse=reverse)
+    ref = np.transpose(ref.reshape(B, d, T, 4), (0, 2, 3, 1))
+    err = np.abs(as_f64(y.cpu()) - ref).max() / (1 + np.abs(ref).max())
+    assert err < 1e-5, err
+
+
+# ---------------------------------------------------------------------------
+# sequential step
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("B,T,d", [(2, 64, 8), (3, 200, 130), (1, 1, 5)])
+def test_sequential_step_matches_oracle(forget, B, T, d, cuda_device):
+    w = Workload("t", B, T, 8, d, "f32", forget, 0.5, 7, 1e-6, 64)
+    inp = make_inputs(w, with_dH=False)
+    g = torch.Generator().manual_seed(5)
+    s0 = torch.stack([torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) + 0.5,
+                      torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) - 0.5], dim=1)
+    P = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    S = api.sequential_step(_dev(torch.from_numpy(P).float()), _dev(inp["R"]), _dev(s0), forget=forget)
+    ref = oracle.sequential_btgd(as_f64(torch.from_numpy(P).float()), as_f64(inp["R"]), as_f64(s0), forget)
+    assert _h_err(as_f64(S.cpu()), ref) <= TOL_F32
+
+
+# ---------------------------------------------------------------------------
+# input projection
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T,d_in,d_h", [(2, 64, 8, 8), (3, 50, 24, 40), (2, 300, 64, 96)])
+def test_preact_gemm_matches_oracle(dtype, B, T, d_in, d_h, cuda_device):
+    w = Workload("t", B, T, d_in, d_h, dtype, "sigmoid", 0.5, 3, 1e-6, 64)
+    inp = make_inputs(w, with_dH=False)
+    P = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    ref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    err = np.abs(as_f64(P.cpu()) - ref).max() / (1 + np.abs(ref).max())
+    assert err < 1e-5, err
+
+
+# ---------------------------------------------------------------------------
+# Newton forward
+# ---------------------------------------------------------------------------
+def _newton_case(w: Workload, fixed_k=None):
+    inp = make_inputs(w, with_dH=False)
+    Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    if fixed_k is None:
+        S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
+                                   max_iters=w.max_iters, fixed=False, tol=w.tol)
+    else:
+        S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
+                                   max_iters=fixed_k, fixed=True, tol=w.tol)
+    stats = api.read_stats(st)
+    Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    return inp, as_f64(S.cpu()), stats, Pref
+
+
+def _check_status_against_oracle(st, ost):
+    """A GPU run either converges (and then the fp64 run converged too) or it
+    stops on a non-finite or large residual; in that case the exact-arithmetic
+    iterate at the same iteration was also far from converged (scaled
+    residual > 1), so the stop is the method's behaviour from the zero guess,
+    not an artefact of the kernels."""
+    if st["converged"]:
+        assert ost["converged"], (st, ost)
+        return True
+    assert st["diverged"] and st["error"] == 3, st
+    k = st["iters"] - 1
+    hist = list(ost["max_scaled_F"])
+    assert k < len(hist) and not (hist[k] <= 1.0), (st, hist[: k + 1])
+    return False
+
+
+def test_newton_tiny_converges_to_sequential(cuda_device):
+    w = WORKLOADS["tiny_f32"]
+    inp, S, st, Pref = _newton_case(w)
+    ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol)
+    print("gpu stats", st, "oracle iters", ost["iters"])
+    assert st["error"] == 0 and not st["diverged"]
+    assert st["converged"]
+    assert abs(st["iters"] - ost["iters"]) <= 1
+    assert _h_err(S, ref) <= TOL_F32
+    # the residual history of the first iterates agrees with the fp64 run
+    for k in range(3):
+        g, o = st["max_scaled_F"][k], ost["max_scaled_F"][k]
+        assert abs(g - o) <= 1e-3 * (1 + o), (k, g, o)
+
+
+@pytest.mark.parametrize("B,T,d", [(2, 50, 40), (1, 1, 1), (2, 31, 33), (3, 64, 70)])
+def test_newton_converges_to_sequential_sigmoid(B, T, d, cuda_device):
+    w = Workload("t", B, T, 16, d, "f32", "sigmoid", 0.5, 11, 1e-6, 64)
+    inp, S, st, Pref = _newton_case(w)
+    ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), "sigmoid")
+    assert st["error"] == 0 and st["converged"], st
+    assert _h_err(S, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256)])
+def test_newton_status_agrees_with_oracle(forget, B, T, d, cuda_device):
+    w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
+    inp, S, st, Pref = _newton_case(w)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol)
+    if _check_status_against_oracle(st, ost):
+        ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget)
+        assert _h_err(S, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_newton_fixed_k_prefix_exact(K, cuda_device):
+    """After K Newton iterations the first K steps equal the sequential
+    trajectory whatever the rest of the iterate looks like."""
+    w = WORKLOADS["slstm_f32_b8_t1024_d256"]
+    inp, S, st, Pref = _newton_case(w, fixed_k=K)
+    assert st["iters"] == K
+    ref = oracle.sequential_btgd(Pref[:, :K], as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
+    assert _h_err(S[:, :K], ref) <= TOL_F32
+
+
+def test_newton_stats_divergence_on_nan(cuda_device):
+    P = torch.full((1, 40, 4, 8), float("nan"), device="cuda")
+    S, st = api.newton_forward(P, torch.zeros(4, 8, device="cuda"), max_iters=3, fixed=False, tol=1e-5)
+    s = api.read_stats(st)
+    assert s["diverged"] and not s["converged"] and s["error"] == 3
+    assert s["iters"] == 1      # a non-finite residual stops the run at once
+
+
+def test_newton_cap_beyond_history(cuda_device):
+    """More iterations than the 64-entry residual history: the run still
+    converges and the record keeps the last 64 residuals."""
+    w = Workload("t", 2, 64, 16, 32, "f32", "sigmoid", 0.5, 11, 1e-30, 100)
+    inp = make_inputs(w, with_dH=False)
+    Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    S, st = api.newton_forward(Pt, _dev(inp["R"]), None, max_iters=100, fixed=True, tol=1e-6)
+    s = api.read_stats(st)
+    assert s["iters"] == 100 and s["converged"]
+    assert len(s["max_scaled_F"]) == 64 and s["history_first_iter"] == 36
+    assert s["max_scaled_F"][-1] <= 1e-6 and s["max_scaled_F"][0] == -1.0
+
+
+def test_newton_bounded_wait_reports_timeout(cuda_device):
+    """Fault injection on the host's request: one tile withholds its carry;
+    its successor's bounded wait expires and the run reports a timeout
+    instead of hanging."""
+    w = Workload("t", 1, 128, 8, 32, "f32", "sigmoid", 0.5, 1, 1e-6, 4)
+    inp = make_inputs(w, with_dH=False)
+    Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    S, st = api.newton_forward(Pt, _dev(inp["R"]), None, max_iters=2, fixed=True, tol=1e-6,
+                               debug_fault=1, wait_limit_us=20000)
+    s = api.read_stats(st)
+    assert s["error"] == 4, s
+    # the context is still usable afterwards
+    S2, st2 = api.newton_forward(Pt, _dev(inp["R"]), None, max_iters=64, fixed=False, tol=1e-6)
+    assert api.read_stats(st2)["converged"]
+
+
+# ---------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("B,T,d_in,d", [(2, 64, 8, 8), (2, 75, 12, 40)])
+def test_backward_matches_oracle_bptt(forget, B, T, d_in, d, cuda_device):
+    w = Workload("t", B, T, d_in, d, "f32", forget, 0.5, 13, 1e-6, 64)
+    inp = make_inputs(w, with_dH=True)
+    g = torch.Generator().manual_seed(9)
+    s0 = torch.stack([torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) + 0.5,
+                      torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) - 0.5], dim=1)
+    x, Wx, R = _dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["R"])
+    Pt = api.preact_gemm(x, Wx, _dev(inp["bias"]))
+    S = api.sequential_step(Pt, R, _dev(s0), forget=forget)
+    out = api.newton_backward(x, Wx, Pt, R, _dev(s0), S, _dev(inp["dH"]), forget=forget)
+    torch.cuda.synchronize()
+    Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    Sref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(s0), forget)
+    ref = oracle.backward_btgd(as_f64(inp["x"]), as_f64(inp["Wx"]), Pref, as_f64(inp["R"]), as_f64(s0), Sref,
+                               as_f64(inp["dH"]), forget)
+    for k in ("dx", "dWx", "dR", "db", "ds0"):
+        got = as_f64(out[k].cpu())
+        err = np.abs(got - ref[k]).max() / (1 + np.abs(ref[k]).max())
+        assert err <= 1e-4, (k, err)
