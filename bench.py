@@ -1,0 +1,337 @@
+#!/usr/bin/env python
+"""Benchmark of the Newton-solved diag-mix sLSTM training step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--newton-iters K_N] [--impl reference]
+
+One step = the whole hot path on one batch of synthetic input already in HBM:
+  input projection GEMM  ->  K_N fixed Newton iterations (fused residual,
+  Jacobian, blocked scan, update)  ->  backward (fused adjoint scan + cell
+  VJP, dR/db reduction, dx and dW_x GEMMs).
+Metric: B*T*d_h elements per second for forward + backward (the JSON
+`value`), with the forward alone reported beside it.  Under torchrun each
+rank runs its own replica of the workload (independent batches, no data-path
+collective): `value` is the sum over ranks of elements divided by the slowest
+rank's device time.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of lanes of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from nonlinear_rnn_pararnn_b200.workloads import ORDER, WORKLOADS, as_f64, make_inputs  # noqa: E402
+
+METRIC = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd+bwd)"
+UNIT = "elems/s"
+DEFAULT_WORKLOAD = "slstm_bf16_train_b8_t8192_d1024"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline leg and --impl reference)
+# ---------------------------------------------------------------------------
+def oracle_sample(w, inp, n_lanes, newton_iters, seed=0):
+    """Run the fp64 oracle, as it stands, on n_lanes (b, j) lanes of the
+    workload: input projection rows, K fixed Newton iterations, BPTT and the
+    lanes' contributions to dx and dW_x.  Returns (seconds, elements)."""
+    import oracle
+    rng = np.random.default_rng(seed)
+    lanes = [(int(rng.integers(0, w.B)), int(rng.integers(0, w.d_h))) for _ in range(n_lanes)]
+    bias = as_f64(inp["bias"])
+    t0 = time.perf_counter()
+    for b, j in lanes:
+        xb = as_f64(inp["x"][b])                                        # (T, d_in)
+        rows = [g * w.d_h + j for g in range(4)]
+        Wr = as_f64(inp["Wx"][rows])                                    # (4, d_in)
+        P = oracle.gemm(xb, Wr, tb=True, bias=bias[:, j])[None]         # (1, T, 4)
+        R = as_f64(inp["R"][:, j])[None]
+        s0 = np.zeros((1, 4))
+        S, _ = oracle.newton(P, R, s0, w.forget, max_iters=newton_iters, fixed=True, tol=w.tol)
+        dH = as_f64(inp["dH"][b, :, j])[None]
+        dP, dR, db, ds0 = oracle.bptt(P, R, s0, S, dH, w.forget)
+        oracle.gemm(dP[0], Wr)                                          # this lane's share of dx
+        oracle.gemm(np.ascontiguousarray(dP[0].T), np.ascontiguousarray(xb.T), tb=True)  # its dW_x rows
+    dt = time.perf_counter() - t0
+    return dt, n_lanes * w.T
+
+
+def run_reference(args, w):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    inp = make_inputs(w)
+    t_lane = 0.0
+    for _ in range(args.warmup):
+        t_lane, _ = oracle_sample(w, inp, 1, args.newton_iters, seed=99)
+    # bounded sample: about a minute of CPU work over all timed steps
+    lanes_per_step = int(max(1, min(args.ref_lanes, 60.0 / max(1e-3, args.steps * t_lane))))
+    total_t, total_e = 0.0, 0
+    for s in range(args.steps):
+        dt, el = oracle_sample(w, inp, lanes_per_step, args.newton_iters, seed=s)
+        total_t += dt
+        total_e += el
+    value = total_e / total_t
+    sample = (f"{lanes_per_step} random (b,j) lanes x T={w.T} per step: fp64 input-projection rows, "
+              f"{args.newton_iters} fixed Newton iterations, BPTT, dx/dW_x contributions")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(w.describe(), newton_iters=args.newton_iters, newton_mode="fixed"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(gpu_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if ws > 1 else 0)
+    torch.cuda.set_device(dev)
+    api._lib.load()
+
+    K = args.newton_iters
+    inp = make_inputs(w)
+    x, Wx, R, bias, s0, dH = (inp[k].to(dev) for k in ("x", "Wx", "R", "bias", "s0", "dH"))
+    P = torch.empty(w.B, w.T, 4, w.d_h, device=dev)
+    S = torch.empty_like(P)
+    stats = api.new_stats(dev)
+    ws_n = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
+    ws_b = api.workspace(_lib.SLSTM_OP_NEWTON_BACKWARD, w.B, w.T, w.d_in, w.d_h, dev)
+    grads = {"dx": torch.empty(w.B, w.T, w.d_in, device=dev), "dWx": torch.empty(4 * w.d_h, w.d_in, device=dev),
+             "dR": torch.empty(4, w.d_h, device=dev), "db": torch.empty(4, w.d_h, device=dev),
+             "ds0": torch.empty(w.B, 4, w.d_h, device=dev)}
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        api.preact_gemm(x, Wx, bias, P=P)
+        if ev is not None:
+            ev[1].record()
+        api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, fixed=True, tol=w.tol, S=S, stats=stats, ws=ws_n)
+        if ev is not None:
+            ev[2].record()
+        api.newton_backward(x, Wx, P, R, s0, S, dH, forget=w.forget, out=grads, ws=ws_b)
+        if ev is not None:
+            ev[3].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    time.sleep(0.25)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for s_ in range(args.steps):
+        step(evs[s_])
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms_total = start.elapsed_time(end)
+    ms_gemm = sum(e[0].elapsed_time(e[1]) for e in evs)
+    ms_newton = sum(e[1].elapsed_time(e[2]) for e in evs)
+    ms_bwd = sum(e[2].elapsed_time(e[3]) for e in evs)
+    st = api.read_stats(stats)
+
+    # ---- end to end through the public API from pinned host buffers ----
+    host_in = {k: inp[k].pin_memory() for k in ("x", "Wx", "R", "bias", "s0", "dH")}
+    dev_in = {"x": x, "Wx": Wx, "R": R, "bias": bias, "s0": s0, "dH": dH}
+    host_out = {k: torch.empty(grads[k].shape, dtype=grads[k].dtype).pin_memory() for k in ("dWx", "dR", "db")}
+    host_stats = torch.empty(stats.shape, dtype=stats.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + host_stats.numel()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        step()
+        for k, t in host_out.items():
+            t.copy_(grads[k], non_blocking=True)
+        host_stats.copy_(stats, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.steps, 20))
+    e_start.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e_end.record()
+    torch.cuda.synchronize()
+    ms_e2e = e_start.elapsed_time(e_end) / e2e_steps
+
+    # max over ranks of the device times
+    vals = torch.tensor([ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd], device=dev, dtype=torch.float64)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd = vals.tolist()
+    ms_step = ms_total / args.steps
+    elems = w.elems
+    value = ws * elems / (ms_step / 1e3)
+    fwd_ms = (ms_gemm + ms_newton) / args.steps
+
+    hbm, peak_kind = _peaks()
+    newton_launch_ms = ms_newton / args.steps / K
+    # algorithmic bytes of one Newton launch: iteration 1 reads P and writes S
+    # (32 B/elem); later ones also read the old S (48 B/elem).  Averaged over
+    # the K launches of a step.
+    newton_bytes = elems * (32 + 48 * (K - 1)) / K
+    achieved = newton_bytes / (newton_launch_ms / 1e3) / 1e9
+    roofline = {"kernel": "newton_iter", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": args.traffic_bytes if args.traffic_bytes else None,
+                "algorithmic_bytes_per_launch": newton_bytes, "avg_launch_ms": newton_launch_ms}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        oracle_sample(w, inp, 1, K, seed=123)              # warm the oracle library
+        dt, el = oracle_sample(w, inp, args.cpu_lanes, K)
+        cpu = {"value": el / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{args.cpu_lanes} random (b,j) lanes x T={w.T}: fp64 input-projection rows, {K} fixed "
+                         f"Newton iterations, BPTT, dx/dW_x contributions ({dt:.1f} s, single thread)"}
+
+    # kernels launched per step: preact GEMM 1, Newton K, backward: adjoint 1 + reduce 1 + 2 GEMMs
+    launches_per_step = 1 + K + 4
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "operand_dtype": "bf16 x/W_x, fp32 state and scans" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": dict(w.describe(), newton_iters=K, newton_mode="fixed",
+                       l2="inputs larger than L2 (P and S are %.2f GB each)" % (elems * 16 / 1e9),
+                       parallelism=f"replicas x{ws}"),
+        "fwd": {"value": ws * elems / (fwd_ms / 1e3), "unit": UNIT, "ms_per_step": fwd_ms},
+        "breakdown_ms_per_step": {"preact_gemm": ms_gemm / args.steps, "newton_forward": ms_newton / args.steps,
+                                  "backward": ms_bwd / args.steps},
+        "newton_stats_last_step": {"iters": st["iters"], "diverged": st["diverged"], "error": st["error"]},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": ws * elems / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=ORDER)
+    ap.add_argument("--newton-iters", type=int, default=4)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-lanes", type=int, default=40)
+    ap.add_argument("--ref-lanes", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="ncu dram read+write bytes per Newton launch, when captured for this build")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    w = WORKLOADS[args.workload]
+    ws, _, _ = _dist()
+    if ws != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
