@@ -56,6 +56,22 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of timings over all ranks (identity when
+    not distributed).  Only timings cross ranks, never data."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate(elems_per_rank, n_ranks, ms_per_step_max):
+    """Whole-job throughput: every rank's elements over the slowest rank's time."""
+    return n_ranks * elems_per_rank / (ms_per_step_max / 1e3)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle sample (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
@@ -250,13 +266,11 @@ def run_gpu(args, w):
     ms_e2e = e_start.elapsed_time(e_end) / e2e_steps
 
     # max over ranks of the device times
-    vals = torch.tensor([ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd], device=dev, dtype=torch.float64)
-    if ws > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd = vals.tolist()
+    ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd = max_over_ranks(
+        [ms_total, ms_e2e, ms_gemm, ms_newton, ms_bwd], device=dev)
     ms_step = ms_total / args.steps
     elems = w.elems
-    value = ws * elems / (ms_step / 1e3)
+    value = aggregate(elems, ws, ms_step)
     fwd_ms = (ms_gemm + ms_newton) / args.steps
 
     hbm, peak_kind = _peaks()
@@ -289,13 +303,13 @@ def run_gpu(args, w):
         "config": dict(w.describe(), newton_iters=K, newton_mode="fixed",
                        l2="inputs larger than L2 (P and S are %.2f GB each)" % (elems * 16 / 1e9),
                        parallelism=f"replicas x{ws}"),
-        "fwd": {"value": ws * elems / (fwd_ms / 1e3), "unit": UNIT, "ms_per_step": fwd_ms},
+        "fwd": {"value": aggregate(elems, ws, fwd_ms), "unit": UNIT, "ms_per_step": fwd_ms},
         "breakdown_ms_per_step": {"preact_gemm": ms_gemm / args.steps, "newton_forward": ms_newton / args.steps,
                                   "backward": ms_bwd / args.steps},
         "newton_stats_last_step": {"iters": st["iters"], "diverged": st["diverged"], "error": st["error"]},
         "roofline": roofline,
         "cpu_baseline": cpu,
-        "e2e": {"value": ws * elems / (ms_e2e / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": aggregate(elems, ws, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
