@@ -198,6 +198,32 @@ int scan_block4(const float *A, const float *b, const float *y0, float *y, int B
                 int flags, void *ws, size_t ws_bytes, slstm_stream_t stream);
 
 /*
+ * scan_block4 for callers that cannot allocate device memory.  (The pages
+ * have no counterpart of this call; it is a service of this library.)
+ * Some callers own no workspace to pass: their own allocator has reserved
+ * every byte of the GPU, or they may not call cudaMalloc because it can
+ * synchronise the device, or they are plugins handed only input and output
+ * pointers.  This entry point takes the same arguments as scan_block4
+ * minus the workspace, and computes the same result, using scratch from one
+ * fixed block of SLSTM_NOALLOC_SCRATCH_BYTES of device memory that the
+ * library reserves on every GPU that loads it, held until the process exits.
+ *   - It allocates nothing.  The first call on each device looks up the
+ *     block's device address (a one-time set-up); make that first call
+ *     before any stream capture begins.
+ *   - All calls on a device share the block.  Calls that overlap on the same
+ *     GPU (other streams, other host threads) race on it: serialise them.
+ *     Each call clears the counters and flags it relies on before use.
+ *   - Returns SLSTM_ERR_UNSUPPORTED when the problem needs more scratch than
+ *     the block holds, that is when slstm_workspace_size(SLSTM_OP_SCAN_BLOCK4,
+ *     B, T, 0, d) > SLSTM_NOALLOC_SCRATCH_BYTES (up to 2727 tiles of 32 steps
+ *     x 32 features: B * ceil(T/32) * ceil(d/32) <= 2727); other errors as
+ *     scan_block4.
+ */
+#define SLSTM_NOALLOC_SCRATCH_BYTES (8u << 20)
+int scan_block4_noalloc(const float *A, const float *b, const float *y0, float *y, int B, int T,
+                        int d, int flags, slstm_stream_t stream);
+
+/*
  * Sequential stepping ("sLSTM in this library", "API notes": the evaluation
  * path; T_steps = 1 is one decode step):
  *   S_t = f(S_{t-1}, P_t) for t = 0 .. T_steps-1, S_{-1} = s0.

@@ -29,6 +29,7 @@ SLSTM_OP_NEWTON_BACKWARD = 3
 SLSTM_MAX_ITERS = 65536
 SLSTM_STATS_HISTORY = 64
 SLSTM_SCAN_REVERSE_T = 1
+SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class NewtonConfig(ctypes.Structure):
@@ -49,6 +50,7 @@ SIGNATURES = {
     "slstm_preact_gemm": (_I, [_V, _V, _I, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
     "slstm_newton_forward": (_I, [_V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _V, _Z, _V]),
     "scan_block4": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
+    "scan_block4_noalloc": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
     "slstm_sequential_step": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
     "slstm_newton_backward": (_I, [_V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I,
                                    _V, _Z, _V]),
