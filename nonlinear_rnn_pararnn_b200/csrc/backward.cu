@@ -36,7 +36,7 @@ template <int FORGET>
 __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
 {
     __shared__ float s_agg[NW][20][32];
-    __shared__ float s_carry[NW][4][32];
+    __shared__ float s_cin[4][32];
     __shared__ float s_part[NW][8][32];
     __shared__ unsigned s_ticket;
     const int lane = threadIdx.x & 31;
@@ -96,16 +96,16 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
     }
     store_aff_smem(s_agg, warp, lane, agg);
     __syncthreads();
+    tile_prefix_tree<NW>(s_agg, agg);
     if (warp == 0) {
         const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_lookback_warp0<NW>(s_agg, s_carry, a.lb, ticket, chunk, zero, false);
+        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, zero, false);
     }
     __syncthreads();
 
     // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
     float lam[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) lam[e] = s_carry[warp][e][lane];
+    warp_carry(s_agg, s_cin, warp, lane, lam);
     float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < L; ++i) {

@@ -44,7 +44,12 @@ struct CellG {
     float gcz, gci, gcf, gni, gnf, gmi, gmf, ghz, ghi, ghf, gho;
 };
 
-SLSTM_DEVINL float sigmoidf_(float x) { return 1.0f / (1.0f + expf(-x)); }
+// Transcendentals on the MUFU pipe through CUDA's fast intrinsics (__expf,
+// __logf, __fdividef), combined by the identities
+//   sigmoid(x) = 1 / (1 + e^{-x}),   tanh(x) = 1 - 2 / (1 + e^{2x}).
+// Both stay finite for any x: e^{..} = inf gives 1/inf = 0.
+SLSTM_DEVINL float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+SLSTM_DEVINL float tanh_fast(float x) { return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * x)); }
 
 // forget: SLSTM_FORGET_SIGMOID or SLSTM_FORGET_EXP.  WANT_J: fill the
 // Jacobian fields.  WANT_G: fill *g.
@@ -57,8 +62,8 @@ SLSTM_DEVINL void cell_eval(float c0, float n0, float m0, float h0, float pz, fl
     const float ai = fmaf(ri, h0, pi);
     const float af = fmaf(rf, h0, pf);
     const float ao = fmaf(ro, h0, po);
-    const float z = tanhf(az);
-    const float og = sigmoidf_(ao);
+    const float z = tanh_fast(az);
+    const float og = sigmoid_fast(ao);
     float lf, dlf;
     if (FORGET == SLSTM_FORGET_EXP) {
         lf = af;
@@ -66,19 +71,20 @@ SLSTM_DEVINL void cell_eval(float c0, float n0, float m0, float h0, float pz, fl
     } else {
         // log sigmoid(af) = min(af, 0) - log1p(exp(-|af|)); its derivative
         // is sigmoid(-af).
-        const float e = expf(-fabsf(af));
-        lf = fminf(af, 0.0f) - log1pf(e);
-        dlf = (af >= 0.0f ? e : 1.0f) / (1.0f + e);
+        const float e = __expf(-fabsf(af));
+        const float ope = 1.0f + e;
+        lf = fminf(af, 0.0f) - __logf(ope);
+        dlf = __fdividef(af >= 0.0f ? e : 1.0f, ope);
     }
     const float u = lf + m0;
     const bool fb = (u >= ai);  // forget branch of the max
     const float m = fb ? u : ai;
-    const float e = expf(-fabsf(u - ai));
+    const float e = __expf(-fabsf(u - ai));
     const float fp = fb ? 1.0f : e;  // exp(u - m)
     const float ip = fb ? e : 1.0f;  // exp(ai - m)
     const float c = fmaf(fp, c0, ip * z);
     const float n = fmaf(fp, n0, ip);
-    const float inv_n = 1.0f / n;
+    const float inv_n = __fdividef(1.0f, n);
     const float y = c * inv_n;
     o.c = c;
     o.n = n;
@@ -240,10 +246,8 @@ SLSTM_DEVINL unsigned wait_flag(const unsigned *flag, unsigned epoch, uint64_t l
     unsigned v = ld_acquire(flag);
     if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
     const uint64_t t0 = globaltimer_ns();
-    unsigned sleep = 32;
-    for (;;) {
-        __nanosleep(sleep);
-        if (sleep < 1024) sleep <<= 1;
+    for (unsigned polls = 0;; ++polls) {
+        if (polls >= 32) __nanosleep(64);
         v = ld_acquire(flag);
         if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
         if (globaltimer_ns() - t0 > limit_ns) return 0u;

@@ -1,0 +1,335 @@
+// bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM, fed by TMA):
+//   C[m][n] = sum_k A[m][k] B[n][k] + bias[n]     (A, B bf16, K-major; C fp32)
+// The input projection P = x W_x^T + b is this product with A = x (rows
+// (b,t)), B = W_x (rows (g,j)) ("sLSTM in this library", section "API
+// notes": W_x is a GEMM).
+//
+// One CTA computes a 128 x 256 tile of C:
+//   warp 0, one lane   TMA producer: A and B k-blocks (64 wide, 128-byte
+//                      swizzle) into a 4-stage ring guarded by mbarriers;
+//   warp 1, one lane   MMA issuer: tcgen05.mma (M=128, N=256, K=16) into a
+//                      256-column fp32 accumulator in TMEM; tcgen05.commit
+//                      frees each stage and finally signals the epilogue;
+//   all 4 warps        epilogue: tcgen05.ld of their 32 TMEM lanes, + bias,
+//                      fp32 stores.
+// No multicast and no clusters.  Every mbarrier wait is bounded in time; on
+// expiry the CTA records an error, waits (bounded) for the loads it issued,
+// frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "launchers.h"
+
+namespace slstm {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr uint32_t A_STAGE = BM * BK * 2;   // 16 KB
+constexpr uint32_t B_STAGE = BN * BK * 2;   // 32 KB
+constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint64_t WAIT_NS = 1000000000ull;   // 1 s bound on any single wait
+
+struct TcArgs {
+    float *C;
+    const float *bias;
+    int M, N, K;
+    unsigned *error;
+};
+
+SLSTM_DEVINL uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SLSTM_DEVINL void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+SLSTM_DEVINL void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+SLSTM_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0u;
+}
+
+// Wait for the phase of `bar` with the given parity to complete; false when
+// the time bound passes first.
+SLSTM_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > WAIT_NS) return false;
+    return true;
+}
+
+SLSTM_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
+// 128-byte swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart.
+SLSTM_DEVINL uint64_t smem_desc_k_sw128(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // start address
+    d |= (uint64_t)1u << 16;                     // leading byte offset (unused when swizzled)
+    d |= (uint64_t)(1024u >> 4) << 32;           // stride byte offset: next 8-row atom
+    d |= (uint64_t)1u << 46;                     // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                     // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, M x N.
+constexpr uint32_t idesc_bf16(int M, int N)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+SLSTM_DEVINL void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+        "}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+SLSTM_DEVINL void umma_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+SLSTM_DEVINL void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+SLSTM_DEVINL void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+SLSTM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(128, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, TcArgs g)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * A_STAGE;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint64_t *empty = full + STAGES;
+    uint64_t *accf = empty + STAGES;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
+    __shared__ int s_abort;
+    __shared__ int s_issued, s_consumed;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM;
+    const int n0 = blockIdx.x * BN;
+    const int nk = (g.K + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accf, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_abort = 0;
+        s_issued = 0;
+        s_consumed = 0;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {
+        // ---- TMA producer ----
+        int kb = 0;
+        for (; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+            if (!mbar_wait(&empty[s], ph ^ 1u) || *(volatile int *)&s_abort) {
+                s_abort = 1;
+                break;
+            }
+            mbar_expect_tx(&full[s], STAGE_BYTES);
+            tma_load_2d(sA + s * A_STAGE, &tma, &full[s], kb * BK, m0);
+            tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kb * BK, n0);
+        }
+        s_issued = kb;
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer ----
+        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        int kb = 0;
+        for (; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+            if (!mbar_wait(&full[s], ph) || *(volatile int *)&s_abort) {
+                s_abort = 1;
+                break;
+            }
+            tc_fence_after();
+            const uint64_t ad = smem_desc_k_sw128(smem_u32(sA + s * A_STAGE));
+            const uint64_t bd = smem_desc_k_sw128(smem_u32(sB + s * B_STAGE));
+#pragma unroll
+            for (int k = 0; k < BK / 16; ++k)   // 16 bf16 = 32 bytes per MMA step
+                umma_bf16(tmem, ad + 2u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            umma_commit(&empty[s]);
+        }
+        s_consumed = kb;
+        umma_commit(accf);   // fires when every MMA issued above has completed
+    }
+
+    // ---- epilogue: all four warps ----
+    const bool acc_ready = mbar_wait(accf, 0u);
+    tc_fence_after();
+    __syncthreads();
+    const bool ok = acc_ready && !s_abort;
+    if (ok) {
+        const int row = m0 + warp * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            float v[32];
+            tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
+            const int col0 = n0 + c * 32;
+            if (row < g.M) {
+                float *dst = g.C + (size_t)row * g.N + col0;
+                if (col0 + 32 <= g.N && (g.N & 3) == 0) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 o;
+                        o.x = v[4 * q + 0] + g.bias[col0 + 4 * q + 0];
+                        o.y = v[4 * q + 1] + g.bias[col0 + 4 * q + 1];
+                        o.z = v[4 * q + 2] + g.bias[col0 + 4 * q + 2];
+                        o.w = v[4 * q + 3] + g.bias[col0 + 4 * q + 3];
+                        reinterpret_cast<float4 *>(dst)[q] = o;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (col0 + i < g.N) dst[i] = v[i] + g.bias[col0 + i];
+                }
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        atomicOr(g.error, 1u);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (!ok && threadIdx.x == 0) {
+        // loads issued but never consumed still land in this CTA's shared
+        // memory: wait for them (bounded) before the CTA exits
+        for (int kb = s_consumed; kb < s_issued; ++kb)
+            (void)mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D K-major bf16 tensor [rows][K] with a (64 x box_rows) box, 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, int rows, int K, int box_rows)
+{
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// C[M][N] = A[M][K] B[N][K]^T + bias[N]; A, B bf16 K-major, K % 8 == 0.
+cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
+                         unsigned *error, cudaStream_t st)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, Bm, N, K, BN)) return cudaErrorInvalidValue;
+    TcArgs g;
+    g.C = C;
+    g.bias = bias;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.error = error;
+    const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
+    gemm_tc_kernel<<<grid, 128, SMEM_BYTES, st>>>(ta, tb, g);
+    return cudaGetLastError();
+}
+
+}  // namespace slstm

@@ -60,7 +60,13 @@ struct GemmDesc {
 };
 cudaError_t gemm_simt(const GemmDesc &g, cudaStream_t st);
 
-// Input projection P = x Wx^T + bias on the tcgen05 tensor cores (bf16).
+// C[M][N] = A[M][K] B[N][K]^T + bias[N] on the tcgen05 tensor cores; A and B
+// bf16, K-major, K % 8 == 0, 16-byte aligned.  `error` (device word) is set
+// nonzero if a bounded wait inside the kernel expires.
+cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
+                         unsigned *error, cudaStream_t st);
+
+// Input projection P = x Wx^T + bias (tcgen05 for bf16, CUDA cores for fp32).
 size_t preact_workspace_bytes(int B, int T, int d_in, int d_h, int dtype);
 cudaError_t preact_launch(const void *x, const void *Wx, int dtype, const float *bias, float *P,
                           int B, int T, int d_in, int d_h, void *ws, cudaStream_t st);

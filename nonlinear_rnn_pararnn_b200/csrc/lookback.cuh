@@ -1,11 +1,13 @@
 // Blocked scan of 4x4 affine maps across CTAs with a decoupled look-back.
 //
 // A "tile" is 32 features x (NW warps x L steps).  Inside a tile every warp
-// folds its own L steps serially (one feature per lane); warp 0 then folds
-// the NW warp aggregates, publishes the tile aggregate, looks back over the
-// tiles before it (same feature group, earlier in processing order) until it
-// meets a published inclusive prefix, publishes its own inclusive prefix and
-// hands every warp its incoming carry through shared memory.
+// folds its own L steps serially (one feature per lane).  The NW warp
+// aggregates are turned into inclusive prefixes by a Kogge-Stone tree in
+// shared memory (all warps work, log2 NW levels).  Warp 0 then publishes the
+// tile aggregate, looks back over the tiles before it (same feature group,
+// earlier in processing order) until it meets a published inclusive prefix,
+// and publishes its own; every warp finally derives its incoming carry from
+// the tile carry and its predecessor's prefix.
 //
 // Tiles take tickets from a global counter in the order CTAs start, and tile
 // (chunk c, group g) has ticket c * n_groups + g, so a tile only ever waits
@@ -32,29 +34,56 @@ struct LookbackArgs {
     int n_groups;      // feature groups (tiles per chunk)
 };
 
-// Called by warp 0 only, after every warp wrote its aggregate (in processing
-// order) to s_agg[w][0..19][lane].  Writes the carry entering each warp to
-// s_carry[w][0..3][lane].  `first_carry` is the value entering chunk 0.
-// `withhold` suppresses this tile's publications (fault injection).
+SLSTM_DEVINL void load_aff_smem(float (*s_agg)[20][32], int w, int lane, Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x.a[e] = s_agg[w][e][lane];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x.b[e] = s_agg[w][16 + e][lane];
+}
+
+SLSTM_DEVINL void store_aff_smem(float (*s_agg)[20][32], int w, int lane, const Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) s_agg[w][e][lane] = x.a[e];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s_agg[w][16 + e][lane] = x.b[e];
+}
+
+// All threads of the CTA.  On entry s_agg[w] holds warp w's aggregate (in
+// processing order) and `mine` the same value in registers; on exit s_agg[w]
+// holds the inclusive prefix agg_w o ... o agg_0.  Ends with a barrier.
 template <int NW>
-SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_carry)[4][32],
+SLSTM_DEVINL void tile_prefix_tree(float (*s_agg)[20][32], Aff &mine)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int off = 1; off < NW; off <<= 1) {
+        Aff left;
+        if (warp >= off) load_aff_smem(s_agg, warp - off, lane, left);
+        __syncthreads();
+        if (warp >= off) {
+            aff_compose(mine, left, mine);
+            store_aff_smem(s_agg, warp, lane, mine);
+        }
+        __syncthreads();
+    }
+}
+
+// Warp 0 only, after tile_prefix_tree.  Publishes the tile aggregate
+// (s_agg[NW-1]), looks back, publishes the inclusive prefix and writes the
+// carry entering the tile to s_cin[0..3][lane].  `first_carry` is the value
+// entering chunk 0.  `withhold` suppresses this tile's publications (fault
+// injection).
+template <int NW>
+SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_cin)[32],
                                       const LookbackArgs &lb, unsigned ticket, int chunk,
                                       const float first_carry[4], bool withhold)
 {
     const int lane = threadIdx.x & 31;
     Aff tile;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) tile.a[e] = s_agg[0][e][lane];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) tile.b[e] = s_agg[0][16 + e][lane];
-    for (int w = 1; w < NW; ++w) {
-        Aff x;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) x.a[e] = s_agg[w][e][lane];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x.b[e] = s_agg[w][16 + e][lane];
-        aff_compose(x, tile, tile);
-    }
+    load_aff_smem(s_agg, NW - 1, lane, tile);
 
     float carry[4];
 #pragma unroll
@@ -75,8 +104,9 @@ SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_carry)[4
         aff_identity(M);
         int q = chunk - 1;
         bool expired = false;
+        const unsigned grp = ticket % (unsigned)lb.n_groups;
         for (;;) {
-            const unsigned tq = (unsigned)q * (unsigned)lb.n_groups + (ticket % (unsigned)lb.n_groups);
+            const unsigned tq = (unsigned)q * (unsigned)lb.n_groups + grp;
             unsigned st = 0;
             if (lane == 0) st = wait_flag(lb.flags + tq, lb.epoch, lb.wait_ns);
             st = __shfl_sync(0xffffffffu, st, 0);
@@ -116,23 +146,26 @@ SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_carry)[4
         __syncwarp();
         if (lane == 0) st_release(lb.flags + ticket, (lb.epoch << 2) | FLAG_INC);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s_cin[e][lane] = carry[e];
+}
 
-    // carries entering each warp of this tile
-    float v[4];
+// Any warp, after the barrier that follows tile_lookback_warp0: the carry
+// entering warp `warp` of the tile.
+SLSTM_DEVINL void warp_carry(float (*s_agg)[20][32], float (*s_cin)[32], int warp, int lane,
+                             float out[4])
+{
+    float cin[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = carry[e];
-    for (int w = 0; w < NW; ++w) {
+    for (int e = 0; e < 4; ++e) cin[e] = s_cin[e][lane];
+    if (warp == 0) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s_carry[w][e][lane] = v[e];
-        if (w + 1 < NW) {
-            Aff x;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) x.a[e] = s_agg[w][e][lane];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) x.b[e] = s_agg[w][16 + e][lane];
-            aff_apply(x, v, v);
-        }
+        for (int e = 0; e < 4; ++e) out[e] = cin[e];
+        return;
     }
+    Aff pre;
+    load_aff_smem(s_agg, warp - 1, lane, pre);
+    aff_apply(pre, cin, out);
 }
 
 // Fold one step's map (J, r) into a running aggregate: agg <- (J, r) o agg.
@@ -165,14 +198,6 @@ SLSTM_DEVINL void cell_identity(Cell &J)
     J.dmh = 0.0f;
     J.jhc = J.jhn = J.jhm = 0.0f;
     J.jhh = 1.0f;
-}
-
-SLSTM_DEVINL void store_aff_smem(float (*s_agg)[20][32], int w, int lane, const Aff &x)
-{
-#pragma unroll
-    for (int e = 0; e < 16; ++e) s_agg[w][e][lane] = x.a[e];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s_agg[w][16 + e][lane] = x.b[e];
 }
 
 }  // namespace slstm

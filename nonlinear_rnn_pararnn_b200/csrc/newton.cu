@@ -87,7 +87,7 @@ template <int FORGET, bool FIRST, bool RESID>
 __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
 {
     __shared__ float s_agg[NW][20][32];
-    __shared__ float s_carry[NW][4][32];
+    __shared__ float s_cin[4][32];
     __shared__ float s_red[2][NW];
     __shared__ unsigned s_ticket;
     __shared__ int s_exit;
@@ -182,18 +182,18 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
     }
     store_aff_smem(s_agg, warp, lane, agg);
     __syncthreads();
+    tile_prefix_tree<NW>(s_agg, agg);
 
     if (warp == 0) {
         const float zero[4] = {0.f, 0.f, 0.f, 0.f};
         const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
-        tile_lookback_warp0<NW>(s_agg, s_carry, a.lb, ticket, chunk, zero, withhold);
+        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, zero, withhold);
     }
     __syncthreads();
 
     // ---- walk B ----
     float dl[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dl[e] = s_carry[warp][e][lane];
+    warp_carry(s_agg, s_cin, warp, lane, dl);
     float snp[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];

@@ -52,7 +52,7 @@ template <bool REVERSE>
 __global__ void __launch_bounds__(NW * 32, 2) scan_kernel(ScanArgs a)
 {
     __shared__ float s_agg[NW][20][32];
-    __shared__ float s_carry[NW][4][32];
+    __shared__ float s_cin[4][32];
     __shared__ unsigned s_ticket;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -85,19 +85,19 @@ __global__ void __launch_bounds__(NW * 32, 2) scan_kernel(ScanArgs a)
     }
     store_aff_smem(s_agg, warp, lane, agg);
     __syncthreads();
+    tile_prefix_tree<NW>(s_agg, agg);
     if (warp == 0) {
         float first[4] = {0.f, 0.f, 0.f, 0.f};
         if (a.y0 && jv) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) first[e] = a.y0[((size_t)bb * 4 + e) * d + jj];
         }
-        tile_lookback_warp0<NW>(s_agg, s_carry, a.lb, ticket, chunk, first, false);
+        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, first, false);
     }
     __syncthreads();
 
     float v[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = s_carry[warp][e][lane];
+    warp_carry(s_agg, s_cin, warp, lane, v);
 #pragma unroll
     for (int i = 0; i < L; ++i) {
         const int p = p_seg + i;
