@@ -8,6 +8,8 @@
 //   dR      += dP_t * h_{t-1},  db += dP_t   (per-tile partials, reduced after)
 //   ds0      = J_0^T lambda_0
 // then dx = dP W_x and dW_x = dP^T x.
+#include <cuda_bf16.h>
+
 #include "launchers.h"
 #include "lookback.cuh"
 
@@ -24,7 +26,11 @@ struct BwdArgs {
     const float *s0;
     const float *S;
     const float *dH;
-    float *dP;        // (B, T, 4, d)
+    float *dP;        // (B, T, 4, d) fp32, when the GEMMs run on CUDA cores
+    // bf16 pair dP ~ hi + lo (|dP - hi - lo| <= 2^-18 |dP|) for the tensor-core
+    // GEMMs, in the layout (B*T, 4d) and transposed (4d, ldT)
+    __nv_bfloat16 *dp_hi, *dp_lo, *dpt_hi, *dpt_lo;
+    long long ldT;
     float *partial;   // [n_tiles][8][32]  dR (4) then db (4)
     float *ds0;       // (B, 4, d) or null
     unsigned *ticket;
@@ -32,12 +38,20 @@ struct BwdArgs {
     int T, d, groups_per_row;
 };
 
-template <int FORGET>
+SLSTM_DEVINL void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
+{
+    hi = __float2bfloat16_rn(v);
+    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
+
+template <int FORGET, bool BF16OUT>
 __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
 {
     __shared__ float s_agg[NW][20][32];
     __shared__ float s_cin[4][32];
     __shared__ float s_part[NW][8][32];
+    // transposed staging of the tile's dP pair: [hi/lo][gate][feature][step]
+    __shared__ __nv_bfloat16 s_dpt[BF16OUT ? 2 : 1][4][32][TT + 2];
     __shared__ unsigned s_ticket;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -132,11 +146,26 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
             const float di = fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3])));
             const float df = fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3])));
             const float dq = g.gho * lam[3];
-            float *pd = a.dP + (row0 + t) * 4 * d + jj;
-            pd[0] = dz;
-            pd[d] = di;
-            pd[2 * d] = df;
-            pd[3 * d] = dq;
+            if (BF16OUT) {
+                const float dv[4] = {dz, di, df, dq};
+                const size_t o = (row0 + t) * 4 * d + jj;
+                const int tl = TT - 1 - (warp * L + i);   // step index inside the tile, ascending in t
+#pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    __nv_bfloat16 hi, lo;
+                    split_bf16(dv[gi], hi, lo);
+                    a.dp_hi[o + gi * d] = hi;
+                    a.dp_lo[o + gi * d] = lo;
+                    s_dpt[0][gi][lane][tl] = hi;
+                    s_dpt[BF16OUT ? 1 : 0][gi][lane][tl] = lo;
+                }
+            } else {
+                float *pd = a.dP + (row0 + t) * 4 * d + jj;
+                pd[0] = dz;
+                pd[d] = di;
+                pd[2 * d] = df;
+                pd[3 * d] = dq;
+            }
             const float hp = prev[3];
             dr[0] = fmaf(dz, hp, dr[0]);
             dr[1] = fmaf(di, hp, dr[1]);
@@ -171,6 +200,52 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
         for (int w = 0; w < NW; ++w) acc += s_part[w][e][lane];
         a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
     }
+    if (BF16OUT) {
+        // rows (g, j) of the transposed pair: 32 consecutive steps each; the
+        // tile covers t in [t_lo, t_lo + TT) clipped to [0, T)
+        const int t_lo = T - (chunk + 1) * TT;
+        const int tl = threadIdx.x & 31;
+        const int t = t_lo + tl;
+        const int j0 = (grp % a.groups_per_row) * 32;
+        for (int r = threadIdx.x >> 5; r < 2 * 4 * 32; r += NW) {
+            const int part = r >> 7;
+            const int gi = (r >> 5) & 3;
+            const int jl = r & 31;
+            if (t >= 0 && j0 + jl < a.d) {
+                __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                dst[((size_t)gi * d + j0 + jl) * a.ldT + row0 + t] = s_dpt[part][gi][jl][tl];
+            }
+        }
+    }
+}
+
+// out[c][r] = in[r][c] for a bf16 matrix of R rows and C columns; row strides
+// ldi (in) and ldo (out) in elements.
+__global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ in, __nv_bfloat16 *__restrict__ out,
+                                      int R, int C, long long ldi, long long ldo)
+{
+    __shared__ __nv_bfloat16 tile[32][34];
+    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    for (int k = ty; k < 32; k += 8) {
+        const int r = r0 + k, c = c0 + tx;
+        if (r < R && c < C) tile[k][tx] = in[(size_t)r * ldi + c];
+    }
+    __syncthreads();
+    for (int k = ty; k < 32; k += 8) {
+        const int c = c0 + k, r = r0 + tx;
+        if (r < R && c < C) out[(size_t)c * ldo + r] = tile[tx][k];
+    }
+}
+
+// out[i] = sum_z part[z][i], z in order (split-K partial sums).
+__global__ void sum_splits_kernel(const float *__restrict__ part, float *__restrict__ out, long long n, int splits)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float acc = 0.0f;
+    for (int z = 0; z < splits; ++z) acc += part[(size_t)z * n + i];
+    out[i] = acc;
 }
 
 // dR[g][j] and db[g][j]: sum of the per-tile partials over chunks and batch
@@ -198,17 +273,33 @@ __global__ void reduce_partials_kernel(const float *__restrict__ partial, float 
 }
 
 struct Layout {
-    size_t ticket, flags, agg, inc, partial, dP, total;
-    int groups_per_row, n_groups, n_chunks, n_tiles;
+    size_t ticket, flags, agg, inc, partial, dP, dpt, xT, wT, wpart, err, total;
+    int groups_per_row, n_groups, n_chunks, n_tiles, splits;
+    long long n, ldT, ld4;
 };
 
-Layout layout(int B, int T, int d_h)
+long long round8(long long v) { return (v + 7) & ~7LL; }
+
+// split-K count of the W_x-gradient GEMM: enough CTAs for two per SM
+int wgrad_splits(int B, int T, int d_in, int d_h)
+{
+    const long long tiles = ((4LL * d_h + 127) / 128) * ((d_in + 255) / 256);
+    int want = (int)((296 + tiles - 1) / tiles);
+    if (want > 16) want = 16;
+    return gemm_tc_splits(4 * d_h, d_in, B * T, 2, want);
+}
+
+Layout layout(int B, int T, int d_in, int d_h)
 {
     Layout l;
     l.groups_per_row = (d_h + 31) / 32;
     l.n_groups = B * l.groups_per_row;
     l.n_chunks = (T + TT - 1) / TT;
     l.n_tiles = l.n_groups * l.n_chunks;
+    l.n = (long long)B * T * 4 * d_h;
+    l.ldT = round8((long long)B * T);
+    l.ld4 = round8(4LL * d_h);
+    l.splits = wgrad_splits(B, T, d_in, d_h);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t at = off;
@@ -220,26 +311,31 @@ Layout layout(int B, int T, int d_h)
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
     l.inc = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.partial = take(sizeof(float) * 8 * 32 * (size_t)l.n_tiles);
-    l.dP = take(sizeof(float) * 4 * (size_t)B * T * d_h);
+    // fp32 dP (CUDA-core GEMMs) and the bf16 pair in the (B*T, 4d) layout
+    // (tensor-core GEMMs) share one region; the transposed pair follows
+    l.dP = take(sizeof(float) * (size_t)l.n);
+    l.dpt = take(2 * sizeof(__nv_bfloat16) * (size_t)(4LL * d_h) * (size_t)l.ldT);
+    l.xT = take(sizeof(__nv_bfloat16) * (size_t)d_in * (size_t)l.ldT);
+    l.wT = take(sizeof(__nv_bfloat16) * (size_t)d_in * (size_t)l.ld4);
+    l.wpart = take(sizeof(float) * (size_t)l.splits * 4 * d_h * d_in);
+    l.err = take(256);
     l.total = off;
     return l;
 }
 
 }  // namespace
 
-size_t backward_workspace_bytes(int B, int T, int d_in, int d_h)
-{
-    (void)d_in;
-    return layout(B, T, d_h).total;
-}
+size_t backward_workspace_bytes(int B, int T, int d_in, int d_h) { return layout(B, T, d_in, d_h).total; }
 
 cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *R,
                             const float *s0, const float *S, const float *dH, float *dx, float *dWx,
                             float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
                             int d_h, void *ws, cudaStream_t st)
 {
-    const Layout l = layout(B, T, d_h);
+    const Layout l = layout(B, T, d_in, d_h);
     char *base = static_cast<char *>(ws);
+    // tensor-core GEMMs need 16-byte TMA strides: (4 d_h) bf16 rows and d_in % 8
+    const bool tc = (dtype == SLSTM_BF16) && (d_h % 2 == 0) && (d_in % 8 == 0);
     BwdArgs a;
     a.P = P;
     a.R = R;
@@ -247,6 +343,11 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.S = S;
     a.dH = dH;
     a.dP = reinterpret_cast<float *>(base + l.dP);
+    a.dp_hi = reinterpret_cast<__nv_bfloat16 *>(base + l.dP);
+    a.dp_lo = a.dp_hi + l.n;
+    a.dpt_hi = reinterpret_cast<__nv_bfloat16 *>(base + l.dpt);
+    a.dpt_lo = a.dpt_hi + 4LL * d_h * l.ldT;
+    a.ldT = l.ldT;
     a.partial = reinterpret_cast<float *>(base + l.partial);
     a.ds0 = ds0;
     a.ticket = reinterpret_cast<unsigned *>(base + l.ticket);
@@ -262,22 +363,52 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.groups_per_row = l.groups_per_row;
     cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
     if (e != cudaSuccess) return e;
-    if (ds0 && !s0) {
-        // ds0 is still defined (the gradient at a zero initial state)
+    if (forget == SLSTM_FORGET_EXP) {
+        if (tc)
+            adjoint_vjp_kernel<SLSTM_FORGET_EXP, true><<<l.n_tiles, NW * 32, 0, st>>>(a);
+        else
+            adjoint_vjp_kernel<SLSTM_FORGET_EXP, false><<<l.n_tiles, NW * 32, 0, st>>>(a);
+    } else {
+        if (tc)
+            adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID, true><<<l.n_tiles, NW * 32, 0, st>>>(a);
+        else
+            adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID, false><<<l.n_tiles, NW * 32, 0, st>>>(a);
     }
-    if (forget == SLSTM_FORGET_EXP)
-        adjoint_vjp_kernel<SLSTM_FORGET_EXP><<<l.n_tiles, NW * 32, 0, st>>>(a);
-    else
-        adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID><<<l.n_tiles, NW * 32, 0, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     reduce_partials_kernel<<<(8 * d_h + 255) / 256, 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     const long long N4 = 4LL * d_h;
+    const int BT = B * T;
+    if (tc) {
+        unsigned *err = reinterpret_cast<unsigned *>(base + l.err);
+        __nv_bfloat16 *xT = reinterpret_cast<__nv_bfloat16 *>(base + l.xT);
+        __nv_bfloat16 *wT = reinterpret_cast<__nv_bfloat16 *>(base + l.wT);
+        float *wpart = reinterpret_cast<float *>(base + l.wpart);
+        if ((e = cudaMemsetAsync(err, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
+        // W_x^T (d_in, 4 d_h) and x^T (d_in, B*T) as K-major operands
+        transpose_bf16_kernel<<<dim3((d_in + 31) / 32, (unsigned)((N4 + 31) / 32)), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(Wx), wT, (int)N4, d_in, d_in, l.ld4);
+        transpose_bf16_kernel<<<dim3((d_in + 31) / 32, (unsigned)((BT + 31) / 32)), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16 *>(x), xT, BT, d_in, d_in, l.ldT);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        // dx = (dP_hi + dP_lo) W_x
+        if ((e = gemm_tc_bf16_ex(a.dp_hi, a.dp_lo, (int)N4, wT, (int)l.ld4, nullptr, dx, BT, d_in, (int)N4, 1, err,
+                                 st)) != cudaSuccess)
+            return e;
+        // dW_x = (dP_hi + dP_lo)^T x, split over B*T, partial sums added in order
+        if ((e = gemm_tc_bf16_ex(a.dpt_hi, a.dpt_lo, (int)l.ldT, xT, (int)l.ldT, nullptr, wpart, (int)N4, d_in, BT,
+                                 l.splits, err, st)) != cudaSuccess)
+            return e;
+        const long long nw = N4 * d_in;
+        sum_splits_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(wpart, dWx, nw, l.splits);
+        return cudaGetLastError();
+    }
+
     // dx[(b,t), k] = sum_{g,j} dP[(b,t), (g,j)] Wx[(g,j), k]
     GemmDesc gx;
-    gx.M = B * T;
+    gx.M = BT;
     gx.N = d_in;
     gx.K = (int)N4;
     gx.A = a.dP;
@@ -295,7 +426,7 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     GemmDesc gw;
     gw.M = (int)N4;
     gw.N = d_in;
-    gw.K = B * T;
+    gw.K = BT;
     gw.A = a.dP;
     gw.a_dtype = SLSTM_F32;
     gw.sam = 1;

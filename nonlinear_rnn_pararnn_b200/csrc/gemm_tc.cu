@@ -35,8 +35,11 @@ constexpr uint64_t WAIT_NS = 1000000000ull;   // 1 s bound on any single wait
 
 struct TcArgs {
     float *C;
-    const float *bias;
+    const float *bias;      // [N] or null
     int M, N, K;
+    int a_parts;            // 1, or 2: C = (A0 + A1) B^T with A1 from the second map
+    int kb_per_split;       // k-blocks of the virtual K (a_parts * ceil(K/64)) per split
+    long long c_split;      // element offset between the C slices of the splits
     unsigned *error;
 };
 
@@ -147,7 +150,8 @@ SLSTM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
 }
 
 __global__ void __launch_bounds__(128, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, TcArgs g)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tma2,
+                   const __grid_constant__ CUtensorMap tmb, TcArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -164,7 +168,11 @@ __global__ void __launch_bounds__(128, 1)
     const int lane = threadIdx.x & 31;
     const int m0 = blockIdx.y * BM;
     const int n0 = blockIdx.x * BN;
-    const int nk = (g.K + BK - 1) / BK;
+    // this CTA's k-blocks: [kb0, kb0 + nkb) of the virtual K that runs over
+    // the a_parts operand parts one after the other
+    const int nk_part = (g.K + BK - 1) / BK;
+    const int kb0 = blockIdx.z * g.kb_per_split;
+    const int nkb = min(g.kb_per_split, g.a_parts * nk_part - kb0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -191,23 +199,26 @@ __global__ void __launch_bounds__(128, 1)
     if (warp == 0 && lane == 0) {
         // ---- TMA producer ----
         int kb = 0;
-        for (; kb < nk; ++kb) {
+        for (; kb < nkb; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
             if (!mbar_wait(&empty[s], ph ^ 1u) || *(volatile int *)&s_abort) {
                 s_abort = 1;
                 break;
             }
+            const int vk = kb0 + kb;
+            const int part = vk / nk_part;
+            const int kk = vk - part * nk_part;
             mbar_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(sA + s * A_STAGE, &tma, &full[s], kb * BK, m0);
-            tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kb * BK, n0);
+            tma_load_2d(sA + s * A_STAGE, part ? &tma2 : &tma, &full[s], kk * BK, m0);
+            tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kk * BK, n0);
         }
         s_issued = kb;
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer ----
         constexpr uint32_t idesc = idesc_bf16(BM, BN);
         int kb = 0;
-        for (; kb < nk; ++kb) {
+        for (; kb < nkb; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
             if (!mbar_wait(&full[s], ph) || *(volatile int *)&s_abort) {
@@ -240,21 +251,21 @@ __global__ void __launch_bounds__(128, 1)
             tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
             const int col0 = n0 + c * 32;
             if (row < g.M) {
-                float *dst = g.C + (size_t)row * g.N + col0;
+                float *dst = g.C + (size_t)blockIdx.z * g.c_split + (size_t)row * g.N + col0;
                 if (col0 + 32 <= g.N && (g.N & 3) == 0) {
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         float4 o;
-                        o.x = v[4 * q + 0] + g.bias[col0 + 4 * q + 0];
-                        o.y = v[4 * q + 1] + g.bias[col0 + 4 * q + 1];
-                        o.z = v[4 * q + 2] + g.bias[col0 + 4 * q + 2];
-                        o.w = v[4 * q + 3] + g.bias[col0 + 4 * q + 3];
+                        o.x = v[4 * q + 0] + (g.bias ? g.bias[col0 + 4 * q + 0] : 0.0f);
+                        o.y = v[4 * q + 1] + (g.bias ? g.bias[col0 + 4 * q + 1] : 0.0f);
+                        o.z = v[4 * q + 2] + (g.bias ? g.bias[col0 + 4 * q + 2] : 0.0f);
+                        o.w = v[4 * q + 3] + (g.bias ? g.bias[col0 + 4 * q + 3] : 0.0f);
                         reinterpret_cast<float4 *>(dst)[q] = o;
                     }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
-                        if (col0 + i < g.N) dst[i] = v[i] + g.bias[col0 + i];
+                        if (col0 + i < g.N) dst[i] = v[i] + (g.bias ? g.bias[col0 + i] : 0.0f);
                 }
             }
         }
@@ -290,13 +301,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 2-D K-major bf16 tensor [rows][K] with a (64 x box_rows) box, 128-byte swizzle.
-bool make_map(CUtensorMap *map, const void *base, int rows, int K, int box_rows)
+// 2-D K-major bf16 tensor [rows][K] (row stride ld elements) with a
+// (64 x box_rows) box, 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, int rows, int K, int ld, int box_rows)
 {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
     cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
@@ -307,9 +319,11 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int K, int box_rows)
 
 }  // namespace
 
-// C[M][N] = A[M][K] B[N][K]^T + bias[N]; A, B bf16 K-major, K % 8 == 0.
-cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
-                         unsigned *error, cudaStream_t st)
+// C = (A0 [+ A1]) B^T (+ bias) with optional split-K into `splits` fp32
+// slices C + z * M * N (the caller sums them); A0, A1: [M][K] bf16 with row
+// stride lda elements, B: [N][K] bf16 with row stride ldb; K-major.
+cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, const void *Bm, int ldb, const float *bias,
+                            float *C, int M, int N, int K, int splits, unsigned *error, cudaStream_t st)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -318,18 +332,45 @@ cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    CUtensorMap ta, tb;
-    if (!make_map(&ta, A, M, K, BM) || !make_map(&tb, Bm, N, K, BN)) return cudaErrorInvalidValue;
+    CUtensorMap ta, ta2, tb;
+    if (!make_map(&ta, A0, M, K, lda, BM) || !make_map(&tb, Bm, N, K, ldb, BN)) return cudaErrorInvalidValue;
+    if (A1 != nullptr) {
+        if (!make_map(&ta2, A1, M, K, lda, BM)) return cudaErrorInvalidValue;
+    } else {
+        ta2 = ta;
+    }
     TcArgs g;
     g.C = C;
     g.bias = bias;
     g.M = M;
     g.N = N;
     g.K = K;
+    g.a_parts = A1 ? 2 : 1;
+    const int total = g.a_parts * ((K + BK - 1) / BK);
+    if (splits < 1) splits = 1;
+    if (splits > total) splits = total;
+    g.kb_per_split = (total + splits - 1) / splits;
+    splits = (total + g.kb_per_split - 1) / g.kb_per_split;   // no empty split
+    g.c_split = (long long)M * N;
     g.error = error;
-    const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-    gemm_tc_kernel<<<grid, 128, SMEM_BYTES, st>>>(ta, tb, g);
+    const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, splits);
+    gemm_tc_kernel<<<grid, 128, SMEM_BYTES, st>>>(ta, ta2, tb, g);
     return cudaGetLastError();
+}
+
+int gemm_tc_splits(int M, int N, int K, int a_parts, int want)
+{
+    const int total = a_parts * ((K + BK - 1) / BK);
+    if (want < 1) want = 1;
+    if (want > total) want = total;
+    const int per = (total + want - 1) / want;
+    return (total + per - 1) / per;
+}
+
+cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
+                         unsigned *error, cudaStream_t st)
+{
+    return gemm_tc_bf16_ex(A, nullptr, K, Bm, K, bias, C, M, N, K, 1, error, st);
 }
 
 }  // namespace slstm

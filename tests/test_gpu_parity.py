@@ -205,9 +205,12 @@ def test_newton_bounded_wait_reports_timeout(cuda_device):
 # backward
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
-@pytest.mark.parametrize("B,T,d_in,d", [(2, 64, 8, 8), (2, 75, 12, 40)])
-def test_backward_matches_oracle_bptt(forget, B, T, d_in, d, cuda_device):
-    w = Workload("t", B, T, d_in, d, "f32", forget, 0.5, 13, 1e-6, 64)
+@pytest.mark.parametrize("B,T,d_in,d,dtype", [(2, 64, 8, 8, "f32"), (2, 75, 12, 40, "f32"),
+                                              (2, 75, 16, 40, "bf16"), (3, 130, 64, 96, "bf16")])
+def test_backward_matches_oracle_bptt(forget, B, T, d_in, d, dtype, cuda_device):
+    """fp32 inputs take the CUDA-core GEMMs; bf16 inputs the tensor-core GEMMs
+    with dP carried as a bf16 pair (transposed copy for the W_x gradient)."""
+    w = Workload("t", B, T, d_in, d, dtype, forget, 0.5, 13, 1e-6, 64)
     inp = make_inputs(w, with_dH=True)
     g = torch.Generator().manual_seed(9)
     s0 = torch.stack([torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) + 0.5,
