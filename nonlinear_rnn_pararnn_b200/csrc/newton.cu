@@ -4,22 +4,41 @@
 // "Cell": the fused diag training cell runs Newton with a 4x4 Jacobian per
 // feature and an O(d) combine; "pararnn-torch structure", section "Current
 // surface": fused kernels prepend h0, residual early stop, divergence after
-// K).  Per tile of 32 features x TT steps:
-//   walk A  each thread (one feature, L consecutive steps) recomputes gates,
-//           stabilizer, f(S_{t-1}, P_t) and J_t in registers from P and the
-//           current guess, keeps (J_t, r_t = f - S_t) in registers and folds
-//           the affine maps delta -> J_t delta + r_t;
-//   scan    warp 0 combines the warps, publishes, looks back across tiles;
-//   walk B  each thread replays its L steps from the incoming carry,
-//           writes S + delta in place and (when asked) evaluates the residual
-//           of the new iterate for the stopping test.
+// K).  The iteration is tiled: a tile is 32 features x 32 steps, handled by
+// one CTA of 8 warps (lane = feature, warp = 4 consecutive steps).
+//
+// Persistent CTAs walk the tiles in ticket order and keep the next tile's P
+// and old S arriving in shared memory (cp.async, double buffered) while they
+// work on the current one:
+//   walk A  each thread recomputes gates, stabilizer, f(S_{t-1}, P_t) and the
+//           4x4 Jacobian J_t in registers for its 4 steps, keeps (J_t, r_t =
+//           f - S_t) in registers and folds the maps delta -> J_t delta + r_t;
+//   scan    the 8 warp aggregates become inclusive prefixes (Kogge-Stone in
+//           shared memory); warp 0 obtains the carry entering the tile from
+//           the tile before it (see below) and publishes this tile's
+//           inclusive prefix;
+//   walk B  each thread replays its steps from its carry, writes S + delta in
+//           place and, when asked, accumulates the residual of the new
+//           iterate for the stopping test.
+//
+// Carry hand-off between tiles.  A tile's inclusive prefix (4 values per
+// feature) is published as 64-bit words (value bits, launch epoch), so a
+// reader validates and reads it in one load and the writer needs no fence.
+// A tile whose predecessor has not published yet first publishes its own
+// aggregate (20 values per feature, gated by a per-tile flag word) and then
+// looks back past unfinished predecessors, composing their aggregates.
+// Tickets are taken in start order and every wait is on a lower ticket that
+// some running CTA holds as its current tile, so every wait ends; waits are
+// also bounded in time (expiry sets an error and continues with a zero
+// carry).
+//
 // In-place update is safe because the only value a tile reads from another
 // tile (the state just before it) comes from a per-tile boundary buffer
 // written by the previous launch.
-#include "lookback.cuh"
-#include "launchers.h"
-
 #include <float.h>
+
+#include "launchers.h"
+#include "lookback.cuh"
 
 namespace slstm {
 namespace {
@@ -34,13 +53,193 @@ struct Args {
     const float *s0;
     float *S;
     NewtonCtrl *ctrl;
-    LookbackArgs lb;
-    float *bnd_in;   // [n_tiles][4][32]  S of the previous iterate at each tile's last step
+    unsigned *flags;              // [n_tiles] aggregate-published flags
+    float *agg;                   // [n_tiles][20][32]
+    unsigned long long *incw;     // [n_tiles][4][32] (value bits | epoch << 32)
+    float *bnd_in;                // [n_tiles][4][32] S of the previous iterate at each tile's last step
     float *bnd_out;
     slstm_newton_stats *stats;
-    int B, T, d, groups_per_row, n_tiles, max_iters, fixed, fault_ticket;
+    unsigned *error;
+    unsigned epoch;
+    unsigned long long wait_ns;
+    int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
     float tol;
 };
+
+struct Smem {
+    float P[2][TT][4][32];
+    float S[2][TT][4][32];
+    float agg[NW][20][32];
+    float cin[4][32];
+    float red[2][NW];
+    unsigned tick[2];
+    int exit_flag;
+};
+
+SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SLSTM_DEVINL void cp_async16(void *dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+SLSTM_DEVINL void cp_async4(void *dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+SLSTM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+SLSTM_DEVINL void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+SLSTM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+SLSTM_DEVINL void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Issue the copies of one tile's P (and old S unless `with_s` is false) into
+// shared-memory stage `st`.  Rows past T and features past d read nothing and
+// arrive as zeros.
+SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, unsigned ticket, bool with_s)
+{
+    if (ticket >= (unsigned)a.n_tiles) return;
+    const int chunk = (int)(ticket / (unsigned)a.n_groups);
+    const int grp = (int)(ticket % (unsigned)a.n_groups);
+    const int b = grp / a.groups_per_row;
+    const int j0 = (grp % a.groups_per_row) * 32;
+    const int t0 = chunk * TT;
+    const size_t d = (size_t)a.d;
+    const int ntens = with_s ? 2 : 1;
+    if (a.vec16) {
+        // 8 chunks of 16 bytes per (step, slot) row of 32 features
+        for (int idx = threadIdx.x; idx < ntens * TT * 4 * 8; idx += NW * 32) {
+            const int tens = idx / (TT * 4 * 8);
+            const int rem = idx % (TT * 4 * 8);
+            const int c = rem & 7;
+            const int rs = rem >> 3;
+            const int step = rs >> 2, slot = rs & 3;
+            const int t = t0 + step;
+            const int jj = j0 + 4 * c;
+            int bytes = 0;
+            if (t < a.T && jj < a.d) bytes = min(16, 4 * (a.d - jj));
+            const float *base = tens ? a.S : a.P;
+            const float *src = bytes ? base + (((size_t)b * a.T + t) * 4 + slot) * d + jj : base;
+            float *dst = tens ? &sm.S[st][step][slot][4 * c] : &sm.P[st][step][slot][4 * c];
+            cp_async16(dst, src, bytes);
+        }
+    } else {
+        for (int idx = threadIdx.x; idx < ntens * TT * 4 * 32; idx += NW * 32) {
+            const int tens = idx / (TT * 4 * 32);
+            const int rem = idx % (TT * 4 * 32);
+            const int jl = rem & 31;
+            const int rs = rem >> 5;
+            const int step = rs >> 2, slot = rs & 3;
+            const int t = t0 + step;
+            const int jj = j0 + jl;
+            const int bytes = (t < a.T && jj < a.d) ? 4 : 0;
+            const float *base = tens ? a.S : a.P;
+            const float *src = bytes ? base + (((size_t)b * a.T + t) * 4 + slot) * d + jj : base;
+            float *dst = tens ? &sm.S[st][step][slot][jl] : &sm.P[st][step][slot][jl];
+            cp_async4(dst, src, bytes);
+        }
+    }
+}
+
+// Inclusive prefix of tile tq for this lane, if published in this launch.
+SLSTM_DEVINL bool read_inc(const Args &a, unsigned tq, int lane, float v[4])
+{
+    const unsigned long long *src = a.incw + (size_t)tq * 4 * 32 + lane;
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const unsigned long long w = ld_relaxed_u64(src + e * 32);
+        ok = ok && ((unsigned)(w >> 32) == a.epoch);
+        v[e] = __uint_as_float((unsigned)w);
+    }
+    return ok;
+}
+
+// Warp 0: carry entering the tile (written to sm.cin) and publication of the
+// tile's inclusive prefix; sm.agg holds the warps' inclusive prefixes.
+SLSTM_DEVINL void tile_carry_warp0(const Args &a, Smem &sm, unsigned ticket, int chunk, int grp, bool withhold)
+{
+    const int lane = threadIdx.x & 31;
+    Aff tile;
+    load_aff_smem(sm.agg, NW - 1, lane, tile);
+    float carry[4] = {0.f, 0.f, 0.f, 0.f};
+    if (chunk > 0) {
+        unsigned tq = ticket - (unsigned)a.n_groups;
+        float v[4];
+        const bool ok = read_inc(a, tq, lane, v);
+        if (__all_sync(0xffffffffu, ok)) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) carry[e] = v[e];
+        } else {
+            // predecessor unfinished: publish the aggregate so that later
+            // tiles can skip over this one, then look back
+            if (!withhold) {
+                float *dst = a.agg + (size_t)ticket * 20 * 32;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(a.flags + ticket, (a.epoch << 2) | FLAG_AGG);
+            }
+            Aff M;
+            aff_identity(M);
+            int q = chunk - 1;
+            const uint64_t t0 = globaltimer_ns();
+            unsigned polls = 0;
+            for (;;) {
+                tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
+                if (read_inc(a, tq, lane, v)) {
+                    aff_apply(M, v, carry);
+                    break;
+                }
+                const unsigned f = ld_acquire(a.flags + tq);
+                if ((f >> 2) == a.epoch && (f & 3u) == FLAG_AGG) {
+                    Aff x;
+                    const float *src = a.agg + (size_t)tq * 20 * 32;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+                    aff_compose(M, x, M);
+                    --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
+                    continue;
+                }
+                if (++polls > 16) __nanosleep(64);
+                if (globaltimer_ns() - t0 > a.wait_ns) {
+                    atomicOr(a.error, 1u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) carry[e] = 0.f;
+                    break;
+                }
+            }
+        }
+    }
+    if (!withhold) {
+        float incv[4];
+        aff_apply(tile, carry, incv);
+        unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            st_relaxed_u64(dst + e * 32, ((unsigned long long)a.epoch << 32) | __float_as_uint(incv[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sm.cin[e][lane] = carry[e];
+}
 
 __device__ void finalize(const Args &a, int k, bool resid)
 {
@@ -86,222 +285,240 @@ __device__ void finalize(const Args &a, int k, bool resid)
 template <int FORGET, bool FIRST, bool RESID>
 __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
 {
-    __shared__ float s_agg[NW][20][32];
-    __shared__ float s_cin[4][32];
-    __shared__ float s_red[2][NW];
-    __shared__ unsigned s_ticket;
-    __shared__ int s_exit;
-
+    extern __shared__ float4 smem_f4[];
+    Smem &sm = *reinterpret_cast<Smem *>(smem_f4);
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    NewtonSlot &slot = a.ctrl->slot[k & 1];
+
     if (threadIdx.x == 0) {
-        const unsigned ex = *(volatile unsigned *)&a.ctrl->done;
-        s_exit = (int)ex;
-        if (!ex) s_ticket = atomicAdd(&a.ctrl->slot[k & 1].ticket, 1u);
+        sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
+        if (!sm.exit_flag) {
+            sm.tick[0] = atomicAdd(&slot.ticket, 1u);
+            sm.tick[1] = atomicAdd(&slot.ticket, 1u);
+        }
     }
     __syncthreads();
-    if (s_exit) return;
+    if (sm.exit_flag) return;
 
-    const unsigned ticket = s_ticket;
-    const int G = a.lb.n_groups;
-    const int chunk = (int)(ticket / (unsigned)G);
-    const int grp = (int)(ticket % (unsigned)G);
-    const int b = grp / a.groups_per_row;
-    const int j = (grp % a.groups_per_row) * 32 + lane;
-    const bool jv = j < a.d;
     const size_t d = (size_t)a.d;
     const int T = a.T;
-    const int t_seg = chunk * TT + warp * L;
-    const size_t row0 = (size_t)b * T;  // (b, t) row = row0 + t
-    const size_t jj = jv ? (size_t)j : 0;
+    const int G = a.n_groups;
+    float mx_raw = 0.f, mx_sc = 0.f;
 
-    float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-    if (jv) {
-        rz = a.R[jj];
-        ri = a.R[d + jj];
-        rf = a.R[2 * d + jj];
-        ro = a.R[3 * d + jj];
-    }
+    unsigned cur = sm.tick[0];
+    unsigned nxt = sm.tick[1];
+    int st = 0;
+    prefetch_tile(a, sm, 0, cur, !FIRST);
+    cp_async_commit();
 
-    // old state just before this warp's segment
-    float sp[4] = {0.f, 0.f, 0.f, 0.f};
-    if (t_seg == 0) {
-        if (a.s0 && jv) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sp[e] = a.s0[((size_t)b * 4 + e) * d + jj];
+    while (cur < (unsigned)a.n_tiles) {
+        // tickets run two tiles ahead: fetch the one after `nxt` now, publish it at the end
+        unsigned after = 0;
+        if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
+        prefetch_tile(a, sm, st ^ 1, nxt, !FIRST);
+        cp_async_commit();
+        cp_async_wait_prev();   // the current tile's copies have landed
+        __syncthreads();
+
+        const unsigned ticket = cur;
+        const int chunk = (int)(ticket / (unsigned)G);
+        const int grp = (int)(ticket % (unsigned)G);
+        const int b = grp / a.groups_per_row;
+        const int j = (grp % a.groups_per_row) * 32 + lane;
+        const bool jv = j < a.d;
+        const size_t jj = jv ? (size_t)j : 0;
+        const int t_seg = chunk * TT + warp * L;
+        const size_t row0 = (size_t)b * T;
+
+        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
+        if (jv) {
+            rz = __ldg(a.R + jj);
+            ri = __ldg(a.R + d + jj);
+            rf = __ldg(a.R + 2 * d + jj);
+            ro = __ldg(a.R + 3 * d + jj);
         }
-    } else if (!FIRST) {
-        if (warp == 0) {
-            const float *src = a.bnd_in + (size_t)(ticket - (unsigned)G) * 4 * 32;
+        // old state just before this warp's segment
+        float sp[4] = {0.f, 0.f, 0.f, 0.f};
+        if (t_seg == 0) {
+            if (a.s0 && jv) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
-        } else if (jv) {
-            const float *src = a.S + (row0 + t_seg - 1) * 4 * d + jj;
+                for (int e = 0; e < 4; ++e) sp[e] = __ldg(a.s0 + ((size_t)b * 4 + e) * d + jj);
+            }
+        } else if (!FIRST) {
+            if (warp == 0) {
+                const float *src = a.bnd_in + (size_t)(ticket - (unsigned)G) * 4 * 32;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sp[e] = src[e * d];
+                for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sp[e] = sm.S[st][warp * L - 1][e][lane];
+            }
         }
-    }
 
-    // ---- walk A ----
-    Cell Jc[L];
-    float rr[L][4];
-    Aff agg;
-    aff_identity(agg);
-    {
-        float cur[4] = {sp[0], sp[1], sp[2], sp[3]};
+        // ---- walk A ----
+        Cell Jc[L];
+        float rr[L][4];
+        Aff agg;
+        aff_identity(agg);
+        {
+            float curS[4] = {sp[0], sp[1], sp[2], sp[3]};
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int t = t_seg + i;
+                const int sl = warp * L + i;
+                if (t < T) {
+                    float so[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (!FIRST) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) so[e] = sm.S[st][sl][e][lane];
+                    }
+                    cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
+                                            sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz,
+                                            ri, rf, ro, Jc[i]);
+                    rr[i][0] = Jc[i].c - so[0];
+                    rr[i][1] = Jc[i].n - so[1];
+                    rr[i][2] = Jc[i].m - so[2];
+                    rr[i][3] = Jc[i].h - so[3];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) curS[e] = so[e];
+                } else {
+                    cell_identity(Jc[i]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) rr[i][e] = 0.f;
+                }
+                fold_jac(agg, Jc[i], rr[i]);
+            }
+        }
+        store_aff_smem(sm.agg, warp, lane, agg);
+        __syncthreads();
+        tile_prefix_tree<NW>(sm.agg, agg);
+        if (warp == 0) tile_carry_warp0(a, sm, ticket, chunk, grp, (k == 0) && ((int)ticket == a.fault_ticket));
+        __syncthreads();
+
+        // ---- walk B ----
+        float dl[4];
+        warp_carry(sm.agg, sm.cin, warp, lane, dl);
+        float snp[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int t = t_seg + i;
+            const int sl = warp * L + i;
             if (t < T) {
-                float p[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
-                if (jv) {
-                    const float *pp = a.P + (row0 + t) * 4 * d + jj;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) p[e] = __ldg(pp + e * d);
-                    if (!FIRST) {
-                        const float *sq = a.S + (row0 + t) * 4 * d + jj;
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) so[e] = sq[e * d];
-                    }
-                }
-                cell_eval<FORGET, true>(cur[0], cur[1], cur[2], cur[3], p[0], p[1], p[2], p[3], rz,
-                                        ri, rf, ro, Jc[i]);
-                rr[i][0] = Jc[i].c - so[0];
-                rr[i][1] = Jc[i].n - so[1];
-                rr[i][2] = Jc[i].m - so[2];
-                rr[i][3] = Jc[i].h - so[3];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) cur[e] = so[e];
-            } else {
-                cell_identity(Jc[i]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) rr[i][e] = 0.f;
-            }
-            fold_jac(agg, Jc[i], rr[i]);
-        }
-    }
-    store_aff_smem(s_agg, warp, lane, agg);
-    __syncthreads();
-    tile_prefix_tree<NW>(s_agg, agg);
-
-    if (warp == 0) {
-        const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-        const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
-        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, zero, withhold);
-    }
-    __syncthreads();
-
-    // ---- walk B ----
-    float dl[4];
-    warp_carry(s_agg, s_cin, warp, lane, dl);
-    float snp[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
-    float mx_raw = 0.f, mx_sc = 0.f;
-#pragma unroll
-    for (int i = 0; i < L; ++i) {
-        const int t = t_seg + i;
-        if (t < T) {
-            jac_mul(Jc[i], dl[0], dl[1], dl[2], dl[3]);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dl[e] += rr[i][e];
-            float sn[4];
-            if (jv) {
-                float *sq = a.S + (row0 + t) * 4 * d + jj;
+                jac_mul(Jc[i], dl[0], dl[1], dl[2], dl[3]);
+                float sn[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float so = FIRST ? 0.f : sq[e * d];
-                    sn[e] = so + dl[e];
-                    sq[e * d] = sn[e];
+                    dl[e] += rr[i][e];
+                    sn[e] = (FIRST ? 0.f : sm.S[st][sl][e][lane]) + dl[e];
                 }
-                if (RESID) {
-                    const float *pp = a.P + (row0 + t) * 4 * d + jj;
-                    Cell f;
-                    cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], __ldg(pp), __ldg(pp + d),
-                                             __ldg(pp + 2 * d), __ldg(pp + 3 * d), rz, ri, rf, ro, f);
-                    const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+                if (jv) {
+                    float *sq = a.S + (row0 + t) * 4 * d + jj;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float af = fabsf(F[e]);
-                        const float sc = af / (1.0f + fabsf(sn[e]));
-                        // propagate NaN: a NaN compares false, so test "not <="
-                        mx_raw = (af <= mx_raw) ? mx_raw : af;
-                        mx_sc = (sc <= mx_sc) ? mx_sc : sc;
+                    for (int e = 0; e < 4; ++e) sq[e * d] = sn[e];
+                    if (RESID) {
+                        Cell f;
+                        cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
+                                                 sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane],
+                                                 rz, ri, rf, ro, f);
+                        const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float af = fabsf(F[e]);
+                            const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
+                            // keep NaN: a NaN compares false, so test "not <="
+                            mx_raw = (af <= mx_raw) ? mx_raw : af;
+                            mx_sc = (sc <= mx_sc) ? mx_sc : sc;
+                        }
                     }
                 }
-            } else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sn[e] = 0.f;
+                for (int e = 0; e < 4; ++e) snp[e] = sn[e];
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) snp[e] = sn[e];
         }
-    }
-    // state at the tile's last step, for the next launch's successor tile
-    if (warp == NW - 1 && t_seg + L - 1 < T) {
-        float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
+        // state at the tile's last step, for the next launch's successor tile
+        if (warp == NW - 1 && t_seg + L - 1 < T) {
+            float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
+            for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
+        }
+
+        if (threadIdx.x == 0) sm.tick[0] = after;
+        __syncthreads();   // stage `st` and sm.agg are free again
+        cur = nxt;
+        nxt = sm.tick[0];
+        st ^= 1;
     }
+    cp_async_wait_all();
 
     if (RESID) {
         mx_raw = warp_max(mx_raw);
         mx_sc = warp_max(mx_sc);
         if (lane == 0) {
-            s_red[0][warp] = mx_raw;
-            s_red[1][warp] = mx_sc;
+            sm.red[0][warp] = mx_raw;
+            sm.red[1][warp] = mx_sc;
         }
     }
     __syncthreads();
     if (threadIdx.x == 0) {
         if (RESID) {
-            float r0 = s_red[0][0], r1 = s_red[1][0];
+            float r0 = sm.red[0][0], r1 = sm.red[1][0];
             for (int w = 1; w < NW; ++w) {
-                r0 = (__float_as_uint(s_red[0][w]) > __float_as_uint(r0)) ? s_red[0][w] : r0;
-                r1 = (__float_as_uint(s_red[1][w]) > __float_as_uint(r1)) ? s_red[1][w] : r1;
+                r0 = (__float_as_uint(sm.red[0][w]) > __float_as_uint(r0)) ? sm.red[0][w] : r0;
+                r1 = (__float_as_uint(sm.red[1][w]) > __float_as_uint(r1)) ? sm.red[1][w] : r1;
             }
-            atomic_max_nonneg(&a.ctrl->slot[k & 1].maxF_raw, r0);
-            atomic_max_nonneg(&a.ctrl->slot[k & 1].maxF_scaled, r1);
+            atomic_max_nonneg(&slot.maxF_raw, r0);
+            atomic_max_nonneg(&slot.maxF_scaled, r1);
         }
         __threadfence();
-        const unsigned fin = atomicAdd(&a.ctrl->slot[k & 1].finished, 1u);
-        if (fin == (unsigned)a.n_tiles - 1u) {
+        const unsigned fin = atomicAdd(&slot.finished, 1u);
+        if (fin == gridDim.x - 1u) {
             __threadfence();
             finalize(a, k, RESID);
         }
     }
 }
 
-template <int FORGET>
-cudaError_t launch_iters(const Args &base, int max_iters, bool fixed, cudaStream_t st)
+template <int FORGET, bool FIRST, bool RESID>
+cudaError_t launch_one(const Args &a, int k, int sms, cudaStream_t st)
 {
-    const dim3 block(NW * 32);
-    const dim3 grid(base.n_tiles);
+    auto kern = newton_iter<FORGET, FIRST, RESID>;
+    static int blocks_per_sm = 0;
+    if (blocks_per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, sizeof(Smem));
+        if (e != cudaSuccess) return e;
+        if (blocks_per_sm < 1) blocks_per_sm = 1;
+    }
+    const int grid = min(a.n_tiles, sms * blocks_per_sm);
+    kern<<<grid, NW * 32, sizeof(Smem), st>>>(a, k);
+    return cudaGetLastError();
+}
+
+template <int FORGET>
+cudaError_t launch_iters(const Args &base, int max_iters, bool fixed, int sms, cudaStream_t st)
+{
     for (int k = 0; k < max_iters; ++k) {
         Args a = base;
-        a.lb.epoch = (unsigned)(k + 1);
+        a.epoch = (unsigned)(k + 1);
         a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
         a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
         const bool resid = !fixed || (k + 1 == max_iters);
-        if (k == 0) {
-            if (resid)
-                newton_iter<FORGET, true, true><<<grid, block, 0, st>>>(a, k);
-            else
-                newton_iter<FORGET, true, false><<<grid, block, 0, st>>>(a, k);
-        } else {
-            if (resid)
-                newton_iter<FORGET, false, true><<<grid, block, 0, st>>>(a, k);
-            else
-                newton_iter<FORGET, false, false><<<grid, block, 0, st>>>(a, k);
-        }
-        const cudaError_t e = cudaGetLastError();
+        cudaError_t e;
+        if (k == 0)
+            e = resid ? launch_one<FORGET, true, true>(a, k, sms, st) : launch_one<FORGET, true, false>(a, k, sms, st);
+        else
+            e = resid ? launch_one<FORGET, false, true>(a, k, sms, st) : launch_one<FORGET, false, false>(a, k, sms, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 struct Layout {
-    size_t ctrl, flags, agg, inc, bnd0, bnd1, total;
+    size_t ctrl, flags, incw, agg, bnd0, bnd1, total;
     int groups_per_row, n_groups, n_chunks, n_tiles;
 };
 
@@ -320,12 +537,24 @@ Layout layout(int B, int T, int d)
     };
     l.ctrl = take(sizeof(NewtonCtrl));
     l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles);
+    l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles);
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
-    l.inc = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.bnd0 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.bnd1 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.total = off;
     return l;
+}
+
+int sm_count()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+    }
+    return n;
 }
 
 }  // namespace
@@ -344,34 +573,38 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     a.s0 = s0;
     a.S = S;
     a.ctrl = reinterpret_cast<NewtonCtrl *>(base + l.ctrl);
-    a.lb.flags = reinterpret_cast<unsigned *>(base + l.flags);
-    a.lb.agg = reinterpret_cast<float *>(base + l.agg);
-    a.lb.inc = reinterpret_cast<float *>(base + l.inc);
-    a.lb.error = &a.ctrl->error;
-    a.lb.epoch = 1;
-    a.lb.wait_ns = (uint64_t)(cfg.wait_limit_us > 0 ? cfg.wait_limit_us : 2000000) * 1000ull;
-    a.lb.n_groups = l.n_groups;
+    a.flags = reinterpret_cast<unsigned *>(base + l.flags);
+    a.agg = reinterpret_cast<float *>(base + l.agg);
+    a.incw = reinterpret_cast<unsigned long long *>(base + l.incw);
     a.bnd_in = reinterpret_cast<float *>(base + l.bnd0);
     a.bnd_out = reinterpret_cast<float *>(base + l.bnd1);
     a.stats = stats;
+    a.error = &a.ctrl->error;
+    a.epoch = 1;
+    a.wait_ns = (unsigned long long)(cfg.wait_limit_us > 0 ? cfg.wait_limit_us : 2000000) * 1000ull;
     a.B = B;
     a.T = T;
     a.d = d;
     a.groups_per_row = l.groups_per_row;
+    a.n_groups = l.n_groups;
     a.n_tiles = l.n_tiles;
     a.max_iters = cfg.max_iters;
     a.fixed = cfg.fixed_iters ? 1 : 0;
     a.tol = cfg.tol;
+    a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(P) & 15) == 0 &&
+               (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
     // fault injection: the first tile of chunk 1 withholds its publications,
     // so the first tile of chunk 2 has nothing to wait for
     a.fault_ticket = (cfg.debug_fault == 1 && l.n_chunks >= 3) ? l.n_groups : -1;
 
-    cudaError_t e = cudaMemsetAsync(base + l.ctrl, 0, sizeof(NewtonCtrl), st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(base + l.flags, 0, sizeof(unsigned) * l.n_tiles, st);
+    // control block, aggregate flags and the epoch tags of the inclusive
+    // prefixes start cleared on every call
+    cudaError_t e = cudaMemsetAsync(base + l.ctrl, 0, l.agg - l.ctrl, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(slstm_newton_stats), st);
     if (e != cudaSuccess) return e;
-    if (cfg.forget == SLSTM_FORGET_EXP) return launch_iters<SLSTM_FORGET_EXP>(a, cfg.max_iters, a.fixed, st);
-    return launch_iters<SLSTM_FORGET_SIGMOID>(a, cfg.max_iters, a.fixed, st);
+    const int sms = sm_count();
+    if (cfg.forget == SLSTM_FORGET_EXP) return launch_iters<SLSTM_FORGET_EXP>(a, cfg.max_iters, a.fixed, sms, st);
+    return launch_iters<SLSTM_FORGET_SIGMOID>(a, cfg.max_iters, a.fixed, sms, st);
 }
 
 }  // namespace slstm
