@@ -70,7 +70,7 @@ struct Smem {
     float P[2][TT][4][32];
     float S[2][TT][4][32];
     float agg[NW][20][32];
-    float cin[4][32];
+    float cin[NW][4][32];
     float red[2][NW];
     unsigned tick[2];
     int exit_flag;
@@ -168,13 +168,14 @@ SLSTM_DEVINL bool read_inc(const Args &a, unsigned tq, int lane, float v[4])
     return ok;
 }
 
-// Warp 0: carry entering the tile (written to sm.cin) and publication of the
-// tile's inclusive prefix; sm.agg holds the warps' inclusive prefixes.
+// Warp 0: carries entering every warp of the tile (written to sm.cin) and
+// publication of the tile's inclusive prefix; sm.agg[w] holds warp w's own
+// aggregate.  When the predecessor has published (the common case) only
+// vectors are propagated: v_{w+1} = A_w v_w + b_w.  The tile aggregate (a
+// fold of 4x4 maps) is formed only when it has to be published.
 SLSTM_DEVINL void tile_carry_warp0(const Args &a, Smem &sm, unsigned ticket, int chunk, int grp, bool withhold)
 {
     const int lane = threadIdx.x & 31;
-    Aff tile;
-    load_aff_smem(sm.agg, NW - 1, lane, tile);
     float carry[4] = {0.f, 0.f, 0.f, 0.f};
     if (chunk > 0) {
         unsigned tq = ticket - (unsigned)a.n_groups;
@@ -186,6 +187,13 @@ SLSTM_DEVINL void tile_carry_warp0(const Args &a, Smem &sm, unsigned ticket, int
         } else {
             // predecessor unfinished: publish the aggregate so that later
             // tiles can skip over this one, then look back
+            Aff tile;
+            load_aff_smem(sm.agg, 0, lane, tile);
+            for (int w = 1; w < NW; ++w) {
+                Aff x;
+                load_aff_smem(sm.agg, w, lane, x);
+                aff_compose(x, tile, tile);
+            }
             if (!withhold) {
                 float *dst = a.agg + (size_t)ticket * 20 * 32;
 #pragma unroll
@@ -229,16 +237,21 @@ SLSTM_DEVINL void tile_carry_warp0(const Args &a, Smem &sm, unsigned ticket, int
             }
         }
     }
+    // carries of the warps, then the tile's inclusive prefix
+    float v[4] = {carry[0], carry[1], carry[2], carry[3]};
+    for (int w = 0; w < NW; ++w) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sm.cin[w][e][lane] = v[e];
+        Aff x;
+        load_aff_smem(sm.agg, w, lane, x);
+        aff_apply(x, v, v);
+    }
     if (!withhold) {
-        float incv[4];
-        aff_apply(tile, carry, incv);
         unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            st_relaxed_u64(dst + e * 32, ((unsigned long long)a.epoch << 32) | __float_as_uint(incv[e]));
+            st_relaxed_u64(dst + e * 32, ((unsigned long long)a.epoch << 32) | __float_as_uint(v[e]));
     }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sm.cin[e][lane] = carry[e];
 }
 
 __device__ void finalize(const Args &a, int k, bool resid)
@@ -357,8 +370,8 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         }
 
         // ---- walk A ----
+        // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B
         Cell Jc[L];
-        float rr[L][4];
         Aff agg;
         aff_identity(agg);
         {
@@ -367,6 +380,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             for (int i = 0; i < L; ++i) {
                 const int t = t_seg + i;
                 const int sl = warp * L + i;
+                float r[4] = {0.f, 0.f, 0.f, 0.f};
                 if (t < T) {
                     float so[4] = {0.f, 0.f, 0.f, 0.f};
                     if (!FIRST) {
@@ -376,29 +390,27 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
                     cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
                                             sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz,
                                             ri, rf, ro, Jc[i]);
-                    rr[i][0] = Jc[i].c - so[0];
-                    rr[i][1] = Jc[i].n - so[1];
-                    rr[i][2] = Jc[i].m - so[2];
-                    rr[i][3] = Jc[i].h - so[3];
+                    r[0] = Jc[i].c - so[0];
+                    r[1] = Jc[i].n - so[1];
+                    r[2] = Jc[i].m - so[2];
+                    r[3] = Jc[i].h - so[3];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) curS[e] = so[e];
                 } else {
                     cell_identity(Jc[i]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) rr[i][e] = 0.f;
                 }
-                fold_jac(agg, Jc[i], rr[i]);
+                fold_jac(agg, Jc[i], r);
             }
         }
         store_aff_smem(sm.agg, warp, lane, agg);
         __syncthreads();
-        tile_prefix_tree<NW>(sm.agg, agg);
         if (warp == 0) tile_carry_warp0(a, sm, ticket, chunk, grp, (k == 0) && ((int)ticket == a.fault_ticket));
         __syncthreads();
 
         // ---- walk B ----
         float dl[4];
-        warp_carry(sm.agg, sm.cin, warp, lane, dl);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dl[e] = sm.cin[warp][e][lane];
         float snp[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
@@ -408,11 +420,13 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             const int sl = warp * L + i;
             if (t < T) {
                 jac_mul(Jc[i], dl[0], dl[1], dl[2], dl[3]);
+                const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
                 float sn[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    dl[e] += rr[i][e];
-                    sn[e] = (FIRST ? 0.f : sm.S[st][sl][e][lane]) + dl[e];
+                    const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
+                    dl[e] += f4[e] - so;   // delta_t = J_t delta_{t-1} + (f_t - S_t)
+                    sn[e] = so + dl[e];
                 }
                 if (jv) {
                     float *sq = a.S + (row0 + t) * 4 * d + jj;
