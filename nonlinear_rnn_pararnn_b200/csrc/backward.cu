@@ -34,8 +34,24 @@ struct BwdArgs {
     float *partial;   // [n_tiles][8][32]  dR (4) then db (4)
     float *ds0;       // (B, 4, d) or null
     unsigned *ticket;
-    LookbackArgs lb;
-    int T, d, groups_per_row;
+    CarryArgs ca;
+    int T, d, groups_per_row, n_tiles, vec16;
+};
+
+// Shared memory of one CTA.  A tile covers steps t in [t_lo, t_hi] with
+// t_hi = T-1-32c and t_lo = t_hi-31 (chunk c in reverse time order); it
+// needs S at t_lo-1 .. t_hi, P at t_lo .. t_hi+1 and dH at t_lo .. t_hi.
+struct BwdSmem {
+    float S[2][TT + 1][4][32];   // row r <-> t = t_lo - 1 + r
+    float P[2][TT + 1][4][32];   // row r <-> t = t_lo + r
+    float dH[2][TT][32];         // row r <-> t = t_lo + r
+    union {
+        float agg[NW][20][32];
+        __nv_bfloat16 dpt[2][4][32][TT + 2];   // transposed staging of the dP pair
+    } u;
+    float cin[NW][4][32];
+    float part[NW][8][32];
+    unsigned tick[2];
 };
 
 SLSTM_DEVINL void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
@@ -44,179 +60,231 @@ SLSTM_DEVINL void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
     lo = __float2bfloat16_rn(v - __bfloat162float(hi));
 }
 
-template <int FORGET, bool BF16OUT>
-__global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
+// Copies of one tile's S, P and dH rows into stage `st`; rows outside [0, T)
+// and features past d arrive as zeros.
+SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, unsigned ticket)
 {
-    __shared__ float s_agg[NW][20][32];
-    __shared__ float s_cin[4][32];
-    __shared__ float s_part[NW][8][32];
-    // transposed staging of the tile's dP pair: [hi/lo][gate][feature][step]
-    __shared__ __nv_bfloat16 s_dpt[BF16OUT ? 2 : 1][4][32][TT + 2];
-    __shared__ unsigned s_ticket;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1u);
-    __syncthreads();
-    const unsigned ticket = s_ticket;
-    const int G = a.lb.n_groups;
+    if (ticket >= (unsigned)a.n_tiles) return;
+    const int G = a.ca.n_groups;
     const int chunk = (int)(ticket / (unsigned)G);
     const int grp = (int)(ticket % (unsigned)G);
     const int b = grp / a.groups_per_row;
-    const int j = (grp % a.groups_per_row) * 32 + lane;
-    const bool jv = j < a.d;
-    const size_t jj = jv ? (size_t)j : 0;
+    const int j0 = (grp % a.groups_per_row) * 32;
+    const int t_lo = a.T - (chunk + 1) * TT;
     const size_t d = (size_t)a.d;
+    const size_t row0 = (size_t)b * a.T;
+    const int valid = min(32, a.d - j0);
+    const int per = a.vec16 ? 8 : 32;         // copies per 32-float row
+    const int rows4 = (TT + 1) * 4;            // (row, slot) pairs of S and of P
+    const int total = (2 * rows4 + TT) * per;
+    for (int idx = threadIdx.x; idx < total; idx += NW * 32) {
+        const int row = idx / per, part = idx % per;
+        float *dst;
+        const float *src;
+        int t;
+        if (row < rows4) {                     // S
+            const int r = row >> 2, slot = row & 3;
+            t = t_lo - 1 + r;
+            dst = &sm.S[st][r][slot][0];
+            src = a.S + ((row0 + (size_t)min(max(t, 0), a.T - 1)) * 4 + slot) * d + j0;
+        } else if (row < 2 * rows4) {          // P
+            const int r = (row - rows4) >> 2, slot = (row - rows4) & 3;
+            t = t_lo + r;
+            dst = &sm.P[st][r][slot][0];
+            src = a.P + ((row0 + (size_t)min(max(t, 0), a.T - 1)) * 4 + slot) * d + j0;
+        } else {                               // dH
+            const int r = row - 2 * rows4;
+            t = t_lo + r;
+            dst = &sm.dH[st][r][0];
+            src = a.dH + (row0 + (size_t)min(max(t, 0), a.T - 1)) * d + j0;
+        }
+        const bool in = (t >= 0 && t < a.T);
+        copy_row32(dst, src, in ? valid : 0, a.vec16 != 0, part);
+    }
+}
+
+template <int FORGET, bool BF16OUT>
+__global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
+{
+    extern __shared__ float4 smem_f4[];
+    BwdSmem &sm = *reinterpret_cast<BwdSmem *>(smem_f4);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int G = a.ca.n_groups;
     const int T = a.T;
-    const size_t row0 = (size_t)b * T;
-    const int p_seg = chunk * TT + warp * L;  // processing position; t = T-1-p
+    const size_t d = (size_t)a.d;
 
-    float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-    if (jv) {
-        rz = a.R[jj];
-        ri = a.R[d + jj];
-        rf = a.R[2 * d + jj];
-        ro = a.R[3 * d + jj];
-    }
-    float s0v[4] = {0.f, 0.f, 0.f, 0.f};
-    if (a.s0 && jv) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s0v[e] = a.s0[((size_t)b * 4 + e) * d + jj];
-    }
-
-    // ---- walk A: fold lambda -> J_{t+1}^T lambda + e_h dH_t, t descending ----
-    Cell Jn[L];  // J_{t+1} for each step of the segment
-    float dh[L];
-    Aff agg;
-    aff_identity(agg);
-#pragma unroll
-    for (int i = 0; i < L; ++i) {
-        const int p = p_seg + i;
-        const int t = T - 1 - p;
-        dh[i] = 0.f;
-        cell_identity(Jn[i]);
-        if (p < T && jv) {
-            dh[i] = a.dH[(row0 + t) * d + jj];
-            if (t + 1 < T) {
-                const float *ps = a.S + (row0 + t) * 4 * d + jj;
-                const float *pp = a.P + (row0 + t + 1) * 4 * d + jj;
-                cell_eval<FORGET, true>(ps[0], ps[d], ps[2 * d], ps[3 * d], __ldg(pp), __ldg(pp + d),
-                                        __ldg(pp + 2 * d), __ldg(pp + 3 * d), rz, ri, rf, ro, Jn[i]);
-            } else {
-                // lambda past the end is zero, so the map's matrix is irrelevant
-            }
-        }
-        const float r[4] = {0.f, 0.f, 0.f, dh[i]};
-        fold_jacT(agg, Jn[i], r);
-    }
-    store_aff_smem(s_agg, warp, lane, agg);
-    __syncthreads();
-    tile_prefix_tree<NW>(s_agg, agg);
-    if (warp == 0) {
-        const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, zero, false);
+    if (threadIdx.x == 0) {
+        sm.tick[0] = atomicAdd(a.ticket, 1u);
+        sm.tick[1] = atomicAdd(a.ticket, 1u);
     }
     __syncthreads();
+    unsigned cur = sm.tick[0];
+    unsigned nxt = sm.tick[1];
+    int st = 0;
+    bwd_prefetch(a, sm, 0, cur);
+    cp_async_commit();
 
-    // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
-    float lam[4];
-    warp_carry(s_agg, s_cin, warp, lane, lam);
-    float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < L; ++i) {
-        const int p = p_seg + i;
-        const int t = T - 1 - p;
-        if (p < T && jv) {
-            jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
-            lam[3] += dh[i];
-            float prev[4];
-            if (t == 0) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = s0v[e];
-            } else {
-                const float *ps = a.S + (row0 + t - 1) * 4 * d + jj;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = ps[e * d];
-            }
-            const float *pp = a.P + (row0 + t) * 4 * d + jj;
-            Cell c;
-            CellG g;
-            cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], __ldg(pp), __ldg(pp + d),
-                                          __ldg(pp + 2 * d), __ldg(pp + 3 * d), rz, ri, rf, ro, c, &g);
-            const float dz = fmaf(g.gcz, lam[0], g.ghz * lam[3]);
-            const float di = fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3])));
-            const float df = fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3])));
-            const float dq = g.gho * lam[3];
-            if (BF16OUT) {
-                const float dv[4] = {dz, di, df, dq};
-                const size_t o = (row0 + t) * 4 * d + jj;
-                const int tl = TT - 1 - (warp * L + i);   // step index inside the tile, ascending in t
-#pragma unroll
-                for (int gi = 0; gi < 4; ++gi) {
-                    __nv_bfloat16 hi, lo;
-                    split_bf16(dv[gi], hi, lo);
-                    a.dp_hi[o + gi * d] = hi;
-                    a.dp_lo[o + gi * d] = lo;
-                    s_dpt[0][gi][lane][tl] = hi;
-                    s_dpt[BF16OUT ? 1 : 0][gi][lane][tl] = lo;
-                }
-            } else {
-                float *pd = a.dP + (row0 + t) * 4 * d + jj;
-                pd[0] = dz;
-                pd[d] = di;
-                pd[2 * d] = df;
-                pd[3 * d] = dq;
-            }
-            const float hp = prev[3];
-            dr[0] = fmaf(dz, hp, dr[0]);
-            dr[1] = fmaf(di, hp, dr[1]);
-            dr[2] = fmaf(df, hp, dr[2]);
-            dr[3] = fmaf(dq, hp, dr[3]);
-            dbs[0] += dz;
-            dbs[1] += di;
-            dbs[2] += df;
-            dbs[3] += dq;
-            if (t == 0 && a.ds0) {
-                float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
-                jacT_mul(c, v0, v1, v2, v3);
-                float *q = a.ds0 + (size_t)b * 4 * d + jj;
-                q[0] = v0;
-                q[d] = v1;
-                q[2 * d] = v2;
-                q[3 * d] = v3;
-            }
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        s_part[warp][e][lane] = dr[e];
-        s_part[warp][4 + e][lane] = dbs[e];
-    }
-    __syncthreads();
-    {
-        // 256 threads: thread (e, lane) sums entry e over the warps
-        const int e = threadIdx.x >> 5;  // 0..7
-        float acc = 0.f;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) acc += s_part[w][e][lane];
-        a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
-    }
-    if (BF16OUT) {
-        // rows (g, j) of the transposed pair: 32 consecutive steps each; the
-        // tile covers t in [t_lo, t_lo + TT) clipped to [0, T)
+    while (cur < (unsigned)a.n_tiles) {
+        unsigned after = 0;
+        if (threadIdx.x == 0) after = atomicAdd(a.ticket, 1u);
+        bwd_prefetch(a, sm, st ^ 1, nxt);
+        cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();
+
+        const unsigned ticket = cur;
+        const int chunk = (int)(ticket / (unsigned)G);
+        const int grp = (int)(ticket % (unsigned)G);
+        const int b = grp / a.groups_per_row;
+        const int j = (grp % a.groups_per_row) * 32 + lane;
+        const bool jv = j < a.d;
+        const size_t jj = jv ? (size_t)j : 0;
+        const size_t row0 = (size_t)b * T;
         const int t_lo = T - (chunk + 1) * TT;
-        const int tl = threadIdx.x & 31;
-        const int t = t_lo + tl;
-        const int j0 = (grp % a.groups_per_row) * 32;
-        for (int r = threadIdx.x >> 5; r < 2 * 4 * 32; r += NW) {
-            const int part = r >> 7;
-            const int gi = (r >> 5) & 3;
-            const int jl = r & 31;
-            if (t >= 0 && j0 + jl < a.d) {
-                __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
-                dst[((size_t)gi * d + j0 + jl) * a.ldT + row0 + t] = s_dpt[part][gi][jl][tl];
+
+        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
+        if (jv) {
+            rz = __ldg(a.R + jj);
+            ri = __ldg(a.R + d + jj);
+            rf = __ldg(a.R + 2 * d + jj);
+            ro = __ldg(a.R + 3 * d + jj);
+        }
+
+        // ---- walk A: fold lambda -> J_{t+1}^T lambda + e_h dH_t, t descending ----
+        Cell Jn[L];   // J_{t+1} of each step
+        Aff agg;
+        aff_identity(agg);
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int rl = TT - 1 - (warp * L + i);   // t - t_lo
+            const int t = t_lo + rl;
+            cell_identity(Jn[i]);
+            float r[4] = {0.f, 0.f, 0.f, 0.f};
+            if (t >= 0) {
+                r[3] = sm.dH[st][rl][lane];
+                if (t + 1 < T)
+                    cell_eval<FORGET, true>(sm.S[st][rl + 1][0][lane], sm.S[st][rl + 1][1][lane],
+                                            sm.S[st][rl + 1][2][lane], sm.S[st][rl + 1][3][lane],
+                                            sm.P[st][rl + 1][0][lane], sm.P[st][rl + 1][1][lane],
+                                            sm.P[st][rl + 1][2][lane], sm.P[st][rl + 1][3][lane], rz, ri, rf, ro, Jn[i]);
+            }
+            fold_jacT(agg, Jn[i], r);
+        }
+        store_aff_smem(sm.u.agg, warp, lane, agg);
+        __syncthreads();
+        if (warp == 0) {
+            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+            tile_carry_serial<NW>(a.ca, sm.u.agg, sm.cin, ticket, chunk, grp, zero, false);
+        }
+        __syncthreads();   // sm.u.agg is dead from here on; sm.u.dpt takes its place
+
+        // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
+        float lam[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][lane];
+        float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int rl = TT - 1 - (warp * L + i);
+            const int t = t_lo + rl;
+            if (t >= 0) {
+                jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
+                lam[3] += sm.dH[st][rl][lane];
+                float prev[4];
+                if (t == 0) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + ((size_t)b * 4 + e) * d + jj) : 0.f;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
+                }
+                Cell c;
+                CellG g;
+                cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
+                                              sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
+                                              ri, rf, ro, c, &g);
+                const float dz = fmaf(g.gcz, lam[0], g.ghz * lam[3]);
+                const float di = fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3])));
+                const float df = fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3])));
+                const float dq = g.gho * lam[3];
+                if (BF16OUT) {
+                    const float dv[4] = {dz, di, df, dq};
+                    const size_t o = (row0 + t) * 4 * d + jj;
+#pragma unroll
+                    for (int gi = 0; gi < 4; ++gi) {
+                        __nv_bfloat16 hi, lo;
+                        split_bf16(dv[gi], hi, lo);
+                        if (jv) {
+                            a.dp_hi[o + gi * d] = hi;
+                            a.dp_lo[o + gi * d] = lo;
+                        }
+                        sm.u.dpt[0][gi][lane][rl] = hi;
+                        sm.u.dpt[1][gi][lane][rl] = lo;
+                    }
+                } else if (jv) {
+                    float *pd = a.dP + (row0 + t) * 4 * d + jj;
+                    pd[0] = dz;
+                    pd[d] = di;
+                    pd[2 * d] = df;
+                    pd[3 * d] = dq;
+                }
+                const float hp = prev[3];
+                dr[0] = fmaf(dz, hp, dr[0]);
+                dr[1] = fmaf(di, hp, dr[1]);
+                dr[2] = fmaf(df, hp, dr[2]);
+                dr[3] = fmaf(dq, hp, dr[3]);
+                dbs[0] += dz;
+                dbs[1] += di;
+                dbs[2] += df;
+                dbs[3] += dq;
+                if (t == 0 && a.ds0 && jv) {
+                    float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
+                    jacT_mul(c, v0, v1, v2, v3);
+                    float *q = a.ds0 + (size_t)b * 4 * d + jj;
+                    q[0] = v0;
+                    q[d] = v1;
+                    q[2 * d] = v2;
+                    q[3 * d] = v3;
+                }
             }
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sm.part[warp][e][lane] = jv ? dr[e] : 0.f;
+            sm.part[warp][4 + e][lane] = jv ? dbs[e] : 0.f;
+        }
+        __syncthreads();
+        {
+            // 256 threads: thread (e, lane) sums entry e over the warps
+            const int e = threadIdx.x >> 5;   // 0..7
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) acc += sm.part[w][e][lane];
+            a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
+        }
+        if (BF16OUT) {
+            // rows (g, j) of the transposed pair: up to 32 consecutive steps each
+            const int tl = threadIdx.x & 31;
+            const int t = t_lo + tl;
+            const int j0 = (grp % a.groups_per_row) * 32;
+            for (int r = threadIdx.x >> 5; r < 2 * 4 * 32; r += NW) {
+                const int part = r >> 7;
+                const int gi = (r >> 5) & 3;
+                const int jl = r & 31;
+                if (t >= 0 && j0 + jl < a.d) {
+                    __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                    dst[((size_t)gi * d + j0 + jl) * a.ldT + row0 + t] = sm.u.dpt[part][gi][jl][tl];
+                }
+            }
+        }
+        if (threadIdx.x == 0) sm.tick[0] = after;
+        __syncthreads();
+        cur = nxt;
+        nxt = sm.tick[0];
+        st ^= 1;
     }
+    cp_async_wait_all();
 }
 
 // out[c][r] = in[r][c] for a bf16 matrix of R rows and C columns; row strides
@@ -272,8 +340,37 @@ __global__ void reduce_partials_kernel(const float *__restrict__ partial, float 
         db[(size_t)(e - 4) * d + j] = (float)acc;
 }
 
+int sm_count_bwd()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+    }
+    return n;
+}
+
+template <int FORGET, bool BF16OUT>
+cudaError_t launch_adjoint(const BwdArgs &a, cudaStream_t st)
+{
+    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT>;
+    static int blocks_per_sm = 0;
+    if (blocks_per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(BwdSmem));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, sizeof(BwdSmem));
+        if (e != cudaSuccess) return e;
+        if (blocks_per_sm < 1) blocks_per_sm = 1;
+    }
+    const int grid = min(a.n_tiles, sm_count_bwd() * blocks_per_sm);
+    kern<<<grid, NW * 32, sizeof(BwdSmem), st>>>(a);
+    return cudaGetLastError();
+}
+
 struct Layout {
-    size_t ticket, flags, agg, inc, partial, dP, dpt, xT, wT, wpart, err, total;
+    size_t ticket, flags, incw, agg, partial, dP, dpt, xT, wT, wpart, err, total;
     int groups_per_row, n_groups, n_chunks, n_tiles, splits;
     long long n, ldT, ld4;
 };
@@ -308,8 +405,8 @@ Layout layout(int B, int T, int d_in, int d_h)
     };
     l.ticket = take(256);
     l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles);
+    l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles);
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
-    l.inc = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.partial = take(sizeof(float) * 8 * 32 * (size_t)l.n_tiles);
     // fp32 dP (CUDA-core GEMMs) and the bf16 pair in the (B*T, 4d) layout
     // (tensor-core GEMMs) share one region; the transposed pair follows
@@ -351,30 +448,29 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.partial = reinterpret_cast<float *>(base + l.partial);
     a.ds0 = ds0;
     a.ticket = reinterpret_cast<unsigned *>(base + l.ticket);
-    a.lb.flags = reinterpret_cast<unsigned *>(base + l.flags);
-    a.lb.agg = reinterpret_cast<float *>(base + l.agg);
-    a.lb.inc = reinterpret_cast<float *>(base + l.inc);
-    a.lb.error = a.ticket + 1;
-    a.lb.epoch = 1;
-    a.lb.wait_ns = 2000000000ull;
-    a.lb.n_groups = l.n_groups;
+    a.ca.flags = reinterpret_cast<unsigned *>(base + l.flags);
+    a.ca.agg = reinterpret_cast<float *>(base + l.agg);
+    a.ca.incw = reinterpret_cast<unsigned long long *>(base + l.incw);
+    a.ca.error = a.ticket + 1;
+    a.ca.epoch = 1;
+    a.ca.wait_ns = 2000000000ull;
+    a.ca.n_groups = l.n_groups;
     a.T = T;
     a.d = d_h;
     a.groups_per_row = l.groups_per_row;
+    a.n_tiles = l.n_tiles;
+    a.vec16 = ((d_h & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
+               (reinterpret_cast<uintptr_t>(P) & 15) == 0 && (reinterpret_cast<uintptr_t>(dH) & 15) == 0) ? 1 : 0;
+    // ticket, error word, flags and the epoch tags of the inclusive prefixes
+    // start cleared
     cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
     if (e != cudaSuccess) return e;
     if (forget == SLSTM_FORGET_EXP) {
-        if (tc)
-            adjoint_vjp_kernel<SLSTM_FORGET_EXP, true><<<l.n_tiles, NW * 32, 0, st>>>(a);
-        else
-            adjoint_vjp_kernel<SLSTM_FORGET_EXP, false><<<l.n_tiles, NW * 32, 0, st>>>(a);
+        e = tc ? launch_adjoint<SLSTM_FORGET_EXP, true>(a, st) : launch_adjoint<SLSTM_FORGET_EXP, false>(a, st);
     } else {
-        if (tc)
-            adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID, true><<<l.n_tiles, NW * 32, 0, st>>>(a);
-        else
-            adjoint_vjp_kernel<SLSTM_FORGET_SIGMOID, false><<<l.n_tiles, NW * 32, 0, st>>>(a);
+        e = tc ? launch_adjoint<SLSTM_FORGET_SIGMOID, true>(a, st) : launch_adjoint<SLSTM_FORGET_SIGMOID, false>(a, st);
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
     reduce_partials_kernel<<<(8 * d_h + 255) / 256, 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -168,6 +168,172 @@ SLSTM_DEVINL void warp_carry(float (*s_agg)[20][32], float (*s_cin)[32], int war
     aff_apply(pre, cin, out);
 }
 
+// ---------------------------------------------------------------------------
+// Carry hand-off used by the persistent kernels (Newton iteration, adjoint).
+// A tile's inclusive prefix (4 values per feature) is published as 64-bit
+// words (value bits | epoch << 32): a reader validates and reads it with one
+// load per word and the writer needs no fence.  The epoch tags are cleared
+// at the start of every call, and each launch of the call has its own epoch.
+// A tile whose predecessor has not published yet publishes its aggregate
+// (gated by the per-tile flag word) and looks back past unfinished tiles.
+// ---------------------------------------------------------------------------
+struct CarryArgs {
+    unsigned *flags;              // [n_tiles]
+    float *agg;                   // [n_tiles][20][32]
+    unsigned long long *incw;     // [n_tiles][4][32]
+    unsigned *error;
+    unsigned epoch;
+    unsigned long long wait_ns;
+    int n_groups;
+};
+
+SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+SLSTM_DEVINL void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// This lane's part of tile tq's inclusive prefix, if published in this launch.
+SLSTM_DEVINL bool read_inc_words(const CarryArgs &ca, unsigned tq, int lane, float v[4])
+{
+    const unsigned long long *src = ca.incw + (size_t)tq * 4 * 32 + lane;
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const unsigned long long w = ld_relaxed_u64(src + e * 32);
+        ok = ok && ((unsigned)(w >> 32) == ca.epoch);
+        v[e] = __uint_as_float((unsigned)w);
+    }
+    return ok;
+}
+
+// Warp 0 only.  s_agg[w] holds warp w's own aggregate (in processing order).
+// Writes the carry entering every warp to s_cin[w] and publishes the tile's
+// inclusive prefix.  `first` enters chunk 0; `withhold` suppresses this
+// tile's publications (fault injection).  In the common case (predecessor
+// published) only 4-vectors move: v_{w+1} = A_w v_w + b_w; the 4x4 tile
+// aggregate is formed only when it must be published.
+template <int NW>
+SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32], float (*s_cin)[4][32],
+                                    unsigned ticket, int chunk, int grp, const float first[4], bool withhold)
+{
+    const int lane = threadIdx.x & 31;
+    float carry[4] = {first[0], first[1], first[2], first[3]};
+    if (chunk > 0) {
+        unsigned tq = ticket - (unsigned)ca.n_groups;
+        float v[4];
+        const bool ok = read_inc_words(ca, tq, lane, v);
+        if (__all_sync(0xffffffffu, ok)) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) carry[e] = v[e];
+        } else {
+            Aff tile;
+            load_aff_smem(s_agg, 0, lane, tile);
+            for (int w = 1; w < NW; ++w) {
+                Aff x;
+                load_aff_smem(s_agg, w, lane, x);
+                aff_compose(x, tile, tile);
+            }
+            if (!withhold) {
+                float *dst = ca.agg + (size_t)ticket * 20 * 32;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) st_release(ca.flags + ticket, (ca.epoch << 2) | FLAG_AGG);
+            }
+            Aff M;
+            aff_identity(M);
+            int q = chunk - 1;
+            const uint64_t t0 = globaltimer_ns();
+            unsigned polls = 0;
+            for (;;) {
+                tq = (unsigned)q * (unsigned)ca.n_groups + (unsigned)grp;
+                if (read_inc_words(ca, tq, lane, v)) {
+                    aff_apply(M, v, carry);
+                    break;
+                }
+                const unsigned f = ld_acquire(ca.flags + tq);
+                if ((f >> 2) == ca.epoch && (f & 3u) == FLAG_AGG) {
+                    Aff x;
+                    const float *src = ca.agg + (size_t)tq * 20 * 32;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+                    aff_compose(M, x, M);
+                    --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
+                    continue;
+                }
+                if (++polls > 16) __nanosleep(64);
+                if (globaltimer_ns() - t0 > ca.wait_ns) {
+                    atomicOr(ca.error, 1u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) carry[e] = 0.f;
+                    break;
+                }
+            }
+        }
+    }
+    float v[4] = {carry[0], carry[1], carry[2], carry[3]};
+    for (int w = 0; w < NW; ++w) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_cin[w][e][lane] = v[e];
+        Aff x;
+        load_aff_smem(s_agg, w, lane, x);
+        aff_apply(x, v, v);
+    }
+    if (!withhold) {
+        unsigned long long *dst = ca.incw + (size_t)ticket * 4 * 32 + lane;
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            st_relaxed_u64(dst + e * 32, ((unsigned long long)ca.epoch << 32) | __float_as_uint(v[e]));
+    }
+}
+
+// cp.async copies into shared memory (zero-fill beyond `bytes`).
+SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+SLSTM_DEVINL void cp_async16(void *dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+SLSTM_DEVINL void cp_async4(void *dst, const void *src, int bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
+                 : "memory");
+}
+
+SLSTM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+SLSTM_DEVINL void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+SLSTM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Copy one row of 32 consecutive floats (src, 16-byte aligned when vec16)
+// into shared memory; only `valid` leading floats are read, the rest become
+// zero.  Called by 8 lanes (vec16: 16 bytes each) or 32 lanes (4 bytes each);
+// `part` is the caller's index within that group.
+SLSTM_DEVINL void copy_row32(float *dst, const float *src, int valid, bool vec16, int part)
+{
+    if (vec16) {
+        const int f0 = 4 * part;
+        const int bytes = valid > f0 ? 4 * min(4, valid - f0) : 0;
+        cp_async16(dst + f0, bytes ? src + f0 : src, bytes);
+    } else {
+        const int bytes = valid > part ? 4 : 0;
+        cp_async4(dst + part, bytes ? src + part : src, bytes);
+    }
+}
+
 // Fold one step's map (J, r) into a running aggregate: agg <- (J, r) o agg.
 SLSTM_DEVINL void fold_jac(Aff &agg, const Cell &J, const float r[4])
 {

@@ -76,36 +76,6 @@ struct Smem {
     int exit_flag;
 };
 
-SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-SLSTM_DEVINL void cp_async16(void *dst, const void *src, int bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
-                 : "memory");
-}
-
-SLSTM_DEVINL void cp_async4(void *dst, const void *src, int bytes)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_addr(dst)), "l"(src), "r"(bytes)
-                 : "memory");
-}
-
-SLSTM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-SLSTM_DEVINL void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-SLSTM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
-{
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-SLSTM_DEVINL void st_relaxed_u64(unsigned long long *p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 // Issue the copies of one tile's P (and old S unless `with_s` is false) into
 // shared-memory stage `st`.  Rows past T and features past d read nothing and
 // arrive as zeros.
@@ -151,106 +121,6 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, unsigned ticket
             float *dst = tens ? &sm.S[st][step][slot][jl] : &sm.P[st][step][slot][jl];
             cp_async4(dst, src, bytes);
         }
-    }
-}
-
-// Inclusive prefix of tile tq for this lane, if published in this launch.
-SLSTM_DEVINL bool read_inc(const Args &a, unsigned tq, int lane, float v[4])
-{
-    const unsigned long long *src = a.incw + (size_t)tq * 4 * 32 + lane;
-    bool ok = true;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const unsigned long long w = ld_relaxed_u64(src + e * 32);
-        ok = ok && ((unsigned)(w >> 32) == a.epoch);
-        v[e] = __uint_as_float((unsigned)w);
-    }
-    return ok;
-}
-
-// Warp 0: carries entering every warp of the tile (written to sm.cin) and
-// publication of the tile's inclusive prefix; sm.agg[w] holds warp w's own
-// aggregate.  When the predecessor has published (the common case) only
-// vectors are propagated: v_{w+1} = A_w v_w + b_w.  The tile aggregate (a
-// fold of 4x4 maps) is formed only when it has to be published.
-SLSTM_DEVINL void tile_carry_warp0(const Args &a, Smem &sm, unsigned ticket, int chunk, int grp, bool withhold)
-{
-    const int lane = threadIdx.x & 31;
-    float carry[4] = {0.f, 0.f, 0.f, 0.f};
-    if (chunk > 0) {
-        unsigned tq = ticket - (unsigned)a.n_groups;
-        float v[4];
-        const bool ok = read_inc(a, tq, lane, v);
-        if (__all_sync(0xffffffffu, ok)) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) carry[e] = v[e];
-        } else {
-            // predecessor unfinished: publish the aggregate so that later
-            // tiles can skip over this one, then look back
-            Aff tile;
-            load_aff_smem(sm.agg, 0, lane, tile);
-            for (int w = 1; w < NW; ++w) {
-                Aff x;
-                load_aff_smem(sm.agg, w, lane, x);
-                aff_compose(x, tile, tile);
-            }
-            if (!withhold) {
-                float *dst = a.agg + (size_t)ticket * 20 * 32;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release(a.flags + ticket, (a.epoch << 2) | FLAG_AGG);
-            }
-            Aff M;
-            aff_identity(M);
-            int q = chunk - 1;
-            const uint64_t t0 = globaltimer_ns();
-            unsigned polls = 0;
-            for (;;) {
-                tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
-                if (read_inc(a, tq, lane, v)) {
-                    aff_apply(M, v, carry);
-                    break;
-                }
-                const unsigned f = ld_acquire(a.flags + tq);
-                if ((f >> 2) == a.epoch && (f & 3u) == FLAG_AGG) {
-                    Aff x;
-                    const float *src = a.agg + (size_t)tq * 20 * 32;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
-                    aff_compose(M, x, M);
-                    --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
-                    continue;
-                }
-                if (++polls > 16) __nanosleep(64);
-                if (globaltimer_ns() - t0 > a.wait_ns) {
-                    atomicOr(a.error, 1u);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) carry[e] = 0.f;
-                    break;
-                }
-            }
-        }
-    }
-    // carries of the warps, then the tile's inclusive prefix
-    float v[4] = {carry[0], carry[1], carry[2], carry[3]};
-    for (int w = 0; w < NW; ++w) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sm.cin[w][e][lane] = v[e];
-        Aff x;
-        load_aff_smem(sm.agg, w, lane, x);
-        aff_apply(x, v, v);
-    }
-    if (!withhold) {
-        unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            st_relaxed_u64(dst + e * 32, ((unsigned long long)a.epoch << 32) | __float_as_uint(v[e]));
     }
 }
 
@@ -404,7 +274,12 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         }
         store_aff_smem(sm.agg, warp, lane, agg);
         __syncthreads();
-        if (warp == 0) tile_carry_warp0(a, sm, ticket, chunk, grp, (k == 0) && ((int)ticket == a.fault_ticket));
+        if (warp == 0) {
+            CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+            tile_carry_serial<NW>(ca, sm.agg, sm.cin, ticket, chunk, grp, zero,
+                                  (k == 0) && ((int)ticket == a.fault_ticket));
+        }
         __syncthreads();
 
         // ---- walk B ----
