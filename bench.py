@@ -293,8 +293,9 @@ def run_gpu(args, w):
                "sample": f"{args.cpu_lanes} random (b,j) lanes x T={w.T}: fp64 input-projection rows, {K} fixed "
                          f"Newton iterations, BPTT, dx/dW_x contributions ({dt:.1f} s, single thread)"}
 
-    # kernels launched per step: preact GEMM 1, Newton K, backward: adjoint 1 + reduce 1 + 2 GEMMs
-    launches_per_step = 1 + K + 4
+    # kernels launched per step: preact GEMM 1, Newton K, backward: adjoint 1 +
+    # dR/db reduction 1 + 2 GEMMs (+ the split-K sum of the tensor-core path)
+    launches_per_step = 1 + K + 4 + (1 if w.dtype == "bf16" else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -28,8 +28,8 @@ struct BwdArgs {
     const float *dH;
     float *dP;        // (B, T, 4, d) fp32, when the GEMMs run on CUDA cores
     // bf16 pair dP ~ hi + lo (|dP - hi - lo| <= 2^-18 |dP|) for the tensor-core
-    // GEMMs, in the layout (B*T, 4d) and transposed (4d, ldT)
-    __nv_bfloat16 *dp_hi, *dp_lo, *dpt_hi, *dpt_lo;
+    // GEMMs, stored transposed: (4d, ldT) with ldT = B*T rounded up to 8
+    __nv_bfloat16 *dpt_hi, *dpt_lo;
     long long ldT;
     float *partial;   // [n_tiles][8][32]  dR (4) then db (4)
     float *ds0;       // (B, 4, d) or null
@@ -210,15 +210,10 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
                 const float dq = g.gho * lam[3];
                 if (BF16OUT) {
                     const float dv[4] = {dz, di, df, dq};
-                    const size_t o = (row0 + t) * 4 * d + jj;
 #pragma unroll
                     for (int gi = 0; gi < 4; ++gi) {
                         __nv_bfloat16 hi, lo;
                         split_bf16(dv[gi], hi, lo);
-                        if (jv) {
-                            a.dp_hi[o + gi * d] = hi;
-                            a.dp_lo[o + gi * d] = lo;
-                        }
                         sm.u.dpt[0][gi][lane][rl] = hi;
                         sm.u.dpt[1][gi][lane][rl] = lo;
                     }
@@ -287,25 +282,6 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
     cp_async_wait_all();
 }
 
-// out[c][r] = in[r][c] for a bf16 matrix of R rows and C columns; row strides
-// ldi (in) and ldo (out) in elements.
-__global__ void transpose_bf16_kernel(const __nv_bfloat16 *__restrict__ in, __nv_bfloat16 *__restrict__ out,
-                                      int R, int C, long long ldi, long long ldo)
-{
-    __shared__ __nv_bfloat16 tile[32][34];
-    const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-    for (int k = ty; k < 32; k += 8) {
-        const int r = r0 + k, c = c0 + tx;
-        if (r < R && c < C) tile[k][tx] = in[(size_t)r * ldi + c];
-    }
-    __syncthreads();
-    for (int k = ty; k < 32; k += 8) {
-        const int c = c0 + k, r = r0 + tx;
-        if (r < R && c < C) out[(size_t)c * ldo + r] = tile[tx][k];
-    }
-}
-
 // out[i] = sum_z part[z][i], z in order (split-K partial sums).
 __global__ void sum_splits_kernel(const float *__restrict__ part, float *__restrict__ out, long long n, int splits)
 {
@@ -318,26 +294,38 @@ __global__ void sum_splits_kernel(const float *__restrict__ part, float *__restr
 
 // dR[g][j] and db[g][j]: sum of the per-tile partials over chunks and batch
 // rows, in a fixed order, accumulated in fp64.
-__global__ void reduce_partials_kernel(const float *__restrict__ partial, float *__restrict__ dR,
-                                       float *__restrict__ db, int B, int n_chunks, int groups_per_row,
-                                       int d)
+// One block per (entry e, group of 32 features); warp w sums the (chunk, b)
+// terms w, w+8, ... for its lane, then the 8 warp sums are added in order.
+__global__ void __launch_bounds__(256) reduce_partials_kernel(const float *__restrict__ partial, float *__restrict__ dR,
+                                                              float *__restrict__ db, int B, int n_chunks,
+                                                              int groups_per_row, int d)
 {
-    const int idx = blockIdx.x * blockDim.x + threadIdx.x;  // over 8 * d
-    if (idx >= 8 * d) return;
-    const int e = idx / d;
-    const int j = idx % d;
-    const int jb = j / 32, lane = j % 32;
+    __shared__ double s_sum[8][32];
+    const int e = blockIdx.y;              // 0..7
+    const int jb = blockIdx.x;             // feature group
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int G = B * groups_per_row;
+    const int terms = n_chunks * B;
     double acc = 0.0;
-    for (int c = 0; c < n_chunks; ++c)
-        for (int b = 0; b < B; ++b) {
-            const size_t ticket = (size_t)c * G + (size_t)b * groups_per_row + jb;
-            acc += partial[(ticket * 8 + e) * 32 + lane];
+    for (int q = warp; q < terms; q += 8) {
+        const int c = q / B, b = q % B;
+        const size_t ticket = (size_t)c * G + (size_t)b * groups_per_row + jb;
+        acc += partial[(ticket * 8 + e) * 32 + lane];
+    }
+    s_sum[warp][lane] = acc;
+    __syncthreads();
+    if (warp == 0) {
+        double t = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += s_sum[w][lane];
+        const int j = jb * 32 + lane;
+        if (j < d) {
+            if (e < 4)
+                dR[(size_t)e * d + j] = (float)t;
+            else
+                db[(size_t)(e - 4) * d + j] = (float)t;
         }
-    if (e < 4)
-        dR[(size_t)e * d + j] = (float)acc;
-    else
-        db[(size_t)(e - 4) * d + j] = (float)acc;
+    }
 }
 
 int sm_count_bwd()
@@ -370,7 +358,7 @@ cudaError_t launch_adjoint(const BwdArgs &a, cudaStream_t st)
 }
 
 struct Layout {
-    size_t ticket, flags, incw, agg, partial, dP, dpt, xT, wT, wpart, err, total;
+    size_t ticket, flags, incw, agg, partial, dP, dpt, wpart, err, total;
     int groups_per_row, n_groups, n_chunks, n_tiles, splits;
     long long n, ldT, ld4;
 };
@@ -408,12 +396,10 @@ Layout layout(int B, int T, int d_in, int d_h)
     l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles);
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
     l.partial = take(sizeof(float) * 8 * 32 * (size_t)l.n_tiles);
-    // fp32 dP (CUDA-core GEMMs) and the bf16 pair in the (B*T, 4d) layout
-    // (tensor-core GEMMs) share one region; the transposed pair follows
+    // fp32 dP for the CUDA-core GEMMs; the transposed bf16 pair for the
+    // tensor-core GEMMs
     l.dP = take(sizeof(float) * (size_t)l.n);
     l.dpt = take(2 * sizeof(__nv_bfloat16) * (size_t)(4LL * d_h) * (size_t)l.ldT);
-    l.xT = take(sizeof(__nv_bfloat16) * (size_t)d_in * (size_t)l.ldT);
-    l.wT = take(sizeof(__nv_bfloat16) * (size_t)d_in * (size_t)l.ld4);
     l.wpart = take(sizeof(float) * (size_t)l.splits * 4 * d_h * d_in);
     l.err = take(256);
     l.total = off;
@@ -432,7 +418,7 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     const Layout l = layout(B, T, d_in, d_h);
     char *base = static_cast<char *>(ws);
     // tensor-core GEMMs need 16-byte TMA strides: (4 d_h) bf16 rows and d_in % 8
-    const bool tc = (dtype == SLSTM_BF16) && (d_h % 2 == 0) && (d_in % 8 == 0);
+    const bool tc = (dtype == SLSTM_BF16) && (d_in % 8 == 0);
     BwdArgs a;
     a.P = P;
     a.R = R;
@@ -440,8 +426,6 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.S = S;
     a.dH = dH;
     a.dP = reinterpret_cast<float *>(base + l.dP);
-    a.dp_hi = reinterpret_cast<__nv_bfloat16 *>(base + l.dP);
-    a.dp_lo = a.dp_hi + l.n;
     a.dpt_hi = reinterpret_cast<__nv_bfloat16 *>(base + l.dpt);
     a.dpt_lo = a.dpt_hi + 4LL * d_h * l.ldT;
     a.ldT = l.ldT;
@@ -471,7 +455,7 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
         e = tc ? launch_adjoint<SLSTM_FORGET_SIGMOID, true>(a, st) : launch_adjoint<SLSTM_FORGET_SIGMOID, false>(a, st);
     }
     if (e != cudaSuccess) return e;
-    reduce_partials_kernel<<<(8 * d_h + 255) / 256, 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
+    reduce_partials_kernel<<<dim3(l.groups_per_row, 8), 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -479,23 +463,17 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     const int BT = B * T;
     if (tc) {
         unsigned *err = reinterpret_cast<unsigned *>(base + l.err);
-        __nv_bfloat16 *xT = reinterpret_cast<__nv_bfloat16 *>(base + l.xT);
-        __nv_bfloat16 *wT = reinterpret_cast<__nv_bfloat16 *>(base + l.wT);
         float *wpart = reinterpret_cast<float *>(base + l.wpart);
         if ((e = cudaMemsetAsync(err, 0, sizeof(unsigned), st)) != cudaSuccess) return e;
-        // W_x^T (d_in, 4 d_h) and x^T (d_in, B*T) as K-major operands
-        transpose_bf16_kernel<<<dim3((d_in + 31) / 32, (unsigned)((N4 + 31) / 32)), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(Wx), wT, (int)N4, d_in, d_in, l.ld4);
-        transpose_bf16_kernel<<<dim3((d_in + 31) / 32, (unsigned)((BT + 31) / 32)), 256, 0, st>>>(
-            static_cast<const __nv_bfloat16 *>(x), xT, BT, d_in, d_in, l.ldT);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        // dx = (dP_hi + dP_lo) W_x
-        if ((e = gemm_tc_bf16_ex(a.dp_hi, a.dp_lo, (int)N4, wT, (int)l.ld4, nullptr, dx, BT, d_in, (int)N4, 1, err,
-                                 st)) != cudaSuccess)
+        // dx = (dP_hi + dP_lo) W_x: the pair is stored (4 d_h, B*T), i.e. an
+        // MN-major A operand; W_x (4 d_h, d_in) is an MN-major B operand
+        if ((e = gemm_tc_bf16_ex(a.dpt_hi, a.dpt_lo, (int)l.ldT, true, Wx, d_in, true, nullptr, dx, BT, d_in,
+                                 (int)N4, 1, err, st)) != cudaSuccess)
             return e;
-        // dW_x = (dP_hi + dP_lo)^T x, split over B*T, partial sums added in order
-        if ((e = gemm_tc_bf16_ex(a.dpt_hi, a.dpt_lo, (int)l.ldT, xT, (int)l.ldT, nullptr, wpart, (int)N4, d_in, BT,
-                                 l.splits, err, st)) != cudaSuccess)
+        // dW_x = (dP_hi + dP_lo)^T x: K-major A, x (B*T, d_in) an MN-major B
+        // operand; split over B*T, partial sums added in order
+        if ((e = gemm_tc_bf16_ex(a.dpt_hi, a.dpt_lo, (int)l.ldT, false, x, d_in, true, nullptr, wpart, (int)N4, d_in,
+                                 BT, l.splits, err, st)) != cudaSuccess)
             return e;
         const long long nw = N4 * d_in;
         sum_splits_kernel<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(wpart, dWx, nw, l.splits);

@@ -103,11 +103,27 @@ SLSTM_DEVINL uint64_t smem_desc_k_sw128(uint32_t saddr)
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, M x N.
-constexpr uint32_t idesc_bf16(int M, int N)
+// Shared-memory matrix descriptor of an MN-major bf16 tile written by TMA as
+// 64-element-wide boxes with 128-byte swizzle: each box is BK K-rows of 128
+// bytes (one 64-element MN atom), boxes `atom_stride` bytes apart; 8-row K
+// groups are 1024 bytes apart.
+SLSTM_DEVINL uint64_t smem_desc_mn_sw128(uint32_t saddr, uint32_t atom_stride)
 {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);        // start address
+    d |= (uint64_t)((atom_stride >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN atom
+    d |= (uint64_t)(1024u >> 4) << 32;                // stride byte offset: next 8-row K group
+    d |= (uint64_t)1u << 46;                          // descriptor version for sm_100
+    d |= (uint64_t)2u << 61;                          // 128-byte swizzle
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, M x N;
+// a_mn / b_mn select MN-major (transposed) operands.
+constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 SLSTM_DEVINL void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
@@ -149,6 +165,9 @@ SLSTM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// A_MN / B_MN: the operand is stored MN-major ([K][M] or [K][N], MN
+// contiguous) instead of K-major; its tile is then loaded as 64-wide boxes.
+template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(128, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tma2,
                    const __grid_constant__ CUtensorMap tmb, TcArgs g)
@@ -210,13 +229,26 @@ __global__ void __launch_bounds__(128, 1)
             const int part = vk / nk_part;
             const int kk = vk - part * nk_part;
             mbar_expect_tx(&full[s], STAGE_BYTES);
-            tma_load_2d(sA + s * A_STAGE, part ? &tma2 : &tma, &full[s], kk * BK, m0);
-            tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kk * BK, n0);
+            const CUtensorMap *am = part ? &tma2 : &tma;
+            if (A_MN) {
+#pragma unroll
+                for (int i = 0; i < BM / 64; ++i)
+                    tma_load_2d(sA + s * A_STAGE + i * (BK * 128), am, &full[s], m0 + 64 * i, kk * BK);
+            } else {
+                tma_load_2d(sA + s * A_STAGE, am, &full[s], kk * BK, m0);
+            }
+            if (B_MN) {
+#pragma unroll
+                for (int i = 0; i < BN / 64; ++i)
+                    tma_load_2d(sB + s * B_STAGE + i * (BK * 128), &tmb, &full[s], n0 + 64 * i, kk * BK);
+            } else {
+                tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kk * BK, n0);
+            }
         }
         s_issued = kb;
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer ----
-        constexpr uint32_t idesc = idesc_bf16(BM, BN);
+        constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
         int kb = 0;
         for (; kb < nkb; ++kb) {
             const int s = kb % STAGES;
@@ -226,11 +258,17 @@ __global__ void __launch_bounds__(128, 1)
                 break;
             }
             tc_fence_after();
-            const uint64_t ad = smem_desc_k_sw128(smem_u32(sA + s * A_STAGE));
-            const uint64_t bd = smem_desc_k_sw128(smem_u32(sB + s * B_STAGE));
+            // per MMA step of K = 16: K-major tiles advance 32 bytes along the
+            // swizzled row, MN-major tiles advance 16 K-rows (2048 bytes)
+            const uint64_t ad = A_MN ? smem_desc_mn_sw128(smem_u32(sA + s * A_STAGE), BK * 128)
+                                     : smem_desc_k_sw128(smem_u32(sA + s * A_STAGE));
+            const uint64_t bd = B_MN ? smem_desc_mn_sw128(smem_u32(sB + s * B_STAGE), BK * 128)
+                                     : smem_desc_k_sw128(smem_u32(sB + s * B_STAGE));
+            constexpr uint64_t a_step = A_MN ? (2048u >> 4) : (32u >> 4);
+            constexpr uint64_t b_step = B_MN ? (2048u >> 4) : (32u >> 4);
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k)   // 16 bf16 = 32 bytes per MMA step
-                umma_bf16(tmem, ad + 2u * k, bd + 2u * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k)
+                umma_bf16(tmem, ad + a_step * k, bd + b_step * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
             umma_commit(&empty[s]);
         }
         s_consumed = kb;
@@ -301,15 +339,17 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// 2-D K-major bf16 tensor [rows][K] (row stride ld elements) with a
-// (64 x box_rows) box, 128-byte swizzle.
-bool make_map(CUtensorMap *map, const void *base, int rows, int K, int ld, int box_rows)
+// 2-D bf16 tensor of `rows` rows of `cols` contiguous elements (row stride
+// ld elements), box of 64 contiguous elements x box_rows rows, 128-byte
+// swizzle.  K-major operands: cols = K, rows = M or N.  MN-major operands:
+// cols = M or N, rows = K.
+bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int ld, int box_rows)
 {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-    cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -317,25 +357,38 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int K, int ld, int b
     return r == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-// C = (A0 [+ A1]) B^T (+ bias) with optional split-K into `splits` fp32
-// slices C + z * M * N (the caller sums them); A0, A1: [M][K] bf16 with row
-// stride lda elements, B: [N][K] bf16 with row stride ldb; K-major.
-cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, const void *Bm, int ldb, const float *bias,
-                            float *C, int M, int N, int K, int splits, unsigned *error, cudaStream_t st)
+template <bool A_MN, bool B_MN>
+cudaError_t launch_tc(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const TcArgs &g,
+                      dim3 grid, cudaStream_t st)
 {
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   SMEM_BYTES);
+        const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    gemm_tc_kernel<A_MN, B_MN><<<grid, 128, SMEM_BYTES, st>>>(ta, ta2, tb, g);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// C = (A0 [+ A1]) B^T (+ bias) with optional split-K into `splits` fp32
+// slices C + z * M * N (the caller sums them).  A0, A1: [M][K] (a_mn = 0) or
+// [K][M] (a_mn = 1) bf16 with row stride lda; B: [N][K] (b_mn = 0) or [K][N]
+// (b_mn = 1) with row stride ldb.
+cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, const void *Bm, int ldb, bool b_mn,
+                            const float *bias, float *C, int M, int N, int K, int splits, unsigned *error,
+                            cudaStream_t st)
+{
     CUtensorMap ta, ta2, tb;
-    if (!make_map(&ta, A0, M, K, lda, BM) || !make_map(&tb, Bm, N, K, ldb, BN)) return cudaErrorInvalidValue;
+    const bool ok_a = a_mn ? make_map(&ta, A0, K, M, lda, BK) : make_map(&ta, A0, M, K, lda, BM);
+    const bool ok_b = b_mn ? make_map(&tb, Bm, K, N, ldb, BK) : make_map(&tb, Bm, N, K, ldb, BN);
+    if (!ok_a || !ok_b) return cudaErrorInvalidValue;
     if (A1 != nullptr) {
-        if (!make_map(&ta2, A1, M, K, lda, BM)) return cudaErrorInvalidValue;
+        const bool ok = a_mn ? make_map(&ta2, A1, K, M, lda, BK) : make_map(&ta2, A1, M, K, lda, BM);
+        if (!ok) return cudaErrorInvalidValue;
     } else {
         ta2 = ta;
     }
@@ -354,12 +407,14 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, const void 
     g.c_split = (long long)M * N;
     g.error = error;
     const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, splits);
-    gemm_tc_kernel<<<grid, 128, SMEM_BYTES, st>>>(ta, ta2, tb, g);
-    return cudaGetLastError();
+    if (a_mn) return b_mn ? launch_tc<true, true>(ta, ta2, tb, g, grid, st) : launch_tc<true, false>(ta, ta2, tb, g, grid, st);
+    return b_mn ? launch_tc<false, true>(ta, ta2, tb, g, grid, st) : launch_tc<false, false>(ta, ta2, tb, g, grid, st);
 }
 
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want)
 {
+    (void)M;
+    (void)N;
     const int total = a_parts * ((K + BK - 1) / BK);
     if (want < 1) want = 1;
     if (want > total) want = total;
@@ -370,7 +425,7 @@ int gemm_tc_splits(int M, int N, int K, int a_parts, int want)
 cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
                          unsigned *error, cudaStream_t st)
 {
-    return gemm_tc_bf16_ex(A, nullptr, K, Bm, K, bias, C, M, N, K, 1, error, st);
+    return gemm_tc_bf16_ex(A, nullptr, K, false, Bm, K, false, bias, C, M, N, K, 1, error, st);
 }
 
 }  // namespace slstm

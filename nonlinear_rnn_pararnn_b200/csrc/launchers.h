@@ -65,11 +65,13 @@ cudaError_t gemm_simt(const GemmDesc &g, cudaStream_t st);
 // nonzero if a bounded wait inside the kernel expires.
 cudaError_t gemm_tc_bf16(const void *A, const void *Bm, const float *bias, float *C, int M, int N, int K,
                          unsigned *error, cudaStream_t st);
-// General form: C = (A0 [+ A1]) B^T (+ bias), A0/A1 [M][K] with row stride
-// lda, B [N][K] with row stride ldb (elements, multiples of 8), split-K into
-// `splits` fp32 slices of C (C + z*M*N) when splits > 1.
-cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, const void *Bm, int ldb, const float *bias,
-                            float *C, int M, int N, int K, int splits, unsigned *error, cudaStream_t st);
+// General form: C = (A0 [+ A1]) B^T (+ bias).  A0, A1: [M][K] (a_mn false)
+// or [K][M] (a_mn true) with row stride lda; B: [N][K] (b_mn false) or
+// [K][N] (b_mn true) with row stride ldb (elements, multiples of 8); split-K
+// into `splits` fp32 slices of C (C + z*M*N) when splits > 1.
+cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, const void *Bm, int ldb, bool b_mn,
+                            const float *bias, float *C, int M, int N, int K, int splits, unsigned *error,
+                            cudaStream_t st);
 // The split count gemm_tc_bf16_ex will actually use for a request of `want`.
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want);
 
