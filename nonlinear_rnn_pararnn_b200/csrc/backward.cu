@@ -73,33 +73,46 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, unsigned t
     const int t_lo = a.T - (chunk + 1) * TT;
     const size_t d = (size_t)a.d;
     const size_t row0 = (size_t)b * a.T;
-    const int valid = min(32, a.d - j0);
-    const int per = a.vec16 ? 8 : 32;         // copies per 32-float row
-    const int rows4 = (TT + 1) * 4;            // (row, slot) pairs of S and of P
-    const int total = (2 * rows4 + TT) * per;
-    for (int idx = threadIdx.x; idx < total; idx += NW * 32) {
-        const int row = idx / per, part = idx % per;
-        float *dst;
-        const float *src;
-        int t;
-        if (row < rows4) {                     // S
-            const int r = row >> 2, slot = row & 3;
-            t = t_lo - 1 + r;
-            dst = &sm.S[st][r][slot][0];
-            src = a.S + ((row0 + (size_t)min(max(t, 0), a.T - 1)) * 4 + slot) * d + j0;
-        } else if (row < 2 * rows4) {          // P
-            const int r = (row - rows4) >> 2, slot = (row - rows4) & 3;
-            t = t_lo + r;
-            dst = &sm.P[st][r][slot][0];
-            src = a.P + ((row0 + (size_t)min(max(t, 0), a.T - 1)) * 4 + slot) * d + j0;
-        } else {                               // dH
-            const int r = row - 2 * rows4;
-            t = t_lo + r;
-            dst = &sm.dH[st][r][0];
-            src = a.dH + (row0 + (size_t)min(max(t, 0), a.T - 1)) * d + j0;
+    const int T = a.T;
+    constexpr int RS = (TT + 1) * 4;           // (row, slot) pairs of S and of P
+    if (a.vec16) {
+        // thread (q, c) copies 16-byte chunk c of (row, slot) pairs q, q+32, ...
+        const int c = threadIdx.x & 7, q = threadIdx.x >> 3;
+        const int jj = j0 + 4 * c;
+        const int fbytes = jj < a.d ? 4 * min(4, a.d - jj) : 0;
+#pragma unroll
+        for (int k = 0; k < (RS + 31) / 32; ++k) {
+            const int rs = q + 32 * k;
+            if (rs < RS) {
+                const int r = rs >> 2, slot = rs & 3;
+                const int tS = t_lo - 1 + r, tP = t_lo + r;   // S row r <-> t_lo-1+r, P row r <-> t_lo+r
+                const int bS = (tS >= 0 && tS < T) ? fbytes : 0;
+                const int bP = (tP >= 0 && tP < T) ? fbytes : 0;
+                cp_async16(&sm.S[st][r][slot][4 * c], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
+                cp_async16(&sm.P[st][r][slot][4 * c], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+            }
         }
-        const bool in = (t >= 0 && t < a.T);
-        copy_row32(dst, src, in ? valid : 0, a.vec16 != 0, part);
+        const int t = t_lo + q;   // dH row q
+        const int bH = (t >= 0 && t < T) ? fbytes : 0;
+        cp_async16(&sm.dH[st][q][4 * c], bH ? a.dH + (row0 + t) * d + jj : a.dH, bH);
+    } else {
+        // 4-byte copies, lane = feature, warp w takes every 8th row
+        const int jl = threadIdx.x & 31, w = threadIdx.x >> 5;
+        const bool fj = j0 + jl < a.d;
+        const size_t jj = (size_t)j0 + jl;
+        for (int rs = w; rs < RS; rs += NW) {
+            const int r = rs >> 2, slot = rs & 3;
+            const int tS = t_lo - 1 + r, tP = t_lo + r;
+            const int bS = (fj && tS >= 0 && tS < T) ? 4 : 0;
+            const int bP = (fj && tP >= 0 && tP < T) ? 4 : 0;
+            cp_async4(&sm.S[st][r][slot][jl], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
+            cp_async4(&sm.P[st][r][slot][jl], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+        }
+        for (int r = w; r < TT; r += NW) {
+            const int t = t_lo + r;
+            const int bH = (fj && t >= 0 && t < T) ? 4 : 0;
+            cp_async4(&sm.dH[st][r][jl], bH ? a.dH + (row0 + t) * d + jj : a.dH, bH);
+        }
     }
 }
 

@@ -88,38 +88,37 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, unsigned ticket
     const int j0 = (grp % a.groups_per_row) * 32;
     const int t0 = chunk * TT;
     const size_t d = (size_t)a.d;
-    const int ntens = with_s ? 2 : 1;
+    const int w = threadIdx.x >> 5;
     if (a.vec16) {
-        // 8 chunks of 16 bytes per (step, slot) row of 32 features
-        for (int idx = threadIdx.x; idx < ntens * TT * 4 * 8; idx += NW * 32) {
-            const int tens = idx / (TT * 4 * 8);
-            const int rem = idx % (TT * 4 * 8);
-            const int c = rem & 7;
-            const int rs = rem >> 3;
-            const int step = rs >> 2, slot = rs & 3;
-            const int t = t0 + step;
-            const int jj = j0 + 4 * c;
-            int bytes = 0;
-            if (t < a.T && jj < a.d) bytes = min(16, 4 * (a.d - jj));
-            const float *base = tens ? a.S : a.P;
-            const float *src = bytes ? base + (((size_t)b * a.T + t) * 4 + slot) * d + jj : base;
-            float *dst = tens ? &sm.S[st][step][slot][4 * c] : &sm.P[st][step][slot][4 * c];
-            cp_async16(dst, src, bytes);
+        // 8 chunks of 16 bytes per (step, slot) row of 32 features; thread
+        // (w, slot, c) copies chunk c of slot `slot` for steps w, w+8, w+16, w+24
+        const int c = threadIdx.x & 7, slot = (threadIdx.x >> 3) & 3;
+        const int jj = j0 + 4 * c;
+        const int fbytes = jj < a.d ? 4 * min(4, a.d - jj) : 0;
+        const size_t off0 = (((size_t)b * a.T + t0 + w) * 4 + slot) * d + jj;
+        const size_t step8 = 32 * d;   // 8 steps of 4 slots
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int step = r * 8 + w;
+            const int bytes = (t0 + step < a.T) ? fbytes : 0;
+            const size_t off = off0 + r * step8;
+            cp_async16(&sm.P[st][step][slot][4 * c], bytes ? a.P + off : a.P, bytes);
+            if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? a.S + off : a.S, bytes);
         }
     } else {
-        for (int idx = threadIdx.x; idx < ntens * TT * 4 * 32; idx += NW * 32) {
-            const int tens = idx / (TT * 4 * 32);
-            const int rem = idx % (TT * 4 * 32);
-            const int jl = rem & 31;
-            const int rs = rem >> 5;
+        // 4-byte copies, lane = feature; warp w copies rows w, w+8, ... of
+        // the 128 (step, slot) rows
+        const int jl = threadIdx.x & 31;
+        const bool fj = j0 + jl < a.d;
+        const size_t base0 = ((size_t)b * a.T + t0) * 4 * d + j0 + jl;
+#pragma unroll 4
+        for (int r = 0; r < 16; ++r) {
+            const int rs = r * 8 + w;
             const int step = rs >> 2, slot = rs & 3;
-            const int t = t0 + step;
-            const int jj = j0 + jl;
-            const int bytes = (t < a.T && jj < a.d) ? 4 : 0;
-            const float *base = tens ? a.S : a.P;
-            const float *src = bytes ? base + (((size_t)b * a.T + t) * 4 + slot) * d + jj : base;
-            float *dst = tens ? &sm.S[st][step][slot][jl] : &sm.P[st][step][slot][jl];
-            cp_async4(dst, src, bytes);
+            const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+            const size_t off = base0 + (size_t)rs * d;
+            cp_async4(&sm.P[st][step][slot][jl], bytes ? a.P + off : a.P, bytes);
+            if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? a.S + off : a.S, bytes);
         }
     }
 }
@@ -289,6 +288,8 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         float snp[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
+        // row pointer of this lane's first step; lanes past d write nothing
+        float *srow = a.S + (row0 + t_seg) * 4 * d + jj;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int t = t_seg + i;
@@ -303,24 +304,22 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
                     dl[e] += f4[e] - so;   // delta_t = J_t delta_{t-1} + (f_t - S_t)
                     sn[e] = so + dl[e];
                 }
-                if (jv) {
-                    float *sq = a.S + (row0 + t) * 4 * d + jj;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sq[e * d] = sn[e];
-                    if (RESID) {
-                        Cell f;
-                        cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
-                                                 sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane],
-                                                 rz, ri, rf, ro, f);
-                        const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+                for (int e = 0; e < 4; ++e)
+                    if (jv) srow[(size_t)i * 4 * d + e * d] = sn[e];
+                if (RESID) {
+                    Cell f;
+                    cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
+                                             sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz,
+                                             ri, rf, ro, f);
+                    const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float af = fabsf(F[e]);
-                            const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
-                            // keep NaN: a NaN compares false, so test "not <="
-                            mx_raw = (af <= mx_raw) ? mx_raw : af;
-                            mx_sc = (sc <= mx_sc) ? mx_sc : sc;
-                        }
+                    for (int e = 0; e < 4; ++e) {
+                        const float af = jv ? fabsf(F[e]) : 0.0f;
+                        const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
+                        // keep NaN: a NaN compares false, so test "not <="
+                        mx_raw = (af <= mx_raw) ? mx_raw : af;
+                        mx_sc = (sc <= mx_sc) ? mx_sc : sc;
                     }
                 }
 #pragma unroll
