@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 from nonlinear_rnn_pararnn_b200.workloads import ORDER, WORKLOADS, as_f64, make_inputs  # noqa: E402
 
 METRIC = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd+bwd)"
+METRIC_FWD = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd)"
 UNIT = "elems/s"
 DEFAULT_WORKLOAD = "slstm_bf16_train_b8_t8192_d1024"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -184,13 +185,15 @@ def run_gpu(args, w):
     api._lib.load()
 
     K = args.newton_iters
+    forward_only = args.mode == "forward"
     inp = make_inputs(w)
     x, Wx, R, bias, s0, dH = (inp[k].to(dev) for k in ("x", "Wx", "R", "bias", "s0", "dH"))
     P = torch.empty(w.B, w.T, 4, w.d_h, device=dev)
     S = torch.empty_like(P)
     stats = api.new_stats(dev)
     ws_n = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
-    ws_b = api.workspace(_lib.SLSTM_OP_NEWTON_BACKWARD, w.B, w.T, w.d_in, w.d_h, dev)
+    ws_b = None if args.mode == "forward" else api.workspace(_lib.SLSTM_OP_NEWTON_BACKWARD, w.B, w.T, w.d_in,
+                                                               w.d_h, dev)
     grads = {"dx": torch.empty(w.B, w.T, w.d_in, device=dev), "dWx": torch.empty(4 * w.d_h, w.d_in, device=dev),
              "dR": torch.empty(4, w.d_h, device=dev), "db": torch.empty(4, w.d_h, device=dev),
              "ds0": torch.empty(w.B, 4, w.d_h, device=dev)}
@@ -204,7 +207,8 @@ def run_gpu(args, w):
         api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, fixed=True, tol=w.tol, S=S, stats=stats, ws=ws_n)
         if ev is not None:
             ev[2].record()
-        api.newton_backward(x, Wx, P, R, s0, S, dH, forget=w.forget, out=grads, ws=ws_b)
+        if not forward_only:
+            api.newton_backward(x, Wx, P, R, s0, S, dH, forget=w.forget, out=grads, ws=ws_b)
         if ev is not None:
             ev[3].record()
 
@@ -295,9 +299,10 @@ def run_gpu(args, w):
 
     # kernels launched per step: preact GEMM 1, Newton K, backward: adjoint 1 +
     # dR/db reduction 1 + 2 GEMMs (+ the split-K sum of the tensor-core path)
-    launches_per_step = 1 + K + 4 + (1 if w.dtype == "bf16" else 0)
+    launches_per_step = 1 + K + (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0))
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "metric": METRIC_FWD if forward_only else METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "operand_dtype": "bf16 x/W_x, fp32 state and scans" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
@@ -323,6 +328,54 @@ def run_gpu(args, w):
     return 0
 
 
+def run_scan(args):
+    """scan_block4 alone: B=4, d=2048, T swept; 96 algorithmic bytes per
+    element (read A 64, b 16, write y 16).  Inputs drawn on the device from a
+    seeded generator (values only set the timing's data, not checked here)."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+    ws_n, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    hbm, peak_kind = _peaks()
+    B, d = 4, 2048
+    sweep = []
+    for T in [int(v) for v in args.scan_T.split(",")]:
+        g = torch.Generator(device=dev)
+        g.manual_seed(T)
+        A = torch.rand(B, T, 4, 4, d, generator=g, device=dev) * 0.6 - 0.3
+        b = torch.randn(B, T, 4, d, generator=g, device=dev)
+        y = torch.empty_like(b)
+        ws = api.workspace(_lib.SLSTM_OP_SCAN_BLOCK4, B, T, 0, d, dev)
+        for _ in range(args.warmup):
+            api.scan_block4(A, b, None, y=y, ws=ws)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            api.scan_block4(A, b, None, y=y, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        elems = B * T * d
+        gbs = elems * 96 / (ms / 1e3) / 1e9
+        sweep.append({"T": T, "ms": ms, "elems_per_s": elems / (ms / 1e3), "achieved_GBs": gbs,
+                      "frac": gbs / hbm})
+        del A, b, y, ws
+        torch.cuda.empty_cache()
+    last = sweep[-1]
+    line = {"metric": "scan_block4 elems/s (B*T*d/s)", "value": last["elems_per_s"], "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": last["ms"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"scan_block4_b{B}_d{d}", "B": B, "T": last["T"], "d": d,
+                       "l2": "inputs larger than L2"},
+            "roofline": {"kernel": "scan_kernel", "bound": "hbm", "achieved": last["achieved_GBs"], "peak": hbm,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": last["frac"], "traffic": None},
+            "sweep": sweep}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,6 +387,10 @@ def main(argv=None):
     ap.add_argument("--cpu-lanes", type=int, default=40)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan"],
+                    help="train: GEMM + Newton + backward (default); forward: GEMM + Newton; "
+                         "scan: scan_block4 alone over T in --scan-T at B=4, d=2048")
+    ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
     args = ap.parse_args(argv)
@@ -345,6 +402,8 @@ def main(argv=None):
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "scan":
+        return run_scan(args)
     return run_gpu(args, w)
 
 

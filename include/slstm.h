@@ -215,8 +215,8 @@ int scan_block4(const float *A, const float *b, const float *y0, float *y, int B
  *     Each call clears the counters and flags it relies on before use.
  *   - Returns SLSTM_ERR_UNSUPPORTED when the problem needs more scratch than
  *     the block holds, that is when slstm_workspace_size(SLSTM_OP_SCAN_BLOCK4,
- *     B, T, 0, d) > SLSTM_NOALLOC_SCRATCH_BYTES (up to 2727 tiles of 32 steps
- *     x 32 features: B * ceil(T/32) * ceil(d/32) <= 2727); other errors as
+ *     B, T, 0, d) > SLSTM_NOALLOC_SCRATCH_BYTES (up to 2337 tiles of 32 steps
+ *     x 32 features: B * ceil(T/32) * ceil(d/32) <= 2337); other errors as
  *     scan_block4.
  */
 #define SLSTM_NOALLOC_SCRATCH_BYTES (8u << 20)

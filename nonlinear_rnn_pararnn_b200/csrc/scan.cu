@@ -5,9 +5,15 @@
 // monoid).
 //   forward:  y_t = A_t y_{t-1} + b_t,   y_{-1} = y0
 //   reverse:  y_t = A_t^T y_{t+1} + b_t, y_T   = y0
-// Blocked: each thread folds L steps of one feature serially, warps of a
-// tile are combined in shared memory, tiles are chained by a decoupled
-// look-back (lookback.cuh).  Composition in fp32.
+// A tile is 32 features x 32 steps (in processing order), one CTA of 8 warps,
+// 4 steps per thread.  Persistent CTAs stage the next tile's A and b (80
+// bytes per element) in shared memory with cp.async while they scan the
+// current one:
+//   walk A   each thread folds its 4 maps (dense 4x4 compositions, fp32);
+//   carry    warp 0 takes the carry entering the tile from the tile before
+//            it (decoupled look-back, lookback.cuh) and hands each warp its
+//            carry;
+//   walk B   each thread applies its maps from its carry and writes y.
 #include "launchers.h"
 #include "lookback.cuh"
 
@@ -24,97 +30,178 @@ struct ScanArgs {
     const float *y0;
     float *y;
     unsigned *ticket;
-    LookbackArgs lb;
-    int T, d, groups_per_row;
+    CarryArgs ca;
+    int T, d, groups_per_row, n_tiles, vec16;
+};
+
+struct ScanSmem {
+    float A[2][TT][16][32];   // [stage][step in processing order][row*4+col][feature]
+    float b[2][TT][4][32];
+    float agg[NW][20][32];
+    float cin[NW][4][32];
+    unsigned tick[2];
 };
 
 template <bool REVERSE>
-SLSTM_DEVINL void load_step(const ScanArgs &a, size_t row, size_t jj, Aff &m)
+SLSTM_DEVINL int step_time(int T, int chunk, int step)
 {
+    const int p = chunk * TT + step;
+    return REVERSE ? T - 1 - p : p;
+}
+
+// Copies of one tile's A and b rows into stage `st`; steps outside [0, T)
+// and features past d arrive as zeros.
+template <bool REVERSE>
+SLSTM_DEVINL void scan_prefetch(const ScanArgs &a, ScanSmem &sm, int st, unsigned ticket)
+{
+    if (ticket >= (unsigned)a.n_tiles) return;
+    const int G = a.ca.n_groups;
+    const int chunk = (int)(ticket / (unsigned)G);
+    const int grp = (int)(ticket % (unsigned)G);
+    const int bb = grp / a.groups_per_row;
+    const int j0 = (grp % a.groups_per_row) * 32;
+    const int T = a.T;
     const size_t d = (size_t)a.d;
-    const float *pa = a.A + row * 16 * d + jj;
-    const float *pb = a.b + row * 4 * d + jj;
+    const size_t row0 = (size_t)bb * T;
+    if (a.vec16) {
+        // thread (q, c): step q, 16-byte chunk c of each of the 20 rows
+        const int c = threadIdx.x & 7, q = threadIdx.x >> 3;
+        const int jj = j0 + 4 * c;
+        const int t = step_time<REVERSE>(T, chunk, q);
+        const int bytes = (jj < a.d && t >= 0 && t < T) ? 4 * min(4, a.d - jj) : 0;
+        const float *pa = bytes ? a.A + (row0 + t) * 16 * d + jj : a.A;
+        const float *pb = bytes ? a.b + (row0 + t) * 4 * d + jj : a.b;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) cp_async16(&sm.A[st][q][e][4 * c], bytes ? pa + e * d : a.A, bytes);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cp_async16(&sm.b[st][q][e][4 * c], bytes ? pb + e * d : a.b, bytes);
+    } else {
+        // 4-byte copies, lane = feature; warp w takes steps w, w+8, ...
+        const int jl = threadIdx.x & 31, w = threadIdx.x >> 5;
+        const bool fj = j0 + jl < a.d;
+        for (int q = w; q < TT; q += NW) {
+            const int t = step_time<REVERSE>(T, chunk, q);
+            const int bytes = (fj && t >= 0 && t < T) ? 4 : 0;
+            const float *pa = bytes ? a.A + (row0 + t) * 16 * d + j0 + jl : a.A;
+            const float *pb = bytes ? a.b + (row0 + t) * 4 * d + j0 + jl : a.b;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) cp_async4(&sm.A[st][q][e][jl], bytes ? pa + e * d : a.A, bytes);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cp_async4(&sm.b[st][q][e][jl], bytes ? pb + e * d : a.b, bytes);
+        }
+    }
+}
+
+// The map of one step from shared memory (transposed matrix in reverse mode).
+template <bool REVERSE>
+SLSTM_DEVINL void load_map(const ScanSmem &sm, int st, int q, int lane, Aff &m)
+{
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const float v = __ldg(pa + (r * 4 + c) * d);
+            const float v = sm.A[st][q][r * 4 + c][lane];
             if (REVERSE)
                 m.a[c * 4 + r] = v;
             else
                 m.a[r * 4 + c] = v;
         }
 #pragma unroll
-    for (int e = 0; e < 4; ++e) m.b[e] = __ldg(pb + e * d);
+    for (int e = 0; e < 4; ++e) m.b[e] = sm.b[st][q][e][lane];
 }
 
 template <bool REVERSE>
-__global__ void __launch_bounds__(NW * 32, 2) scan_kernel(ScanArgs a)
+__global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
 {
-    __shared__ float s_agg[NW][20][32];
-    __shared__ float s_cin[4][32];
-    __shared__ unsigned s_ticket;
+    extern __shared__ float4 smem_f4[];
+    ScanSmem &sm = *reinterpret_cast<ScanSmem *>(smem_f4);
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    if (threadIdx.x == 0) s_ticket = atomicAdd(a.ticket, 1u);
-    __syncthreads();
-    const unsigned ticket = s_ticket;
-    const int G = a.lb.n_groups;
-    const int chunk = (int)(ticket / (unsigned)G);
-    const int grp = (int)(ticket % (unsigned)G);
-    const int bb = grp / a.groups_per_row;
-    const int j = (grp % a.groups_per_row) * 32 + lane;
-    const bool jv = j < a.d;
-    const size_t jj = jv ? (size_t)j : 0;
-    const size_t d = (size_t)a.d;
+    const int G = a.ca.n_groups;
     const int T = a.T;
-    const int p_seg = chunk * TT + warp * L;
-    const size_t row0 = (size_t)bb * T;
+    const size_t d = (size_t)a.d;
 
-    Aff agg;
-    aff_identity(agg);
-#pragma unroll
-    for (int i = 0; i < L; ++i) {
-        const int p = p_seg + i;
-        if (p < T && jv) {
-            const int t = REVERSE ? T - 1 - p : p;
-            Aff m;
-            load_step<REVERSE>(a, row0 + t, jj, m);
-            aff_compose(m, agg, agg);
-        }
-    }
-    store_aff_smem(s_agg, warp, lane, agg);
-    __syncthreads();
-    tile_prefix_tree<NW>(s_agg, agg);
-    if (warp == 0) {
-        float first[4] = {0.f, 0.f, 0.f, 0.f};
-        if (a.y0 && jv) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) first[e] = a.y0[((size_t)bb * 4 + e) * d + jj];
-        }
-        tile_lookback_warp0<NW>(s_agg, s_cin, a.lb, ticket, chunk, first, false);
+    if (threadIdx.x == 0) {
+        sm.tick[0] = atomicAdd(a.ticket, 1u);
+        sm.tick[1] = atomicAdd(a.ticket, 1u);
     }
     __syncthreads();
+    unsigned cur = sm.tick[0];
+    unsigned nxt = sm.tick[1];
+    int st = 0;
+    scan_prefetch<REVERSE>(a, sm, 0, cur);
+    cp_async_commit();
 
-    float v[4];
-    warp_carry(s_agg, s_cin, warp, lane, v);
+    while (cur < (unsigned)a.n_tiles) {
+        unsigned after = 0;
+        if (threadIdx.x == 0) after = atomicAdd(a.ticket, 1u);
+        scan_prefetch<REVERSE>(a, sm, st ^ 1, nxt);
+        cp_async_commit();
+        cp_async_wait_prev();
+        __syncthreads();
+
+        const unsigned ticket = cur;
+        const int chunk = (int)(ticket / (unsigned)G);
+        const int grp = (int)(ticket % (unsigned)G);
+        const int bb = grp / a.groups_per_row;
+        const int j = (grp % a.groups_per_row) * 32 + lane;
+        const bool jv = j < a.d;
+        const size_t jj = jv ? (size_t)j : 0;
+        const size_t row0 = (size_t)bb * T;
+
+        // ---- walk A ----
+        Aff agg;
+        aff_identity(agg);
 #pragma unroll
-    for (int i = 0; i < L; ++i) {
-        const int p = p_seg + i;
-        if (p < T && jv) {
-            const int t = REVERSE ? T - 1 - p : p;
-            Aff m;
-            load_step<REVERSE>(a, row0 + t, jj, m);
-            aff_apply(m, v, v);
-            float *py = a.y + (row0 + t) * 4 * d + jj;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) py[e * d] = v[e];
+        for (int i = 0; i < L; ++i) {
+            const int q = warp * L + i;
+            if (chunk * TT + q < T) {
+                Aff m;
+                load_map<REVERSE>(sm, st, q, lane, m);
+                aff_compose(m, agg, agg);
+            }
         }
+        store_aff_smem(sm.agg, warp, lane, agg);
+        __syncthreads();
+        if (warp == 0) {
+            float first[4] = {0.f, 0.f, 0.f, 0.f};
+            if (a.y0 && jv) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) first[e] = __ldg(a.y0 + ((size_t)bb * 4 + e) * d + jj);
+            }
+            tile_carry_serial<NW>(a.ca, sm.agg, sm.cin, ticket, chunk, grp, first, false);
+        }
+        __syncthreads();
+
+        // ---- walk B ----
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = sm.cin[warp][e][lane];
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int q = warp * L + i;
+            if (chunk * TT + q < T) {
+                const int t = step_time<REVERSE>(T, chunk, q);
+                Aff m;
+                load_map<REVERSE>(sm, st, q, lane, m);
+                aff_apply(m, v, v);
+                float *py = a.y + (row0 + t) * 4 * d + jj;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (jv) py[e * d] = v[e];
+            }
+        }
+        if (threadIdx.x == 0) sm.tick[0] = after;
+        __syncthreads();
+        cur = nxt;
+        nxt = sm.tick[0];
+        st ^= 1;
     }
+    cp_async_wait_all();
 }
 
 struct Layout {
-    size_t ticket, flags, agg, inc, total;
+    size_t ticket, flags, incw, agg, total;
     int groups_per_row, n_groups, n_chunks, n_tiles;
 };
 
@@ -133,10 +220,39 @@ Layout layout(int B, int T, int d)
     };
     l.ticket = take(256);
     l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles);
+    l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles);
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
-    l.inc = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.total = off;
     return l;
+}
+
+int sm_count_scan()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+    }
+    return n;
+}
+
+template <bool REVERSE>
+cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st)
+{
+    auto kern = scan_kernel<REVERSE>;
+    static int blocks_per_sm = 0;
+    if (blocks_per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(ScanSmem));
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, sizeof(ScanSmem));
+        if (e != cudaSuccess) return e;
+        if (blocks_per_sm < 1) blocks_per_sm = 1;
+    }
+    const int grid = min(a.n_tiles, sm_count_scan() * blocks_per_sm);
+    kern<<<grid, NW * 32, sizeof(ScanSmem), st>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -154,24 +270,24 @@ cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, 
     a.y0 = y0;
     a.y = y;
     a.ticket = reinterpret_cast<unsigned *>(base + l.ticket);
-    a.lb.flags = reinterpret_cast<unsigned *>(base + l.flags);
-    a.lb.agg = reinterpret_cast<float *>(base + l.agg);
-    a.lb.inc = reinterpret_cast<float *>(base + l.inc);
-    a.lb.error = a.ticket + 1;
-    a.lb.epoch = 1;
-    a.lb.wait_ns = 2000000000ull;
-    a.lb.n_groups = l.n_groups;
+    a.ca.flags = reinterpret_cast<unsigned *>(base + l.flags);
+    a.ca.agg = reinterpret_cast<float *>(base + l.agg);
+    a.ca.incw = reinterpret_cast<unsigned long long *>(base + l.incw);
+    a.ca.error = a.ticket + 1;
+    a.ca.epoch = 1;
+    a.ca.wait_ns = 2000000000ull;
+    a.ca.n_groups = l.n_groups;
     a.T = T;
     a.d = d;
     a.groups_per_row = l.groups_per_row;
-    // the ticket counter, the error word and every flag start at zero
+    a.n_tiles = l.n_tiles;
+    a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(A) & 15) == 0 &&
+               (reinterpret_cast<uintptr_t>(b) & 15) == 0) ? 1 : 0;
+    // the ticket counter, the error word, every flag and the epoch tags of
+    // the inclusive prefixes start at zero
     cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
     if (e != cudaSuccess) return e;
-    if (reverse)
-        scan_kernel<true><<<l.n_tiles, NW * 32, 0, st>>>(a);
-    else
-        scan_kernel<false><<<l.n_tiles, NW * 32, 0, st>>>(a);
-    return cudaGetLastError();
+    return reverse ? launch_scan<true>(a, st) : launch_scan<false>(a, st);
 }
 
 }  // namespace slstm

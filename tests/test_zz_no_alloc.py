@@ -51,12 +51,12 @@ def test_noalloc_matches_scan_block4_twice(cuda_device):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_device):
-    # 2728 tiles of 32 steps x 32 features need more than the fixed block;
+    # 2338 tiles of 32 steps x 32 features need more than the fixed block;
     # rejected on the host, so the fake pointers are never touched
     fake = ctypes.c_void_p(0x10000)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     lib = _lib.load()
-    assert lib.scan_block4_noalloc(fake, fake, None, ctypes.c_void_p(0x20000), 1, 2728 * 32, 32, 0,
+    assert lib.scan_block4_noalloc(fake, fake, None, ctypes.c_void_p(0x20000), 1, 2338 * 32, 32, 0,
                                    stream) == _lib.SLSTM_ERR_UNSUPPORTED
     assert lib.scan_block4_noalloc(fake, fake, None, ctypes.c_void_p(0x20000), 1, 0, 32, 0,
                                    stream) == _lib.SLSTM_ERR_INVALID_ARG
