@@ -218,17 +218,25 @@ SLSTM_DEVINL bool read_inc_words(const CarryArgs &ca, unsigned tq, int lane, flo
 // inclusive prefix.  `first` enters chunk 0; `withhold` suppresses this
 // tile's publications (fault injection).  In the common case (predecessor
 // published) only 4-vectors move: v_{w+1} = A_w v_w + b_w; the 4x4 tile
-// aggregate is formed only when it must be published.
+// aggregate is formed only when it must be published.  `pre_ok` / `pre`: the
+// predecessor's prefix as read earlier by the caller (to overlap the load's
+// latency with other work); it is read again here when that read was early.
 template <int NW>
 SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32], float (*s_cin)[4][32],
-                                    unsigned ticket, int chunk, int grp, const float first[4], bool withhold)
+                                    unsigned ticket, int chunk, int grp, const float first[4], bool withhold,
+                                    bool pre_ok = false, const float *pre = nullptr)
 {
     const int lane = threadIdx.x & 31;
     float carry[4] = {first[0], first[1], first[2], first[3]};
     if (chunk > 0) {
         unsigned tq = ticket - (unsigned)ca.n_groups;
         float v[4];
-        const bool ok = read_inc_words(ca, tq, lane, v);
+        bool ok = pre_ok && (pre != nullptr);
+        if (ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = pre[e];
+        }
+        if (!__all_sync(0xffffffffu, ok)) ok = read_inc_words(ca, tq, lane, v);
         if (__all_sync(0xffffffffu, ok)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) carry[e] = v[e];
@@ -283,13 +291,18 @@ SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32],
             }
         }
     }
+    // the next warp's map is loaded while the current one is applied
     float v[4] = {carry[0], carry[1], carry[2], carry[3]};
+    Aff x;
+    load_aff_smem(s_agg, 0, lane, x);
+#pragma unroll
     for (int w = 0; w < NW; ++w) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) s_cin[w][e][lane] = v[e];
-        Aff x;
-        load_aff_smem(s_agg, w, lane, x);
+        Aff xn;
+        if (w + 1 < NW) load_aff_smem(s_agg, w + 1, lane, xn);
         aff_apply(x, v, v);
+        if (w + 1 < NW) x = xn;
     }
     if (!withhold) {
         unsigned long long *dst = ca.incw + (size_t)ticket * 4 * 32 + lane;
@@ -298,6 +311,15 @@ SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32],
             st_relaxed_u64(dst + e * 32, ((unsigned long long)ca.epoch << 32) | __float_as_uint(v[e]));
     }
 }
+
+// Value component e (slot order c, n, m, h) of a cell evaluation; e is a
+// compile-time constant after unrolling.
+SLSTM_DEVINL float cell_f(const Cell &c, int e) { return e == 0 ? c.c : (e == 1 ? c.n : (e == 2 ? c.m : c.h)); }
+
+// Named CTA barriers for a producer warp handing a value to a consumer warp:
+// the producer arrives, the consumer waits; `n` counts both warps' threads.
+SLSTM_DEVINL void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+SLSTM_DEVINL void named_bar_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // cp.async copies into shared memory (zero-fill beyond `bytes`).
 SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }

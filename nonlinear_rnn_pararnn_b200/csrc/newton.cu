@@ -238,6 +238,15 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             }
         }
 
+        // warp 0 issues the load of the previous tile's inclusive prefix now
+        // and checks it after walk A, so that the load's latency is hidden
+        unsigned long long prew[4] = {0ull, 0ull, 0ull, 0ull};
+        if (warp == 0 && chunk > 0) {
+            const unsigned long long *src = a.incw + (size_t)(ticket - (unsigned)G) * 4 * 32 + lane;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) prew[e] = ld_relaxed_u64(src + e * 32);
+        }
+
         // ---- walk A ----
         // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B
         Cell Jc[L];
@@ -276,8 +285,15 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         if (warp == 0) {
             CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
             const float zero[4] = {0.f, 0.f, 0.f, 0.f};
+            bool pre_ok = chunk > 0;
+            float pre[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                pre_ok = pre_ok && ((unsigned)(prew[e] >> 32) == a.epoch);
+                pre[e] = __uint_as_float((unsigned)prew[e]);
+            }
             tile_carry_serial<NW>(ca, sm.agg, sm.cin, ticket, chunk, grp, zero,
-                                  (k == 0) && ((int)ticket == a.fault_ticket));
+                                  (k == 0) && ((int)ticket == a.fault_ticket), pre_ok, pre);
         }
         __syncthreads();
 
