@@ -213,12 +213,11 @@ SLSTM_DEVINL void jacT_mul(const Cell &J, float &x0, float &x1, float &x2, float
 }
 
 // ---------------------------------------------------------------------------
-// Publish / look-back flags.  A flag word holds (epoch << 2) | state, with
-// state 1 = aggregate published, 2 = inclusive prefix published.  A fresh
-// epoch per launch means stale words never match.
+// Look-back flag word of a tile: (epoch << 2) | FLAG_AGG once the tile's
+// aggregate is published.  A fresh epoch per launch means stale words never
+// match.
 // ---------------------------------------------------------------------------
 constexpr unsigned FLAG_AGG = 1u;
-constexpr unsigned FLAG_INC = 2u;
 
 SLSTM_DEVINL unsigned ld_acquire(const unsigned *p)
 {
@@ -237,21 +236,6 @@ SLSTM_DEVINL uint64_t globaltimer_ns()
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
-}
-
-// Spin (one lane) until flag's epoch matches and its state is nonzero, or the
-// time limit passes.  Returns the state (1 or 2), or 0 on timeout.
-SLSTM_DEVINL unsigned wait_flag(const unsigned *flag, unsigned epoch, uint64_t limit_ns)
-{
-    unsigned v = ld_acquire(flag);
-    if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
-    const uint64_t t0 = globaltimer_ns();
-    for (unsigned polls = 0;; ++polls) {
-        if (polls >= 32) __nanosleep(64);
-        v = ld_acquire(flag);
-        if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
-        if (globaltimer_ns() - t0 > limit_ns) return 0u;
-    }
 }
 
 // Non-negative float max through its bit pattern (NaN sorts above +inf).

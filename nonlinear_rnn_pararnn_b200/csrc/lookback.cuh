@@ -1,39 +1,83 @@
-// Blocked scan of 4x4 affine maps across CTAs with a decoupled look-back.
+// Carry hand-off between the tiles of a blocked scan of 4x4 affine maps
+// (a block-bidiagonal solve) with a decoupled look-back.
 //
-// A "tile" is 32 features x (NW warps x L steps).  Inside a tile every warp
-// folds its own L steps serially (one feature per lane).  The NW warp
-// aggregates are turned into inclusive prefixes by a Kogge-Stone tree in
-// shared memory (all warps work, log2 NW levels).  Warp 0 then publishes the
-// tile aggregate, looks back over the tiles before it (same feature group,
-// earlier in processing order) until it meets a published inclusive prefix,
-// and publishes its own; every warp finally derives its incoming carry from
-// the tile carry and its predecessor's prefix.
+// A tile is 32 features x (NW warps x L steps).  Each warp folds its own L
+// steps into one affine map per feature (lane = feature) and stores it in
+// shared memory.  The carry entering the tile is the inclusive prefix of the
+// tile before it in the same feature group (ticket - n_groups); from it the
+// carry entering every warp follows by applying the warp maps in order, and
+// the last of these values is the tile's own inclusive prefix, which it
+// publishes for its successor.
 //
-// Tiles take tickets from a global counter in the order CTAs start, and tile
-// (chunk c, group g) has ticket c * n_groups + g, so a tile only ever waits
-// on tiles that started before it: every wait ends.  Waits are bounded in
-// time anyway; on expiry the tile records an error, continues with a zero
-// carry and still publishes, so that no other tile waits on it.
+// Publication.  An inclusive prefix (4 values per feature) is published as
+// 64-bit words (value bits | epoch << 32), so a reader validates and reads it
+// with one load per word and the writer needs no fence.  The epoch tags are
+// cleared at the start of every call and each launch of the call has its own
+// epoch.  A tile whose predecessor has not published yet publishes its own
+// aggregate (gated by a per-tile flag word) and looks back past unfinished
+// tiles, composing their aggregates until it meets a published prefix.
 //
-// Global state per tile (ticket):  flag word, aggregate [20][32] and
-// inclusive prefix [4][32] (feature-contiguous so that a warp moves 128-byte
-// rows).
+// Progress.  Tiles take tickets from a global counter in the order CTAs ask
+// for them, tile (chunk c, group g) has ticket c * n_groups + g, and a CTA
+// only waits on lower tickets, each held by a running CTA as its current
+// tile: every wait ends.  Waits are also bounded in time; on expiry the tile
+// records an error and continues with a zero carry.
+//
+// Two layouts of the per-warp maps are supported.  The plain one,
+// s_agg[w][20][32] (entry-major), is walked by warp 0 alone.  TileMaps stores
+// the maps column-major with a padded row stride so that four warps can walk
+// them at once with one (feature, row) pair per lane (carry_chain4): the
+// carry's serial dependence over the NW maps then costs one 4-term dot
+// product per map and lane instead of a 4x4 matrix-vector product.
 #pragma once
 
 #include "common.cuh"
 
 namespace slstm {
 
-struct LookbackArgs {
-    unsigned *flags;   // [n_tiles]
-    float *agg;        // [n_tiles][20][32]
-    float *inc;        // [n_tiles][4][32]
-    unsigned *error;   // set to nonzero when a wait expires
-    unsigned epoch;    // nonzero, unique per launch since the flags were cleared
-    uint64_t wait_ns;  // bound of one wait
-    int n_groups;      // feature groups (tiles per chunk)
+struct CarryArgs {
+    unsigned *flags;              // [n_tiles] aggregate-published flags
+    float *agg;                   // [n_tiles][20][32] published aggregates
+    unsigned long long *incw;     // [n_tiles][4][32] inclusive prefixes (value bits | epoch << 32)
+    unsigned *error;              // set to nonzero when a wait expires
+    unsigned epoch;               // nonzero, unique per launch since the tags were cleared
+    unsigned long long wait_ns;   // bound of one wait
+    int n_groups;                 // feature groups (tiles per chunk)
 };
 
+SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+SLSTM_DEVINL void st_relaxed_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+SLSTM_DEVINL unsigned long long inc_word(unsigned epoch, float v)
+{
+    return ((unsigned long long)epoch << 32) | __float_as_uint(v);
+}
+
+// This lane's part (feature `lane`, 4 slots) of tile tq's inclusive prefix,
+// if published in this launch.
+SLSTM_DEVINL bool read_inc_words(const CarryArgs &ca, unsigned tq, int lane, float v[4])
+{
+    const unsigned long long *src = ca.incw + (size_t)tq * 4 * 32 + lane;
+    bool ok = true;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const unsigned long long w = ld_relaxed_u64(src + e * 32);
+        ok = ok && ((unsigned)(w >> 32) == ca.epoch);
+        v[e] = __uint_as_float((unsigned)w);
+    }
+    return ok;
+}
+
+// ---- plain layout -----------------------------------------------------------
 SLSTM_DEVINL void load_aff_smem(float (*s_agg)[20][32], int w, int lane, Aff &x)
 {
 #pragma unroll
@@ -50,266 +94,218 @@ SLSTM_DEVINL void store_aff_smem(float (*s_agg)[20][32], int w, int lane, const 
     for (int e = 0; e < 4; ++e) s_agg[w][16 + e][lane] = x.b[e];
 }
 
-// All threads of the CTA.  On entry s_agg[w] holds warp w's aggregate (in
-// processing order) and `mine` the same value in registers; on exit s_agg[w]
-// holds the inclusive prefix agg_w o ... o agg_0.  Ends with a barrier.
-template <int NW>
-SLSTM_DEVINL void tile_prefix_tree(float (*s_agg)[20][32], Aff &mine)
-{
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int off = 1; off < NW; off <<= 1) {
-        Aff left;
-        if (warp >= off) load_aff_smem(s_agg, warp - off, lane, left);
-        __syncthreads();
-        if (warp >= off) {
-            aff_compose(mine, left, mine);
-            store_aff_smem(s_agg, warp, lane, mine);
-        }
-        __syncthreads();
-    }
-}
-
-// Warp 0 only, after tile_prefix_tree.  Publishes the tile aggregate
-// (s_agg[NW-1]), looks back, publishes the inclusive prefix and writes the
-// carry entering the tile to s_cin[0..3][lane].  `first_carry` is the value
-// entering chunk 0.  `withhold` suppresses this tile's publications (fault
-// injection).
-template <int NW>
-SLSTM_DEVINL void tile_lookback_warp0(float (*s_agg)[20][32], float (*s_cin)[32],
-                                      const LookbackArgs &lb, unsigned ticket, int chunk,
-                                      const float first_carry[4], bool withhold)
+// ---- look-back (warp 0, lane = feature) -------------------------------------
+// The predecessor has not published its prefix: publish this tile's
+// aggregate (composed from the warp maps that load(w, x) returns, in
+// processing order) unless `withhold`, then walk back over earlier tiles of
+// the group.  Returns this lane's carry entering the tile in `carry`.
+template <int NW, class LoadMap>
+SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned ticket, int chunk, int grp,
+                                bool withhold, float carry[4])
 {
     const int lane = threadIdx.x & 31;
     Aff tile;
-    load_aff_smem(s_agg, NW - 1, lane, tile);
-
-    float carry[4];
+    load(0, tile);
+    for (int w = 1; w < NW; ++w) {
+        Aff x;
+        load(w, x);
+        aff_compose(x, tile, tile);
+    }
+    if (!withhold) {
+        float *dst = ca.agg + (size_t)ticket * 20 * 32;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) carry[e] = first_carry[e];
-
-    if (chunk > 0) {
-        if (!withhold) {
-            float *dst = lb.agg + (size_t)ticket * 20 * 32;
+        for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release(lb.flags + ticket, (lb.epoch << 2) | FLAG_AGG);
+        for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release(ca.flags + ticket, (ca.epoch << 2) | FLAG_AGG);
+    }
+    Aff M;  // composition of the aggregates met so far (latest first)
+    aff_identity(M);
+    int q = chunk - 1;
+    const uint64_t t0 = globaltimer_ns();
+    unsigned polls = 0;
+    for (;;) {
+        const unsigned tq = (unsigned)q * (unsigned)ca.n_groups + (unsigned)grp;
+        float v[4];
+        const bool got = read_inc_words(ca, tq, lane, v);
+        if (__all_sync(0xffffffffu, got)) {
+            aff_apply(M, v, carry);
+            return;
         }
-        Aff M;  // composition of the aggregates met so far (latest first)
-        aff_identity(M);
-        int q = chunk - 1;
-        bool expired = false;
-        const unsigned grp = ticket % (unsigned)lb.n_groups;
-        for (;;) {
-            const unsigned tq = (unsigned)q * (unsigned)lb.n_groups + grp;
-            unsigned st = 0;
-            if (lane == 0) st = wait_flag(lb.flags + tq, lb.epoch, lb.wait_ns);
-            st = __shfl_sync(0xffffffffu, st, 0);
-            if (st == 0u) {
-                expired = true;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) carry[e] = 0.0f;
-                break;
-            }
-            if (st == FLAG_INC) {
-                float v[4];
-                const float *src = lb.inc + (size_t)tq * 4 * 32;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) v[e] = __ldcg(src + e * 32 + lane);
-                aff_apply(M, v, carry);
-                break;
-            }
+        const unsigned f = ld_acquire(ca.flags + tq);
+        if ((f >> 2) == ca.epoch && (f & 3u) == FLAG_AGG) {
             Aff x;
-            const float *src = lb.agg + (size_t)tq * 20 * 32;
+            const float *src = ca.agg + (size_t)tq * 20 * 32;
 #pragma unroll
             for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
 #pragma unroll
             for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
             aff_compose(M, x, M);
-            --q;  // chunk 0 always publishes an inclusive prefix, so q stays >= 0
+            --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
+            continue;
         }
-        if (expired && lane == 0) atomicOr(lb.error, 1u);
+        if (++polls > 16) __nanosleep(64);
+        if (globaltimer_ns() - t0 > ca.wait_ns) {
+            atomicOr(ca.error, 1u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) carry[e] = 0.f;
+            return;
+        }
     }
-
-    if (!withhold) {
-        float incv[4];
-        aff_apply(tile, carry, incv);
-        float *dst = lb.inc + (size_t)ticket * 4 * 32;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = incv[e];
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) st_release(lb.flags + ticket, (lb.epoch << 2) | FLAG_INC);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s_cin[e][lane] = carry[e];
 }
 
-// Any warp, after the barrier that follows tile_lookback_warp0: the carry
-// entering warp `warp` of the tile.
-SLSTM_DEVINL void warp_carry(float (*s_agg)[20][32], float (*s_cin)[32], int warp, int lane,
-                             float out[4])
-{
-    float cin[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) cin[e] = s_cin[e][lane];
-    if (warp == 0) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) out[e] = cin[e];
-        return;
-    }
-    Aff pre;
-    load_aff_smem(s_agg, warp - 1, lane, pre);
-    aff_apply(pre, cin, out);
-}
-
-// ---------------------------------------------------------------------------
-// Carry hand-off used by the persistent kernels (Newton iteration, adjoint).
-// A tile's inclusive prefix (4 values per feature) is published as 64-bit
-// words (value bits | epoch << 32): a reader validates and reads it with one
-// load per word and the writer needs no fence.  The epoch tags are cleared
-// at the start of every call, and each launch of the call has its own epoch.
-// A tile whose predecessor has not published yet publishes its aggregate
-// (gated by the per-tile flag word) and looks back past unfinished tiles.
-// ---------------------------------------------------------------------------
-struct CarryArgs {
-    unsigned *flags;              // [n_tiles]
-    float *agg;                   // [n_tiles][20][32]
-    unsigned long long *incw;     // [n_tiles][4][32]
-    unsigned *error;
-    unsigned epoch;
-    unsigned long long wait_ns;
-    int n_groups;
-};
-
-SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
-{
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-SLSTM_DEVINL void st_relaxed_u64(unsigned long long *p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// This lane's part of tile tq's inclusive prefix, if published in this launch.
-SLSTM_DEVINL bool read_inc_words(const CarryArgs &ca, unsigned tq, int lane, float v[4])
-{
-    const unsigned long long *src = ca.incw + (size_t)tq * 4 * 32 + lane;
-    bool ok = true;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const unsigned long long w = ld_relaxed_u64(src + e * 32);
-        ok = ok && ((unsigned)(w >> 32) == ca.epoch);
-        v[e] = __uint_as_float((unsigned)w);
-    }
-    return ok;
-}
-
-// Warp 0 only.  s_agg[w] holds warp w's own aggregate (in processing order).
-// Writes the carry entering every warp to s_cin[w] and publishes the tile's
-// inclusive prefix.  `first` enters chunk 0; `withhold` suppresses this
-// tile's publications (fault injection).  In the common case (predecessor
-// published) only 4-vectors move: v_{w+1} = A_w v_w + b_w; the 4x4 tile
-// aggregate is formed only when it must be published.  `pre_ok` / `pre`: the
-// predecessor's prefix as read earlier by the caller (to overlap the load's
-// latency with other work); it is read again here when that read was early.
-template <int NW>
-SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32], float (*s_cin)[4][32],
-                                    unsigned ticket, int chunk, int grp, const float first[4], bool withhold,
-                                    bool pre_ok = false, const float *pre = nullptr)
+// Warp 0, lane = feature: v_{w+1} = A_w v_w + b_w through the tile from
+// `carry`; put(w, v_w) stores the carry entering warp w; the final value, the
+// tile's inclusive prefix, is published unless `withhold`.
+template <int NW, class LoadMap, class PutCarry>
+SLSTM_DEVINL void carry_serial(const CarryArgs &ca, LoadMap load, PutCarry put, unsigned ticket, bool withhold,
+                               const float carry[4])
 {
     const int lane = threadIdx.x & 31;
-    float carry[4] = {first[0], first[1], first[2], first[3]};
-    if (chunk > 0) {
-        unsigned tq = ticket - (unsigned)ca.n_groups;
-        float v[4];
-        bool ok = pre_ok && (pre != nullptr);
-        if (ok) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = pre[e];
-        }
-        if (!__all_sync(0xffffffffu, ok)) ok = read_inc_words(ca, tq, lane, v);
-        if (__all_sync(0xffffffffu, ok)) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) carry[e] = v[e];
-        } else {
-            Aff tile;
-            load_aff_smem(s_agg, 0, lane, tile);
-            for (int w = 1; w < NW; ++w) {
-                Aff x;
-                load_aff_smem(s_agg, w, lane, x);
-                aff_compose(x, tile, tile);
-            }
-            if (!withhold) {
-                float *dst = ca.agg + (size_t)ticket * 20 * 32;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
-                __threadfence();
-                __syncwarp();
-                if (lane == 0) st_release(ca.flags + ticket, (ca.epoch << 2) | FLAG_AGG);
-            }
-            Aff M;
-            aff_identity(M);
-            int q = chunk - 1;
-            const uint64_t t0 = globaltimer_ns();
-            unsigned polls = 0;
-            for (;;) {
-                tq = (unsigned)q * (unsigned)ca.n_groups + (unsigned)grp;
-                if (read_inc_words(ca, tq, lane, v)) {
-                    aff_apply(M, v, carry);
-                    break;
-                }
-                const unsigned f = ld_acquire(ca.flags + tq);
-                if ((f >> 2) == ca.epoch && (f & 3u) == FLAG_AGG) {
-                    Aff x;
-                    const float *src = ca.agg + (size_t)tq * 20 * 32;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
-                    aff_compose(M, x, M);
-                    --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
-                    continue;
-                }
-                if (++polls > 16) __nanosleep(64);
-                if (globaltimer_ns() - t0 > ca.wait_ns) {
-                    atomicOr(ca.error, 1u);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) carry[e] = 0.f;
-                    break;
-                }
-            }
-        }
-    }
     // the next warp's map is loaded while the current one is applied
     float v[4] = {carry[0], carry[1], carry[2], carry[3]};
     Aff x;
-    load_aff_smem(s_agg, 0, lane, x);
+    load(0, x);
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s_cin[w][e][lane] = v[e];
+        put(w, v);
         Aff xn;
-        if (w + 1 < NW) load_aff_smem(s_agg, w + 1, lane, xn);
+        if (w + 1 < NW) load(w + 1, xn);
         aff_apply(x, v, v);
         if (w + 1 < NW) x = xn;
     }
     if (!withhold) {
         unsigned long long *dst = ca.incw + (size_t)ticket * 4 * 32 + lane;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            st_relaxed_u64(dst + e * 32, ((unsigned long long)ca.epoch << 32) | __float_as_uint(v[e]));
+        for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(ca.epoch, v[e]));
     }
+}
+
+// Warp 0 only, plain layout.  Writes the carry entering every warp to
+// s_cin[w] and publishes the tile's inclusive prefix.  `first` enters chunk
+// 0; `withhold` suppresses this tile's publications (fault injection).
+// `pre_ok` / `pre`: the predecessor's prefix as read earlier by the caller
+// (to overlap the load's latency with other work); it is read again here
+// when that read was early.
+template <int NW>
+SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32], float (*s_cin)[4][32],
+                                    unsigned ticket, int chunk, int grp, const float first[4], bool withhold,
+                                    bool pre_ok = false, const float *pre = nullptr)
+{
+    const int lane = threadIdx.x & 31;
+    auto load = [&](int w, Aff &x) { load_aff_smem(s_agg, w, lane, x); };
+    float carry[4] = {first[0], first[1], first[2], first[3]};
+    if (chunk > 0) {
+        bool ok = pre_ok && (pre != nullptr);
+        if (ok) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) carry[e] = pre[e];
+        }
+        if (!__all_sync(0xffffffffu, ok)) ok = read_inc_words(ca, ticket - (unsigned)ca.n_groups, lane, carry);
+        if (!__all_sync(0xffffffffu, ok)) tile_lookback<NW>(ca, load, ticket, chunk, grp, withhold, carry);
+    }
+    carry_serial<NW>(
+        ca, load,
+        [&](int w, const float v[4]) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s_cin[w][e][lane] = v[e];
+        },
+        ticket, withhold, carry);
+}
+
+// ---- chain layout -------------------------------------------------------------
+// Row stride of TileMaps: with 40 floats, (row, feature) pairs of one chain
+// warp (8 features x 4 rows) fall in 32 distinct banks.
+constexpr int MAP_LD = 40;
+
+template <int NW>
+struct TileMaps {
+    float m[NW][5][4][MAP_LD];   // [warp][column k, k = 4: offset b][row][feature]
+    float cin[NW][4][MAP_LD];    // [warp][slot][feature]: carry entering the warp's steps
+};
+
+// Lane = feature.
+template <int NW>
+SLSTM_DEVINL void maps_store(TileMaps<NW> &t, int w, int lane, const Aff &x)
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) t.m[w][k][r][lane] = x.a[r * 4 + k];
+        t.m[w][4][r][lane] = x.b[r];
+    }
+}
+
+template <int NW>
+SLSTM_DEVINL void maps_load(const TileMaps<NW> &t, int w, int lane, Aff &x)
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x.a[r * 4 + k] = t.m[w][k][r][lane];
+        x.b[r] = t.m[w][4][r][lane];
+    }
+}
+
+// Chain lanes: warps 0..3, lane (row = lane >> 3, feature = 8 * warp + (lane & 7)).
+SLSTM_DEVINL int chain_feature(int warp, int lane) { return ((warp & 3) << 3) | (lane & 7); }
+SLSTM_DEVINL int chain_row(int lane) { return lane >> 3; }
+
+// Word of tile tq's inclusive prefix that chain lane (warp, lane) owns.
+SLSTM_DEVINL size_t chain_word(unsigned tq, int warp, int lane)
+{
+    return ((size_t)tq * 4 + chain_row(lane)) * 32 + chain_feature(warp, lane);
+}
+
+// Chain warps only.  c: this lane's component of the carry entering the
+// tile.  Stores the carry entering every warp in t.cin and returns this
+// lane's component of the tile's inclusive prefix.  The arithmetic (order of
+// the fused multiply-adds) is that of aff_apply, so both walks give the same
+// bits.
+template <int NW>
+SLSTM_DEVINL float carry_chain4(TileMaps<NW> &t, float c, int warp, int lane)
+{
+    const int f = chain_feature(warp, lane);
+    const int r = chain_row(lane);
+    const int i8 = lane & 7;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        t.cin[w][r][f] = c;
+        const float a0 = t.m[w][0][r][f];
+        const float a1 = t.m[w][1][r][f];
+        const float a2 = t.m[w][2][r][f];
+        const float a3 = t.m[w][3][r][f];
+        const float bb = t.m[w][4][r][f];
+        const float v0 = __shfl_sync(0xffffffffu, c, i8);
+        const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
+        const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
+        const float v3 = __shfl_sync(0xffffffffu, c, 24 + i8);
+        c = fmaf(a3, v3, fmaf(a2, v2, fmaf(a1, v1, fmaf(a0, v0, bb))));
+    }
+    return c;
+}
+
+// Warp 0 only, chain layout, when some chain lane found no published
+// predecessor prefix: reads it again, else looks back; then walks the maps
+// serially (lane = feature).  chunk > 0.
+template <int NW>
+SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, TileMaps<NW> &t, unsigned ticket, int chunk, int grp,
+                                      bool withhold)
+{
+    const int lane = threadIdx.x & 31;
+    auto load = [&](int w, Aff &x) { maps_load(t, w, lane, x); };
+    float carry[4];
+    const bool ok = read_inc_words(ca, ticket - (unsigned)ca.n_groups, lane, carry);
+    if (!__all_sync(0xffffffffu, ok)) tile_lookback<NW>(ca, load, ticket, chunk, grp, withhold, carry);
+    carry_serial<NW>(
+        ca, load,
+        [&](int w, const float v[4]) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t.cin[w][e][lane] = v[e];
+        },
+        ticket, withhold, carry);
 }
 
 // Value component e (slot order c, n, m, h) of a cell evaluation; e is a

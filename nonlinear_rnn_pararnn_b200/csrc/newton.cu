@@ -13,24 +13,14 @@
 //   walk A  each thread recomputes gates, stabilizer, f(S_{t-1}, P_t) and the
 //           4x4 Jacobian J_t in registers for its 4 steps, keeps (J_t, r_t =
 //           f - S_t) in registers and folds the maps delta -> J_t delta + r_t;
-//   scan    the 8 warp aggregates become inclusive prefixes (Kogge-Stone in
-//           shared memory); warp 0 obtains the carry entering the tile from
-//           the tile before it (see below) and publishes this tile's
-//           inclusive prefix;
+//   carry   the carry entering the tile is the predecessor tile's inclusive
+//           prefix (looked at twice: before and after walk A); warps 0-3
+//           apply the 8 warp maps to it, one (feature, slot) pair per lane,
+//           and publish this tile's prefix; a tile whose predecessor has not
+//           published falls back to the look-back in lookback.cuh;
 //   walk B  each thread replays its steps from its carry, writes S + delta in
 //           place and, when asked, accumulates the residual of the new
 //           iterate for the stopping test.
-//
-// Carry hand-off between tiles.  A tile's inclusive prefix (4 values per
-// feature) is published as 64-bit words (value bits, launch epoch), so a
-// reader validates and reads it in one load and the writer needs no fence.
-// A tile whose predecessor has not published yet first publishes its own
-// aggregate (20 values per feature, gated by a per-tile flag word) and then
-// looks back past unfinished predecessors, composing their aggregates.
-// Tickets are taken in start order and every wait is on a lower ticket that
-// some running CTA holds as its current tile, so every wait ends; waits are
-// also bounded in time (expiry sets an error and continues with a zero
-// carry).
 //
 // In-place update is safe because the only value a tile reads from another
 // tile (the state just before it) comes from a per-tile boundary buffer
@@ -66,59 +56,86 @@ struct Args {
     float tol;
 };
 
+// A ticket decoded once (by thread 0) for the whole CTA.
+struct TileInfo {
+    unsigned ticket;
+    int chunk;
+    int b;
+    int j0;
+    unsigned long long off;   // element offset of (b, chunk * TT, slot 0, feature j0) in P and S
+    unsigned long long pad;
+};
+
 struct Smem {
     float P[2][TT][4][32];
     float S[2][TT][4][32];
-    float agg[NW][20][32];
-    float cin[NW][4][32];
+    TileMaps<NW> maps;
+    TileInfo info[3];   // ring: current, next and the one after
     float red[2][NW];
-    unsigned tick[2];
     int exit_flag;
 };
 
+SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
+{
+    ti.ticket = ticket;
+    ti.chunk = ti.b = ti.j0 = 0;
+    ti.off = 0;
+    if (ticket < (unsigned)a.n_tiles) {
+        const unsigned chunk = ticket / (unsigned)a.n_groups;
+        const unsigned grp = ticket - chunk * (unsigned)a.n_groups;
+        const unsigned b = grp / (unsigned)a.groups_per_row;
+        ti.chunk = (int)chunk;
+        ti.b = (int)b;
+        ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
+        ti.off = ((size_t)b * a.T + (size_t)chunk * TT) * 4 * (size_t)a.d + (size_t)ti.j0;
+    }
+}
+
+// Per-thread part of the copy offsets (see prefetch_tile).
+SLSTM_DEVINL size_t prefetch_offset(const Args &a)
+{
+    const int w = threadIdx.x >> 5;
+    if (a.vec16) return (size_t)(w * 4 + ((threadIdx.x >> 3) & 3)) * a.d + 4 * (threadIdx.x & 7);
+    return (size_t)w * a.d + (threadIdx.x & 31);
+}
+
 // Issue the copies of one tile's P (and old S unless `with_s` is false) into
 // shared-memory stage `st`.  Rows past T and features past d read nothing and
-// arrive as zeros.
-SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, unsigned ticket, bool with_s)
+// arrive as zeros.  `toff` = prefetch_offset(a).
+SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo &ti, size_t toff, bool with_s)
 {
-    if (ticket >= (unsigned)a.n_tiles) return;
-    const int chunk = (int)(ticket / (unsigned)a.n_groups);
-    const int grp = (int)(ticket % (unsigned)a.n_groups);
-    const int b = grp / a.groups_per_row;
-    const int j0 = (grp % a.groups_per_row) * 32;
-    const int t0 = chunk * TT;
-    const size_t d = (size_t)a.d;
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const int t0 = ti.chunk * TT;
     const int w = threadIdx.x >> 5;
+    const float *p = a.P + ti.off + toff;
+    const float *s = a.S + ti.off + toff;
     if (a.vec16) {
         // 8 chunks of 16 bytes per (step, slot) row of 32 features; thread
         // (w, slot, c) copies chunk c of slot `slot` for steps w, w+8, w+16, w+24
         const int c = threadIdx.x & 7, slot = (threadIdx.x >> 3) & 3;
-        const int jj = j0 + 4 * c;
-        const int fbytes = jj < a.d ? 4 * min(4, a.d - jj) : 0;
-        const size_t off0 = (((size_t)b * a.T + t0 + w) * 4 + slot) * d + jj;
-        const size_t step8 = 32 * d;   // 8 steps of 4 slots
+        const int rem = a.d - ti.j0 - 4 * c;
+        const int fbytes = rem > 0 ? 4 * min(4, rem) : 0;
+        const size_t step8 = 32 * (size_t)a.d;   // 8 steps of 4 slots
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int step = r * 8 + w;
             const int bytes = (t0 + step < a.T) ? fbytes : 0;
-            const size_t off = off0 + r * step8;
-            cp_async16(&sm.P[st][step][slot][4 * c], bytes ? a.P + off : a.P, bytes);
-            if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? a.S + off : a.S, bytes);
+            cp_async16(&sm.P[st][step][slot][4 * c], bytes ? p + r * step8 : a.P, bytes);
+            if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? s + r * step8 : a.S, bytes);
         }
     } else {
         // 4-byte copies, lane = feature; warp w copies rows w, w+8, ... of
         // the 128 (step, slot) rows
         const int jl = threadIdx.x & 31;
-        const bool fj = j0 + jl < a.d;
-        const size_t base0 = ((size_t)b * a.T + t0) * 4 * d + j0 + jl;
+        const bool fj = ti.j0 + jl < a.d;
+        const size_t row8 = 8 * (size_t)a.d;
 #pragma unroll 4
         for (int r = 0; r < 16; ++r) {
             const int rs = r * 8 + w;
             const int step = rs >> 2, slot = rs & 3;
             const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
-            const size_t off = base0 + (size_t)rs * d;
-            cp_async4(&sm.P[st][step][slot][jl], bytes ? a.P + off : a.P, bytes);
-            if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? a.S + off : a.S, bytes);
+            cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * row8 : a.P, bytes);
+            if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? s + r * row8 : a.S, bytes);
         }
     }
 }
@@ -176,8 +193,8 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
     if (threadIdx.x == 0) {
         sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
         if (!sm.exit_flag) {
-            sm.tick[0] = atomicAdd(&slot.ticket, 1u);
-            sm.tick[1] = atomicAdd(&slot.ticket, 1u);
+            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[0]);
+            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[1]);
         }
     }
     __syncthreads();
@@ -185,33 +202,33 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
 
     const size_t d = (size_t)a.d;
     const int T = a.T;
-    const int G = a.n_groups;
+    const unsigned G = (unsigned)a.n_groups;
+    const size_t toff = prefetch_offset(a);
+    const bool chain_warp = warp < 4;
     float mx_raw = 0.f, mx_sc = 0.f;
 
-    unsigned cur = sm.tick[0];
-    unsigned nxt = sm.tick[1];
-    int st = 0;
-    prefetch_tile(a, sm, 0, cur, !FIRST);
+    int ring = 0, st = 0;
+    prefetch_tile(a, sm, 0, sm.info[0], toff, !FIRST);
     cp_async_commit();
 
-    while (cur < (unsigned)a.n_tiles) {
-        // tickets run two tiles ahead: fetch the one after `nxt` now, publish it at the end
+    for (;;) {
+        const TileInfo ti = sm.info[ring];
+        if (ti.ticket >= (unsigned)a.n_tiles) break;
+        const int rn = ring == 2 ? 0 : ring + 1;
+        // tickets run two tiles ahead: fetch the one after the next now,
+        // decode it into the ring at the end of this tile
         unsigned after = 0;
         if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
-        prefetch_tile(a, sm, st ^ 1, nxt, !FIRST);
+        prefetch_tile(a, sm, st ^ 1, sm.info[rn], toff, !FIRST);
         cp_async_commit();
         cp_async_wait_prev();   // the current tile's copies have landed
         __syncthreads();
 
-        const unsigned ticket = cur;
-        const int chunk = (int)(ticket / (unsigned)G);
-        const int grp = (int)(ticket % (unsigned)G);
-        const int b = grp / a.groups_per_row;
-        const int j = (grp % a.groups_per_row) * 32 + lane;
-        const bool jv = j < a.d;
-        const size_t jj = jv ? (size_t)j : 0;
+        const unsigned ticket = ti.ticket;
+        const int chunk = ti.chunk;
+        const bool jv = ti.j0 + lane < a.d;
+        const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
         const int t_seg = chunk * TT + warp * L;
-        const size_t row0 = (size_t)b * T;
 
         float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
         if (jv) {
@@ -225,11 +242,11 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         if (t_seg == 0) {
             if (a.s0 && jv) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sp[e] = __ldg(a.s0 + ((size_t)b * 4 + e) * d + jj);
+                for (int e = 0; e < 4; ++e) sp[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
             }
         } else if (!FIRST) {
             if (warp == 0) {
-                const float *src = a.bnd_in + (size_t)(ticket - (unsigned)G) * 4 * 32;
+                const float *src = a.bnd_in + (size_t)(ticket - G) * 4 * 32;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
             } else {
@@ -238,14 +255,12 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             }
         }
 
-        // warp 0 issues the load of the previous tile's inclusive prefix now
-        // and checks it after walk A, so that the load's latency is hidden
-        unsigned long long prew[4] = {0ull, 0ull, 0ull, 0ull};
-        if (warp == 0 && chunk > 0) {
-            const unsigned long long *src = a.incw + (size_t)(ticket - (unsigned)G) * 4 * 32 + lane;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) prew[e] = ld_relaxed_u64(src + e * 32);
-        }
+        // first look at the predecessor's inclusive prefix (chain lanes); the
+        // load's latency is hidden behind walk A
+        const bool look = chain_warp && chunk > 0;
+        const unsigned long long *predw = a.incw + chain_word(ticket - G, warp, lane);
+        unsigned long long w1 = 0ull;
+        if (look) w1 = ld_relaxed_u64(predw);
 
         // ---- walk A ----
         // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B
@@ -280,32 +295,40 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
                 fold_jac(agg, Jc[i], r);
             }
         }
-        store_aff_smem(sm.agg, warp, lane, agg);
-        __syncthreads();
-        if (warp == 0) {
-            CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-            bool pre_ok = chunk > 0;
-            float pre[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                pre_ok = pre_ok && ((unsigned)(prew[e] >> 32) == a.epoch);
-                pre[e] = __uint_as_float((unsigned)prew[e]);
+        // second look, for a predecessor that published during walk A
+        unsigned long long w2 = 0ull;
+        if (look) w2 = ld_relaxed_u64(predw);
+        maps_store(sm.maps, warp, lane, agg);
+
+        // ---- carry ----
+        float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
+        bool ok = true;
+        if (look) {
+            const bool ok1 = (unsigned)(w1 >> 32) == a.epoch;
+            ok = ok1 || (unsigned)(w2 >> 32) == a.epoch;
+            c = __uint_as_float((unsigned)(ok1 ? w1 : w2));
+        }
+        const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
+        if (__syncthreads_and(ok)) {
+            if (chain_warp) {
+                c = carry_chain4(sm.maps, c, warp, lane);
+                if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
             }
-            tile_carry_serial<NW>(ca, sm.agg, sm.cin, ticket, chunk, grp, zero,
-                                  (k == 0) && ((int)ticket == a.fault_ticket), pre_ok, pre);
+        } else if (warp == 0) {
+            const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+            tile_carry_fallback<NW>(ca, sm.maps, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold);
         }
         __syncthreads();
 
         // ---- walk B ----
         float dl[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dl[e] = sm.cin[warp][e][lane];
+        for (int e = 0; e < 4; ++e) dl[e] = sm.maps.cin[warp][e][lane];
         float snp[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
         // row pointer of this lane's first step; lanes past d write nothing
-        float *srow = a.S + (row0 + t_seg) * 4 * d + jj;
+        float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int t = t_seg + i;
@@ -349,10 +372,9 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
         }
 
-        if (threadIdx.x == 0) sm.tick[0] = after;
-        __syncthreads();   // stage `st` and sm.agg are free again
-        cur = nxt;
-        nxt = sm.tick[0];
+        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
+        __syncthreads();   // stage `st`, the maps and the oldest ring entry are free again
+        ring = rn;
         st ^= 1;
     }
     cp_async_wait_all();
