@@ -215,6 +215,114 @@ SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32],
         ticket, withhold, carry);
 }
 
+// ---- packed fold ---------------------------------------------------------
+// A fold's running aggregate with its matrix columns paired, so that the
+// 4x4 products run on the packed fp32x2 pipe (__ffma2_rn / __fmul2_rn, two
+// lanes of the same scalar operation per instruction).  Each packed lane
+// performs exactly the scalar jac_mul / jacT_mul sequence, so the bits equal
+// those of fold_jac / fold_jacT.
+struct AffP {
+    float2 a01[4];   // row r: (A[r][0], A[r][1])
+    float2 a23[4];   // row r: (A[r][2], A[r][3])
+    float b[4];
+};
+
+SLSTM_DEVINL float2 dup2(float v) { return make_float2(v, v); }
+
+// Columns x_k <- J x_k for a pair of columns (rows in x[0..3]).
+SLSTM_DEVINL void jac_mul_p(const float2 j[11], float2 x[4])
+{
+    // j: fp, jcm, jch, jnm, jnh, beta, dmh, jhc, jhn, jhm, jhh
+    const float2 y0 = __ffma2_rn(j[0], x[0], __ffma2_rn(j[1], x[2], __fmul2_rn(j[2], x[3])));
+    const float2 y1 = __ffma2_rn(j[0], x[1], __ffma2_rn(j[3], x[2], __fmul2_rn(j[4], x[3])));
+    const float2 y2 = __ffma2_rn(j[5], x[2], __fmul2_rn(j[6], x[3]));
+    const float2 y3 = __ffma2_rn(j[7], x[0], __ffma2_rn(j[8], x[1], __ffma2_rn(j[9], x[2], __fmul2_rn(j[10], x[3]))));
+    x[0] = y0;
+    x[1] = y1;
+    x[2] = y2;
+    x[3] = y3;
+}
+
+// Columns x_k <- J^T x_k for a pair of columns.
+SLSTM_DEVINL void jacT_mul_p(const float2 j[11], float2 x[4])
+{
+    const float2 y0 = __ffma2_rn(j[0], x[0], __fmul2_rn(j[7], x[3]));
+    const float2 y1 = __ffma2_rn(j[0], x[1], __fmul2_rn(j[8], x[3]));
+    const float2 y2 = __ffma2_rn(j[1], x[0], __ffma2_rn(j[3], x[1], __ffma2_rn(j[5], x[2], __fmul2_rn(j[9], x[3]))));
+    const float2 y3 = __ffma2_rn(j[2], x[0], __ffma2_rn(j[4], x[1], __ffma2_rn(j[6], x[2], __fmul2_rn(j[10], x[3]))));
+    x[0] = y0;
+    x[1] = y1;
+    x[2] = y2;
+    x[3] = y3;
+}
+
+SLSTM_DEVINL void cell_pairs(const Cell &J, float2 j[11])
+{
+    j[0] = dup2(J.fp);
+    j[1] = dup2(J.jcm);
+    j[2] = dup2(J.jch);
+    j[3] = dup2(J.jnm);
+    j[4] = dup2(J.jnh);
+    j[5] = dup2(J.beta);
+    j[6] = dup2(J.dmh);
+    j[7] = dup2(J.jhc);
+    j[8] = dup2(J.jhn);
+    j[9] = dup2(J.jhm);
+    j[10] = dup2(J.jhh);
+}
+
+// agg <- (J, r) o agg (TRANS: J^T).
+template <bool TRANS>
+SLSTM_DEVINL void fold_p(AffP &agg, const Cell &J, const float r[4])
+{
+    float2 j[11];
+    cell_pairs(J, j);
+    float2 x[4] = {agg.a01[0], agg.a01[1], agg.a01[2], agg.a01[3]};
+    if (TRANS) jacT_mul_p(j, x); else jac_mul_p(j, x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) agg.a01[i] = x[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = agg.a23[i];
+    if (TRANS) jacT_mul_p(j, x); else jac_mul_p(j, x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) agg.a23[i] = x[i];
+    if (TRANS) jacT_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
+    else jac_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
+}
+
+// The aggregate of a single step: (J, r) (TRANS: (J^T, r)).
+template <bool TRANS>
+SLSTM_DEVINL void affp_from_cell(AffP &x, const Cell &J, const float r[4])
+{
+    if (TRANS) {
+        x.a01[0] = make_float2(J.fp, 0.f);   x.a23[0] = make_float2(0.f, J.jhc);
+        x.a01[1] = make_float2(0.f, J.fp);   x.a23[1] = make_float2(0.f, J.jhn);
+        x.a01[2] = make_float2(J.jcm, J.jnm); x.a23[2] = make_float2(J.beta, J.jhm);
+        x.a01[3] = make_float2(J.jch, J.jnh); x.a23[3] = make_float2(J.dmh, J.jhh);
+    } else {
+        x.a01[0] = make_float2(J.fp, 0.f);   x.a23[0] = make_float2(J.jcm, J.jch);
+        x.a01[1] = make_float2(0.f, J.fp);   x.a23[1] = make_float2(J.jnm, J.jnh);
+        x.a01[2] = make_float2(0.f, 0.f);    x.a23[2] = make_float2(J.beta, J.dmh);
+        x.a01[3] = make_float2(J.jhc, J.jhn); x.a23[3] = make_float2(J.jhm, J.jhh);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x.b[e] = r[e];
+}
+
+SLSTM_DEVINL void affp_to_aff(const AffP &p, Aff &x)
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        x.a[r * 4 + 0] = p.a01[r].x;
+        x.a[r * 4 + 1] = p.a01[r].y;
+        x.a[r * 4 + 2] = p.a23[r].x;
+        x.a[r * 4 + 3] = p.a23[r].y;
+        x.b[r] = p.b[r];
+    }
+}
+
 // ---- chain layout -------------------------------------------------------------
 // Row stride of TileMaps: with 40 floats, (row, feature) pairs of one chain
 // warp (8 features x 4 rows) fall in 32 distinct banks.
@@ -234,6 +342,19 @@ SLSTM_DEVINL void maps_store(TileMaps<NW> &t, int w, int lane, const Aff &x)
     for (int r = 0; r < 4; ++r) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) t.m[w][k][r][lane] = x.a[r * 4 + k];
+        t.m[w][4][r][lane] = x.b[r];
+    }
+}
+
+template <int NW>
+SLSTM_DEVINL void maps_store(TileMaps<NW> &t, int w, int lane, const AffP &x)
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        t.m[w][0][r][lane] = x.a01[r].x;
+        t.m[w][1][r][lane] = x.a01[r].y;
+        t.m[w][2][r][lane] = x.a23[r].x;
+        t.m[w][3][r][lane] = x.a23[r].y;
         t.m[w][4][r][lane] = x.b[r];
     }
 }

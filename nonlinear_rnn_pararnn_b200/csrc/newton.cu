@@ -265,8 +265,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         // ---- walk A ----
         // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B
         Cell Jc[L];
-        Aff agg;
-        aff_identity(agg);
+        AffP agg;
         {
             float curS[4] = {sp[0], sp[1], sp[2], sp[3]};
 #pragma unroll
@@ -292,7 +291,8 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
                 } else {
                     cell_identity(Jc[i]);
                 }
-                fold_jac(agg, Jc[i], r);
+                if (i == 0) affp_from_cell<false>(agg, Jc[0], r);
+                else fold_p<false>(agg, Jc[i], r);
             }
         }
         // second look, for a predecessor that published during walk A
