@@ -199,6 +199,16 @@ SLSTM_DEVINL void jac_mul(const Cell &J, float &x0, float &x1, float &x2, float 
     x3 = y3;
 }
 
+// y = J x + a for the sparse cell Jacobian, with a entering the innermost
+// fused multiply-add of each row.
+SLSTM_DEVINL void jac_mul_add(const Cell &J, const float x[4], const float a[4], float y[4])
+{
+    y[0] = fmaf(J.fp, x[0], fmaf(J.jcm, x[2], fmaf(J.jch, x[3], a[0])));
+    y[1] = fmaf(J.fp, x[1], fmaf(J.jnm, x[2], fmaf(J.jnh, x[3], a[1])));
+    y[2] = fmaf(J.beta, x[2], fmaf(J.dmh, x[3], a[2]));
+    y[3] = fmaf(J.jhc, x[0], fmaf(J.jhn, x[1], fmaf(J.jhm, x[2], fmaf(J.jhh, x[3], a[3]))));
+}
+
 // x <- J^T x for the sparse cell Jacobian.
 SLSTM_DEVINL void jacT_mul(const Cell &J, float &x0, float &x1, float &x2, float &x3)
 {

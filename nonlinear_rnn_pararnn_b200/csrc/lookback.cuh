@@ -219,8 +219,7 @@ SLSTM_DEVINL void tile_carry_serial(const CarryArgs &ca, float (*s_agg)[20][32],
 // A fold's running aggregate with its matrix columns paired, so that the
 // 4x4 products run on the packed fp32x2 pipe (__ffma2_rn / __fmul2_rn, two
 // lanes of the same scalar operation per instruction).  Each packed lane
-// performs exactly the scalar jac_mul / jacT_mul sequence, so the bits equal
-// those of fold_jac / fold_jacT.
+// performs exactly the scalar jac_mul / jacT_mul sequence.
 struct AffP {
     float2 a01[4];   // row r: (A[r][0], A[r][1])
     float2 a23[4];   // row r: (A[r][2], A[r][3])
@@ -286,10 +285,14 @@ SLSTM_DEVINL void fold_p(AffP &agg, const Cell &J, const float r[4])
     if (TRANS) jacT_mul_p(j, x); else jac_mul_p(j, x);
 #pragma unroll
     for (int i = 0; i < 4; ++i) agg.a23[i] = x[i];
-    if (TRANS) jacT_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
-    else jac_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
+    if (TRANS) {
+        jacT_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
+        for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
+    } else {
+        const float b[4] = {agg.b[0], agg.b[1], agg.b[2], agg.b[3]};
+        jac_mul_add(J, b, r, agg.b);
+    }
 }
 
 // The aggregate of a single step: (J, r) (TRANS: (J^T, r)).

@@ -263,34 +263,27 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         if (look) w1 = ld_relaxed_u64(predw);
 
         // ---- walk A ----
-        // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B
+        // Jc[i] keeps J_t and f(S_{t-1}, P_t) of step i for walk B.  Steps past
+        // T (only in a group's last tile) run on zero-filled rows; nothing
+        // downstream of them is stored or published.
         Cell Jc[L];
         AffP agg;
         {
             float curS[4] = {sp[0], sp[1], sp[2], sp[3]};
 #pragma unroll
             for (int i = 0; i < L; ++i) {
-                const int t = t_seg + i;
                 const int sl = warp * L + i;
-                float r[4] = {0.f, 0.f, 0.f, 0.f};
-                if (t < T) {
-                    float so[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (!FIRST) {
+                float so[4] = {0.f, 0.f, 0.f, 0.f};
+                if (!FIRST) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) so[e] = sm.S[st][sl][e][lane];
-                    }
-                    cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
-                                            sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz,
-                                            ri, rf, ro, Jc[i]);
-                    r[0] = Jc[i].c - so[0];
-                    r[1] = Jc[i].n - so[1];
-                    r[2] = Jc[i].m - so[2];
-                    r[3] = Jc[i].h - so[3];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) curS[e] = so[e];
-                } else {
-                    cell_identity(Jc[i]);
+                    for (int e = 0; e < 4; ++e) so[e] = sm.S[st][sl][e][lane];
                 }
+                cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
+                                        sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
+                                        rf, ro, Jc[i]);
+                const float r[4] = {Jc[i].c - so[0], Jc[i].n - so[1], Jc[i].m - so[2], Jc[i].h - so[3]};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) curS[e] = so[e];
                 if (i == 0) affp_from_cell<false>(agg, Jc[0], r);
                 else fold_p<false>(agg, Jc[i], r);
             }
@@ -327,43 +320,42 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         float snp[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
-        // row pointer of this lane's first step; lanes past d write nothing
+        // row pointer of this lane's first step; lanes past d and steps past T
+        // write nothing
         float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
-            const int t = t_seg + i;
             const int sl = warp * L + i;
-            if (t < T) {
-                jac_mul(Jc[i], dl[0], dl[1], dl[2], dl[3]);
-                const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
-                float sn[4];
+            const bool wr = jv && (t_seg + i < T);
+            // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
+            const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
+            float sn[4];
+            jac_mul_add(Jc[i], dl, f4, sn);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
+                dl[e] = sn[e] - so;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+            if (RESID) {
+                Cell f;
+                cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
+                                         sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
+                                         rf, ro, f);
+                const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
-                    dl[e] += f4[e] - so;   // delta_t = J_t delta_{t-1} + (f_t - S_t)
-                    sn[e] = so + dl[e];
+                    const float af = wr ? fabsf(F[e]) : 0.0f;
+                    const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
+                    // keep NaN: a NaN compares false, so test "not <="
+                    mx_raw = (af <= mx_raw) ? mx_raw : af;
+                    mx_sc = (sc <= mx_sc) ? mx_sc : sc;
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (jv) srow[(size_t)i * 4 * d + e * d] = sn[e];
-                if (RESID) {
-                    Cell f;
-                    cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
-                                             sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz,
-                                             ri, rf, ro, f);
-                    const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float af = jv ? fabsf(F[e]) : 0.0f;
-                        const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
-                        // keep NaN: a NaN compares false, so test "not <="
-                        mx_raw = (af <= mx_raw) ? mx_raw : af;
-                        mx_sc = (sc <= mx_sc) ? mx_sc : sc;
-                    }
-                }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) snp[e] = sn[e];
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) snp[e] = sn[e];
         }
         // state at the tile's last step, for the next launch's successor tile
         if (warp == NW - 1 && t_seg + L - 1 < T) {
