@@ -15,12 +15,10 @@
 // No multicast and no clusters.  Every mbarrier wait is bounded in time; on
 // expiry the CTA records an error, waits (bounded) for the loads it issued,
 // frees its TMEM and returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
-#include "common.cuh"
 #include "launchers.h"
+#include "tma.cuh"
 
 namespace slstm {
 namespace {
@@ -42,53 +40,6 @@ struct TcArgs {
     long long c_split;      // element offset between the C slices of the splits
     unsigned *error;
 };
-
-SLSTM_DEVINL uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-SLSTM_DEVINL void mbar_init(uint64_t *bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-SLSTM_DEVINL void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-}
-
-SLSTM_DEVINL bool mbar_try_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n"
-        " .reg .pred p;\n"
-        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n"
-        "}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0u;
-}
-
-// Wait for the phase of `bar` with the given parity to complete; false when
-// the time bound passes first.
-SLSTM_DEVINL bool mbar_wait(uint64_t *bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer_ns() - t0 > WAIT_NS) return false;
-    return true;
-}
-
-SLSTM_DEVINL void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-        : "memory");
-}
 
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
 // 128-byte swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart.
@@ -199,7 +150,7 @@ __global__ void __launch_bounds__(128, 1)
             mbar_init(&empty[s], 1);
         }
         mbar_init(accf, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
         s_abort = 0;
         s_issued = 0;
         s_consumed = 0;
@@ -221,7 +172,7 @@ __global__ void __launch_bounds__(128, 1)
         for (; kb < nkb; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (!mbar_wait(&empty[s], ph ^ 1u) || *(volatile int *)&s_abort) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, WAIT_NS) || *(volatile int *)&s_abort) {
                 s_abort = 1;
                 break;
             }
@@ -253,7 +204,7 @@ __global__ void __launch_bounds__(128, 1)
         for (; kb < nkb; ++kb) {
             const int s = kb % STAGES;
             const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (!mbar_wait(&full[s], ph) || *(volatile int *)&s_abort) {
+            if (!mbar_wait(&full[s], ph, WAIT_NS) || *(volatile int *)&s_abort) {
                 s_abort = 1;
                 break;
             }
@@ -276,7 +227,7 @@ __global__ void __launch_bounds__(128, 1)
     }
 
     // ---- epilogue: all four warps ----
-    const bool acc_ready = mbar_wait(accf, 0u);
+    const bool acc_ready = mbar_wait(accf, 0u, WAIT_NS);
     tc_fence_after();
     __syncthreads();
     const bool ok = acc_ready && !s_abort;
@@ -317,7 +268,7 @@ __global__ void __launch_bounds__(128, 1)
         // loads issued but never consumed still land in this CTA's shared
         // memory: wait for them (bounded) before the CTA exits
         for (int kb = s_consumed; kb < s_issued; ++kb)
-            (void)mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u);
+            (void)mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u, WAIT_NS);
     }
     __syncthreads();
     if (warp == 0) {
@@ -326,26 +277,13 @@ __global__ void __launch_bounds__(128, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 // 2-D bf16 tensor of `rows` rows of `cols` contiguous elements (row stride
 // ld elements), box of 64 contiguous elements x box_rows rows, 128-byte
 // swizzle.  K-major operands: cols = K, rows = M or N.  MN-major operands:
 // cols = M or N, rows = K.
 bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int ld, int box_rows)
 {
-    auto fn = encode_fn();
+    auto fn = tensor_map_encoder();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)ld * 2};

@@ -26,9 +26,11 @@
 // tile (the state just before it) comes from a per-tile boundary buffer
 // written by the previous launch.
 #include <float.h>
+#include <string.h>
 
 #include "launchers.h"
 #include "lookback.cuh"
+#include "tma.cuh"
 
 namespace slstm {
 namespace {
@@ -67,13 +69,33 @@ struct TileInfo {
 };
 
 struct Smem {
-    float P[2][TT][4][32];
+    float P[2][TT][4][32];   // stage s: rows (step, slot) of 32 features; TMA boxes land here
     float S[2][TT][4][32];
     TileMaps<NW> maps;
     TileInfo info[3];   // ring: current, next and the one after
+    uint64_t bar[2];    // TMA completion, one per stage
     float red[2][NW];
     int exit_flag;
 };
+constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + room to align the stages to 1 KB
+constexpr int TMA_THREAD = (NW - 1) * 32;            // issues the tile loads (warp NW-1 carries no chain lane)
+constexpr uint64_t TMA_WAIT_NS = 1000000000ull;
+
+// Tensor maps of P and S viewed as (d, 4T, B): boxes of 32 features x 128
+// (step, slot) rows for the tile loads, 32 x 16 rows for a warp's stores.
+struct NewtonMaps {
+    CUtensorMap P, S, Sw;
+};
+
+// TMA_THREAD only: start the loads of one tile into stage `st`.
+SLSTM_DEVINL void issue_tile_load(const Args &a, const NewtonMaps &m, Smem &sm, int st, const TileInfo &ti, bool with_s)
+{
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const int row = ti.chunk * TT * 4;
+    mbar_expect_tx(&sm.bar[st], (with_s ? 2u : 1u) * (uint32_t)sizeof(sm.P[0]));
+    tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, row, ti.b);
+    if (with_s) tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, row, ti.b);
+}
 
 SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
 {
@@ -181,11 +203,14 @@ __device__ void finalize(const Args &a, int k, bool resid)
     if (done) atomicExch(&c->done, 1u);
 }
 
-template <int FORGET, bool FIRST, bool RESID>
-__global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
+// TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
+// stage, stores per warp from the stage walk B wrote); otherwise by cp.async
+// and plain stores.
+template <int FORGET, bool FIRST, bool RESID, bool TMA>
+__global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
-    extern __shared__ float4 smem_f4[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_f4);
+    extern __shared__ unsigned char smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     NewtonSlot &slot = a.ctrl->slot[k & 1];
@@ -196,6 +221,11 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[0]);
             decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[1]);
         }
+    }
+    if (TMA && threadIdx.x == TMA_THREAD) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        mbar_init_fence();
     }
     __syncthreads();
     if (sm.exit_flag) return;
@@ -208,8 +238,14 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
     float mx_raw = 0.f, mx_sc = 0.f;
 
     int ring = 0, st = 0;
-    prefetch_tile(a, sm, 0, sm.info[0], toff, !FIRST);
-    cp_async_commit();
+    unsigned it = 0;       // tiles done by this CTA; stage it & 1, TMA phase (it >> 1) & 1
+    bool tma_ok = true;    // false after a TMA wait expired: no further waits
+    if (TMA) {
+        if (threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, 0, sm.info[0], !FIRST);
+    } else {
+        prefetch_tile(a, sm, 0, sm.info[0], toff, !FIRST);
+        cp_async_commit();
+    }
 
     for (;;) {
         const TileInfo ti = sm.info[ring];
@@ -219,10 +255,20 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         // decode it into the ring at the end of this tile
         unsigned after = 0;
         if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
-        prefetch_tile(a, sm, st ^ 1, sm.info[rn], toff, !FIRST);
-        cp_async_commit();
-        cp_async_wait_prev();   // the current tile's copies have landed
-        __syncthreads();
+        if (TMA) {
+            // the current tile's boxes have landed (the next tile's loads
+            // start after walk A, once this stage's old stores are read out)
+            if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS)) {
+                atomicOr(a.error, 2u);
+                (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS);
+                tma_ok = false;
+            }
+        } else {
+            prefetch_tile(a, sm, st ^ 1, sm.info[rn], toff, !FIRST);
+            cp_async_commit();
+            cp_async_wait_prev();   // the current tile's copies have landed
+            __syncthreads();
+        }
 
         const unsigned ticket = ti.ticket;
         const int chunk = ti.chunk;
@@ -292,6 +338,9 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         unsigned long long w2 = 0ull;
         if (look) w2 = ld_relaxed_u64(predw);
         maps_store(sm.maps, warp, lane, agg);
+        // this warp's stores of the previous tile have been read out of the
+        // other stage, which the next tile's loads overwrite after the barrier
+        if (TMA && lane == 0) bulk_wait_read_all();
 
         // ---- carry ----
         float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
@@ -302,7 +351,9 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
             c = __uint_as_float((unsigned)(ok1 ? w1 : w2));
         }
         const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
-        if (__syncthreads_and(ok)) {
+        const bool fast = __syncthreads_and(ok);
+        if (TMA && threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st ^ 1, sm.info[rn], !FIRST);
+        if (fast) {
             if (chain_warp) {
                 c = carry_chain4(sm.maps, c, warp, lane);
                 if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
@@ -336,9 +387,16 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
                 const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
                 dl[e] = sn[e] - so;
             }
+            if (TMA) {
+                // in place over S_old in the stage; rows past T and features
+                // past d fall outside the tensor and are not stored
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+                for (int e = 0; e < 4; ++e) sm.S[st][sl][e][lane] = sn[e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+            }
             if (RESID) {
                 Cell f;
                 cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
@@ -357,6 +415,14 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
 #pragma unroll
             for (int e = 0; e < 4; ++e) snp[e] = sn[e];
         }
+        if (TMA) {
+            tma_store_fence();
+            __syncwarp();
+            if (lane == 0 && t_seg < T) {
+                tma_store_3d(&maps.Sw, &sm.S[st][warp * L][0][0], ti.j0, t_seg * 4, ti.b);
+                bulk_commit();
+            }
+        }
         // state at the tile's last step, for the next launch's successor tile
         if (warp == NW - 1 && t_seg + L - 1 < T) {
             float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
@@ -368,8 +434,13 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
         __syncthreads();   // stage `st`, the maps and the oldest ring entry are free again
         ring = rn;
         st ^= 1;
+        ++it;
     }
-    cp_async_wait_all();
+    if (TMA) {
+        if (lane == 0) bulk_wait_all();
+    } else {
+        cp_async_wait_all();
+    }
 
     if (RESID) {
         mx_raw = warp_max(mx_raw);
@@ -399,25 +470,25 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k)
     }
 }
 
-template <int FORGET, bool FIRST, bool RESID>
-cudaError_t launch_one(const Args &a, int k, int sms, cudaStream_t st)
+template <int FORGET, bool FIRST, bool RESID, bool TMA>
+cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = newton_iter<FORGET, FIRST, RESID>;
+    auto kern = newton_iter<FORGET, FIRST, RESID, TMA>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem));
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, sizeof(Smem));
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (blocks_per_sm < 1) blocks_per_sm = 1;
     }
     const int grid = min(a.n_tiles, sms * blocks_per_sm);
-    kern<<<grid, NW * 32, sizeof(Smem), st>>>(a, k);
+    kern<<<grid, NW * 32, SMEM_BYTES, st>>>(a, k, m);
     return cudaGetLastError();
 }
 
-template <int FORGET>
-cudaError_t launch_iters(const Args &base, int max_iters, bool fixed, int sms, cudaStream_t st)
+template <int FORGET, bool TMA>
+cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, int sms, cudaStream_t st)
 {
     for (int k = 0; k < max_iters; ++k) {
         Args a = base;
@@ -427,9 +498,11 @@ cudaError_t launch_iters(const Args &base, int max_iters, bool fixed, int sms, c
         const bool resid = !fixed || (k + 1 == max_iters);
         cudaError_t e;
         if (k == 0)
-            e = resid ? launch_one<FORGET, true, true>(a, k, sms, st) : launch_one<FORGET, true, false>(a, k, sms, st);
+            e = resid ? launch_one<FORGET, true, true, TMA>(a, m, k, sms, st)
+                      : launch_one<FORGET, true, false, TMA>(a, m, k, sms, st);
         else
-            e = resid ? launch_one<FORGET, false, true>(a, k, sms, st) : launch_one<FORGET, false, false>(a, k, sms, st);
+            e = resid ? launch_one<FORGET, false, true, TMA>(a, m, k, sms, st)
+                      : launch_one<FORGET, false, false, TMA>(a, m, k, sms, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -521,8 +594,20 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(slstm_newton_stats), st);
     if (e != cudaSuccess) return e;
     const int sms = sm_count();
-    if (cfg.forget == SLSTM_FORGET_EXP) return launch_iters<SLSTM_FORGET_EXP>(a, cfg.max_iters, a.fixed, sms, st);
-    return launch_iters<SLSTM_FORGET_SIGMOID>(a, cfg.max_iters, a.fixed, sms, st);
+    // TMA moves the tiles when the rows are 16-byte aligned and every row
+    // coordinate fits a signed 32-bit box coordinate
+    NewtonMaps m;
+    memset(&m, 0, sizeof(m));
+    const uint64_t rows = 4 * (uint64_t)T, bstride = rows * (uint64_t)d;
+    const bool tma = a.vec16 && rows < (1ull << 31) &&
+                     make_map_f32_3d(&m.P, P, d, rows, B, d, bstride, 32, TT * 4) &&
+                     make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
+                     make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);
+    if (cfg.forget == SLSTM_FORGET_EXP)
+        return tma ? launch_iters<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, sms, st)
+                   : launch_iters<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, sms, st);
+    return tma ? launch_iters<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, sms, st)
+               : launch_iters<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, sms, st);
 }
 
 }  // namespace slstm
