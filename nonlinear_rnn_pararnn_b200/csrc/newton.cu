@@ -71,6 +71,8 @@ struct TileInfo {
 struct Smem {
     float P[2][TT][4][32];   // stage s: rows (step, slot) of 32 features; TMA boxes land here
     float S[2][TT][4][32];
+    float R[2][4][32];     // TMA path: the tile's recurrent weights (gate-major)
+    float bnd[2][4][32];   // TMA path: S_old just before the tile (previous launch's boundary)
     TileMaps<NW> maps;
     TileInfo info[3];   // ring: current, next and the one after
     uint64_t bar[2];    // TMA completion, one per stage
@@ -87,14 +89,24 @@ struct NewtonMaps {
     CUtensorMap P, S, Sw;
 };
 
-// TMA_THREAD only: start the loads of one tile into stage `st`.
+// TMA_THREAD only: start the loads of one tile into stage `st`: the P (and
+// S_old) boxes, the R entries of its features and, after the first launch,
+// the boundary state before it, all counted on the stage's mbarrier.
 SLSTM_DEVINL void issue_tile_load(const Args &a, const NewtonMaps &m, Smem &sm, int st, const TileInfo &ti, bool with_s)
 {
     if (ti.ticket >= (unsigned)a.n_tiles) return;
     const int row = ti.chunk * TT * 4;
-    mbar_expect_tx(&sm.bar[st], (with_s ? 2u : 1u) * (uint32_t)sizeof(sm.P[0]));
+    const uint32_t rbytes = 4u * (uint32_t)min(32, a.d - ti.j0);   // a multiple of 16 (d % 4 == 0)
+    const bool bnd = with_s && ti.chunk > 0;
+    mbar_expect_tx(&sm.bar[st], (with_s ? 2u : 1u) * (uint32_t)sizeof(sm.P[0]) + 4u * rbytes +
+                                    (bnd ? (uint32_t)sizeof(sm.bnd[0]) : 0u));
     tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, row, ti.b);
     if (with_s) tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, row, ti.b);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    if (bnd)
+        bulk_load(&sm.bnd[st][0][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32,
+                  (uint32_t)sizeof(sm.bnd[0]), &sm.bar[st]);
 }
 
 SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
@@ -277,7 +289,14 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         const int t_seg = chunk * TT + warp * L;
 
         float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-        if (jv) {
+        if (TMA) {
+            if (jv) {
+                rz = sm.R[st][0][lane];
+                ri = sm.R[st][1][lane];
+                rf = sm.R[st][2][lane];
+                ro = sm.R[st][3][lane];
+            }
+        } else if (jv) {
             rz = __ldg(a.R + jj);
             ri = __ldg(a.R + d + jj);
             rf = __ldg(a.R + 2 * d + jj);
@@ -292,9 +311,14 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             }
         } else if (!FIRST) {
             if (warp == 0) {
-                const float *src = a.bnd_in + (size_t)(ticket - G) * 4 * 32;
+                if (TMA) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
+                    for (int e = 0; e < 4; ++e) sp[e] = sm.bnd[st][e][lane];
+                } else {
+                    const float *src = a.bnd_in + (size_t)(ticket - G) * 4 * 32;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
+                }
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sp[e] = sm.S[st][warp * L - 1][e][lane];
@@ -338,6 +362,8 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         unsigned long long w2 = 0ull;
         if (look) w2 = ld_relaxed_u64(predw);
         maps_store(sm.maps, warp, lane, agg);
+        // the tile after the next one, visible to all after the vote barrier
+        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
         // this warp's stores of the previous tile have been read out of the
         // other stage, which the next tile's loads overwrite after the barrier
         if (TMA && lane == 0) bulk_wait_read_all();
@@ -430,8 +456,11 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
         }
 
-        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
-        __syncthreads();   // stage `st`, the maps and the oldest ring entry are free again
+        // TMA: no barrier here.  The next tile's loads go to the other stage,
+        // and the vote barrier after its walk A orders every warp's walk B
+        // here before the stage, the maps or the carries are written again.
+        // The cp.async path prefetches at the top of the tile and needs one.
+        if (!TMA) __syncthreads();
         ring = rn;
         st ^= 1;
         ++it;
@@ -599,7 +628,7 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     NewtonMaps m;
     memset(&m, 0, sizeof(m));
     const uint64_t rows = 4 * (uint64_t)T, bstride = rows * (uint64_t)d;
-    const bool tma = a.vec16 && rows < (1ull << 31) &&
+    const bool tma = a.vec16 && (reinterpret_cast<uintptr_t>(R) & 15) == 0 && rows < (1ull << 31) &&
                      make_map_f32_3d(&m.P, P, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);

@@ -71,6 +71,15 @@ SLSTM_DEVINL void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, 
         : "memory");
 }
 
+// Contiguous bulk copy global -> shared; size, src and dst multiples of 16 bytes.
+SLSTM_DEVINL void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // Store a box from shared memory; elements outside the tensor are not
 // written.  The caller makes its shared-memory writes visible first
 // (tma_store_fence by every writing thread, then a barrier or __syncwarp).
