@@ -325,11 +325,12 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             }
         }
 
-        // first look at the predecessor's inclusive prefix (chain lanes); the
-        // load's latency is hidden behind walk A
+        // looks at the predecessor's inclusive prefix (chain lanes): before
+        // and halfway through walk A, so that both loads' latency is hidden;
+        // the second is read only when the first found nothing
         const bool look = chain_warp && chunk > 0;
         const unsigned long long *predw = a.incw + chain_word(ticket - G, warp, lane);
-        unsigned long long w1 = 0ull;
+        unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
 
         // ---- walk A ----
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             float curS[4] = {sp[0], sp[1], sp[2], sp[3]};
 #pragma unroll
             for (int i = 0; i < L; ++i) {
+                if (i == L / 2 && look) w2 = ld_relaxed_u64(predw);
                 const int sl = warp * L + i;
                 float so[4] = {0.f, 0.f, 0.f, 0.f};
                 if (!FIRST) {
@@ -358,9 +360,6 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
                 else fold_p<false>(agg, Jc[i], r);
             }
         }
-        // second look, for a predecessor that published during walk A
-        unsigned long long w2 = 0ull;
-        if (look) w2 = ld_relaxed_u64(predw);
         maps_store(sm.maps, warp, lane, agg);
         // the tile after the next one, visible to all after the vote barrier
         if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
@@ -372,9 +371,12 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
         bool ok = true;
         if (look) {
-            const bool ok1 = (unsigned)(w1 >> 32) == a.epoch;
-            ok = ok1 || (unsigned)(w2 >> 32) == a.epoch;
-            c = __uint_as_float((unsigned)(ok1 ? w1 : w2));
+            if ((unsigned)(w1 >> 32) == a.epoch) {
+                c = __uint_as_float((unsigned)w1);
+            } else {
+                ok = (unsigned)(w2 >> 32) == a.epoch;
+                c = __uint_as_float((unsigned)w2);
+            }
         }
         const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
         const bool fast = __syncthreads_and(ok);
