@@ -9,9 +9,11 @@
 //   ds0      = J_0^T lambda_0
 // then dx = dP W_x and dW_x = dP^T x.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "launchers.h"
 #include "lookback.cuh"
+#include "tma.cuh"
 
 namespace slstm {
 namespace {
@@ -19,6 +21,7 @@ namespace {
 constexpr int NW = 8;
 constexpr int L = 4;
 constexpr int TT = NW * L;
+constexpr int DPT_LD = 36;   // bf16 row stride of the dP staging: 8-byte rows, conflict-free 8-byte stores
 
 struct BwdArgs {
     const float *P;
@@ -35,44 +38,72 @@ struct BwdArgs {
     float *ds0;       // (B, 4, d) or null
     unsigned *ticket;
     CarryArgs ca;
-    int T, d, groups_per_row, n_tiles, vec16;
+    int T, d, groups_per_row, n_tiles, vec16, dpt_vec8;
 };
 
-// Shared memory of one CTA.  A tile covers steps t in [t_lo, t_hi] with
-// t_hi = T-1-32c and t_lo = t_hi-31 (chunk c in reverse time order); it
-// needs S at t_lo-1 .. t_hi, P at t_lo .. t_hi+1 and dH at t_lo .. t_hi.
+// A ticket decoded once (by thread 0) for the whole CTA.  The tile covers
+// steps t in [t_lo, t_lo + 31], chunk c in reverse time order.
+struct BwdInfo {
+    unsigned ticket;
+    int chunk;
+    int b;
+    int j0;
+    int t_lo;
+    int pad[3];
+};
+
+// Shared memory of one CTA.  A tile needs S at t_lo-1 .. t_hi, P at
+// t_lo .. t_hi+1 and dH at t_lo .. t_hi (t_hi = t_lo + 31).
 struct BwdSmem {
     float S[2][TT + 1][4][32];   // row r <-> t = t_lo - 1 + r
     float P[2][TT + 1][4][32];   // row r <-> t = t_lo + r
     float dH[2][TT][32];         // row r <-> t = t_lo + r
+    float R[2][4][32];           // TMA path: the tile's recurrent weights
     union {
-        float agg[NW][20][32];
-        __nv_bfloat16 dpt[2][4][32][TT + 2];   // transposed staging of the dP pair
+        MapArr m[NW];            // warp maps, dead once the carries are known
+        struct {
+            __nv_bfloat16 dpt[2][4][32][DPT_LD];   // transposed staging of the dP pair: [part][gate][feature][t]
+            float part[NW][8][32];                 // per-warp dR, db partial sums
+        } o;
     } u;
-    float cin[NW][4][32];
-    float part[NW][8][32];
-    unsigned tick[2];
+    CinArr cin[NW];
+    BwdInfo info[3];
+    uint64_t bar[2];
+};
+constexpr size_t BWD_SMEM_BYTES = sizeof(BwdSmem) + 1024;
+constexpr int BWD_TMA_THREAD = (NW - 1) * 32;
+constexpr uint64_t BWD_TMA_WAIT_NS = 1000000000ull;
+
+// Tensor maps: S and P as (d, 4T, B) with boxes of 32 features x 132 (step,
+// slot) rows, dH as (d, T, B) with boxes of 32 x 32.
+struct BwdMaps {
+    CUtensorMap S, P, H;
 };
 
-SLSTM_DEVINL void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo)
+SLSTM_DEVINL void bwd_decode(const BwdArgs &a, unsigned ticket, BwdInfo &ti)
 {
-    hi = __float2bfloat16_rn(v);
-    lo = __float2bfloat16_rn(v - __bfloat162float(hi));
+    ti.ticket = ticket;
+    ti.chunk = ti.b = ti.j0 = ti.t_lo = 0;
+    if (ticket < (unsigned)a.n_tiles) {
+        const unsigned G = (unsigned)a.ca.n_groups;
+        const unsigned chunk = ticket / G;
+        const unsigned grp = ticket - chunk * G;
+        const unsigned b = grp / (unsigned)a.groups_per_row;
+        ti.chunk = (int)chunk;
+        ti.b = (int)b;
+        ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
+        ti.t_lo = a.T - ((int)chunk + 1) * TT;
+    }
 }
 
-// Copies of one tile's S, P and dH rows into stage `st`; rows outside [0, T)
-// and features past d arrive as zeros.
-SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, unsigned ticket)
+// cp.async path: copies of one tile's S, P and dH rows into stage `st`; rows
+// outside [0, T) and features past d arrive as zeros.
+SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdInfo &ti)
 {
-    if (ticket >= (unsigned)a.n_tiles) return;
-    const int G = a.ca.n_groups;
-    const int chunk = (int)(ticket / (unsigned)G);
-    const int grp = (int)(ticket % (unsigned)G);
-    const int b = grp / a.groups_per_row;
-    const int j0 = (grp % a.groups_per_row) * 32;
-    const int t_lo = a.T - (chunk + 1) * TT;
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const int j0 = ti.j0, t_lo = ti.t_lo;
     const size_t d = (size_t)a.d;
-    const size_t row0 = (size_t)b * a.T;
+    const size_t row0 = (size_t)ti.b * a.T;
     const int T = a.T;
     constexpr int RS = (TT + 1) * 4;           // (row, slot) pairs of S and of P
     if (a.vec16) {
@@ -85,7 +116,7 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, unsigned t
             const int rs = q + 32 * k;
             if (rs < RS) {
                 const int r = rs >> 2, slot = rs & 3;
-                const int tS = t_lo - 1 + r, tP = t_lo + r;   // S row r <-> t_lo-1+r, P row r <-> t_lo+r
+                const int tS = t_lo - 1 + r, tP = t_lo + r;
                 const int bS = (tS >= 0 && tS < T) ? fbytes : 0;
                 const int bP = (tP >= 0 && tP < T) ? fbytes : 0;
                 cp_async16(&sm.S[st][r][slot][4 * c], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
@@ -116,151 +147,223 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, unsigned t
     }
 }
 
-template <int FORGET, bool BF16OUT>
-__global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
+// TMA path, BWD_TMA_THREAD only: start the loads of one tile into stage st.
+// Boxes that start before t = 0 or end past T - 1 read zeros there.
+SLSTM_DEVINL void bwd_issue_load(const BwdArgs &a, const BwdMaps &m, BwdSmem &sm, int st, const BwdInfo &ti)
 {
-    extern __shared__ float4 smem_f4[];
-    BwdSmem &sm = *reinterpret_cast<BwdSmem *>(smem_f4);
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const uint32_t rbytes = 4u * (uint32_t)min(32, a.d - ti.j0);
+    mbar_expect_tx(&sm.bar[st], (uint32_t)(sizeof(sm.S[0]) + sizeof(sm.P[0]) + sizeof(sm.dH[0])) + 4u * rbytes);
+    tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, (ti.t_lo - 1) * 4, ti.b);
+    tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, ti.t_lo * 4, ti.b);
+    tma_load_3d(&sm.dH[st][0][0], &m.H, &sm.bar[st], ti.j0, ti.t_lo, ti.b);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+}
+
+// TMA: tiles arrive by TMA (BWD_TMA_THREAD, mbarrier per stage); otherwise by
+// cp.async.  BF16OUT: dP leaves as the transposed bf16 pair, else as fp32.
+template <int FORGET, bool BF16OUT, bool TMA>
+__global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps)
+{
+    extern __shared__ unsigned char smem_raw[];
+    BwdSmem &sm = *reinterpret_cast<BwdSmem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int G = a.ca.n_groups;
+    const unsigned G = (unsigned)a.ca.n_groups;
     const int T = a.T;
     const size_t d = (size_t)a.d;
+    const bool chain_warp = warp < 4;
 
     if (threadIdx.x == 0) {
-        sm.tick[0] = atomicAdd(a.ticket, 1u);
-        sm.tick[1] = atomicAdd(a.ticket, 1u);
+        bwd_decode(a, atomicAdd(a.ticket, 1u), sm.info[0]);
+        bwd_decode(a, atomicAdd(a.ticket, 1u), sm.info[1]);
+    }
+    if (TMA && threadIdx.x == BWD_TMA_THREAD) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        mbar_init_fence();
     }
     __syncthreads();
-    unsigned cur = sm.tick[0];
-    unsigned nxt = sm.tick[1];
-    int st = 0;
-    bwd_prefetch(a, sm, 0, cur);
-    cp_async_commit();
+    int ring = 0, st = 0;
+    unsigned it = 0;
+    bool tma_ok = true;
+    if (TMA) {
+        if (threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, 0, sm.info[0]);
+    } else {
+        bwd_prefetch(a, sm, 0, sm.info[0]);
+        cp_async_commit();
+    }
 
-    while (cur < (unsigned)a.n_tiles) {
+    for (;;) {
+        const BwdInfo ti = sm.info[ring];
+        if (ti.ticket >= (unsigned)a.n_tiles) break;
+        const int rn = ring == 2 ? 0 : ring + 1;
         unsigned after = 0;
         if (threadIdx.x == 0) after = atomicAdd(a.ticket, 1u);
-        bwd_prefetch(a, sm, st ^ 1, nxt);
-        cp_async_commit();
-        cp_async_wait_prev();
-        __syncthreads();
+        if (TMA) {
+            if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, BWD_TMA_WAIT_NS)) {
+                atomicOr(a.ca.error, 2u);
+                (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, BWD_TMA_WAIT_NS);
+                tma_ok = false;
+            }
+        } else {
+            bwd_prefetch(a, sm, st ^ 1, sm.info[rn]);
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncthreads();
+        }
 
-        const unsigned ticket = cur;
-        const int chunk = (int)(ticket / (unsigned)G);
-        const int grp = (int)(ticket % (unsigned)G);
-        const int b = grp / a.groups_per_row;
-        const int j = (grp % a.groups_per_row) * 32 + lane;
-        const bool jv = j < a.d;
-        const size_t jj = jv ? (size_t)j : 0;
-        const size_t row0 = (size_t)b * T;
-        const int t_lo = T - (chunk + 1) * TT;
+        const unsigned ticket = ti.ticket;
+        const int chunk = ti.chunk;
+        const bool jv = ti.j0 + lane < a.d;
+        const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
+        const size_t row0 = (size_t)ti.b * T;
+        const int t_lo = ti.t_lo;
 
         float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-        if (jv) {
+        if (TMA) {
+            if (jv) {
+                rz = sm.R[st][0][lane];
+                ri = sm.R[st][1][lane];
+                rf = sm.R[st][2][lane];
+                ro = sm.R[st][3][lane];
+            }
+        } else if (jv) {
             rz = __ldg(a.R + jj);
             ri = __ldg(a.R + d + jj);
             rf = __ldg(a.R + 2 * d + jj);
             ro = __ldg(a.R + 3 * d + jj);
         }
 
+        // looks at the predecessor's (later-in-time) inclusive prefix
+        const bool look = chain_warp && chunk > 0;
+        const unsigned long long *predw = a.ca.incw + chain_word(ticket - G, warp, lane);
+        unsigned long long w1 = 0ull, w2 = 0ull;
+        if (look) w1 = ld_relaxed_u64(predw);
+
         // ---- walk A: fold lambda -> J_{t+1}^T lambda + e_h dH_t, t descending ----
+        // Rows past T or before 0 are zero-filled: J_T (the step past the
+        // end) is finite and only ever meets the zero carry entering the
+        // sequence's last step; steps before 0 come last in this order and
+        // reach nothing that is stored.
         Cell Jn[L];   // J_{t+1} of each step
-        Aff agg;
-        aff_identity(agg);
+        AffP agg;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
+            if (i == L / 2 && look) w2 = ld_relaxed_u64(predw);
             const int rl = TT - 1 - (warp * L + i);   // t - t_lo
-            const int t = t_lo + rl;
-            cell_identity(Jn[i]);
-            float r[4] = {0.f, 0.f, 0.f, 0.f};
-            if (t >= 0) {
-                r[3] = sm.dH[st][rl][lane];
-                if (t + 1 < T)
-                    cell_eval<FORGET, true>(sm.S[st][rl + 1][0][lane], sm.S[st][rl + 1][1][lane],
-                                            sm.S[st][rl + 1][2][lane], sm.S[st][rl + 1][3][lane],
-                                            sm.P[st][rl + 1][0][lane], sm.P[st][rl + 1][1][lane],
-                                            sm.P[st][rl + 1][2][lane], sm.P[st][rl + 1][3][lane], rz, ri, rf, ro, Jn[i]);
+            cell_eval<FORGET, true>(sm.S[st][rl + 1][0][lane], sm.S[st][rl + 1][1][lane], sm.S[st][rl + 1][2][lane],
+                                    sm.S[st][rl + 1][3][lane], sm.P[st][rl + 1][0][lane], sm.P[st][rl + 1][1][lane],
+                                    sm.P[st][rl + 1][2][lane], sm.P[st][rl + 1][3][lane], rz, ri, rf, ro, Jn[i]);
+            const float r[4] = {0.f, 0.f, 0.f, sm.dH[st][rl][lane]};
+            if (i == 0) affp_from_cell<true>(agg, Jn[0], r);
+            else fold_p<true>(agg, Jn[i], r);
+        }
+        maps_store(sm.u.m, warp, lane, agg);
+        if (threadIdx.x == 0) bwd_decode(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
+
+        // ---- carry ----
+        float c = 0.f;   // chunk 0: nothing enters after the sequence's last step
+        bool ok = true;
+        if (look) {
+            if ((unsigned)(w1 >> 32) == a.ca.epoch) {
+                c = __uint_as_float((unsigned)w1);
+            } else {
+                ok = (unsigned)(w2 >> 32) == a.ca.epoch;
+                c = __uint_as_float((unsigned)w2);
             }
-            fold_jacT(agg, Jn[i], r);
         }
-        store_aff_smem(sm.u.agg, warp, lane, agg);
-        __syncthreads();
-        if (warp == 0) {
-            const float zero[4] = {0.f, 0.f, 0.f, 0.f};
-            tile_carry_serial<NW>(a.ca, sm.u.agg, sm.cin, ticket, chunk, grp, zero, false);
+        const bool fast = __syncthreads_and(ok);
+        if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
+        if (fast) {
+            if (chain_warp) {
+                c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane);
+                st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+            }
+        } else if (warp == 0) {
+            tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false);
         }
-        __syncthreads();   // sm.u.agg is dead from here on; sm.u.dpt takes its place
+        __syncthreads();   // the maps are dead from here on; the dP staging takes their place
 
         // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
         float lam[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][lane];
         float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
+        float dv[L][4];   // dP of the thread's steps (gate order z, i, f, o)
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int rl = TT - 1 - (warp * L + i);
             const int t = t_lo + rl;
-            if (t >= 0) {
-                jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
-                lam[3] += sm.dH[st][rl][lane];
-                float prev[4];
-                if (t == 0) {
+            jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
+            lam[3] += sm.dH[st][rl][lane];
+            float prev[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + ((size_t)b * 4 + e) * d + jj) : 0.f;
-                } else {
+            for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
+            Cell cc;
+            CellG g;
+            if (t == 0) {
+                // the state before the sequence is s0; ds0 = J_0^T lambda_0
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
-                }
-                Cell c;
-                CellG g;
+                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj) : 0.f;
                 cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
                                               sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
-                                              ri, rf, ro, c, &g);
-                const float dz = fmaf(g.gcz, lam[0], g.ghz * lam[3]);
-                const float di = fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3])));
-                const float df = fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3])));
-                const float dq = g.gho * lam[3];
-                if (BF16OUT) {
-                    const float dv[4] = {dz, di, df, dq};
-#pragma unroll
-                    for (int gi = 0; gi < 4; ++gi) {
-                        __nv_bfloat16 hi, lo;
-                        split_bf16(dv[gi], hi, lo);
-                        sm.u.dpt[0][gi][lane][rl] = hi;
-                        sm.u.dpt[1][gi][lane][rl] = lo;
-                    }
-                } else if (jv) {
-                    float *pd = a.dP + (row0 + t) * 4 * d + jj;
-                    pd[0] = dz;
-                    pd[d] = di;
-                    pd[2 * d] = df;
-                    pd[3 * d] = dq;
-                }
-                const float hp = prev[3];
-                dr[0] = fmaf(dz, hp, dr[0]);
-                dr[1] = fmaf(di, hp, dr[1]);
-                dr[2] = fmaf(df, hp, dr[2]);
-                dr[3] = fmaf(dq, hp, dr[3]);
-                dbs[0] += dz;
-                dbs[1] += di;
-                dbs[2] += df;
-                dbs[3] += dq;
-                if (t == 0 && a.ds0 && jv) {
+                                              ri, rf, ro, cc, &g);
+                if (a.ds0 && jv) {
                     float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
-                    jacT_mul(c, v0, v1, v2, v3);
-                    float *q = a.ds0 + (size_t)b * 4 * d + jj;
+                    jacT_mul(cc, v0, v1, v2, v3);
+                    float *q = a.ds0 + (size_t)ti.b * 4 * d + jj;
                     q[0] = v0;
                     q[d] = v1;
                     q[2 * d] = v2;
                     q[3 * d] = v3;
                 }
+            } else {
+                cell_eval<FORGET, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
+                                               sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
+                                               ri, rf, ro, cc, &g);
+            }
+            const bool tv = t >= 0;   // steps before 0 (last chunk only) contribute nothing
+            dv[i][0] = tv ? fmaf(g.gcz, lam[0], g.ghz * lam[3]) : 0.f;
+            dv[i][1] = tv ? fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3]))) : 0.f;
+            dv[i][2] = tv ? fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3]))) : 0.f;
+            dv[i][3] = tv ? g.gho * lam[3] : 0.f;
+            if (!BF16OUT && jv && tv) {
+                float *pd = a.dP + (row0 + t) * 4 * d + jj;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pd[e * d] = dv[i][e];
+            }
+            const float hp = prev[3];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                dr[e] = fmaf(dv[i][e], hp, dr[e]);
+                dbs[e] += dv[i][e];
             }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            sm.part[warp][e][lane] = jv ? dr[e] : 0.f;
-            sm.part[warp][4 + e][lane] = jv ? dbs[e] : 0.f;
+            sm.u.o.part[warp][e][lane] = jv ? dr[e] : 0.f;
+            sm.u.o.part[warp][4 + e][lane] = jv ? dbs[e] : 0.f;
+        }
+        if (BF16OUT) {
+            // the thread's 4 steps are 4 consecutive t: t_lo + 28 - 4w .. t_lo + 31 - 4w
+            const int rb = TT - L - warp * L;
+#pragma unroll
+            for (int gi = 0; gi < 4; ++gi) {
+                const __nv_bfloat162 h01 = __floats2bfloat162_rn(dv[3][gi], dv[2][gi]);
+                const __nv_bfloat162 h23 = __floats2bfloat162_rn(dv[1][gi], dv[0][gi]);
+                const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+                const __nv_bfloat162 l01 = __floats2bfloat162_rn(dv[3][gi] - f01.x, dv[2][gi] - f01.y);
+                const __nv_bfloat162 l23 = __floats2bfloat162_rn(dv[1][gi] - f23.x, dv[0][gi] - f23.y);
+                uint2 hv, lv;
+                hv.x = *reinterpret_cast<const unsigned *>(&h01);
+                hv.y = *reinterpret_cast<const unsigned *>(&h23);
+                lv.x = *reinterpret_cast<const unsigned *>(&l01);
+                lv.y = *reinterpret_cast<const unsigned *>(&l23);
+                *reinterpret_cast<uint2 *>(&sm.u.o.dpt[0][gi][lane][rb]) = hv;
+                *reinterpret_cast<uint2 *>(&sm.u.o.dpt[1][gi][lane][rb]) = lv;
+            }
         }
         __syncthreads();
         {
@@ -268,31 +371,44 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a)
             const int e = threadIdx.x >> 5;   // 0..7
             float acc = 0.f;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) acc += sm.part[w][e][lane];
+            for (int w = 0; w < NW; ++w) acc += sm.u.o.part[w][e][lane];
             a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
         }
         if (BF16OUT) {
-            // rows (g, j) of the transposed pair: up to 32 consecutive steps each
-            const int tl = threadIdx.x & 31;
-            const int t = t_lo + tl;
-            const int j0 = (grp % a.groups_per_row) * 32;
-            for (int r = threadIdx.x >> 5; r < 2 * 4 * 32; r += NW) {
-                const int part = r >> 7;
-                const int gi = (r >> 5) & 3;
-                const int jl = r & 31;
-                if (t >= 0 && j0 + jl < a.d) {
-                    __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
-                    dst[((size_t)gi * d + j0 + jl) * a.ldT + row0 + t] = sm.u.dpt[part][gi][jl][tl];
+            // rows (part, gate, feature) of the transposed pair, 32 steps each;
+            // nothing before t = 0 (those addresses hold the previous batch row)
+            if (a.dpt_vec8) {
+                // 8-byte pieces of 4 steps: piece q of row r is index 8 r + q
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int idx = threadIdx.x + NW * 32 * k;
+                    const int r = idx >> 3, q = idx & 7;
+                    const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
+                    const int t = t_lo + 4 * q;
+                    if (t >= 0 && ti.j0 + jl < a.d) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
+                        __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                        *reinterpret_cast<uint2 *>(dst + ((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t) = v;
+                    }
+                }
+            } else {
+                const int tl = threadIdx.x & 31;
+                const int t = t_lo + tl;
+                for (int r = warp; r < 2 * 4 * 32; r += NW) {
+                    const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
+                    if (t >= 0 && ti.j0 + jl < a.d) {
+                        __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                        dst[((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t] = sm.u.o.dpt[part][gi][jl][tl];
+                    }
                 }
             }
         }
-        if (threadIdx.x == 0) sm.tick[0] = after;
-        __syncthreads();
-        cur = nxt;
-        nxt = sm.tick[0];
+        __syncthreads();   // the staging and the stage are free again
+        ring = rn;
         st ^= 1;
+        ++it;
     }
-    cp_async_wait_all();
+    if (!TMA) cp_async_wait_all();
 }
 
 // out[i] = sum_z part[z][i], z in order (split-K partial sums).
@@ -353,21 +469,28 @@ int sm_count_bwd()
     return n;
 }
 
-template <int FORGET, bool BF16OUT>
-cudaError_t launch_adjoint(const BwdArgs &a, cudaStream_t st)
+template <int FORGET, bool BF16OUT, bool TMA>
+cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
 {
-    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT>;
+    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT, TMA>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(BwdSmem));
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BWD_SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, sizeof(BwdSmem));
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, NW * 32, BWD_SMEM_BYTES);
         if (e != cudaSuccess) return e;
         if (blocks_per_sm < 1) blocks_per_sm = 1;
     }
     const int grid = min(a.n_tiles, sm_count_bwd() * blocks_per_sm);
-    kern<<<grid, NW * 32, sizeof(BwdSmem), st>>>(a);
+    kern<<<grid, NW * 32, BWD_SMEM_BYTES, st>>>(a, m);
     return cudaGetLastError();
+}
+
+template <int FORGET>
+cudaError_t launch_adjoint_any(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, cudaStream_t st)
+{
+    if (tma) return bf16out ? launch_adjoint<FORGET, true, true>(a, m, st) : launch_adjoint<FORGET, false, true>(a, m, st);
+    return bf16out ? launch_adjoint<FORGET, true, false>(a, m, st) : launch_adjoint<FORGET, false, false>(a, m, st);
 }
 
 struct Layout {
@@ -456,17 +579,24 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.d = d_h;
     a.groups_per_row = l.groups_per_row;
     a.n_tiles = l.n_tiles;
+    a.dpt_vec8 = (T % 4 == 0) ? 1 : 0;   // 8-byte pieces of the transposed pair stay aligned
     a.vec16 = ((d_h & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&
                (reinterpret_cast<uintptr_t>(P) & 15) == 0 && (reinterpret_cast<uintptr_t>(dH) & 15) == 0) ? 1 : 0;
     // ticket, error word, flags and the epoch tags of the inclusive prefixes
     // start cleared
     cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
     if (e != cudaSuccess) return e;
-    if (forget == SLSTM_FORGET_EXP) {
-        e = tc ? launch_adjoint<SLSTM_FORGET_EXP, true>(a, st) : launch_adjoint<SLSTM_FORGET_EXP, false>(a, st);
-    } else {
-        e = tc ? launch_adjoint<SLSTM_FORGET_SIGMOID, true>(a, st) : launch_adjoint<SLSTM_FORGET_SIGMOID, false>(a, st);
-    }
+    // TMA moves the tiles when the rows are 16-byte aligned and every row
+    // coordinate fits a signed 32-bit box coordinate
+    BwdMaps m;
+    memset(&m, 0, sizeof(m));
+    const uint64_t rows = 4 * (uint64_t)T;
+    const bool tma = a.vec16 && (reinterpret_cast<uintptr_t>(R) & 15) == 0 && rows < (1ull << 31) &&
+                     make_map_f32_3d(&m.S, S, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
+                     make_map_f32_3d(&m.P, P, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
+                     make_map_f32_3d(&m.H, dH, d_h, T, B, d_h, (uint64_t)T * d_h, 32, TT);
+    e = (forget == SLSTM_FORGET_EXP) ? launch_adjoint_any<SLSTM_FORGET_EXP>(a, m, tma, tc, st)
+                                     : launch_adjoint_any<SLSTM_FORGET_SIGMOID>(a, m, tma, tc, st);
     if (e != cudaSuccess) return e;
     reduce_partials_kernel<<<dim3(l.groups_per_row, 8), 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);

@@ -331,45 +331,47 @@ SLSTM_DEVINL void affp_to_aff(const AffP &p, Aff &x)
 // warp (8 features x 4 rows) fall in 32 distinct banks.
 constexpr int MAP_LD = 40;
 
+// Per-warp maps of a tile, [warp][column k, k = 4: offset b][row][feature],
+// and the carries entering the warps, [warp][slot][feature].
+typedef float MapArr[5][4][MAP_LD];
+typedef float CinArr[4][MAP_LD];
+
 template <int NW>
 struct TileMaps {
-    float m[NW][5][4][MAP_LD];   // [warp][column k, k = 4: offset b][row][feature]
-    float cin[NW][4][MAP_LD];    // [warp][slot][feature]: carry entering the warp's steps
+    MapArr m[NW];
+    CinArr cin[NW];
 };
 
 // Lane = feature.
-template <int NW>
-SLSTM_DEVINL void maps_store(TileMaps<NW> &t, int w, int lane, const Aff &x)
+SLSTM_DEVINL void maps_store(MapArr *m, int w, int lane, const Aff &x)
 {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) t.m[w][k][r][lane] = x.a[r * 4 + k];
-        t.m[w][4][r][lane] = x.b[r];
+        for (int k = 0; k < 4; ++k) m[w][k][r][lane] = x.a[r * 4 + k];
+        m[w][4][r][lane] = x.b[r];
     }
 }
 
-template <int NW>
-SLSTM_DEVINL void maps_store(TileMaps<NW> &t, int w, int lane, const AffP &x)
+SLSTM_DEVINL void maps_store(MapArr *m, int w, int lane, const AffP &x)
 {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        t.m[w][0][r][lane] = x.a01[r].x;
-        t.m[w][1][r][lane] = x.a01[r].y;
-        t.m[w][2][r][lane] = x.a23[r].x;
-        t.m[w][3][r][lane] = x.a23[r].y;
-        t.m[w][4][r][lane] = x.b[r];
+        m[w][0][r][lane] = x.a01[r].x;
+        m[w][1][r][lane] = x.a01[r].y;
+        m[w][2][r][lane] = x.a23[r].x;
+        m[w][3][r][lane] = x.a23[r].y;
+        m[w][4][r][lane] = x.b[r];
     }
 }
 
-template <int NW>
-SLSTM_DEVINL void maps_load(const TileMaps<NW> &t, int w, int lane, Aff &x)
+SLSTM_DEVINL void maps_load(const MapArr *m, int w, int lane, Aff &x)
 {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x.a[r * 4 + k] = t.m[w][k][r][lane];
-        x.b[r] = t.m[w][4][r][lane];
+        for (int k = 0; k < 4; ++k) x.a[r * 4 + k] = m[w][k][r][lane];
+        x.b[r] = m[w][4][r][lane];
     }
 }
 
@@ -384,24 +386,24 @@ SLSTM_DEVINL size_t chain_word(unsigned tq, int warp, int lane)
 }
 
 // Chain warps only.  c: this lane's component of the carry entering the
-// tile.  Stores the carry entering every warp in t.cin and returns this
+// tile.  Stores the carry entering every warp in cin and returns this
 // lane's component of the tile's inclusive prefix.  The arithmetic (order of
 // the fused multiply-adds) is that of aff_apply, so both walks give the same
 // bits.
 template <int NW>
-SLSTM_DEVINL float carry_chain4(TileMaps<NW> &t, float c, int warp, int lane)
+SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane)
 {
     const int f = chain_feature(warp, lane);
     const int r = chain_row(lane);
     const int i8 = lane & 7;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-        t.cin[w][r][f] = c;
-        const float a0 = t.m[w][0][r][f];
-        const float a1 = t.m[w][1][r][f];
-        const float a2 = t.m[w][2][r][f];
-        const float a3 = t.m[w][3][r][f];
-        const float bb = t.m[w][4][r][f];
+        cin[w][r][f] = c;
+        const float a0 = m[w][0][r][f];
+        const float a1 = m[w][1][r][f];
+        const float a2 = m[w][2][r][f];
+        const float a3 = m[w][3][r][f];
+        const float bb = m[w][4][r][f];
         const float v0 = __shfl_sync(0xffffffffu, c, i8);
         const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
         const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
@@ -415,11 +417,11 @@ SLSTM_DEVINL float carry_chain4(TileMaps<NW> &t, float c, int warp, int lane)
 // predecessor prefix: reads it again, else looks back; then walks the maps
 // serially (lane = feature).  chunk > 0.
 template <int NW>
-SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, TileMaps<NW> &t, unsigned ticket, int chunk, int grp,
-                                      bool withhold)
+SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, const MapArr *m, CinArr *cin, unsigned ticket, int chunk,
+                                      int grp, bool withhold)
 {
     const int lane = threadIdx.x & 31;
-    auto load = [&](int w, Aff &x) { maps_load(t, w, lane, x); };
+    auto load = [&](int w, Aff &x) { maps_load(m, w, lane, x); };
     float carry[4];
     const bool ok = read_inc_words(ca, ticket - (unsigned)ca.n_groups, lane, carry);
     if (!__all_sync(0xffffffffu, ok)) tile_lookback<NW>(ca, load, ticket, chunk, grp, withhold, carry);
@@ -427,7 +429,7 @@ SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, TileMaps<NW> &t, unsi
         ca, load,
         [&](int w, const float v[4]) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) t.cin[w][e][lane] = v[e];
+            for (int e = 0; e < 4; ++e) cin[w][e][lane] = v[e];
         },
         ticket, withhold, carry);
 }

@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
                 else fold_p<false>(agg, Jc[i], r);
             }
         }
-        maps_store(sm.maps, warp, lane, agg);
+        maps_store(sm.maps.m, warp, lane, agg);
         // the tile after the next one, visible to all after the vote barrier
         if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
         // this warp's stores of the previous tile have been read out of the
@@ -383,12 +383,12 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         if (TMA && threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st ^ 1, sm.info[rn], !FIRST);
         if (fast) {
             if (chain_warp) {
-                c = carry_chain4(sm.maps, c, warp, lane);
+                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane);
                 if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
             }
         } else if (warp == 0) {
             const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-            tile_carry_fallback<NW>(ca, sm.maps, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold);
+            tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold);
         }
         __syncthreads();
 
