@@ -4,18 +4,22 @@
 // (b,t)), B = W_x (rows (g,j)) ("sLSTM in this library", section "API
 // notes": W_x is a GEMM).
 //
-// One CTA computes a 128 x 256 tile of C:
+// Persistent CTAs (one per SM) walk 128 x 256 tiles of C (and split-K
+// slices), n fastest so that the A rows of a tile row are reused from L2:
 //   warp 0, one lane   TMA producer: A and B k-blocks (64 wide, 128-byte
 //                      swizzle) into a 4-stage ring guarded by mbarriers;
-//   warp 1, one lane   MMA issuer: tcgen05.mma (M=128, N=256, K=16) into a
-//                      256-column fp32 accumulator in TMEM; tcgen05.commit
-//                      frees each stage and finally signals the epilogue;
-//   all 4 warps        epilogue: tcgen05.ld of their 32 TMEM lanes, + bias,
-//                      fp32 stores.
+//   warp 1, one lane   MMA issuer: tcgen05.mma (M=128, N=256, K=16) into one
+//                      of two 256-column fp32 accumulators in TMEM, so that a
+//                      tile's epilogue overlaps the next tile's main loop;
+//   warps 2-5          epilogue: tcgen05.ld of their TMEM lane quarter, + bias,
+//                      32-column slices staged in shared memory and written
+//                      by TMA stores (plain stores when C rows are not
+//                      16-byte aligned).
 // No multicast and no clusters.  Every mbarrier wait is bounded in time; on
-// expiry the CTA records an error, waits (bounded) for the loads it issued,
-// frees its TMEM and returns.
+// expiry the CTA records an error, waits (bounded) for the loads and MMAs it
+// issued, frees its TMEM and returns.
 #include <cuda_bf16.h>
+#include <string.h>
 
 #include "launchers.h"
 #include "tma.cuh"
@@ -27,8 +31,11 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr uint32_t A_STAGE = BM * BK * 2;   // 16 KB
 constexpr uint32_t B_STAGE = BN * BK * 2;   // 32 KB
 constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;
-constexpr uint32_t TMEM_COLS = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+constexpr uint32_t TMEM_COLS = 2 * BN;      // two accumulators: one tile's epilogue overlaps the next one's MMAs
+constexpr int EPI_COLS = 32;                // columns per epilogue store box (128 bytes of fp32)
+constexpr uint32_t EPI_BYTES = BM * EPI_COLS * 4;   // 16 KB, two of them
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * EPI_BYTES + 1024 + 256;
+constexpr int THREADS = 192;                // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint64_t WAIT_NS = 1000000000ull;   // 1 s bound on any single wait
 
 struct TcArgs {
@@ -37,9 +44,31 @@ struct TcArgs {
     int M, N, K;
     int a_parts;            // 1, or 2: C = (A0 + A1) B^T with A1 from the second map
     int kb_per_split;       // k-blocks of the virtual K (a_parts * ceil(K/64)) per split
+    int m_tiles, n_tiles, n_work;   // work item w = (split, m tile, n tile), n fastest
+    int tma_out;            // the epilogue stores through the C tensor map
     long long c_split;      // element offset between the C slices of the splits
     unsigned *error;
 };
+
+// Named barrier with an OR reduction over `n` threads: every participant
+// gets the same answer.
+SLSTM_DEVINL bool bar_or(int id, int n, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n"
+        " .reg .pred p, q;\n"
+        " setp.ne.u32 p, %1, 0;\n"
+        " bar.red.or.pred q, %2, %3, p;\n"
+        " selp.u32 %0, 1, 0, q;\n"
+        "}\n"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(n)
+        : "memory");
+    return r != 0u;
+}
+
+SLSTM_DEVINL void bar_named(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // Shared-memory matrix descriptor of a K-major bf16 tile written by TMA with
 // 128-byte swizzle: rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart.
@@ -118,38 +147,50 @@ SLSTM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
 
 // A_MN / B_MN: the operand is stored MN-major ([K][M] or [K][N], MN
 // contiguous) instead of K-major; its tile is then loaded as 64-wide boxes.
+//
+// Persistent: CTA c takes work items c, c + gridDim.x, ...  Roles:
+//   warp 0, one lane   TMA producer over every item's k-blocks (4-stage ring);
+//   warp 1, one lane   MMA issuer; item i accumulates in TMEM columns
+//                      [256 (i & 1), 256 (i & 1) + 256), handed to the
+//                      epilogue by tcgen05.commit and back by an mbarrier;
+//   warps 2-5          epilogue: TMEM lane quarter (warp & 3), + bias, then
+//                      32-column slices staged in shared memory (128-byte
+//                      swizzle) and written by TMA stores, two staging buffers.
 template <bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tma2,
-                   const __grid_constant__ CUtensorMap tmb, TcArgs g)
+                   const __grid_constant__ CUtensorMap tmb, const __grid_constant__ CUtensorMap tmc, TcArgs g)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * A_STAGE;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    uint8_t *sE = smem + STAGES * STAGE_BYTES;   // 1024-aligned: the swizzle pattern is address based
+    uint64_t *full = reinterpret_cast<uint64_t *>(sE + 2 * EPI_BYTES);
     uint64_t *empty = full + STAGES;
-    uint64_t *accf = empty + STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accf + 1);
+    uint64_t *tfull = empty + STAGES;    // [2] accumulator ready
+    uint64_t *tempty = tfull + 2;        // [2] accumulator drained (4 epilogue warps)
+    uint64_t *fin = tempty + 2;          // every MMA issued has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(fin + 1);
     __shared__ int s_abort;
     __shared__ int s_issued, s_consumed;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM;
-    const int n0 = blockIdx.x * BN;
-    // this CTA's k-blocks: [kb0, kb0 + nkb) of the virtual K that runs over
-    // the a_parts operand parts one after the other
     const int nk_part = (g.K + BK - 1) / BK;
-    const int kb0 = blockIdx.z * g.kb_per_split;
-    const int nkb = min(g.kb_per_split, g.a_parts * nk_part - kb0);
+    const int total_kb = g.a_parts * nk_part;
+    const int per_split = g.m_tiles * g.n_tiles;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(accf, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(fin, 1);
         mbar_init_fence();
         s_abort = 0;
         s_issued = 0;
@@ -166,110 +207,162 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0 && lane == 0) {
-        // ---- TMA producer ----
-        int kb = 0;
-        for (; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (!mbar_wait(&empty[s], ph ^ 1u, WAIT_NS) || *(volatile int *)&s_abort) {
-                s_abort = 1;
-                break;
-            }
-            const int vk = kb0 + kb;
-            const int part = vk / nk_part;
-            const int kk = vk - part * nk_part;
-            mbar_expect_tx(&full[s], STAGE_BYTES);
-            const CUtensorMap *am = part ? &tma2 : &tma;
-            if (A_MN) {
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---- TMA producer ----
+            int gkb = 0;
+            bool stop = false;
+            for (int w = blockIdx.x; w < g.n_work && !stop; w += gridDim.x) {
+                const int z = w / per_split;
+                const int r = w - z * per_split;
+                const int m0 = (r / g.n_tiles) * BM, n0 = (r % g.n_tiles) * BN;
+                const int kb0 = z * g.kb_per_split;
+                const int nkb = min(g.kb_per_split, total_kb - kb0);
+                for (int kb = 0; kb < nkb; ++kb, ++gkb) {
+                    const int s = gkb % STAGES;
+                    const uint32_t ph = (uint32_t)(gkb / STAGES) & 1u;
+                    if (*(volatile int *)&s_abort || !mbar_wait(&empty[s], ph ^ 1u, WAIT_NS)) {
+                        s_abort = 1;
+                        stop = true;
+                        break;
+                    }
+                    const int vk = kb0 + kb;
+                    const int part = vk / nk_part;
+                    const int kk = vk - part * nk_part;
+                    mbar_expect_tx(&full[s], STAGE_BYTES);
+                    const CUtensorMap *am = part ? &tma2 : &tma;
+                    if (A_MN) {
 #pragma unroll
-                for (int i = 0; i < BM / 64; ++i)
-                    tma_load_2d(sA + s * A_STAGE + i * (BK * 128), am, &full[s], m0 + 64 * i, kk * BK);
-            } else {
-                tma_load_2d(sA + s * A_STAGE, am, &full[s], kk * BK, m0);
-            }
-            if (B_MN) {
+                        for (int i = 0; i < BM / 64; ++i)
+                            tma_load_2d(sA + s * A_STAGE + i * (BK * 128), am, &full[s], m0 + 64 * i, kk * BK);
+                    } else {
+                        tma_load_2d(sA + s * A_STAGE, am, &full[s], kk * BK, m0);
+                    }
+                    if (B_MN) {
 #pragma unroll
-                for (int i = 0; i < BN / 64; ++i)
-                    tma_load_2d(sB + s * B_STAGE + i * (BK * 128), &tmb, &full[s], n0 + 64 * i, kk * BK);
-            } else {
-                tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kk * BK, n0);
+                        for (int i = 0; i < BN / 64; ++i)
+                            tma_load_2d(sB + s * B_STAGE + i * (BK * 128), &tmb, &full[s], n0 + 64 * i, kk * BK);
+                    } else {
+                        tma_load_2d(sB + s * B_STAGE, &tmb, &full[s], kk * BK, n0);
+                    }
+                }
             }
+            s_issued = gkb;
         }
-        s_issued = kb;
-    } else if (warp == 1 && lane == 0) {
-        // ---- MMA issuer ----
-        constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
-        int kb = 0;
-        for (; kb < nkb; ++kb) {
-            const int s = kb % STAGES;
-            const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-            if (!mbar_wait(&full[s], ph, WAIT_NS) || *(volatile int *)&s_abort) {
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---- MMA issuer ----
+            constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+            constexpr uint64_t a_step = A_MN ? (2048u >> 4) : (32u >> 4);
+            constexpr uint64_t b_step = B_MN ? (2048u >> 4) : (32u >> 4);
+            int gkb = 0, lt = 0;
+            bool stop = false;
+            for (int w = blockIdx.x; w < g.n_work && !stop; w += gridDim.x, ++lt) {
+                const int z = w / per_split;
+                const int nkb = min(g.kb_per_split, total_kb - z * g.kb_per_split);
+                const int buf = lt & 1;
+                if (*(volatile int *)&s_abort || !mbar_wait(&tempty[buf], ((uint32_t)(lt >> 1) & 1u) ^ 1u, WAIT_NS)) {
+                    s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < nkb; ++kb, ++gkb) {
+                    const int s = gkb % STAGES;
+                    const uint32_t ph = (uint32_t)(gkb / STAGES) & 1u;
+                    if (*(volatile int *)&s_abort || !mbar_wait(&full[s], ph, WAIT_NS)) {
+                        s_abort = 1;
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    // per MMA step of K = 16: K-major tiles advance 32 bytes along
+                    // the swizzled row, MN-major tiles advance 16 K-rows (2048 bytes)
+                    const uint64_t ad = A_MN ? smem_desc_mn_sw128(smem_u32(sA + s * A_STAGE), BK * 128)
+                                             : smem_desc_k_sw128(smem_u32(sA + s * A_STAGE));
+                    const uint64_t bd = B_MN ? smem_desc_mn_sw128(smem_u32(sB + s * B_STAGE), BK * 128)
+                                             : smem_desc_k_sw128(smem_u32(sB + s * B_STAGE));
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k)
+                        umma_bf16(acc, ad + a_step * k, bd + b_step * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                }
+                if (!stop) umma_commit(&tfull[buf]);
+            }
+            s_consumed = gkb;
+            umma_commit(fin);   // fires when every MMA issued above has completed
+        }
+    } else {
+        // ---- epilogue: warps 2-5, TMEM lane quarter q = warp & 3 ----
+        const int q = warp & 3;
+        const int et = threadIdx.x - 64;   // 0..127
+        const int row = q * 32 + lane;     // row within the tile
+        int lt = 0, chunk = 0;
+        for (int w = blockIdx.x; w < g.n_work; w += gridDim.x, ++lt) {
+            const int z = w / per_split;
+            const int r = w - z * per_split;
+            const int m0 = (r / g.n_tiles) * BM, n0 = (r % g.n_tiles) * BN;
+            const int buf = lt & 1;
+            const bool got = !*(volatile int *)&s_abort && mbar_wait(&tfull[buf], (uint32_t)(lt >> 1) & 1u, WAIT_NS);
+            if (bar_or(1, 128, !got)) {
                 s_abort = 1;
                 break;
             }
             tc_fence_after();
-            // per MMA step of K = 16: K-major tiles advance 32 bytes along the
-            // swizzled row, MN-major tiles advance 16 K-rows (2048 bytes)
-            const uint64_t ad = A_MN ? smem_desc_mn_sw128(smem_u32(sA + s * A_STAGE), BK * 128)
-                                     : smem_desc_k_sw128(smem_u32(sA + s * A_STAGE));
-            const uint64_t bd = B_MN ? smem_desc_mn_sw128(smem_u32(sB + s * B_STAGE), BK * 128)
-                                     : smem_desc_k_sw128(smem_u32(sB + s * B_STAGE));
-            constexpr uint64_t a_step = A_MN ? (2048u >> 4) : (32u >> 4);
-            constexpr uint64_t b_step = B_MN ? (2048u >> 4) : (32u >> 4);
-#pragma unroll
-            for (int k = 0; k < BK / 16; ++k)
-                umma_bf16(tmem, ad + a_step * k, bd + b_step * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-            umma_commit(&empty[s]);
-        }
-        s_consumed = kb;
-        umma_commit(accf);   // fires when every MMA issued above has completed
-    }
-
-    // ---- epilogue: all four warps ----
-    const bool acc_ready = mbar_wait(accf, 0u, WAIT_NS);
-    tc_fence_after();
-    __syncthreads();
-    const bool ok = acc_ready && !s_abort;
-    if (ok) {
-        const int row = m0 + warp * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+            const uint32_t lane_addr = tmem + (uint32_t)(buf * BN) + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            float v[32];
-            tmem_ld32(lane_addr + (uint32_t)(c * 32), v);
-            const int col0 = n0 + c * 32;
-            if (row < g.M) {
-                float *dst = g.C + (size_t)blockIdx.z * g.c_split + (size_t)row * g.N + col0;
-                if (col0 + 32 <= g.N && (g.N & 3) == 0) {
+            for (int c = 0; c < BN / EPI_COLS; ++c, ++chunk) {
+                float v[32];
+                tmem_ld32(lane_addr + (uint32_t)(c * EPI_COLS), v);
+                const int col0 = n0 + c * EPI_COLS;
+                if (g.bias) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 o;
-                        o.x = v[4 * q + 0] + (g.bias ? g.bias[col0 + 4 * q + 0] : 0.0f);
-                        o.y = v[4 * q + 1] + (g.bias ? g.bias[col0 + 4 * q + 1] : 0.0f);
-                        o.z = v[4 * q + 2] + (g.bias ? g.bias[col0 + 4 * q + 2] : 0.0f);
-                        o.w = v[4 * q + 3] + (g.bias ? g.bias[col0 + 4 * q + 3] : 0.0f);
-                        reinterpret_cast<float4 *>(dst)[q] = o;
+                    for (int i = 0; i < 32; ++i) v[i] += (col0 + i < g.N) ? __ldg(g.bias + col0 + i) : 0.0f;
+                }
+                if (g.tma_out) {
+                    uint8_t *buf_e = sE + (chunk & 1) * EPI_BYTES;
+                    // the store that last read this staging buffer is done with it
+                    if (et == 0) bulk_wait_read_1();
+                    bar_named(1, 128);
+                    // row `row`, 16-byte piece j at piece j ^ (row & 7): the
+                    // tensor map's 128-byte swizzle
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4 *>(buf_e + row * 128 + ((j ^ (row & 7)) << 4)) =
+                            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+                    tma_store_fence();
+                    bar_named(1, 128);
+                    if (et == 0) {
+                        tma_store_3d(&tmc, buf_e, col0, m0, z);
+                        bulk_commit();
                     }
                 } else {
+                    const int grow = m0 + row;
+                    if (grow < g.M) {
+                        float *dst = g.C + (size_t)z * g.c_split + (size_t)grow * g.N + col0;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (col0 + i < g.N) dst[i] = v[i] + (g.bias ? g.bias[col0 + i] : 0.0f);
+                        for (int i = 0; i < 32; ++i)
+                            if (col0 + i < g.N) dst[i] = v[i];
+                    }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
         }
-    } else if (threadIdx.x == 0) {
-        atomicOr(g.error, 1u);
+        if (et == 0) bulk_wait_all();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (!ok && threadIdx.x == 0) {
+    if (threadIdx.x == 0 && s_abort) {
+        atomicOr(g.error, 1u);
         // loads issued but never consumed still land in this CTA's shared
-        // memory: wait for them (bounded) before the CTA exits
+        // memory, and issued MMAs still write TMEM: wait for both (bounded)
         for (int kb = s_consumed; kb < s_issued; ++kb)
             (void)mbar_wait(&full[kb % STAGES], (uint32_t)(kb / STAGES) & 1u, WAIT_NS);
     }
+    if (threadIdx.x == 0) (void)mbar_wait(fin, 0u, WAIT_NS);
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -295,9 +388,37 @@ bool make_map(CUtensorMap *map, const void *base, int rows, int cols, int ld, in
     return r == CUDA_SUCCESS;
 }
 
+// fp32 C viewed as (N, M, splits), box 32 x 128 x 1, 128-byte swizzle: the
+// epilogue's store boxes.  Rows past M and columns past N are not written.
+bool make_c_map(CUtensorMap *map, float *C, int M, int N, int splits)
+{
+    auto fn = tensor_map_encoder();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)splits};
+    cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
+    cuuint32_t box[3] = {(cuuint32_t)EPI_COLS, (cuuint32_t)BM, 1u};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, C, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count_tc()
+{
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+    }
+    return n;
+}
+
 template <bool A_MN, bool B_MN>
-cudaError_t launch_tc(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const TcArgs &g,
-                      dim3 grid, cudaStream_t st)
+cudaError_t launch_tc(const CUtensorMap &ta, const CUtensorMap &ta2, const CUtensorMap &tb, const CUtensorMap &tc,
+                      const TcArgs &g, cudaStream_t st)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -306,7 +427,8 @@ cudaError_t launch_tc(const CUtensorMap &ta, const CUtensorMap &ta2, const CUten
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    gemm_tc_kernel<A_MN, B_MN><<<grid, 128, SMEM_BYTES, st>>>(ta, ta2, tb, g);
+    const int grid = min(g.n_work, sm_count_tc());
+    gemm_tc_kernel<A_MN, B_MN><<<grid, THREADS, SMEM_BYTES, st>>>(ta, ta2, tb, tc, g);
     return cudaGetLastError();
 }
 
@@ -344,9 +466,14 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, 
     splits = (total + g.kb_per_split - 1) / g.kb_per_split;   // no empty split
     g.c_split = (long long)M * N;
     g.error = error;
-    const dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, splits);
-    if (a_mn) return b_mn ? launch_tc<true, true>(ta, ta2, tb, g, grid, st) : launch_tc<true, false>(ta, ta2, tb, g, grid, st);
-    return b_mn ? launch_tc<false, true>(ta, ta2, tb, g, grid, st) : launch_tc<false, false>(ta, ta2, tb, g, grid, st);
+    g.m_tiles = (M + BM - 1) / BM;
+    g.n_tiles = (N + BN - 1) / BN;
+    g.n_work = g.m_tiles * g.n_tiles * splits;
+    CUtensorMap tc;
+    memset(&tc, 0, sizeof(tc));
+    g.tma_out = ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 && make_c_map(&tc, C, M, N, splits)) ? 1 : 0;
+    if (a_mn) return b_mn ? launch_tc<true, true>(ta, ta2, tb, tc, g, st) : launch_tc<true, false>(ta, ta2, tb, tc, g, st);
+    return b_mn ? launch_tc<false, true>(ta, ta2, tb, tc, g, st) : launch_tc<false, false>(ta, ta2, tb, tc, g, st);
 }
 
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want)

@@ -91,6 +91,23 @@ SLSTM_DEVINL void tma_store_3d(const CUtensorMap *map, const void *src, int c0, 
                  : "memory");
 }
 
+SLSTM_DEVINL void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+SLSTM_DEVINL void tma_store_2d(const CUtensorMap *map, const void *src, int c0, int c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+// The source shared memory of all but the most recent committed bulk store
+// group may be reused.
+SLSTM_DEVINL void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
 SLSTM_DEVINL void tma_store_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 SLSTM_DEVINL void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // The source shared memory of every committed bulk store may be reused.
