@@ -501,13 +501,25 @@ struct Layout {
 
 long long round8(long long v) { return (v + 7) & ~7LL; }
 
-// split-K count of the W_x-gradient GEMM: enough CTAs for two per SM
+// split-K count of the W_x-gradient GEMM: the count (up to 16) whose work
+// items fill whole waves of the persistent CTAs best; a larger count only
+// when it fills them at least 2% better (each split adds an M x N partial).
 int wgrad_splits(int B, int T, int d_in, int d_h)
 {
     const long long tiles = ((4LL * d_h + 127) / 128) * ((d_in + 255) / 256);
-    int want = (int)((296 + tiles - 1) / tiles);
-    if (want > 16) want = 16;
-    return gemm_tc_splits(4 * d_h, d_in, B * T, 2, want);
+    const long long sms = sm_count_bwd();
+    int best = 1;
+    double best_eff = 0.0;
+    for (int want = 1; want <= 16; ++want) {
+        const int s = gemm_tc_splits(4 * d_h, d_in, B * T, 2, want);
+        const long long work = tiles * s;
+        const double eff = (double)work / (double)(((work + sms - 1) / sms) * sms);
+        if (eff > best_eff + 0.02) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    return best;
 }
 
 Layout layout(int B, int T, int d_in, int d_h)

@@ -205,11 +205,16 @@ def test_newton_bounded_wait_reports_timeout(cuda_device):
 # backward
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
-@pytest.mark.parametrize("B,T,d_in,d,dtype", [(2, 64, 8, 8, "f32"), (2, 75, 12, 40, "f32"),
-                                              (2, 75, 16, 40, "bf16"), (3, 130, 64, 96, "bf16")])
+@pytest.mark.parametrize("B,T,d_in,d,dtype", [(2, 64, 8, 8, "f32"), (2, 75, 12, 40, "f32"), (2, 33, 8, 10, "f32"),
+                                              (2, 75, 16, 40, "bf16"), (3, 130, 64, 96, "bf16"),
+                                              (2, 96, 16, 40, "bf16"), (2, 100, 24, 36, "bf16"),
+                                              (2, 70, 16, 18, "bf16")])
 def test_backward_matches_oracle_bptt(forget, B, T, d_in, d, dtype, cuda_device):
     """fp32 inputs take the CUDA-core GEMMs; bf16 inputs the tensor-core GEMMs
-    with dP carried as a bf16 pair (transposed copy for the W_x gradient)."""
+    with dP carried as a bf16 pair (transposed copy for the W_x gradient).
+    d % 4 != 0 takes the cp.async tile path of the adjoint kernel, d % 4 == 0
+    the TMA one; T % 4 == 0 writes the transposed pair in 8-byte pieces
+    (with T % 32 != 0 the last tile starts before t = 0), other T per element."""
     w = Workload("t", B, T, d_in, d, dtype, forget, 0.5, 13, 1e-6, 64)
     inp = make_inputs(w, with_dH=True)
     g = torch.Generator().manual_seed(9)
