@@ -31,7 +31,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from nonlinear_rnn_pararnn_b200.workloads import ORDER, WORKLOADS, as_f64, make_inputs  # noqa: E402
+from nonlinear_rnn_pararnn_b200.workloads import ORDER, WORKLOADS, as_f64, make_inputs, scaled  # noqa: E402
 
 METRIC = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd+bwd)"
 METRIC_FWD = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd)"
@@ -393,10 +393,17 @@ def main(argv=None):
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="run the workload with T shortened to this length (small cases for ncu "
+                         "captures; the bench line then names the shortened workload)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = WORKLOADS[args.workload]
+    if args.seq_len is not None:
+        if not 1 <= args.seq_len <= w.T:
+            ap.error(f"--seq-len must be in [1, {w.T}]")
+        w = scaled(w, T=args.seq_len, name=f"{w.name}_T{args.seq_len}")
     ws, _, _ = _dist()
     if ws != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
