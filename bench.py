@@ -20,6 +20,7 @@ bounded sample of lanes of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import subprocess
@@ -284,9 +285,9 @@ def run_gpu(args, w):
     # the K launches of a step.
     newton_bytes = elems * (32 + 48 * (K - 1)) / K
     achieved = newton_bytes / (newton_launch_ms / 1e3) / 1e9
+    traffic = args.traffic_bytes if args.traffic_bytes else newton_traffic_bytes(elems, K)
     roofline = {"kernel": "newton_iter", "bound": "hbm", "achieved": achieved, "peak": hbm,
-                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": args.traffic_bytes if args.traffic_bytes else None,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                 "algorithmic_bytes_per_launch": newton_bytes, "avg_launch_ms": newton_launch_ms}
 
     cpu = None
@@ -374,6 +375,33 @@ def run_scan(args):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+# DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
+# last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
+# (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
+# this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
+# (every tile moves the same bytes), so it scales to a full launch by the element count.
+NEWTON_TRAFFIC = {"sources_sha256": "bcf8928af9c19e747b45a6a0c09c7e52bb16cb3270ce693cfa511b5f66e41be1", "first": 31.66, "middle": 48.28, "last": 48.05}
+NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
+
+
+def newton_sources_sha256() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nonlinear_rnn_pararnn_b200", "csrc")
+    for name in NEWTON_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def newton_traffic_bytes(elems: int, K: int):
+    """Measured DRAM bytes of one Newton launch averaged over the K launches of a step, or None."""
+    if newton_sources_sha256() != NEWTON_TRAFFIC["sources_sha256"]:
+        return None
+    t = NEWTON_TRAFFIC
+    per = t["first"] if K == 1 else (t["first"] + t["middle"] * (K - 2) + t["last"]) / K
+    return per * elems
 
 
 def main(argv=None):
