@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
         float lam[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][lane];
+        for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][sw(e, lane)];
         float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
         float dv[L][4];   // dP of the thread's steps (gate order z, i, f, o)
 #pragma unroll

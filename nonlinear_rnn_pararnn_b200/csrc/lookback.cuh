@@ -25,7 +25,7 @@
 //
 // Two layouts of the per-warp maps are supported.  The plain one,
 // s_agg[w][20][32] (entry-major), is walked by warp 0 alone.  TileMaps stores
-// the maps column-major with a padded row stride so that four warps can walk
+// the maps column-major with XOR-swizzled rows so that four warps can walk
 // them at once with one (feature, row) pair per lane (carry_chain4): the
 // carry's serial dependence over the NW maps then costs one 4-term dot
 // product per map and lane instead of a 4x4 matrix-vector product.
@@ -327,9 +327,12 @@ SLSTM_DEVINL void affp_to_aff(const AffP &p, Aff &x)
 }
 
 // ---- chain layout -------------------------------------------------------------
-// Row stride of TileMaps: with 40 floats, (row, feature) pairs of one chain
-// warp (8 features x 4 rows) fall in 32 distinct banks.
-constexpr int MAP_LD = 40;
+// Row length of TileMaps.  Feature f of row r sits at position f ^ (8 r)
+// (sw(r, f)): a row written by 32 feature lanes is a permutation of 32 banks,
+// and the 32 (row, feature) pairs a chain warp reads (8 features x 4 rows)
+// also fall in 32 distinct banks.
+constexpr int MAP_LD = 32;
+SLSTM_DEVINL int sw(int r, int f) { return f ^ (r << 3); }
 
 // Per-warp maps of a tile, [warp][column k, k = 4: offset b][row][feature],
 // and the carries entering the warps, [warp][slot][feature].
@@ -348,8 +351,8 @@ SLSTM_DEVINL void maps_store(MapArr *m, int w, int lane, const Aff &x)
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) m[w][k][r][lane] = x.a[r * 4 + k];
-        m[w][4][r][lane] = x.b[r];
+        for (int k = 0; k < 4; ++k) m[w][k][r][sw(r, lane)] = x.a[r * 4 + k];
+        m[w][4][r][sw(r, lane)] = x.b[r];
     }
 }
 
@@ -357,11 +360,11 @@ SLSTM_DEVINL void maps_store(MapArr *m, int w, int lane, const AffP &x)
 {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        m[w][0][r][lane] = x.a01[r].x;
-        m[w][1][r][lane] = x.a01[r].y;
-        m[w][2][r][lane] = x.a23[r].x;
-        m[w][3][r][lane] = x.a23[r].y;
-        m[w][4][r][lane] = x.b[r];
+        m[w][0][r][sw(r, lane)] = x.a01[r].x;
+        m[w][1][r][sw(r, lane)] = x.a01[r].y;
+        m[w][2][r][sw(r, lane)] = x.a23[r].x;
+        m[w][3][r][sw(r, lane)] = x.a23[r].y;
+        m[w][4][r][sw(r, lane)] = x.b[r];
     }
 }
 
@@ -370,8 +373,8 @@ SLSTM_DEVINL void maps_load(const MapArr *m, int w, int lane, Aff &x)
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x.a[r * 4 + k] = m[w][k][r][lane];
-        x.b[r] = m[w][4][r][lane];
+        for (int k = 0; k < 4; ++k) x.a[r * 4 + k] = m[w][k][r][sw(r, lane)];
+        x.b[r] = m[w][4][r][sw(r, lane)];
     }
 }
 
@@ -398,12 +401,13 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
     const int i8 = lane & 7;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-        cin[w][r][f] = c;
-        const float a0 = m[w][0][r][f];
-        const float a1 = m[w][1][r][f];
-        const float a2 = m[w][2][r][f];
-        const float a3 = m[w][3][r][f];
-        const float bb = m[w][4][r][f];
+        const int fs = sw(r, f);
+        cin[w][r][fs] = c;
+        const float a0 = m[w][0][r][fs];
+        const float a1 = m[w][1][r][fs];
+        const float a2 = m[w][2][r][fs];
+        const float a3 = m[w][3][r][fs];
+        const float bb = m[w][4][r][fs];
         const float v0 = __shfl_sync(0xffffffffu, c, i8);
         const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
         const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
@@ -429,7 +433,7 @@ SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, const MapArr *m, CinA
         ca, load,
         [&](int w, const float v[4]) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cin[w][e][lane] = v[e];
+            for (int e = 0; e < 4; ++e) cin[w][e][sw(e, lane)] = v[e];
         },
         ticket, withhold, carry);
 }

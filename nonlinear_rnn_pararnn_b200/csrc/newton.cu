@@ -8,8 +8,8 @@
 // one CTA of 8 warps (lane = feature, warp = 4 consecutive steps).
 //
 // Persistent CTAs walk the tiles in ticket order and keep the next tile's P
-// and old S arriving in shared memory (cp.async, double buffered) while they
-// work on the current one:
+// and old S arriving in shared memory (TMA, or cp.async when rows are not
+// 16-byte aligned; double buffered) while they work on the current one:
 //   walk A  each thread recomputes gates, stabilizer, f(S_{t-1}, P_t) and the
 //           4x4 Jacobian J_t in registers for its 4 steps, keeps (J_t, r_t =
 //           f - S_t) in registers and folds the maps delta -> J_t delta + r_t;
@@ -71,6 +71,7 @@ struct TileInfo {
 struct Smem {
     float P[2][TT][4][32];   // stage s: rows (step, slot) of 32 features; TMA boxes land here
     float S[2][TT][4][32];
+    float O[TT][4][32];    // TMA path: S_new of the tile, source of the warps' TMA stores
     float R[2][4][32];     // TMA path: the tile's recurrent weights (gate-major)
     float bnd[2][4][32];   // TMA path: S_old just before the tile (previous launch's boundary)
     TileMaps<NW> maps;
@@ -268,8 +269,10 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         unsigned after = 0;
         if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
         if (TMA) {
-            // the current tile's boxes have landed (the next tile's loads
-            // start after walk A, once this stage's old stores are read out)
+            // the other stage is free (every warp passed the barrier that
+            // ends the previous tile): start the next tile's loads a whole
+            // tile ahead, then wait for the current tile's boxes
+            if (threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st ^ 1, sm.info[rn], !FIRST);
             if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS)) {
                 atomicOr(a.error, 2u);
                 (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS);
@@ -363,9 +366,6 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         maps_store(sm.maps.m, warp, lane, agg);
         // the tile after the next one, visible to all after the vote barrier
         if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
-        // this warp's stores of the previous tile have been read out of the
-        // other stage, which the next tile's loads overwrite after the barrier
-        if (TMA && lane == 0) bulk_wait_read_all();
 
         // ---- carry ----
         float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
@@ -380,7 +380,6 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         }
         const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
         const bool fast = __syncthreads_and(ok);
-        if (TMA && threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st ^ 1, sm.info[rn], !FIRST);
         if (fast) {
             if (chain_warp) {
                 c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane);
@@ -393,9 +392,14 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         __syncthreads();
 
         // ---- walk B ----
+        // this warp's store of the previous tile has read its rows of O
+        if (TMA) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        }
         float dl[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dl[e] = sm.maps.cin[warp][e][lane];
+        for (int e = 0; e < 4; ++e) dl[e] = sm.maps.cin[warp][e][sw(e, lane)];
         float snp[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
@@ -416,10 +420,10 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
                 dl[e] = sn[e] - so;
             }
             if (TMA) {
-                // in place over S_old in the stage; rows past T and features
-                // past d fall outside the tensor and are not stored
+                // rows past T and features past d fall outside the tensor and
+                // are not stored
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sm.S[st][sl][e][lane] = sn[e];
+                for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sn[e];
             } else {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
@@ -447,7 +451,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             tma_store_fence();
             __syncwarp();
             if (lane == 0 && t_seg < T) {
-                tma_store_3d(&maps.Sw, &sm.S[st][warp * L][0][0], ti.j0, t_seg * 4, ti.b);
+                tma_store_3d(&maps.Sw, &sm.O[warp * L][0][0], ti.j0, t_seg * 4, ti.b);
                 bulk_commit();
             }
         }
@@ -458,11 +462,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
         }
 
-        // TMA: no barrier here.  The next tile's loads go to the other stage,
-        // and the vote barrier after its walk A orders every warp's walk B
-        // here before the stage, the maps or the carries are written again.
-        // The cp.async path prefetches at the top of the tile and needs one.
-        if (!TMA) __syncthreads();
+        __syncthreads();   // this stage is free for the loads of the tile after next
         ring = rn;
         st ^= 1;
         ++it;
