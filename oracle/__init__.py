@@ -243,3 +243,61 @@ def backward_btgd(x, Wx, P, R, s0, S, dH, forget="sigmoid"):
     db_g = db.reshape(B, d, 4).sum(axis=0).T.copy()
     return {"dx": dx, "dWx": dWx, "dR": dR_g, "db": db_g,
             "ds0": bgd_from_lanes(ds0, B, d), "dP": dP_b}
+
+
+# ----------------------------------------------------------------------------
+# packed ragged sequences ("sLSTM in this library", section "Packed sequences":
+# sequences concatenated along time, exclusive-prefix offsets cu_seqlens, one
+# initial state per sequence).  The packed problem is, by definition, the
+# independent problems of its sequences; these functions cut the packed
+# arrays at the offsets and run the pinned per-sequence functions above.
+# ----------------------------------------------------------------------------
+def _segments(cu):
+    cu = [int(v) for v in np.asarray(cu).reshape(-1)]
+    return [(k, cu[k], cu[k + 1]) for k in range(len(cu) - 1)]
+
+
+def sequential_varlen(P, R, s0, cu, forget="sigmoid") -> np.ndarray:
+    """P (total_T, 4, d) packed; s0 (n, 4, d) or None -> S (total_T, 4, d)."""
+    P = _f64(P)
+    d = P.shape[2]
+    S = np.zeros_like(P)
+    for k, a, b in _segments(cu):
+        if b > a:
+            s0k = np.zeros((1, 4, d)) if s0 is None else _f64(s0)[k:k + 1]
+            S[a:b] = sequential_btgd(P[None, a:b], R, s0k, forget)[0]
+    return S
+
+
+def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4) -> np.ndarray:
+    """K Newton iterations from the zero guess on every sequence (fixed-K mode)."""
+    P = _f64(P)
+    d = P.shape[2]
+    S = np.zeros_like(P)
+    for k, a, b in _segments(cu):
+        if b > a:
+            s0k = np.zeros((1, 4, d)) if s0 is None else _f64(s0)[k:k + 1]
+            S[a:b] = newton_btgd(P[None, a:b], R, s0k, forget, max_iters=K, fixed=True, tol=0.0)[0][0]
+    return S
+
+
+def backward_varlen(x, Wx, P, R, s0, S, dH, cu, forget="sigmoid"):
+    """Gradients of L = sum dH * h over all sequences: dx (total_T, d_in), dWx, dR, db
+    (summed over sequences) and ds0 (n, 4, d; zero for empty sequences)."""
+    x, P, S, dH = _f64(x), _f64(P), _f64(S), _f64(dH)
+    Wx = _f64(Wx)
+    d = P.shape[2]
+    segs = _segments(cu)
+    out = {"dx": np.zeros_like(x), "dWx": np.zeros(Wx.shape), "dR": np.zeros((4, d)), "db": np.zeros((4, d)),
+           "ds0": np.zeros((len(segs), 4, d)), "dP": np.zeros_like(P)}
+    for k, a, b in segs:
+        if b == a:
+            continue
+        s0k = np.zeros((1, 4, d)) if s0 is None else _f64(s0)[k:k + 1]
+        g = backward_btgd(x[None, a:b], Wx, P[None, a:b], R, s0k, S[None, a:b], dH[None, a:b], forget)
+        out["dx"][a:b] = g["dx"][0]
+        out["dP"][a:b] = g["dP"][0]
+        out["ds0"][k] = g["ds0"][0]
+        for key in ("dWx", "dR", "db"):
+            out[key] += g[key]
+    return out

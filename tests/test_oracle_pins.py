@@ -319,3 +319,67 @@ def test_gemm_matches_numpy():
     np.testing.assert_allclose(oracle.gemm(A, Bm, bias=bias), A @ Bm + bias, rtol=1e-13)
     np.testing.assert_allclose(oracle.gemm(A.T.copy(), Bm, ta=True), A @ Bm, rtol=1e-13)
     np.testing.assert_allclose(oracle.gemm(A, Bm.T.copy(), tb=True), A @ Bm, rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# packed ragged sequences: the packed problem is the independent problems of
+# its sequences ("sLSTM in this library", section "Packed sequences").  These
+# pin the cutting and gathering at the offsets against the batched functions.
+# ---------------------------------------------------------------------------
+def _packed_case(rng, B, T, d, d_in):
+    x = rng.normal(size=(B, T, d_in))
+    Wx = rng.normal(size=(4 * d, d_in)) / math.sqrt(d_in)
+    bias = np.zeros((4, d))
+    bias[2] = np.linspace(3, 6, d)
+    R = rng.uniform(-0.5, 0.5, size=(4, d))
+    s0 = np.stack([rng.normal(size=(B, d)), rng.uniform(0.5, 1.5, size=(B, d)), rng.normal(size=(B, d)),
+                   rng.uniform(-0.5, 0.5, size=(B, d))], axis=1)
+    dH = rng.normal(size=(B, T, d))
+    return x, Wx, bias, R, s0, dH
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_varlen_equal_lengths_equals_batched(forget):
+    rng = np.random.default_rng(51)
+    B, T, d, d_in = 3, 7, 4, 5
+    x, Wx, bias, R, s0, dH = _packed_case(rng, B, T, d, d_in)
+    P = oracle.preact(x, Wx, bias)
+    cu = np.arange(B + 1) * T
+    pk = lambda a: a.reshape((B * T,) + a.shape[2:])
+    S_b = oracle.sequential_btgd(P, R, s0, forget)
+    np.testing.assert_array_equal(oracle.sequential_varlen(pk(P), R, s0, cu, forget), pk(S_b))
+    N_b, _ = oracle.newton_btgd(P, R, s0, forget, max_iters=3, fixed=True, tol=0.0)
+    np.testing.assert_array_equal(oracle.newton_varlen_fixed(pk(P), R, s0, cu, forget, 3), pk(N_b))
+    g_b = oracle.backward_btgd(x, Wx, P, R, s0, S_b, dH, forget)
+    g_v = oracle.backward_varlen(pk(x), Wx, pk(P), R, s0, pk(S_b), pk(dH), cu, forget)
+    np.testing.assert_allclose(g_v["dx"], pk(g_b["dx"]), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g_v["ds0"], g_b["ds0"], rtol=0, atol=1e-12)
+    for k in ("dWx", "dR", "db"):
+        np.testing.assert_allclose(g_v[k], g_b[k], rtol=1e-12, atol=1e-12)
+
+
+def test_varlen_empty_sequences_and_independence():
+    rng = np.random.default_rng(52)
+    d, d_in = 3, 4
+    x, Wx, bias, R, s0, dH = _packed_case(rng, 5, 6, d, d_in)
+    P = oracle.preact(x, Wx, bias)
+    total = 13
+    xp, Pp, dHp = x.reshape(-1, d_in)[:total], P.reshape(-1, 4, d)[:total], dH.reshape(-1, d)[:total]
+    cu = np.array([0, 5, 5, 6, 13, 13])        # lengths 5, 0, 1, 7, 0
+    S = oracle.sequential_varlen(Pp, R, s0, cu)
+    # a sequence of length one is one step from its own s0
+    one = oracle.sequential_btgd(Pp[None, 5:6], R, s0[2:3])[0]
+    np.testing.assert_array_equal(S[5:6], one)
+    # changing the initial state of sequence 3 changes nothing outside [6, 13)
+    s0b = s0.copy()
+    s0b[3] += 0.7
+    S2 = oracle.sequential_varlen(Pp, R, s0b, cu)
+    np.testing.assert_array_equal(S2[:6], S[:6])
+    assert np.abs(S2[6:] - S[6:]).max() > 1e-6
+    g = oracle.backward_varlen(xp, Wx, Pp, R, s0, S, dHp, cu)
+    assert not g["ds0"][1].any() and not g["ds0"][4].any()    # empty sequences get no gradient
+    # dropping the empty sequences changes no gradient of the others
+    cu2 = np.array([0, 5, 6, 13])
+    g2 = oracle.backward_varlen(xp, Wx, Pp, R, s0[[0, 2, 3]], S, dHp, cu2)
+    np.testing.assert_array_equal(g2["dx"], g["dx"])
+    np.testing.assert_array_equal(g2["ds0"], g["ds0"][[0, 2, 3]])
