@@ -79,7 +79,9 @@ typedef enum {
     SLSTM_OP_PREACT_GEMM = 0,
     SLSTM_OP_NEWTON_FORWARD = 1,
     SLSTM_OP_SCAN_BLOCK4 = 2,
-    SLSTM_OP_NEWTON_BACKWARD = 3
+    SLSTM_OP_NEWTON_BACKWARD = 3,
+    SLSTM_OP_NEWTON_FORWARD_VARLEN = 4,   /* B = number of sequences, T = total packed length */
+    SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5   /* B = number of sequences, T = total packed length */
 } slstm_op;
 
 #define SLSTM_MAX_ITERS 65536     /* largest accepted max_iters              */
@@ -249,6 +251,38 @@ int slstm_newton_backward(const void *x, const void *Wx, int dtype, const float 
                           float *dx, float *dWx, float *dR, float *db, float *ds0, int forget,
                           int B, int T, int d_in, int d_h, void *ws, size_t ws_bytes,
                           slstm_stream_t stream);
+
+/*
+ * Packed ragged sequences ("sLSTM in this library", "Packed sequences": time
+ * packed as (1, N, ...) with FlashAttention-style exclusive-prefix offsets,
+ * one initial state per sequence, the Newton inner solve a segmented scan on
+ * the (J, r) monoid with a head flag at each sequence start).
+ *   cu_seqlens  device int32 array of n_seq + 1 offsets: cu_seqlens[0] = 0,
+ *               nondecreasing, cu_seqlens[n_seq] = total_T; sequence k
+ *               occupies packed steps [cu_seqlens[k], cu_seqlens[k+1]) and
+ *               may be empty
+ *   P, S        (total_T, 4, d_h) fp32;  dH (total_T, d_h);  x (total_T, d_in)
+ *   s0, ds0     (n_seq, 4, d_h) fp32, s0 may be NULL (zeros), ds0 may be NULL
+ * At a sequence's first step the previous state is its own s0 and the step
+ * does not depend on the step before it (a zero Jacobian: the head flag), so
+ * every sequence is solved exactly as on its own; the stopping test and the
+ * stats are over all sequences together.  The offsets are read on the
+ * device: the forward checks them and, when they are malformed, writes
+ * SLSTM_ERR_INVALID_ARG to stats->error and leaves S untouched; both calls
+ * clamp every offset into [0, total_T], so malformed offsets never lead to an
+ * access outside the arrays.  Workspace: slstm_workspace_size with
+ * SLSTM_OP_NEWTON_FORWARD_VARLEN / _BACKWARD_VARLEN, B = n_seq, T = total_T.
+ * Other arguments and errors as slstm_newton_forward / slstm_newton_backward.
+ */
+int slstm_newton_forward_varlen(const float *P, const float *R, const float *s0, const int *cu_seqlens,
+                                int n_seq, float *S, const slstm_newton_config *cfg, slstm_newton_stats *stats,
+                                int total_T, int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+int slstm_newton_backward_varlen(const void *x, const void *Wx, int dtype, const float *P, const float *R,
+                                 const float *s0, const int *cu_seqlens, int n_seq, const float *S,
+                                 const float *dH, float *dx, float *dWx, float *dR, float *db, float *ds0,
+                                 int forget, int total_T, int d_in, int d_h, void *ws, size_t ws_bytes,
+                                 slstm_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -26,6 +26,8 @@ SLSTM_OP_PREACT_GEMM = 0
 SLSTM_OP_NEWTON_FORWARD = 1
 SLSTM_OP_SCAN_BLOCK4 = 2
 SLSTM_OP_NEWTON_BACKWARD = 3
+SLSTM_OP_NEWTON_FORWARD_VARLEN = 4
+SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5
 SLSTM_MAX_ITERS = 65536
 SLSTM_STATS_HISTORY = 64
 SLSTM_SCAN_REVERSE_T = 1
@@ -54,6 +56,10 @@ SIGNATURES = {
     "slstm_sequential_step": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
     "slstm_newton_backward": (_I, [_V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I,
                                    _V, _Z, _V]),
+    "slstm_newton_forward_varlen": (_I, [_V, _V, _V, _V, _I, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _V, _Z,
+                                         _V]),
+    "slstm_newton_backward_varlen": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I,
+                                          _I, _V, _Z, _V]),
 }
 
 _lib = None

@@ -171,3 +171,69 @@ def newton_backward(x, Wx, P, R, s0, S, dH, *, forget="sigmoid", out: dict = Non
         _ptr(out["dWx"]), _ptr(out["dR"]), _ptr(out["db"]), _ptr(out.get("ds0")), forget_code(forget), B, T,
         d_in, d_h, _ptr(ws), ws.numel(), _stream()))
     return out
+
+
+# ---------------------------------------------------------------------------
+# packed ragged sequences (cu_seqlens)
+# ---------------------------------------------------------------------------
+def _need_cu(cu: torch.Tensor, n_seq: int):
+    if cu.device.type != "cuda" or cu.dtype != torch.int32 or not cu.is_contiguous() or cu.dim() != 1 \
+            or cu.numel() != n_seq + 1:
+        raise ValueError(f"cu_seqlens must be a contiguous int32 CUDA tensor of {n_seq + 1} offsets")
+
+
+def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu_seqlens: torch.Tensor, *,
+                          forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
+                          S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None):
+    """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
+    cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats)."""
+    total_T, four, d_h = P.shape
+    n_seq = cu_seqlens.numel() - 1
+    _need(P, "P", (total_T, 4, d_h))
+    _need(R, "R", (4, d_h))
+    _need_cu(cu_seqlens, n_seq)
+    if s0 is not None:
+        _need(s0, "s0", (n_seq, 4, d_h))
+    if S is None:
+        S = torch.empty_like(P)
+    _need(S, "S", (total_T, 4, d_h))
+    if stats is None:
+        stats = new_stats(P.device)
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
+    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0)
+    check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
+        _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
+        _ptr(ws), ws.numel(), _stream()))
+    return S, stats
+
+
+def newton_backward_varlen(x, Wx, P, R, s0, cu_seqlens, S, dH, *, forget="sigmoid", out: dict = None,
+                           ws: torch.Tensor = None):
+    """Gradients of sum(dH * h) over packed sequences: x (total_T, d_in), P and S (total_T, 4, d_h),
+    dH (total_T, d_h); returns dict dx, dWx, dR, db, ds0 (n_seq, 4, d_h)."""
+    total_T, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    n_seq = cu_seqlens.numel() - 1
+    dt = x.dtype
+    _need(x, "x", (total_T, d_in), dt)
+    _need(Wx, "Wx", (4 * d_h, d_in), dt)
+    _need(P, "P", (total_T, 4, d_h))
+    _need(R, "R", (4, d_h))
+    _need_cu(cu_seqlens, n_seq)
+    if s0 is not None:
+        _need(s0, "s0", (n_seq, 4, d_h))
+    _need(S, "S", (total_T, 4, d_h))
+    _need(dH, "dH", (total_T, d_h))
+    dev = x.device
+    if out is None:
+        out = {"dx": torch.empty(total_T, d_in, device=dev), "dWx": torch.empty(4 * d_h, d_in, device=dev),
+               "dR": torch.empty(4, d_h, device=dev), "db": torch.empty(4, d_h, device=dev),
+               "ds0": torch.empty(n_seq, 4, d_h, device=dev)}
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_BACKWARD_VARLEN, n_seq, total_T, d_in, d_h, dev)
+    check("slstm_newton_backward_varlen", load().slstm_newton_backward_varlen(
+        _ptr(x), _ptr(Wx), _DTYPE[dt], _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), _ptr(dH),
+        _ptr(out["dx"]), _ptr(out["dWx"]), _ptr(out["dR"]), _ptr(out["db"]), _ptr(out.get("ds0")),
+        forget_code(forget), total_T, d_in, d_h, _ptr(ws), ws.numel(), _stream()))
+    return out

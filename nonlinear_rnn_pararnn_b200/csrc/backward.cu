@@ -38,6 +38,8 @@ struct BwdArgs {
     float *ds0;       // (B, 4, d) or null
     unsigned *ticket;
     CarryArgs ca;
+    const unsigned *vmask;   // packed sequences: head-flag words (one per 32 steps), else null
+    const int *vseq;         // packed sequences: sequence index at each head step
     int T, d, groups_per_row, n_tiles, vec16, dpt_vec8;
 };
 
@@ -49,7 +51,8 @@ struct BwdInfo {
     int b;
     int j0;
     int t_lo;
-    int pad[3];
+    int pad;
+    unsigned long long hmask;   // packed sequences: bit r set when step t_lo + r (r <= 32) starts a sequence
 };
 
 // Shared memory of one CTA.  A tile needs S at t_lo-1 .. t_hi, P at
@@ -84,6 +87,7 @@ SLSTM_DEVINL void bwd_decode(const BwdArgs &a, unsigned ticket, BwdInfo &ti)
 {
     ti.ticket = ticket;
     ti.chunk = ti.b = ti.j0 = ti.t_lo = 0;
+    ti.hmask = 0ull;
     if (ticket < (unsigned)a.n_tiles) {
         const unsigned G = (unsigned)a.ca.n_groups;
         const unsigned chunk = ticket / G;
@@ -93,6 +97,16 @@ SLSTM_DEVINL void bwd_decode(const BwdArgs &a, unsigned ticket, BwdInfo &ti)
         ti.b = (int)b;
         ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
         ti.t_lo = a.T - ((int)chunk + 1) * TT;
+        if (a.vmask) {
+            // bits of steps t_lo .. t_lo + 32 from the (up to three) words they span
+            const int q = (ti.t_lo >= 0) ? (ti.t_lo >> 5) : -((31 - ti.t_lo) >> 5);
+            const int sh = ti.t_lo - 32 * q;   // 0 .. 31
+            const int nw = (a.T + 31) >> 5;
+            unsigned long long w[3];
+#pragma unroll
+            for (int i = 0; i < 3; ++i) w[i] = (q + i >= 0 && q + i < nw) ? a.vmask[q + i] : 0u;
+            ti.hmask = (w[0] >> sh) | (w[1] << (32 - sh)) | (sh ? (w[2] << (64 - sh)) : 0ull);
+        }
     }
 }
 
@@ -163,7 +177,10 @@ SLSTM_DEVINL void bwd_issue_load(const BwdArgs &a, const BwdMaps &m, BwdSmem &sm
 
 // TMA: tiles arrive by TMA (BWD_TMA_THREAD, mbarrier per stage); otherwise by
 // cp.async.  BF16OUT: dP leaves as the transposed bf16 pair, else as fp32.
-template <int FORGET, bool BF16OUT, bool TMA>
+// VARLEN: packed ragged sequences (B = 1): J_{t+1} is zero when step t + 1
+// starts a sequence, and a sequence's first step takes its s0 (and yields its
+// ds0) as the dense kernel does at t = 0.
+template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN>
 __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -256,8 +273,11 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             cell_eval<FORGET, true>(sm.S[st][rl + 1][0][lane], sm.S[st][rl + 1][1][lane], sm.S[st][rl + 1][2][lane],
                                     sm.S[st][rl + 1][3][lane], sm.P[st][rl + 1][0][lane], sm.P[st][rl + 1][1][lane],
                                     sm.P[st][rl + 1][2][lane], sm.P[st][rl + 1][3][lane], rz, ri, rf, ro, Jn[i]);
+            // step t + 1 starts a sequence: lambda_t does not depend on lambda_{t+1}
+            const bool reset = VARLEN && ((ti.hmask >> (rl + 1)) & 1ull);
+            if (reset) cell_zero_jac(Jn[i]);
             const float r[4] = {0.f, 0.f, 0.f, sm.dH[st][rl][lane]};
-            if (i == 0) affp_from_cell<true>(agg, Jn[0], r);
+            if (i == 0 || reset) affp_from_cell<true>(agg, Jn[i], r);
             else fold_p<true>(agg, Jn[i], r);
         }
         maps_store(sm.u.m, warp, lane, agg);
@@ -274,15 +294,23 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 c = __uint_as_float((unsigned)w2);
             }
         }
+        // warps whose steps contain such a reset (bits rl + 1 of their steps)
+        unsigned whead = 0u;
+        if (VARLEN) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w)
+                whead |= (((ti.hmask >> (TT - L - w * L + 1)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
+        }
         const bool fast = __syncthreads_and(ok);
         if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
         if (fast) {
             if (chain_warp) {
-                c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane);
+                c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead);
                 st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
             }
         } else if (warp == 0) {
-            tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false);
+            tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false,
+                                    whead);
         }
         __syncthreads();   // the maps are dead from here on; the dP staging takes their place
 
@@ -296,6 +324,10 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         for (int i = 0; i < L; ++i) {
             const int rl = TT - 1 - (warp * L + i);
             const int t = t_lo + rl;
+            if (VARLEN && ((ti.hmask >> (rl + 1)) & 1ull)) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) lam[e] = 0.0f;
+            }
             jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
             lam[3] += sm.dH[st][rl][lane];
             float prev[4];
@@ -303,17 +335,19 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
             Cell cc;
             CellG g;
-            if (t == 0) {
-                // the state before the sequence is s0; ds0 = J_0^T lambda_0
+            const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
+            if (head) {
+                // the state before the sequence is its s0; ds0 = J^T lambda at its first step
+                const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj) : 0.f;
+                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
                 cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
                                               sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
                                               ri, rf, ro, cc, &g);
                 if (a.ds0 && jv) {
                     float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
                     jacT_mul(cc, v0, v1, v2, v3);
-                    float *q = a.ds0 + (size_t)ti.b * 4 * d + jj;
+                    float *q = a.ds0 + sq * 4 * d + jj;
                     q[0] = v0;
                     q[d] = v1;
                     q[2 * d] = v2;
@@ -469,10 +503,10 @@ int sm_count_bwd()
     return n;
 }
 
-template <int FORGET, bool BF16OUT, bool TMA>
+template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN>
 cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
 {
-    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT, TMA>;
+    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT, TMA, VARLEN>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BWD_SMEM_BYTES);
@@ -486,11 +520,22 @@ cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
     return cudaGetLastError();
 }
 
-template <int FORGET>
-cudaError_t launch_adjoint_any(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, cudaStream_t st)
+template <int FORGET, bool VARLEN>
+cudaError_t launch_adjoint_v(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, cudaStream_t st)
 {
-    if (tma) return bf16out ? launch_adjoint<FORGET, true, true>(a, m, st) : launch_adjoint<FORGET, false, true>(a, m, st);
-    return bf16out ? launch_adjoint<FORGET, true, false>(a, m, st) : launch_adjoint<FORGET, false, false>(a, m, st);
+    if (tma)
+        return bf16out ? launch_adjoint<FORGET, true, true, VARLEN>(a, m, st)
+                       : launch_adjoint<FORGET, false, true, VARLEN>(a, m, st);
+    return bf16out ? launch_adjoint<FORGET, true, false, VARLEN>(a, m, st)
+                   : launch_adjoint<FORGET, false, false, VARLEN>(a, m, st);
+}
+
+template <int FORGET>
+cudaError_t launch_adjoint_any(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, bool varlen,
+                               cudaStream_t st)
+{
+    return varlen ? launch_adjoint_v<FORGET, true>(a, m, tma, bf16out, st)
+                  : launch_adjoint_v<FORGET, false>(a, m, tma, bf16out, st);
 }
 
 struct Layout {
@@ -561,7 +606,7 @@ size_t backward_workspace_bytes(int B, int T, int d_in, int d_h) { return layout
 cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *R,
                             const float *s0, const float *S, const float *dH, float *dx, float *dWx,
                             float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
-                            int d_h, void *ws, cudaStream_t st)
+                            int d_h, void *ws, cudaStream_t st, const Varlen *vl)
 {
     const Layout l = layout(B, T, d_in, d_h);
     char *base = static_cast<char *>(ws);
@@ -598,6 +643,16 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     // start cleared
     cudaError_t e = cudaMemsetAsync(base, 0, l.agg, st);
     if (e != cudaSuccess) return e;
+    a.vmask = nullptr;
+    a.vseq = nullptr;
+    if (vl) {
+        if ((e = varlen_build(*vl, T, nullptr, nullptr, st)) != cudaSuccess) return e;
+        a.vmask = vl->mask;
+        a.vseq = vl->seq;
+        // empty sequences get a zero ds0; the others are written at their first step
+        if (ds0 && (e = cudaMemsetAsync(ds0, 0, sizeof(float) * 4 * (size_t)d_h * vl->n_seq, st)) != cudaSuccess)
+            return e;
+    }
     // TMA moves the tiles when the rows are 16-byte aligned and every row
     // coordinate fits a signed 32-bit box coordinate
     BwdMaps m;
@@ -607,8 +662,8 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
                      make_map_f32_3d(&m.S, S, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
                      make_map_f32_3d(&m.P, P, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
                      make_map_f32_3d(&m.H, dH, d_h, T, B, d_h, (uint64_t)T * d_h, 32, TT);
-    e = (forget == SLSTM_FORGET_EXP) ? launch_adjoint_any<SLSTM_FORGET_EXP>(a, m, tma, tc, st)
-                                     : launch_adjoint_any<SLSTM_FORGET_SIGMOID>(a, m, tma, tc, st);
+    e = (forget == SLSTM_FORGET_EXP) ? launch_adjoint_any<SLSTM_FORGET_EXP>(a, m, tma, tc, vl != nullptr, st)
+                                     : launch_adjoint_any<SLSTM_FORGET_SIGMOID>(a, m, tma, tc, vl != nullptr, st);
     if (e != cudaSuccess) return e;
     reduce_partials_kernel<<<dim3(l.groups_per_row, 8), 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);

@@ -35,6 +35,13 @@ struct Cell {
     float fp, jcm, jch, jnm, jnh, beta, dmh, jhc, jhn, jhm, jhh;
 };
 
+// The step's Jacobian set to zero: the step does not depend on the one before
+// (the first step of a packed sequence).
+SLSTM_DEVINL void cell_zero_jac(Cell &J)
+{
+    J.fp = J.jcm = J.jch = J.jnm = J.jnh = J.beta = J.dmh = J.jhc = J.jhn = J.jhm = J.jhh = 0.0f;
+}
+
 // Gate-space derivative G = d s_t / d a_t, nonzero pattern (columns z,i,f,o):
 //   [ gcz gci gcf 0   ]
 //   [ 0   gni gnf 0   ]

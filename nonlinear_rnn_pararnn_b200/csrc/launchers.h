@@ -26,10 +26,31 @@ struct NewtonCtrl {
     NewtonSlot slot[2];
 };
 
+// Packed ragged sequences: the head flags of the packed time axis, built on
+// the device from cu_seqlens.  mask[c] bit i: step 32 c + i is the first step
+// of a nonempty sequence, whose index is seq[32 c + i].  err: nonzero when
+// the offsets are malformed.
+struct Varlen {
+    const int *cu;     // the caller's offsets (n_seq + 1)
+    int n_seq;
+    unsigned *mask;    // [ceil(total_T / 32)]
+    int *seq;          // [total_T]
+    unsigned *err;
+};
+size_t varlen_table_bytes(int total_T);
+// Carve the table out of `ws` (varlen_table_bytes(total_T) bytes, 256-aligned).
+Varlen varlen_layout(const int *cu, int n_seq, int total_T, void *ws);
+// Build the table on `st`.  On malformed offsets: *err = 1 and, when given,
+// stats->error = SLSTM_ERR_INVALID_ARG and *done = 1.  Offsets are clamped to
+// [0, total_T] either way.
+cudaError_t varlen_build(const Varlen &v, int total_T, slstm_newton_stats *stats, unsigned *done,
+                         cudaStream_t st);
+
 size_t newton_workspace_bytes(int B, int T, int d);
+// vl: packed ragged sequences (B = 1, T = total_T), or null for B sequences of T.
 cudaError_t newton_forward(const float *P, const float *R, const float *s0, float *S,
                            const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
-                           int d, void *ws, cudaStream_t st);
+                           int d, void *ws, cudaStream_t st, const Varlen *vl = nullptr);
 
 size_t scan_workspace_bytes(int B, int T, int d);
 cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, float *y, int B,
@@ -39,10 +60,11 @@ cudaError_t sequential_launch(const float *P, const float *R, const float *s0, f
                               int T, int d, int forget, cudaStream_t st);
 
 size_t backward_workspace_bytes(int B, int T, int d_in, int d_h);
+// vl: packed ragged sequences (B = 1, T = total_T; s0 and ds0 per sequence).
 cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *R,
                             const float *s0, const float *S, const float *dH, float *dx, float *dWx,
                             float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,
-                            int d_h, void *ws, cudaStream_t st);
+                            int d_h, void *ws, cudaStream_t st, const Varlen *vl = nullptr);
 
 // C[M][N] = sum_k A(m,k) B(k,n) (+ bias[n]) with fp32 accumulation.
 // A(m,k) = A[m*sam + k*sak], B(k,n) = B[k*sbk + n*sbn]; element types as

@@ -95,13 +95,21 @@ SLSTM_DEVINL void store_aff_smem(float (*s_agg)[20][32], int w, int lane, const 
 }
 
 // ---- look-back (warp 0, lane = feature) -------------------------------------
+// Segment heads.  Bit w of `whead` marks a warp map that starts a new segment
+// (packed sequences): it ignores what enters it, so applying or composing it
+// selects its own map instead of multiplying by its zero matrix (a zero
+// matrix times a non-finite carry would not give zero).  A tile aggregate
+// that contains a head is published with FLAG_HEAD, and a look-back that
+// meets one stops there: its offset is that tile's inclusive prefix.
+constexpr unsigned FLAG_HEAD = 2u;
+
 // The predecessor has not published its prefix: publish this tile's
 // aggregate (composed from the warp maps that load(w, x) returns, in
 // processing order) unless `withhold`, then walk back over earlier tiles of
 // the group.  Returns this lane's carry entering the tile in `carry`.
 template <int NW, class LoadMap>
 SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned ticket, int chunk, int grp,
-                                bool withhold, float carry[4])
+                                bool withhold, float carry[4], unsigned whead = 0u)
 {
     const int lane = threadIdx.x & 31;
     Aff tile;
@@ -109,7 +117,8 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
     for (int w = 1; w < NW; ++w) {
         Aff x;
         load(w, x);
-        aff_compose(x, tile, tile);
+        if ((whead >> w) & 1u) tile = x;
+        else aff_compose(x, tile, tile);
     }
     if (!withhold) {
         float *dst = ca.agg + (size_t)ticket * 20 * 32;
@@ -119,7 +128,9 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
         for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = tile.b[e];
         __threadfence();
         __syncwarp();
-        if (lane == 0) st_release(ca.flags + ticket, (ca.epoch << 2) | FLAG_AGG);
+        // with a head inside, successors need not look past this tile (the
+        // warps before the head still take the carry found below)
+        if (lane == 0) st_release(ca.flags + ticket, (ca.epoch << 2) | FLAG_AGG | (whead ? FLAG_HEAD : 0u));
     }
     Aff M;  // composition of the aggregates met so far (latest first)
     aff_identity(M);
@@ -135,13 +146,18 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
             return;
         }
         const unsigned f = ld_acquire(ca.flags + tq);
-        if ((f >> 2) == ca.epoch && (f & 3u) == FLAG_AGG) {
+        if ((f >> 2) == ca.epoch && (f & FLAG_AGG)) {
             Aff x;
             const float *src = ca.agg + (size_t)tq * 20 * 32;
 #pragma unroll
             for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
 #pragma unroll
             for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+            if (f & FLAG_HEAD) {
+                // that tile's prefix is its offset
+                aff_apply(M, x.b, carry);
+                return;
+            }
             aff_compose(M, x, M);
             --q;   // chunk 0 never publishes an aggregate, so q stays >= 0
             continue;
@@ -161,7 +177,7 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
 // tile's inclusive prefix, is published unless `withhold`.
 template <int NW, class LoadMap, class PutCarry>
 SLSTM_DEVINL void carry_serial(const CarryArgs &ca, LoadMap load, PutCarry put, unsigned ticket, bool withhold,
-                               const float carry[4])
+                               const float carry[4], unsigned whead = 0u)
 {
     const int lane = threadIdx.x & 31;
     // the next warp's map is loaded while the current one is applied
@@ -173,7 +189,12 @@ SLSTM_DEVINL void carry_serial(const CarryArgs &ca, LoadMap load, PutCarry put, 
         put(w, v);
         Aff xn;
         if (w + 1 < NW) load(w + 1, xn);
-        aff_apply(x, v, v);
+        if ((whead >> w) & 1u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
+        } else {
+            aff_apply(x, v, v);
+        }
         if (w + 1 < NW) x = xn;
     }
     if (!withhold) {
@@ -394,7 +415,7 @@ SLSTM_DEVINL size_t chain_word(unsigned tq, int warp, int lane)
 // the fused multiply-adds) is that of aff_apply, so both walks give the same
 // bits.
 template <int NW>
-SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane)
+SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane, unsigned whead = 0u)
 {
     const int f = chain_feature(warp, lane);
     const int r = chain_row(lane);
@@ -412,7 +433,8 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
         const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
         const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
         const float v3 = __shfl_sync(0xffffffffu, c, 24 + i8);
-        c = fmaf(a3, v3, fmaf(a2, v2, fmaf(a1, v1, fmaf(a0, v0, bb))));
+        const float nc = fmaf(a3, v3, fmaf(a2, v2, fmaf(a1, v1, fmaf(a0, v0, bb))));
+        c = ((whead >> w) & 1u) ? bb : nc;
     }
     return c;
 }
@@ -422,20 +444,20 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
 // serially (lane = feature).  chunk > 0.
 template <int NW>
 SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, const MapArr *m, CinArr *cin, unsigned ticket, int chunk,
-                                      int grp, bool withhold)
+                                      int grp, bool withhold, unsigned whead = 0u)
 {
     const int lane = threadIdx.x & 31;
     auto load = [&](int w, Aff &x) { maps_load(m, w, lane, x); };
     float carry[4];
     const bool ok = read_inc_words(ca, ticket - (unsigned)ca.n_groups, lane, carry);
-    if (!__all_sync(0xffffffffu, ok)) tile_lookback<NW>(ca, load, ticket, chunk, grp, withhold, carry);
+    if (!__all_sync(0xffffffffu, ok)) tile_lookback<NW>(ca, load, ticket, chunk, grp, withhold, carry, whead);
     carry_serial<NW>(
         ca, load,
         [&](int w, const float v[4]) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) cin[w][e][sw(e, lane)] = v[e];
         },
-        ticket, withhold, carry);
+        ticket, withhold, carry, whead);
 }
 
 // Value component e (slot order c, n, m, h) of a cell evaluation; e is a

@@ -52,6 +52,8 @@ struct Args {
     float *bnd_out;
     slstm_newton_stats *stats;
     unsigned *error;
+    const unsigned *vmask;        // packed sequences: head-flag words (one per chunk), else null
+    const int *vseq;              // packed sequences: sequence index at each head step
     unsigned epoch;
     unsigned long long wait_ns;
     int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
@@ -65,7 +67,8 @@ struct TileInfo {
     int b;
     int j0;
     unsigned long long off;   // element offset of (b, chunk * TT, slot 0, feature j0) in P and S
-    unsigned long long pad;
+    unsigned mask;            // packed sequences: bit i set when step chunk * TT + i starts a sequence
+    unsigned pad;
 };
 
 struct Smem {
@@ -115,6 +118,7 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
     ti.ticket = ticket;
     ti.chunk = ti.b = ti.j0 = 0;
     ti.off = 0;
+    ti.mask = 0u;
     if (ticket < (unsigned)a.n_tiles) {
         const unsigned chunk = ticket / (unsigned)a.n_groups;
         const unsigned grp = ticket - chunk * (unsigned)a.n_groups;
@@ -123,7 +127,16 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
         ti.b = (int)b;
         ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
         ti.off = ((size_t)b * a.T + (size_t)chunk * TT) * 4 * (size_t)a.d + (size_t)ti.j0;
+        if (a.vmask) ti.mask = a.vmask[chunk];
     }
+}
+
+// Packed sequences: the initial state of the sequence that starts at step t.
+SLSTM_DEVINL void head_state(const Args &a, int t, size_t jj, bool jv, float s[4])
+{
+    const size_t k = (size_t)a.vseq[t];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] = (a.s0 && jv) ? __ldg(a.s0 + (k * 4 + e) * (size_t)a.d + jj) : 0.0f;
 }
 
 // Per-thread part of the copy offsets (see prefetch_tile).
@@ -219,7 +232,9 @@ __device__ void finalize(const Args &a, int k, bool resid)
 // TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
 // stage, stores per warp from the stage walk B wrote); otherwise by cp.async
 // and plain stores.
-template <int FORGET, bool FIRST, bool RESID, bool TMA>
+// VARLEN: packed ragged sequences (B = 1); at a head step the previous state is
+// the sequence's s0 and the Jacobian is zero, which makes the scan segmented.
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN>
 __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -308,7 +323,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         // old state just before this warp's segment
         float sp[4] = {0.f, 0.f, 0.f, 0.f};
         if (t_seg == 0) {
-            if (a.s0 && jv) {
+            if (!VARLEN && a.s0 && jv) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sp[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
             }
@@ -353,13 +368,18 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
 #pragma unroll
                     for (int e = 0; e < 4; ++e) so[e] = sm.S[st][sl][e][lane];
                 }
+                const bool head = VARLEN && ((ti.mask >> sl) & 1u);
+                if (head) head_state(a, t_seg + i, jj, jv, curS);
                 cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
                                         sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
                                         rf, ro, Jc[i]);
+                if (head) cell_zero_jac(Jc[i]);
                 const float r[4] = {Jc[i].c - so[0], Jc[i].n - so[1], Jc[i].m - so[2], Jc[i].h - so[3]};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) curS[e] = so[e];
-                if (i == 0) affp_from_cell<false>(agg, Jc[0], r);
+                // a head starts the warp's map afresh: select, never multiply
+                // what came before by its zero Jacobian
+                if (i == 0 || head) affp_from_cell<false>(agg, Jc[i], r);
                 else fold_p<false>(agg, Jc[i], r);
             }
         }
@@ -379,15 +399,22 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
             }
         }
         const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
+        // warps whose steps contain a sequence start (packed sequences)
+        unsigned whead = 0u;
+        if (VARLEN) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) whead |= (((ti.mask >> (w * L)) & ((1u << L) - 1u)) != 0u) ? (1u << w) : 0u;
+        }
         const bool fast = __syncthreads_and(ok);
         if (fast) {
             if (chain_warp) {
-                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane);
+                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead);
                 if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
             }
         } else if (warp == 0) {
             const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-            tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold);
+            tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold,
+                                    whead);
         }
         __syncthreads();
 
@@ -410,6 +437,11 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         for (int i = 0; i < L; ++i) {
             const int sl = warp * L + i;
             const bool wr = jv && (t_seg + i < T);
+            if (VARLEN && ((ti.mask >> sl) & 1u)) {
+                // a sequence starts here: nothing from before enters it
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
+            }
             // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
             const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
             float sn[4];
@@ -430,6 +462,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
                     if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
             }
             if (RESID) {
+                if (VARLEN && ((ti.mask >> sl) & 1u)) head_state(a, t_seg + i, jj, jv, snp);
                 Cell f;
                 cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
                                          sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
@@ -501,10 +534,10 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
     }
 }
 
-template <int FORGET, bool FIRST, bool RESID, bool TMA>
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN>
 cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = newton_iter<FORGET, FIRST, RESID, TMA>;
+    auto kern = newton_iter<FORGET, FIRST, RESID, TMA, VARLEN>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -518,7 +551,7 @@ cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaS
     return cudaGetLastError();
 }
 
-template <int FORGET, bool TMA>
+template <int FORGET, bool TMA, bool VARLEN>
 cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, int sms, cudaStream_t st)
 {
     for (int k = 0; k < max_iters; ++k) {
@@ -529,11 +562,11 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         const bool resid = !fixed || (k + 1 == max_iters);
         cudaError_t e;
         if (k == 0)
-            e = resid ? launch_one<FORGET, true, true, TMA>(a, m, k, sms, st)
-                      : launch_one<FORGET, true, false, TMA>(a, m, k, sms, st);
+            e = resid ? launch_one<FORGET, true, true, TMA, VARLEN>(a, m, k, sms, st)
+                      : launch_one<FORGET, true, false, TMA, VARLEN>(a, m, k, sms, st);
         else
-            e = resid ? launch_one<FORGET, false, true, TMA>(a, m, k, sms, st)
-                      : launch_one<FORGET, false, false, TMA>(a, m, k, sms, st);
+            e = resid ? launch_one<FORGET, false, true, TMA, VARLEN>(a, m, k, sms, st)
+                      : launch_one<FORGET, false, false, TMA, VARLEN>(a, m, k, sms, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -579,13 +612,21 @@ int sm_count()
     return n;
 }
 
+template <int FORGET, bool TMA>
+cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, bool fixed, int sms, bool varlen,
+                             cudaStream_t st)
+{
+    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, sms, st)
+                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, sms, st);
+}
+
 }  // namespace
 
 size_t newton_workspace_bytes(int B, int T, int d) { return layout(B, T, d).total; }
 
 cudaError_t newton_forward(const float *P, const float *R, const float *s0, float *S,
                            const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
-                           int d, void *ws, cudaStream_t st)
+                           int d, void *ws, cudaStream_t st, const Varlen *vl)
 {
     const Layout l = layout(B, T, d);
     char *base = static_cast<char *>(ws);
@@ -624,6 +665,14 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     cudaError_t e = cudaMemsetAsync(base + l.ctrl, 0, l.agg - l.ctrl, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(slstm_newton_stats), st);
     if (e != cudaSuccess) return e;
+    a.vmask = nullptr;
+    a.vseq = nullptr;
+    if (vl) {
+        // malformed offsets mark the call done before any iteration runs
+        if ((e = varlen_build(*vl, T, stats, &a.ctrl->done, st)) != cudaSuccess) return e;
+        a.vmask = vl->mask;
+        a.vseq = vl->seq;
+    }
     const int sms = sm_count();
     // TMA moves the tiles when the rows are 16-byte aligned and every row
     // coordinate fits a signed 32-bit box coordinate
@@ -634,11 +683,12 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
                      make_map_f32_3d(&m.P, P, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);
+    const bool v = vl != nullptr;
     if (cfg.forget == SLSTM_FORGET_EXP)
-        return tma ? launch_iters<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, sms, st)
-                   : launch_iters<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, sms, st);
-    return tma ? launch_iters<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, sms, st)
-               : launch_iters<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, sms, st);
+        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, sms, v, st)
+                   : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, sms, v, st);
+    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, sms, v, st)
+               : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, sms, v, st);
 }
 
 }  // namespace slstm

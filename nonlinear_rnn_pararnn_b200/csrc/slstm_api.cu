@@ -27,6 +27,12 @@ bool sizes_ok(int B, int T, int d_a, int d_b)
     return tiles <= kIndexLimit;
 }
 
+// Packed sequences: n_seq sequences over total_T packed steps (one batch row).
+bool varlen_sizes_ok(int n_seq, int total_T, int d_a, int d_b)
+{
+    return n_seq >= 1 && n_seq <= total_T && sizes_ok(1, total_T, d_a, d_b);
+}
+
 bool ws_ok(void *ws, size_t have, size_t need)
 {
     if (need == 0) return true;
@@ -67,6 +73,12 @@ size_t slstm_workspace_size(int op, int B, int T, int d_in, int d_h)
     case SLSTM_OP_NEWTON_BACKWARD:
         if (!sizes_ok(B, T, d_in, d_h)) return 0;
         return backward_workspace_bytes(B, T, d_in, d_h);
+    case SLSTM_OP_NEWTON_FORWARD_VARLEN:
+        if (!varlen_sizes_ok(B, T, d_h, d_h)) return 0;
+        return varlen_table_bytes(T) + newton_workspace_bytes(1, T, d_h);
+    case SLSTM_OP_NEWTON_BACKWARD_VARLEN:
+        if (!varlen_sizes_ok(B, T, d_in, d_h)) return 0;
+        return varlen_table_bytes(T) + backward_workspace_bytes(1, T, d_in, d_h);
     default: return 0;
     }
 }
@@ -136,6 +148,47 @@ int slstm_newton_backward(const void *x, const void *Wx, int dtype, const float 
     if (!ws_ok(ws, ws_bytes, backward_workspace_bytes(B, T, d_in, d_h))) return SLSTM_ERR_INVALID_ARG;
     return cuda_status(backward_launch(x, Wx, dtype, P, R, s0, S, dH, dx, dWx, dR, db, ds0, forget, B, T,
                                        d_in, d_h, ws, static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_newton_forward_varlen(const float *P, const float *R, const float *s0, const int *cu_seqlens, int n_seq,
+                                float *S, const slstm_newton_config *cfg, slstm_newton_stats *stats, int total_T,
+                                int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (cfg == nullptr || cu_seqlens == nullptr) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
+    if (!varlen_sizes_ok(n_seq, total_T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
+        return SLSTM_ERR_INVALID_ARG;
+    const size_t vt = varlen_table_bytes(total_T);
+    if (!ws_ok(ws, ws_bytes, vt + newton_workspace_bytes(1, total_T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    const Varlen vl = varlen_layout(cu_seqlens, n_seq, total_T, ws);
+    return cuda_status(newton_forward(P, R, s0, S, *cfg, stats, 1, total_T, d_h, static_cast<char *>(ws) + vt,
+                                      static_cast<cudaStream_t>(stream), &vl));
+}
+
+int slstm_newton_backward_varlen(const void *x, const void *Wx, int dtype, const float *P, const float *R,
+                                 const float *s0, const int *cu_seqlens, int n_seq, const float *S,
+                                 const float *dH, float *dx, float *dWx, float *dR, float *db, float *ds0,
+                                 int forget, int total_T, int d_in, int d_h, void *ws, size_t ws_bytes,
+                                 slstm_stream_t stream)
+{
+    if (dtype != SLSTM_F32 && dtype != SLSTM_BF16) return SLSTM_ERR_INVALID_ARG;
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (cu_seqlens == nullptr || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return SLSTM_ERR_INVALID_ARG;
+    if (!varlen_sizes_ok(n_seq, total_T, d_in, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wx) || !aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) ||
+        !aligned16(S) || !aligned16(dH) || !aligned16(dx) || !aligned16(dWx) || !aligned16(dR) ||
+        !aligned16(db) || !aligned16_or_null(ds0))
+        return SLSTM_ERR_INVALID_ARG;
+    const size_t vt = varlen_table_bytes(total_T);
+    if (!ws_ok(ws, ws_bytes, vt + backward_workspace_bytes(1, total_T, d_in, d_h))) return SLSTM_ERR_INVALID_ARG;
+    const Varlen vl = varlen_layout(cu_seqlens, n_seq, total_T, ws);
+    return cuda_status(backward_launch(x, Wx, dtype, P, R, s0, S, dH, dx, dWx, dR, db, ds0, forget, 1, total_T,
+                                       d_in, d_h, static_cast<char *>(ws) + vt, static_cast<cudaStream_t>(stream),
+                                       &vl));
 }
 
 }  // extern "C"

@@ -1,0 +1,144 @@
+"""GPU parity of the packed ragged-sequence entry points (cu_seqlens) against
+the fp64 oracle, which solves every sequence on its own.
+
+Lengths mix empty sequences, single steps, sequences shorter than a tile and
+sequences that cross several 32-step tiles, so that tiles start and end in
+the middle of sequences and several sequences start inside one tile.  d = 40
+takes the TMA tile path, d = 33 and d = 18 the cp.async one.  Tolerances as
+in test_gpu_parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from nonlinear_rnn_pararnn_b200 import api
+from nonlinear_rnn_pararnn_b200.workloads import Workload, as_f64, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+
+
+def _dev(t):
+    return None if t is None else t.to("cuda").contiguous()
+
+
+def _case(lengths, d, d_in, dtype, forget, seed):
+    """Packed inputs: x (total_T, d_in), W_x, bias, R, dH (total_T, d), s0 (n, 4, d), cu (n + 1,)."""
+    total = int(sum(lengths))
+    w = Workload("v", 1, total, d_in, d, dtype, forget, 0.5, seed, 1e-6, 64)
+    inp = make_inputs(w, with_dH=True)
+    g = torch.Generator().manual_seed(seed + 1000)
+    n = len(lengths)
+    s0 = torch.stack([torch.randn(n, d, generator=g), torch.rand(n, d, generator=g) + 0.5,
+                      torch.randn(n, d, generator=g), torch.rand(n, d, generator=g) - 0.5], dim=1)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32)
+    return {"x": inp["x"][0], "Wx": inp["Wx"], "bias": inp["bias"], "R": inp["R"], "dH": inp["dH"][0],
+            "s0": s0, "cu": cu}
+
+
+def _preact(c):
+    P = api.preact_gemm(_dev(c["x"])[None], _dev(c["Wx"]), _dev(c["bias"]))[0].contiguous()
+    Pref = oracle.preact(as_f64(c["x"])[None], as_f64(c["Wx"]), as_f64(c["bias"]))[0]
+    return P, Pref
+
+
+def _h_err(S_gpu, S_ref):
+    h = S_ref[:, 3, :]
+    return float((np.abs(S_gpu[:, 3, :] - h) / (1 + np.abs(h))).max())
+
+
+LENGTHS = [[5, 0, 1, 40, 33, 64, 7, 0], [70, 3], [32, 32, 32], [1, 1, 1, 1, 1], [17]]
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("d", [40, 33])
+@pytest.mark.parametrize("lengths", LENGTHS)
+def test_varlen_fixed_k_matches_oracle(lengths, d, forget, cuda_device):
+    K = 3
+    c = _case(lengths, d, 12, "f32", forget, 41)
+    P, Pref = _preact(c)
+    S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), forget=forget, max_iters=K,
+                                      fixed=True, tol=1e-6)
+    torch.cuda.synchronize()
+    got = as_f64(S.cpu())
+    assert api.read_stats(st)["iters"] == K
+    # The iterate after K steps from the zero guess is far from the solution
+    # and amplifies rounding (as in the dense fixed-K tests, only what fp32
+    # pins is compared).  Newton's prefix exactness, per sequence: after K
+    # iterations the first K steps of every sequence are the sequential
+    # trajectory; a carry leaking across a sequence start would break it.
+    seq = oracle.sequential_varlen(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy(), forget)
+    cu = c["cu"].numpy()
+    for k in range(len(lengths)):
+        a = int(cu[k])
+        b = min(int(cu[k + 1]), a + K)
+        if b > a:
+            assert _h_err(got[a:b], seq[a:b]) <= TOL_F32, (k, a, b)
+
+
+@pytest.mark.parametrize("d", [40, 33])
+def test_varlen_converges_to_sequential(d, cuda_device):
+    lengths = [12, 0, 1, 40, 33, 9]
+    c = _case(lengths, d, 16, "f32", "sigmoid", 42)
+    P, Pref = _preact(c)
+    S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), max_iters=64, tol=1e-6)
+    torch.cuda.synchronize()
+    s = api.read_stats(st)
+    assert s["error"] == 0 and s["converged"], s
+    ref = oracle.sequential_varlen(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy())
+    assert _h_err(as_f64(S.cpu()), ref) <= TOL_F32
+
+
+def test_varlen_equal_lengths_matches_batched(cuda_device):
+    B, T, d = 3, 50, 40
+    c = _case([T] * B, d, 16, "f32", "sigmoid", 43)
+    P, _ = _preact(c)
+    R, s0 = _dev(c["R"]), _dev(c["s0"])
+    # converged solutions (fixed-K iterates amplify the different rounding
+    # order of packed and batched tiles)
+    Sv, stv = api.newton_forward_varlen(P, R, s0, _dev(c["cu"]), max_iters=64, tol=1e-6)
+    Sb, stb = api.newton_forward(P.view(B, T, 4, d), R, s0, max_iters=64, tol=1e-6)
+    torch.cuda.synchronize()
+    assert api.read_stats(stv)["converged"] and api.read_stats(stb)["converged"]
+    a, b = as_f64(Sv.cpu()).reshape(B, T, 4, d), as_f64(Sb.cpu())
+    assert float((np.abs(a - b) / (1 + np.abs(b))).max()) <= TOL_F32
+
+
+@pytest.mark.parametrize("bad", [[0, 5, 3, 10], [0, 4, 9], [1, 4, 10]])
+def test_varlen_malformed_offsets_report_invalid_arg(bad, cuda_device):
+    total, d = 10, 8
+    c = _case([total], d, 8, "f32", "sigmoid", 44)
+    P, _ = _preact(c)
+    cu = torch.tensor(bad, dtype=torch.int32, device="cuda")
+    n = len(bad) - 1
+    s0 = torch.zeros(n, 4, d, device="cuda")
+    S = torch.full_like(P, float("nan"))
+    S, st = api.newton_forward_varlen(P, _dev(c["R"]), s0, cu, max_iters=3, S=S)
+    torch.cuda.synchronize()
+    s = api.read_stats(st)
+    assert s["error"] == 1 and s["iters"] == 0, s     # SLSTM_ERR_INVALID_ARG, nothing ran
+    assert torch.isnan(S).all()                       # S untouched
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("d_in,d,dtype", [(12, 40, "f32"), (16, 40, "bf16"), (16, 18, "bf16")])
+def test_varlen_backward_matches_oracle(d_in, d, dtype, forget, cuda_device):
+    lengths = [5, 0, 1, 40, 33, 36, 7, 0]
+    c = _case(lengths, d, d_in, dtype, forget, 45)
+    P, Pref = _preact(c)
+    cu = c["cu"].numpy()
+    Sref = oracle.sequential_varlen(Pref, as_f64(c["R"]), as_f64(c["s0"]), cu, forget)
+    S = torch.from_numpy(Sref).float().cuda()
+    out = api.newton_backward_varlen(_dev(c["x"]), _dev(c["Wx"]), P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]),
+                                     S, _dev(c["dH"]), forget=forget)
+    torch.cuda.synchronize()
+    ref = oracle.backward_varlen(as_f64(c["x"]), as_f64(c["Wx"]), Pref, as_f64(c["R"]), as_f64(c["s0"]), Sref,
+                                 as_f64(c["dH"]), cu, forget)
+    for k in ("dx", "dWx", "dR", "db", "ds0"):
+        got = as_f64(out[k].cpu())
+        err = np.abs(got - ref[k]).max() / (1 + np.abs(ref[k]).max())
+        assert err <= 1e-4, (k, err)
+    # empty sequences get exactly zero
+    assert not out["ds0"][1].any() and not out["ds0"][7].any()
