@@ -424,6 +424,80 @@ def run_scan(args):
     return 0
 
 
+def run_varlen(args, w):
+    """Packed ragged sequences: the workload's B*T steps repacked into sequences whose lengths are
+    drawn (seeded) uniformly from [T/8, 2T), the last one cut to fit; the same inputs, each
+    sequence from s0 = 0.  A step is the input-projection GEMM, K fixed Newton iterations and the
+    backward, all through the packed entry points."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+    _, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    K = args.newton_iters
+    total = w.B * w.T
+    rng = np.random.default_rng(7)
+    lengths = []
+    while sum(lengths) < total:
+        lengths.append(int(rng.integers(max(1, w.T // 8), 2 * w.T)))
+    lengths[-1] -= sum(lengths) - total
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device=dev)
+    n_seq = len(lengths)
+    inp = make_inputs(w)
+    x = inp["x"].reshape(total, w.d_in).to(dev)
+    Wx, R, bias = inp["Wx"].to(dev), inp["R"].to(dev), inp["bias"].to(dev)
+    dH = inp["dH"].reshape(total, w.d_h).to(dev)
+    s0 = torch.zeros(n_seq, 4, w.d_h, device=dev)
+    P = torch.empty(1, total, 4, w.d_h, device=dev)
+    S = torch.empty(total, 4, w.d_h, device=dev)
+    stats = api.new_stats(dev)
+    ws_f = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total, 0, w.d_h, dev)
+    ws_b = api.workspace(_lib.SLSTM_OP_NEWTON_BACKWARD_VARLEN, n_seq, total, w.d_in, w.d_h, dev)
+    grads = {"dx": torch.empty(total, w.d_in, device=dev), "dWx": torch.empty(4 * w.d_h, w.d_in, device=dev),
+             "dR": torch.empty(4, w.d_h, device=dev), "db": torch.empty(4, w.d_h, device=dev),
+             "ds0": torch.empty(n_seq, 4, w.d_h, device=dev)}
+
+    def step(ev=None):
+        api.preact_gemm(x[None], Wx, bias, P=P)
+        if ev is not None:
+            ev[0].record()
+        api.newton_forward_varlen(P[0], R, s0, cu, forget=w.forget, max_iters=K, fixed=True, tol=w.tol, S=S,
+                                  stats=stats, ws=ws_f)
+        if ev is not None:
+            ev[1].record()
+        api.newton_backward_varlen(x, Wx, P[0], R, s0, cu, S, dH, forget=w.forget, out=grads, ws=ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        step(evs[i])
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    newton_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps / K
+    hbm, peak_kind = _peaks()
+    nbytes = total * w.d_h * (32 + 48 * (K - 1)) / K
+    gbs = nbytes / (newton_ms / 1e3) / 1e9
+    st = api.read_stats(stats)
+    line = {"metric": METRIC + ", packed ragged sequences", "value": total * w.d_h / (ms / 1e3), "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{w.name}_packed", "total_T": total, "n_seq": n_seq,
+                       "lengths": f"uniform integers in [{max(1, w.T // 8)}, {2 * w.T}), seed 7, last cut to fit",
+                       "d_in": w.d_in, "d_h": w.d_h, "x_dtype": w.dtype, "forget": w.forget, "newton_iters": K,
+                       "newton_mode": "fixed", "l2": "inputs larger than L2"},
+            "roofline": {"kernel": "newton_iter (packed)", "bound": "hbm", "achieved": gbs, "peak": hbm,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm, "traffic": None,
+                         "avg_launch_ms": newton_ms},
+            "newton_stats": {"iters": st["iters"], "error": st["error"]}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
 # last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
@@ -462,9 +536,10 @@ def main(argv=None):
     ap.add_argument("--cpu-lanes", type=int, default=40)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan"],
+    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen"],
                     help="train: GEMM + Newton + backward (default); forward: GEMM + Newton; "
-                         "scan: scan_block4 alone over T in --scan-T at B=4, d=2048")
+                         "scan: scan_block4 alone over T in --scan-T at B=4, d=2048; "
+                         "varlen: the workload repacked into ragged sequences (cu_seqlens)")
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
@@ -486,6 +561,8 @@ def main(argv=None):
         return run_reference(args, w)
     if args.mode == "scan":
         return run_scan(args)
+    if args.mode == "varlen":
+        return run_varlen(args, w)
     return run_gpu(args, w)
 
 
