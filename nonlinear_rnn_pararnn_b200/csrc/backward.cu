@@ -41,6 +41,7 @@ struct BwdArgs {
     const unsigned *vmask;   // packed sequences: head-flag words (one per 32 steps), else null
     const int *vseq;         // packed sequences: sequence index at each head step
     int T, d, groups_per_row, n_tiles, vec16, dpt_vec8;
+    FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
 // A ticket decoded once (by thread 0) for the whole CTA.  The tile covers
@@ -90,9 +91,9 @@ SLSTM_DEVINL void bwd_decode(const BwdArgs &a, unsigned ticket, BwdInfo &ti)
     ti.hmask = 0ull;
     if (ticket < (unsigned)a.n_tiles) {
         const unsigned G = (unsigned)a.ca.n_groups;
-        const unsigned chunk = ticket / G;
+        const unsigned chunk = fast_div(ticket, a.div_groups);
         const unsigned grp = ticket - chunk * G;
-        const unsigned b = grp / (unsigned)a.groups_per_row;
+        const unsigned b = fast_div(grp, a.div_gpr);
         ti.chunk = (int)chunk;
         ti.b = (int)b;
         ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
@@ -635,6 +636,8 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.T = T;
     a.d = d_h;
     a.groups_per_row = l.groups_per_row;
+    a.div_groups = make_fastdiv((unsigned)l.n_groups);
+    a.div_gpr = make_fastdiv((unsigned)l.groups_per_row);
     a.n_tiles = l.n_tiles;
     a.dpt_vec8 = (T % 4 == 0) ? 1 : 0;   // 8-byte pieces of the transposed pair stay aligned
     a.vec16 = ((d_h & 3) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0 &&

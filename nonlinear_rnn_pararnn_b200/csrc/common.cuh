@@ -255,6 +255,33 @@ SLSTM_DEVINL uint64_t globaltimer_ns()
     return t;
 }
 
+// Division by a divisor d >= 1 that is fixed for a launch, for dividends below
+// 2^31: q = (n * M) >> (32 + s) with s = ceil(log2 d) and the round-up
+// multiplier M = ceil(2^(32+s) / d) < 2^33 (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994).  Turns the
+// per-tile ticket decode into a multiply and a shift.
+struct FastDiv {
+    unsigned long long mul;
+    unsigned shift;
+    unsigned d;
+};
+
+inline FastDiv make_fastdiv(unsigned d)
+{
+    unsigned s = 0;
+    while ((1ull << s) < d) ++s;
+    FastDiv f;
+    f.mul = ((1ull << (32 + s)) + d - 1) / d;
+    f.shift = 32 + s;
+    f.d = d;
+    return f;
+}
+
+SLSTM_DEVINL unsigned fast_div(unsigned n, const FastDiv &f)
+{
+    return (unsigned)(((unsigned long long)n * f.mul) >> f.shift);
+}
+
 // Non-negative float max through its bit pattern (NaN sorts above +inf).
 SLSTM_DEVINL void atomic_max_nonneg(unsigned *slot, float v)
 {

@@ -58,6 +58,7 @@ struct Args {
     unsigned long long wait_ns;
     int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
     float tol;
+    FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
 // A ticket decoded once (by thread 0) for the whole CTA.
@@ -120,9 +121,9 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
     ti.off = 0;
     ti.mask = 0u;
     if (ticket < (unsigned)a.n_tiles) {
-        const unsigned chunk = ticket / (unsigned)a.n_groups;
+        const unsigned chunk = fast_div(ticket, a.div_groups);
         const unsigned grp = ticket - chunk * (unsigned)a.n_groups;
-        const unsigned b = grp / (unsigned)a.groups_per_row;
+        const unsigned b = fast_div(grp, a.div_gpr);
         ti.chunk = (int)chunk;
         ti.b = (int)b;
         ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
@@ -650,6 +651,8 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     a.d = d;
     a.groups_per_row = l.groups_per_row;
     a.n_groups = l.n_groups;
+    a.div_groups = make_fastdiv((unsigned)l.n_groups);
+    a.div_gpr = make_fastdiv((unsigned)l.groups_per_row);
     a.n_tiles = l.n_tiles;
     a.max_iters = cfg.max_iters;
     a.fixed = cfg.fixed_iters ? 1 : 0;

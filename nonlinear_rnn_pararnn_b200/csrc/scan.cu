@@ -32,6 +32,7 @@ struct ScanArgs {
     unsigned *ticket;
     CarryArgs ca;
     int T, d, groups_per_row, n_tiles, vec16;
+    FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
 struct ScanSmem {
@@ -56,10 +57,10 @@ SLSTM_DEVINL void scan_prefetch(const ScanArgs &a, ScanSmem &sm, int st, unsigne
 {
     if (ticket >= (unsigned)a.n_tiles) return;
     const int G = a.ca.n_groups;
-    const int chunk = (int)(ticket / (unsigned)G);
-    const int grp = (int)(ticket % (unsigned)G);
-    const int bb = grp / a.groups_per_row;
-    const int j0 = (grp % a.groups_per_row) * 32;
+    const int chunk = (int)fast_div(ticket, a.div_groups);
+    const int grp = (int)(ticket - (unsigned)chunk * (unsigned)G);
+    const int bb = (int)fast_div((unsigned)grp, a.div_gpr);
+    const int j0 = (grp - bb * a.groups_per_row) * 32;
     const int T = a.T;
     const size_t d = (size_t)a.d;
     const size_t row0 = (size_t)bb * T;
@@ -141,10 +142,10 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
         __syncthreads();
 
         const unsigned ticket = cur;
-        const int chunk = (int)(ticket / (unsigned)G);
-        const int grp = (int)(ticket % (unsigned)G);
-        const int bb = grp / a.groups_per_row;
-        const int j = (grp % a.groups_per_row) * 32 + lane;
+        const int chunk = (int)fast_div(ticket, a.div_groups);
+        const int grp = (int)(ticket - (unsigned)chunk * (unsigned)G);
+        const int bb = (int)fast_div((unsigned)grp, a.div_gpr);
+        const int j = (grp - bb * a.groups_per_row) * 32 + lane;
         const bool jv = j < a.d;
         const size_t jj = jv ? (size_t)j : 0;
         const size_t row0 = (size_t)bb * T;
@@ -280,6 +281,8 @@ cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, 
     a.T = T;
     a.d = d;
     a.groups_per_row = l.groups_per_row;
+    a.div_groups = make_fastdiv((unsigned)l.n_groups);
+    a.div_gpr = make_fastdiv((unsigned)l.groups_per_row);
     a.n_tiles = l.n_tiles;
     a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(A) & 15) == 0 &&
                (reinterpret_cast<uintptr_t>(b) & 15) == 0) ? 1 : 0;
