@@ -503,7 +503,7 @@ def run_varlen(args, w):
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
 # this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
 # (every tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "bcf8928af9c19e747b45a6a0c09c7e52bb16cb3270ce693cfa511b5f66e41be1", "first": 31.66, "middle": 48.28, "last": 48.05}
+NEWTON_TRAFFIC = {"sources_sha256": "55d62befc76fd9daab62999b316cfe2b8898b2f92412aee6ae4a39a2d10f36fd", "first": 31.76, "middle": 48.38, "last": 48.09}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
