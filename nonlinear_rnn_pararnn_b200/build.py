@@ -51,13 +51,28 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    """Compile every source to an object in parallel (one nvcc per file),
+    then link the shared library; objects live in a temporary folder."""
     if not force and not verbose_ptxas and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
-    if verbose_ptxas:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.check_call(cmd)
+    import concurrent.futures
+    import tempfile
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    with tempfile.TemporaryDirectory(prefix="slstm_build_") as tmpdir:
+        def compile_one(src):
+            obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
+            cmd = [_nvcc(), *compile_flags, "-I", INCLUDE, "-c", "-o", obj, src]
+            if verbose_ptxas:
+                cmd.insert(1, "-Xptxas=-v")
+            subprocess.check_call(cmd)
+            return obj
+        srcs = sources()
+        workers = max(1, min(len(srcs), os.cpu_count() or 1))
+        with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+            objs = list(pool.map(compile_one, srcs))
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler",
+                               "-fPIC", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 
