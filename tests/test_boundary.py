@@ -112,6 +112,42 @@ def test_other_entry_points_reject_bad_arguments():
     assert lib.slstm_newton_backward(args[0], args[1], 5, *args[2:12], 0, 2, 8, 8, 8, FAKE, big, NULL) == E
 
 
+def test_varlen_entry_points_reject_bad_arguments():
+    lib = _lib.load()
+    E = _lib.SLSTM_ERR_INVALID_ARG
+    big = ctypes.c_size_t(1 << 40)
+    cu = FAKE
+
+    def fwd(P=FAKE, R=FAKE, s0=NULL, cu=cu, n=3, S=FAKE, cfg=None, stats=FAKE, total=64, d=8, wb=big):
+        c = cfg if cfg is not None else _cfg()
+        return lib.slstm_newton_forward_varlen(P, R, s0, cu, n, S, ctypes.byref(c), stats, total, d, FAKE, wb, NULL)
+
+    assert fwd(cu=NULL) == E                          # offsets missing
+    assert fwd(cu=ctypes.c_void_p(0x10002)) == E      # offsets not int32-aligned
+    assert fwd(n=0) == E
+    assert fwd(n=65, total=64) == E                   # more sequences than steps
+    assert fwd(total=0) == E
+    assert fwd(S=FAKE_MIS) == E
+    assert fwd(cfg=_cfg(max_iters=0)) == E
+    assert fwd(wb=ctypes.c_size_t(64)) == E
+    assert lib.slstm_newton_forward_varlen(FAKE, FAKE, NULL, cu, 3, FAKE, None, FAKE, 64, 8, FAKE, big, NULL) == E
+    # (x, Wx, dtype, P, R, s0, cu, n_seq, S, dH, dx, dWx, dR, db, ds0, forget, total_T, d_in, d_h, ws, bytes, stream)
+
+    def bwd(dtype=0, cu=cu, n=3, forget=0, total=64, d_in=8, d=8, ds0=NULL):
+        return lib.slstm_newton_backward_varlen(FAKE, FAKE, dtype, FAKE, FAKE, NULL, cu, n, FAKE, FAKE, FAKE, FAKE,
+                                                FAKE, FAKE, ds0, forget, total, d_in, d, FAKE, big, NULL)
+    assert bwd(dtype=5) == E
+    assert bwd(forget=3) == E
+    assert bwd(cu=NULL) == E
+    assert bwd(n=0) == E
+    assert bwd(total=0) == E
+    assert bwd(ds0=FAKE_MIS) == E
+    ws_f = lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, 3, 64, 0, 8)
+    assert ws_f > lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD, 1, 64, 0, 8)
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, 65, 64, 0, 8) == 0
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_NEWTON_BACKWARD_VARLEN, 3, 64, 8, 8) > 0
+
+
 def test_python_binding_validates_before_calling():
     import torch
     from nonlinear_rnn_pararnn_b200 import api
