@@ -503,7 +503,7 @@ def run_varlen(args, w):
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
 # this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
 # (every tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "55d62befc76fd9daab62999b316cfe2b8898b2f92412aee6ae4a39a2d10f36fd", "first": 31.76, "middle": 48.38, "last": 48.09}
+NEWTON_TRAFFIC = {"sources_sha256": "864dde235fc834f99aa72eb7e382b0fcdcd60028a8cfcce2897b27e2be3ba221", "first": 31.76, "middle": 48.38, "last": 48.09}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 

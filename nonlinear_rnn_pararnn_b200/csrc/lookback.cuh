@@ -335,18 +335,6 @@ SLSTM_DEVINL void affp_from_cell(AffP &x, const Cell &J, const float r[4])
     for (int e = 0; e < 4; ++e) x.b[e] = r[e];
 }
 
-SLSTM_DEVINL void affp_to_aff(const AffP &p, Aff &x)
-{
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        x.a[r * 4 + 0] = p.a01[r].x;
-        x.a[r * 4 + 1] = p.a01[r].y;
-        x.a[r * 4 + 2] = p.a23[r].x;
-        x.a[r * 4 + 3] = p.a23[r].y;
-        x.b[r] = p.b[r];
-    }
-}
-
 // ---- chain layout -------------------------------------------------------------
 // Row length of TileMaps.  Feature f of row r sits at position f ^ (8 r)
 // (sw(r, f)): a row written by 32 feature lanes is a permutation of 32 banks,
@@ -460,15 +448,6 @@ SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, const MapArr *m, CinA
         ticket, withhold, carry, whead);
 }
 
-// Value component e (slot order c, n, m, h) of a cell evaluation; e is a
-// compile-time constant after unrolling.
-SLSTM_DEVINL float cell_f(const Cell &c, int e) { return e == 0 ? c.c : (e == 1 ? c.n : (e == 2 ? c.m : c.h)); }
-
-// Named CTA barriers for a producer warp handing a value to a consumer warp:
-// the producer arrives, the consumer waits; `n` counts both warps' threads.
-SLSTM_DEVINL void named_bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-SLSTM_DEVINL void named_bar_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
 // cp.async copies into shared memory (zero-fill beyond `bytes`).
 SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -487,53 +466,5 @@ SLSTM_DEVINL void cp_async4(void *dst, const void *src, int bytes)
 SLSTM_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 SLSTM_DEVINL void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 SLSTM_DEVINL void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-// Copy one row of 32 consecutive floats (src, 16-byte aligned when vec16)
-// into shared memory; only `valid` leading floats are read, the rest become
-// zero.  Called by 8 lanes (vec16: 16 bytes each) or 32 lanes (4 bytes each);
-// `part` is the caller's index within that group.
-SLSTM_DEVINL void copy_row32(float *dst, const float *src, int valid, bool vec16, int part)
-{
-    if (vec16) {
-        const int f0 = 4 * part;
-        const int bytes = valid > f0 ? 4 * min(4, valid - f0) : 0;
-        cp_async16(dst + f0, bytes ? src + f0 : src, bytes);
-    } else {
-        const int bytes = valid > part ? 4 : 0;
-        cp_async4(dst + part, bytes ? src + part : src, bytes);
-    }
-}
-
-// Fold one step's map (J, r) into a running aggregate: agg <- (J, r) o agg.
-SLSTM_DEVINL void fold_jac(Aff &agg, const Cell &J, const float r[4])
-{
-#pragma unroll
-    for (int col = 0; col < 4; ++col)
-        jac_mul(J, agg.a[col], agg.a[4 + col], agg.a[8 + col], agg.a[12 + col]);
-    jac_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
-}
-
-// Same with the transposed Jacobian: agg <- (J^T, r) o agg.
-SLSTM_DEVINL void fold_jacT(Aff &agg, const Cell &J, const float r[4])
-{
-#pragma unroll
-    for (int col = 0; col < 4; ++col)
-        jacT_mul(J, agg.a[col], agg.a[4 + col], agg.a[8 + col], agg.a[12 + col]);
-    jacT_mul(J, agg.b[0], agg.b[1], agg.b[2], agg.b[3]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) agg.b[e] += r[e];
-}
-
-SLSTM_DEVINL void cell_identity(Cell &J)
-{
-    J.fp = 1.0f;
-    J.jcm = J.jch = J.jnm = J.jnh = 0.0f;
-    J.beta = 1.0f;
-    J.dmh = 0.0f;
-    J.jhc = J.jhn = J.jhm = 0.0f;
-    J.jhh = 1.0f;
-}
 
 }  // namespace slstm
