@@ -4,8 +4,8 @@
 // "Cell": the fused diag training cell runs Newton with a 4x4 Jacobian per
 // feature and an O(d) combine; "pararnn-torch structure", section "Current
 // surface": fused kernels prepend h0, residual early stop, divergence after
-// K).  The iteration is tiled: a tile is 32 features x 32 steps, handled by
-// one CTA of 8 warps (lane = feature, warp = 4 consecutive steps).
+// K).  The iteration is tiled: a tile is 32 features x 64 steps, handled by
+// one CTA of 16 warps (lane = feature, warp = 4 consecutive steps).
 //
 // Persistent CTAs walk the tiles in ticket order and keep the next tile's P
 // and old S arriving in shared memory (TMA, or cp.async when rows are not
@@ -35,7 +35,7 @@
 namespace slstm {
 namespace {
 
-constexpr int NW = 8;   // warps per tile (time segments)
+constexpr int NW = 16;   // warps per tile (time segments)
 constexpr int L = 4;    // steps per thread
 constexpr int TT = NW * L;
 
@@ -52,7 +52,7 @@ struct Args {
     float *bnd_out;
     slstm_newton_stats *stats;
     unsigned *error;
-    const unsigned *vmask;        // packed sequences: head-flag words (one per chunk), else null
+    const unsigned *vmask;        // packed sequences: head-flag words (one per 32 steps), else null
     const int *vseq;              // packed sequences: sequence index at each head step
     unsigned epoch;
     unsigned long long wait_ns;
@@ -67,9 +67,8 @@ struct TileInfo {
     int chunk;
     int b;
     int j0;
-    unsigned long long off;   // element offset of (b, chunk * TT, slot 0, feature j0) in P and S
-    unsigned mask;            // packed sequences: bit i set when step chunk * TT + i starts a sequence
-    unsigned pad;
+    unsigned long long off;    // element offset of (b, chunk * TT, slot 0, feature j0) in P and S
+    unsigned long long mask;   // packed sequences: bit i set when step chunk * TT + i starts a sequence
 };
 
 struct Smem {
@@ -119,7 +118,7 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
     ti.ticket = ticket;
     ti.chunk = ti.b = ti.j0 = 0;
     ti.off = 0;
-    ti.mask = 0u;
+    ti.mask = 0ull;
     if (ticket < (unsigned)a.n_tiles) {
         const unsigned chunk = fast_div(ticket, a.div_groups);
         const unsigned grp = ticket - chunk * (unsigned)a.n_groups;
@@ -128,7 +127,18 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
         ti.b = (int)b;
         ti.j0 = (int)(grp - b * (unsigned)a.groups_per_row) * 32;
         ti.off = ((size_t)b * a.T + (size_t)chunk * TT) * 4 * (size_t)a.d + (size_t)ti.j0;
-        if (a.vmask) ti.mask = a.vmask[chunk];
+        if (a.vmask) {
+            // head flags of steps chunk * TT .. chunk * TT + TT - 1, from the
+            // words of 32 steps that hold them
+            const unsigned t0 = chunk * (unsigned)TT;
+            const unsigned nwords = ((unsigned)a.T + 31u) >> 5;
+            unsigned long long mk = 0ull;
+#pragma unroll
+            for (int q = 0; q < (TT + 31) / 32; ++q)
+                if ((t0 >> 5) + q < nwords) mk |= (unsigned long long)a.vmask[(t0 >> 5) + q] << (32 * q);
+            if constexpr (TT < 32) mk = (mk >> (t0 & 31u)) & ((1ull << (TT % 32)) - 1ull);
+            ti.mask = mk;
+        }
     }
 }
 
@@ -160,31 +170,31 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo 
     const float *s = a.S + ti.off + toff;
     if (a.vec16) {
         // 8 chunks of 16 bytes per (step, slot) row of 32 features; thread
-        // (w, slot, c) copies chunk c of slot `slot` for steps w, w+8, w+16, w+24
+        // (w, slot, c) copies chunk c of slot `slot` for steps w, w + NW, ...
         const int c = threadIdx.x & 7, slot = (threadIdx.x >> 3) & 3;
         const int rem = a.d - ti.j0 - 4 * c;
         const int fbytes = rem > 0 ? 4 * min(4, rem) : 0;
-        const size_t step8 = 32 * (size_t)a.d;   // 8 steps of 4 slots
+        const size_t stepw = (size_t)NW * 4 * a.d;   // NW steps of 4 slots
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int step = r * 8 + w;
+        for (int r = 0; r < L; ++r) {
+            const int step = r * NW + w;
             const int bytes = (t0 + step < a.T) ? fbytes : 0;
-            cp_async16(&sm.P[st][step][slot][4 * c], bytes ? p + r * step8 : a.P, bytes);
-            if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? s + r * step8 : a.S, bytes);
+            cp_async16(&sm.P[st][step][slot][4 * c], bytes ? p + r * stepw : a.P, bytes);
+            if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? s + r * stepw : a.S, bytes);
         }
     } else {
-        // 4-byte copies, lane = feature; warp w copies rows w, w+8, ... of
-        // the 128 (step, slot) rows
+        // 4-byte copies, lane = feature; warp w copies rows w, w + NW, ... of
+        // the 4 TT (step, slot) rows
         const int jl = threadIdx.x & 31;
         const bool fj = ti.j0 + jl < a.d;
-        const size_t row8 = 8 * (size_t)a.d;
+        const size_t roww = (size_t)NW * a.d;
 #pragma unroll 4
-        for (int r = 0; r < 16; ++r) {
-            const int rs = r * 8 + w;
+        for (int r = 0; r < 4 * L; ++r) {
+            const int rs = r * NW + w;
             const int step = rs >> 2, slot = rs & 3;
             const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
-            cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * row8 : a.P, bytes);
-            if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? s + r * row8 : a.S, bytes);
+            cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * roww : a.P, bytes);
+            if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? s + r * roww : a.S, bytes);
         }
     }
 }
@@ -236,7 +246,7 @@ __device__ void finalize(const Args &a, int k, bool resid)
 // VARLEN: packed ragged sequences (B = 1); at a head step the previous state is
 // the sequence's s0 and the Jacobian is zero, which makes the scan segmented.
 template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN>
-__global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
+__global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -369,7 +379,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
 #pragma unroll
                     for (int e = 0; e < 4; ++e) so[e] = sm.S[st][sl][e][lane];
                 }
-                const bool head = VARLEN && ((ti.mask >> sl) & 1u);
+                const bool head = VARLEN && ((ti.mask >> sl) & 1ull);
                 if (head) head_state(a, t_seg + i, jj, jv, curS);
                 cell_eval<FORGET, true>(curS[0], curS[1], curS[2], curS[3], sm.P[st][sl][0][lane],
                                         sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
@@ -404,7 +414,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         unsigned whead = 0u;
         if (VARLEN) {
 #pragma unroll
-            for (int w = 0; w < NW; ++w) whead |= (((ti.mask >> (w * L)) & ((1u << L) - 1u)) != 0u) ? (1u << w) : 0u;
+            for (int w = 0; w < NW; ++w) whead |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
         }
         const bool fast = __syncthreads_and(ok);
         if (fast) {
@@ -438,7 +448,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
         for (int i = 0; i < L; ++i) {
             const int sl = warp * L + i;
             const bool wr = jv && (t_seg + i < T);
-            if (VARLEN && ((ti.mask >> sl) & 1u)) {
+            if (VARLEN && ((ti.mask >> sl) & 1ull)) {
                 // a sequence starts here: nothing from before enters it
 #pragma unroll
                 for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
@@ -463,7 +473,7 @@ __global__ void __launch_bounds__(NW * 32, 2) newton_iter(Args a, int k, const _
                     if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
             }
             if (RESID) {
-                if (VARLEN && ((ti.mask >> sl) & 1u)) head_state(a, t_seg + i, jj, jv, snp);
+                if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
                 Cell f;
                 cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
                                          sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,

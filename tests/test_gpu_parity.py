@@ -143,7 +143,7 @@ def test_newton_converges_to_sequential_sigmoid(B, T, d, cuda_device):
 
 
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
-@pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256)])
+@pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256), (1, 300, 36), (2, 200, 40)])
 def test_newton_status_agrees_with_oracle(forget, B, T, d, cuda_device):
     w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
     inp, S, st, Pref = _newton_case(w)
@@ -189,7 +189,7 @@ def test_newton_bounded_wait_reports_timeout(cuda_device):
     """Fault injection on the host's request: one tile withholds its carry;
     its successor's bounded wait expires and the run reports a timeout
     instead of hanging."""
-    w = Workload("t", 1, 128, 8, 32, "f32", "sigmoid", 0.5, 1, 1e-6, 4)
+    w = Workload("t", 1, 256, 8, 32, "f32", "sigmoid", 0.5, 1, 1e-6, 4)
     inp = make_inputs(w, with_dH=False)
     Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
     S, st = api.newton_forward(Pt, _dev(inp["R"]), None, max_iters=2, fixed=True, tol=1e-6,
