@@ -283,6 +283,18 @@ SLSTM_DEVINL unsigned fast_div(unsigned n, const FastDiv &f)
 }
 
 // Non-negative float max through its bit pattern (NaN sorts above +inf).
+// Named CTA barriers (ids 1..15; id 0 is __syncthreads).  `count` threads,
+// a multiple of 32, take part; whole warps call these.
+SLSTM_DEVINL void named_bar_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+SLSTM_DEVINL void named_bar_arrive(int id, int count)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 SLSTM_DEVINL void atomic_max_nonneg(unsigned *slot, float v)
 {
     atomicMax(slot, __float_as_uint(fabsf(v)));

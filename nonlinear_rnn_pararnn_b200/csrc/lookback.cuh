@@ -402,8 +402,13 @@ SLSTM_DEVINL size_t chain_word(unsigned tq, int warp, int lane)
 // lane's component of the tile's inclusive prefix.  The arithmetic (order of
 // the fused multiply-adds) is that of aff_apply, so both walks give the same
 // bits.
+//
+// release > 0: named barrier 1 + w (release + ... threads: the 4 chain
+// warps and warp w) is arrived at once the carry entering warp w < release is
+// stored, so that warp can go on while the chain walks the later maps.
 template <int NW>
-SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane, unsigned whead = 0u)
+SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane, unsigned whead = 0u,
+                                int release = 0)
 {
     const int f = chain_feature(warp, lane);
     const int r = chain_row(lane);
@@ -412,6 +417,7 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
     for (int w = 0; w < NW; ++w) {
         const int fs = sw(r, f);
         cin[w][r][fs] = c;
+        if (w < release) named_bar_arrive(1 + w, 5 * 32);
         const float a0 = m[w][0][r][fs];
         const float a1 = m[w][1][r][fs];
         const float a2 = m[w][2][r][fs];

@@ -84,7 +84,12 @@ struct Smem {
     int exit_flag;
 };
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + room to align the stages to 1 KB
-constexpr int TMA_THREAD = (NW - 1) * 32;            // issues the tile loads (warp NW-1 carries no chain lane)
+// Warps CHAIN0 .. NW-1 walk the carry through the warp maps (chain lanes);
+// warp w < CHAIN0 starts walk B as soon as the carry entering it is stored
+// (named barrier 1 + w), the chain warps themselves after CHAIN_BAR.
+constexpr int CHAIN0 = NW - 4;
+constexpr int CHAIN_BAR = CHAIN0 + 1;   // the chain warps' own barrier (ids 1 .. CHAIN0 are per warp)
+constexpr int TMA_THREAD = (CHAIN0 - 1) * 32;   // issues the tile loads (a warp with no chain lane)
 constexpr uint64_t TMA_WAIT_NS = 1000000000ull;
 
 // Tensor maps of P and S viewed as (d, 4T, B): boxes of 32 features x 128
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     const int T = a.T;
     const unsigned G = (unsigned)a.n_groups;
     const size_t toff = prefetch_offset(a);
-    const bool chain_warp = warp < 4;
+    const bool chain_warp = warp >= CHAIN0;
     float mx_raw = 0.f, mx_sc = 0.f;
 
     int ring = 0, st = 0;
@@ -417,17 +422,24 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             for (int w = 0; w < NW; ++w) whead |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
         }
         const bool fast = __syncthreads_and(ok);
-        if (fast) {
-            if (chain_warp) {
-                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead);
+        if (chain_warp) {
+            if (fast) {
+                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead, CHAIN0);
                 if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
+                named_bar_sync(CHAIN_BAR, 4 * 32);
+            } else {
+                if (warp == CHAIN0) {
+                    const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                    tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk,
+                                            (int)(ticket - (unsigned)chunk * G), withhold, whead);
+                }
+                named_bar_sync(CHAIN_BAR, 4 * 32);
+#pragma unroll 1
+                for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
             }
-        } else if (warp == 0) {
-            const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-            tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), withhold,
-                                    whead);
+        } else {
+            named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
         }
-        __syncthreads();
 
         // ---- walk B ----
         // this warp's store of the previous tile has read its rows of O
