@@ -186,9 +186,10 @@ SLSTM_DEVINL void carry_serial(const CarryArgs &ca, LoadMap load, PutCarry put, 
     load(0, x);
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-        put(w, v);
+        // the next map is read before the store, which loads may not pass
         Aff xn;
         if (w + 1 < NW) load(w + 1, xn);
+        put(w, v);
         if ((whead >> w) & 1u) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) v[e] = x.b[e];
@@ -403,8 +404,8 @@ SLSTM_DEVINL size_t chain_word(unsigned tq, int warp, int lane)
 // the fused multiply-adds) is that of aff_apply, so both walks give the same
 // bits.
 //
-// release > 0: named barrier 1 + w (release + ... threads: the 4 chain
-// warps and warp w) is arrived at once the carry entering warp w < release is
+// release > 0: each chain warp arrives at named barrier 1 + w (160 threads:
+// the 4 chain warps and warp w) once the carry entering warp w < release is
 // stored, so that warp can go on while the chain walks the later maps.
 template <int NW>
 SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp, int lane, unsigned whead = 0u,
@@ -412,23 +413,29 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
 {
     const int f = chain_feature(warp, lane);
     const int r = chain_row(lane);
+    const int fs = sw(r, f);
     const int i8 = lane & 7;
+    // the map entries are read two maps ahead, before the stores and barrier
+    // arrivals of the current map, which the compiler may not move loads past
+    float q[3][5];
+    auto load = [&](int w, float *o) {
+#pragma unroll
+        for (int k = 0; k < 5; ++k) o[k] = m[w][k][r][fs];
+    };
+    load(0, q[0]);
+    if (NW > 1) load(1, q[1]);
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-        const int fs = sw(r, f);
+        if (w + 2 < NW) load(w + 2, q[(w + 2) % 3]);
         cin[w][r][fs] = c;
         if (w < release) named_bar_arrive(1 + w, 5 * 32);
-        const float a0 = m[w][0][r][fs];
-        const float a1 = m[w][1][r][fs];
-        const float a2 = m[w][2][r][fs];
-        const float a3 = m[w][3][r][fs];
-        const float bb = m[w][4][r][fs];
+        const float *a = q[w % 3];
         const float v0 = __shfl_sync(0xffffffffu, c, i8);
         const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
         const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
         const float v3 = __shfl_sync(0xffffffffu, c, 24 + i8);
-        const float nc = fmaf(a3, v3, fmaf(a2, v2, fmaf(a1, v1, fmaf(a0, v0, bb))));
-        c = ((whead >> w) & 1u) ? bb : nc;
+        const float nc = fmaf(a[3], v3, fmaf(a[2], v2, fmaf(a[1], v1, fmaf(a[0], v0, a[4]))));
+        c = ((whead >> w) & 1u) ? a[4] : nc;
     }
     return c;
 }
