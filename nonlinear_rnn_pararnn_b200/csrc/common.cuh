@@ -300,14 +300,19 @@ SLSTM_DEVINL void atomic_max_nonneg(unsigned *slot, float v)
     atomicMax(slot, __float_as_uint(fabsf(v)));
 }
 
+// max(a, b), NaN when either is NaN (fmaxf would drop it): a non-finite
+// residual stays visible through every reduction.
+SLSTM_DEVINL float fmax_nan(float a, float b)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
 SLSTM_DEVINL float warp_max(float v)
 {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float w = __shfl_xor_sync(0xffffffffu, v, o);
-        // keep NaN: fmaxf drops NaN, so compare bit patterns of |v|
-        v = (__float_as_uint(w) > __float_as_uint(v)) ? w : v;
-    }
+    for (int o = 16; o > 0; o >>= 1) v = fmax_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 

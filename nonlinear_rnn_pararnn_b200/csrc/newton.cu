@@ -495,9 +495,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                 for (int e = 0; e < 4; ++e) {
                     const float af = wr ? fabsf(F[e]) : 0.0f;
                     const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
-                    // keep NaN: a NaN compares false, so test "not <="
-                    mx_raw = (af <= mx_raw) ? mx_raw : af;
-                    mx_sc = (sc <= mx_sc) ? mx_sc : sc;
+                    mx_raw = fmax_nan(mx_raw, af);
+                    mx_sc = fmax_nan(mx_sc, sc);
                 }
             }
 #pragma unroll

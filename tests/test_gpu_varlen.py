@@ -142,3 +142,21 @@ def test_varlen_backward_matches_oracle(d_in, d, dtype, forget, cuda_device):
         assert err <= 1e-4, (k, err)
     # empty sequences get exactly zero
     assert not out["ds0"][1].any() and not out["ds0"][7].any()
+
+
+def test_varlen_nan_in_one_sequence_reports_divergence(cuda_device):
+    """A non-finite value inside a short sequence does not leak into the next
+    sequence (its start ignores the state before it), so the steps after it in
+    the same thread are finite again; the residual maximum must still keep the
+    NaN and the run must report divergence."""
+    lengths = [2, 3, 40]
+    c = _case(lengths, 40, 12, "f32", "sigmoid", 46)
+    P, _ = _preact(c)
+    P[0, 1, 5] = float("nan")    # first sequence, step 0, gate i of feature 5
+    S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), max_iters=2, fixed=True,
+                                      tol=1e-6)
+    torch.cuda.synchronize()
+    s = api.read_stats(st)
+    assert s["diverged"] and s["error"] == 3, s
+    # the later sequences are untouched by it
+    assert torch.isfinite(S[2:]).all()
