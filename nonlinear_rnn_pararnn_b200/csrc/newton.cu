@@ -89,7 +89,8 @@ constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + room to align the stag
 // (named barrier 1 + w), the chain warps themselves after CHAIN_BAR.
 constexpr int CHAIN0 = NW - 4;
 constexpr int CHAIN_BAR = CHAIN0 + 1;   // the chain warps' own barrier (ids 1 .. CHAIN0 are per warp)
-constexpr int TMA_THREAD = (CHAIN0 - 1) * 32;   // issues the tile loads (a warp with no chain lane)
+constexpr int TMA_THREAD = (CHAIN0 - 1) * 32;   // issues the first tile's loads (a warp with no chain lane)
+constexpr int TMA_WARP0 = CHAIN0 - 4;           // lane 0 of warps TMA_WARP0 .. +3 issue the later tiles' loads
 constexpr uint64_t TMA_WAIT_NS = 1000000000ull;
 
 // Tensor maps of P and S viewed as (d, 4T, B): boxes of 32 features x 128
@@ -116,6 +117,32 @@ SLSTM_DEVINL void issue_tile_load(const Args &a, const NewtonMaps &m, Smem &sm, 
     if (bnd)
         bulk_load(&sm.bnd[st][0][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32,
                   (uint32_t)sizeof(sm.bnd[0]), &sm.bar[st]);
+}
+
+// The same loads split over four issuing threads (lane 0 of warps
+// TMA_WARP0 .. TMA_WARP0 + 3), so that no single warp starts its walk late:
+// part 0 announces the stage's bytes and loads P, part 1 S_old, part 2 the R
+// rows, part 3 the boundary block.  Bytes may land before they are announced.
+SLSTM_DEVINL void issue_tile_load_part(const Args &a, const NewtonMaps &m, Smem &sm, int st, const TileInfo &ti,
+                                       bool with_s, int part)
+{
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const int row = ti.chunk * TT * 4;
+    const uint32_t rbytes = 4u * (uint32_t)min(32, a.d - ti.j0);
+    const bool bnd = with_s && ti.chunk > 0;
+    if (part == 0) {
+        mbar_expect_tx(&sm.bar[st], (with_s ? 2u : 1u) * (uint32_t)sizeof(sm.P[0]) + 4u * rbytes +
+                                        (bnd ? (uint32_t)sizeof(sm.bnd[0]) : 0u));
+        tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, row, ti.b);
+    } else if (part == 1) {
+        if (with_s) tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, row, ti.b);
+    } else if (part == 2) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    } else if (bnd) {
+        bulk_load(&sm.bnd[st][0][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32,
+                  (uint32_t)sizeof(sm.bnd[0]), &sm.bar[st]);
+    }
 }
 
 SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
@@ -303,7 +330,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             // the other stage is free (every warp passed the barrier that
             // ends the previous tile): start the next tile's loads a whole
             // tile ahead, then wait for the current tile's boxes
-            if (threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st ^ 1, sm.info[rn], !FIRST);
+            if (lane == 0 && warp >= TMA_WARP0 && warp < TMA_WARP0 + 4)
+                issue_tile_load_part(a, maps, sm, st ^ 1, sm.info[rn], !FIRST, warp - TMA_WARP0);
             if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS)) {
                 atomicOr(a.error, 2u);
                 (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS);
@@ -400,8 +428,6 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             }
         }
         maps_store(sm.maps.m, warp, lane, agg);
-        // the tile after the next one, visible to all after the vote barrier
-        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
 
         // ---- carry ----
         float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
@@ -510,6 +536,9 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                 bulk_commit();
             }
         }
+        // the tile after the next one (read two tiles from now), decoded where
+        // warp 0 would otherwise wait for the chain warps
+        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
         // state at the tile's last step, for the next launch's successor tile
         if (warp == NW - 1 && t_seg + L - 1 < T) {
             float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
