@@ -388,7 +388,8 @@ SLSTM_DEVINL void maps_load(const MapArr *m, int w, int lane, Aff &x)
     }
 }
 
-// Chain lanes: warps 0..3, lane (row = lane >> 3, feature = 8 * warp + (lane & 7)).
+// Chain lanes: four warps with warp & 3 = 0 .. 3, lane (row = lane >> 3,
+// feature = 8 * (warp & 3) + (lane & 7)).
 SLSTM_DEVINL int chain_feature(int warp, int lane) { return ((warp & 3) << 3) | (lane & 7); }
 SLSTM_DEVINL int chain_row(int lane) { return lane >> 3; }
 
@@ -440,7 +441,7 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
     return c;
 }
 
-// Warp 0 only, chain layout, when some chain lane found no published
+// One warp only, chain layout, when some chain lane found no published
 // predecessor prefix: reads it again, else looks back; then walks the maps
 // serially (lane = feature).  chunk > 0.
 template <int NW>

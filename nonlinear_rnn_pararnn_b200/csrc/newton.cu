@@ -14,10 +14,12 @@
 //           4x4 Jacobian J_t in registers for its 4 steps, keeps (J_t, r_t =
 //           f - S_t) in registers and folds the maps delta -> J_t delta + r_t;
 //   carry   the carry entering the tile is the predecessor tile's inclusive
-//           prefix (looked at twice: before and after walk A); warps 0-3
-//           apply the 8 warp maps to it, one (feature, slot) pair per lane,
-//           and publish this tile's prefix; a tile whose predecessor has not
-//           published falls back to the look-back in lookback.cuh;
+//           prefix (looked at twice: before and after walk A); the last four
+//           warps apply the 16 warp maps to it, one (feature, slot) pair per
+//           lane, release every other warp as soon as the carry entering it
+//           is stored, and publish this tile's prefix; a tile whose
+//           predecessor has not published falls back to the look-back in
+//           lookback.cuh;
 //   walk B  each thread replays its steps from its carry, writes S + delta in
 //           place and, when asked, accumulates the residual of the new
 //           iterate for the stopping test.
