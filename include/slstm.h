@@ -106,7 +106,19 @@ typedef enum {
  *               stats.error; results are not meaningful).
  *   wait_limit_us  upper bound of one bounded wait, in microseconds
  *               (0 = the default of 2 seconds).
+ *   carry_mode  how a tile gets the scan carry entering it (same results up
+ *               to rounding): SLSTM_CARRY_FUSED, one launch per iteration in
+ *               which each tile takes its predecessor's published prefix
+ *               (decoupled look-back); SLSTM_CARRY_TWO_PASS, a pass that
+ *               stores every tile's aggregate map, a scan of the aggregates
+ *               of each feature group, and a pass that applies the carries
+ *               (no tile waits on another; cheaper with few feature groups);
+ *               SLSTM_CARRY_AUTO (0) picks two passes when there are at
+ *               most SMs / 4 feature groups (B * ceil(d_h/32)) and at least
+ *               256 chunks of 64 steps, and debug_fault is 0.
  */
+typedef enum { SLSTM_CARRY_AUTO = 0, SLSTM_CARRY_FUSED = 1, SLSTM_CARRY_TWO_PASS = 2 } slstm_carry_mode;
+
 typedef struct {
     int max_iters;
     int fixed_iters;
@@ -114,6 +126,7 @@ typedef struct {
     int forget;
     int debug_fault;
     int wait_limit_us;
+    int carry_mode;
 } slstm_newton_config;
 
 /*

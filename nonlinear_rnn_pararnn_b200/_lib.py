@@ -36,7 +36,8 @@ SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 class NewtonConfig(ctypes.Structure):
     _fields_ = [("max_iters", ctypes.c_int), ("fixed_iters", ctypes.c_int), ("tol", ctypes.c_float),
-                ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int)]
+                ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int),
+                ("carry_mode", ctypes.c_int)]
 
 
 STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY

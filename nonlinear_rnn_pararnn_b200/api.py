@@ -91,7 +91,7 @@ def read_stats(stats: torch.Tensor) -> dict:
 def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
                    max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
                    stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
-                   wait_limit_us: int = 0):
+                   wait_limit_us: int = 0, carry_mode: int = 0):
     """Newton solve; returns (S, stats) with stats a device record (see read_stats)."""
     B, T, four, d_h = P.shape
     _need(P, "P", (B, T, 4, d_h))
@@ -106,7 +106,7 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
     cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
-                       int(wait_limit_us))
+                       int(wait_limit_us), int(carry_mode))
     check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
                                                               ctypes.byref(cfg), _ptr(stats), B, T, d_h,
                                                               _ptr(ws), ws.numel(), _stream()))
@@ -184,7 +184,8 @@ def _need_cu(cu: torch.Tensor, n_seq: int):
 
 def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu_seqlens: torch.Tensor, *,
                           forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
-                          S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None):
+                          S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None,
+                          carry_mode: int = 0):
     """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
     cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats)."""
     total_T, four, d_h = P.shape
@@ -201,7 +202,7 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
-    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0)
+    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0, int(carry_mode))
     check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
         _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
         _ptr(ws), ws.numel(), _stream()))

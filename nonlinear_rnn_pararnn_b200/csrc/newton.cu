@@ -38,6 +38,15 @@ namespace slstm {
 namespace {
 
 constexpr int NW = 16;   // warps per tile (time segments)
+// How a launch gets the carry entering each tile.  FUSED: from the tile
+// before it in the same launch (decoupled look-back).  With few feature
+// groups most tiles would wait on their predecessors, so an iteration can
+// instead run as two passes over the tiles with a scan in between: AGG
+// stores each tile's aggregate map, a blocked scan (scan_block_agg,
+// scan_block_carry, scan_tile_carry) turns the aggregates of every feature
+// group into the carry entering each tile, and APPLY is the fused iteration
+// with that carry known.
+constexpr int MODE_FUSED = 0, MODE_AGG = 1, MODE_APPLY = 2;
 constexpr int L = 4;    // steps per thread
 constexpr int TT = NW * L;
 
@@ -52,6 +61,10 @@ struct Args {
     unsigned long long *incw;     // [n_tiles][4][32] (value bits | epoch << 32)
     float *bnd_in;                // [n_tiles][4][32] S of the previous iterate at each tile's last step
     float *bnd_out;
+    float *cin_buf;               // two-pass carry: [n_tiles][4][32] carry entering each tile (chain layout)
+    float *blk_agg;               // two-pass scan scratch (see scan_block_agg)
+    unsigned *blk_head;
+    float *blk_cin;
     slstm_newton_stats *stats;
     unsigned *error;
     const unsigned *vmask;        // packed sequences: head-flag words (one per 32 steps), else null
@@ -274,12 +287,128 @@ __device__ void finalize(const Args &a, int k, bool resid)
     if (done) atomicExch(&c->done, 1u);
 }
 
+// Between the two passes of an iteration: the carry entering every tile,
+// from the aggregates of the tiles before it in its feature group (chunk 0
+// gets none).  A group's chunks are cut into blocks of SCAN_BLK: the
+// aggregates of every block are composed (scan_block_agg), the blocks of a
+// group are walked in order (scan_block_carry), and every block applies its
+// aggregates from the carry entering it (scan_tile_carry).  One warp per
+// (group, block), lane = feature; a tile with a sequence start passes on its
+// offset whatever enters it.
+constexpr int SCAN_BLK = 32;
+
+SLSTM_DEVINL void load_agg(const float *src, int lane, Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+}
+
+SLSTM_DEVINL void store_agg(float *dst, int lane, const Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = x.a[e];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = x.b[e];
+}
+
+struct ScanArgs {
+    const float *agg;          // [n_tiles][20][32] tile aggregates
+    const unsigned *head;      // [n_tiles] nonzero: the tile holds a sequence start
+    float *blk_agg;            // [n_groups][n_blk][20][32]
+    unsigned *blk_head;        // [n_groups][n_blk]
+    float *blk_cin;            // [n_groups][n_blk][4][32]
+    float *cin;                // [n_tiles][4][32] the carry entering each tile
+    const unsigned *done;
+    int n_groups, n_chunks, n_blk;
+};
+
+// (group, block) per warp: the composition of the block's tile aggregates.
+__global__ void __launch_bounds__(256) scan_block_agg(ScanArgs s)
+{
+    if (*(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= (long long)s.n_groups * s.n_blk) return;
+    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
+    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
+    const size_t G = (size_t)s.n_groups;
+    Aff acc, x;
+    load_agg(s.agg + ((size_t)c0 * G + g) * 640, lane, acc);
+    bool hd = s.head[(size_t)c0 * G + g] != 0u;
+    for (int c = c0 + 1; c < c1; ++c) {
+        load_agg(s.agg + ((size_t)c * G + g) * 640, lane, x);
+        if (s.head[(size_t)c * G + g] != 0u) {
+            acc = x;   // starts afresh: ignores what came before
+            hd = true;
+        } else {
+            aff_compose(x, acc, acc);
+        }
+    }
+    store_agg(s.blk_agg + (size_t)wid * 640, lane, acc);
+    if (lane == 0) s.blk_head[wid] = hd ? 1u : 0u;
+}
+
+// One warp per group: the carry entering each block.
+__global__ void __launch_bounds__(256) scan_block_carry(ScanArgs s)
+{
+    if (*(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (g >= s.n_groups) return;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    Aff x;
+    for (int k = 0; k < s.n_blk; ++k) {
+        const size_t w = (size_t)g * s.n_blk + k;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.blk_cin[w * 128 + e * 32 + lane] = v[e];
+        if (k + 1 == s.n_blk) break;
+        load_agg(s.blk_agg + w * 640, lane, x);
+        if (s.blk_head[w] != 0u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
+        } else {
+            aff_apply(x, v, v);
+        }
+    }
+}
+
+// (group, block) per warp: the carry entering each tile of the block.
+__global__ void __launch_bounds__(256) scan_tile_carry(ScanArgs s)
+{
+    if (*(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= (long long)s.n_groups * s.n_blk) return;
+    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
+    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
+    const size_t G = (size_t)s.n_groups;
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = s.blk_cin[(size_t)wid * 128 + e * 32 + lane];
+    Aff x;
+    for (int c = c0; c < c1; ++c) {
+        const size_t t = (size_t)c * G + g;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.cin[t * 128 + e * 32 + lane] = v[e];
+        if (c + 1 == c1) break;
+        load_agg(s.agg + t * 640, lane, x);
+        if (s.head[t] != 0u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
+        } else {
+            aff_apply(x, v, v);
+        }
+    }
+}
+
 // TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
 // stage, stores per warp from the stage walk B wrote); otherwise by cp.async
 // and plain stores.
 // VARLEN: packed ragged sequences (B = 1); at a head step the previous state is
 // the sequence's s0 and the Jacobian is zero, which makes the scan segmented.
-template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN>
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE>
 __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -291,8 +420,9 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     if (threadIdx.x == 0) {
         sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
         if (!sm.exit_flag) {
-            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[0]);
-            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[1]);
+            // AGG tiles are independent: a static order needs no counter
+            decode_tile(a, MODE == MODE_AGG ? blockIdx.x : atomicAdd(&slot.ticket, 1u), sm.info[0]);
+            decode_tile(a, MODE == MODE_AGG ? blockIdx.x + gridDim.x : atomicAdd(&slot.ticket, 1u), sm.info[1]);
         }
     }
     if (TMA && threadIdx.x == TMA_THREAD) {
@@ -327,7 +457,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // tickets run two tiles ahead: fetch the one after the next now,
         // decode it into the ring at the end of this tile
         unsigned after = 0;
-        if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
+        if (threadIdx.x == 0)
+            after = MODE == MODE_AGG ? blockIdx.x + (it + 2u) * gridDim.x : atomicAdd(&slot.ticket, 1u);
         if (TMA) {
             // the other stage is free (every warp passed the barrier that
             // ends the previous tile): start the next tile's loads a whole
@@ -392,7 +523,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // looks at the predecessor's inclusive prefix (chain lanes): before
         // and halfway through walk A, so that both loads' latency is hidden;
         // the second is read only when the first found nothing
-        const bool look = chain_warp && chunk > 0;
+        const bool look = MODE == MODE_FUSED && chain_warp && chunk > 0;
         const unsigned long long *predw = a.incw + chain_word(ticket - G, warp, lane);
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
@@ -431,122 +562,159 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         }
         maps_store(sm.maps.m, warp, lane, agg);
 
-        // ---- carry ----
-        float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
-        bool ok = true;
-        if (look) {
-            if ((unsigned)(w1 >> 32) == a.epoch) {
-                c = __uint_as_float((unsigned)w1);
-            } else {
-                ok = (unsigned)(w2 >> 32) == a.epoch;
-                c = __uint_as_float((unsigned)w2);
-            }
-        }
-        const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
         // warps whose steps contain a sequence start (packed sequences)
         unsigned whead = 0u;
         if (VARLEN) {
 #pragma unroll
             for (int w = 0; w < NW; ++w) whead |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
         }
-        const bool fast = __syncthreads_and(ok);
-        if (chain_warp) {
-            if (fast) {
-                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead, CHAIN0);
-                if (!withhold) st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
-                named_bar_sync(CHAIN_BAR, 4 * 32);
-            } else {
-                if (warp == CHAIN0) {
-                    const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-                    tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk,
-                                            (int)(ticket - (unsigned)chunk * G), withhold, whead);
+        if constexpr (MODE == MODE_AGG) {
+            // the tile's aggregate map: a tree over the warp maps (at step h,
+            // warp w composes slot (2w+2)h - 1 with slot (2w+1)h - 1 into the
+            // former; a part that holds a sequence start ignores what enters
+            // it and is kept as it is)
+#pragma unroll
+            for (int h = 1; h < NW; h *= 2) {
+                __syncthreads();
+                if (warp < NW / (2 * h)) {
+                    const int hi = (2 * warp + 2) * h - 1, lo = (2 * warp + 1) * h - 1;
+                    const bool hhead = VARLEN && (((whead >> ((2 * warp + 1) * h)) & ((1u << h) - 1u)) != 0u);
+                    Aff x, y;
+                    maps_load(sm.maps.m, hi, lane, x);
+                    if (!hhead) {
+                        maps_load(sm.maps.m, lo, lane, y);
+                        aff_compose(x, y, x);
+                        maps_store(sm.maps.m, hi, lane, x);
+                    }
                 }
-                named_bar_sync(CHAIN_BAR, 4 * 32);
-#pragma unroll 1
-                for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                Aff x;
+                maps_load(sm.maps.m, NW - 1, lane, x);
+                float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
+                if (lane == 0) a.flags[ticket] = whead ? 1u : 0u;
             }
         } else {
-            named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
-        }
 
-        // ---- walk B ----
-        // this warp's store of the previous tile has read its rows of O
-        if (TMA) {
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
-        }
-        float dl[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dl[e] = sm.maps.cin[warp][e][sw(e, lane)];
-        float snp[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
-        // row pointer of this lane's first step; lanes past d and steps past T
-        // write nothing
-        float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
-#pragma unroll
-        for (int i = 0; i < L; ++i) {
-            const int sl = warp * L + i;
-            const bool wr = jv && (t_seg + i < T);
-            if (VARLEN && ((ti.mask >> sl) & 1ull)) {
-                // a sequence starts here: nothing from before enters it
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
-            }
-            // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
-            const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
-            float sn[4];
-            jac_mul_add(Jc[i], dl, f4, sn);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
-                dl[e] = sn[e] - so;
-            }
-            if (TMA) {
-                // rows past T and features past d fall outside the tensor and
-                // are not stored
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sn[e];
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
-            }
-            if (RESID) {
-                if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
-                Cell f;
-                cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
-                                         sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
-                                         rf, ro, f);
-                const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float af = wr ? fabsf(F[e]) : 0.0f;
-                    const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
-                    mx_raw = fmax_nan(mx_raw, af);
-                    mx_sc = fmax_nan(mx_sc, sc);
+            // ---- carry ----
+            float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
+            bool ok = true;
+            if (MODE == MODE_APPLY && chain_warp) c = a.cin_buf[chain_word(ticket, warp, lane)];
+            if (look) {
+                if ((unsigned)(w1 >> 32) == a.epoch) {
+                    c = __uint_as_float((unsigned)w1);
+                } else {
+                    ok = (unsigned)(w2 >> 32) == a.epoch;
+                    c = __uint_as_float((unsigned)w2);
                 }
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) snp[e] = sn[e];
-        }
-        if (TMA) {
-            tma_store_fence();
-            __syncwarp();
-            if (lane == 0 && t_seg < T) {
-                tma_store_3d(&maps.Sw, &sm.O[warp * L][0][0], ti.j0, t_seg * 4, ti.b);
-                bulk_commit();
+            const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
+            const bool fast = __syncthreads_and(ok);
+            if (chain_warp) {
+                if (fast) {
+                    c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead, CHAIN0);
+                    if (MODE == MODE_FUSED && !withhold)
+                        st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
+                    named_bar_sync(CHAIN_BAR, 4 * 32);
+                } else {
+                    if (warp == CHAIN0) {
+                        const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                        tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk,
+                                                (int)(ticket - (unsigned)chunk * G), withhold, whead);
+                    }
+                    named_bar_sync(CHAIN_BAR, 4 * 32);
+    #pragma unroll 1
+                    for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
+                }
+            } else {
+                named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
             }
+
+            // ---- walk B ----
+            // this warp's store of the previous tile has read its rows of O
+            if (TMA) {
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+            }
+            float dl[4];
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) dl[e] = sm.maps.cin[warp][e][sw(e, lane)];
+            float snp[4];
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) snp[e] = sp[e] + dl[e];
+            // row pointer of this lane's first step; lanes past d and steps past T
+            // write nothing
+            float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
+    #pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int sl = warp * L + i;
+                const bool wr = jv && (t_seg + i < T);
+                if (VARLEN && ((ti.mask >> sl) & 1ull)) {
+                    // a sequence starts here: nothing from before enters it
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
+                }
+                // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
+                const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
+                float sn[4];
+                jac_mul_add(Jc[i], dl, f4, sn);
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
+                    dl[e] = sn[e] - so;
+                }
+                if (TMA) {
+                    // rows past T and features past d fall outside the tensor and
+                    // are not stored
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sn[e];
+                } else {
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+                }
+                if (RESID) {
+                    if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
+                    Cell f;
+                    cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
+                                             sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
+                                             rf, ro, f);
+                    const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float af = wr ? fabsf(F[e]) : 0.0f;
+                        const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
+                        mx_raw = fmax_nan(mx_raw, af);
+                        mx_sc = fmax_nan(mx_sc, sc);
+                    }
+                }
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) snp[e] = sn[e];
+            }
+            if (TMA) {
+                tma_store_fence();
+                __syncwarp();
+                if (lane == 0 && t_seg < T) {
+                    tma_store_3d(&maps.Sw, &sm.O[warp * L][0][0], ti.j0, t_seg * 4, ti.b);
+                    bulk_commit();
+                }
+            }
+            // state at the tile's last step, for the next launch's successor tile
+            if (warp == NW - 1 && t_seg + L - 1 < T) {
+                float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
+            }
+
         }
         // the tile after the next one (read two tiles from now), decoded where
         // warp 0 would otherwise wait for the chain warps
         if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
-        // state at the tile's last step, for the next launch's successor tile
-        if (warp == NW - 1 && t_seg + L - 1 < T) {
-            float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
-        }
 
         __syncthreads();   // this stage is free for the loads of the tile after next
         ring = rn;
@@ -558,6 +726,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     } else {
         cp_async_wait_all();
     }
+    if constexpr (MODE == MODE_AGG) return;   // the iteration itself is the APPLY launch
 
     if (RESID) {
         mx_raw = warp_max(mx_raw);
@@ -587,10 +756,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     }
 }
 
-template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN>
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE>
 cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = newton_iter<FORGET, FIRST, RESID, TMA, VARLEN>;
+    auto kern = newton_iter<FORGET, FIRST, RESID, TMA, VARLEN, MODE>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -604,8 +773,19 @@ cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaS
     return cudaGetLastError();
 }
 
+template <int FORGET, bool TMA, bool VARLEN, int MODE>
+cudaError_t launch_pass(const Args &a, const NewtonMaps &m, int k, bool resid, int sms, cudaStream_t st)
+{
+    if (k == 0)
+        return resid ? launch_one<FORGET, true, true, TMA, VARLEN, MODE>(a, m, k, sms, st)
+                     : launch_one<FORGET, true, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
+    return resid ? launch_one<FORGET, false, true, TMA, VARLEN, MODE>(a, m, k, sms, st)
+                 : launch_one<FORGET, false, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
+}
+
 template <int FORGET, bool TMA, bool VARLEN>
-cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, int sms, cudaStream_t st)
+cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
+                         cudaStream_t st)
 {
     for (int k = 0; k < max_iters; ++k) {
         Args a = base;
@@ -614,19 +794,28 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
         const bool resid = !fixed || (k + 1 == max_iters);
         cudaError_t e;
-        if (k == 0)
-            e = resid ? launch_one<FORGET, true, true, TMA, VARLEN>(a, m, k, sms, st)
-                      : launch_one<FORGET, true, false, TMA, VARLEN>(a, m, k, sms, st);
-        else
-            e = resid ? launch_one<FORGET, false, true, TMA, VARLEN>(a, m, k, sms, st)
-                      : launch_one<FORGET, false, false, TMA, VARLEN>(a, m, k, sms, st);
+        if (two_pass) {
+            if ((e = launch_pass<FORGET, TMA, VARLEN, MODE_AGG>(a, m, k, false, sms, st)) != cudaSuccess) return e;
+            const int n_chunks = a.n_tiles / a.n_groups;
+            const int n_blk = (n_chunks + SCAN_BLK - 1) / SCAN_BLK;
+            const ScanArgs sa{a.agg, a.flags, a.blk_agg, a.blk_head, a.blk_cin, a.cin_buf, &a.ctrl->done,
+                              a.n_groups, n_chunks, n_blk};
+            const long long nw = (long long)a.n_groups * n_blk;
+            scan_block_agg<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
+            scan_block_carry<<<(a.n_groups + 7) / 8, 256, 0, st>>>(sa);
+            scan_tile_carry<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            e = launch_pass<FORGET, TMA, VARLEN, MODE_APPLY>(a, m, k, resid, sms, st);
+        } else {
+            e = launch_pass<FORGET, TMA, VARLEN, MODE_FUSED>(a, m, k, resid, sms, st);
+        }
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 struct Layout {
-    size_t ctrl, flags, incw, agg, bnd0, bnd1, total;
+    size_t ctrl, flags, incw, agg, bnd0, bnd1, cin, blk_agg, blk_head, blk_cin, total;
     int groups_per_row, n_groups, n_chunks, n_tiles;
 };
 
@@ -649,6 +838,11 @@ Layout layout(int B, int T, int d)
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
     l.bnd0 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.bnd1 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
+    l.cin = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
+    const size_t nblk = (size_t)l.n_groups * ((l.n_chunks + SCAN_BLK - 1) / SCAN_BLK);
+    l.blk_agg = take(sizeof(float) * 20 * 32 * nblk);
+    l.blk_head = take(sizeof(unsigned) * nblk);
+    l.blk_cin = take(sizeof(float) * 4 * 32 * nblk);
     l.total = off;
     return l;
 }
@@ -666,11 +860,11 @@ int sm_count()
 }
 
 template <int FORGET, bool TMA>
-cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, bool fixed, int sms, bool varlen,
-                             cudaStream_t st)
+cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
+                             bool varlen, cudaStream_t st)
 {
-    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, sms, st)
-                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, sms, st);
+    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, two_pass, sms, st)
+                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, two_pass, sms, st);
 }
 
 }  // namespace
@@ -694,6 +888,10 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     a.incw = reinterpret_cast<unsigned long long *>(base + l.incw);
     a.bnd_in = reinterpret_cast<float *>(base + l.bnd0);
     a.bnd_out = reinterpret_cast<float *>(base + l.bnd1);
+    a.cin_buf = reinterpret_cast<float *>(base + l.cin);
+    a.blk_agg = reinterpret_cast<float *>(base + l.blk_agg);
+    a.blk_head = reinterpret_cast<unsigned *>(base + l.blk_head);
+    a.blk_cin = reinterpret_cast<float *>(base + l.blk_cin);
     a.stats = stats;
     a.error = &a.ctrl->error;
     a.epoch = 1;
@@ -739,11 +937,19 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
                      make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);
     const bool v = vl != nullptr;
+    // With few feature groups and many chunks, most tiles of a fused launch
+    // would wait for their predecessor: take the two passes instead (measured
+    // on B200: faster from 1024 chunks down to 256 with 8-32 groups, slower
+    // with 64 groups or 128 chunks).  Fault injection acts on the fused
+    // launch's publications.
+    const bool two_pass = cfg.carry_mode == SLSTM_CARRY_TWO_PASS ||
+                          (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 && 4 * l.n_groups <= sms &&
+                           l.n_chunks >= 256);
     if (cfg.forget == SLSTM_FORGET_EXP)
-        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, sms, v, st)
-                   : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, sms, v, st);
-    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, sms, v, st)
-               : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, sms, v, st);
+        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st)
+                   : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st);
+    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st)
+               : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st);
 }
 
 }  // namespace slstm

@@ -103,6 +103,7 @@ int slstm_newton_forward(const float *P, const float *R, const float *s0, float 
     if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
     if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
     if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
     if (!sizes_ok(B, T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
         return SLSTM_ERR_INVALID_ARG;
@@ -158,6 +159,7 @@ int slstm_newton_forward_varlen(const float *P, const float *R, const float *s0,
     if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
     if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
     if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
     if (!varlen_sizes_ok(n_seq, total_T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))

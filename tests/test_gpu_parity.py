@@ -87,15 +87,20 @@ def test_preact_gemm_matches_oracle(dtype, B, T, d_in, d_h, cuda_device):
 # ---------------------------------------------------------------------------
 # Newton forward
 # ---------------------------------------------------------------------------
-def _newton_case(w: Workload, fixed_k=None):
+# carry modes: 1 = one fused launch per iteration (decoupled look-back),
+# 2 = two passes with a scan of tile aggregates in between
+CARRY_MODES = [1, 2]
+
+
+def _newton_case(w: Workload, fixed_k=None, carry_mode=0):
     inp = make_inputs(w, with_dH=False)
     Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
     if fixed_k is None:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
-                                   max_iters=w.max_iters, fixed=False, tol=w.tol)
+                                   max_iters=w.max_iters, fixed=False, tol=w.tol, carry_mode=carry_mode)
     else:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
-                                   max_iters=fixed_k, fixed=True, tol=w.tol)
+                                   max_iters=fixed_k, fixed=True, tol=w.tol, carry_mode=carry_mode)
     stats = api.read_stats(st)
     Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
     return inp, as_f64(S.cpu()), stats, Pref
@@ -133,32 +138,35 @@ def test_newton_tiny_converges_to_sequential(cuda_device):
         assert abs(g - o) <= 1e-3 * (1 + o), (k, g, o)
 
 
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("B,T,d", [(2, 50, 40), (1, 1, 1), (2, 31, 33), (3, 64, 70)])
-def test_newton_converges_to_sequential_sigmoid(B, T, d, cuda_device):
+def test_newton_converges_to_sequential_sigmoid(B, T, d, carry_mode, cuda_device):
     w = Workload("t", B, T, 16, d, "f32", "sigmoid", 0.5, 11, 1e-6, 64)
-    inp, S, st, Pref = _newton_case(w)
+    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode)
     ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), "sigmoid")
     assert st["error"] == 0 and st["converged"], st
     assert _h_err(S, ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 @pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256), (1, 300, 36), (2, 200, 40)])
-def test_newton_status_agrees_with_oracle(forget, B, T, d, cuda_device):
+def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, cuda_device):
     w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
-    inp, S, st, Pref = _newton_case(w)
+    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode)
     _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol)
     if _check_status_against_oracle(st, ost):
         ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget)
         assert _h_err(S, ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("K", [1, 3])
-def test_newton_fixed_k_prefix_exact(K, cuda_device):
+def test_newton_fixed_k_prefix_exact(K, carry_mode, cuda_device):
     """After K Newton iterations the first K steps equal the sequential
     trajectory whatever the rest of the iterate looks like."""
     w = WORKLOADS["slstm_f32_b8_t1024_d256"]
-    inp, S, st, Pref = _newton_case(w, fixed_k=K)
+    inp, S, st, Pref = _newton_case(w, fixed_k=K, carry_mode=carry_mode)
     assert st["iters"] == K
     ref = oracle.sequential_btgd(Pref[:, :K], as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
     assert _h_err(S[:, :K], ref) <= TOL_F32

@@ -52,15 +52,21 @@ def _h_err(S_gpu, S_ref):
 LENGTHS = [[5, 0, 1, 40, 33, 64, 7, 0], [70, 3], [32, 32, 32], [1, 1, 1, 1, 1], [17]]
 
 
+# carry modes: 1 = one fused launch per iteration (decoupled look-back),
+# 2 = two passes with a scan of tile aggregates in between
+CARRY_MODES = [1, 2]
+
+
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 @pytest.mark.parametrize("d", [40, 33])
 @pytest.mark.parametrize("lengths", LENGTHS)
-def test_varlen_fixed_k_matches_oracle(lengths, d, forget, cuda_device):
+def test_varlen_fixed_k_matches_oracle(lengths, d, forget, carry_mode, cuda_device):
     K = 3
     c = _case(lengths, d, 12, "f32", forget, 41)
     P, Pref = _preact(c)
     S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), forget=forget, max_iters=K,
-                                      fixed=True, tol=1e-6)
+                                      fixed=True, tol=1e-6, carry_mode=carry_mode)
     torch.cuda.synchronize()
     got = as_f64(S.cpu())
     assert api.read_stats(st)["iters"] == K
@@ -78,12 +84,14 @@ def test_varlen_fixed_k_matches_oracle(lengths, d, forget, cuda_device):
             assert _h_err(got[a:b], seq[a:b]) <= TOL_F32, (k, a, b)
 
 
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("d", [40, 33])
-def test_varlen_converges_to_sequential(d, cuda_device):
+def test_varlen_converges_to_sequential(d, carry_mode, cuda_device):
     lengths = [12, 0, 1, 40, 33, 9]
     c = _case(lengths, d, 16, "f32", "sigmoid", 42)
     P, Pref = _preact(c)
-    S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), max_iters=64, tol=1e-6)
+    S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), max_iters=64, tol=1e-6,
+                                      carry_mode=carry_mode)
     torch.cuda.synchronize()
     s = api.read_stats(st)
     assert s["error"] == 0 and s["converged"], s
@@ -144,7 +152,8 @@ def test_varlen_backward_matches_oracle(d_in, d, dtype, forget, cuda_device):
     assert not out["ds0"][1].any() and not out["ds0"][7].any()
 
 
-def test_varlen_nan_in_one_sequence_reports_divergence(cuda_device):
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+def test_varlen_nan_in_one_sequence_reports_divergence(carry_mode, cuda_device):
     """A non-finite value inside a short sequence does not leak into the next
     sequence (its start ignores the state before it), so the steps after it in
     the same thread are finite again; the residual maximum must still keep the
@@ -154,7 +163,7 @@ def test_varlen_nan_in_one_sequence_reports_divergence(cuda_device):
     P, _ = _preact(c)
     P[0, 1, 5] = float("nan")    # first sequence, step 0, gate i of feature 5
     S, st = api.newton_forward_varlen(P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]), max_iters=2, fixed=True,
-                                      tol=1e-6)
+                                      tol=1e-6, carry_mode=carry_mode)
     torch.cuda.synchronize()
     s = api.read_stats(st)
     assert s["diverged"] and s["error"] == 3, s
