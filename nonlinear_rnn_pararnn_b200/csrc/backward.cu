@@ -38,6 +38,7 @@ struct BwdArgs {
     float *ds0;       // (B, 4, d) or null
     unsigned *ticket;
     CarryArgs ca;
+    float *cin_buf;   // two-pass carry: [n_tiles][4][32] carry entering each tile (chain layout)
     const unsigned *vmask;   // packed sequences: head-flag words (one per 32 steps), else null
     const int *vseq;         // packed sequences: sequence index at each head step
     int T, d, groups_per_row, n_tiles, vec16, dpt_vec8;
@@ -181,7 +182,12 @@ SLSTM_DEVINL void bwd_issue_load(const BwdArgs &a, const BwdMaps &m, BwdSmem &sm
 // VARLEN: packed ragged sequences (B = 1): J_{t+1} is zero when step t + 1
 // starts a sequence, and a sequence's first step takes its s0 (and yields its
 // ds0) as the dense kernel does at t = 0.
-template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN>
+// MODE: as the Newton iteration's (BWD_FUSED: carry by decoupled look-back;
+// BWD_AGG: store each tile's aggregate map only; BWD_APPLY: the fused pass
+// with the carry entering every tile known from the scan of the aggregates).
+constexpr int BWD_FUSED = 0, BWD_AGG = 1, BWD_APPLY = 2;
+
+template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN, int MODE>
 __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, const __grid_constant__ BwdMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -194,8 +200,9 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
     const bool chain_warp = warp < 4;
 
     if (threadIdx.x == 0) {
-        bwd_decode(a, atomicAdd(a.ticket, 1u), sm.info[0]);
-        bwd_decode(a, atomicAdd(a.ticket, 1u), sm.info[1]);
+        // BWD_AGG tiles are independent: a static order needs no counter
+        bwd_decode(a, MODE == BWD_AGG ? blockIdx.x : atomicAdd(a.ticket, 1u), sm.info[0]);
+        bwd_decode(a, MODE == BWD_AGG ? blockIdx.x + gridDim.x : atomicAdd(a.ticket, 1u), sm.info[1]);
     }
     if (TMA && threadIdx.x == BWD_TMA_THREAD) {
         mbar_init(&sm.bar[0], 1);
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         if (ti.ticket >= (unsigned)a.n_tiles) break;
         const int rn = ring == 2 ? 0 : ring + 1;
         unsigned after = 0;
-        if (threadIdx.x == 0) after = atomicAdd(a.ticket, 1u);
+        if (threadIdx.x == 0) after = MODE == BWD_AGG ? blockIdx.x + (it + 2u) * gridDim.x : atomicAdd(a.ticket, 1u);
         if (TMA) {
             if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, BWD_TMA_WAIT_NS)) {
                 atomicOr(a.ca.error, 2u);
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         }
 
         // looks at the predecessor's (later-in-time) inclusive prefix
-        const bool look = chain_warp && chunk > 0;
+        const bool look = MODE == BWD_FUSED && chain_warp && chunk > 0;
         const unsigned long long *predw = a.ca.incw + chain_word(ticket - G, warp, lane);
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
@@ -284,17 +291,6 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         maps_store(sm.u.m, warp, lane, agg);
         if (threadIdx.x == 0) bwd_decode(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
 
-        // ---- carry ----
-        float c = 0.f;   // chunk 0: nothing enters after the sequence's last step
-        bool ok = true;
-        if (look) {
-            if ((unsigned)(w1 >> 32) == a.ca.epoch) {
-                c = __uint_as_float((unsigned)w1);
-            } else {
-                ok = (unsigned)(w2 >> 32) == a.ca.epoch;
-                c = __uint_as_float((unsigned)w2);
-            }
-        }
         // warps whose steps contain such a reset (bits rl + 1 of their steps)
         unsigned whead = 0u;
         if (VARLEN) {
@@ -302,138 +298,185 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             for (int w = 0; w < NW; ++w)
                 whead |= (((ti.hmask >> (TT - L - w * L + 1)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
         }
-        const bool fast = __syncthreads_and(ok);
-        if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
-        if (fast) {
-            if (chain_warp) {
-                c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead);
-                st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
-            }
-        } else if (warp == 0) {
-            tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false,
-                                    whead);
-        }
-        __syncthreads();   // the maps are dead from here on; the dP staging takes their place
-
-        // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
-        float lam[4];
+        if constexpr (MODE == BWD_AGG) {
+            if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
+            // the tile's aggregate map: a tree over the warp maps in processing
+            // order (at step h, warp w composes slot (2w+2)h - 1 with slot
+            // (2w+1)h - 1 into the former; a part holding a reset ignores what
+            // enters it and is kept as it is)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][sw(e, lane)];
-        float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
-        float dv[L][4];   // dP of the thread's steps (gate order z, i, f, o)
-#pragma unroll
-        for (int i = 0; i < L; ++i) {
-            const int rl = TT - 1 - (warp * L + i);
-            const int t = t_lo + rl;
-            if (VARLEN && ((ti.hmask >> (rl + 1)) & 1ull)) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) lam[e] = 0.0f;
-            }
-            jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
-            lam[3] += sm.dH[st][rl][lane];
-            float prev[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
-            Cell cc;
-            CellG g;
-            const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
-            if (head) {
-                // the state before the sequence is its s0; ds0 = J^T lambda at its first step
-                const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
-                cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
-                                              sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
-                                              ri, rf, ro, cc, &g);
-                if (a.ds0 && jv) {
-                    float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
-                    jacT_mul(cc, v0, v1, v2, v3);
-                    float *q = a.ds0 + sq * 4 * d + jj;
-                    q[0] = v0;
-                    q[d] = v1;
-                    q[2 * d] = v2;
-                    q[3 * d] = v3;
-                }
-            } else {
-                cell_eval<FORGET, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
-                                               sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
-                                               ri, rf, ro, cc, &g);
-            }
-            const bool tv = t >= 0;   // steps before 0 (last chunk only) contribute nothing
-            dv[i][0] = tv ? fmaf(g.gcz, lam[0], g.ghz * lam[3]) : 0.f;
-            dv[i][1] = tv ? fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3]))) : 0.f;
-            dv[i][2] = tv ? fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3]))) : 0.f;
-            dv[i][3] = tv ? g.gho * lam[3] : 0.f;
-            if (!BF16OUT && jv && tv) {
-                float *pd = a.dP + (row0 + t) * 4 * d + jj;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pd[e * d] = dv[i][e];
-            }
-            const float hp = prev[3];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                dr[e] = fmaf(dv[i][e], hp, dr[e]);
-                dbs[e] += dv[i][e];
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            sm.u.o.part[warp][e][lane] = jv ? dr[e] : 0.f;
-            sm.u.o.part[warp][4 + e][lane] = jv ? dbs[e] : 0.f;
-        }
-        if (BF16OUT) {
-            // the thread's 4 steps are 4 consecutive t: t_lo + 28 - 4w .. t_lo + 31 - 4w
-            const int rb = TT - L - warp * L;
-#pragma unroll
-            for (int gi = 0; gi < 4; ++gi) {
-                const __nv_bfloat162 h01 = __floats2bfloat162_rn(dv[3][gi], dv[2][gi]);
-                const __nv_bfloat162 h23 = __floats2bfloat162_rn(dv[1][gi], dv[0][gi]);
-                const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
-                const __nv_bfloat162 l01 = __floats2bfloat162_rn(dv[3][gi] - f01.x, dv[2][gi] - f01.y);
-                const __nv_bfloat162 l23 = __floats2bfloat162_rn(dv[1][gi] - f23.x, dv[0][gi] - f23.y);
-                uint2 hv, lv;
-                hv.x = *reinterpret_cast<const unsigned *>(&h01);
-                hv.y = *reinterpret_cast<const unsigned *>(&h23);
-                lv.x = *reinterpret_cast<const unsigned *>(&l01);
-                lv.y = *reinterpret_cast<const unsigned *>(&l23);
-                *reinterpret_cast<uint2 *>(&sm.u.o.dpt[0][gi][lane][rb]) = hv;
-                *reinterpret_cast<uint2 *>(&sm.u.o.dpt[1][gi][lane][rb]) = lv;
-            }
-        }
-        __syncthreads();
-        {
-            // 256 threads: thread (e, lane) sums entry e over the warps
-            const int e = threadIdx.x >> 5;   // 0..7
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < NW; ++w) acc += sm.u.o.part[w][e][lane];
-            a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
-        }
-        if (BF16OUT) {
-            // rows (part, gate, feature) of the transposed pair, 32 steps each;
-            // nothing before t = 0 (those addresses hold the previous batch row)
-            if (a.dpt_vec8) {
-                // 8-byte pieces of 4 steps: piece q of row r is index 8 r + q
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int idx = threadIdx.x + NW * 32 * k;
-                    const int r = idx >> 3, q = idx & 7;
-                    const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
-                    const int t = t_lo + 4 * q;
-                    if (t >= 0 && ti.j0 + jl < a.d) {
-                        const uint2 v = *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
-                        __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
-                        *reinterpret_cast<uint2 *>(dst + ((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t) = v;
+            for (int h = 1; h < NW; h *= 2) {
+                __syncthreads();
+                if (warp < NW / (2 * h)) {
+                    const int hi = (2 * warp + 2) * h - 1, lo = (2 * warp + 1) * h - 1;
+                    const bool hhead = VARLEN && (((whead >> ((2 * warp + 1) * h)) & ((1u << h) - 1u)) != 0u);
+                    if (!hhead) {
+                        Aff x, y;
+                        maps_load(sm.u.m, hi, lane, x);
+                        maps_load(sm.u.m, lo, lane, y);
+                        aff_compose(x, y, x);
+                        maps_store(sm.u.m, hi, lane, x);
                     }
                 }
-            } else {
-                const int tl = threadIdx.x & 31;
-                const int t = t_lo + tl;
-                for (int r = warp; r < 2 * 4 * 32; r += NW) {
-                    const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
-                    if (t >= 0 && ti.j0 + jl < a.d) {
-                        __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
-                        dst[((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t] = sm.u.o.dpt[part][gi][jl][tl];
+            }
+            __syncthreads();
+            if (warp == 0) {
+                Aff x;
+                maps_load(sm.u.m, NW - 1, lane, x);
+                float *dst = a.ca.agg + (size_t)ticket * 20 * 32 + lane;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
+                if (lane == 0) a.ca.flags[ticket] = whead ? 1u : 0u;
+            }
+        } else {
+
+            // ---- carry ----
+            float c = 0.f;   // chunk 0: nothing enters after the sequence's last step
+            bool ok = true;
+            if (MODE == BWD_APPLY && chain_warp) c = a.cin_buf[chain_word(ticket, warp, lane)];
+            if (look) {
+                if ((unsigned)(w1 >> 32) == a.ca.epoch) {
+                    c = __uint_as_float((unsigned)w1);
+                } else {
+                    ok = (unsigned)(w2 >> 32) == a.ca.epoch;
+                    c = __uint_as_float((unsigned)w2);
+                }
+            }
+            const bool fast = __syncthreads_and(ok);
+            if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
+            if (fast) {
+                if (chain_warp) {
+                    c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead);
+                    if (MODE == BWD_FUSED) st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+                }
+            } else if (warp == 0) {
+                tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false,
+                                        whead);
+            }
+            __syncthreads();   // the maps are dead from here on; the dP staging takes their place
+
+            // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
+            float lam[4];
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][sw(e, lane)];
+            float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
+            float dv[L][4];   // dP of the thread's steps (gate order z, i, f, o)
+    #pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int rl = TT - 1 - (warp * L + i);
+                const int t = t_lo + rl;
+                if (VARLEN && ((ti.hmask >> (rl + 1)) & 1ull)) {
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) lam[e] = 0.0f;
+                }
+                jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
+                lam[3] += sm.dH[st][rl][lane];
+                float prev[4];
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
+                Cell cc;
+                CellG g;
+                const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
+                if (head) {
+                    // the state before the sequence is its s0; ds0 = J^T lambda at its first step
+                    const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
+                    cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
+                                                  sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
+                                                  ri, rf, ro, cc, &g);
+                    if (a.ds0 && jv) {
+                        float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
+                        jacT_mul(cc, v0, v1, v2, v3);
+                        float *q = a.ds0 + sq * 4 * d + jj;
+                        q[0] = v0;
+                        q[d] = v1;
+                        q[2 * d] = v2;
+                        q[3 * d] = v3;
+                    }
+                } else {
+                    cell_eval<FORGET, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
+                                                   sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
+                                                   ri, rf, ro, cc, &g);
+                }
+                const bool tv = t >= 0;   // steps before 0 (last chunk only) contribute nothing
+                dv[i][0] = tv ? fmaf(g.gcz, lam[0], g.ghz * lam[3]) : 0.f;
+                dv[i][1] = tv ? fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3]))) : 0.f;
+                dv[i][2] = tv ? fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3]))) : 0.f;
+                dv[i][3] = tv ? g.gho * lam[3] : 0.f;
+                if (!BF16OUT && jv && tv) {
+                    float *pd = a.dP + (row0 + t) * 4 * d + jj;
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) pd[e * d] = dv[i][e];
+                }
+                const float hp = prev[3];
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    dr[e] = fmaf(dv[i][e], hp, dr[e]);
+                    dbs[e] += dv[i][e];
+                }
+            }
+    #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sm.u.o.part[warp][e][lane] = jv ? dr[e] : 0.f;
+                sm.u.o.part[warp][4 + e][lane] = jv ? dbs[e] : 0.f;
+            }
+            if (BF16OUT) {
+                // the thread's 4 steps are 4 consecutive t: t_lo + 28 - 4w .. t_lo + 31 - 4w
+                const int rb = TT - L - warp * L;
+    #pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    const __nv_bfloat162 h01 = __floats2bfloat162_rn(dv[3][gi], dv[2][gi]);
+                    const __nv_bfloat162 h23 = __floats2bfloat162_rn(dv[1][gi], dv[0][gi]);
+                    const float2 f01 = __bfloat1622float2(h01), f23 = __bfloat1622float2(h23);
+                    const __nv_bfloat162 l01 = __floats2bfloat162_rn(dv[3][gi] - f01.x, dv[2][gi] - f01.y);
+                    const __nv_bfloat162 l23 = __floats2bfloat162_rn(dv[1][gi] - f23.x, dv[0][gi] - f23.y);
+                    uint2 hv, lv;
+                    hv.x = *reinterpret_cast<const unsigned *>(&h01);
+                    hv.y = *reinterpret_cast<const unsigned *>(&h23);
+                    lv.x = *reinterpret_cast<const unsigned *>(&l01);
+                    lv.y = *reinterpret_cast<const unsigned *>(&l23);
+                    *reinterpret_cast<uint2 *>(&sm.u.o.dpt[0][gi][lane][rb]) = hv;
+                    *reinterpret_cast<uint2 *>(&sm.u.o.dpt[1][gi][lane][rb]) = lv;
+                }
+            }
+            __syncthreads();
+            {
+                // 256 threads: thread (e, lane) sums entry e over the warps
+                const int e = threadIdx.x >> 5;   // 0..7
+                float acc = 0.f;
+    #pragma unroll
+                for (int w = 0; w < NW; ++w) acc += sm.u.o.part[w][e][lane];
+                a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
+            }
+            if (BF16OUT) {
+                // rows (part, gate, feature) of the transposed pair, 32 steps each;
+                // nothing before t = 0 (those addresses hold the previous batch row)
+                if (a.dpt_vec8) {
+                    // 8-byte pieces of 4 steps: piece q of row r is index 8 r + q
+    #pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int idx = threadIdx.x + NW * 32 * k;
+                        const int r = idx >> 3, q = idx & 7;
+                        const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
+                        const int t = t_lo + 4 * q;
+                        if (t >= 0 && ti.j0 + jl < a.d) {
+                            const uint2 v = *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
+                            __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                            *reinterpret_cast<uint2 *>(dst + ((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t) = v;
+                        }
+                    }
+                } else {
+                    const int tl = threadIdx.x & 31;
+                    const int t = t_lo + tl;
+                    for (int r = warp; r < 2 * 4 * 32; r += NW) {
+                        const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
+                        if (t >= 0 && ti.j0 + jl < a.d) {
+                            __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
+                            dst[((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t] = sm.u.o.dpt[part][gi][jl][tl];
+                        }
                     }
                 }
             }
@@ -504,10 +547,10 @@ int sm_count_bwd()
     return n;
 }
 
-template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN>
-cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
+template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN, int MODE>
+cudaError_t launch_adjoint_mode(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
 {
-    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT, TMA, VARLEN>;
+    auto kern = adjoint_vjp_kernel<FORGET, BF16OUT, TMA, VARLEN, MODE>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)BWD_SMEM_BYTES);
@@ -521,26 +564,42 @@ cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, cudaStream_t st)
     return cudaGetLastError();
 }
 
+// Scratch of the two-pass carry (null scan.cin: one fused pass).
+struct TwoPass {
+    TileScanArgs scan;
+};
+
+template <int FORGET, bool BF16OUT, bool TMA, bool VARLEN>
+cudaError_t launch_adjoint(const BwdArgs &a, const BwdMaps &m, const TwoPass &tp, cudaStream_t st)
+{
+    if (!tp.scan.cin) return launch_adjoint_mode<FORGET, BF16OUT, TMA, VARLEN, BWD_FUSED>(a, m, st);
+    cudaError_t e = launch_adjoint_mode<FORGET, BF16OUT, TMA, VARLEN, BWD_AGG>(a, m, st);
+    if (e == cudaSuccess) e = launch_tile_scan(tp.scan, st);
+    if (e == cudaSuccess) e = launch_adjoint_mode<FORGET, BF16OUT, TMA, VARLEN, BWD_APPLY>(a, m, st);
+    return e;
+}
+
 template <int FORGET, bool VARLEN>
-cudaError_t launch_adjoint_v(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, cudaStream_t st)
+cudaError_t launch_adjoint_v(const BwdArgs &a, const BwdMaps &m, const TwoPass &tp, bool tma, bool bf16out,
+                             cudaStream_t st)
 {
     if (tma)
-        return bf16out ? launch_adjoint<FORGET, true, true, VARLEN>(a, m, st)
-                       : launch_adjoint<FORGET, false, true, VARLEN>(a, m, st);
-    return bf16out ? launch_adjoint<FORGET, true, false, VARLEN>(a, m, st)
-                   : launch_adjoint<FORGET, false, false, VARLEN>(a, m, st);
+        return bf16out ? launch_adjoint<FORGET, true, true, VARLEN>(a, m, tp, st)
+                       : launch_adjoint<FORGET, false, true, VARLEN>(a, m, tp, st);
+    return bf16out ? launch_adjoint<FORGET, true, false, VARLEN>(a, m, tp, st)
+                   : launch_adjoint<FORGET, false, false, VARLEN>(a, m, tp, st);
 }
 
 template <int FORGET>
-cudaError_t launch_adjoint_any(const BwdArgs &a, const BwdMaps &m, bool tma, bool bf16out, bool varlen,
-                               cudaStream_t st)
+cudaError_t launch_adjoint_any(const BwdArgs &a, const BwdMaps &m, const TwoPass &tp, bool tma, bool bf16out,
+                               bool varlen, cudaStream_t st)
 {
-    return varlen ? launch_adjoint_v<FORGET, true>(a, m, tma, bf16out, st)
-                  : launch_adjoint_v<FORGET, false>(a, m, tma, bf16out, st);
+    return varlen ? launch_adjoint_v<FORGET, true>(a, m, tp, tma, bf16out, st)
+                  : launch_adjoint_v<FORGET, false>(a, m, tp, tma, bf16out, st);
 }
 
 struct Layout {
-    size_t ticket, flags, incw, agg, partial, dP, dpt, wpart, err, total;
+    size_t ticket, flags, incw, agg, partial, dP, dpt, wpart, err, cin, blk_agg, blk_head, blk_cin, total;
     int groups_per_row, n_groups, n_chunks, n_tiles, splits;
     long long n, ldT, ld4;
 };
@@ -596,6 +655,11 @@ Layout layout(int B, int T, int d_in, int d_h)
     l.dpt = take(2 * sizeof(__nv_bfloat16) * (size_t)(4LL * d_h) * (size_t)l.ldT);
     l.wpart = take(sizeof(float) * (size_t)l.splits * 4 * d_h * d_in);
     l.err = take(256);
+    l.cin = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
+    const size_t nblk = (size_t)l.n_groups * scan_blocks(l.n_chunks);
+    l.blk_agg = take(sizeof(float) * 20 * 32 * nblk);
+    l.blk_head = take(sizeof(unsigned) * nblk);
+    l.blk_cin = take(sizeof(float) * 4 * 32 * nblk);
     l.total = off;
     return l;
 }
@@ -665,8 +729,19 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
                      make_map_f32_3d(&m.S, S, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
                      make_map_f32_3d(&m.P, P, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
                      make_map_f32_3d(&m.H, dH, d_h, T, B, d_h, (uint64_t)T * d_h, 32, TT);
-    e = (forget == SLSTM_FORGET_EXP) ? launch_adjoint_any<SLSTM_FORGET_EXP>(a, m, tma, tc, vl != nullptr, st)
-                                     : launch_adjoint_any<SLSTM_FORGET_SIGMOID>(a, m, tma, tc, vl != nullptr, st);
+    // few feature groups and a long time axis: two passes with a scan of the
+    // tile aggregates in between instead of waiting for predecessors
+    TwoPass tp;
+    memset(&tp, 0, sizeof(tp));
+    a.cin_buf = nullptr;
+    if (prefer_two_pass(l.n_groups, (long long)l.n_chunks * TT, sm_count_bwd())) {
+        a.cin_buf = reinterpret_cast<float *>(base + l.cin);
+        tp.scan = TileScanArgs{a.ca.agg, a.ca.flags, reinterpret_cast<float *>(base + l.blk_agg),
+                               reinterpret_cast<unsigned *>(base + l.blk_head), reinterpret_cast<float *>(base + l.blk_cin),
+                               a.cin_buf, nullptr, l.n_groups, l.n_chunks, scan_blocks(l.n_chunks)};
+    }
+    e = (forget == SLSTM_FORGET_EXP) ? launch_adjoint_any<SLSTM_FORGET_EXP>(a, m, tp, tma, tc, vl != nullptr, st)
+                                     : launch_adjoint_any<SLSTM_FORGET_SIGMOID>(a, m, tp, tma, tc, vl != nullptr, st);
     if (e != cudaSuccess) return e;
     reduce_partials_kernel<<<dim3(l.groups_per_row, 8), 256, 0, st>>>(a.partial, dR, db, B, l.n_chunks,
                                                                    l.groups_per_row, d_h);

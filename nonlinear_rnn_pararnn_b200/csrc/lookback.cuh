@@ -462,6 +462,145 @@ SLSTM_DEVINL void tile_carry_fallback(const CarryArgs &ca, const MapArr *m, CinA
         ticket, withhold, carry, whead);
 }
 
+namespace {
+
+// ---- two-pass carry ----------------------------------------------------------
+// Between the two passes of a blocked scan: the carry entering every tile,
+// from the aggregates of the tiles before it in its feature group (chunk 0
+// gets none).  Tile aggregates are [tile][20][32] (entry-major, lane =
+// feature; A row-major, then b), carries [tile][4][32].  A group's chunks are cut into blocks of SCAN_BLK: the
+// aggregates of every block are composed (scan_block_agg), the blocks of a
+// group are walked in order (scan_block_carry), and every block applies its
+// aggregates from the carry entering it (scan_tile_carry).  One warp per
+// (group, block), lane = feature; a tile with a sequence start passes on its
+// offset whatever enters it.
+constexpr int SCAN_BLK = 32;
+
+SLSTM_DEVINL void load_agg(const float *src, int lane, Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
+}
+
+SLSTM_DEVINL void store_agg(float *dst, int lane, const Aff &x)
+{
+#pragma unroll
+    for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = x.a[e];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = x.b[e];
+}
+
+struct TileScanArgs {
+    const float *agg;          // [n_tiles][20][32] tile aggregates
+    const unsigned *head;      // [n_tiles] nonzero: the tile holds a sequence start
+    float *blk_agg;            // [n_groups][n_blk][20][32]
+    unsigned *blk_head;        // [n_groups][n_blk]
+    float *blk_cin;            // [n_groups][n_blk][4][32]
+    float *cin;                // [n_tiles][4][32] the carry entering each tile
+    const unsigned *done;      // nonzero: the call has finished (or null)
+    int n_groups, n_chunks, n_blk;
+};
+
+// (group, block) per warp: the composition of the block's tile aggregates.
+__global__ void __launch_bounds__(256) scan_block_agg(TileScanArgs s)
+{
+    if (s.done && *(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= (long long)s.n_groups * s.n_blk) return;
+    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
+    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
+    const size_t G = (size_t)s.n_groups;
+    Aff acc, x;
+    load_agg(s.agg + ((size_t)c0 * G + g) * 640, lane, acc);
+    bool hd = s.head[(size_t)c0 * G + g] != 0u;
+    for (int c = c0 + 1; c < c1; ++c) {
+        load_agg(s.agg + ((size_t)c * G + g) * 640, lane, x);
+        if (s.head[(size_t)c * G + g] != 0u) {
+            acc = x;   // starts afresh: ignores what came before
+            hd = true;
+        } else {
+            aff_compose(x, acc, acc);
+        }
+    }
+    store_agg(s.blk_agg + (size_t)wid * 640, lane, acc);
+    if (lane == 0) s.blk_head[wid] = hd ? 1u : 0u;
+}
+
+// One warp per group: the carry entering each block.
+__global__ void __launch_bounds__(256) scan_block_carry(TileScanArgs s)
+{
+    if (s.done && *(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (g >= s.n_groups) return;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    Aff x;
+    for (int k = 0; k < s.n_blk; ++k) {
+        const size_t w = (size_t)g * s.n_blk + k;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.blk_cin[w * 128 + e * 32 + lane] = v[e];
+        if (k + 1 == s.n_blk) break;
+        load_agg(s.blk_agg + w * 640, lane, x);
+        if (s.blk_head[w] != 0u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
+        } else {
+            aff_apply(x, v, v);
+        }
+    }
+}
+
+// (group, block) per warp: the carry entering each tile of the block.
+__global__ void __launch_bounds__(256) scan_tile_carry(TileScanArgs s)
+{
+    if (s.done && *(volatile const unsigned *)s.done) return;
+    const int lane = threadIdx.x & 31;
+    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (wid >= (long long)s.n_groups * s.n_blk) return;
+    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
+    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
+    const size_t G = (size_t)s.n_groups;
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = s.blk_cin[(size_t)wid * 128 + e * 32 + lane];
+    Aff x;
+    for (int c = c0; c < c1; ++c) {
+        const size_t t = (size_t)c * G + g;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.cin[t * 128 + e * 32 + lane] = v[e];
+        if (c + 1 == c1) break;
+        load_agg(s.agg + t * 640, lane, x);
+        if (s.head[t] != 0u) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
+        } else {
+            aff_apply(x, v, v);
+        }
+    }
+}
+
+// The three scan launches on `st`.
+inline cudaError_t launch_tile_scan(const TileScanArgs &s, cudaStream_t st)
+{
+    const long long nw = (long long)s.n_groups * s.n_blk;
+    scan_block_agg<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(s);
+    scan_block_carry<<<(s.n_groups + 7) / 8, 256, 0, st>>>(s);
+    scan_tile_carry<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(s);
+    return cudaGetLastError();
+}
+
+inline int scan_blocks(int n_chunks) { return (n_chunks + SCAN_BLK - 1) / SCAN_BLK; }
+
+// Two passes pay off with few feature groups and a long time axis (measured
+// on B200 for the Newton iteration: faster with 8-32 groups from 16 384 steps
+// on, slower with 64 groups or 8192 steps).
+inline bool prefer_two_pass(int n_groups, long long steps, int sms) { return 4 * n_groups <= sms && steps >= 16384; }
+
+}  // namespace
+
 // cp.async copies into shared memory (zero-fill beyond `bytes`).
 SLSTM_DEVINL uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 

@@ -287,122 +287,6 @@ __device__ void finalize(const Args &a, int k, bool resid)
     if (done) atomicExch(&c->done, 1u);
 }
 
-// Between the two passes of an iteration: the carry entering every tile,
-// from the aggregates of the tiles before it in its feature group (chunk 0
-// gets none).  A group's chunks are cut into blocks of SCAN_BLK: the
-// aggregates of every block are composed (scan_block_agg), the blocks of a
-// group are walked in order (scan_block_carry), and every block applies its
-// aggregates from the carry entering it (scan_tile_carry).  One warp per
-// (group, block), lane = feature; a tile with a sequence start passes on its
-// offset whatever enters it.
-constexpr int SCAN_BLK = 32;
-
-SLSTM_DEVINL void load_agg(const float *src, int lane, Aff &x)
-{
-#pragma unroll
-    for (int e = 0; e < 16; ++e) x.a[e] = __ldcg(src + e * 32 + lane);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) x.b[e] = __ldcg(src + (16 + e) * 32 + lane);
-}
-
-SLSTM_DEVINL void store_agg(float *dst, int lane, const Aff &x)
-{
-#pragma unroll
-    for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = x.a[e];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dst[(16 + e) * 32 + lane] = x.b[e];
-}
-
-struct ScanArgs {
-    const float *agg;          // [n_tiles][20][32] tile aggregates
-    const unsigned *head;      // [n_tiles] nonzero: the tile holds a sequence start
-    float *blk_agg;            // [n_groups][n_blk][20][32]
-    unsigned *blk_head;        // [n_groups][n_blk]
-    float *blk_cin;            // [n_groups][n_blk][4][32]
-    float *cin;                // [n_tiles][4][32] the carry entering each tile
-    const unsigned *done;
-    int n_groups, n_chunks, n_blk;
-};
-
-// (group, block) per warp: the composition of the block's tile aggregates.
-__global__ void __launch_bounds__(256) scan_block_agg(ScanArgs s)
-{
-    if (*(volatile const unsigned *)s.done) return;
-    const int lane = threadIdx.x & 31;
-    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (wid >= (long long)s.n_groups * s.n_blk) return;
-    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
-    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
-    const size_t G = (size_t)s.n_groups;
-    Aff acc, x;
-    load_agg(s.agg + ((size_t)c0 * G + g) * 640, lane, acc);
-    bool hd = s.head[(size_t)c0 * G + g] != 0u;
-    for (int c = c0 + 1; c < c1; ++c) {
-        load_agg(s.agg + ((size_t)c * G + g) * 640, lane, x);
-        if (s.head[(size_t)c * G + g] != 0u) {
-            acc = x;   // starts afresh: ignores what came before
-            hd = true;
-        } else {
-            aff_compose(x, acc, acc);
-        }
-    }
-    store_agg(s.blk_agg + (size_t)wid * 640, lane, acc);
-    if (lane == 0) s.blk_head[wid] = hd ? 1u : 0u;
-}
-
-// One warp per group: the carry entering each block.
-__global__ void __launch_bounds__(256) scan_block_carry(ScanArgs s)
-{
-    if (*(volatile const unsigned *)s.done) return;
-    const int lane = threadIdx.x & 31;
-    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (g >= s.n_groups) return;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    Aff x;
-    for (int k = 0; k < s.n_blk; ++k) {
-        const size_t w = (size_t)g * s.n_blk + k;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s.blk_cin[w * 128 + e * 32 + lane] = v[e];
-        if (k + 1 == s.n_blk) break;
-        load_agg(s.blk_agg + w * 640, lane, x);
-        if (s.blk_head[w] != 0u) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
-        } else {
-            aff_apply(x, v, v);
-        }
-    }
-}
-
-// (group, block) per warp: the carry entering each tile of the block.
-__global__ void __launch_bounds__(256) scan_tile_carry(ScanArgs s)
-{
-    if (*(volatile const unsigned *)s.done) return;
-    const int lane = threadIdx.x & 31;
-    const long long wid = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (wid >= (long long)s.n_groups * s.n_blk) return;
-    const int g = (int)(wid / s.n_blk), k = (int)(wid % s.n_blk);
-    const int c0 = k * SCAN_BLK, c1 = min(c0 + SCAN_BLK, s.n_chunks);
-    const size_t G = (size_t)s.n_groups;
-    float v[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) v[e] = s.blk_cin[(size_t)wid * 128 + e * 32 + lane];
-    Aff x;
-    for (int c = c0; c < c1; ++c) {
-        const size_t t = (size_t)c * G + g;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s.cin[t * 128 + e * 32 + lane] = v[e];
-        if (c + 1 == c1) break;
-        load_agg(s.agg + t * 640, lane, x);
-        if (s.head[t] != 0u) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = x.b[e];
-        } else {
-            aff_apply(x, v, v);
-        }
-    }
-}
-
 // TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
 // stage, stores per warp from the stage walk B wrote); otherwise by cp.async
 // and plain stores.
@@ -797,14 +681,9 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         if (two_pass) {
             if ((e = launch_pass<FORGET, TMA, VARLEN, MODE_AGG>(a, m, k, false, sms, st)) != cudaSuccess) return e;
             const int n_chunks = a.n_tiles / a.n_groups;
-            const int n_blk = (n_chunks + SCAN_BLK - 1) / SCAN_BLK;
-            const ScanArgs sa{a.agg, a.flags, a.blk_agg, a.blk_head, a.blk_cin, a.cin_buf, &a.ctrl->done,
-                              a.n_groups, n_chunks, n_blk};
-            const long long nw = (long long)a.n_groups * n_blk;
-            scan_block_agg<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
-            scan_block_carry<<<(a.n_groups + 7) / 8, 256, 0, st>>>(sa);
-            scan_tile_carry<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            const TileScanArgs sa{a.agg, a.flags, a.blk_agg, a.blk_head, a.blk_cin, a.cin_buf, &a.ctrl->done,
+                              a.n_groups, n_chunks, scan_blocks(n_chunks)};
+            if ((e = launch_tile_scan(sa, st)) != cudaSuccess) return e;
             e = launch_pass<FORGET, TMA, VARLEN, MODE_APPLY>(a, m, k, resid, sms, st);
         } else {
             e = launch_pass<FORGET, TMA, VARLEN, MODE_FUSED>(a, m, k, resid, sms, st);
@@ -839,7 +718,7 @@ Layout layout(int B, int T, int d)
     l.bnd0 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.bnd1 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.cin = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
-    const size_t nblk = (size_t)l.n_groups * ((l.n_chunks + SCAN_BLK - 1) / SCAN_BLK);
+    const size_t nblk = (size_t)l.n_groups * scan_blocks(l.n_chunks);
     l.blk_agg = take(sizeof(float) * 20 * 32 * nblk);
     l.blk_head = take(sizeof(unsigned) * nblk);
     l.blk_cin = take(sizeof(float) * 4 * 32 * nblk);
@@ -937,14 +816,12 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
                      make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
                      make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);
     const bool v = vl != nullptr;
-    // With few feature groups and many chunks, most tiles of a fused launch
-    // would wait for their predecessor: take the two passes instead (measured
-    // on B200: faster from 1024 chunks down to 256 with 8-32 groups, slower
-    // with 64 groups or 128 chunks).  Fault injection acts on the fused
-    // launch's publications.
+    // With few feature groups and a long time axis, most tiles of a fused
+    // launch would wait for their predecessor: take the two passes instead.
+    // Fault injection acts on the fused launch's publications.
     const bool two_pass = cfg.carry_mode == SLSTM_CARRY_TWO_PASS ||
-                          (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 && 4 * l.n_groups <= sms &&
-                           l.n_chunks >= 256);
+                          (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 &&
+                           prefer_two_pass(l.n_groups, (long long)l.n_chunks * TT, sms));
     if (cfg.forget == SLSTM_FORGET_EXP)
         return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st)
                    : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st);

@@ -214,6 +214,7 @@ def test_newton_bounded_wait_reports_timeout(cuda_device):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 @pytest.mark.parametrize("B,T,d_in,d,dtype", [(2, 64, 8, 8, "f32"), (2, 75, 12, 40, "f32"), (2, 33, 8, 10, "f32"),
+                                              (1, 16400, 16, 36, "bf16"),
                                               (2, 75, 16, 40, "bf16"), (3, 130, 64, 96, "bf16"),
                                               (2, 96, 16, 40, "bf16"), (2, 100, 24, 36, "bf16"),
                                               (2, 70, 16, 18, "bf16")])

@@ -169,3 +169,27 @@ def test_varlen_nan_in_one_sequence_reports_divergence(carry_mode, cuda_device):
     assert s["diverged"] and s["error"] == 3, s
     # the later sequences are untouched by it
     assert torch.isfinite(S[2:]).all()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_varlen_backward_two_pass_matches_oracle(dtype, cuda_device):
+    """Few feature groups and a long packed axis: the adjoint takes the two
+    passes (tile aggregates, blocked scan, then the fused pass with known
+    carries) instead of the look-back."""
+    lengths = [5000, 0, 3000, 7000, 1700]
+    d = 40
+    c = _case(lengths, d, 16, dtype, "sigmoid", 47)
+    P, Pref = _preact(c)
+    cu = c["cu"].numpy()
+    Sref = oracle.sequential_varlen(Pref, as_f64(c["R"]), as_f64(c["s0"]), cu, "sigmoid")
+    S = torch.from_numpy(Sref).float().cuda()
+    out = api.newton_backward_varlen(_dev(c["x"]), _dev(c["Wx"]), P, _dev(c["R"]), _dev(c["s0"]), _dev(c["cu"]),
+                                     S, _dev(c["dH"]), forget="sigmoid")
+    torch.cuda.synchronize()
+    ref = oracle.backward_varlen(as_f64(c["x"]), as_f64(c["Wx"]), Pref, as_f64(c["R"]), as_f64(c["s0"]), Sref,
+                                 as_f64(c["dH"]), cu, "sigmoid")
+    for k in ("dx", "dWx", "dR", "db", "ds0"):
+        got = as_f64(out[k].cpu())
+        err = np.abs(got - ref[k]).max() / (1 + np.abs(ref[k]).max())
+        assert err <= 1e-4, (k, err)
+    assert not out["ds0"][1].any()
