@@ -503,7 +503,7 @@ def run_varlen(args, w):
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
 # this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
 # (every tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "581550f131f13aee150e36474ed5fceacd6944dbfc3580ea77c4c0572558163b", "first": 30.01, "middle": 46.36, "last": 46.34}
+NEWTON_TRAFFIC = {"sources_sha256": "433c5e1cd5aa899d3ac0dcf696ed7dbfc118ef343a36b2a5ba34a515f1d1785f", "first": 30.11, "middle": 46.40, "last": 46.46}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
