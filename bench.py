@@ -498,6 +498,63 @@ def run_varlen(args, w):
     return 0
 
 
+def run_decode(args, w):
+    """Decode: the workload's B rows, d_in and d_h stepped one token at a time with the fused decode
+    kernel (input projection + cell update); a step is 128 tokens replayed from one CUDA graph.
+    The roofline counts the bytes a token must read: all of W_x, x and the state, and the new state
+    written; W_x (8.4 MB at d_in = d_h = 1024, bf16) stays in L2 between tokens, so the achieved rate
+    can exceed the HBM copy bandwidth."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import api
+    _, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    T_dec = 128
+    inp = make_inputs(w, with_dH=False)
+    xs = inp["x"][:, :T_dec].transpose(0, 1).contiguous().to(dev)   # (T_dec, B, d_in)
+    Wx, R, bias = inp["Wx"].to(dev), inp["R"].to(dev), inp["bias"].to(dev)
+    s0 = inp["s0"].to(dev)
+    S = torch.empty(T_dec, w.B, 4, w.d_h, device=dev)
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(stream):
+        api.decode(xs, Wx, bias, R, s0, forget=w.forget, S=S)
+    torch.cuda.current_stream().wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        api.decode(xs, Wx, bias, R, s0, forget=w.forget, S=S)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    us_token = ms * 1e3 / T_dec
+    esz = 2 if w.dtype == "bf16" else 4
+    nbytes = 4 * w.d_h * w.d_in * esz + w.B * w.d_in * esz + 2 * w.B * 4 * w.d_h * 4
+    gbs = nbytes / (us_token / 1e6) / 1e9
+    hbm, peak_kind = _peaks()
+    launches = T_dec * ((w.B + 15) // 16)
+    line = {"metric": "sLSTM decode tokens/s (B rows x steps / s)", "value": w.B * T_dec / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "operand_dtype": f"{w.dtype} x/W_x, fp32 state", "data": "synthetic",
+            "config": {"workload": f"{w.name}_decode", "B": w.B, "d_in": w.d_in, "d_h": w.d_h,
+                       "x_dtype": w.dtype, "forget": w.forget, "tokens_per_step": T_dec,
+                       "us_per_token": us_token, "cuda_graph": True,
+                       "l2": "W_x stays in L2 between tokens (decode reuses it every token)"},
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": gbs, "peak": hbm,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm, "traffic": None,
+                         "bytes_per_token": nbytes},
+            "gpu_launches": launches * args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
 # last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
@@ -536,7 +593,7 @@ def main(argv=None):
     ap.add_argument("--cpu-lanes", type=int, default=40)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen"],
+    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen", "decode"],
                     help="train: GEMM + Newton + backward (default); forward: GEMM + Newton; "
                          "scan: scan_block4 alone over T in --scan-T at B=4, d=2048; "
                          "varlen: the workload repacked into ragged sequences (cu_seqlens)")
@@ -563,6 +620,8 @@ def main(argv=None):
         return run_scan(args)
     if args.mode == "varlen":
         return run_varlen(args, w)
+    if args.mode == "decode":
+        return run_decode(args, w)
     return run_gpu(args, w)
 
 

@@ -248,6 +248,27 @@ int slstm_sequential_step(const float *P, const float *R, const float *s0, float
                           int T_steps, int d_h, int forget, slstm_stream_t stream);
 
 /*
+ * One decode step for B batch rows ("sLSTM in this library", "API notes": at
+ * T = 1 evaluation is one recurrent step; "pararnn-torch structure": the T = 1
+ * step is replayed under CUDA graphs): the input projection fused with the
+ * cell update,
+ *   P[b, g, j]     = sum_k Wx[g d_h + j, k] x[b, k] + bias[g, j]
+ *   s_next[b, :, j] = f(s_prev[b, :, j], P[b, :, j])      (f as in slstm_newton_forward)
+ * x: (B, d_in), Wx: (4 d_h, d_in), both of `dtype` (SLSTM_F32 or SLSTM_BF16),
+ * d_in a multiple of 4 (f32) or 8 (bf16).  bias, R: (4, d_h) fp32.  s_prev:
+ * (B, 4, d_h) fp32 or NULL (zero state); s_next: (B, 4, d_h) fp32, which may
+ * be s_prev itself (in-place step) but must not overlap it otherwise.  All
+ * pointers device memory owned by the caller, 16-byte aligned.  W_x is read
+ * once per 16 batch rows; accumulation in fp32.  One launch per 16 rows, no
+ * workspace, no synchronisation, so a sequence of steps can be captured in a
+ * CUDA graph.  Returns SLSTM_ERR_INVALID_ARG for bad sizes, dtype, forget mode
+ * or alignment (before touching the GPU), SLSTM_ERR_CUDA for a launch error.
+ */
+int slstm_decode_step(const void *x, const void *Wx, int dtype, const float *bias, const float *R,
+                      const float *s_prev, float *s_next, int forget, int B, int d_in, int d_h,
+                      slstm_stream_t stream);
+
+/*
  * Gradients of L = sum_{b,t,j} dH[b,t,j] * h[b,t,j] at the solution S
  * ("sLSTM in this library", "Backward": one reverse associative scan of J^T,
  * then the packed cell VJP):

@@ -61,6 +61,7 @@ SIGNATURES = {
                                          _V]),
     "slstm_newton_backward_varlen": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I,
                                           _I, _V, _Z, _V]),
+    "slstm_decode_step": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _I, _I, _I, _V]),
 }
 
 _lib = None

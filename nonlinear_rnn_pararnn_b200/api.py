@@ -146,6 +146,45 @@ def sequential_step(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *
     return S
 
 
+def decode_step(x: torch.Tensor, Wx: torch.Tensor, bias: torch.Tensor, R: torch.Tensor, s_prev: torch.Tensor = None,
+                *, forget="sigmoid", out: torch.Tensor = None) -> torch.Tensor:
+    """One decode step: x (B, d_in) and Wx (4 d_h, d_in) of one dtype, bias and R (4, d_h), s_prev
+    (B, 4, d_h) or None (zero state); returns s_next (B, 4, d_h), written into `out` when given
+    (`out` may be `s_prev`)."""
+    B, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    dt = x.dtype
+    _need(x, "x", (B, d_in), dt)
+    _need(Wx, "Wx", (4 * d_h, d_in), dt)
+    _need(bias, "bias", (4, d_h))
+    _need(R, "R", (4, d_h))
+    if s_prev is not None:
+        _need(s_prev, "s_prev", (B, 4, d_h))
+    if out is None:
+        out = torch.empty(B, 4, d_h, device=x.device, dtype=torch.float32)
+    _need(out, "out", (B, 4, d_h))
+    check("slstm_decode_step", load().slstm_decode_step(_ptr(x), _ptr(Wx), _DTYPE[dt], _ptr(bias), _ptr(R),
+                                                        _ptr(s_prev), _ptr(out), forget_code(forget), B, d_in, d_h,
+                                                        _stream()))
+    return out
+
+
+def decode(xs: torch.Tensor, Wx: torch.Tensor, bias: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
+           forget="sigmoid", S: torch.Tensor = None) -> torch.Tensor:
+    """T decode steps over xs (T, B, d_in) from s0 (B, 4, d_h) or zero; returns S (T, B, 4, d_h), the
+    state after every step.  One launch per step on the current stream (capturable in a CUDA graph)."""
+    T, B, d_in = xs.shape
+    d_h = Wx.shape[0] // 4
+    if S is None:
+        S = torch.empty(T, B, 4, d_h, device=xs.device, dtype=torch.float32)
+    _need(S, "S", (T, B, 4, d_h))
+    prev = s0
+    for t in range(T):
+        decode_step(xs[t], Wx, bias, R, prev, forget=forget, out=S[t])
+        prev = S[t]
+    return S
+
+
 def newton_backward(x, Wx, P, R, s0, S, dH, *, forget="sigmoid", out: dict = None, ws: torch.Tensor = None):
     """Gradients of sum(dH * h); returns dict dx, dWx, dR, db, ds0."""
     B, T, d_in = x.shape

@@ -56,6 +56,8 @@ size_t scan_workspace_bytes(int B, int T, int d);
 cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, float *y, int B,
                                int T, int d, bool reverse, void *ws, cudaStream_t st);
 
+cudaError_t decode_launch(const void *x, const void *Wx, int dtype, const float *bias, const float *R,
+                          const float *s_prev, float *s_next, int forget, int B, int d_in, int d, cudaStream_t st);
 cudaError_t sequential_launch(const float *P, const float *R, const float *s0, float *S, int B,
                               int T, int d, int forget, cudaStream_t st);
 

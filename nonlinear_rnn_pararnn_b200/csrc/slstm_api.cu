@@ -134,6 +134,21 @@ int slstm_sequential_step(const float *P, const float *R, const float *s0, float
                                          static_cast<cudaStream_t>(stream)));
 }
 
+int slstm_decode_step(const void *x, const void *Wx, int dtype, const float *bias, const float *R,
+                      const float *s_prev, float *s_next, int forget, int B, int d_in, int d_h,
+                      slstm_stream_t stream)
+{
+    if (dtype != SLSTM_F32 && dtype != SLSTM_BF16) return SLSTM_ERR_INVALID_ARG;
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, 1, d_in, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (d_in % (dtype == SLSTM_BF16 ? 8 : 4) != 0) return SLSTM_ERR_INVALID_ARG;   // 16-byte rows
+    if (!aligned16(x) || !aligned16(Wx) || !aligned16(bias) || !aligned16(R) || !aligned16_or_null(s_prev) ||
+        !aligned16(s_next))
+        return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(decode_launch(x, Wx, dtype, bias, R, s_prev, s_next, forget, B, d_in, d_h,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 int slstm_newton_backward(const void *x, const void *Wx, int dtype, const float *P, const float *R,
                           const float *s0, const float *S, const float *dH, float *dx, float *dWx,
                           float *dR, float *db, float *ds0, int forget, int B, int T, int d_in,

@@ -112,6 +112,14 @@ def test_other_entry_points_reject_bad_arguments():
     args = [FAKE] * 13
     assert lib.slstm_newton_backward(args[0], args[1], 0, *args[2:12], 0, 2, 0, 8, 8, FAKE, big, NULL) == E
     assert lib.slstm_newton_backward(args[0], args[1], 5, *args[2:12], 0, 2, 8, 8, 8, FAKE, big, NULL) == E
+    # decode: dtype, forget mode, sizes, 16-byte rows, alignment
+    assert lib.slstm_decode_step(FAKE, FAKE, 7, FAKE, FAKE, NULL, FAKE, 0, 2, 8, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE, FAKE, 0, FAKE, FAKE, NULL, FAKE, 3, 2, 8, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE, FAKE, 0, FAKE, FAKE, NULL, FAKE, 0, 0, 8, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE, FAKE, _lib.SLSTM_BF16, FAKE, FAKE, NULL, FAKE, 0, 2, 12, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE, FAKE, 0, FAKE, FAKE, NULL, FAKE, 0, 2, 6, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE_MIS, FAKE, 0, FAKE, FAKE, NULL, FAKE, 0, 2, 8, 8, NULL) == E
+    assert lib.slstm_decode_step(FAKE, FAKE, 0, FAKE, FAKE, FAKE_MIS, FAKE, 0, 2, 8, 8, NULL) == E
 
 
 def test_varlen_entry_points_reject_bad_arguments():
