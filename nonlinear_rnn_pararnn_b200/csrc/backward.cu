@@ -455,17 +455,21 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 // rows (part, gate, feature) of the transposed pair, 32 steps each;
                 // nothing before t = 0 (those addresses hold the previous batch row)
                 if (a.dpt_vec8) {
-                    // 8-byte pieces of 4 steps: piece q of row r is index 8 r + q
+                    // 8-byte pieces of 4 steps: thread (feature jl, piece q) copies
+                    // piece q of the 8 rows (part, gate) of feature jl
+                    static_assert(NW * 32 == 256, "one thread per (feature, piece)");
+                    const int q = threadIdx.x & 7, jl = threadIdx.x >> 3;
+                    const int t = t_lo + 4 * q;
+                    if (t >= 0 && ti.j0 + jl < a.d) {
+                        const size_t base = (size_t)(ti.j0 + jl) * a.ldT + row0 + t;
+                        const size_t gstride = d * (size_t)a.ldT;
     #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int idx = threadIdx.x + NW * 32 * k;
-                        const int r = idx >> 3, q = idx & 7;
-                        const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
-                        const int t = t_lo + 4 * q;
-                        if (t >= 0 && ti.j0 + jl < a.d) {
-                            const uint2 v = *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
-                            __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
-                            *reinterpret_cast<uint2 *>(dst + ((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t) = v;
+                        for (int part = 0; part < 2; ++part) {
+                            __nv_bfloat16 *dst = (part ? a.dpt_lo : a.dpt_hi) + base;
+    #pragma unroll
+                            for (int gi = 0; gi < 4; ++gi)
+                                *reinterpret_cast<uint2 *>(dst + gi * gstride) =
+                                    *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
                         }
                     }
                 } else {
