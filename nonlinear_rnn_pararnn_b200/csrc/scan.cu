@@ -151,16 +151,19 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
         const size_t row0 = (size_t)bb * T;
 
         // ---- walk A ----
+        // the thread's maps stay in registers for walk B (one CTA per SM
+        // leaves the whole register file to its 256 threads); steps past T
+        // (only in a group's last tile) are skipped
+        Aff mp[L];
         Aff agg;
-        aff_identity(agg);
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int q = warp * L + i;
-            if (chunk * TT + q < T) {
-                Aff m;
-                load_map<REVERSE>(sm, st, q, lane, m);
-                aff_compose(m, agg, agg);
-            }
+            const bool valid = chunk * TT + q < T;
+            if (valid) load_map<REVERSE>(sm, st, q, lane, mp[i]);
+            else aff_identity(mp[i]);
+            if (i == 0) agg = mp[0];
+            else if (valid) aff_compose(mp[i], agg, agg);
         }
         store_aff_smem(sm.agg, warp, lane, agg);
         __syncthreads();
@@ -183,9 +186,7 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
             const int q = warp * L + i;
             if (chunk * TT + q < T) {
                 const int t = step_time<REVERSE>(T, chunk, q);
-                Aff m;
-                load_map<REVERSE>(sm, st, q, lane, m);
-                aff_apply(m, v, v);
+                aff_apply(mp[i], v, v);
                 float *py = a.y + (row0 + t) * 4 * d + jj;
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
