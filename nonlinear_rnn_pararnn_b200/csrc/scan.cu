@@ -10,9 +10,11 @@
 // bytes per element) in shared memory with cp.async while they scan the
 // current one:
 //   walk A   each thread folds its 4 maps (dense 4x4 compositions, fp32);
-//   carry    warp 0 takes the carry entering the tile from the tile before
-//            it (decoupled look-back, lookback.cuh) and hands each warp its
-//            carry;
+//   carry    the last four warps take the carry entering the tile from the
+//            tile before it (its published prefix, read during walk A; the
+//            decoupled look-back of lookback.cuh when it is missing) and walk
+//            it through the warp maps, one (feature, slot) pair per lane,
+//            releasing each other warp as soon as its carry is stored;
 //   walk B   each thread applies its maps from its carry and writes y.
 #include "launchers.h"
 #include "lookback.cuh"
@@ -23,6 +25,8 @@ namespace {
 constexpr int NW = 8;
 constexpr int L = 4;
 constexpr int TT = NW * L;
+constexpr int CHAIN0 = NW - 4;          // first chain warp
+constexpr int CHAIN_BAR = CHAIN0 + 1;   // the chain warps' own barrier (ids 1 .. CHAIN0: per warp)
 
 struct ScanArgs {
     const float *A;
@@ -38,8 +42,7 @@ struct ScanArgs {
 struct ScanSmem {
     float A[2][TT][16][32];   // [stage][step in processing order][row*4+col][feature]
     float b[2][TT][4][32];
-    float agg[NW][20][32];
-    float cin[NW][4][32];
+    TileMaps<NW> maps;
     unsigned tick[2];
 };
 
@@ -149,6 +152,14 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
         const bool jv = j < a.d;
         const size_t jj = jv ? (size_t)j : 0;
         const size_t row0 = (size_t)bb * T;
+        const bool chain_warp = warp >= CHAIN0;
+
+        // the predecessor's inclusive prefix (chain lanes), looked at before
+        // and halfway through walk A
+        const bool look = chain_warp && chunk > 0;
+        const unsigned long long *predw = a.ca.incw + chain_word(ticket - (unsigned)G, warp, lane);
+        unsigned long long w1 = 0ull, w2 = 0ull;
+        if (look) w1 = ld_relaxed_u64(predw);
 
         // ---- walk A ----
         // the thread's maps stay in registers for walk B (one CTA per SM
@@ -164,23 +175,46 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
             else aff_identity(mp[i]);
             if (i == 0) agg = mp[0];
             else if (valid) aff_compose(mp[i], agg, agg);
+            if (i == L / 2 && look) w2 = ld_relaxed_u64(predw);
         }
-        store_aff_smem(sm.agg, warp, lane, agg);
-        __syncthreads();
-        if (warp == 0) {
-            float first[4] = {0.f, 0.f, 0.f, 0.f};
-            if (a.y0 && jv) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) first[e] = __ldg(a.y0 + ((size_t)bb * 4 + e) * d + jj);
+        maps_store(sm.maps.m, warp, lane, agg);
+
+        // ---- carry ----
+        float c = 0.f;
+        bool ok = true;
+        if (chain_warp && chunk == 0 && a.y0) {
+            // chunk 0: y0 enters (chain lane (row, feature))
+            const int jf = (grp - bb * a.groups_per_row) * 32 + chain_feature(warp, lane);
+            if (jf < a.d) c = __ldg(a.y0 + ((size_t)bb * 4 + chain_row(lane)) * d + jf);
+        }
+        if (look) {
+            if ((unsigned)(w1 >> 32) == a.ca.epoch) {
+                c = __uint_as_float((unsigned)w1);
+            } else {
+                ok = (unsigned)(w2 >> 32) == a.ca.epoch;
+                c = __uint_as_float((unsigned)w2);
             }
-            tile_carry_serial<NW>(a.ca, sm.agg, sm.cin, ticket, chunk, grp, first, false);
         }
-        __syncthreads();
+        const bool fast = __syncthreads_and(ok);
+        if (chain_warp) {
+            if (fast) {
+                c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, 0u, CHAIN0);
+                st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+                named_bar_sync(CHAIN_BAR, 4 * 32);
+            } else {
+                if (warp == CHAIN0) tile_carry_fallback<NW>(a.ca, sm.maps.m, sm.maps.cin, ticket, chunk, grp, false);
+                named_bar_sync(CHAIN_BAR, 4 * 32);
+#pragma unroll 1
+                for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
+            }
+        } else {
+            named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
+        }
 
         // ---- walk B ----
         float v[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = sm.cin[warp][e][lane];
+        for (int e = 0; e < 4; ++e) v[e] = sm.maps.cin[warp][e][sw(e, lane)];
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int q = warp * L + i;
