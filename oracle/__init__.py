@@ -301,3 +301,59 @@ def backward_varlen(x, Wx, P, R, s0, S, dH, cu, forget="sigmoid"):
         for key in ("dWx", "dR", "db"):
             out[key] += g[key]
     return out
+
+
+# ----------------------------------------------------------------------------
+# the trunk layer ("sLSTM in this library", section "Stacking":
+# RMSNorm -> ParaRNN(ParaSLSTM) -> residual -> RMSNorm -> SwiGLU -> residual).
+# Readings where the section is silent: RMSNorm(v) = v / sqrt(mean(v^2) + eps)
+# * w over the model axis; SwiGLU(z) = W_down (silu(W_gate z) * (W_up z)) with
+# no biases; the cell has d_in = d_h = d_model and starts from the zero state.
+# Its GEMM operands are bf16 (the library's compute type): with
+# ``bf16_operands`` the normalised activations and the SwiGLU product are
+# rounded to bf16 (nearest, ties to even) where they enter a GEMM.
+# ----------------------------------------------------------------------------
+def round_bf16(a) -> np.ndarray:
+    """Nearest bf16 value of each fp64 entry (ties to even), as fp64."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(_f64(a))).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def rmsnorm(v, w, eps=1e-6) -> np.ndarray:
+    v = _f64(v)
+    return v / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps) * _f64(w)
+
+
+def silu(a) -> np.ndarray:
+    a = _f64(a)
+    return a / (1.0 + np.exp(-a))
+
+
+def swiglu(z, W_gate, W_up, W_down, bf16_operands=False) -> np.ndarray:
+    """z (M, D), W_gate / W_up (F, D), W_down (D, F) -> (M, D)."""
+    z = _f64(z)
+    g = gemm(z, W_gate, tb=True)
+    u = gemm(z, W_up, tb=True)
+    a = silu(g) * u
+    if bf16_operands:
+        a = round_bf16(a)
+    return gemm(a, W_down, tb=True)
+
+
+def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gate, W_up, W_down, forget="sigmoid", eps=1e-6,
+                  bf16_operands=False):
+    """x (B, T, D) -> (y (B, T, D), S (B, T, 4, D)), the cell solved exactly
+    (sequentially) from the zero state."""
+    x = _f64(x)
+    B, T, D = x.shape
+    z1 = rmsnorm(x, norm1_w, eps)
+    if bf16_operands:
+        z1 = round_bf16(z1)
+    P = preact(z1, Wx, bias)
+    S = sequential_btgd(P, R, np.zeros((B, 4, D)), forget)
+    u = x + S[:, :, 3, :]
+    z2 = rmsnorm(u, norm2_w, eps)
+    if bf16_operands:
+        z2 = round_bf16(z2)
+    y = u + swiglu(z2.reshape(B * T, D), W_gate, W_up, W_down, bf16_operands).reshape(B, T, D)
+    return y, S

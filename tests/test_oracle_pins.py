@@ -383,3 +383,84 @@ def test_varlen_empty_sequences_and_independence():
     g2 = oracle.backward_varlen(xp, Wx, Pp, R, s0[[0, 2, 3]], S, dHp, cu2)
     np.testing.assert_array_equal(g2["dx"], g["dx"])
     np.testing.assert_array_equal(g2["ds0"], g["ds0"][[0, 2, 3]])
+
+
+# ---------------------------------------------------------------------------
+# the trunk layer: RMSNorm, SwiGLU, the block's wiring, bf16 rounding
+# ---------------------------------------------------------------------------
+def test_round_bf16_known_values():
+    # bf16: 8 significant bits, so the spacing just above 1 is 2^-7
+    v = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 3 * 2.0 ** -9, -2.0 ** -130, 0.1, 3.0e38])
+    got = oracle.round_bf16(v)
+    assert got[0] == 1.0                       # tie between 1 and 1 + 2^-7: to the even one
+    assert got[1] == 1 + 2.0 ** -6             # tie between 1 + 2^-7 and 1 + 2^-6: to the even one
+    assert got[2] == 1 + 2.0 ** -7             # nearest, no tie
+    assert got[3] == -2.0 ** -130              # subnormals are kept
+    assert got[4] == 0.10009765625             # bf16 0x3DCD
+    assert abs(got[5] - 3.0e38) / 3.0e38 < 2.0 ** -8
+
+
+def test_rmsnorm_closed_forms():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((5, 37)) * 3
+    eps = 1e-6
+    y = oracle.rmsnorm(v, np.ones(37), eps)
+    ms = np.mean(v * v, axis=-1)
+    # mean of squares after the norm is ms / (ms + eps)
+    np.testing.assert_allclose(np.mean(y * y, axis=-1), ms / (ms + eps), rtol=1e-13)
+    # positive scaling of a row leaves the output (eps = 0) unchanged, w scales columns
+    w = rng.standard_normal(37)
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * v, w, 0.0), oracle.rmsnorm(v, w, 0.0), rtol=1e-13)
+    np.testing.assert_allclose(oracle.rmsnorm(v, w, 0.0), oracle.rmsnorm(v, np.ones(37), 0.0) * w, rtol=1e-13)
+    # one feature: v / |v| * w
+    np.testing.assert_allclose(oracle.rmsnorm(np.array([[-2.5]]), np.array([0.5]), 0.0), [[-0.5]], rtol=1e-15)
+
+
+def test_silu_and_swiglu_known_values():
+    # logistic(1) = 1 / (1 + e^-1) = 0.7310585786300049
+    np.testing.assert_allclose(oracle.silu(np.array([0.0, 1.0, -1.0, 40.0])),
+                               [0.0, 0.7310585786300049, -0.2689414213699951, 40.0], rtol=1e-15)
+    # identity projections: SwiGLU(z) = silu(z) * z elementwise
+    z = np.array([[1.0, -1.0, 2.0]])
+    I3 = np.eye(3)
+    np.testing.assert_allclose(oracle.swiglu(z, I3, I3, I3), [[0.7310585786300049, 0.2689414213699951,
+                                                               2.0 * 2.0 / (1 + math.exp(-2.0))]], rtol=1e-15)
+    # F = 2 hidden units, D = 1: W_down mixes them, the gate and the up projection
+    # are separate rows (a swapped gate/up would give another value)
+    z = np.array([[2.0]])
+    Wg, Wu, Wd = np.array([[1.0], [0.0]]), np.array([[3.0], [1.0]]), np.array([[1.0, 10.0]])
+    want = (2.0 / (1 + math.exp(-2.0))) * 6.0 + 0.0
+    np.testing.assert_allclose(oracle.swiglu(z, Wg, Wu, Wd), [[want]], rtol=1e-15)
+
+
+def test_block_wiring():
+    rng = np.random.default_rng(4)
+    B, T, D, F = 2, 9, 6, 12
+    x = rng.standard_normal((B, T, D))
+    w1, w2 = rng.uniform(0.5, 1.5, D), rng.uniform(0.5, 1.5, D)
+    Wx = rng.standard_normal((4 * D, D)) / np.sqrt(D)
+    bias = np.zeros((4, D))
+    bias[2] = 3.0
+    R = rng.uniform(-0.5, 0.5, (4, D))
+    Wg, Wu, Wd = rng.standard_normal((F, D)), rng.standard_normal((F, D)), rng.standard_normal((D, F)) / F
+    y, S = oracle.block_forward(x, w1, Wx, bias, R, w2, Wg, Wu, Wd)
+    # the cell sees the normalised input and starts from zero
+    P = oracle.preact(oracle.rmsnorm(x, w1), Wx, bias)
+    np.testing.assert_allclose(S, oracle.sequential_btgd(P, R, np.zeros((B, 4, D))), rtol=0, atol=0)
+    # W_down = 0: the block is x + h
+    y0, _ = oracle.block_forward(x, w1, Wx, bias, R, w2, Wg, Wu, 0 * Wd)
+    np.testing.assert_allclose(y0, x + S[:, :, 3, :], rtol=0, atol=0)
+    # the FFN part is a function of the residual u = x + h alone: moving an
+    # amount into x and the opposite into nothing else changes y by that amount
+    # only through u (check: y - u equals SwiGLU(RMSNorm(u)))
+    u = x + S[:, :, 3, :]
+    ffn = oracle.swiglu(oracle.rmsnorm(u, w2).reshape(-1, D), Wg, Wu, Wd).reshape(B, T, D)
+    np.testing.assert_allclose(y - u, ffn, rtol=1e-12, atol=1e-12)
+    # a causal layer: changing x at step t leaves the outputs before t alone
+    x2 = x.copy()
+    x2[:, 5] += 1.0
+    y2, _ = oracle.block_forward(x2, w1, Wx, bias, R, w2, Wg, Wu, Wd)
+    assert np.array_equal(y2[:, :5], y[:, :5]) and np.abs(y2[:, 5:] - y[:, 5:]).max() > 1e-3
+    # bf16 operands move the result by about the bf16 step, no more
+    yb, _ = oracle.block_forward(x, w1, Wx, bias, R, w2, Wg, Wu, Wd, bf16_operands=True)
+    assert 0 < np.abs(yb - y).max() < 2e-2
