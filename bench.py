@@ -555,6 +555,84 @@ def run_decode(args, w):
     return 0
 
 
+def run_block(args, w):
+    """The trunk layer's forward (RMSNorm -> cell -> residual -> RMSNorm -> SwiGLU -> residual) at the
+    workload's B and T with d_model = d_h and d_ff = 4 d_model: one slstm_block_forward call per step
+    (7 launches + the Newton iterations), fixed K Newton iterations.  There is no single dominant
+    kernel, so the roofline line compares the step with its floor: the three GEMMs' flops at the
+    sustained bf16 tensor peak plus the Newton and norm kernels' algorithmic bytes at the HBM copy
+    bandwidth; frac = floor / measured step time."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import api
+    _, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    K = args.newton_iters
+    B, T, D = w.B, w.T, w.d_h
+    F = 4 * D
+    g = torch.Generator().manual_seed(w.seed)
+    x = torch.randn(B, T, D, generator=g).to(dev)
+    w1 = (torch.rand(D, generator=g) + 0.5).to(dev)
+    w2 = (torch.rand(D, generator=g) + 0.5).to(dev)
+    Wx = (torch.randn(4 * D, D, generator=g) * D ** -0.5).to(torch.bfloat16).to(dev)
+    bias = torch.zeros(4, D)
+    bias[2] = torch.linspace(3.0, 6.0, D)
+    bias = bias.to(dev)
+    R = ((torch.rand(4, D, generator=g) * 2 - 1) * w.r_scale).to(dev)
+    W_gu = (torch.randn(2 * F, D, generator=g) * D ** -0.5).to(torch.bfloat16).to(dev)
+    W_down = (torch.randn(D, F, generator=g) * F ** -0.5).to(torch.bfloat16).to(dev)
+    y = torch.empty_like(x)
+    S = torch.empty(B, T, 4, D, device=dev)
+    stats = api.new_stats(dev)
+    wsb = api.block_workspace(B, T, D, F, dev)
+
+    def step():
+        api.block_forward(x, w1, Wx, bias, R, w2, W_gu, W_down, forget=w.forget, max_iters=K, fixed=True,
+                          y=y, S=S, stats=stats, ws=wsb)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    time.sleep(0.25)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    st = api.read_stats(stats)
+    M = B * T
+    flops = 2.0 * M * D * (4 * D + 2 * F + F)
+    nbytes = M * D * (32 + 48 * (K - 1)) + M * D * (4 + 2) + M * D * (4 + 16 + 4 + 2)
+    hbm, peak_kind = _peaks()
+    try:
+        with open(PEAKS_PATH) as f:
+            tflops = float(json.load(f)["bf16_tflops_sustained"])
+        tkind = "measured"
+    except Exception:
+        tflops, tkind = 1400.0, "fallback"
+    floor_ms = flops / (tflops * 1e12) * 1e3 + nbytes / (hbm * 1e9) * 1e3
+    line = {"metric": "trunk-layer forward tokens/s (B*T / s)", "value": M / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "operand_dtype": "bf16 GEMM operands, fp32 accumulation, state and residual stream", "data": "synthetic",
+            "config": {"workload": f"{w.name}_block", "B": B, "T": T, "d_model": D, "d_ff": F, "forget": w.forget,
+                       "newton_iters": K, "newton_mode": "fixed", "error": st["error"],
+                       "l2": "inputs larger than L2"},
+            "roofline": {"kernel": "whole layer (3 GEMMs + Newton + norms)", "bound": "tensor+hbm",
+                         "achieved": floor_ms, "peak": ms, "unit": "ms (floor vs measured)",
+                         "frac": floor_ms / ms, "traffic": None, "gemm_tflop_per_step": flops / 1e12,
+                         "tensor_peak_tflops": tflops, "tensor_peak_kind": tkind, "hbm_gbs": hbm,
+                         "hbm_peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes},
+            "clocks": clocks,
+            "gpu_launches": (5 + K) * args.steps}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 # DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
 # last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
 # (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
@@ -593,10 +671,11 @@ def main(argv=None):
     ap.add_argument("--cpu-lanes", type=int, default=40)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen", "decode"],
+    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen", "decode", "block"],
                     help="train: GEMM + Newton + backward (default); forward: GEMM + Newton; "
                          "scan: scan_block4 alone over T in --scan-T at B=4, d=2048; "
-                         "varlen: the workload repacked into ragged sequences (cu_seqlens)")
+                         "varlen: the workload repacked into ragged sequences (cu_seqlens); "
+                         "decode: T = 1 steps under a CUDA graph; block: the trunk layer's forward")
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
@@ -622,6 +701,8 @@ def main(argv=None):
         return run_varlen(args, w)
     if args.mode == "decode":
         return run_decode(args, w)
+    if args.mode == "block":
+        return run_block(args, w)
     return run_gpu(args, w)
 
 

@@ -318,6 +318,37 @@ int slstm_newton_backward_varlen(const void *x, const void *Wx, int dtype, const
                                  int forget, int total_T, int d_in, int d_h, void *ws, size_t ws_bytes,
                                  slstm_stream_t stream);
 
+/*
+ * The trunk layer, forward ("sLSTM in this library", section "Stacking":
+ * RMSNorm -> ParaRNN(ParaSLSTM) -> residual -> RMSNorm -> SwiGLU -> residual):
+ *   z1 = RMSNorm(x) * norm1_w,  P = z1 Wx^T + bias,  S = the cell's solution
+ *        on P from the zero state (Newton, as slstm_newton_forward with cfg)
+ *   u  = x + h  (h = slot 3 of S),  z2 = RMSNorm(u) * norm2_w
+ *   y  = u + W_down (silu(W_gate z2) * (W_up z2))
+ * with RMSNorm(v) = v / sqrt(mean over the d_model axis of v^2 + eps).
+ *   x, y     (B, T, d_model) fp32; y may be x (in place), must not overlap S
+ *   norm1_w, norm2_w  (d_model) fp32;  bias, R (4, d_model) fp32
+ *   Wx       (4 d_model, d_model) bf16, gate-major rows g d_model + j
+ *   W_gu     (2 d_ff, d_model) bf16: W_gate and W_up interleaved in blocks
+ *            of 32 rows (rows 64 k .. 64 k + 31 = W_gate rows 32 k .. 32 k + 31,
+ *            rows 64 k + 32 .. 64 k + 63 = W_up rows 32 k .. 32 k + 31)
+ *   W_down   (d_model, d_ff) bf16
+ *   S        (B, T, 4, d_model) fp32, the cell's states (kept for a backward pass)
+ * d_model a multiple of 8, d_ff a multiple of 32.  The GEMM operands z1, z2
+ * and the SwiGLU product are rounded to bf16; accumulation and everything
+ * else in fp32.  The SwiGLU product and the residual are formed in the GEMM
+ * epilogues.  Workspace: slstm_block_workspace_size(B, T, d_model, d_ff) bytes,
+ * 256-byte aligned.  Stats and errors as slstm_newton_forward (argument errors
+ * before touching the GPU); a bounded wait that expires inside a GEMM sets
+ * the first 4-byte word of the workspace nonzero.
+ */
+size_t slstm_block_workspace_size(int B, int T, int d_model, int d_ff);
+
+int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, const float *bias, const float *R,
+                        const float *norm2_w, const void *W_gu, const void *W_down, float *y, float *S,
+                        const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T, int d_model,
+                        int d_ff, float eps, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -62,6 +62,9 @@ SIGNATURES = {
     "slstm_newton_backward_varlen": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I,
                                           _I, _V, _Z, _V]),
     "slstm_decode_step": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _I, _I, _I, _V]),
+    "slstm_block_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "slstm_block_forward": (_I, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V,
+                                 _I, _I, _I, _I, ctypes.c_float, _V, _Z, _V]),
 }
 
 _lib = None

@@ -277,3 +277,55 @@ def newton_backward_varlen(x, Wx, P, R, s0, cu_seqlens, S, dH, *, forget="sigmoi
         _ptr(out["dx"]), _ptr(out["dWx"]), _ptr(out["dR"]), _ptr(out["db"]), _ptr(out.get("ds0")),
         forget_code(forget), total_T, d_in, d_h, _ptr(ws), ws.numel(), _stream()))
     return out
+
+
+# ---------------------------------------------------------------------------
+# the trunk layer (RMSNorm -> cell -> residual -> RMSNorm -> SwiGLU -> residual)
+# ---------------------------------------------------------------------------
+def interleave_gate_up(W_gate: torch.Tensor, W_up: torch.Tensor) -> torch.Tensor:
+    """(d_ff, d_model) W_gate and W_up -> the (2 d_ff, d_model) W_gu of
+    block_forward: blocks of 32 gate rows followed by the 32 up rows of the
+    same hidden features.  A one-time weight layout change (d_ff % 32 == 0)."""
+    F, D = W_gate.shape
+    if tuple(W_up.shape) != (F, D) or F % 32:
+        raise ValueError("W_gate and W_up must both be (d_ff, d_model) with d_ff % 32 == 0")
+    return torch.stack([W_gate.reshape(F // 32, 32, D), W_up.reshape(F // 32, 32, D)], dim=1).reshape(2 * F, D)
+
+
+def block_workspace(B: int, T: int, d_model: int, d_ff: int, device=None) -> torch.Tensor:
+    n = int(load().slstm_block_workspace_size(B, T, d_model, d_ff))
+    if n == 0:
+        raise ValueError("unsupported trunk-layer sizes (d_model % 8, d_ff % 32)")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sigmoid", max_iters: int = 8,
+                  fixed: bool = False, tol: float = 1e-5, eps: float = 1e-6, y: torch.Tensor = None,
+                  S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None, carry_mode: int = 0):
+    """The trunk layer's forward; returns (y, S, stats).  x (B, T, d_model)
+    fp32; Wx, W_gu (interleave_gate_up), W_down bf16."""
+    B, T, D = x.shape
+    F = W_down.shape[1]
+    _need(x, "x", (B, T, D))
+    _need(norm1_w, "norm1_w", (D,))
+    _need(norm2_w, "norm2_w", (D,))
+    _need(Wx, "Wx", (4 * D, D), torch.bfloat16)
+    _need(bias, "bias", (4, D))
+    _need(R, "R", (4, D))
+    _need(W_gu, "W_gu", (2 * F, D), torch.bfloat16)
+    _need(W_down, "W_down", (D, F), torch.bfloat16)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", (B, T, D))
+    if S is None:
+        S = torch.empty(B, T, 4, D, dtype=torch.float32, device=x.device)
+    _need(S, "S", (B, T, 4, D))
+    if stats is None:
+        stats = new_stats(x.device)
+    if ws is None:
+        ws = block_workspace(B, T, D, F, x.device)
+    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0, int(carry_mode))
+    check("slstm_block_forward", load().slstm_block_forward(
+        _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(y),
+        _ptr(S), ctypes.byref(cfg), _ptr(stats), B, T, D, F, float(eps), _ptr(ws), ws.numel(), _stream()))
+    return y, S, stats

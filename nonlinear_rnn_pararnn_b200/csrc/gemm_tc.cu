@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 #include <string.h>
 
+#include "block.h"
 #include "launchers.h"
 #include "tma.cuh"
 
@@ -48,6 +49,9 @@ struct TcArgs {
     int tma_out;            // the epilogue stores through the C tensor map
     long long c_split;      // element offset between the C slices of the splits
     unsigned *error;
+    int epi;                // GEMM_EPI_STORE, GEMM_EPI_SWIGLU or GEMM_EPI_RESIDUAL
+    __nv_bfloat16 *Cb;      // GEMM_EPI_SWIGLU: the [M][N/2] bf16 product
+    const float *res;       // GEMM_EPI_RESIDUAL: C = acc + res, res [M][N] (may be C)
 };
 
 // Named barrier with an OR reduction over `n` threads: every participant
@@ -315,6 +319,55 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float v[32];
                 tmem_ld32(lane_addr + (uint32_t)(c * EPI_COLS), v);
                 const int col0 = n0 + c * EPI_COLS;
+                if (g.epi == GEMM_EPI_SWIGLU) {
+                    // columns 64k .. 64k+31 are the gate of features 32k ..
+                    // 32k+31, columns 64k+32 .. 64k+63 their up projection:
+                    // write silu(gate) * up of the 32 features as bf16
+                    float u[32];
+                    tmem_ld32(lane_addr + (uint32_t)((c + 1) * EPI_COLS), u);
+                    ++c;
+                    ++chunk;
+                    const int grow = m0 + row;
+                    if (grow < g.M && col0 < g.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(g.Cb + (size_t)grow * (g.N >> 1) + (col0 >> 1));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const int i = 8 * j + 2 * h;
+                                // silu(v) = v / (1 + e^-v); the fast divide returns 0 once
+                                // the denominator passes 2^126, where silu is 0 to fp32 anyway
+                                const float a0 = __fdividef(v[i], 1.0f + __expf(-v[i])) * u[i];
+                                const float a1 = __fdividef(v[i + 1], 1.0f + __expf(-v[i + 1])) * u[i + 1];
+                                const __nv_bfloat162 pr = __floats2bfloat162_rn(a0, a1);
+                                w[h] = *reinterpret_cast<const uint32_t *>(&pr);
+                            }
+                            dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                    continue;
+                }
+                if (g.epi == GEMM_EPI_RESIDUAL) {
+                    const int grow = m0 + row;
+                    if (grow < g.M) {
+                        const float *src = g.res + (size_t)grow * g.N + col0;
+                        if ((g.N & 3) == 0 && col0 + 32 <= g.N) {
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 r4 = *reinterpret_cast<const float4 *>(src + 4 * j);
+                                v[4 * j] += r4.x;
+                                v[4 * j + 1] += r4.y;
+                                v[4 * j + 2] += r4.z;
+                                v[4 * j + 3] += r4.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (col0 + i < g.N) v[i] += src[i];
+                        }
+                    }
+                }
                 if (g.bias) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] += (col0 + i < g.N) ? __ldg(g.bias + col0 + i) : 0.0f;
@@ -453,6 +506,7 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, 
         ta2 = ta;
     }
     TcArgs g;
+    memset(&g, 0, sizeof(g));   // epi = GEMM_EPI_STORE
     g.C = C;
     g.bias = bias;
     g.M = M;
@@ -474,6 +528,40 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, 
     g.tma_out = ((N & 3) == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 && make_c_map(&tc, C, M, N, splits)) ? 1 : 0;
     if (a_mn) return b_mn ? launch_tc<true, true>(ta, ta2, tb, tc, g, st) : launch_tc<true, false>(ta, ta2, tb, tc, g, st);
     return b_mn ? launch_tc<false, true>(ta, ta2, tb, tc, g, st) : launch_tc<false, false>(ta, ta2, tb, tc, g, st);
+}
+
+cudaError_t gemm_tc_bf16_epi(const void *A, const void *Bm, float *C, __nv_bfloat16 *Cb, const float *res, int M,
+                             int N, int K, int epi, unsigned *error, cudaStream_t st)
+{
+    if (epi == GEMM_EPI_SWIGLU ? (Cb == nullptr || N % 64 != 0) : (C == nullptr || epi != GEMM_EPI_RESIDUAL ||
+                                                                    res == nullptr))
+        return cudaErrorInvalidValue;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, A, M, K, K, BM) || !make_map(&tb, Bm, N, K, K, BN)) return cudaErrorInvalidValue;
+    TcArgs g;
+    memset(&g, 0, sizeof(g));
+    g.C = C;
+    g.bias = nullptr;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.a_parts = 1;
+    g.kb_per_split = (K + BK - 1) / BK;   // no split-K: the epilogue sees whole sums
+    g.c_split = (long long)M * N;
+    g.error = error;
+    g.m_tiles = (M + BM - 1) / BM;
+    g.n_tiles = (N + BN - 1) / BN;
+    g.n_work = g.m_tiles * g.n_tiles;
+    g.epi = epi;
+    g.Cb = Cb;
+    g.res = res;
+    CUtensorMap tc;
+    memset(&tc, 0, sizeof(tc));
+    g.tma_out = (epi == GEMM_EPI_RESIDUAL && (N & 3) == 0 && (reinterpret_cast<uintptr_t>(C) & 15) == 0 &&
+                 make_c_map(&tc, C, M, N, 1))
+                    ? 1
+                    : 0;
+    return launch_tc<false, false>(ta, ta, tb, tc, g, st);
 }
 
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want)

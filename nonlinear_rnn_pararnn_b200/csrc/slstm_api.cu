@@ -3,6 +3,7 @@
 // launchers in launchers.h do the work.
 #include <stdint.h>
 
+#include "block.h"
 #include "launchers.h"
 
 using namespace slstm;
@@ -40,6 +41,13 @@ bool ws_ok(void *ws, size_t have, size_t need)
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SLSTM_OK : SLSTM_ERR_CUDA; }
+
+// The trunk layer: K-major bf16 GEMMs over d_model (rows of 16 bytes) and a
+// SwiGLU epilogue over blocks of 32 hidden features.
+bool block_sizes_ok(int B, int T, int D, int F)
+{
+    return sizes_ok(B, T, D, F) && D % 8 == 0 && F % 32 == 0;
+}
 
 }  // namespace
 
@@ -206,6 +214,36 @@ int slstm_newton_backward_varlen(const void *x, const void *Wx, int dtype, const
     return cuda_status(backward_launch(x, Wx, dtype, P, R, s0, S, dH, dx, dWx, dR, db, ds0, forget, 1, total_T,
                                        d_in, d_h, static_cast<char *>(ws) + vt, static_cast<cudaStream_t>(stream),
                                        &vl));
+}
+
+size_t slstm_block_workspace_size(int B, int T, int d_model, int d_ff)
+{
+    if (!block_sizes_ok(B, T, d_model, d_ff)) return 0;
+    return block_workspace_bytes(B, T, d_model, d_ff);
+}
+
+int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, const float *bias, const float *R,
+                        const float *norm2_w, const void *W_gu, const void *W_down, float *y, float *S,
+                        const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T, int d_model,
+                        int d_ff, float eps, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (cfg == nullptr) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
+    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
+    if (!block_sizes_ok(B, T, d_model, d_ff)) return SLSTM_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !(eps < 1e30f)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(norm1_w) || !aligned16(Wx) || !aligned16(bias) || !aligned16(R) ||
+        !aligned16(norm2_w) || !aligned16(W_gu) || !aligned16(W_down) || !aligned16(y) || !aligned16(S) ||
+        !aligned16(stats))
+        return SLSTM_ERR_INVALID_ARG;
+    const size_t M = (size_t)B * T;
+    const char *yb = reinterpret_cast<const char *>(y), *sb = reinterpret_cast<const char *>(S);
+    if (yb < sb + M * 16 * d_model && sb < yb + M * 4 * d_model) return SLSTM_ERR_INVALID_ARG;   // y overlaps S
+    if (!ws_ok(ws, ws_bytes, block_workspace_bytes(B, T, d_model, d_ff))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(block_forward_launch(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, y, S, *cfg, stats, B, T,
+                                            d_model, d_ff, eps, ws, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

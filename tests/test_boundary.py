@@ -164,3 +164,30 @@ def test_python_binding_validates_before_calling():
     P = torch.zeros(2, 8, 4, 8)
     with pytest.raises(ValueError):
         api.newton_forward(P, torch.zeros(4, 8))     # CPU tensors are refused
+
+
+def test_block_entry_point_rejects_bad_arguments():
+    lib = _lib.load()
+    E = _lib.SLSTM_ERR_INVALID_ARG
+    big = ctypes.c_size_t(1 << 40)
+    # (x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, y, S, cfg, stats, B, T, D, F, eps, ws, bytes, stream)
+
+    def fwd(x=FAKE, y=ctypes.c_void_p(0x10000), S=ctypes.c_void_p(0x20000000), cfg=None, B=2, T=16, D=64, F=256,
+            eps=1e-6, wb=big):
+        c = cfg if cfg is not None else _cfg()
+        return lib.slstm_block_forward(x, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, y, S, ctypes.byref(c), FAKE,
+                                       B, T, D, F, eps, FAKE, wb, NULL)
+
+    assert fwd(D=60) == E                       # d_model % 8
+    assert fwd(F=250) == E                      # d_ff % 32
+    assert fwd(B=0) == E and fwd(T=0) == E
+    assert fwd(eps=-1.0) == E and fwd(eps=float("nan")) == E
+    assert fwd(x=FAKE_MIS) == E
+    assert fwd(cfg=_cfg(max_iters=0)) == E
+    assert fwd(wb=ctypes.c_size_t(64)) == E     # workspace too small
+    assert fwd(S=ctypes.c_void_p(0x10000 + 256)) == E   # y and S overlap
+    assert lib.slstm_block_workspace_size(2, 16, 60, 256) == 0
+    assert lib.slstm_block_workspace_size(2, 16, 64, 250) == 0
+    n = lib.slstm_block_workspace_size(2, 16, 64, 256)
+    # at least the bf16 activations and the fp32 pre-activations
+    assert n >= 2 * 16 * 64 * 2 + 2 * 16 * 4 * 64 * 4
