@@ -357,3 +357,50 @@ def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gate, W_up, W_down, forget
         z2 = round_bf16(z2)
     y = u + swiglu(z2.reshape(B * T, D), W_gate, W_up, W_down, bf16_operands).reshape(B, T, D)
     return y, S
+
+
+def rmsnorm_backward(v, w, dz, eps=1e-6):
+    """Gradients of sum(dz * rmsnorm(v, w)) with respect to v and w.
+    With r = (mean(v^2) + eps)^(-1/2) and z_i = w_i v_i r over the model axis
+    of size D: dv_j = r w_j dz_j - (r^3 v_j / D) sum_i dz_i w_i v_i and
+    dw_i = sum over rows of dz_i v_i r."""
+    v, w, dz = _f64(v), _f64(w), _f64(dz)
+    D = v.shape[-1]
+    r = 1.0 / np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    s = np.sum(dz * w * v, axis=-1, keepdims=True)
+    dv = r * w * dz - (r ** 3) * v * s / D
+    dw = np.sum((dz * v * r).reshape(-1, D), axis=0)
+    return dv, dw
+
+
+def block_backward(x, norm1_w, Wx, bias, R, norm2_w, W_gate, W_up, W_down, dY, forget="sigmoid", eps=1e-6):
+    """Gradients of L = sum(dY * y) for y = block_forward(...) without operand
+    rounding (the rounded forward is piecewise constant in its operands; its
+    gradient is read as that of the unrounded function).  Returns dict dx,
+    dnorm1_w, dWx, dbias, dR, dnorm2_w, dW_gate, dW_up, dW_down."""
+    x, dY = _f64(x), _f64(dY)
+    B, T, D = x.shape
+    M = B * T
+    z1 = rmsnorm(x, norm1_w, eps)
+    P = preact(z1, Wx, bias)
+    S = sequential_btgd(P, R, np.zeros((B, 4, D)), forget)
+    u = x + S[:, :, 3, :]
+    z2 = rmsnorm(u, norm2_w, eps).reshape(M, D)
+    g = gemm(z2, W_gate, tb=True)
+    v = gemm(z2, W_up, tb=True)
+    sg = 1.0 / (1.0 + np.exp(-g))
+    a = g * sg * v
+    dY2 = dY.reshape(M, D)
+    dW_down = gemm(dY2, a, ta=True)                       # (D, F)
+    da = gemm(dY2, W_down)                                # (M, F)
+    dg = da * v * sg * (1.0 + g * (1.0 - sg))             # silu'(g) = s (1 + g (1 - s))
+    dv = da * g * sg
+    dW_gate = gemm(dg, z2, ta=True)
+    dW_up = gemm(dv, z2, ta=True)
+    dz2 = gemm(dg, W_gate) + gemm(dv, W_up)
+    du_n, dnorm2_w = rmsnorm_backward(u.reshape(M, D), norm2_w, dz2, eps)
+    du = dY + du_n.reshape(B, T, D)
+    cell = backward_btgd(z1, Wx, P, R, np.zeros((B, 4, D)), S, du, forget)
+    dx_n, dnorm1_w = rmsnorm_backward(x, norm1_w, cell["dx"], eps)
+    return {"dx": du + dx_n, "dnorm1_w": dnorm1_w, "dWx": cell["dWx"], "dbias": cell["db"], "dR": cell["dR"],
+            "dnorm2_w": dnorm2_w, "dW_gate": dW_gate, "dW_up": dW_up, "dW_down": dW_down}

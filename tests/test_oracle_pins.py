@@ -464,3 +464,34 @@ def test_block_wiring():
     # bf16 operands move the result by about the bf16 step, no more
     yb, _ = oracle.block_forward(x, w1, Wx, bias, R, w2, Wg, Wu, Wd, bf16_operands=True)
     assert 0 < np.abs(yb - y).max() < 2e-2
+
+
+def test_block_backward_matches_finite_differences():
+    """Central differences of L = sum(dY * y) along one random direction per
+    argument pin every gradient of the trunk layer (norms, SwiGLU, the cell)."""
+    rng = np.random.default_rng(5)
+    B, T, D, F = 2, 6, 4, 8
+    args = {"x": rng.standard_normal((B, T, D)), "norm1_w": rng.uniform(0.5, 1.5, D),
+            "Wx": rng.standard_normal((4 * D, D)) / 2, "bias": np.zeros((4, D)), "R": rng.uniform(-0.5, 0.5, (4, D)),
+            "norm2_w": rng.uniform(0.5, 1.5, D), "W_gate": rng.standard_normal((F, D)) / 2,
+            "W_up": rng.standard_normal((F, D)) / 2, "W_down": rng.standard_normal((D, F)) / 3}
+    args["bias"][2] = 3.0
+    dY = rng.standard_normal((B, T, D))
+    names = list(args)
+
+    def loss(a):
+        y, _ = oracle.block_forward(*[a[k] for k in names])
+        return float(np.sum(dY * y))
+
+    grads = oracle.block_backward(*[args[k] for k in names], dY)
+    key = {"x": "dx", "norm1_w": "dnorm1_w", "Wx": "dWx", "bias": "dbias", "R": "dR", "norm2_w": "dnorm2_w",
+           "W_gate": "dW_gate", "W_up": "dW_up", "W_down": "dW_down"}
+    h = 1e-6
+    for k in names:
+        e = rng.standard_normal(args[k].shape)
+        ap, am = dict(args), dict(args)
+        ap[k] = args[k] + h * e
+        am[k] = args[k] - h * e
+        fd = (loss(ap) - loss(am)) / (2 * h)
+        an = float(np.sum(grads[key[k]] * e))
+        assert abs(fd - an) <= 1e-6 * (1 + abs(an)), (k, fd, an)
