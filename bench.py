@@ -635,7 +635,7 @@ def run_block(args, w):
 
 # DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
 # last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
-# (profiles/newton_iter_train_b8_t2048_d1024.md).  The counters describe the kernel sources with
+# (the newton_iter capture summarised under profiles/).  The counters describe the kernel sources with
 # this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
 # (every tile moves the same bytes), so it scales to a full launch by the element count.
 NEWTON_TRAFFIC = {"sources_sha256": "a1354d490b4ffca0023f55f55b9b12a31166f1d56c4ea2ff2b1e91f2ce16bad2", "first": 29.95, "middle": 46.33, "last": 46.35}

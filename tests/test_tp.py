@@ -97,8 +97,8 @@ def _worker(rank, world, port, q):
     q.put((rank, j0, j1, S, dx.numpy(), g["dWx"], g["dR"], g["db"], g["ds0"]))
 
 
-def test_tensor_parallel_shards_match_full_problem_gloo_world2():
-    world = 2
+@pytest.mark.parametrize("world", [2, 3])
+def test_tensor_parallel_shards_match_full_problem_gloo(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     s = socket.socket()
@@ -118,7 +118,10 @@ def test_tensor_parallel_shards_match_full_problem_gloo_world2():
     x, Wx, bias, R, s0, dH = _problem()
     S, g = _oracle_pass(x, Wx, bias, R, s0, dH)
     d = R.shape[1]
-    assert got[0][0] == 0 and got[0][1] == 32 and got[1][0] == 32 and got[1][1] == d
+    # 72 features = three 32-feature groups: [0, 32) + [32, 72) for two ranks,
+    # [0, 32) + [32, 64) + [64, 72) for three
+    want = {2: [(0, 32), (32, 72)], 3: [(0, 32), (32, 64), (64, 72)]}[world]
+    assert [(got[r][0], got[r][1]) for r in range(world)] == want and want[-1][1] == d
     for r in range(world):
         j0, j1, Sr, dx, dWx, dR, db, ds0 = got[r]
         np.testing.assert_allclose(Sr, S[..., j0:j1], rtol=0, atol=1e-12)
