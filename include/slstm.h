@@ -349,6 +349,31 @@ int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, co
                         const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T, int d_model,
                         int d_ff, float eps, void *ws, size_t ws_bytes, slstm_stream_t stream);
 
+/*
+ * Gradients of L = sum(dY * y) for y = slstm_block_forward(...), given x, the
+ * weights and the forward's S (the layer's activations are recomputed):
+ *   dx (B, T, d_model), dnorm1_w, dnorm2_w (d_model), dWx (4 d_model,
+ *   d_model), dbias, dR (4, d_model), dW_gu (2 d_ff, d_model; the interleaved
+ *   row order of W_gu), dW_down (d_model, d_ff), all fp32, caller-owned,
+ *   16-byte aligned, none overlapping an input.
+ * Read as the gradient of the layer with unrounded operands (the bf16
+ * rounding of z1, z2 and the SwiGLU product is piecewise constant): the
+ * recomputed z1 and z2 are the forward's bf16 values, every gradient is
+ * formed in fp32.  The cell's part is slstm_newton_backward's (dH = dL/du,
+ * zero initial state, its tensor-core GEMMs); the SwiGLU and norm gradients
+ * use CUDA-core fp32 GEMMs.  Sizes as slstm_block_forward; workspace:
+ * slstm_block_backward_workspace_size(B, T, d_model, d_ff) bytes, 256-byte
+ * aligned.  Returns SLSTM_ERR_INVALID_ARG before touching the GPU for bad
+ * sizes, forget mode, eps, alignment or workspace.
+ */
+size_t slstm_block_backward_workspace_size(int B, int T, int d_model, int d_ff);
+
+int slstm_block_backward(const float *x, const float *norm1_w, const void *Wx, const float *bias, const float *R,
+                         const float *norm2_w, const void *W_gu, const void *W_down, const float *S, const float *dY,
+                         float *dx, float *dnorm1_w, float *dWx, float *dbias, float *dR, float *dnorm2_w,
+                         float *dW_gu, float *dW_down, int forget, int B, int T, int d_model, int d_ff, float eps,
+                         void *ws, size_t ws_bytes, slstm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,8 @@ SIGNATURES = {
                                           _I, _V, _Z, _V]),
     "slstm_decode_step": (_I, [_V, _V, _I, _V, _V, _V, _V, _I, _I, _I, _I, _V]),
     "slstm_block_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "slstm_block_backward_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "slstm_block_backward": (_I, [_V] * 18 + [_I, _I, _I, _I, _I, ctypes.c_float, _V, _Z, _V]),
     "slstm_block_forward": (_I, [_V, _V, _V, _V, _V, _V, _V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V,
                                  _I, _I, _I, _I, ctypes.c_float, _V, _Z, _V]),
 }

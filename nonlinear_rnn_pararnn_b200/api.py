@@ -329,3 +329,39 @@ def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sig
         _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(y),
         _ptr(S), ctypes.byref(cfg), _ptr(stats), B, T, D, F, float(eps), _ptr(ws), ws.numel(), _stream()))
     return y, S, stats
+
+
+def block_backward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, S, dY, *, forget="sigmoid", eps: float = 1e-6,
+                   out: dict = None, ws: torch.Tensor = None) -> dict:
+    """Gradients of sum(dY * y) of the trunk layer at x, given the forward's S;
+    returns dict dx, dnorm1_w, dWx, dbias, dR, dnorm2_w, dW_gu (interleaved
+    like W_gu), dW_down."""
+    B, T, D = x.shape
+    F = W_down.shape[1]
+    _need(x, "x", (B, T, D))
+    _need(norm1_w, "norm1_w", (D,))
+    _need(norm2_w, "norm2_w", (D,))
+    _need(Wx, "Wx", (4 * D, D), torch.bfloat16)
+    _need(bias, "bias", (4, D))
+    _need(R, "R", (4, D))
+    _need(W_gu, "W_gu", (2 * F, D), torch.bfloat16)
+    _need(W_down, "W_down", (D, F), torch.bfloat16)
+    _need(S, "S", (B, T, 4, D))
+    _need(dY, "dY", (B, T, D))
+    dev = x.device
+    if out is None:
+        out = {"dx": torch.empty(B, T, D, device=dev), "dnorm1_w": torch.empty(D, device=dev),
+               "dWx": torch.empty(4 * D, D, device=dev), "dbias": torch.empty(4, D, device=dev),
+               "dR": torch.empty(4, D, device=dev), "dnorm2_w": torch.empty(D, device=dev),
+               "dW_gu": torch.empty(2 * F, D, device=dev), "dW_down": torch.empty(D, F, device=dev)}
+    if ws is None:
+        n = int(load().slstm_block_backward_workspace_size(B, T, D, F))
+        if n == 0:
+            raise ValueError("unsupported trunk-layer sizes (d_model % 8, d_ff % 32)")
+        ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    names = ("dx", "dnorm1_w", "dWx", "dbias", "dR", "dnorm2_w", "dW_gu", "dW_down")
+    check("slstm_block_backward", load().slstm_block_backward(
+        _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(S),
+        _ptr(dY), *[_ptr(out[k]) for k in names], forget_code(forget), B, T, D, F, float(eps), _ptr(ws), ws.numel(),
+        _stream()))
+    return out

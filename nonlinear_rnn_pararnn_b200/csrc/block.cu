@@ -92,7 +92,224 @@ BlockLayout block_layout(void *ws, int B, int T, int D, int F)
     return l;
 }
 
+// ---------------------------------------------------------------------------
+// backward
+// ---------------------------------------------------------------------------
+
+// RMSNorm backward, one warp per row, for z = w v r with r = (mean(v^2) + eps)^(-1/2):
+//   out = base + r w dz - r^3 v (sum_i dz_i w_i v_i) / D
+// and dz is overwritten with the row's weight-gradient terms dz v r.  out may
+// be base and each element of dz_c is read, then written, by the same lane.
+__global__ void __launch_bounds__(NORM_ROWS * 32) norm_bwd_kernel(const float *v, const float *__restrict__ w,
+                                                                  float *dz_c, const float *base, float *out, int M,
+                                                                  int D, float eps)
+{
+    const int r = blockIdx.x * NORM_ROWS + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= M) return;
+    const int n4 = D >> 2;
+    const float4 *vr = reinterpret_cast<const float4 *>(v + (size_t)r * D);
+    float4 *dr = reinterpret_cast<float4 *>(dz_c + (size_t)r * D);
+    const float4 *br = reinterpret_cast<const float4 *>(base + (size_t)r * D);
+    float4 *orow = reinterpret_cast<float4 *>(out + (size_t)r * D);
+    const float4 *w4 = reinterpret_cast<const float4 *>(w);
+    float ss = 0.0f, sd = 0.0f;
+    for (int i = lane; i < n4; i += 32) {
+        const float4 a = vr[i], g = dr[i], wv = __ldg(w4 + i);
+        ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
+        sd = fmaf(g.x * wv.x, a.x, fmaf(g.y * wv.y, a.y, fmaf(g.z * wv.z, a.z, fmaf(g.w * wv.w, a.w, sd))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        sd += __shfl_xor_sync(0xffffffffu, sd, o);
+    }
+    const float rs = rsqrtf(ss / (float)D + eps);
+    const float k3 = rs * rs * rs * sd / (float)D;
+    for (int i = lane; i < n4; i += 32) {
+        const float4 a = vr[i], g = dr[i], wv = __ldg(w4 + i), b = br[i];
+        orow[i] = make_float4(b.x + rs * wv.x * g.x - k3 * a.x, b.y + rs * wv.y * g.y - k3 * a.y,
+                              b.z + rs * wv.z * g.z - k3 * a.z, b.w + rs * wv.w * g.w - k3 * a.w);
+        dr[i] = make_float4(g.x * a.x * rs, g.y * a.y * rs, g.z * a.z * rs, g.w * a.w * rs);
+    }
+}
+
+// SwiGLU backward, one thread per (row m, hidden feature f): gv holds the
+// gate/up projections in the interleaved column order (gate of f at column
+// 64 (f / 32) + f % 32, up 32 columns later); da[m][f] = dL/da.  Writes
+// dL/dgate and dL/dup over gv and the product a = silu(gate) up over da.
+__global__ void __launch_bounds__(256) swiglu_bwd_kernel(float *gv, float *da, long long total, int F)
+{
+    const long long q = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (q >= total) return;
+    const long long m = q / F;
+    const int f = (int)(q - m * F);
+    float *row = gv + m * 2 * F;
+    const int cg = (f >> 5) * 64 + (f & 31);
+    const float g = row[cg], u = row[cg + 32], d = da[q];
+    const float sg = __fdividef(1.0f, 1.0f + __expf(-g));   // 0 once e^-g passes 2^126
+    const float silu = g * sg;
+    row[cg] = d * u * sg * fmaf(g, 1.0f - sg, 1.0f);        // silu'(g) = s (1 + g (1 - s))
+    row[cg + 32] = d * silu;
+    da[q] = silu * u;
+}
+
+// Column sums of c (M x D) in a fixed order: chunk k of rows_per_chunk rows
+// into partial[k][:], then the chunks in order.
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const float *__restrict__ c, int M, int D,
+                                                             int rows_per_chunk, float *__restrict__ partial)
+{
+    const int i = blockIdx.x * 256 + threadIdx.x;
+    if (i >= D) return;
+    const int r0 = blockIdx.y * rows_per_chunk;
+    const int r1 = min(M, r0 + rows_per_chunk);
+    float acc = 0.0f;
+    for (int r = r0; r < r1; ++r) acc += c[(size_t)r * D + i];
+    partial[(size_t)blockIdx.y * D + i] = acc;
+}
+
+__global__ void __launch_bounds__(256) colsum_final_kernel(const float *__restrict__ partial, int n_chunks, int D,
+                                                           float *__restrict__ out)
+{
+    const int i = blockIdx.x * 256 + threadIdx.x;
+    if (i >= D) return;
+    float acc = 0.0f;
+    for (int k = 0; k < n_chunks; ++k) acc += partial[(size_t)k * D + i];
+    out[i] = acc;
+}
+
+constexpr int COLSUM_ROWS = 256;
+
+struct BlockBwdLayout {
+    unsigned *err;
+    __nv_bfloat16 *z1, *z2;   // (M, D) each
+    float *P;                 // (M, 4D)
+    float *u;                 // (M, D)
+    float *gv;                // (M, 2F): gate/up, then their gradients
+    float *da;                // (M, F): dL/da, then a
+    float *dz2, *dz1;         // (M, D) each
+    float *partial;           // (M / COLSUM_ROWS + 1, D)
+    void *cell_ws;
+};
+
+BlockBwdLayout block_bwd_layout(void *ws, int B, int T, int D, int F)
+{
+    const size_t M = (size_t)B * T;
+    const size_t chunks = (M + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    char *p = static_cast<char *>(ws);
+    BlockBwdLayout l;
+    l.err = reinterpret_cast<unsigned *>(p);
+    p += 256;
+    l.z1 = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += al256(M * D * 2);
+    l.z2 = reinterpret_cast<__nv_bfloat16 *>(p);
+    p += al256(M * D * 2);
+    l.P = reinterpret_cast<float *>(p);
+    p += al256(M * 4 * D * 4);
+    l.u = reinterpret_cast<float *>(p);
+    p += al256(M * D * 4);
+    l.gv = reinterpret_cast<float *>(p);
+    p += al256(M * 2 * F * 4);
+    l.da = reinterpret_cast<float *>(p);
+    p += al256(M * F * 4);
+    l.dz2 = reinterpret_cast<float *>(p);
+    p += al256(M * D * 4);
+    l.dz1 = reinterpret_cast<float *>(p);
+    p += al256(M * D * 4);
+    l.partial = reinterpret_cast<float *>(p);
+    p += al256(chunks * D * 4);
+    l.cell_ws = p;
+    return l;
+}
+
+cudaError_t colsum(const float *c, int M, int D, float *partial, float *out, cudaStream_t st)
+{
+    const int chunks = (M + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    colsum_partial_kernel<<<dim3((D + 255) / 256, chunks), 256, 0, st>>>(c, M, D, COLSUM_ROWS, partial);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    colsum_final_kernel<<<(D + 255) / 256, 256, 0, st>>>(partial, chunks, D, out);
+    return cudaGetLastError();
+}
+
+GemmDesc simt_desc(int M, int N, int K, const void *A, int adt, long long sam, long long sak, const void *Bm, int bdt,
+                   long long sbk, long long sbn, float *C)
+{
+    GemmDesc g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.A = A;
+    g.a_dtype = adt;
+    g.sam = sam;
+    g.sak = sak;
+    g.B = Bm;
+    g.b_dtype = bdt;
+    g.sbk = sbk;
+    g.sbn = sbn;
+    g.bias = nullptr;
+    g.C = C;
+    return g;
+}
+
 }  // namespace
+
+size_t block_backward_workspace_bytes(int B, int T, int D, int F)
+{
+    const size_t M = (size_t)B * T;
+    const size_t chunks = (M + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    return 256 + 2 * al256(M * D * 2) + al256(M * 4 * D * 4) + 3 * al256(M * D * 4) + al256(M * 2 * F * 4) +
+           al256(M * F * 4) + al256(chunks * D * 4) + backward_workspace_bytes(B, T, D, D);
+}
+
+cudaError_t block_backward_launch(const float *x, const float *norm1_w, const void *Wx, const float *bias,
+                                  const float *R, const float *norm2_w, const void *W_gu, const void *W_down,
+                                  const float *S, const float *dY, float *dx, float *dnorm1_w, float *dWx,
+                                  float *dbias, float *dR, float *dnorm2_w, float *dW_gu, float *dW_down, int forget,
+                                  int B, int T, int D, int F, float eps, void *ws, cudaStream_t st)
+{
+    const BlockBwdLayout l = block_bwd_layout(ws, B, T, D, F);
+    const int M = B * T;
+    const dim3 rows((M + NORM_ROWS - 1) / NORM_ROWS);
+    cudaError_t e = cudaMemsetAsync(l.err, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return e;
+    // the forward's activations: z1, P = z1 W_x^T + b, u = x + h, z2
+    block_norm_kernel<false><<<rows, NORM_ROWS * 32, 0, st>>>(x, nullptr, norm1_w, nullptr, l.z1, M, D, eps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = gemm_tc_bf16(l.z1, Wx, bias, l.P, M, 4 * D, D, l.err, st)) != cudaSuccess) return e;
+    block_norm_kernel<true><<<rows, NORM_ROWS * 32, 0, st>>>(x, S, norm2_w, l.u, l.z2, M, D, eps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // gate/up projections (interleaved columns) and dL/da = dY W_down
+    if ((e = gemm_simt(simt_desc(M, 2 * F, D, l.z2, SLSTM_BF16, D, 1, W_gu, SLSTM_BF16, 1, D, l.gv), st)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_simt(simt_desc(M, F, D, dY, SLSTM_F32, D, 1, W_down, SLSTM_BF16, F, 1, l.da), st)) != cudaSuccess)
+        return e;
+    const long long total = (long long)M * F;
+    swiglu_bwd_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(l.gv, l.da, total, F);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dW_down = dY^T a, dz2 = dgv W_gu, dW_gu = dgv^T z2
+    if ((e = gemm_simt(simt_desc(D, F, M, dY, SLSTM_F32, 1, D, l.da, SLSTM_F32, F, 1, dW_down), st)) != cudaSuccess)
+        return e;
+    if ((e = gemm_simt(simt_desc(M, D, 2 * F, l.gv, SLSTM_F32, 2LL * F, 1, W_gu, SLSTM_BF16, D, 1, l.dz2), st)) !=
+        cudaSuccess)
+        return e;
+    if ((e = gemm_simt(simt_desc(2 * F, D, M, l.gv, SLSTM_F32, 1, 2LL * F, l.z2, SLSTM_BF16, D, 1, dW_gu), st)) !=
+        cudaSuccess)
+        return e;
+    // du = dY + RMSNorm2 backward (into dx), dnorm2_w
+    norm_bwd_kernel<<<rows, NORM_ROWS * 32, 0, st>>>(l.u, norm2_w, l.dz2, dY, dx, M, D, eps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = colsum(l.dz2, M, D, l.partial, dnorm2_w, st)) != cudaSuccess) return e;
+    // the cell: dH = du; its input gradient is dz1
+    if ((e = backward_launch(l.z1, Wx, SLSTM_BF16, l.P, R, nullptr, S, dx, l.dz1, dWx, dR, dbias, nullptr, forget, B,
+                             T, D, D, l.cell_ws, st)) != cudaSuccess)
+        return e;
+    // dx = du + RMSNorm1 backward, dnorm1_w
+    norm_bwd_kernel<<<rows, NORM_ROWS * 32, 0, st>>>(x, norm1_w, l.dz1, dx, dx, M, D, eps);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return colsum(l.dz1, M, D, l.partial, dnorm1_w, st);
+}
 
 size_t block_workspace_bytes(int B, int T, int D, int F)
 {

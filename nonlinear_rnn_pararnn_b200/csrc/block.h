@@ -26,4 +26,13 @@ cudaError_t block_forward_launch(const float *x, const float *norm1_w, const voi
                                  float *S, const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
                                  int D, int F, float eps, void *ws, cudaStream_t st);
 
+// Gradients of sum(dY * y) for the forward above (recomputes its activations
+// from x and the forward's S).
+size_t block_backward_workspace_bytes(int B, int T, int D, int F);
+cudaError_t block_backward_launch(const float *x, const float *norm1_w, const void *Wx, const float *bias,
+                                  const float *R, const float *norm2_w, const void *W_gu, const void *W_down,
+                                  const float *S, const float *dY, float *dx, float *dnorm1_w, float *dWx,
+                                  float *dbias, float *dR, float *dnorm2_w, float *dW_gu, float *dW_down, int forget,
+                                  int B, int T, int D, int F, float eps, void *ws, cudaStream_t st);
+
 }  // namespace slstm

@@ -246,4 +246,29 @@ int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, co
                                             d_model, d_ff, eps, ws, static_cast<cudaStream_t>(stream)));
 }
 
+size_t slstm_block_backward_workspace_size(int B, int T, int d_model, int d_ff)
+{
+    if (!block_sizes_ok(B, T, d_model, d_ff)) return 0;
+    return block_backward_workspace_bytes(B, T, d_model, d_ff);
+}
+
+int slstm_block_backward(const float *x, const float *norm1_w, const void *Wx, const float *bias, const float *R,
+                         const float *norm2_w, const void *W_gu, const void *W_down, const float *S, const float *dY,
+                         float *dx, float *dnorm1_w, float *dWx, float *dbias, float *dR, float *dnorm2_w,
+                         float *dW_gu, float *dW_down, int forget, int B, int T, int d_model, int d_ff, float eps,
+                         void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!block_sizes_ok(B, T, d_model, d_ff)) return SLSTM_ERR_INVALID_ARG;
+    if (!(eps >= 0.0f) || !(eps < 1e30f)) return SLSTM_ERR_INVALID_ARG;
+    const void *ptrs[] = {x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, S, dY,
+                          dx, dnorm1_w, dWx, dbias, dR, dnorm2_w, dW_gu, dW_down};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, block_backward_workspace_bytes(B, T, d_model, d_ff))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(block_backward_launch(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, S, dY, dx, dnorm1_w, dWx,
+                                             dbias, dR, dnorm2_w, dW_gu, dW_down, forget, B, T, d_model, d_ff, eps, ws,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

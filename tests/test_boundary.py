@@ -191,3 +191,20 @@ def test_block_entry_point_rejects_bad_arguments():
     n = lib.slstm_block_workspace_size(2, 16, 64, 256)
     # at least the bf16 activations and the fp32 pre-activations
     assert n >= 2 * 16 * 64 * 2 + 2 * 16 * 4 * 64 * 4
+
+
+def test_block_backward_entry_point_rejects_bad_arguments():
+    lib = _lib.load()
+    E = _lib.SLSTM_ERR_INVALID_ARG
+    big = ctypes.c_size_t(1 << 40)
+
+    def bwd(x=FAKE, forget=0, B=2, T=16, D=64, F=256, eps=1e-6, wb=big):
+        return lib.slstm_block_backward(x, *([FAKE] * 17), forget, B, T, D, F, eps, FAKE, wb, NULL)
+
+    assert bwd(forget=5) == E
+    assert bwd(D=60) == E and bwd(F=100) == E and bwd(B=0) == E
+    assert bwd(eps=-1.0) == E
+    assert bwd(x=FAKE_MIS) == E
+    assert bwd(wb=ctypes.c_size_t(64)) == E
+    assert lib.slstm_block_backward_workspace_size(2, 16, 64, 250) == 0
+    assert lib.slstm_block_backward_workspace_size(2, 16, 64, 256) > lib.slstm_block_workspace_size(2, 16, 64, 256)

@@ -74,3 +74,32 @@ def test_block_forward_in_place(cuda_device):
     y2, _, _ = _run(p, "sigmoid", y=x, x_override=x)
     torch.cuda.synchronize()
     assert y2.data_ptr() == x.data_ptr() and torch.equal(y2, y)
+
+
+@pytest.mark.parametrize("B,T,D,F,forget", [(2, 40, 64, 256, "sigmoid"), (1, 33, 96, 384, "sigmoid"),
+                                            (2, 8, 64, 256, "exp")])
+def test_block_backward_matches_oracle(B, T, D, F, forget, cuda_device):
+    """Gradients of sum(dY * y) from the forward's S against the oracle's
+    gradient of the unrounded layer; the GPU's recomputed z1, z2 are the
+    forward's bf16 values, so the per-tensor bound is the bf16 one for
+    gradients, 1e-2 (1 + max |g|)."""
+    p = _params(B, T, D, F, 83)
+    x, w1, w2, Wx, bias, R, Wg, Wu, Wd = p
+    y, S, st = _run(p, forget)
+    torch.cuda.synchronize()
+    assert api.read_stats(st)["converged"]
+    dY = torch.randn(B, T, D, generator=torch.Generator().manual_seed(84))
+    d = [t.cuda() for t in (x, w1, Wx, bias, R, w2)]
+    W_gu = api.interleave_gate_up(Wg, Wu).contiguous().cuda()
+    out = api.block_backward(d[0], d[1], d[2], d[3], d[4], d[5], W_gu, Wd.cuda(), S, dY.cuda(), forget=forget)
+    torch.cuda.synchronize()
+    ref = oracle.block_backward(as_f64(x), as_f64(w1), as_f64(Wx), as_f64(bias), as_f64(R), as_f64(w2), as_f64(Wg),
+                                as_f64(Wu), as_f64(Wd), as_f64(dY), forget)
+    gu = as_f64(out["dW_gu"].cpu()).reshape(F // 32, 2, 32, D)
+    got = {k: as_f64(out[k].cpu()) for k in ("dx", "dnorm1_w", "dWx", "dbias", "dR", "dnorm2_w", "dW_down")}
+    got["dW_gate"] = gu[:, 0].reshape(F, D)
+    got["dW_up"] = gu[:, 1].reshape(F, D)
+    for k, g in got.items():
+        r = ref[k]
+        err = float(np.abs(g - r).max() / (1 + np.abs(r).max()))
+        assert err <= 1e-2, (k, err)
