@@ -361,7 +361,8 @@ int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, co
  * recomputed z1 and z2 are the forward's bf16 values, every gradient is
  * formed in fp32.  The cell's part is slstm_newton_backward's (dH = dL/du,
  * zero initial state, its tensor-core GEMMs); the SwiGLU and norm gradients
- * use CUDA-core fp32 GEMMs.  Sizes as slstm_block_forward; workspace:
+ * use CUDA-core fp32 GEMMs.  Sizes as slstm_block_forward and B * T <=
+ * 8 388 480 (65535 row tiles of 128 for those GEMMs); workspace:
  * slstm_block_backward_workspace_size(B, T, d_model, d_ff) bytes, 256-byte
  * aligned.  Returns SLSTM_ERR_INVALID_ARG before touching the GPU for bad
  * sizes, forget mode, eps, alignment or workspace.

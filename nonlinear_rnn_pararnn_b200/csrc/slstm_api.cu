@@ -49,6 +49,10 @@ bool block_sizes_ok(int B, int T, int D, int F)
     return sizes_ok(B, T, D, F) && D % 8 == 0 && F % 32 == 0;
 }
 
+// The trunk backward's CUDA-core GEMMs tile the B*T rows 128 at a time on the
+// grid's y axis (at most 65535 tiles).
+constexpr long long kBlockBwdMaxRows = 65535LL * 128;
+
 }  // namespace
 
 extern "C" {
@@ -260,6 +264,7 @@ int slstm_block_backward(const float *x, const float *norm1_w, const void *Wx, c
 {
     if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
     if (!block_sizes_ok(B, T, d_model, d_ff)) return SLSTM_ERR_INVALID_ARG;
+    if ((long long)B * T > kBlockBwdMaxRows) return SLSTM_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SLSTM_ERR_INVALID_ARG;
     const void *ptrs[] = {x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, S, dY,
                           dx, dnorm1_w, dWx, dbias, dR, dnorm2_w, dW_gu, dW_down};

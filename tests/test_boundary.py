@@ -203,6 +203,7 @@ def test_block_backward_entry_point_rejects_bad_arguments():
 
     assert bwd(forget=5) == E
     assert bwd(D=60) == E and bwd(F=100) == E and bwd(B=0) == E
+    assert bwd(B=2, T=65535 * 64 + 1) == E            # more row tiles than the grid's y axis
     assert bwd(eps=-1.0) == E
     assert bwd(x=FAKE_MIS) == E
     assert bwd(wb=ctypes.c_size_t(64)) == E
