@@ -136,3 +136,18 @@ def test_tensor_parallel_shards_match_full_problem_gloo(world):
     Wl, bl, Rl = tp.shard_params(Wx, bias, R, 0, 32)
     _, gp = _oracle_pass(x, Wl, bl, Rl, tp.shard_state(s0, 0, 32), tp.shard_state(dH, 0, 32))
     assert np.abs(gp["dx"] - g["dx"]).max() > 1e-3
+
+
+def test_empty_shard_forward_and_backward_need_no_kernels():
+    """A rank beyond the group count owns no features: its forward returns
+    empty (B, T, 4, 0) tensors and its backward a zero input gradient of the
+    full shape (its share of the all-reduce) without calling the library."""
+    B, T, d_in = 2, 5, 8
+    x = torch.randn(B, T, d_in)
+    Wl, bl, Rl = tp.shard_params(torch.zeros(4 * 32, d_in), torch.zeros(4, 32), torch.zeros(4, 32), 32, 32)
+    assert Wl.shape == (0, d_in) and bl.shape == (4, 0) and Rl.shape == (4, 0)
+    P, S, st = tp.forward(x, Wl, bl, Rl)
+    assert P.shape == (B, T, 4, 0) and S.shape == (B, T, 4, 0) and st is None
+    out = tp.backward(x, Wl, P, Rl, None, S, torch.empty(B, T, 0))
+    assert out["dx"].shape == (B, T, d_in) and not out["dx"].any()
+    assert out["dWx"].shape == (0, d_in) and out["dR"].shape == (4, 0)
