@@ -42,6 +42,15 @@ bool ws_ok(void *ws, size_t have, size_t need)
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SLSTM_OK : SLSTM_ERR_CUDA; }
 
+// The Newton configuration fields every forward entry point checks.
+bool config_ok(const slstm_newton_config &c)
+{
+    if (c.max_iters < 1 || c.max_iters > SLSTM_MAX_ITERS) return false;
+    if (c.forget != SLSTM_FORGET_SIGMOID && c.forget != SLSTM_FORGET_EXP) return false;
+    if (!(c.tol >= 0.0f) || c.wait_limit_us < 0) return false;
+    return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
+}
+
 // The trunk layer: K-major bf16 GEMMs over d_model (rows of 16 bytes) and a
 // SwiGLU epilogue over blocks of 32 hidden features.
 bool block_sizes_ok(int B, int T, int D, int F)
@@ -112,10 +121,7 @@ int slstm_newton_forward(const float *P, const float *R, const float *s0, float 
                          int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
 {
     if (cfg == nullptr) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
-    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
+    if (!config_ok(*cfg)) return SLSTM_ERR_INVALID_ARG;
     if (!sizes_ok(B, T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
         return SLSTM_ERR_INVALID_ARG;
@@ -183,10 +189,7 @@ int slstm_newton_forward_varlen(const float *P, const float *R, const float *s0,
                                 int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
 {
     if (cfg == nullptr || cu_seqlens == nullptr) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
-    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
+    if (!config_ok(*cfg)) return SLSTM_ERR_INVALID_ARG;
     if (!varlen_sizes_ok(n_seq, total_T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
@@ -232,10 +235,7 @@ int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, co
                         int d_ff, float eps, void *ws, size_t ws_bytes, slstm_stream_t stream)
 {
     if (cfg == nullptr) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->max_iters < 1 || cfg->max_iters > SLSTM_MAX_ITERS) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->forget != SLSTM_FORGET_SIGMOID && cfg->forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
-    if (!(cfg->tol >= 0.0f) || cfg->wait_limit_us < 0) return SLSTM_ERR_INVALID_ARG;
-    if (cfg->carry_mode < SLSTM_CARRY_AUTO || cfg->carry_mode > SLSTM_CARRY_TWO_PASS) return SLSTM_ERR_INVALID_ARG;
+    if (!config_ok(*cfg)) return SLSTM_ERR_INVALID_ARG;
     if (!block_sizes_ok(B, T, d_model, d_ff)) return SLSTM_ERR_INVALID_ARG;
     if (!(eps >= 0.0f) || !(eps < 1e30f)) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(norm1_w) || !aligned16(Wx) || !aligned16(bias) || !aligned16(R) ||
