@@ -404,3 +404,114 @@ def block_backward(x, norm1_w, Wx, bias, R, norm2_w, W_gate, W_up, W_down, dY, f
     dx_n, dnorm1_w = rmsnorm_backward(x, norm1_w, cell["dx"], eps)
     return {"dx": du + dx_n, "dnorm1_w": dnorm1_w, "dWx": cell["dWx"], "dbias": cell["db"], "dR": cell["dR"],
             "dnorm2_w": dnorm2_w, "dW_gate": dW_gate, "dW_up": dW_up, "dW_down": dW_down}
+
+
+# ----------------------------------------------------------------------------
+# head-wise recurrent mixing ("sLSTM in this library", section on mix='head':
+# block-diagonal R of shape (4, n_heads, d_head, d_head) run through the same
+# Newton loop; the dense-Jacobian form is the reference for factorised
+# kernels).  The gate pre-activations of feature j = head * d_head + i are
+#   a_g[j] = P_g[j] + sum_k R[g, head, i, k] h_{t-1}[head * d_head + k],
+# and the rest of the step is the diag cell's: the pinned lane step is called
+# with r = 0 on the mixed pre-activations.  Small problems only (Python loops).
+# ----------------------------------------------------------------------------
+def _head_mix(Rh, h):
+    """Rh (4, H, dh, dh), h (B, d) -> (B, 4, d) recurrent contributions."""
+    B, d = h.shape
+    _, H, dh, _ = Rh.shape
+    return np.einsum("ghik,bhk->bghi", Rh, h.reshape(B, H, dh)).reshape(B, 4, d)
+
+
+def _head_step_all(S_prev, Pt, Rh, forget):
+    """One step for every (b, j): returns s (B, 4, d), Jl (B, d, 4, 4) with the
+    recurrent path left out, G (B, d, 4, 4)."""
+    B, _, d = S_prev.shape
+    A = Pt + _head_mix(Rh, S_prev[:, 3, :])
+    s = np.zeros((B, 4, d))
+    Jl = np.zeros((B, d, 4, 4))
+    G = np.zeros((B, d, 4, 4))
+    z = np.zeros(4)
+    for b in range(B):
+        for j in range(d):
+            s[b, :, j], Jl[b, j], G[b, j] = step(S_prev[b, :, j], A[b, :, j], z, forget)
+    return s, Jl, G
+
+
+def sequential_head(P, Rh, s0, forget="sigmoid") -> np.ndarray:
+    """P (B, T, 4, d), Rh (4, H, dh, dh) with H dh = d, s0 (B, 4, d) -> S (B, T, 4, d)."""
+    P, Rh = _f64(P), _f64(Rh)
+    B, T, _, d = P.shape
+    S = np.zeros((B, T, 4, d))
+    prev = np.zeros((B, 4, d)) if s0 is None else _f64(s0).copy()
+    for t in range(T):
+        prev, _, _ = _head_step_all(prev, P[:, t], Rh, forget)
+        S[:, t] = prev
+    return S
+
+
+def head_jacobian(Jl, G, Rh):
+    """Dense per-head Jacobian ds_t / ds_{t-1}: (B, H, 4 dh, 4 dh), state index
+    e * dh + i for slot e of head feature i.  J = diag-lane part + G R routed
+    into the h column: d s[e, i] / d h[k] += sum_g G[i][e, g] R[g, head, i, k]."""
+    B, d = Jl.shape[:2]
+    _, H, dh, _ = Rh.shape
+    J = np.zeros((B, H, 4 * dh, 4 * dh))
+    for hd in range(H):
+        for i in range(dh):
+            j = hd * dh + i
+            for e in range(4):
+                for e2 in range(4):
+                    J[:, hd, e * dh + i, e2 * dh + i] += Jl[:, j, e, e2]
+                for k in range(dh):
+                    J[:, hd, e * dh + i, 3 * dh + k] += np.einsum("bg,g->b", G[:, j, e, :], Rh[:, hd, i, k])
+    return J
+
+
+def newton_head(P, Rh, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
+    """Newton over time with dense per-head Jacobian blocks, the same update,
+    stopping rule (max |F| / (1 + |s|) <= tol) and zero initial guess as the
+    diag oracle.  Returns (S, stats)."""
+    P, Rh = _f64(P), _f64(Rh)
+    B, T, _, d = P.shape
+    _, H, dh, _ = Rh.shape
+    s0v = np.zeros((B, 4, d)) if s0 is None else _f64(s0)
+    S = np.zeros((B, T, 4, d))
+    hist = []
+    conv = div = False
+    it = 0
+
+    def residual_and_jac(S):
+        F = np.zeros_like(S)
+        Js = []
+        for t in range(T):
+            prev = s0v if t == 0 else S[:, t - 1]
+            f, Jl, G = _head_step_all(prev, P[:, t], Rh, forget)
+            F[:, t] = S[:, t] - f
+            Js.append(head_jacobian(Jl, G, Rh))
+        return F, Js
+
+    def to_heads(x):   # (B, 4, d) -> (B, H, 4 dh)
+        return x.reshape(B, 4, H, dh).transpose(0, 2, 1, 3).reshape(B, H, 4 * dh)
+
+    def from_heads(y):
+        return y.reshape(B, H, 4, dh).transpose(0, 2, 1, 3).reshape(B, 4, d)
+
+    F, Js = residual_and_jac(S)
+    for it in range(1, max_iters + 1):
+        delta = np.zeros((B, H, 4 * dh))
+        for t in range(T):
+            delta = (np.einsum("bhij,bhj->bhi", Js[t], delta) if t > 0 else 0.0) - to_heads(F[:, t])
+            S[:, t] += from_heads(delta)
+        F, Js = residual_and_jac(S)
+        raw = float(np.max(np.abs(F)))
+        scaled = float(np.max(np.abs(F) / (1.0 + np.abs(S))))
+        hist.append((raw, scaled))
+        if not np.isfinite(raw):
+            div = True
+            break
+        if not fixed and scaled <= tol:
+            conv = True
+            break
+    if not conv and hist and hist[-1][0] > 1.0:
+        div = True
+    return S, {"iters": it, "converged": conv, "diverged": div, "max_abs_F": [h[0] for h in hist]}

@@ -495,3 +495,84 @@ def test_block_backward_matches_finite_differences():
         fd = (loss(ap) - loss(am)) / (2 * h)
         an = float(np.sum(grads[key[k]] * e))
         assert abs(fd - an) <= 1e-6 * (1 + abs(an)), (k, fd, an)
+
+
+# ---------------------------------------------------------------------------
+# head-wise recurrent mixing (dense per-head Jacobians)
+# ---------------------------------------------------------------------------
+def _head_case(B=2, T=7, H=2, dh=3, seed=6, scale=0.4):
+    rng = np.random.default_rng(seed)
+    d = H * dh
+    P = rng.standard_normal((B, T, 4, d))
+    P[:, :, 2, :] += 3.0
+    Rh = rng.uniform(-scale, scale, (4, H, dh, dh))
+    s0 = np.stack([rng.standard_normal((B, d)), rng.uniform(0.5, 1.5, (B, d)), rng.standard_normal((B, d)),
+                   rng.uniform(-0.5, 0.5, (B, d))], axis=1)
+    return P, Rh, s0
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_head_mixing_with_diagonal_blocks_is_diag_mixing(forget):
+    P, Rh, s0 = _head_case()
+    _, H, dh, _ = Rh.shape
+    r = np.stack([np.concatenate([np.diag(Rh[g, h]) for h in range(H)]) for g in range(4)])
+    Rdiag = np.zeros_like(Rh)
+    for g in range(4):
+        for h in range(H):
+            Rdiag[g, h] = np.diag(np.diag(Rh[g, h]))
+    np.testing.assert_allclose(oracle.sequential_head(P, Rdiag, s0, forget), oracle.sequential_btgd(P, r, s0, forget),
+                               rtol=1e-14, atol=1e-14)
+    # d_head = 1 is diag mixing too
+    P1, R1, s01 = _head_case(H=6, dh=1)
+    np.testing.assert_allclose(oracle.sequential_head(P1, R1, s01, forget),
+                               oracle.sequential_btgd(P1, R1[:, :, 0, 0], s01, forget), rtol=1e-14, atol=1e-14)
+
+
+def test_head_mixing_direction_of_the_weight():
+    """R[g, head, i, k] carries h of feature k into feature i: with only the
+    (0, 1) entries set, feature 1 of the head has no recurrence at all (the diag
+    cell with r = 0) while feature 0 depends on feature 1's trajectory."""
+    P, _, s0 = _head_case(B=1, H=1, dh=2)
+    Rh = np.zeros((4, 1, 2, 2))
+    Rh[:, 0, 0, 1] = [0.3, -0.4, 0.5, 0.2]
+    S = oracle.sequential_head(P, Rh, s0)
+    free = oracle.sequential_btgd(P[..., 1:], np.zeros((4, 1)), s0[..., 1:])
+    np.testing.assert_allclose(S[..., 1:], free, rtol=0, atol=1e-15)
+    plain0 = oracle.sequential_btgd(P[..., :1], np.zeros((4, 1)), s0[..., :1])
+    assert np.abs(S[..., 0] - plain0[..., 0]).max() > 1e-3
+
+
+def test_head_jacobian_matches_finite_differences():
+    P, Rh, s0 = _head_case(B=1, T=1)
+    _, H, dh, _ = Rh.shape
+    d = H * dh
+    _, Jl, G = oracle._head_step_all(s0, P[:, 0], Rh, "sigmoid")
+    J = oracle.head_jacobian(Jl, G, Rh)
+    eps = 1e-6
+    for hd in range(H):
+        for e2 in range(4):
+            for k in range(dh):
+                sp, sm = s0.copy(), s0.copy()
+                sp[0, e2, hd * dh + k] += eps
+                sm[0, e2, hd * dh + k] -= eps
+                fp, _, _ = oracle._head_step_all(sp, P[:, 0], Rh, "sigmoid")
+                fm, _, _ = oracle._head_step_all(sm, P[:, 0], Rh, "sigmoid")
+                col = (fp - fm)[0] / (2 * eps)          # (4, d)
+                for e in range(4):
+                    for i in range(dh):
+                        got = J[0, hd, e * dh + i, e2 * dh + k]
+                        assert abs(got - col[e, hd * dh + i]) <= 1e-6 * (1 + abs(got)), (hd, e, i, e2, k)
+                # no coupling across heads
+                other = [j for j in range(d) if j // dh != hd]
+                assert np.abs(col[:, other]).max() == 0.0
+
+
+def test_head_newton_prefix_exact_and_converges():
+    P, Rh, s0 = _head_case(T=6)
+    ref = oracle.sequential_head(P, Rh, s0)
+    for K in (1, 3):
+        S, _ = oracle.newton_head(P, Rh, s0, max_iters=K, fixed=True)
+        np.testing.assert_allclose(S[:, :K], ref[:, :K], rtol=1e-12, atol=1e-12)
+    S, st = oracle.newton_head(P, Rh, s0, max_iters=20, tol=1e-12)
+    assert st["converged"] and not st["diverged"]
+    np.testing.assert_allclose(S, ref, rtol=1e-10, atol=1e-10)
