@@ -209,3 +209,20 @@ def test_block_backward_entry_point_rejects_bad_arguments():
     assert bwd(wb=ctypes.c_size_t(64)) == E
     assert lib.slstm_block_backward_workspace_size(2, 16, 64, 250) == 0
     assert lib.slstm_block_backward_workspace_size(2, 16, 64, 256) > lib.slstm_block_workspace_size(2, 16, 64, 256)
+
+
+def test_interleave_gate_up_layout():
+    """W_gu rows 64 k .. 64 k + 31 are W_gate rows 32 k .. 32 k + 31 and rows
+    64 k + 32 .. 64 k + 63 the W_up rows of the same features."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import api
+    F, D = 96, 5
+    Wg = torch.arange(F * D, dtype=torch.float32).reshape(F, D)
+    Wu = -1 - Wg
+    W = api.interleave_gate_up(Wg, Wu)
+    assert W.shape == (2 * F, D)
+    for k in range(F // 32):
+        assert torch.equal(W[64 * k:64 * k + 32], Wg[32 * k:32 * k + 32])
+        assert torch.equal(W[64 * k + 32:64 * k + 64], Wu[32 * k:32 * k + 32])
+    with pytest.raises(ValueError):
+        api.interleave_gate_up(Wg[:40], Wu[:40])
