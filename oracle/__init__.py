@@ -53,7 +53,8 @@ def _load():
         lib.oracle_sequential.argtypes = [I, I, D, D, D, I, D]
         lib.oracle_sequential_unstabilised.argtypes = [I, I, D, D, D, I, D, D, D]
         lib.oracle_affine_solve.argtypes = [I, I, D, D, D, I, D]
-        lib.oracle_newton.argtypes = [I, I, D, D, D, I, I, I, ctypes.c_double, D, D, D, IP, IP, IP]
+        lib.oracle_newton.argtypes = [I, I, D, D, D, I, I, I, ctypes.c_double, I, I, D, D, D, D,
+                                      IP, IP, IP]
         lib.oracle_bptt.argtypes = [I, I, D, D, D, D, D, I, D, D, D, D]
         lib.oracle_gemm.argtypes = [I, I, I, D, I, D, I, D, D]
         for f in ("oracle_step", "oracle_sequential", "oracle_sequential_unstabilised",
@@ -160,20 +161,42 @@ def affine_solve(A, b, y0=None, reverse=False) -> np.ndarray:
     return y
 
 
-def newton(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
-    """fp64 Newton; returns (S, stats dict)."""
+INIT_DECOUPLED = 0
+INIT_ZERO = 1
+INIT_GIVEN = 2
+_INITS = {"decoupled": INIT_DECOUPLED, "zero": INIT_ZERO, "given": INIT_GIVEN}
+_RESIDUAL_MODES = {"scaled": 0, "raw": 1}
+
+
+def newton(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init="decoupled",
+           residual_mode="scaled", S_init=None):
+    """fp64 Newton; returns (S, stats dict).
+
+    init: "decoupled" (the trajectory with R = 0, the default), "zero", or
+    "given" with S_init (L, T, 4) as the initial guess.  residual_mode:
+    "scaled" (max |F| / (1 + |s|) <= tol) or "raw" (max |F| <= tol)."""
     lib = _load()
     P, R, s0 = _f64(P), _f64(R), _f64(s0)
     L, T, _ = P.shape
-    S = np.zeros((L, T, 4))
-    hr = np.full(max_iters, np.nan)
-    hs = np.full(max_iters, np.nan)
+    code = _INITS[init]
+    if code == INIT_GIVEN:
+        if S_init is None:
+            raise ValueError("init='given' needs S_init")
+        S = _f64(S_init).copy()
+        if S.shape != (L, T, 4):
+            raise ValueError(f"S_init shape {S.shape} != {(L, T, 4)}")
+    else:
+        S = np.zeros((L, T, 4))
+    hr = np.full(max(max_iters, 1), np.nan)
+    hs = np.full(max(max_iters, 1), np.nan)
+    ir = np.zeros(2)
     it, conv, div = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     lib.oracle_newton(L, T, _ptr(P), _ptr(R), _ptr(s0), _forget_code(forget), int(max_iters),
-                      1 if fixed else 0, float(tol), _ptr(S), _ptr(hr), _ptr(hs),
-                      ctypes.byref(it), ctypes.byref(conv), ctypes.byref(div))
+                      1 if fixed else 0, float(tol), code, _RESIDUAL_MODES[residual_mode], _ptr(S),
+                      _ptr(hr), _ptr(hs), _ptr(ir), ctypes.byref(it), ctypes.byref(conv), ctypes.byref(div))
     return S, {"iters": it.value, "converged": bool(conv.value), "diverged": bool(div.value),
-               "max_abs_F": hr[: it.value].copy(), "max_scaled_F": hs[: it.value].copy()}
+               "max_abs_F": hr[: it.value].copy(), "max_scaled_F": hs[: it.value].copy(),
+               "init_max_abs_F": float(ir[0]), "init_max_scaled_F": float(ir[1])}
 
 
 def bptt(P, R, s0, S, dH, forget="sigmoid"):
@@ -221,10 +244,12 @@ def sequential_btgd(P, R, s0, forget="sigmoid") -> np.ndarray:
     return btgd_from_lanes(S, B, d)
 
 
-def newton_btgd(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
+def newton_btgd(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init="decoupled",
+                residual_mode="scaled", S_init=None):
     B, T, _, d = P.shape
+    Si = lanes_from_btgd(S_init) if S_init is not None else None
     S, st = newton(lanes_from_btgd(P), lanes_from_gd(R, B), lanes_from_bgd(s0), forget,
-                   max_iters, fixed, tol)
+                   max_iters, fixed, tol, init, residual_mode, Si)
     return btgd_from_lanes(S, B, d), st
 
 
@@ -269,15 +294,17 @@ def sequential_varlen(P, R, s0, cu, forget="sigmoid") -> np.ndarray:
     return S
 
 
-def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4) -> np.ndarray:
-    """K Newton iterations from the zero guess on every sequence (fixed-K mode)."""
+def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4, init="decoupled") -> np.ndarray:
+    """K Newton iterations from the given kind of guess ("decoupled" or "zero")
+    on every sequence (fixed-K mode)."""
     P = _f64(P)
     d = P.shape[2]
     S = np.zeros_like(P)
     for k, a, b in _segments(cu):
         if b > a:
             s0k = np.zeros((1, 4, d)) if s0 is None else _f64(s0)[k:k + 1]
-            S[a:b] = newton_btgd(P[None, a:b], R, s0k, forget, max_iters=K, fixed=True, tol=0.0)[0][0]
+            S[a:b] = newton_btgd(P[None, a:b], R, s0k, forget, max_iters=K, fixed=True, tol=0.0,
+                                  init=init)[0][0]
     return S
 
 

@@ -260,26 +260,79 @@ void oracle_affine_solve(int lanes, int T, const double *A, const double *b,
 }
 
 /*
+ * The decoupled trajectory: the cell run with the recurrent weights set to
+ * zero, so that no gate sees h_{t-1} while c, n and m still recur exactly.
+ * It is one of the initial guesses of oracle_newton below.  The pages give
+ * no initial guess beyond prepending h0 ([structure] "Current surface"); this
+ * is the reading taken for the default one.
+ */
+static void decoupled_trajectory(int T, const double *P, const double *s0, int forget, double *S)
+{
+    const double zero[4] = {0.0, 0.0, 0.0, 0.0};
+    const double *prev = s0;
+    for (int t = 0; t < T; ++t) {
+        oracle_step(prev, P + (size_t)t * 4, zero, forget, S + (size_t)t * 4, NULL, NULL);
+        prev = S + (size_t)t * 4;
+    }
+}
+
+/* Raw and scaled maxima of the residual of every lane at S; returns 1 when
+ * some residual or state entry is not finite. */
+static int residual_maxima(int lanes, int T, const double *P, const double *R, const double *s0,
+                           int forget, const double *S, double *F, double *raw, double *scaled)
+{
+    const size_t n4 = (size_t)T * 4;
+    int bad = 0;
+    *raw = 0.0;
+    *scaled = 0.0;
+    for (int l = 0; l < lanes; ++l) {
+        const double *Sl = S + (size_t)l * n4;
+        residual_and_jacobian(T, P + (size_t)l * n4, R + 4 * l, s0 + 4 * l, forget, Sl, F, NULL);
+        for (size_t q = 0; q < n4; ++q) {
+            const double a = fabs(F[q]);
+            if (!isfinite(a) || !isfinite(Sl[q])) bad = 1;
+            if (a > *raw) *raw = a;
+            const double sc = a / (1.0 + fabs(Sl[q]));
+            if (sc > *scaled) *scaled = sc;
+        }
+    }
+    if (bad) {
+        *raw = INFINITY;
+        *scaled = INFINITY;
+    }
+    return bad;
+}
+
+/*
  * Newton solve of the whole trajectory (ParaRNN Newton, as described in
  * [pararnn] "Cell" and [structure] "Current surface"):
- *   guess S = 0 for every t (s0 is fixed and enters as the step before t=0)
+ *   initial guess (s0 is fixed and enters as the step before t = 0):
+ *     init 0: the decoupled trajectory (decoupled_trajectory above); in
+ *             tolerance mode its residual is evaluated first, and a guess
+ *             that already meets the test ends the solve after 0 iterations;
+ *     init 1: S = 0 for every t;
+ *     init 2: S as given on entry (its residual is not evaluated);
  *   repeat k = 1..max_iters:
  *     F_t = S_t - f(S_{t-1}, P_t),  J_t = d f / d s_{t-1} at the guess
  *     solve delta_t = J_t delta_{t-1} - F_t,  delta_{-1} = 0
  *     S <- S + delta
  *     Fn = residual at the new S; record max|Fn| and max |Fn|/(1+|S|)
- *     stop when (not fixed) and max |Fn|/(1+|S|) <= tol
+ *     stop when (not fixed) and the test holds: max |Fn|/(1+|S|) <= tol
+ *     (residual_mode 0) or max|Fn| <= tol (residual_mode 1)
  *   diverged when not converged and (max|Fn| > 1 or non-finite) after the
  *   last iteration ([structure] "Current surface": NewtonDivergenceError if
  *   max|F| > 1 after K).  In fixed mode "converged" reports whether the final
- *   scaled residual meets tol.
+ *   residual meets the test.
  * All lanes iterate together and stop together (the residual is a max over
  * every lane, step and slot).
- * hist_raw / hist_scaled receive one value per iteration (max_iters long).
+ * hist_raw / hist_scaled receive one value per iteration (max_iters long);
+ * init_res (2 values, may be NULL) the raw and scaled residual of the initial
+ * guess, or -1 when it is not evaluated.
  */
 void oracle_newton(int lanes, int T, const double *P, const double *R,
                    const double *s0, int forget, int max_iters, int fixed,
-                   double tol, double *S, double *hist_raw, double *hist_scaled,
+                   double tol, int init, int residual_mode, double *S,
+                   double *hist_raw, double *hist_scaled, double *init_res,
                    int *iters, int *converged, int *diverged)
 {
     const size_t n4 = (size_t)T * 4;
@@ -287,12 +340,31 @@ void oracle_newton(int lanes, int T, const double *P, const double *R,
     double *J = malloc(sizeof(double) * n4 * 4);
     double *negF = malloc(sizeof(double) * n4);
     double *delta = malloc(sizeof(double) * n4);
-    memset(S, 0, sizeof(double) * n4 * lanes);
+    if (init == 0) {
+        for (int l = 0; l < lanes; ++l)
+            decoupled_trajectory(T, P + (size_t)l * n4, s0 + 4 * l, forget, S + (size_t)l * n4);
+    } else if (init == 1) {
+        memset(S, 0, sizeof(double) * n4 * lanes);
+    }
     *iters = 0;
     *converged = 0;
     *diverged = 0;
+    if (init_res) init_res[0] = init_res[1] = -1.0;
     double raw = INFINITY, scaled = INFINITY;
-    for (int k = 1; k <= max_iters; ++k) {
+    int done = 0;
+    if (init == 0 && !fixed) {
+        const int bad = residual_maxima(lanes, T, P, R, s0, forget, S, F, &raw, &scaled);
+        if (init_res) {
+            init_res[0] = raw;
+            init_res[1] = scaled;
+        }
+        const double test = residual_mode ? raw : scaled;
+        if (!bad && test <= tol) {
+            *converged = 1;
+            done = 1;
+        }
+    }
+    for (int k = 1; k <= max_iters && !done; ++k) {
         for (int l = 0; l < lanes; ++l) {
             double *Sl = S + (size_t)l * n4;
             residual_and_jacobian(T, P + (size_t)l * n4, R + 4 * l, s0 + 4 * l,
@@ -301,35 +373,18 @@ void oracle_newton(int lanes, int T, const double *P, const double *R,
             oracle_affine_solve(1, T, J, negF, NULL, 0, delta);
             for (size_t q = 0; q < n4; ++q) Sl[q] += delta[q];
         }
-        raw = 0.0;
-        scaled = 0.0;
-        int bad = 0;
-        for (int l = 0; l < lanes; ++l) {
-            double *Sl = S + (size_t)l * n4;
-            residual_and_jacobian(T, P + (size_t)l * n4, R + 4 * l, s0 + 4 * l,
-                                  forget, Sl, F, NULL);
-            for (size_t q = 0; q < n4; ++q) {
-                const double a = fabs(F[q]);
-                if (!isfinite(a) || !isfinite(Sl[q])) bad = 1;
-                if (a > raw) raw = a;
-                const double sc = a / (1.0 + fabs(Sl[q]));
-                if (sc > scaled) scaled = sc;
-            }
-        }
-        if (bad) {
-            raw = INFINITY;
-            scaled = INFINITY;
-        }
+        const int bad = residual_maxima(lanes, T, P, R, s0, forget, S, F, &raw, &scaled);
         hist_raw[k - 1] = raw;
         hist_scaled[k - 1] = scaled;
         *iters = k;
         if (bad) break;
-        if (!fixed && scaled <= tol) {
+        const double test = residual_mode ? raw : scaled;
+        if (!fixed && test <= tol) {
             *converged = 1;
             break;
         }
     }
-    if (fixed && scaled <= tol) *converged = 1;
+    if (fixed && (residual_mode ? raw : scaled) <= tol) *converged = 1;
     if (!*converged && !(raw <= 1.0)) *diverged = 1;
     free(F);
     free(J);

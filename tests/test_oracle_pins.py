@@ -265,6 +265,124 @@ def test_newton_divergence_flag():
     assert st["diverged"] and not st["converged"]
 
 
+def _closed_form_h_zero_recurrence(P, forget):
+    """h of the R = 0 cell from the zero state, by the log-space weighted
+    average h_t = o_t sum_s w_ts z_s / sum_s w_ts (the closed form pinned in
+    test_zero_recurrence_closed_form), for every lane and step."""
+    L, T, _ = P.shape
+    H = np.zeros((L, T))
+    for l in range(L):
+        z = np.tanh(P[l, :, 0])
+        o = 1 / (1 + np.exp(-P[l, :, 3]))
+        lf = P[l, :, 2] if forget == "exp" else -np.logaddexp(0, -P[l, :, 2])
+        cum = np.concatenate([[0.0], np.cumsum(lf)])
+        for t in range(T):
+            lw = P[l, : t + 1, 1] + (cum[t + 1] - cum[1 : t + 2])
+            w = np.exp(lw - lw.max())
+            H[l, t] = o[t] * (w @ z[: t + 1]) / w.sum()
+    return H
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_decoupled_guess_is_the_zero_recurrence_solution(forget):
+    """The default initial guess is the trajectory with R = 0.  With R = 0 it
+    is therefore the solution itself: the solve ends after 0 iterations with
+    a zero residual and h equal to the closed form."""
+    rng = np.random.default_rng(71)
+    P, _, _ = _rand_lane_inputs(rng, 3, 30, forget)
+    R = np.zeros((3, 4))
+    s0 = np.zeros((3, 4))
+    S, st = oracle.newton(P, R, s0, forget, max_iters=5, tol=1e-12)
+    assert st["iters"] == 0 and st["converged"] and not st["diverged"]
+    assert st["init_max_abs_F"] == 0.0
+    H = _closed_form_h_zero_recurrence(P, forget)
+    np.testing.assert_allclose(S[:, :, 3], H, rtol=0, atol=1e-12)
+    # with R != 0 the guess keeps the R = 0 gates: its h is still the closed
+    # form of the R = 0 cell, and its residual is nonzero
+    R2 = rng.uniform(-0.5, 0.5, size=(3, 4))
+    S2, st2 = oracle.newton(P, R2, s0, forget, max_iters=1, fixed=True, init="decoupled")
+    Sg, stg = oracle.newton(P, R2, s0, forget, max_iters=1, tol=1e30)
+    assert stg["iters"] == 0 and stg["init_max_abs_F"] > 1e-3
+    np.testing.assert_allclose(Sg[:, :, 3], H, rtol=0, atol=1e-12)
+    # a fixed-K solve does not stop at the guess
+    assert st2["iters"] == 1 and st2["init_max_abs_F"] == -1.0
+
+
+def _workload_lanes(rng, L, T, forget, r_scale):
+    """Lanes drawn like the workloads: P ~ N(0, 1) per gate (x ~ N(0,1) through
+    W_x ~ N(0, 1/d_in)), forget bias spread over [3, 6], R ~ U(-a, a)."""
+    P = rng.normal(size=(L, T, 4))
+    P[:, :, 2] += np.linspace(3.0, 6.0, L)[:, None]
+    R = rng.uniform(-r_scale, r_scale, size=(L, 4))
+    return P, R, np.zeros((L, 4))
+
+
+@pytest.mark.parametrize("forget,T", [("sigmoid", 1024), ("exp", 512)])
+def test_decoupled_guess_converges_where_the_zero_guess_diverges(forget, T):
+    """From the zero guess the iterates blow up on these lengths; from the
+    decoupled guess the solve converges in a few iterations, and a converged
+    iterate is the unique sequential trajectory."""
+    rng = np.random.default_rng(73)
+    P, R, s0 = _workload_lanes(rng, 6, T, forget, 0.5)
+    Sseq = oracle.sequential(P, R, s0, forget)
+    _, stz = oracle.newton(P, R, s0, forget, max_iters=8, tol=1e-8, init="zero")
+    assert not stz["converged"]
+    S, st = oracle.newton(P, R, s0, forget, max_iters=8, tol=1e-8)
+    assert st["converged"] and st["iters"] <= 6, st
+    np.testing.assert_allclose(S, Sseq, rtol=0, atol=1e-7 * (1 + np.abs(Sseq)).max())
+
+
+@pytest.mark.parametrize("init", ["decoupled", "zero", "given"])
+def test_newton_prefix_exact_from_every_guess(init):
+    """Prefix exactness holds whatever the guess: after k iterations the first
+    k steps are the sequential trajectory."""
+    rng = np.random.default_rng(79)
+    T = 10
+    P, R, s0 = _rand_lane_inputs(rng, 3, T, "sigmoid")
+    Sseq = oracle.sequential(P, R, s0, "sigmoid")
+    guess = np.abs(rng.normal(size=(3, T, 4))) + 0.5
+    for k in (1, 3):
+        S, st = oracle.newton(P, R, s0, "sigmoid", max_iters=k, fixed=True, init=init,
+                              S_init=guess if init == "given" else None)
+        assert st["iters"] == k
+        np.testing.assert_allclose(S[:, :k], Sseq[:, :k], rtol=0, atol=1e-12 * (1 + np.abs(Sseq).max()))
+        if init != "decoupled":   # from these guesses the rest is not exact yet
+            assert np.abs(S[:, k:] - Sseq[:, k:]).max() > 1e-9
+
+
+def test_newton_given_guess():
+    rng = np.random.default_rng(83)
+    P, R, s0 = _rand_lane_inputs(rng, 3, 16, "exp")
+    Sseq = oracle.sequential(P, R, s0, "exp")
+    # a guess at the solution stays there: F = 0, so delta = 0
+    S, st = oracle.newton(P, R, s0, "exp", max_iters=1, fixed=True, init="given", S_init=Sseq)
+    np.testing.assert_allclose(S, Sseq, rtol=0, atol=1e-12 * (1 + np.abs(Sseq).max()))
+    assert st["max_abs_F"][0] <= 1e-12 * (1 + np.abs(Sseq).max())
+    # a zero guess given explicitly is the zero init
+    Sz, stz = oracle.newton(P, R, s0, "exp", max_iters=3, fixed=True, init="zero")
+    Sg, stg = oracle.newton(P, R, s0, "exp", max_iters=3, fixed=True, init="given", S_init=np.zeros_like(P))
+    np.testing.assert_array_equal(Sz, Sg)
+    np.testing.assert_array_equal(stz["max_abs_F"], stg["max_abs_F"])
+
+
+def test_newton_residual_modes():
+    """residual_mode 'raw' stops at the first iteration with max|F| <= tol,
+    'scaled' at the first with max |F|/(1+|s|) <= tol; both histories are
+    the same iterates, so each stop is the first crossing of its column."""
+    rng = np.random.default_rng(89)
+    P, R, s0 = _workload_lanes(rng, 4, 256, "sigmoid", 0.5)
+    _, full = oracle.newton(P, R, s0, "sigmoid", max_iters=8, fixed=True, tol=0.0)
+    for mode, col in (("raw", "max_abs_F"), ("scaled", "max_scaled_F")):
+        tol = 1e-6
+        _, st = oracle.newton(P, R, s0, "sigmoid", max_iters=8, tol=tol, residual_mode=mode)
+        first = int(np.argmax(full[col] <= tol)) + 1
+        assert full[col][first - 1] <= tol
+        assert st["converged"] and st["iters"] == first
+        np.testing.assert_array_equal(st[col], full[col][:first])
+    # the scaled residual never exceeds the raw one
+    assert np.all(full["max_scaled_F"] <= full["max_abs_F"])
+
+
 # ---------------------------------------------------------------------------
 # backward
 # ---------------------------------------------------------------------------
