@@ -97,8 +97,8 @@ typedef enum {
  *               exact iteration count (fixed mode).
  *   fixed_iters 0: stop at the first iteration whose new iterate meets tol;
  *               1: run exactly max_iters iterations.
- *   tol         tolerance on the scaled residual max |F| / (1 + |s|), taken
- *               over every (b, t, slot, j) of the new iterate.
+ *   tol         tolerance of the stopping test (residual_mode), taken over
+ *               every (b, t, slot, j) of the new iterate.
  *   forget      slstm_forget.
  *   debug_fault 0 in normal use.  1 makes one tile of the first iteration
  *               withhold its scan carry, so that its successor's bounded
@@ -116,8 +116,28 @@ typedef enum {
  *               SLSTM_CARRY_AUTO (0) picks two passes when there are at
  *               most SMs / 4 feature groups (B * ceil(d_h/32)) and at least
  *               256 chunks of 64 steps, and debug_fault is 0.
+ *   init        the initial guess (the pages give none beyond prepending
+ *               h0; the default is this library's reading):
+ *               SLSTM_INIT_DECOUPLED (0): the trajectory of the cell with
+ *               its gates blind to h_{t-1} (R taken as 0: z, o, log i, log f
+ *               from P alone, c, n, m recurring exactly), computed by an
+ *               associative scan in one launch that reads P and writes S.
+ *               In tolerance mode the guess's own residual is tested first
+ *               and a guess that meets the test ends the solve after 0
+ *               iterations.  From this guess the solve converges in a few
+ *               iterations on long sequences where the zero guess overflows;
+ *               SLSTM_INIT_ZERO: S = 0 at every step;
+ *               SLSTM_INIT_GIVEN: S holds the guess on entry (warm start;
+ *               its residual is not tested, at least one iteration runs).
+ *   residual_mode  the stopping test: SLSTM_RESIDUAL_SCALED (0),
+ *               max |F| / (1 + |s|) <= tol; SLSTM_RESIDUAL_RAW, max|F| <= tol
+ *               (the pages' own norm).  Both maxima are recorded either way.
  */
 typedef enum { SLSTM_CARRY_AUTO = 0, SLSTM_CARRY_FUSED = 1, SLSTM_CARRY_TWO_PASS = 2 } slstm_carry_mode;
+
+typedef enum { SLSTM_INIT_DECOUPLED = 0, SLSTM_INIT_ZERO = 1, SLSTM_INIT_GIVEN = 2 } slstm_init;
+
+typedef enum { SLSTM_RESIDUAL_SCALED = 0, SLSTM_RESIDUAL_RAW = 1 } slstm_residual_mode;
 
 typedef struct {
     int max_iters;
@@ -127,13 +147,15 @@ typedef struct {
     int debug_fault;
     int wait_limit_us;
     int carry_mode;
+    int init;
+    int residual_mode;
 } slstm_newton_config;
 
 /*
  * Newton outcome, in DEVICE memory owned by the caller (zeroing it is not
  * required; slstm_newton_forward initialises it on the stream).
- *   iters        Newton iterations performed.
- *   converged    1 when the last iterate's scaled residual <= tol.
+ *   iters        Newton iterations performed (the initial guess is not one).
+ *   converged    1 when the last iterate meets the stopping test.
  *   diverged     1 when not converged and max|F| > 1 or non-finite after the
  *                last iteration ("NewtonDivergenceError" of the pages).
  *   error        0, SLSTM_ERR_DIVERGED when diverged, or SLSTM_ERR_TIMEOUT.
@@ -141,6 +163,9 @@ typedef struct {
  *                produced by iteration k (max over every element), for the
  *                last min(iters, 64) iterations.  In fixed mode only the final
  *                iteration evaluates its residual; the others hold -1.
+ *   init_max_abs_F, init_max_scaled_F   residual of the initial guess when
+ *                it was tested (SLSTM_INIT_DECOUPLED in tolerance mode),
+ *                else -1.
  */
 typedef struct {
     int iters;
@@ -149,6 +174,8 @@ typedef struct {
     int error;
     float max_abs_F[SLSTM_STATS_HISTORY];
     float max_scaled_F[SLSTM_STATS_HISTORY];
+    float init_max_abs_F;
+    float init_max_scaled_F;
 } slstm_newton_stats;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -178,7 +205,7 @@ int slstm_preact_gemm(const void *x, const void *Wx, int dtype, const float *bia
 /*
  * Newton solve of the whole trajectory ("sLSTM in this library", "Cell";
  * "pararnn-torch structure", "Current surface"):
- *   guess S = 0 for every step; s0 enters as the step before t = 0;
+ *   initial guess as cfg->init selects; s0 enters as the step before t = 0;
  *   each iteration evaluates F_t = S_t - f(S_{t-1}, P_t) and J_t = df/ds_{t-1}
  *   at the guess, solves delta_t = J_t delta_{t-1} - F_t (delta_{-1} = 0) by a
  *   blocked associative scan of 4x4 affine maps, and sets S <- S + delta;

@@ -31,16 +31,21 @@ SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5
 SLSTM_MAX_ITERS = 65536
 SLSTM_STATS_HISTORY = 64
 SLSTM_SCAN_REVERSE_T = 1
+SLSTM_INIT_DECOUPLED = 0
+SLSTM_INIT_ZERO = 1
+SLSTM_INIT_GIVEN = 2
+SLSTM_RESIDUAL_SCALED = 0
+SLSTM_RESIDUAL_RAW = 1
 SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class NewtonConfig(ctypes.Structure):
     _fields_ = [("max_iters", ctypes.c_int), ("fixed_iters", ctypes.c_int), ("tol", ctypes.c_float),
                 ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int),
-                ("carry_mode", ctypes.c_int)]
+                ("carry_mode", ctypes.c_int), ("init", ctypes.c_int), ("residual_mode", ctypes.c_int)]
 
 
-STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY
+STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY + 2 * 4
 
 _V = ctypes.c_void_p
 _I = ctypes.c_int

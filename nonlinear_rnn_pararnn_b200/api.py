@@ -70,6 +70,19 @@ def preact_gemm(x: torch.Tensor, Wx: torch.Tensor, bias: torch.Tensor, P: torch.
     return P
 
 
+_INIT = {"decoupled": _lib.SLSTM_INIT_DECOUPLED, "zero": _lib.SLSTM_INIT_ZERO, "given": _lib.SLSTM_INIT_GIVEN}
+_RESIDUAL = {"scaled": _lib.SLSTM_RESIDUAL_SCALED, "raw": _lib.SLSTM_RESIDUAL_RAW}
+
+
+def newton_config(max_iters: int, fixed: bool, tol: float, forget, debug_fault: int = 0, wait_limit_us: int = 0,
+                  carry_mode: int = 0, init="decoupled", residual_mode="scaled") -> NewtonConfig:
+    """The C ABI's slstm_newton_config.  init: "decoupled" (default), "zero"
+    or "given" (S holds the guess on entry); residual_mode: "scaled" or "raw"."""
+    return NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
+                        int(wait_limit_us), int(carry_mode), _INIT[init] if isinstance(init, str) else int(init),
+                        _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode))
+
+
 def new_stats(device=None) -> torch.Tensor:
     return torch.zeros(_lib.STATS_BYTES, dtype=torch.uint8, device=device or "cuda")
 
@@ -82,31 +95,34 @@ def read_stats(stats: torch.Tensor) -> dict:
     it = ints[0]
     m = _lib.SLSTM_STATS_HISTORY
     ks = list(range(max(0, it - m), it))     # the iterations the ring still holds
-    raw_h, sc_h = fl[:m].tolist(), fl[m:].tolist()
+    raw_h, sc_h = fl[:m].tolist(), fl[m:2 * m].tolist()
     return {"iters": it, "converged": bool(ints[1]), "diverged": bool(ints[2]), "error": ints[3],
             "history_first_iter": ks[0] if ks else 0,
-            "max_abs_F": [raw_h[k % m] for k in ks], "max_scaled_F": [sc_h[k % m] for k in ks]}
+            "max_abs_F": [raw_h[k % m] for k in ks], "max_scaled_F": [sc_h[k % m] for k in ks],
+            "init_max_abs_F": float(fl[2 * m]), "init_max_scaled_F": float(fl[2 * m + 1])}
 
 
 def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
                    max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
                    stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
-                   wait_limit_us: int = 0, carry_mode: int = 0):
-    """Newton solve; returns (S, stats) with stats a device record (see read_stats)."""
+                   wait_limit_us: int = 0, carry_mode: int = 0, init="decoupled", residual_mode="scaled"):
+    """Newton solve; returns (S, stats) with stats a device record (see read_stats).
+    With init="given", S must be passed and holds the initial guess."""
     B, T, four, d_h = P.shape
     _need(P, "P", (B, T, 4, d_h))
     _need(R, "R", (4, d_h))
     if s0 is not None:
         _need(s0, "s0", (B, 4, d_h))
     if S is None:
+        if init == "given":
+            raise ValueError("init='given' needs S holding the initial guess")
         S = torch.empty_like(P)
     _need(S, "S", (B, T, 4, d_h))
     if stats is None:
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
-    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
-                       int(wait_limit_us), int(carry_mode))
+    cfg = newton_config(max_iters, fixed, tol, forget, debug_fault, wait_limit_us, carry_mode, init, residual_mode)
     check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
                                                               ctypes.byref(cfg), _ptr(stats), B, T, d_h,
                                                               _ptr(ws), ws.numel(), _stream()))
@@ -224,7 +240,7 @@ def _need_cu(cu: torch.Tensor, n_seq: int):
 def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu_seqlens: torch.Tensor, *,
                           forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
                           S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None,
-                          carry_mode: int = 0):
+                          carry_mode: int = 0, init="decoupled", residual_mode="scaled"):
     """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
     cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats)."""
     total_T, four, d_h = P.shape
@@ -241,7 +257,7 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
-    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0, int(carry_mode))
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode)
     check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
         _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
         _ptr(ws), ws.numel(), _stream()))
@@ -301,7 +317,8 @@ def block_workspace(B: int, T: int, d_model: int, d_ff: int, device=None) -> tor
 
 def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sigmoid", max_iters: int = 8,
                   fixed: bool = False, tol: float = 1e-5, eps: float = 1e-6, y: torch.Tensor = None,
-                  S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None, carry_mode: int = 0):
+                  S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None, carry_mode: int = 0,
+                  init="decoupled", residual_mode="scaled"):
     """The trunk layer's forward; returns (y, S, stats).  x (B, T, d_model)
     fp32; Wx, W_gu (interleave_gate_up), W_down bf16."""
     B, T, D = x.shape
@@ -324,7 +341,7 @@ def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sig
         stats = new_stats(x.device)
     if ws is None:
         ws = block_workspace(B, T, D, F, x.device)
-    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), 0, 0, int(carry_mode))
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode)
     check("slstm_block_forward", load().slstm_block_forward(
         _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(y),
         _ptr(S), ctypes.byref(cfg), _ptr(stats), B, T, D, F, float(eps), _ptr(ws), ws.numel(), _stream()))

@@ -72,6 +72,9 @@ struct Args {
     unsigned epoch;
     unsigned long long wait_ns;
     int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
+    int k0;             // launches before the first Newton iteration (the guess): 0 or 1
+    int resid_raw;      // stopping test on max|F| (else on the scaled residual)
+    int guess_tested;   // the guess launch evaluated and recorded its own residual
     float tol;
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
@@ -246,6 +249,8 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo 
     }
 }
 
+// Last CTA of launch k: records the residual of Newton iteration n = k - k0
+// and decides whether the solve goes on.
 __device__ void finalize(const Args &a, int k, bool resid)
 {
     NewtonCtrl *c = a.ctrl;
@@ -254,7 +259,8 @@ __device__ void finalize(const Args &a, int k, bool resid)
     const float raw = __uint_as_float(atomicOr(&s.maxF_raw, 0u));
     const float sc = __uint_as_float(atomicOr(&s.maxF_scaled, 0u));
     const unsigned err = atomicOr(&c->error, 0u);
-    const bool last = (k + 1 == a.max_iters);
+    const int n = k - a.k0;
+    const bool last = (n + 1 == a.max_iters);
     // the next iteration starts from a clean slot (its previous user,
     // iteration k - 1, finished before this launch began)
     NewtonSlot &nx = c->slot[(k + 1) & 1];
@@ -262,9 +268,14 @@ __device__ void finalize(const Args &a, int k, bool resid)
     nx.finished = 0u;
     nx.maxF_raw = 0u;
     nx.maxF_scaled = 0u;
-    st->iters = k + 1;
-    st->max_abs_F[k % SLSTM_STATS_HISTORY] = resid ? raw : -1.0f;
-    st->max_scaled_F[k % SLSTM_STATS_HISTORY] = resid ? sc : -1.0f;
+    st->iters = n + 1;
+    st->max_abs_F[n % SLSTM_STATS_HISTORY] = resid ? raw : -1.0f;
+    st->max_scaled_F[n % SLSTM_STATS_HISTORY] = resid ? sc : -1.0f;
+    if (n == 0 && !a.guess_tested) {
+        st->init_max_abs_F = -1.0f;
+        st->init_max_scaled_F = -1.0f;
+    }
+    const float test = a.resid_raw ? raw : sc;
     bool done = last;
     if (err) {
         st->error = SLSTM_ERR_TIMEOUT;
@@ -275,7 +286,7 @@ __device__ void finalize(const Args &a, int k, bool resid)
             st->diverged = 1;
             st->error = SLSTM_ERR_DIVERGED;
             done = true;
-        } else if (sc <= a.tol && (!a.fixed || last)) {
+        } else if (test <= a.tol && (!a.fixed || last)) {
             st->converged = 1;
             done = done || !a.fixed;
         } else if (last && raw > 1.0f) {
@@ -285,6 +296,485 @@ __device__ void finalize(const Args &a, int k, bool resid)
     }
     __threadfence();
     if (done) atomicExch(&c->done, 1u);
+}
+
+// ---- the decoupled initial guess --------------------------------------------
+// The default initial guess is the trajectory of the cell with its gates
+// blind to h_{t-1} (R taken as 0): z, o, log i and log f then depend on P
+// alone and only c, n, m recur.  In unstabilised form (C, N) = (c, n) e^m that
+// recurrence is linear, C_t = f_t C_{t-1} + i_t z_t, so a run of steps maps
+// (C, N) to e^A (C, N) + e^mu (u, v) with A = sum log f, and the guess is an
+// associative scan over such runs, kept stabilised: the run is stored as
+// (A, mu, u, v) with mu the largest exponent of its own inputs.  The launch
+// has the Newton iteration's tiles, tickets and look-back, with five floats
+// per run instead of a 4x4 affine map, reads P and writes S (and the tile
+// boundary states the first Newton iteration reads).
+
+// A run of steps.  head: the run contains a sequence start, so its result
+// ignores what enters it; (mu, u, v) then hold the state (m, c, n) at its
+// end and A is unused.
+struct Seg {
+    float A, mu, u, v;
+    float o;      // output gate of the run's last step (h = o c / n there)
+    bool head;
+};
+
+// (m, c, n) <- the run (A, mu, u, v) applied to the state (m, c, n):
+//   m' = max(A + m, mu),  (c', n') = e^{A + m - m'} (c, n) + e^{mu - m'} (u, v).
+// With (A, mu, u, v) = (log f_t, log i_t, z_t, 1) this is one step of the cell
+// with R = 0, ties going to the forget branch as in the cell.
+SLSTM_DEVINL void seg_apply(float A, float mu, float u, float v, float &m, float &c, float &n)
+{
+    const float x = A + m;
+    const bool fb = x >= mu;
+    const float e = __expf(-fabsf(x - mu));
+    const float f1 = fb ? 1.0f : e;
+    const float f2 = fb ? e : 1.0f;
+    m = fb ? x : mu;
+    c = fmaf(f1, c, f2 * u);
+    n = fmaf(f1, n, f2 * v);
+}
+
+// out = second o first (the run `first`, then the run `second`).
+SLSTM_DEVINL void seg_compose(const Seg &second, const Seg &first, Seg &out)
+{
+    if (second.head) {
+        out = second;
+        return;
+    }
+    Seg r = first;
+    seg_apply(second.A, second.mu, second.u, second.v, r.mu, r.u, r.v);
+    r.A = first.A + second.A;
+    r.o = second.o;
+    out = r;
+}
+
+// h = o c / n, written the same way wherever the guess forms it.
+SLSTM_DEVINL float guess_h(float o, float c, float n) { return o * (c * __fdividef(1.0f, n)); }
+
+// Gates of one step with R = 0.
+template <int FORGET>
+SLSTM_DEVINL void guess_gates(float pz, float pf, float po, float &z, float &lf, float &o)
+{
+    z = tanh_fast(pz);
+    o = sigmoid_fast(po);
+    if (FORGET == SLSTM_FORGET_EXP) {
+        lf = pf;
+    } else {
+        lf = fminf(pf, 0.0f) - __logf(1.0f + __expf(-fabsf(pf)));
+    }
+}
+
+struct GuessSmem {
+    float P[2][TT][4][32];   // stage s: rows (step, slot) of 32 features; TMA boxes land here
+    float O[TT][4][32];      // TMA path: S of the tile, source of the warps' TMA stores
+    float R[2][4][32];       // TMA path: the tile's recurrent weights (gate-major)
+    float seg[NW][5][32];    // each warp's run: A, mu, u, v, o
+    float cin[NW][4][32];    // state (c, n, m, h) entering each warp
+    TileInfo info[3];
+    uint64_t bar[2];
+    float red[2][NW];
+    unsigned whead;
+    int exit_flag;
+};
+constexpr size_t GUESS_SMEM_BYTES = sizeof(GuessSmem) + 1024;
+
+SLSTM_DEVINL void guess_issue_load(const Args &a, const NewtonMaps &m, GuessSmem &sm, int st, const TileInfo &ti)
+{
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const uint32_t rbytes = 4u * (uint32_t)min(32, a.d - ti.j0);   // a multiple of 16 (d % 4 == 0)
+    mbar_expect_tx(&sm.bar[st], (uint32_t)sizeof(sm.P[0]) + 4u * rbytes);
+    tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, ti.chunk * TT * 4, ti.b);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+}
+
+// cp.async path: 4-byte copies, lane = feature; rows past T and features
+// past d arrive as zeros.
+SLSTM_DEVINL void guess_prefetch(const Args &a, GuessSmem &sm, int st, const TileInfo &ti)
+{
+    if (ti.ticket >= (unsigned)a.n_tiles) return;
+    const int w = threadIdx.x >> 5, jl = threadIdx.x & 31;
+    const bool fj = ti.j0 + jl < a.d;
+    const float *p = a.P + ti.off + (size_t)w * a.d + jl;
+    const size_t roww = (size_t)NW * a.d;
+    const int t0 = ti.chunk * TT;
+#pragma unroll 4
+    for (int r = 0; r < 4 * L; ++r) {
+        const int rs = r * NW + w;
+        const int step = rs >> 2, slot = rs & 3;
+        const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+        cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * roww : a.P, bytes);
+    }
+}
+
+// The guess's look-back when the predecessor's state is not published yet
+// (warp 0, lane = feature, chunk > 0): publishes this tile's run, then
+// composes the runs of unfinished predecessors until it meets a published
+// state.  Returns the state (c, n, m, h) entering the tile in v.
+SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket, int chunk, int grp, float v[4])
+{
+    const int lane = threadIdx.x & 31;
+    {
+        float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
+        dst[0] = tile.A;
+        dst[32] = tile.mu;
+        dst[64] = tile.u;
+        dst[96] = tile.v;
+        dst[128] = tile.o;
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release(a.flags + ticket, (a.epoch << 2) | FLAG_AGG | (tile.head ? FLAG_HEAD : 0u));
+    }
+    Seg M;            // composition of the runs met so far (latest last)
+    bool have = false;
+    int q = chunk - 1;
+    const uint64_t t0 = globaltimer_ns();
+    unsigned polls = 0;
+    const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+    for (;;) {
+        const unsigned tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
+        float w[4];
+        if (__all_sync(0xffffffffu, read_inc_words(ca, tq, lane, w))) {
+            if (have) {
+                seg_apply(M.A, M.mu, M.u, M.v, w[2], w[0], w[1]);
+                w[3] = guess_h(M.o, w[0], w[1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = w[e];
+            return;
+        }
+        const unsigned f = ld_acquire(a.flags + tq);
+        if ((f >> 2) == a.epoch && (f & FLAG_AGG)) {
+            const float *src = a.agg + (size_t)tq * 20 * 32 + lane;
+            Seg x;
+            x.A = __ldcg(src);
+            x.mu = __ldcg(src + 32);
+            x.u = __ldcg(src + 64);
+            x.v = __ldcg(src + 96);
+            x.o = __ldcg(src + 128);
+            x.head = (f & FLAG_HEAD) != 0u;
+            if (have) seg_compose(M, x, M);
+            else M = x;
+            have = true;
+            if (M.head) {
+                // a sequence starts inside: the state is the run's own end
+                v[0] = M.u;
+                v[1] = M.v;
+                v[2] = M.mu;
+                v[3] = guess_h(M.o, M.u, M.v);
+                return;
+            }
+            --q;   // chunk 0 never publishes a run, so q stays >= 0
+            continue;
+        }
+        if (++polls > 16) __nanosleep(64);
+        if (globaltimer_ns() - t0 > a.wait_ns) {
+            atomicOr(a.error, 1u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = 0.f;
+            return;
+        }
+    }
+}
+
+// The guess: one launch over every tile.  RESID: also evaluate the guess's
+// residual with the true R (tolerance mode), recorded as the initial
+// residual; a guess that meets the test ends the solve.
+template <int FORGET, bool RESID, bool TMA, bool VARLEN>
+__global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_constant__ NewtonMaps maps)
+{
+    extern __shared__ unsigned char smem_raw[];
+    GuessSmem &sm = *reinterpret_cast<GuessSmem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    NewtonSlot &slot = a.ctrl->slot[0];
+
+    if (threadIdx.x == 0) {
+        sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
+        if (!sm.exit_flag) {
+            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[0]);
+            decode_tile(a, atomicAdd(&slot.ticket, 1u), sm.info[1]);
+        }
+    }
+    if (TMA && threadIdx.x == 0) {
+        mbar_init(&sm.bar[0], 1);
+        mbar_init(&sm.bar[1], 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    if (sm.exit_flag) return;
+
+    const size_t d = (size_t)a.d;
+    const int T = a.T;
+    const unsigned G = (unsigned)a.n_groups;
+    float mx_raw = 0.f, mx_sc = 0.f;
+    int ring = 0, st = 0;
+    unsigned it = 0;
+    bool tma_ok = true;
+    if (TMA) {
+        if (threadIdx.x == 0) guess_issue_load(a, maps, sm, 0, sm.info[0]);
+    } else {
+        guess_prefetch(a, sm, 0, sm.info[0]);
+        cp_async_commit();
+    }
+
+    for (;;) {
+        const TileInfo ti = sm.info[ring];
+        if (ti.ticket >= (unsigned)a.n_tiles) break;
+        const int rn = ring == 2 ? 0 : ring + 1;
+        unsigned after = 0;
+        if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
+        if (TMA) {
+            if (threadIdx.x == 32) guess_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
+            if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS)) {
+                atomicOr(a.error, 2u);
+                (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS);
+                tma_ok = false;
+            }
+        } else {
+            guess_prefetch(a, sm, st ^ 1, sm.info[rn]);
+            cp_async_commit();
+            cp_async_wait_prev();
+            __syncthreads();
+        }
+
+        const unsigned ticket = ti.ticket;
+        const int chunk = ti.chunk;
+        const bool jv = ti.j0 + lane < a.d;
+        const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
+        const int t_seg = chunk * TT + warp * L;
+
+        // ---- walk A: this warp's run, lane = feature ----
+        float gz[L], glf[L], go[L], gi[L];
+        Seg run;
+        {
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int sl = warp * L + i;
+                guess_gates<FORGET>(sm.P[st][sl][0][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], gz[i],
+                                    glf[i], go[i]);
+                gi[i] = sm.P[st][sl][1][lane];
+                const bool head = VARLEN && ((ti.mask >> sl) & 1ull);
+                if (head) {
+                    float s0v[4];
+                    head_state(a, t_seg + i, jj, jv, s0v);
+                    run.mu = s0v[2];
+                    run.u = s0v[0];
+                    run.v = s0v[1];
+                    seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
+                    run.head = true;
+                } else if (i == 0) {
+                    run.A = glf[i];
+                    run.mu = gi[i];
+                    run.u = gz[i];
+                    run.v = 1.0f;
+                    run.head = false;
+                } else {
+                    seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
+                    run.A += glf[i];
+                }
+                run.o = go[i];
+            }
+            sm.seg[warp][0][lane] = run.A;
+            sm.seg[warp][1][lane] = run.mu;
+            sm.seg[warp][2][lane] = run.u;
+            sm.seg[warp][3][lane] = run.v;
+            sm.seg[warp][4][lane] = run.o;
+        }
+        if (VARLEN && threadIdx.x == 0) {
+            unsigned wh = 0u;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) wh |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
+            sm.whead = wh;
+        }
+        __syncthreads();
+
+        // ---- carry: warp 0 walks the runs; warp w goes on once its state is stored ----
+        if (warp == 0) {
+            const unsigned whead = VARLEN ? sm.whead : 0u;
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            if (chunk == 0) {
+                if (!VARLEN && a.s0 && jv) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
+                }
+            } else {
+                const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                const bool ok = read_inc_words(ca, ticket - G, lane, v);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    Seg tile;
+#pragma unroll 1
+                    for (int w = 0; w < NW; ++w) {
+                        Seg x;
+                        x.A = sm.seg[w][0][lane];
+                        x.mu = sm.seg[w][1][lane];
+                        x.u = sm.seg[w][2][lane];
+                        x.v = sm.seg[w][3][lane];
+                        x.o = sm.seg[w][4][lane];
+                        x.head = ((whead >> w) & 1u) != 0u;
+                        if (w == 0) tile = x;
+                        else seg_compose(x, tile, tile);
+                    }
+                    guess_lookback(a, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
+                }
+            }
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sm.cin[w][e][lane] = v[e];
+                if (w > 0) named_bar_arrive(w, 2 * 32);
+                if ((whead >> w) & 1u) {
+                    v[0] = sm.seg[w][2][lane];
+                    v[1] = sm.seg[w][3][lane];
+                    v[2] = sm.seg[w][1][lane];
+                } else {
+                    seg_apply(sm.seg[w][0][lane], sm.seg[w][1][lane], sm.seg[w][2][lane], sm.seg[w][3][lane], v[2],
+                              v[0], v[1]);
+                }
+                v[3] = guess_h(sm.seg[w][4][lane], v[0], v[1]);
+            }
+            unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, v[e]));
+        } else {
+            named_bar_sync(warp, 2 * 32);   // the state entering this warp is stored
+        }
+
+        // ---- walk B: replay the steps from the entering state ----
+        if (TMA) {
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        }
+        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
+        if (RESID && jv) {
+            if (TMA) {
+                rz = sm.R[st][0][lane];
+                ri = sm.R[st][1][lane];
+                rf = sm.R[st][2][lane];
+                ro = sm.R[st][3][lane];
+            } else {
+                rz = __ldg(a.R + jj);
+                ri = __ldg(a.R + d + jj);
+                rf = __ldg(a.R + 2 * d + jj);
+                ro = __ldg(a.R + 3 * d + jj);
+            }
+        }
+        float sv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sv[e] = sm.cin[warp][e][lane];
+        float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
+#pragma unroll
+        for (int i = 0; i < L; ++i) {
+            const int sl = warp * L + i;
+            const bool wr = jv && (t_seg + i < T);
+            if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, sv);
+            const float prev[4] = {sv[0], sv[1], sv[2], sv[3]};
+            seg_apply(glf[i], gi[i], gz[i], 1.0f, sv[2], sv[0], sv[1]);
+            sv[3] = guess_h(go[i], sv[0], sv[1]);
+            if (TMA) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sv[e];
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (wr) srow[(size_t)i * 4 * d + e * d] = sv[e];
+            }
+            if (RESID) {
+                Cell f;
+                cell_eval<FORGET, false>(prev[0], prev[1], prev[2], prev[3], sm.P[st][sl][0][lane], gi[i],
+                                         sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri, rf, ro, f);
+                const float F[4] = {sv[0] - f.c, sv[1] - f.n, sv[2] - f.m, sv[3] - f.h};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float af = wr ? fabsf(F[e]) : 0.0f;
+                    mx_raw = fmax_nan(mx_raw, af);
+                    mx_sc = fmax_nan(mx_sc, __fdividef(af, 1.0f + fabsf(sv[e])));
+                }
+            }
+        }
+        if (TMA) {
+            tma_store_fence();
+            __syncwarp();
+            if (lane == 0 && t_seg < T) {
+                tma_store_3d(&maps.Sw, &sm.O[warp * L][0][0], ti.j0, t_seg * 4, ti.b);
+                bulk_commit();
+            }
+        }
+        // state at the tile's last step, read by the first Newton iteration
+        if (warp == NW - 1 && t_seg + L - 1 < T) {
+            float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = sv[e];
+        }
+        if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
+        __syncthreads();   // this stage is free for the loads of the tile after next
+        ring = rn;
+        st ^= 1;
+        ++it;
+    }
+    if (TMA) {
+        if (lane == 0) bulk_wait_all();
+    } else {
+        cp_async_wait_all();
+    }
+    if (!RESID) return;
+    mx_raw = warp_max(mx_raw);
+    mx_sc = warp_max(mx_sc);
+    if (lane == 0) {
+        sm.red[0][warp] = mx_raw;
+        sm.red[1][warp] = mx_sc;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float r0 = sm.red[0][0], r1 = sm.red[1][0];
+        for (int w = 1; w < NW; ++w) {
+            r0 = (__float_as_uint(sm.red[0][w]) > __float_as_uint(r0)) ? sm.red[0][w] : r0;
+            r1 = (__float_as_uint(sm.red[1][w]) > __float_as_uint(r1)) ? sm.red[1][w] : r1;
+        }
+        atomic_max_nonneg(&slot.maxF_raw, r0);
+        atomic_max_nonneg(&slot.maxF_scaled, r1);
+        __threadfence();
+        const unsigned fin = atomicAdd(&slot.finished, 1u);
+        if (fin == gridDim.x - 1u) {
+            __threadfence();
+            const float raw = __uint_as_float(atomicOr(&slot.maxF_raw, 0u));
+            const float sc = __uint_as_float(atomicOr(&slot.maxF_scaled, 0u));
+            slstm_newton_stats *stt = a.stats;
+            stt->init_max_abs_F = raw;
+            stt->init_max_scaled_F = sc;
+            const unsigned err = atomicOr(a.error, 0u);
+            const float test = a.resid_raw ? raw : sc;
+            if (err) {
+                stt->error = SLSTM_ERR_TIMEOUT;
+                __threadfence();
+                atomicExch(&a.ctrl->done, 1u);
+            } else if (raw <= FLT_MAX && sc <= FLT_MAX && test <= a.tol) {
+                stt->converged = 1;
+                __threadfence();
+                atomicExch(&a.ctrl->done, 1u);
+            }
+        }
+    }
+}
+
+// Caller-given guess: the state at the last step of every tile that has a
+// successor, in the boundary layout the first Newton iteration reads
+// ([tile][slot][32 features]).
+__global__ void gather_boundaries(Args a)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)a.n_tiles * 128) return;
+    const unsigned tile = (unsigned)(idx >> 7);
+    const int e = (int)((idx >> 5) & 3), lane = (int)(idx & 31);
+    const unsigned chunk = tile / (unsigned)a.n_groups;
+    const unsigned grp = tile - chunk * (unsigned)a.n_groups;
+    const unsigned b = grp / (unsigned)a.groups_per_row;
+    const int j = (int)(grp - b * (unsigned)a.groups_per_row) * 32 + lane;
+    const long long t = (long long)chunk * TT + TT - 1;
+    float v = 0.0f;
+    if (t < a.T && j < a.d) v = a.S[(((size_t)b * a.T + (size_t)t) * 4 + e) * (size_t)a.d + j];
+    a.bnd_out[idx] = v;
 }
 
 // TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
@@ -497,7 +987,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                     c = __uint_as_float((unsigned)w2);
                 }
             }
-            const bool withhold = (k == 0) && ((int)ticket == a.fault_ticket);
+            const bool withhold = (k == a.k0) && ((int)ticket == a.fault_ticket);
             const bool fast = __syncthreads_and(ok);
             if (chain_warp) {
                 if (fast) {
@@ -667,16 +1157,47 @@ cudaError_t launch_pass(const Args &a, const NewtonMaps &m, int k, bool resid, i
                  : launch_one<FORGET, false, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
 }
 
+template <int FORGET, bool RESID, bool TMA, bool VARLEN>
+cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int sms, cudaStream_t st)
+{
+    auto kern = guess_kernel<FORGET, RESID, TMA, VARLEN>;
+    static bool ready = false;
+    if (!ready) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GUESS_SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        ready = true;
+    }
+    kern<<<min(a.n_tiles, sms), NW * 32, GUESS_SMEM_BYTES, st>>>(a, m);
+    return cudaGetLastError();
+}
+
+// The launches of one solve: the initial guess as launch 0 (decoupled: the
+// guess kernel; given: the boundary gather), then Newton iterations
+// k = k0 .. k0 + max_iters - 1.  Launch k has epoch k + 1 and writes the
+// boundary buffer that launch k + 1 reads.
 template <int FORGET, bool TMA, bool VARLEN>
 cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
-                         cudaStream_t st)
+                         int init, cudaStream_t st)
 {
-    for (int k = 0; k < max_iters; ++k) {
+    if (init == SLSTM_INIT_DECOUPLED) {
+        Args a = base;
+        a.epoch = 1u;
+        const cudaError_t e = fixed ? launch_guess<FORGET, false, TMA, VARLEN>(a, m, sms, st)
+                                    : launch_guess<FORGET, true, TMA, VARLEN>(a, m, sms, st);
+        if (e != cudaSuccess) return e;
+    } else if (init == SLSTM_INIT_GIVEN) {
+        const long long n = (long long)base.n_tiles * 128;
+        gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(base);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    for (int k = base.k0; k < base.k0 + max_iters; ++k) {
         Args a = base;
         a.epoch = (unsigned)(k + 1);
         a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
         a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
-        const bool resid = !fixed || (k + 1 == max_iters);
+        const bool resid = !fixed || (k + 1 - base.k0 == max_iters);
         cudaError_t e;
         if (two_pass) {
             if ((e = launch_pass<FORGET, TMA, VARLEN, MODE_AGG>(a, m, k, false, sms, st)) != cudaSuccess) return e;
@@ -740,10 +1261,10 @@ int sm_count()
 
 template <int FORGET, bool TMA>
 cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
-                             bool varlen, cudaStream_t st)
+                             bool varlen, int init, cudaStream_t st)
 {
-    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, two_pass, sms, st)
-                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, two_pass, sms, st);
+    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, two_pass, sms, init, st)
+                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, two_pass, sms, init, st);
 }
 
 }  // namespace
@@ -786,6 +1307,9 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     a.max_iters = cfg.max_iters;
     a.fixed = cfg.fixed_iters ? 1 : 0;
     a.tol = cfg.tol;
+    a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : 1;
+    a.resid_raw = cfg.residual_mode == SLSTM_RESIDUAL_RAW ? 1 : 0;
+    a.guess_tested = (cfg.init == SLSTM_INIT_DECOUPLED && !a.fixed) ? 1 : 0;
     a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(P) & 15) == 0 &&
                (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
     // fault injection: the first tile of chunk 1 withholds its publications,
@@ -822,11 +1346,14 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     const bool two_pass = cfg.carry_mode == SLSTM_CARRY_TWO_PASS ||
                           (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 &&
                            prefer_two_pass(l.n_groups, (long long)l.n_chunks * TT, sms));
+    const int init = cfg.init;
     if (cfg.forget == SLSTM_FORGET_EXP)
-        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st)
-                   : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st);
-    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st)
-               : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, st);
+        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
+                   : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
+                                                               st);
+    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
+               : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
+                                                               st);
 }
 
 }  // namespace slstm

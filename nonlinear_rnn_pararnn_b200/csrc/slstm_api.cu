@@ -48,6 +48,8 @@ bool config_ok(const slstm_newton_config &c)
     if (c.max_iters < 1 || c.max_iters > SLSTM_MAX_ITERS) return false;
     if (c.forget != SLSTM_FORGET_SIGMOID && c.forget != SLSTM_FORGET_EXP) return false;
     if (!(c.tol >= 0.0f) || c.wait_limit_us < 0) return false;
+    if (c.init < SLSTM_INIT_DECOUPLED || c.init > SLSTM_INIT_GIVEN) return false;
+    if (c.residual_mode != SLSTM_RESIDUAL_SCALED && c.residual_mode != SLSTM_RESIDUAL_RAW) return false;
     return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
 }
 

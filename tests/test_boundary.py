@@ -64,7 +64,8 @@ def test_workspace_sizes():
 
 
 def _cfg(**kw):
-    base = dict(max_iters=4, fixed_iters=0, tol=1e-5, forget=0, debug_fault=0, wait_limit_us=0, carry_mode=0)
+    base = dict(max_iters=4, fixed_iters=0, tol=1e-5, forget=0, debug_fault=0, wait_limit_us=0, carry_mode=0,
+                init=0, residual_mode=0)
     base.update(kw)
     return _lib.NewtonConfig(**base)
 
@@ -92,6 +93,9 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(cfg=_cfg(tol=float("nan"))) == E
     assert call(cfg=_cfg(carry_mode=3)) == E
     assert call(cfg=_cfg(carry_mode=-1)) == E
+    assert call(cfg=_cfg(init=3)) == E
+    assert call(cfg=_cfg(init=-1)) == E
+    assert call(cfg=_cfg(residual_mode=2)) == E
     assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
     assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
     assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E

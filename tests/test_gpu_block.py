@@ -45,10 +45,8 @@ def _run(p, forget, y=None, x_override=None):
     return api.block_forward(x, w1, Wx, bias, R, w2, W_gu, Wd, forget=forget, max_iters=64, tol=1e-6, y=y)
 
 
-# Newton from the zero guess needs short sequences to converge in fp32 with the
-# exponential forget gate (its first iterates overflow on longer ones, as in
-# the cell's own tests), so that case is 8 steps long
 @pytest.mark.parametrize("B,T,D,F,forget", [(2, 64, 64, 256, "sigmoid"), (2, 8, 96, 384, "exp"),
+                                            (2, 300, 96, 384, "exp"), (2, 700, 64, 256, "sigmoid"),
                                             (3, 40, 136, 544, "sigmoid"), (1, 33, 264, 1056, "sigmoid"),
                                             (3, 60, 64, 256, "sigmoid")])
 def test_block_forward_matches_oracle(B, T, D, F, forget, cuda_device):

@@ -35,8 +35,8 @@ def _capture(step):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_training_step_replays_under_cuda_graph(dtype, cuda_device):
-    # solved to convergence (a fixed-K iterate from the zero guess is far from
-    # the solution and amplifies rounding differences)
+    # solved to convergence, so that replay and eager runs are compared on the
+    # solution
     w = Workload("graph", 2, 64, 32, 64, dtype, "sigmoid", 0.5, 91, 1e-6, 64)
     inp = make_inputs(w)
     x, Wx, R, bias, s0, dH = (inp[k].cuda() for k in ("x", "Wx", "R", "bias", "s0", "dH"))

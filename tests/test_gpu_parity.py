@@ -92,15 +92,17 @@ def test_preact_gemm_matches_oracle(dtype, B, T, d_in, d_h, cuda_device):
 CARRY_MODES = [1, 2]
 
 
-def _newton_case(w: Workload, fixed_k=None, carry_mode=0):
+def _newton_case(w: Workload, fixed_k=None, carry_mode=0, init="decoupled", residual_mode="scaled"):
     inp = make_inputs(w, with_dH=False)
     Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
     if fixed_k is None:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
-                                   max_iters=w.max_iters, fixed=False, tol=w.tol, carry_mode=carry_mode)
+                                   max_iters=w.max_iters, fixed=False, tol=w.tol, carry_mode=carry_mode,
+                                   init=init, residual_mode=residual_mode)
     else:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
-                                   max_iters=fixed_k, fixed=True, tol=w.tol, carry_mode=carry_mode)
+                                   max_iters=fixed_k, fixed=True, tol=w.tol, carry_mode=carry_mode, init=init,
+                                   residual_mode=residual_mode)
     stats = api.read_stats(st)
     Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
     return inp, as_f64(S.cpu()), stats, Pref
@@ -110,7 +112,7 @@ def _check_status_against_oracle(st, ost):
     """A GPU run either converges (and then the fp64 run converged too) or it
     stops on a non-finite or large residual; in that case the exact-arithmetic
     iterate at the same iteration was also far from converged (scaled
-    residual > 1), so the stop is the method's behaviour from the zero guess,
+    residual > 1), so the stop is the method's behaviour from that guess,
     not an artefact of the kernels."""
     if st["converged"]:
         assert ost["converged"], (st, ost)
@@ -132,8 +134,10 @@ def test_newton_tiny_converges_to_sequential(cuda_device):
     assert st["converged"]
     assert abs(st["iters"] - ost["iters"]) <= 1
     assert _h_err(S, ref) <= TOL_F32
-    # the residual history of the first iterates agrees with the fp64 run
-    for k in range(3):
+    # the residual of the guess and of the first iterates agrees with the fp64 run
+    g, o = st["init_max_scaled_F"], ost["init_max_scaled_F"]
+    assert abs(g - o) <= 1e-3 * (1 + o), (g, o)
+    for k in range(min(2, len(st["max_scaled_F"]), len(ost["max_scaled_F"]))):
         g, o = st["max_scaled_F"][k], ost["max_scaled_F"][k]
         assert abs(g - o) <= 1e-3 * (1 + o), (k, g, o)
 
@@ -148,16 +152,115 @@ def test_newton_converges_to_sequential_sigmoid(B, T, d, carry_mode, cuda_device
     assert _h_err(S, ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("init", ["decoupled", "zero"])
 @pytest.mark.parametrize("carry_mode", CARRY_MODES)
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 @pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256), (1, 300, 36), (2, 200, 40)])
-def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, cuda_device):
+def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, init, cuda_device):
     w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
-    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode)
-    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol)
-    if _check_status_against_oracle(st, ost):
+    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode, init=init)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol,
+                                init=init)
+    converged = _check_status_against_oracle(st, ost)
+    if init == "decoupled":
+        assert converged, (st, ost["iters"])
+    if converged:
         ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget)
         assert _h_err(S, ref) <= TOL_F32
+
+
+def _s_err(S_gpu, S_ref):
+    """max over every slot of |dS| / (1 + |S|)."""
+    return float((np.abs(S_gpu - S_ref) / (1 + np.abs(S_ref))).max())
+
+
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+@pytest.mark.parametrize("B,T,d,s0_random", [(2, 50, 40, True), (1, 1, 1, False), (3, 64, 70, True),
+                                              (1, 3000, 36, True), (2, 4100, 64, False)])
+def test_newton_decoupled_guess_matches_oracle(forget, B, T, d, s0_random, carry_mode, cuda_device):
+    """The guess launch alone (its test passes at any tolerance): every slot of
+    the decoupled trajectory against the oracle's, across many tiles and the
+    look-back over up to 65 chunks of 64 steps."""
+    w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 17, 1e30, 4)
+    inp = make_inputs(w, with_dH=False)
+    s0 = inp["s0"]
+    if s0_random:
+        g = torch.Generator().manual_seed(19)
+        s0 = torch.stack([torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) + 0.5,
+                          torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) - 0.5], dim=1)
+    Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(s0), forget=forget, max_iters=4, fixed=False, tol=1e30,
+                               carry_mode=carry_mode)
+    s = api.read_stats(st)
+    assert s["iters"] == 0 and s["converged"] and s["error"] == 0, s
+    Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    Sg, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(s0), forget, 4, False, 1e30)
+    assert ost["iters"] == 0
+    assert _s_err(as_f64(S.cpu()), Sg) <= TOL_F32
+    g, o = s["init_max_scaled_F"], ost["init_max_scaled_F"]
+    assert abs(g - o) <= 1e-3 * (1 + o), (g, o)
+
+
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+@pytest.mark.parametrize("forget,T", [("sigmoid", 1024), ("exp", 512), ("sigmoid", 2500)])
+def test_newton_converges_where_zero_guess_diverges(forget, T, carry_mode, cuda_device):
+    """Lengths at which the zero guess overflows: from the decoupled guess the
+    GPU solve converges, to the sequential trajectory, in about as many
+    iterations as the fp64 run."""
+    w = Workload("t", 2, T, 16, 40, "f32", forget, 0.5, 23, 1e-5, 16)
+    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol)
+    print("gpu", st["iters"], st["max_scaled_F"], "oracle", ost["iters"], list(ost["max_scaled_F"]))
+    assert st["converged"] and st["error"] == 0, st
+    assert ost["converged"] and abs(st["iters"] - ost["iters"]) <= 1
+    ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget)
+    assert _h_err(S, ref) <= TOL_F32
+
+
+def test_newton_raw_residual_mode(cuda_device):
+    """residual_mode 'raw': the stop uses max|F| (the pages' norm); the run
+    stops where the fp64 run with the same rule stops, give or take one.  The
+    tolerance is one fp32 can reach on max|F| (the normaliser n reaches tens,
+    so |F| has a rounding floor of a few 1e-6)."""
+    w = scaled(WORKLOADS["tiny_f32"], tol=1e-4)
+    inp, S, st, Pref = _newton_case(w, residual_mode="raw")
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol,
+                                residual_mode="raw")
+    print("gpu", st, "oracle", ost)
+    assert st["converged"] and ost["converged"]
+    assert st["max_abs_F"][-1] <= w.tol
+    assert abs(st["iters"] - ost["iters"]) <= 1
+    ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
+    assert _h_err(S, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_newton_given_guess_one_iteration(forget, carry_mode, cuda_device):
+    """Warm start: S holds a guess near the solution (the sequential
+    trajectory, perturbed); one iteration from it matches the fp64 iteration
+    from the same guess at every step and slot."""
+    w = Workload("t", 3, 700, 16, 40, "f32", forget, 0.5, 29, 1e-6, 1)
+    inp = make_inputs(w, with_dH=False)
+    # both sides read the same fp32 P and guess, made on the host by the oracle
+    P32 = torch.from_numpy(oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))).float()
+    Sseq = oracle.sequential_btgd(as_f64(P32), as_f64(inp["R"]), as_f64(inp["s0"]), forget)
+    # relative noise of 1e-3 on c, n, h and absolute 1e-3 on the stabiliser m
+    u = np.random.default_rng(31).uniform(-1, 1, size=Sseq.shape)
+    g64 = Sseq * (1 + 1e-3 * u)
+    g64[:, :, 2] = Sseq[:, :, 2] + 1e-3 * u[:, :, 2]
+    guess32 = torch.from_numpy(g64).float()
+    S = _dev(guess32)
+    S, st = api.newton_forward(_dev(P32), _dev(inp["R"]), None, forget=forget, max_iters=1, fixed=True, tol=1e-6,
+                               S=S, init="given", carry_mode=carry_mode)
+    s = api.read_stats(st)
+    assert s["iters"] == 1 and s["init_max_abs_F"] == -1.0
+    So, ost = oracle.newton_btgd(as_f64(P32), as_f64(inp["R"]), as_f64(inp["s0"]), forget, 1, True, 1e-6,
+                                 init="given", S_init=as_f64(guess32))
+    assert _s_err(as_f64(S.cpu()), So) <= TOL_F32
+    g_r, o_r = s["max_abs_F"][0], ost["max_abs_F"][0]
+    assert abs(g_r - o_r) <= 1e-3 * (1 + o_r) + 1e-5, (g_r, o_r)
 
 
 @pytest.mark.parametrize("carry_mode", CARRY_MODES)

@@ -70,11 +70,13 @@ def test_varlen_fixed_k_matches_oracle(lengths, d, forget, carry_mode, cuda_devi
     torch.cuda.synchronize()
     got = as_f64(S.cpu())
     assert api.read_stats(st)["iters"] == K
-    # The iterate after K steps from the zero guess is far from the solution
-    # and amplifies rounding (as in the dense fixed-K tests, only what fp32
-    # pins is compared).  Newton's prefix exactness, per sequence: after K
-    # iterations the first K steps of every sequence are the sequential
-    # trajectory; a carry leaking across a sequence start would break it.
+    # The whole iterate after K iterations from the decoupled guess of every
+    # sequence, against the fp64 iterate of each sequence on its own.
+    ref = oracle.newton_varlen_fixed(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy(), forget, K)
+    assert float((np.abs(got - ref) / (1 + np.abs(ref))).max()) <= TOL_F32
+    # Newton's prefix exactness, per sequence: after K iterations the first K
+    # steps of every sequence are the sequential trajectory; a carry leaking
+    # across a sequence start would break it.
     seq = oracle.sequential_varlen(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy(), forget)
     cu = c["cu"].numpy()
     for k in range(len(lengths)):
@@ -104,8 +106,7 @@ def test_varlen_equal_lengths_matches_batched(cuda_device):
     c = _case([T] * B, d, 16, "f32", "sigmoid", 43)
     P, _ = _preact(c)
     R, s0 = _dev(c["R"]), _dev(c["s0"])
-    # converged solutions (fixed-K iterates amplify the different rounding
-    # order of packed and batched tiles)
+    # converged solutions (packed and batched tiles round in different orders)
     Sv, stv = api.newton_forward_varlen(P, R, s0, _dev(c["cu"]), max_iters=64, tol=1e-6)
     Sb, stb = api.newton_forward(P.view(B, T, 4, d), R, s0, max_iters=64, tol=1e-6)
     torch.cuda.synchronize()
