@@ -494,15 +494,22 @@ def head_jacobian(Jl, G, Rh):
     return J
 
 
-def newton_head(P, Rh, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5):
-    """Newton over time with dense per-head Jacobian blocks, the same update,
-    stopping rule (max |F| / (1 + |s|) <= tol) and zero initial guess as the
-    diag oracle.  Returns (S, stats)."""
+def newton_head(P, Rh, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init="decoupled"):
+    """Newton over time with dense per-head Jacobian blocks, the same update
+    and stopping rule (max |F| / (1 + |s|) <= tol) as the diag oracle.  The
+    initial guess is the decoupled trajectory (the cell with no recurrent
+    input, which does not depend on the mixing) or, with init="zero", S = 0.
+    Returns (S, stats)."""
     P, Rh = _f64(P), _f64(Rh)
     B, T, _, d = P.shape
     _, H, dh, _ = Rh.shape
     s0v = np.zeros((B, 4, d)) if s0 is None else _f64(s0)
-    S = np.zeros((B, T, 4, d))
+    if init == "decoupled":
+        S = sequential_btgd(P, np.zeros((4, d)), s0v, forget)
+    elif init == "zero":
+        S = np.zeros((B, T, 4, d))
+    else:
+        raise ValueError(f"unknown init {init!r}")
     hist = []
     conv = div = False
     it = 0
@@ -542,3 +549,48 @@ def newton_head(P, Rh, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5)
     if not conv and hist and hist[-1][0] > 1.0:
         div = True
     return S, {"iters": it, "converged": conv, "diverged": div, "max_abs_F": [h[0] for h in hist]}
+
+
+def backward_head(x, Wx, P, Rh, s0, S, dH, forget="sigmoid"):
+    """Gradients of L = sum dH * h for head mixing at the trajectory S, by the
+    reverse loop of the diag backward with the dense per-head Jacobian
+    (head_jacobian) in place of the 4x4 one:
+      lambda_t = e_h dH_t + J_{t+1}^T lambda_{t+1}
+      dP_t = G_t^T lambda_t per feature (G = d s_t / d a_t, as step() gives it)
+      dRh[g, head, i, k] = sum_{b,t} dP_t[g, (head, i)] h_{t-1}[(head, k)]
+      db = sum dP, ds0 = J_0^T lambda_0, dx = dP W_x, dW_x = dP^T x.
+    Returns dict dx, dWx, dRh (4, H, dh, dh), db (4, d), ds0 (B, 4, d), dP."""
+    P, Rh, S, dH = _f64(P), _f64(Rh), _f64(S), _f64(dH)
+    B, T, _, d = P.shape
+    _, H, dh, _ = Rh.shape
+    d_in = np.asarray(Wx).shape[1]
+    s0v = np.zeros((B, 4, d)) if s0 is None else _f64(s0)
+
+    def to_heads(v):     # (B, 4, d) -> (B, H, 4 dh), state index e * dh + i
+        return v.reshape(B, 4, H, dh).transpose(0, 2, 1, 3).reshape(B, H, 4 * dh)
+
+    def from_heads(y):
+        return y.reshape(B, H, 4, dh).transpose(0, 2, 1, 3).reshape(B, 4, d)
+
+    dP = np.zeros((B, T, 4, d))
+    dRh = np.zeros_like(Rh)
+    lam = np.zeros((B, 4, d))
+    J_next = None
+    for t in range(T - 1, -1, -1):
+        prev = s0v if t == 0 else S[:, t - 1]
+        _, Jl, G = _head_step_all(prev, P[:, t], Rh, forget)
+        lam_t = np.zeros((B, 4, d))
+        lam_t[:, 3, :] = dH[:, t]
+        if J_next is not None:
+            lam_t += from_heads(np.einsum("bhji,bhj->bhi", J_next, to_heads(lam)))
+        dp = np.einsum("bjeg,bej->bgj", G, lam_t)                 # (B, 4, d)
+        dP[:, t] = dp
+        hp = prev[:, 3, :].reshape(B, H, dh)
+        dRh += np.einsum("bghi,bhk->ghik", dp.reshape(B, 4, H, dh), hp)
+        lam = lam_t
+        J_next = head_jacobian(Jl, G, Rh)
+    ds0 = from_heads(np.einsum("bhji,bhj->bhi", J_next, to_heads(lam)))
+    dP2 = dP.reshape(B * T, 4 * d)
+    x2 = _f64(x).reshape(B * T, d_in)
+    return {"dx": (dP2 @ _f64(Wx)).reshape(B, T, d_in), "dWx": dP2.T @ x2, "dRh": dRh,
+            "db": dP.sum(axis=(0, 1)), "ds0": ds0, "dP": dP}

@@ -694,3 +694,79 @@ def test_head_newton_prefix_exact_and_converges():
     S, st = oracle.newton_head(P, Rh, s0, max_iters=20, tol=1e-12)
     assert st["converged"] and not st["diverged"]
     np.testing.assert_allclose(S, ref, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("init", ["decoupled", "zero"])
+def test_head_newton_from_either_guess(init):
+    """Prefix exactness and convergence hold from both initial guesses; the
+    decoupled guess is the diag cell's R = 0 trajectory whatever the mixing."""
+    P, Rh, s0 = _head_case(T=9, seed=8)
+    ref = oracle.sequential_head(P, Rh, s0)
+    S1, _ = oracle.newton_head(P, Rh, s0, max_iters=1, fixed=True, init=init)
+    np.testing.assert_allclose(S1[:, :1], ref[:, :1], rtol=1e-12, atol=1e-12)
+    S, st = oracle.newton_head(P, Rh, s0, max_iters=30, tol=1e-12, init=init)
+    assert st["converged"]
+    np.testing.assert_allclose(S, ref, rtol=1e-10, atol=1e-10)
+
+
+def _head_grad_case(B=2, T=5, H=2, dh=3, d_in=4, seed=12):
+    rng = np.random.default_rng(seed)
+    d = H * dh
+    x = rng.standard_normal((B, T, d_in))
+    Wx = rng.standard_normal((4 * d, d_in)) / math.sqrt(d_in)
+    bias = np.zeros((4, d))
+    bias[2] = np.linspace(3, 6, d)
+    Rh = rng.uniform(-0.4, 0.4, (4, H, dh, dh))
+    s0 = np.stack([rng.standard_normal((B, d)), rng.uniform(0.5, 1.5, (B, d)), rng.standard_normal((B, d)),
+                   rng.uniform(-0.5, 0.5, (B, d))], axis=1)
+    dH = rng.standard_normal((B, T, d))
+    return x, Wx, bias, Rh, s0, dH
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_head_backward_matches_finite_differences(forget):
+    """Every gradient of L = sum dH * h for head mixing against central
+    differences of the sequential head recurrence (step 1e-6)."""
+    x, Wx, bias, Rh, s0, dH = _head_grad_case()
+
+    def loss(x, Wx, bias, Rh, s0):
+        P_ = oracle.preact(x, Wx, bias)
+        return float((oracle.sequential_head(P_, Rh, s0, forget)[:, :, 3, :] * dH).sum())
+
+    P = oracle.preact(x, Wx, bias)
+    S = oracle.sequential_head(P, Rh, s0, forget)
+    g = oracle.backward_head(x, Wx, P, Rh, s0, S, dH, forget)
+    eps = 1e-6
+    args = {"x": x, "Wx": Wx, "bias": bias, "Rh": Rh, "s0": s0}
+    names = {"x": "dx", "Wx": "dWx", "bias": "db", "Rh": "dRh", "s0": "ds0"}
+    rng = np.random.default_rng(3)
+    for k, gname in names.items():
+        a = args[k]
+        idx = [tuple(rng.integers(0, n) for n in a.shape) for _ in range(6)]
+        for ix in idx:
+            ap, am = a.copy(), a.copy()
+            ap[ix] += eps
+            am[ix] -= eps
+            fp = loss(**{**args, k: ap})
+            fm = loss(**{**args, k: am})
+            fd = (fp - fm) / (2 * eps)
+            got = g[gname][ix]
+            assert abs(got - fd) <= 1e-6 * (1 + abs(fd)), (k, ix, got, fd)
+
+
+def test_head_backward_with_diagonal_blocks_is_the_diag_backward():
+    x, Wx, bias, Rh, s0, dH = _head_grad_case(seed=14)
+    _, H, dh, _ = Rh.shape
+    Rdiag = np.zeros_like(Rh)
+    for g_ in range(4):
+        for h_ in range(H):
+            Rdiag[g_, h_] = np.diag(np.diag(Rh[g_, h_]))
+    r = np.stack([np.concatenate([np.diag(Rh[g_, h_]) for h_ in range(H)]) for g_ in range(4)])
+    P = oracle.preact(x, Wx, bias)
+    S = oracle.sequential_btgd(P, r, s0, "sigmoid")
+    gh = oracle.backward_head(x, Wx, P, Rdiag, s0, S, dH, "sigmoid")
+    gd = oracle.backward_btgd(x, Wx, P, r, s0, S, dH, "sigmoid")
+    for k in ("dx", "dWx", "db", "ds0", "dP"):
+        np.testing.assert_allclose(gh[k], gd[k], rtol=1e-12, atol=1e-12)
+    dR_diag = np.stack([np.concatenate([np.diag(gh["dRh"][g_, h_]) for h_ in range(H)]) for g_ in range(4)])
+    np.testing.assert_allclose(dR_diag, gd["dR"], rtol=1e-12, atol=1e-12)
