@@ -53,7 +53,7 @@ def _load():
         lib.oracle_sequential.argtypes = [I, I, D, D, D, I, D]
         lib.oracle_sequential_unstabilised.argtypes = [I, I, D, D, D, I, D, D, D]
         lib.oracle_affine_solve.argtypes = [I, I, D, D, D, I, D]
-        lib.oracle_newton.argtypes = [I, I, D, D, D, I, I, I, ctypes.c_double, I, I, D, D, D, D,
+        lib.oracle_newton.argtypes = [I, I, D, D, D, I, I, I, ctypes.c_double, I, I, I, D, D, D, D,
                                       IP, IP, IP]
         lib.oracle_bptt.argtypes = [I, I, D, D, D, D, D, I, D, D, D, D]
         lib.oracle_gemm.argtypes = [I, I, I, D, I, D, I, D, D]
@@ -169,12 +169,13 @@ _RESIDUAL_MODES = {"scaled": 0, "raw": 1}
 
 
 def newton(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init="decoupled",
-           residual_mode="scaled", S_init=None):
+           residual_mode="scaled", S_init=None, sweeps=0):
     """fp64 Newton; returns (S, stats dict).
 
-    init: "decoupled" (the trajectory with R = 0, the default), "zero", or
-    "given" with S_init (L, T, 4) as the initial guess.  residual_mode:
-    "scaled" (max |F| / (1 + |s|) <= tol) or "raw" (max |F| <= tol)."""
+    init: "decoupled" (the trajectory with R = 0, then `sweeps` refinement
+    sweeps; the default), "zero", or "given" with S_init (L, T, 4) as the
+    initial guess.  residual_mode: "scaled" (max |F| / (1 + |s|) <= tol) or
+    "raw" (max |F| <= tol)."""
     lib = _load()
     P, R, s0 = _f64(P), _f64(R), _f64(s0)
     L, T, _ = P.shape
@@ -192,7 +193,7 @@ def newton(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init=
     ir = np.zeros(2)
     it, conv, div = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     lib.oracle_newton(L, T, _ptr(P), _ptr(R), _ptr(s0), _forget_code(forget), int(max_iters),
-                      1 if fixed else 0, float(tol), code, _RESIDUAL_MODES[residual_mode], _ptr(S),
+                      1 if fixed else 0, float(tol), code, int(sweeps), _RESIDUAL_MODES[residual_mode], _ptr(S),
                       _ptr(hr), _ptr(hs), _ptr(ir), ctypes.byref(it), ctypes.byref(conv), ctypes.byref(div))
     return S, {"iters": it.value, "converged": bool(conv.value), "diverged": bool(div.value),
                "max_abs_F": hr[: it.value].copy(), "max_scaled_F": hs[: it.value].copy(),
@@ -245,11 +246,11 @@ def sequential_btgd(P, R, s0, forget="sigmoid") -> np.ndarray:
 
 
 def newton_btgd(P, R, s0, forget="sigmoid", max_iters=8, fixed=False, tol=1e-5, init="decoupled",
-                residual_mode="scaled", S_init=None):
+                residual_mode="scaled", S_init=None, sweeps=0):
     B, T, _, d = P.shape
     Si = lanes_from_btgd(S_init) if S_init is not None else None
     S, st = newton(lanes_from_btgd(P), lanes_from_gd(R, B), lanes_from_bgd(s0), forget,
-                   max_iters, fixed, tol, init, residual_mode, Si)
+                   max_iters, fixed, tol, init, residual_mode, Si, sweeps)
     return btgd_from_lanes(S, B, d), st
 
 
@@ -294,7 +295,7 @@ def sequential_varlen(P, R, s0, cu, forget="sigmoid") -> np.ndarray:
     return S
 
 
-def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4, init="decoupled") -> np.ndarray:
+def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4, init="decoupled", sweeps=0) -> np.ndarray:
     """K Newton iterations from the given kind of guess ("decoupled" or "zero")
     on every sequence (fixed-K mode)."""
     P = _f64(P)
@@ -304,7 +305,7 @@ def newton_varlen_fixed(P, R, s0, cu, forget="sigmoid", K=4, init="decoupled") -
         if b > a:
             s0k = np.zeros((1, 4, d)) if s0 is None else _f64(s0)[k:k + 1]
             S[a:b] = newton_btgd(P[None, a:b], R, s0k, forget, max_iters=K, fixed=True, tol=0.0,
-                                  init=init)[0][0]
+                                  init=init, sweeps=sweeps)[0][0]
     return S
 
 

@@ -276,6 +276,29 @@ static void decoupled_trajectory(int T, const double *P, const double *s0, int f
     }
 }
 
+/*
+ * One refinement sweep of the decoupled guess: the gates of step t see the
+ * previous guess's h_{t-1} (Sold), while c, n and m recur exactly from the
+ * new sweep's own previous state, as in decoupled_trajectory:
+ *   a_t = P_t + r h^old_{t-1}  (h^old_{-1} = s0's h),  Snew_t = step(Snew_{t-1}, a_t) with r = 0.
+ * It is a fixed-point (Picard) sweep of the recurrence on h: the solution is
+ * its fixed point, and after k sweeps the first k steps are exact.  Reading
+ * taken for the guess's refinement: the pages give no initial guess.
+ */
+static void guess_sweep(int T, const double *P, const double *r, const double *s0, int forget,
+                        const double *Sold, double *Snew)
+{
+    const double zero[4] = {0.0, 0.0, 0.0, 0.0};
+    const double *prev = s0;
+    for (int t = 0; t < T; ++t) {
+        const double h_old = (t == 0) ? s0[3] : Sold[(size_t)(t - 1) * 4 + 3];
+        double a[4];
+        for (int g = 0; g < 4; ++g) a[g] = P[(size_t)t * 4 + g] + r[g] * h_old;
+        oracle_step(prev, a, zero, forget, Snew + (size_t)t * 4, NULL, NULL);
+        prev = Snew + (size_t)t * 4;
+    }
+}
+
 /* Raw and scaled maxima of the residual of every lane at S; returns 1 when
  * some residual or state entry is not finite. */
 static int residual_maxima(int lanes, int T, const double *P, const double *R, const double *s0,
@@ -307,11 +330,15 @@ static int residual_maxima(int lanes, int T, const double *P, const double *R, c
  * Newton solve of the whole trajectory (ParaRNN Newton, as described in
  * [pararnn] "Cell" and [structure] "Current surface"):
  *   initial guess (s0 is fixed and enters as the step before t = 0):
- *     init 0: the decoupled trajectory (decoupled_trajectory above); in
- *             tolerance mode its residual is evaluated first, and a guess
- *             that already meets the test ends the solve after 0 iterations;
+ *     init 0: the decoupled trajectory (decoupled_trajectory above), then
+ *             `sweeps` refinement sweeps (guess_sweep above);
  *     init 1: S = 0 for every t;
- *     init 2: S as given on entry (its residual is not evaluated);
+ *     init 2: S as given on entry;
+ *   the residual of the initial guess is recorded in init_res (raw, scaled)
+ *   when init is 0, the mode is tolerance and max_iters >= 1, else init_res
+ *   holds -1; it does not stop the solve: the test starts with iteration 1;
+ *   max_iters = 0 returns the initial guess itself (iters 0, neither
+ *   converged nor diverged);
  *   repeat k = 1..max_iters:
  *     F_t = S_t - f(S_{t-1}, P_t),  J_t = d f / d s_{t-1} at the guess
  *     solve delta_t = J_t delta_{t-1} - F_t,  delta_{-1} = 0
@@ -331,7 +358,7 @@ static int residual_maxima(int lanes, int T, const double *P, const double *R, c
  */
 void oracle_newton(int lanes, int T, const double *P, const double *R,
                    const double *s0, int forget, int max_iters, int fixed,
-                   double tol, int init, int residual_mode, double *S,
+                   double tol, int init, int sweeps, int residual_mode, double *S,
                    double *hist_raw, double *hist_scaled, double *init_res,
                    int *iters, int *converged, int *diverged)
 {
@@ -341,8 +368,14 @@ void oracle_newton(int lanes, int T, const double *P, const double *R,
     double *negF = malloc(sizeof(double) * n4);
     double *delta = malloc(sizeof(double) * n4);
     if (init == 0) {
-        for (int l = 0; l < lanes; ++l)
-            decoupled_trajectory(T, P + (size_t)l * n4, s0 + 4 * l, forget, S + (size_t)l * n4);
+        for (int l = 0; l < lanes; ++l) {
+            double *Sl = S + (size_t)l * n4;
+            decoupled_trajectory(T, P + (size_t)l * n4, s0 + 4 * l, forget, Sl);
+            for (int k = 0; k < sweeps; ++k) {
+                guess_sweep(T, P + (size_t)l * n4, R + 4 * l, s0 + 4 * l, forget, Sl, delta);
+                memcpy(Sl, delta, sizeof(double) * n4);
+            }
+        }
     } else if (init == 1) {
         memset(S, 0, sizeof(double) * n4 * lanes);
     }
@@ -351,20 +384,9 @@ void oracle_newton(int lanes, int T, const double *P, const double *R,
     *diverged = 0;
     if (init_res) init_res[0] = init_res[1] = -1.0;
     double raw = INFINITY, scaled = INFINITY;
-    int done = 0;
-    if (init == 0 && !fixed) {
-        const int bad = residual_maxima(lanes, T, P, R, s0, forget, S, F, &raw, &scaled);
-        if (init_res) {
-            init_res[0] = raw;
-            init_res[1] = scaled;
-        }
-        const double test = residual_mode ? raw : scaled;
-        if (!bad && test <= tol) {
-            *converged = 1;
-            done = 1;
-        }
-    }
-    for (int k = 1; k <= max_iters && !done; ++k) {
+    if (init == 0 && !fixed && max_iters >= 1 && init_res)
+        (void)residual_maxima(lanes, T, P, R, s0, forget, S, F, &init_res[0], &init_res[1]);
+    for (int k = 1; k <= max_iters; ++k) {
         for (int l = 0; l < lanes; ++l) {
             double *Sl = S + (size_t)l * n4;
             residual_and_jacobian(T, P + (size_t)l * n4, R + 4 * l, s0 + 4 * l,
@@ -384,8 +406,8 @@ void oracle_newton(int lanes, int T, const double *P, const double *R,
             break;
         }
     }
-    if (fixed && (residual_mode ? raw : scaled) <= tol) *converged = 1;
-    if (!*converged && !(raw <= 1.0)) *diverged = 1;
+    if (fixed && max_iters >= 1 && (residual_mode ? raw : scaled) <= tol) *converged = 1;
+    if (*iters > 0 && !*converged && !(raw <= 1.0)) *diverged = 1;
     free(F);
     free(J);
     free(negF);

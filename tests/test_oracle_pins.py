@@ -286,26 +286,61 @@ def _closed_form_h_zero_recurrence(P, forget):
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 def test_decoupled_guess_is_the_zero_recurrence_solution(forget):
     """The default initial guess is the trajectory with R = 0.  With R = 0 it
-    is therefore the solution itself: the solve ends after 0 iterations with
-    a zero residual and h equal to the closed form."""
+    is therefore the solution itself: its residual is zero, one iteration
+    leaves it where it is, and h is the closed form.  max_iters = 0 returns
+    the guess."""
     rng = np.random.default_rng(71)
     P, _, _ = _rand_lane_inputs(rng, 3, 30, forget)
     R = np.zeros((3, 4))
     s0 = np.zeros((3, 4))
     S, st = oracle.newton(P, R, s0, forget, max_iters=5, tol=1e-12)
-    assert st["iters"] == 0 and st["converged"] and not st["diverged"]
-    assert st["init_max_abs_F"] == 0.0
+    assert st["iters"] == 1 and st["converged"] and not st["diverged"]
+    assert st["init_max_abs_F"] == 0.0 and st["max_abs_F"][0] == 0.0
     H = _closed_form_h_zero_recurrence(P, forget)
     np.testing.assert_allclose(S[:, :, 3], H, rtol=0, atol=1e-12)
     # with R != 0 the guess keeps the R = 0 gates: its h is still the closed
     # form of the R = 0 cell, and its residual is nonzero
     R2 = rng.uniform(-0.5, 0.5, size=(3, 4))
-    S2, st2 = oracle.newton(P, R2, s0, forget, max_iters=1, fixed=True, init="decoupled")
-    Sg, stg = oracle.newton(P, R2, s0, forget, max_iters=1, tol=1e30)
-    assert stg["iters"] == 0 and stg["init_max_abs_F"] > 1e-3
+    Sg, stg = oracle.newton(P, R2, s0, forget, max_iters=0)
+    assert stg["iters"] == 0 and not stg["converged"] and not stg["diverged"]
     np.testing.assert_allclose(Sg[:, :, 3], H, rtol=0, atol=1e-12)
-    # a fixed-K solve does not stop at the guess
-    assert st2["iters"] == 1 and st2["init_max_abs_F"] == -1.0
+    _, st2 = oracle.newton(P, R2, s0, forget, max_iters=1, tol=1e-30)
+    assert st2["init_max_abs_F"] > 1e-3
+    # a fixed-K solve does not record the guess's residual
+    _, st3 = oracle.newton(P, R2, s0, forget, max_iters=1, fixed=True)
+    assert st3["iters"] == 1 and st3["init_max_abs_F"] == -1.0
+
+
+@pytest.mark.parametrize("forget", ["sigmoid", "exp"])
+def test_guess_sweeps(forget):
+    """Refinement sweeps of the guess: a sweep's gates see the previous
+    guess's h, so (1) with R = 0 a sweep leaves the decoupled guess unchanged,
+    (2) the solution is a fixed point of the sweep, (3) after k sweeps the
+    first k steps are the sequential trajectory (prefix exactness of the
+    fixed-point iteration), and (4) on the workloads' lanes each sweep shrinks
+    the residual and the sweeps converge to the solution."""
+    rng = np.random.default_rng(97)
+    T = 40
+    P, R, s0 = _rand_lane_inputs(rng, 3, T, forget)
+    Sseq = oracle.sequential(P, R, s0, forget)
+    Z = np.zeros((3, 4))
+    g0, _ = oracle.newton(P, Z, s0, forget, max_iters=0)
+    g2, _ = oracle.newton(P, Z, s0, forget, max_iters=0, sweeps=2)
+    np.testing.assert_array_equal(g0, g2)
+    for k in (1, 2, 5):
+        gk, _ = oracle.newton(P, R, s0, forget, max_iters=0, sweeps=k)
+        np.testing.assert_allclose(gk[:, :k], Sseq[:, :k], rtol=0, atol=1e-12 * (1 + np.abs(Sseq).max()))
+        if k < T:
+            assert np.abs(gk[:, k:] - Sseq[:, k:]).max() > 1e-12
+    # the solution is the sweeps' fixed point: T sweeps and more reach it
+    g_many, _ = oracle.newton(P, R, s0, forget, max_iters=0, sweeps=T + 5)
+    np.testing.assert_allclose(g_many, Sseq, rtol=0, atol=1e-10 * (1 + np.abs(Sseq).max()))
+    P2, R2, s02 = _workload_lanes(rng, 4, 512, forget, 0.5)
+    res = []
+    for k in range(4):
+        _, st = oracle.newton(P2, R2, s02, forget, max_iters=1, tol=1e-30, sweeps=k)
+        res.append(st["init_max_scaled_F"])
+    assert all(b < a for a, b in zip(res, res[1:])), res
 
 
 def _workload_lanes(rng, L, T, forget, r_scale):
