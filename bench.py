@@ -2,17 +2,24 @@
 """Benchmark of the Newton-solved diag-mix sLSTM training step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--newton-iters K_N] [--impl reference]
+                    [--newton-mode tol|fixed] [--newton-iters K_N] [--impl reference]
 
 One step = the whole hot path on one batch of synthetic input already in HBM:
-  input projection GEMM  ->  K_N fixed Newton iterations (fused residual,
-  Jacobian, blocked scan, update)  ->  backward (fused adjoint scan + cell
-  VJP, dR/db reduction, dx and dW_x GEMMs).
+  input projection GEMM  ->  Newton solve to the workload's tolerance (the
+  decoupled initial guess, then iterations with fused residual, Jacobian,
+  blocked scan and update until max |F| / (1 + |s|) <= tol)  ->  backward
+  (fused adjoint scan + cell VJP, dR/db reduction, dx and dW_x GEMMs).
 Metric: B*T*d_h elements per second for forward + backward (the JSON
 `value`), with the forward alone reported beside it.  Under torchrun each
 rank runs its own replica of the workload (independent batches, no data-path
 collective): `value` is the sum over ranks of elements divided by the slowest
 rank's device time.
+
+With no flags the line also carries, measured in the same run on rank 0: the
+long-sequence workload's forward (B=4, T=65536, d=2048: input projection and
+the converged Newton solve, and the fixed K=4 solve) with the Newton solve's
+HBM roofline fraction, and the scan_block4 sweep at B=4, d=2048 over
+T = 4096, 16384, 65536.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of lanes of the same workload.
@@ -77,54 +84,184 @@ def aggregate(elems_per_rank, n_ranks, ms_per_step_max):
 # ---------------------------------------------------------------------------
 # CPU oracle sample (cpu_baseline leg and --impl reference)
 # ---------------------------------------------------------------------------
-def oracle_sample(w, inp, n_lanes, newton_iters, seed=0):
-    """Run the fp64 oracle, as it stands, on n_lanes (b, j) lanes of the
-    workload: input projection rows, K fixed Newton iterations, BPTT and the
-    lanes' contributions to dx and dW_x.  Returns (seconds, elements)."""
-    import oracle
+def _sample_lanes(w, n_lanes, seed):
     rng = np.random.default_rng(seed)
-    lanes = [(int(rng.integers(0, w.B)), int(rng.integers(0, w.d_h))) for _ in range(n_lanes)]
+    return [(int(rng.integers(0, w.B)), int(rng.integers(0, w.d_h))) for _ in range(n_lanes)]
+
+
+def oracle_lane(w, inp, b, j, newton):
+    """The fp64 oracle, as it stands, on one (b, j) lane of the workload: its
+    input-projection rows, the Newton solve (newton = ("tol", cap, sweeps) or
+    ("fixed", K, sweeps), from the decoupled guess with that many refinement
+    sweeps), BPTT and the lane's
+    contributions to dx and dW_x."""
+    import oracle
     bias = as_f64(inp["bias"])
+    xb = as_f64(inp["x"][b])                                        # (T, d_in)
+    rows = [g * w.d_h + j for g in range(4)]
+    Wr = as_f64(inp["Wx"][rows])                                    # (4, d_in)
+    P = oracle.gemm(xb, Wr, tb=True, bias=bias[:, j])[None]         # (1, T, 4)
+    R = as_f64(inp["R"][:, j])[None]
+    s0 = np.zeros((1, 4))
+    mode, k, sweeps = newton
+    S, st = oracle.newton(P, R, s0, w.forget, max_iters=k, fixed=(mode == "fixed"), tol=w.tol, sweeps=sweeps)
+    dH = as_f64(inp["dH"][b, :, j])[None]
+    dP, dR, db, ds0 = oracle.bptt(P, R, s0, S, dH, w.forget)
+    oracle.gemm(dP[0], Wr)                                          # this lane's share of dx
+    oracle.gemm(np.ascontiguousarray(dP[0].T), np.ascontiguousarray(xb.T), tb=True)  # its dW_x rows
+    return st["iters"]
+
+
+_POOL_STATE = {}
+_SHARED_KEYS = ("x", "Wx", "R", "bias", "dH")
+
+
+def _share_inputs(inp):
+    """Copy the workload's input tensors into shared memory once, so that the
+    oracle's worker processes read them instead of each drawing its own copy.
+    Returns (segments to keep alive, metadata for the workers)."""
+    import torch
+    from multiprocessing import shared_memory
+    segs, meta = [], {}
+    for k in _SHARED_KEYS:
+        t = inp[k].contiguous()
+        raw = t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+        arr = raw.numpy()
+        shm = shared_memory.SharedMemory(create=True, size=max(1, arr.nbytes))
+        np.ndarray(arr.shape, dtype=arr.dtype, buffer=shm.buf)[...] = arr
+        segs.append(shm)
+        meta[k] = (shm.name, tuple(t.shape), str(t.dtype))
+    return segs, meta
+
+
+def _pool_init(name, T, meta):
+    import torch
+    from multiprocessing import shared_memory
+    w = WORKLOADS[name] if T == WORKLOADS[name].T else scaled(WORKLOADS[name], T=T)
+    inp, keep = {}, []
+    for k, (shm_name, shape, dt) in meta.items():
+        shm = shared_memory.SharedMemory(name=shm_name)
+        keep.append(shm)
+        if dt == "torch.bfloat16":
+            arr = np.ndarray(shape, dtype=np.int16, buffer=shm.buf)
+            inp[k] = torch.from_numpy(arr).view(torch.bfloat16)
+        else:
+            inp[k] = torch.from_numpy(np.ndarray(shape, dtype=np.float32, buffer=shm.buf))
+    _POOL_STATE.update(w=w, inp=inp, keep=keep)
+
+
+def _pool_lane(task):
+    b, j, newton = task
+    return oracle_lane(_POOL_STATE["w"], _POOL_STATE["inp"], b, j, newton)
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_timing(w, inp, newton, single_lanes, seed=0, pool=None, pool_lanes=0):
+    """Elements per second of the oracle on sampled lanes: on one core in this
+    process, and (pool given) on every core with one worker process per core,
+    each lane one task.  Returns a dict."""
+    out = {}
+    oracle_lane(w, inp, 0, 0, newton)                               # warm the oracle library
+    lanes = _sample_lanes(w, single_lanes, seed)
     t0 = time.perf_counter()
-    for b, j in lanes:
-        xb = as_f64(inp["x"][b])                                        # (T, d_in)
-        rows = [g * w.d_h + j for g in range(4)]
-        Wr = as_f64(inp["Wx"][rows])                                    # (4, d_in)
-        P = oracle.gemm(xb, Wr, tb=True, bias=bias[:, j])[None]         # (1, T, 4)
-        R = as_f64(inp["R"][:, j])[None]
-        s0 = np.zeros((1, 4))
-        S, _ = oracle.newton(P, R, s0, w.forget, max_iters=newton_iters, fixed=True, tol=w.tol)
-        dH = as_f64(inp["dH"][b, :, j])[None]
-        dP, dR, db, ds0 = oracle.bptt(P, R, s0, S, dH, w.forget)
-        oracle.gemm(dP[0], Wr)                                          # this lane's share of dx
-        oracle.gemm(np.ascontiguousarray(dP[0].T), np.ascontiguousarray(xb.T), tb=True)  # its dW_x rows
+    iters = [oracle_lane(w, inp, b, j, newton) for b, j in lanes]
     dt = time.perf_counter() - t0
-    return dt, n_lanes * w.T
+    out["single"] = {"value": single_lanes * w.T / dt, "cores": 1, "seconds": dt, "lanes": single_lanes,
+                     "newton_iters": iters}
+    if pool is not None and pool_lanes:
+        lanes = _sample_lanes(w, pool_lanes, seed + 1)
+        pool.map(_pool_lane, [(0, 0, newton)] * pool.cores)                  # every worker warmed
+        t0 = time.perf_counter()
+        pool.map(_pool_lane, [(b, j, newton) for b, j in lanes])
+        dt = time.perf_counter() - t0
+        out["all_cores"] = {"value": pool_lanes * w.T / dt, "cores": pool.cores, "seconds": dt,
+                            "lanes": pool_lanes}
+    return out
+
+
+class OraclePool:
+    """One spawned worker process per host core (at most 64), reading the
+    workload's inputs from shared memory.  Spawned, not forked, so that it is
+    safe whether or not this process has touched the GPU."""
+
+    def __init__(self, w, inp):
+        import concurrent.futures
+        import multiprocessing as mp
+        self.cores = min(host_cores(), 64)
+        self.segs, meta = _share_inputs(inp)
+        base = w.name.split("_T")[0] if w.name not in WORKLOADS else w.name
+        self.ex = concurrent.futures.ProcessPoolExecutor(max_workers=self.cores, mp_context=mp.get_context("spawn"),
+                                                         initializer=_pool_init, initargs=(base, w.T, meta))
+
+    def map(self, fn, tasks):
+        return list(self.ex.map(fn, tasks))
+
+    def shutdown(self):
+        self.ex.shutdown()
+        for s in self.segs:
+            s.close()
+            s.unlink()
+
+
+def _newton_desc(newton):
+    mode, k, sweeps = newton
+    it = f"Newton to the workload's tolerance (cap {k})" if mode == "tol" else f"{k} fixed Newton iterations"
+    return f"{it} from the decoupled guess with {sweeps} refinement sweeps"
 
 
 def run_reference(args, w):
     ws, rank, _ = _dist()
     if rank != 0:
         return 0
+    newton = (("tol", w.max_iters) if args.newton_mode == "tol" else ("fixed", args.newton_iters)) + (args.guess_sweeps,)
     inp = make_inputs(w)
-    t_lane = 0.0
-    for _ in range(args.warmup):
-        t_lane, _ = oracle_sample(w, inp, 1, args.newton_iters, seed=99)
-    # bounded sample: about a minute of CPU work over all timed steps
-    lanes_per_step = int(max(1, min(args.ref_lanes, 60.0 / max(1e-3, args.steps * t_lane))))
+    pool = OraclePool(w, inp)
+    cores = pool.cores
+    lanes = _sample_lanes(w, cores, 99)
+    pool.map(_pool_lane, [(b, j, newton) for b, j in lanes])   # warm-up: every worker ready
+    for _ in range(args.warmup - 1):
+        pool.map(_pool_lane, [(b, j, newton) for b, j in lanes])
+    t0 = time.perf_counter()
+    pool.map(_pool_lane, [(b, j, newton) for b, j in lanes])
+    per_round = time.perf_counter() - t0
+    # bounded sample: about a minute of wall time over all timed steps
+    rounds = int(max(1, min(args.ref_lanes, 60.0 / max(1e-3, args.steps * per_round))))
     total_t, total_e = 0.0, 0
-    for s in range(args.steps):
-        dt, el = oracle_sample(w, inp, lanes_per_step, args.newton_iters, seed=s)
-        total_t += dt
-        total_e += el
+    for s_ in range(args.steps):
+        lanes = _sample_lanes(w, rounds * cores, s_)
+        t0 = time.perf_counter()
+        pool.map(_pool_lane, [(b, j, newton) for b, j in lanes])
+        total_t += time.perf_counter() - t0
+        total_e += len(lanes) * w.T
+    pool.shutdown()
     value = total_e / total_t
-    sample = (f"{lanes_per_step} random (b,j) lanes x T={w.T} per step: fp64 input-projection rows, "
-              f"{args.newton_iters} fixed Newton iterations, BPTT, dx/dW_x contributions")
+    sample = (f"{rounds * cores} random (b,j) lanes x T={w.T} per step on {cores} worker processes "
+              f"({cpu_model()}): fp64 input-projection rows, {_newton_desc(newton)}, "
+              f"BPTT, dx/dW_x contributions")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": dict(w.describe(), newton_iters=args.newton_iters, newton_mode="fixed"),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "data": "synthetic",
+            "config": dict(w.describe(), newton_mode=newton[0], newton_max_iters=newton[1], guess_sweeps=newton[2]),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -185,9 +322,13 @@ def run_gpu(args, w):
     torch.cuda.set_device(dev)
     api._lib.load()
 
-    K = args.newton_iters
+    tol_mode = args.newton_mode == "tol"
+    K = w.max_iters if tol_mode else args.newton_iters
     forward_only = args.mode == "forward"
     inp = make_inputs(w)
+    pool = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        pool = OraclePool(w, inp)            # spawned workers, started before the GPU work
     x, Wx, R, bias, s0, dH = (inp[k].to(dev) for k in ("x", "Wx", "R", "bias", "s0", "dH"))
     P = torch.empty(w.B, w.T, 4, w.d_h, device=dev)
     S = torch.empty_like(P)
@@ -209,8 +350,8 @@ def run_gpu(args, w):
         api.preact_gemm(dv["x"], dv["Wx"], dv["bias"], P=P)
         if ev is not None:
             ev[1].record()
-        api.newton_forward(P, dv["R"], dv["s0"], forget=w.forget, max_iters=K, fixed=True, tol=w.tol, S=S,
-                           stats=stats, ws=ws_n)
+        api.newton_forward(P, dv["R"], dv["s0"], forget=w.forget, max_iters=K, fixed=not tol_mode, tol=w.tol, S=S,
+                           stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps)
         if ev is not None:
             ev[2].record()
         if not forward_only:
@@ -245,6 +386,7 @@ def run_gpu(args, w):
     ms_newton = sum(e[1].elapsed_time(e[2]) for e in evs)
     ms_bwd = sum(e[2].elapsed_time(e[3]) for e in evs)
     st = api.read_stats(stats)
+    S_finite = bool(torch.isfinite(S).all().item())
 
     # ---- end to end through the public API from pinned host buffers ----
     # Every step copies its inputs (x, W_x, R, b, s0, dH) host -> device and
@@ -326,41 +468,66 @@ def run_gpu(args, w):
     fwd_ms = (ms_gemm + ms_newton) / args.steps
 
     hbm, peak_kind = _peaks()
-    newton_launch_ms = ms_newton / args.steps / K
-    # algorithmic bytes of one Newton launch: iteration 1 reads P and writes S
-    # (32 B/elem); later ones also read the old S (48 B/elem).  Averaged over
-    # the K launches of a step.
-    newton_bytes = elems * (32 + 48 * (K - 1)) / K
-    achieved = newton_bytes / (newton_launch_ms / 1e3) / 1e9
-    traffic = args.traffic_bytes if args.traffic_bytes else newton_traffic_bytes(elems, K)
-    roofline = {"kernel": "newton_iter", "bound": "hbm", "achieved": achieved, "peak": hbm,
-                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
-                "algorithmic_bytes_per_launch": newton_bytes, "avg_launch_ms": newton_launch_ms}
+    # The Newton solve is one C call: the guess launch (reads P, writes S: 32
+    # algorithmic B/elem), its refinement sweeps (read P and h, write S: 36
+    # B/elem each) and n iterations (read P and the old S, write S: 48 B/elem
+    # each); in tolerance mode the launches after convergence return at once.
+    # Its CUDA-event time over the timed region against those bytes.
+    n_it = st["iters"]
+    sw = args.guess_sweeps
+    newton_ms = ms_newton / args.steps
+    newton_bytes = elems * solve_bytes_per_elem(n_it, sw)
+    achieved = newton_bytes / (newton_ms / 1e3) / 1e9
+    traffic = args.traffic_bytes if args.traffic_bytes else newton_traffic_bytes(elems, n_it, sw)
+    roofline = {"kernel": "newton solve (guess_kernel x (1 + sweeps) + newton_iter x iters)", "bound": "hbm",
+                "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "algorithmic_bytes_per_solve": newton_bytes,
+                "working_launches_per_solve": 1 + sw + n_it, "avg_launch_ms": newton_ms / (1 + sw + n_it),
+                "solve_ms": newton_ms}
 
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        oracle_sample(w, inp, 1, K, seed=123)              # warm the oracle library
-        dt, el = oracle_sample(w, inp, args.cpu_lanes, K)
-        cpu = {"value": el / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{args.cpu_lanes} random (b,j) lanes x T={w.T}: fp64 input-projection rows, {K} fixed "
-                         f"Newton iterations, BPTT, dx/dW_x contributions ({dt:.1f} s, single thread)"}
+    if pool is not None:
+        newton = ("tol", w.max_iters, args.guess_sweeps) if tol_mode else ("fixed", K, args.guess_sweeps)
+        t = oracle_timing(w, inp, newton, args.cpu_lanes, seed=123, pool=pool,
+                          pool_lanes=args.cpu_lanes * pool.cores)
+        pool.shutdown()
+        cpu = {"value": t["all_cores"]["value"], "unit": UNIT, "cores": t["all_cores"]["cores"], "kind": "oracle",
+               "cpu_model": cpu_model(),
+               "sample": f"{t['all_cores']['lanes']} random (b,j) lanes x T={w.T} on {t['all_cores']['cores']} "
+                         f"worker processes ({t['all_cores']['seconds']:.1f} s): fp64 input-projection rows, "
+                         f"{_newton_desc(newton)}, BPTT, dx/dW_x contributions",
+               "single_core": {"value": t["single"]["value"], "lanes": t["single"]["lanes"],
+                               "seconds": t["single"]["seconds"]}}
 
-    # kernels launched per step: preact GEMM 1, Newton K, backward: adjoint 1 +
-    # dR/db reduction 1 + 2 GEMMs (+ the split-K sum of the tensor-core path)
-    launches_per_step = 1 + K + (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0))
+    extra = {}
+    if rank == 0 and ws == 1 and args.mode == "train" and not args.no_extra and args.seq_len is None:
+        del P, S, grads, dev_bufs, grad_bufs, ws_n, ws_b
+        torch.cuda.empty_cache()
+        extra["long_forward"] = long_forward(args, dev, hbm, peak_kind)
+        torch.cuda.empty_cache()
+        extra["scan_block4_sweep"] = scan_sweep(args, dev, hbm, peak_kind)
+
+    # kernels launched per step: preact GEMM 1, Newton: the guess + K iteration
+    # launches (in tolerance mode those after convergence exit at once),
+    # backward: adjoint 1 + dR/db reduction 1 + 2 GEMMs (+ the split-K sum of
+    # the tensor-core path)
+    launches_per_step = 1 + 1 + args.guess_sweeps + K + (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0))
     line = {
         "metric": METRIC_FWD if forward_only else METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "operand_dtype": "bf16 x/W_x, fp32 state and scans" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
-        "config": dict(w.describe(), newton_iters=K, newton_mode="fixed",
+        "config": dict(w.describe(), newton_mode=args.newton_mode, newton_max_iters=K, newton_init="decoupled",
+                       guess_sweeps=args.guess_sweeps,
                        l2="inputs larger than L2 (P and S are %.2f GB each)" % (elems * 16 / 1e9),
                        parallelism=f"replicas x{ws}"),
         "fwd": {"value": aggregate(elems, ws, fwd_ms), "unit": UNIT, "ms_per_step": fwd_ms},
         "breakdown_ms_per_step": {"preact_gemm": ms_gemm / args.steps, "newton_forward": ms_newton / args.steps,
                                   "backward": ms_bwd / args.steps},
-        "newton_stats_last_step": {"iters": st["iters"], "diverged": st["diverged"], "error": st["error"]},
+        "newton_stats_last_step": {"iters": st["iters"], "converged": st["converged"], "diverged": st["diverged"],
+                                   "error": st["error"], "max_scaled_F": st["max_scaled_F"],
+                                   "init_max_scaled_F": st["init_max_scaled_F"], "S_finite": S_finite},
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": aggregate(elems, ws, ms_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -368,6 +535,7 @@ def run_gpu(args, w):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    line.update(extra)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -376,18 +544,15 @@ def run_gpu(args, w):
     return 0
 
 
-def run_scan(args):
+def scan_sweep(args, dev, hbm, peak_kind, T_list=None):
     """scan_block4 alone: B=4, d=2048, T swept; 96 algorithmic bytes per
     element (read A 64, b 16, write y 16).  Inputs drawn on the device from a
     seeded generator (values only set the timing's data, not checked here)."""
     import torch
     from nonlinear_rnn_pararnn_b200 import _lib, api
-    ws_n, rank, _ = _dist()
-    dev = torch.device("cuda", 0)
-    hbm, peak_kind = _peaks()
     B, d = 4, 2048
     sweep = []
-    for T in [int(v) for v in args.scan_T.split(",")]:
+    for T in (T_list or [int(v) for v in args.scan_T.split(",")]):
         g = torch.Generator(device=dev)
         g.manual_seed(T)
         A = torch.rand(B, T, 4, 4, d, generator=g, device=dev) * 0.6 - 0.3
@@ -398,23 +563,86 @@ def run_scan(args):
             api.scan_block4(A, b, None, y=y, ws=ws)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(3, min(args.steps, 20))
         e0.record()
-        for _ in range(args.steps):
+        for _ in range(n):
             api.scan_block4(A, b, None, y=y, ws=ws)
         e1.record()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
+        ms = e0.elapsed_time(e1) / n
         elems = B * T * d
         gbs = elems * 96 / (ms / 1e3) / 1e9
-        sweep.append({"T": T, "ms": ms, "elems_per_s": elems / (ms / 1e3), "achieved_GBs": gbs,
-                      "frac": gbs / hbm})
+        sweep.append({"workload": f"scan_block4_b{B}_t{T}_d{d}", "T": T, "ms": ms, "elems_per_s": elems / (ms / 1e3),
+                      "achieved_GBs": gbs, "peak": hbm, "peak_kind": peak_kind, "frac": gbs / hbm, "steps": n})
         del A, b, y, ws
         torch.cuda.empty_cache()
+    return sweep
+
+
+def long_forward(args, dev, hbm, peak_kind):
+    """The long-sequence workload's forward (B=4, T=65536, d_in=d_h=2048, bf16
+    x/W_x, R ~ U(-0.3, 0.3)): input projection + the Newton solve, converged
+    to its tolerance and with K=4 fixed iterations, timed with CUDA events;
+    the Newton solve's roofline as for the training step."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+    w = WORKLOADS["slstm_bf16_long_b4_t65536_d2048"]
+    inp = make_inputs(w, with_dH=False)
+    x, Wx, R, bias, s0 = (inp[k].to(dev) for k in ("x", "Wx", "R", "bias", "s0"))
+    P = torch.empty(w.B, w.T, 4, w.d_h, device=dev)
+    S = torch.empty_like(P)
+    stats = api.new_stats(dev)
+    ws_n = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
+    out = {"workload": w.name, "B": w.B, "T": w.T, "d_h": w.d_h, "forget": w.forget, "tol": w.tol}
+    for mode, K in (("tol", w.max_iters), ("fixed", (w.fixed_iters or (4,))[0])):
+        def step(ev):
+            ev[0].record()
+            api.preact_gemm(x, Wx, bias, P=P)
+            ev[1].record()
+            api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, fixed=(mode == "fixed"), tol=w.tol, S=S,
+                               stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps)
+            ev[2].record()
+        n = 5
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.warmup + n)]
+        for i in range(args.warmup):
+            step(evs[i])
+        torch.cuda.synchronize()
+        for i in range(n):
+            step(evs[args.warmup + i])
+        torch.cuda.synchronize()
+        timed = evs[args.warmup:]
+        gemm_ms = sum(e[0].elapsed_time(e[1]) for e in timed) / n
+        newton_ms = sum(e[1].elapsed_time(e[2]) for e in timed) / n
+        st = api.read_stats(stats)
+        it = st["iters"]
+        nbytes = w.elems * solve_bytes_per_elem(it, args.guess_sweeps)
+        gbs = nbytes / (newton_ms / 1e3) / 1e9
+        out[mode] = {"newton_mode": mode, "max_iters": K, "iters": it, "guess_sweeps": args.guess_sweeps,
+                     "converged": st["converged"],
+                     "error": st["error"], "max_scaled_F": st["max_scaled_F"],
+                     "S_finite": bool(torch.isfinite(S).all().item()),
+                     "fwd_elems_per_s": w.elems / ((gemm_ms + newton_ms) / 1e3), "ms_preact_gemm": gemm_ms,
+                     "ms_newton": newton_ms, "steps": n,
+                     "roofline": {"kernel": "newton solve (guess_kernel x (1 + sweeps) + newton_iter x iters)",
+                                  "bound": "hbm",
+                                  "achieved": gbs, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                                  "frac": gbs / hbm, "algorithmic_bytes_per_solve": nbytes}}
+    del x, Wx, R, bias, s0, P, S, ws_n
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_scan(args):
+    import torch
+    ws_n, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    hbm, peak_kind = _peaks()
+    sweep = scan_sweep(args, dev, hbm, peak_kind)
     last = sweep[-1]
     line = {"metric": "scan_block4 elems/s (B*T*d/s)", "value": last["elems_per_s"], "unit": UNIT, "n_gpus": 1,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": last["ms"], "higher_is_better": True,
+            "steps": last["steps"], "warmup": args.warmup, "ms_per_step": last["ms"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"scan_block4_b{B}_d{d}", "B": B, "T": last["T"], "d": d,
+            "config": {"workload": last["workload"], "B": 4, "T": last["T"], "d": 2048,
                        "l2": "inputs larger than L2"},
             "roofline": {"kernel": "scan_kernel", "bound": "hbm", "achieved": last["achieved_GBs"], "peak": hbm,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": last["frac"], "traffic": None},
@@ -427,13 +655,14 @@ def run_scan(args):
 def run_varlen(args, w):
     """Packed ragged sequences: the workload's B*T steps repacked into sequences whose lengths are
     drawn (seeded) uniformly from [T/8, 2T), the last one cut to fit; the same inputs, each
-    sequence from s0 = 0.  A step is the input-projection GEMM, K fixed Newton iterations and the
+    sequence from s0 = 0.  A step is the input-projection GEMM, the Newton solve (to tolerance, or K fixed) and the
     backward, all through the packed entry points."""
     import torch
     from nonlinear_rnn_pararnn_b200 import _lib, api
     _, rank, _ = _dist()
     dev = torch.device("cuda", 0)
-    K = args.newton_iters
+    tol_mode = args.newton_mode == "tol"
+    K = w.max_iters if tol_mode else args.newton_iters
     total = w.B * w.T
     rng = np.random.default_rng(7)
     lengths = []
@@ -460,8 +689,8 @@ def run_varlen(args, w):
         api.preact_gemm(x[None], Wx, bias, P=P)
         if ev is not None:
             ev[0].record()
-        api.newton_forward_varlen(P[0], R, s0, cu, forget=w.forget, max_iters=K, fixed=True, tol=w.tol, S=S,
-                                  stats=stats, ws=ws_f)
+        api.newton_forward_varlen(P[0], R, s0, cu, forget=w.forget, max_iters=K, fixed=not tol_mode, tol=w.tol, S=S,
+                                  stats=stats, ws=ws_f, guess_sweeps=args.guess_sweeps)
         if ev is not None:
             ev[1].record()
         api.newton_backward_varlen(x, Wx, P[0], R, s0, cu, S, dH, forget=w.forget, out=grads, ws=ws_b)
@@ -477,22 +706,24 @@ def run_varlen(args, w):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    newton_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps / K
+    newton_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
     hbm, peak_kind = _peaks()
-    nbytes = total * w.d_h * (32 + 48 * (K - 1)) / K
-    gbs = nbytes / (newton_ms / 1e3) / 1e9
     st = api.read_stats(stats)
+    nbytes = total * w.d_h * solve_bytes_per_elem(st["iters"], args.guess_sweeps)
+    gbs = nbytes / (newton_ms / 1e3) / 1e9
     line = {"metric": METRIC + ", packed ragged sequences", "value": total * w.d_h / (ms / 1e3), "unit": UNIT,
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": f"{w.name}_packed", "total_T": total, "n_seq": n_seq,
                        "lengths": f"uniform integers in [{max(1, w.T // 8)}, {2 * w.T}), seed 7, last cut to fit",
-                       "d_in": w.d_in, "d_h": w.d_h, "x_dtype": w.dtype, "forget": w.forget, "newton_iters": K,
-                       "newton_mode": "fixed", "l2": "inputs larger than L2"},
-            "roofline": {"kernel": "newton_iter (packed)", "bound": "hbm", "achieved": gbs, "peak": hbm,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm, "traffic": None,
-                         "avg_launch_ms": newton_ms},
-            "newton_stats": {"iters": st["iters"], "error": st["error"]}}
+                       "d_in": w.d_in, "d_h": w.d_h, "x_dtype": w.dtype, "forget": w.forget, "newton_max_iters": K,
+                       "newton_mode": args.newton_mode, "guess_sweeps": args.guess_sweeps,
+                       "l2": "inputs larger than L2"},
+            "roofline": {"kernel": "newton solve, packed (guess_kernel x (1 + sweeps) + newton_iter x iters)",
+                         "bound": "hbm",
+                         "achieved": gbs, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": None, "solve_ms": newton_ms},
+            "newton_stats": {"iters": st["iters"], "converged": st["converged"], "error": st["error"]}}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -558,7 +789,7 @@ def run_decode(args, w):
 def run_block(args, w):
     """The trunk layer's forward (RMSNorm -> cell -> residual -> RMSNorm -> SwiGLU -> residual) at the
     workload's B and T with d_model = d_h and d_ff = 4 d_model: one slstm_block_forward call per step
-    (7 launches + the Newton iterations), fixed K Newton iterations.  There is no single dominant
+    (7 launches + the Newton launches), the Newton solve to the workload's tolerance (or fixed K).  There is no single dominant
     kernel, so the roofline line compares the step with its floor: the three GEMMs' flops at the
     sustained bf16 tensor peak plus the Newton and norm kernels' algorithmic bytes at the HBM copy
     bandwidth; frac = floor / measured step time."""
@@ -566,7 +797,8 @@ def run_block(args, w):
     from nonlinear_rnn_pararnn_b200 import api
     _, rank, _ = _dist()
     dev = torch.device("cuda", 0)
-    K = args.newton_iters
+    tol_mode = args.newton_mode == "tol"
+    K = w.max_iters if tol_mode else args.newton_iters
     B, T, D = w.B, w.T, w.d_h
     F = 4 * D
     g = torch.Generator().manual_seed(w.seed)
@@ -585,27 +817,45 @@ def run_block(args, w):
     stats = api.new_stats(dev)
     wsb = api.block_workspace(B, T, D, F, dev)
 
-    def step():
-        api.block_forward(x, w1, Wx, bias, R, w2, W_gu, W_down, forget=w.forget, max_iters=K, fixed=True,
-                          y=y, S=S, stats=stats, ws=wsb)
+    dY = torch.randn(B, T, D, generator=g).to(dev)
+    grads = {"dx": torch.empty(B, T, D, device=dev), "dnorm1_w": torch.empty(D, device=dev),
+             "dWx": torch.empty(4 * D, D, device=dev), "dbias": torch.empty(4, D, device=dev),
+             "dR": torch.empty(4, D, device=dev), "dnorm2_w": torch.empty(D, device=dev),
+             "dW_gu": torch.empty(2 * F, D, device=dev), "dW_down": torch.empty(D, F, device=dev)}
+    wsbb = torch.empty(int(api.load().slstm_block_backward_workspace_size(B, T, D, F)), dtype=torch.uint8,
+                       device=dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        api.block_forward(x, w1, Wx, bias, R, w2, W_gu, W_down, forget=w.forget, max_iters=K, fixed=not tol_mode,
+                          tol=w.tol, y=y, S=S, stats=stats, ws=wsb, guess_sweeps=args.guess_sweeps)
+        if ev is not None:
+            ev[1].record()
+        api.block_backward(x, w1, Wx, bias, R, w2, W_gu, W_down, S, dY, forget=w.forget, out=grads, ws=wsbb)
+        if ev is not None:
+            ev[2].record()
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev.index)
     time.sleep(0.25)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        step(evs[i])
     e1.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms_all = e0.elapsed_time(e1) / args.steps
+    ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    ms_bwd = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     st = api.read_stats(stats)
     M = B * T
     flops = 2.0 * M * D * (4 * D + 2 * F + F)
-    nbytes = M * D * (32 + 48 * (K - 1)) + M * D * (4 + 2) + M * D * (4 + 16 + 4 + 2)
+    nbytes = M * D * solve_bytes_per_elem(st["iters"], args.guess_sweeps) + M * D * (4 + 2) + M * D * (4 + 16 + 4 + 2)
     hbm, peak_kind = _peaks()
     try:
         with open(PEAKS_PATH) as f:
@@ -614,12 +864,19 @@ def run_block(args, w):
     except Exception:
         tflops, tkind = 1400.0, "fallback"
     floor_ms = flops / (tflops * 1e12) * 1e3 + nbytes / (hbm * 1e9) * 1e3
+    # the backward: eight GEMMs on the tensor cores (the forward's two recomputed, the five of the
+    # SwiGLU and norm gradients, the cell's dx and dW_x with the bf16 pair doubling their flops)
+    bwd_flops = 2.0 * M * D * (4 * D + 2 * F) + 2.0 * 2 * M * D * (F + F + 2 * F + 2 * F) + 2.0 * 2 * M * D * (4 * D) * 2
     line = {"metric": "trunk-layer forward tokens/s (B*T / s)", "value": M / (ms / 1e3), "unit": "tokens/s",
+            "fwd_bwd": {"value": M / (ms_all / 1e3), "unit": "tokens/s", "ms_per_step": ms_all,
+                        "ms_backward": ms_bwd, "backward_gemm_tflop": bwd_flops / 1e12,
+                        "backward_tensor_floor_ms": bwd_flops / (tflops * 1e12) * 1e3},
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "operand_dtype": "bf16 GEMM operands, fp32 accumulation, state and residual stream", "data": "synthetic",
             "config": {"workload": f"{w.name}_block", "B": B, "T": T, "d_model": D, "d_ff": F, "forget": w.forget,
-                       "newton_iters": K, "newton_mode": "fixed", "error": st["error"],
+                       "newton_max_iters": K, "newton_mode": args.newton_mode, "newton_iters": st["iters"],
+                       "converged": st["converged"], "error": st["error"],
                        "l2": "inputs larger than L2"},
             "roofline": {"kernel": "whole layer (3 GEMMs + Newton + norms)", "bound": "tensor+hbm",
                          "achieved": floor_ms, "peak": ms, "unit": "ms (floor vs measured)",
@@ -627,18 +884,18 @@ def run_block(args, w):
                          "tensor_peak_tflops": tflops, "tensor_peak_kind": tkind, "hbm_gbs": hbm,
                          "hbm_peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes},
             "clocks": clocks,
-            "gpu_launches": (5 + K) * args.steps}
+            "gpu_launches": (6 + K + 20) * args.steps}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
 
 
-# DRAM bytes (read + write) per element of B*T*d_h of the newton_iter launches (first, middle and
-# last iteration of a step), from one ncu capture of the training workload shortened to T = 2048
-# (the newton_iter capture summarised under profiles/).  The counters describe the kernel sources with
-# this SHA-256; any other build reports traffic null.  Traffic per element does not depend on T
-# (every tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "a1354d490b4ffca0023f55f55b9b12a31166f1d56c4ea2ff2b1e91f2ce16bad2", "first": 29.95, "middle": 46.33, "last": 46.35}
+# DRAM bytes (read + write) per element of B*T*d_h of the Newton solve's kernels, from one ncu
+# capture of the training workload shortened to T = 2048 (summarised under profiles/): the guess
+# launch, a refinement sweep and a Newton iteration that evaluates its residual.  The counters describe the kernel
+# sources with this SHA-256; any other build reports traffic null.  Traffic per element does not
+# depend on T (every tile moves the same bytes), so it scales to a full launch by the element count.
+NEWTON_TRAFFIC = {"sources_sha256": None, "guess": None, "sweep": None, "iter": None}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
@@ -651,13 +908,21 @@ def newton_sources_sha256() -> str:
     return h.hexdigest()
 
 
-def newton_traffic_bytes(elems: int, K: int):
-    """Measured DRAM bytes of one Newton launch averaged over the K launches of a step, or None."""
-    if newton_sources_sha256() != NEWTON_TRAFFIC["sources_sha256"]:
-        return None
+def solve_bytes_per_elem(iters: int, sweeps: int) -> int:
+    """Algorithmic bytes per element of B*T*d_h of one Newton solve: the
+    decoupled guess reads P and writes S (32), a refinement sweep also reads
+    the previous guess's h (36), an iteration reads P and the old S and writes
+    S (48)."""
+    return 32 + 36 * sweeps + 48 * iters
+
+
+def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
+    """Measured DRAM bytes of one Newton solve (the guess, its sweeps and
+    `iters` iterations), or None when the counters are not for this build."""
     t = NEWTON_TRAFFIC
-    per = t["first"] if K == 1 else (t["first"] + t["middle"] * (K - 2) + t["last"]) / K
-    return per * elems
+    if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
+        return None
+    return (t["guess"] + t["sweep"] * sweeps + t["iter"] * iters) * elems
 
 
 def main(argv=None):
@@ -666,9 +931,15 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=ORDER)
+    ap.add_argument("--newton-mode", default="tol", choices=["tol", "fixed"],
+                    help="tol: Newton to the workload's tolerance (its cap as max_iters); fixed: --newton-iters")
     ap.add_argument("--newton-iters", type=int, default=4)
+    ap.add_argument("--guess-sweeps", type=int, default=2,
+                    help="refinement sweeps of the decoupled initial guess (the library's Python default)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the long-sequence forward and the scan sweep that the default line carries")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-lanes", type=int, default=40)
+    ap.add_argument("--cpu-lanes", type=int, default=16)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen", "decode", "block"],

@@ -47,6 +47,12 @@
  *     convergence, divergence, bounded-wait timeouts) are written to the
  *     device-side stats record and read by the caller after synchronising.
  *   - No call aborts, traps or throws.
+ *   - Tiles hand scan carries to one another through the workspace with
+ *     bounded waits.  A wait that expires (it should never happen; it means
+ *     a tile was not scheduled within the limit) makes the carry it waited
+ *     for NaN, so every output that depends on it is NaN instead of silently
+ *     wrong, and sets a nonzero error word in the workspace.
+ *     slstm_newton_forward also reports it as SLSTM_ERR_TIMEOUT in its stats.
  *   - Sizes: 1 <= B <= 65535, 1 <= T, 1 <= d_in, d_h, d <= 2^20, B*T < 2^31
  *     and B * ceil(T/32) * ceil(max(d_in, d_h)/32) < 2^31.
  */
@@ -81,20 +87,26 @@ typedef enum {
     SLSTM_OP_SCAN_BLOCK4 = 2,
     SLSTM_OP_NEWTON_BACKWARD = 3,
     SLSTM_OP_NEWTON_FORWARD_VARLEN = 4,   /* B = number of sequences, T = total packed length */
-    SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5   /* B = number of sequences, T = total packed length */
+    SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5,  /* B = number of sequences, T = total packed length */
+    SLSTM_OP_NEWTON_BACKWARD_HEAD = 6,    /* sized for the largest head width, SLSTM_MAX_HEAD_DIM */
+    SLSTM_OP_CONTEXT_PARALLEL = 7         /* one rank's time slice: T = the slice's length */
 } slstm_op;
 
 #define SLSTM_MAX_ITERS 65536     /* largest accepted max_iters              */
+#define SLSTM_MAX_HEAD_DIM 32     /* largest head width of the head-mixing calls */
+#define SLSTM_MAX_GUESS_SWEEPS 64 /* largest guess_sweeps                       */
 #define SLSTM_STATS_HISTORY 64    /* residual history kept in the stats record */
 
 /* scan_block4 flags */
 #define SLSTM_SCAN_REVERSE_T 1
+#define SLSTM_SCAN_DEBUG_WITHHOLD 2   /* fault injection, see scan_block4 */
 
 /*
  * Newton solver settings ("pararnn-torch structure", "Current surface":
  * NewtonConfig(max_iters), residual early stop, fixed-K compile-safe preset).
- *   max_iters   1..SLSTM_MAX_ITERS: iteration cap (tolerance mode) or the
- *               exact iteration count (fixed mode).
+ *   max_iters   1..SLSTM_MAX_ITERS (0 allowed with SLSTM_INIT_DECOUPLED):
+ *               iteration cap (tolerance mode) or the exact iteration count
+ *               (fixed mode).
  *   fixed_iters 0: stop at the first iteration whose new iterate meets tol;
  *               1: run exactly max_iters iterations.
  *   tol         tolerance of the stopping test (residual_mode), taken over
@@ -121,14 +133,20 @@ typedef enum {
  *               SLSTM_INIT_DECOUPLED (0): the trajectory of the cell with
  *               its gates blind to h_{t-1} (R taken as 0: z, o, log i, log f
  *               from P alone, c, n, m recurring exactly), computed by an
- *               associative scan in one launch that reads P and writes S.
- *               In tolerance mode the guess's own residual is tested first
- *               and a guess that meets the test ends the solve after 0
- *               iterations.  From this guess the solve converges in a few
- *               iterations on long sequences where the zero guess overflows;
+ *               associative scan in one launch that reads P and writes S,
+ *               then refined by guess_sweeps fixed-point sweeps (each a
+ *               launch of the same scan whose gates see R h_{t-1} of the
+ *               previous guess; it reads P and h, writes S).  From this
+ *               guess the solve converges in a few iterations on long
+ *               sequences where the zero guess overflows.  In tolerance mode
+ *               the first iteration records the guess's residual
+ *               (stats.init_max_*); max_iters may then be 0, which returns
+ *               the guess itself;
  *               SLSTM_INIT_ZERO: S = 0 at every step;
- *               SLSTM_INIT_GIVEN: S holds the guess on entry (warm start;
- *               its residual is not tested, at least one iteration runs).
+ *               SLSTM_INIT_GIVEN: S holds the guess on entry (warm start).
+ *               The stopping test starts with iteration 1 in every case.
+ *   guess_sweeps  0..SLSTM_MAX_GUESS_SWEEPS refinement sweeps of the
+ *               decoupled guess (ignored by the other inits).
  *   residual_mode  the stopping test: SLSTM_RESIDUAL_SCALED (0),
  *               max |F| / (1 + |s|) <= tol; SLSTM_RESIDUAL_RAW, max|F| <= tol
  *               (the pages' own norm).  Both maxima are recorded either way.
@@ -149,6 +167,7 @@ typedef struct {
     int carry_mode;
     int init;
     int residual_mode;
+    int guess_sweeps;
 } slstm_newton_config;
 
 /*
@@ -163,9 +182,9 @@ typedef struct {
  *                produced by iteration k (max over every element), for the
  *                last min(iters, 64) iterations.  In fixed mode only the final
  *                iteration evaluates its residual; the others hold -1.
- *   init_max_abs_F, init_max_scaled_F   residual of the initial guess when
- *                it was tested (SLSTM_INIT_DECOUPLED in tolerance mode),
- *                else -1.
+ *   init_max_abs_F, init_max_scaled_F   residual of the initial guess,
+ *                recorded by the first iteration (SLSTM_INIT_DECOUPLED in
+ *                tolerance mode), else -1.
  */
 typedef struct {
     int iters;
@@ -234,7 +253,15 @@ int slstm_newton_forward(const float *P, const float *R, const float *s0, float 
  *   b   (B, T, 4, d) fp32
  *   y0  (B, 4, d) fp32, or NULL for zeros
  *   y   (B, T, 4, d) fp32 output; may not alias A or b
- * Composition is in fp32.
+ * Composition is in fp32.  The reverse mode pairs A_t^T with b_t at the same
+ * index t; the map that carries y_{t+1} back to step t is the one stored at
+ * t (a deliberate reading: the caller stores, at step t, the transpose it
+ * wants applied there).
+ * flags may also hold SLSTM_SCAN_DEBUG_WITHHOLD (tests only, needs T > 64):
+ * the tile of steps 32..63 (in processing order) of batch row 0, features
+ * 0..31 withholds its carry; the next tile's bounded wait (20 ms in this
+ * mode) expires, and the outputs of those features from step 64 (in
+ * processing order) on are NaN.  The rest is computed as usual.
  */
 int scan_block4(const float *A, const float *b, const float *y0, float *y, int B, int T, int d,
                 int flags, void *ws, size_t ws_bytes, slstm_stream_t stream);
@@ -344,6 +371,99 @@ int slstm_newton_backward_varlen(const void *x, const void *Wx, int dtype, const
                                  const float *dH, float *dx, float *dWx, float *dR, float *db, float *ds0,
                                  int forget, int total_T, int d_in, int d_h, void *ws, size_t ws_bytes,
                                  slstm_stream_t stream);
+
+/*
+ * Time context parallel ("sLSTM in this library", section "Tensor parallel":
+ * context parallel splits time).  Rank r of n holds the steps of its time
+ * slice of every sequence: P and S are (B, T, 4, d_h) with T the slice's
+ * length (it may differ between ranks; B and d_h may not).  A solve keeps the
+ * single-GPU call's arithmetic, with every scan split into three phases:
+ * each rank composes its slice into one map (…_run / …_map), the caller
+ * gathers every rank's map on every rank (an all-gather: NCCL over NVLink in
+ * the Python layer; nothing here communicates), and each rank enters its
+ * slice through the maps of the ranks before it (…_apply).  The solve:
+ *   guess:  slstm_cp_guess_run(sweep 0) -> gather runs -> slstm_cp_guess_apply(sweep 0)
+ *   each refinement sweep: gather every rank's last state of the current
+ *           guess, then slstm_cp_guess_run(sweep 1) -> gather runs ->
+ *           slstm_cp_guess_apply(sweep 1)
+ *   each Newton iteration: gather last states, slstm_cp_newton_map ->
+ *           gather maps -> slstm_cp_newton_apply, whose stats record
+ *           (max_abs_F[0], max_scaled_F[0]) holds the slice's residual
+ *           maxima of the new iterate; the caller takes the maximum over
+ *           ranks for the stopping test.
+ * Arguments:
+ *   s_before  (B, 4, d_h) the current iterate's (or, for a sweep, the
+ *             previous guess's) state just before the slice: the last state
+ *             of rank r - 1, or the sequences' s0 on rank 0 (NULL: zero)
+ *   s0        (B, 4, d_h) the sequences' initial state (NULL: zero); only its
+ *             value on the ranks' apply matters
+ *   run       (B, 5, d_h) output: the slice's run of the guess's monoid
+ *             (log f sum, stabiliser, u, v, last output gate)
+ *   runs      (n, B, 5, d_h) every rank's run in rank order (ranks before
+ *             `rank` are read; may be NULL on rank 0)
+ *   map       (B, 20, d_h) output: the slice's affine map of the linear
+ *             solve (4x4 row-major, then the offset)
+ *   maps      (n, B, 20, d_h) every rank's map in rank order
+ *   cfg       tol and residual_mode are used (the rest is fixed: one
+ *             iteration from the given iterate)
+ * slstm_cp_newton_map and slstm_cp_newton_apply of one iteration share the
+ * workspace (the apply reuses the tile maps the map call left there).
+ * Workspace: slstm_workspace_size(SLSTM_OP_CONTEXT_PARALLEL, B, T, 0, d_h).
+ */
+int slstm_cp_guess_run(const float *P, const float *R, const float *s_before, const float *S, int sweep,
+                       int forget, float *run, int B, int T, int d_h, void *ws, size_t ws_bytes,
+                       slstm_stream_t stream);
+
+int slstm_cp_guess_apply(const float *P, const float *R, const float *s0, const float *s_before,
+                         const float *runs, int rank, float *S, int sweep, int forget, int B, int T, int d_h,
+                         void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+int slstm_cp_newton_map(const float *P, const float *R, const float *s_before, const float *S, int forget,
+                        float *map, int B, int T, int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+int slstm_cp_newton_apply(const float *P, const float *R, const float *s_before, const float *maps, int rank,
+                          float *S, const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
+                          int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+/*
+ * Head mixing ("sLSTM in this library", section "Cell", row 'head': Beck's
+ * block-diagonal R of shape (4, n_heads, d_head, d_head), n_heads d_head =
+ * d_h; the factorised Newton, reverse pass and packed VJP that never form
+ * the dense (4 d_head)^2 Jacobian, fused for d_head <= 32).  The recurrent
+ * input of gate g of feature i of head hd is
+ *   sum_k R_head[g][hd][i][k] h_{t-1}[hd d_head + k]
+ * in place of diag mixing's R[g][j] h_{t-1}[j]; everything else is the cell
+ * of slstm_newton_forward.  R_head is (4, n_heads, d_head, d_head) fp32,
+ * 1 <= d_head <= SLSTM_MAX_HEAD_DIM and d_head divides d_h; other tensors and
+ * conventions as the diag calls.  One warp serves one (batch row, head):
+ * the Jacobian's h column is applied as G (R_head delta_h) (G = ds/da per
+ * feature), so the Newton linear solve runs as a recurrence of these
+ * matrix-vector products over time, in parallel over batch rows and heads.
+ *
+ * slstm_sequential_step_head: S_t = f(S_{t-1}, P_t) stepped over T_steps.
+ * slstm_newton_forward_head: the Newton solve; cfg as slstm_newton_forward
+ *   (debug_fault and guess_sweeps must be 0; carry_mode is ignored).  With
+ *   SLSTM_INIT_DECOUPLED the guess is the same decoupled trajectory (it does
+ *   not depend on the mixing); its residual is not recorded.  Workspace: slstm_workspace_size(
+ *   SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h).
+ * slstm_newton_backward_head: gradients of L = sum dH * h as
+ *   slstm_newton_backward, with dR_head (4, n_heads, d_head, d_head) in
+ *   place of dR.  Workspace: slstm_workspace_size(
+ *   SLSTM_OP_NEWTON_BACKWARD_HEAD, B, T, d_in, d_h).
+ * Errors: SLSTM_ERR_INVALID_ARG for a d_head outside 1..32 or not dividing
+ * d_h, and as the diag calls otherwise.
+ */
+int slstm_sequential_step_head(const float *P, const float *R_head, const float *s0, float *S, int B,
+                               int T_steps, int d_h, int d_head, int forget, slstm_stream_t stream);
+
+int slstm_newton_forward_head(const float *P, const float *R_head, const float *s0, float *S,
+                              const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
+                              int d_h, int d_head, void *ws, size_t ws_bytes, slstm_stream_t stream);
+
+int slstm_newton_backward_head(const void *x, const void *Wx, int dtype, const float *P, const float *R_head,
+                               const float *s0, const float *S, const float *dH, float *dx, float *dWx,
+                               float *dR_head, float *db, float *ds0, int forget, int B, int T, int d_in,
+                               int d_h, int d_head, void *ws, size_t ws_bytes, slstm_stream_t stream);
 
 /*
  * The trunk layer, forward ("sLSTM in this library", section "Stacking":

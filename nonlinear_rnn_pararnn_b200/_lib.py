@@ -28,9 +28,14 @@ SLSTM_OP_SCAN_BLOCK4 = 2
 SLSTM_OP_NEWTON_BACKWARD = 3
 SLSTM_OP_NEWTON_FORWARD_VARLEN = 4
 SLSTM_OP_NEWTON_BACKWARD_VARLEN = 5
+SLSTM_OP_NEWTON_BACKWARD_HEAD = 6
+SLSTM_OP_CONTEXT_PARALLEL = 7
+SLSTM_MAX_HEAD_DIM = 32
+SLSTM_MAX_GUESS_SWEEPS = 64
 SLSTM_MAX_ITERS = 65536
 SLSTM_STATS_HISTORY = 64
 SLSTM_SCAN_REVERSE_T = 1
+SLSTM_SCAN_DEBUG_WITHHOLD = 2
 SLSTM_INIT_DECOUPLED = 0
 SLSTM_INIT_ZERO = 1
 SLSTM_INIT_GIVEN = 2
@@ -42,7 +47,8 @@ SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 class NewtonConfig(ctypes.Structure):
     _fields_ = [("max_iters", ctypes.c_int), ("fixed_iters", ctypes.c_int), ("tol", ctypes.c_float),
                 ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int),
-                ("carry_mode", ctypes.c_int), ("init", ctypes.c_int), ("residual_mode", ctypes.c_int)]
+                ("carry_mode", ctypes.c_int), ("init", ctypes.c_int), ("residual_mode", ctypes.c_int),
+                ("guess_sweeps", ctypes.c_int)]
 
 
 STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY + 2 * 4
@@ -60,6 +66,16 @@ SIGNATURES = {
     "scan_block4": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
     "scan_block4_noalloc": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
     "slstm_sequential_step": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),
+    "slstm_sequential_step_head": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _I, _V]),
+    "slstm_cp_guess_run": (_I, [_V, _V, _V, _V, _I, _I, _V, _I, _I, _I, _V, _Z, _V]),
+    "slstm_cp_guess_apply": (_I, [_V, _V, _V, _V, _V, _I, _V, _I, _I, _I, _I, _I, _V, _Z, _V]),
+    "slstm_cp_newton_map": (_I, [_V, _V, _V, _V, _I, _V, _I, _I, _I, _V, _Z, _V]),
+    "slstm_cp_newton_apply": (_I, [_V, _V, _V, _V, _I, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _V, _Z,
+                                   _V]),
+    "slstm_newton_forward_head": (_I, [_V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _I, _V, _Z,
+                                       _V]),
+    "slstm_newton_backward_head": (_I, [_V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I,
+                                        _I, _V, _Z, _V]),
     "slstm_newton_backward": (_I, [_V, _V, _I, _V, _V, _V, _V, _V, _V, _V, _V, _V, _V, _I, _I, _I, _I, _I,
                                    _V, _Z, _V]),
     "slstm_newton_forward_varlen": (_I, [_V, _V, _V, _V, _I, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _V, _Z,

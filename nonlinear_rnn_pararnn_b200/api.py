@@ -74,13 +74,20 @@ _INIT = {"decoupled": _lib.SLSTM_INIT_DECOUPLED, "zero": _lib.SLSTM_INIT_ZERO, "
 _RESIDUAL = {"scaled": _lib.SLSTM_RESIDUAL_SCALED, "raw": _lib.SLSTM_RESIDUAL_RAW}
 
 
+# refinement sweeps of the decoupled guess used when the caller names none
+DEFAULT_GUESS_SWEEPS = 2
+
+
 def newton_config(max_iters: int, fixed: bool, tol: float, forget, debug_fault: int = 0, wait_limit_us: int = 0,
-                  carry_mode: int = 0, init="decoupled", residual_mode="scaled") -> NewtonConfig:
-    """The C ABI's slstm_newton_config.  init: "decoupled" (default), "zero"
-    or "given" (S holds the guess on entry); residual_mode: "scaled" or "raw"."""
+                  carry_mode: int = 0, init="decoupled", residual_mode="scaled",
+                  guess_sweeps: int = DEFAULT_GUESS_SWEEPS) -> NewtonConfig:
+    """The C ABI's slstm_newton_config.  init: "decoupled" (default; with
+    guess_sweeps refinement sweeps), "zero" or "given" (S holds the guess on
+    entry); residual_mode: "scaled" or "raw"."""
     return NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
                         int(wait_limit_us), int(carry_mode), _INIT[init] if isinstance(init, str) else int(init),
-                        _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode))
+                        _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode),
+                        int(guess_sweeps))
 
 
 def new_stats(device=None) -> torch.Tensor:
@@ -105,7 +112,8 @@ def read_stats(stats: torch.Tensor) -> dict:
 def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
                    max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
                    stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
-                   wait_limit_us: int = 0, carry_mode: int = 0, init="decoupled", residual_mode="scaled"):
+                   wait_limit_us: int = 0, carry_mode: int = 0, init="decoupled", residual_mode="scaled",
+                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS):
     """Newton solve; returns (S, stats) with stats a device record (see read_stats).
     With init="given", S must be passed and holds the initial guess."""
     B, T, four, d_h = P.shape
@@ -122,7 +130,8 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
-    cfg = newton_config(max_iters, fixed, tol, forget, debug_fault, wait_limit_us, carry_mode, init, residual_mode)
+    cfg = newton_config(max_iters, fixed, tol, forget, debug_fault, wait_limit_us, carry_mode, init, residual_mode,
+                        guess_sweeps)
     check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
                                                               ctypes.byref(cfg), _ptr(stats), B, T, d_h,
                                                               _ptr(ws), ws.numel(), _stream()))
@@ -240,7 +249,8 @@ def _need_cu(cu: torch.Tensor, n_seq: int):
 def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu_seqlens: torch.Tensor, *,
                           forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
                           S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None,
-                          carry_mode: int = 0, init="decoupled", residual_mode="scaled"):
+                          carry_mode: int = 0, init="decoupled", residual_mode="scaled",
+                          guess_sweeps: int = DEFAULT_GUESS_SWEEPS):
     """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
     cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats)."""
     total_T, four, d_h = P.shape
@@ -257,7 +267,7 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
-    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode)
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode, guess_sweeps)
     check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
         _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
         _ptr(ws), ws.numel(), _stream()))
@@ -318,7 +328,7 @@ def block_workspace(B: int, T: int, d_model: int, d_ff: int, device=None) -> tor
 def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sigmoid", max_iters: int = 8,
                   fixed: bool = False, tol: float = 1e-5, eps: float = 1e-6, y: torch.Tensor = None,
                   S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None, carry_mode: int = 0,
-                  init="decoupled", residual_mode="scaled"):
+                  init="decoupled", residual_mode="scaled", guess_sweeps: int = DEFAULT_GUESS_SWEEPS):
     """The trunk layer's forward; returns (y, S, stats).  x (B, T, d_model)
     fp32; Wx, W_gu (interleave_gate_up), W_down bf16."""
     B, T, D = x.shape
@@ -341,7 +351,7 @@ def block_forward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, *, forget="sig
         stats = new_stats(x.device)
     if ws is None:
         ws = block_workspace(B, T, D, F, x.device)
-    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode)
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode, guess_sweeps)
     check("slstm_block_forward", load().slstm_block_forward(
         _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(y),
         _ptr(S), ctypes.byref(cfg), _ptr(stats), B, T, D, F, float(eps), _ptr(ws), ws.numel(), _stream()))
@@ -381,4 +391,85 @@ def block_backward(x, norm1_w, Wx, bias, R, norm2_w, W_gu, W_down, S, dY, *, for
         _ptr(x), _ptr(norm1_w), _ptr(Wx), _ptr(bias), _ptr(R), _ptr(norm2_w), _ptr(W_gu), _ptr(W_down), _ptr(S),
         _ptr(dY), *[_ptr(out[k]) for k in names], forget_code(forget), B, T, D, F, float(eps), _ptr(ws), ws.numel(),
         _stream()))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# head mixing: block-diagonal R (4, n_heads, d_head, d_head)
+# ---------------------------------------------------------------------------
+def _head_dims(R_head: torch.Tensor, d_h: int):
+    if R_head.dim() != 4 or R_head.shape[0] != 4 or R_head.shape[2] != R_head.shape[3]:
+        raise ValueError(f"R_head must be (4, n_heads, d_head, d_head), got {tuple(R_head.shape)}")
+    H, dh = R_head.shape[1], R_head.shape[2]
+    if H * dh != d_h:
+        raise ValueError(f"n_heads * d_head = {H * dh} != d_h = {d_h}")
+    _need(R_head, "R_head", (4, H, dh, dh))
+    return H, dh
+
+
+def sequential_step_head(P: torch.Tensor, R_head: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
+                         S: torch.Tensor = None) -> torch.Tensor:
+    B, T, four, d_h = P.shape
+    _need(P, "P", (B, T, 4, d_h))
+    H, dh = _head_dims(R_head, d_h)
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    if S is None:
+        S = torch.empty_like(P)
+    _need(S, "S", (B, T, 4, d_h))
+    check("slstm_sequential_step_head", load().slstm_sequential_step_head(
+        _ptr(P), _ptr(R_head), _ptr(s0), _ptr(S), B, T, d_h, dh, forget_code(forget), _stream()))
+    return S
+
+
+def newton_forward_head(P: torch.Tensor, R_head: torch.Tensor, s0: torch.Tensor = None, *, forget="sigmoid",
+                        max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
+                        stats: torch.Tensor = None, ws: torch.Tensor = None, init="decoupled", residual_mode="scaled"):
+    """Newton solve with head mixing; returns (S, stats)."""
+    B, T, four, d_h = P.shape
+    _need(P, "P", (B, T, 4, d_h))
+    H, dh = _head_dims(R_head, d_h)
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    if S is None:
+        if init == "given":
+            raise ValueError("init='given' needs S holding the initial guess")
+        S = torch.empty_like(P)
+    _need(S, "S", (B, T, 4, d_h))
+    if stats is None:
+        stats = new_stats(P.device)
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, 0, init, residual_mode, 0)
+    check("slstm_newton_forward_head", load().slstm_newton_forward_head(
+        _ptr(P), _ptr(R_head), _ptr(s0), _ptr(S), ctypes.byref(cfg), _ptr(stats), B, T, d_h, dh, _ptr(ws),
+        ws.numel(), _stream()))
+    return S, stats
+
+
+def newton_backward_head(x, Wx, P, R_head, s0, S, dH, *, forget="sigmoid", out: dict = None,
+                         ws: torch.Tensor = None):
+    """Gradients of sum(dH * h) with head mixing; returns dict dx, dWx, dR_head, db, ds0."""
+    B, T, d_in = x.shape
+    d_h = Wx.shape[0] // 4
+    dt = x.dtype
+    _need(x, "x", (B, T, d_in), dt)
+    _need(Wx, "Wx", (4 * d_h, d_in), dt)
+    _need(P, "P", (B, T, 4, d_h))
+    H, dh = _head_dims(R_head, d_h)
+    if s0 is not None:
+        _need(s0, "s0", (B, 4, d_h))
+    _need(S, "S", (B, T, 4, d_h))
+    _need(dH, "dH", (B, T, d_h))
+    dev = x.device
+    if out is None:
+        out = {"dx": torch.empty(B, T, d_in, device=dev), "dWx": torch.empty(4 * d_h, d_in, device=dev),
+               "dR_head": torch.empty(4, H, dh, dh, device=dev), "db": torch.empty(4, d_h, device=dev),
+               "ds0": torch.empty(B, 4, d_h, device=dev)}
+    if ws is None:
+        ws = workspace(_lib.SLSTM_OP_NEWTON_BACKWARD_HEAD, B, T, d_in, d_h, dev)
+    check("slstm_newton_backward_head", load().slstm_newton_backward_head(
+        _ptr(x), _ptr(Wx), _DTYPE[dt], _ptr(P), _ptr(R_head), _ptr(s0), _ptr(S), _ptr(dH), _ptr(out["dx"]),
+        _ptr(out["dWx"]), _ptr(out["dR_head"]), _ptr(out["db"]), _ptr(out.get("ds0")), forget_code(forget), B, T,
+        d_in, d_h, dh, _ptr(ws), ws.numel(), _stream()))
     return out

@@ -503,6 +503,16 @@ __global__ void sum_splits_kernel(const float *__restrict__ part, float *__restr
     out[i] = acc;
 }
 
+}  // namespace
+
+cudaError_t sum_splits(const float *part, float *out, long long n, int splits, cudaStream_t st)
+{
+    sum_splits_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(part, out, n, splits);
+    return cudaGetLastError();
+}
+
+namespace {
+
 // dR[g][j] and db[g][j]: sum of the per-tile partials over chunks and batch
 // rows, in a fixed order, accumulated in fp64.
 // One block per (entry e, group of 32 features); warp w sums the (chunk, b)

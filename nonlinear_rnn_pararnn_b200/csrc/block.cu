@@ -134,24 +134,46 @@ __global__ void __launch_bounds__(NORM_ROWS * 32) norm_bwd_kernel(const float *v
     }
 }
 
+// fp32 -> a pair of bf16 with v ~ hi + lo (|v - hi - lo| <= 2^-16 |v|), the
+// tensor-core operand form of an fp32 matrix.
+__global__ void __launch_bounds__(256) split_pair_kernel(const float *__restrict__ v, __nv_bfloat16 *__restrict__ hi,
+                                                         __nv_bfloat16 *__restrict__ lo, long long n)
+{
+    const long long q = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (q >= n) return;
+    const float x = v[q];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi[q] = h;
+    lo[q] = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
 // SwiGLU backward, one thread per (row m, hidden feature f): gv holds the
 // gate/up projections in the interleaved column order (gate of f at column
-// 64 (f / 32) + f % 32, up 32 columns later); da[m][f] = dL/da.  Writes
-// dL/dgate and dL/dup over gv and the product a = silu(gate) up over da.
-__global__ void __launch_bounds__(256) swiglu_bwd_kernel(float *gv, float *da, long long total, int F)
+// 64 (f / 32) + f % 32, up 32 columns later); da[m][f] = dL/da.  The
+// gradients of the gate and up projections go out as a bf16 pair in the same
+// column order (tensor-core A operands), the product a = silu(gate) up as
+// bf16, the forward's own rounding of that GEMM operand.
+__global__ void __launch_bounds__(256) swiglu_bwd_pair_kernel(const float *__restrict__ gv, const float *__restrict__ da,
+                                                              __nv_bfloat16 *__restrict__ dgv_hi,
+                                                              __nv_bfloat16 *__restrict__ dgv_lo,
+                                                              __nv_bfloat16 *__restrict__ a, long long total, int F)
 {
     const long long q = (long long)blockIdx.x * 256 + threadIdx.x;
     if (q >= total) return;
     const long long m = q / F;
     const int f = (int)(q - m * F);
-    float *row = gv + m * 2 * F;
-    const int cg = (f >> 5) * 64 + (f & 31);
-    const float g = row[cg], u = row[cg + 32], d = da[q];
-    const float sg = __fdividef(1.0f, 1.0f + __expf(-g));   // 0 once e^-g passes 2^126
+    const long long cg = m * 2 * F + (f >> 5) * 64 + (f & 31);
+    const float g = gv[cg], u = gv[cg + 32], d = da[q];
+    const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
     const float silu = g * sg;
-    row[cg] = d * u * sg * fmaf(g, 1.0f - sg, 1.0f);        // silu'(g) = s (1 + g (1 - s))
-    row[cg + 32] = d * silu;
-    da[q] = silu * u;
+    const float dg = d * u * sg * fmaf(g, 1.0f - sg, 1.0f);
+    const float du = d * silu;
+    const __nv_bfloat16 hg = __float2bfloat16_rn(dg), hu = __float2bfloat16_rn(du);
+    dgv_hi[cg] = hg;
+    dgv_lo[cg] = __float2bfloat16_rn(dg - __bfloat162float(hg));
+    dgv_hi[cg + 32] = hu;
+    dgv_lo[cg + 32] = __float2bfloat16_rn(du - __bfloat162float(hu));
+    a[q] = __float2bfloat16_rn(silu * u);
 }
 
 // Column sums of c (M x D) in a fixed order: chunk k of rows_per_chunk rows
@@ -185,40 +207,107 @@ struct BlockBwdLayout {
     __nv_bfloat16 *z1, *z2;   // (M, D) each
     float *P;                 // (M, 4D)
     float *u;                 // (M, D)
-    float *gv;                // (M, 2F): gate/up, then their gradients
-    float *da;                // (M, F): dL/da, then a
+    float *gv;                // (M, 2F): gate/up
+    float *da;                // (M, F): dL/da
+    __nv_bfloat16 *dy_hi, *dy_lo;     // (M, D): dY as a bf16 pair
+    __nv_bfloat16 *dgv_hi, *dgv_lo;   // (M, 2F): gate/up gradients as a bf16 pair
+    __nv_bfloat16 *a;                 // (M, F): silu(gate) up in bf16
+    float *wpart;             // split-K partial sums of the weight gradients
     float *dz2, *dz1;         // (M, D) each
     float *partial;           // (M / COLSUM_ROWS + 1, D)
     void *cell_ws;
+    int splits_down, splits_gu;
 };
 
-BlockBwdLayout block_bwd_layout(void *ws, int B, int T, int D, int F)
+// split-K count of a weight-gradient GEMM (M x N output, K = B*T rows, two A
+// parts): the count (up to 16) whose work items fill whole waves of the
+// persistent CTAs (128 x 256 output tiles) best.
+int block_wgrad_splits(int M, int N, int K)
+{
+    const long long tiles = ((long long)(M + 127) / 128) * ((N + 255) / 256);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                   cudaSuccess || sms < 1)
+        sms = 148;
+    int best = 1;
+    double best_eff = 0.0;
+    for (int want = 1; want <= 16; ++want) {
+        const int s = gemm_tc_splits(M, N, K, 2, want);
+        const long long work = tiles * s;
+        const double eff = (double)work / (double)(((work + sms - 1) / sms) * sms);
+        if (eff > best_eff + 0.02) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    return best;
+}
+
+// Byte offsets of the backward's buffers inside its workspace; `total` is
+// where the cell backward's own workspace starts.
+struct BlockBwdOffsets {
+    size_t err, z1, z2, P, u, gv, da, dy_hi, dy_lo, dgv_hi, dgv_lo, a, wpart, dz2, dz1, partial, total;
+    int splits_down, splits_gu;
+};
+
+BlockBwdOffsets block_bwd_offsets(int B, int T, int D, int F)
 {
     const size_t M = (size_t)B * T;
     const size_t chunks = (M + COLSUM_ROWS - 1) / COLSUM_ROWS;
+    BlockBwdOffsets o;
+    o.splits_down = block_wgrad_splits(D, F, (int)M);
+    o.splits_gu = block_wgrad_splits(2 * F, D, (int)M);
+    const size_t wpart = (size_t)(o.splits_down > o.splits_gu ? o.splits_down : o.splits_gu) * 2 * F * D;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off += al256(bytes);
+        return at;
+    };
+    o.err = take(256);
+    o.z1 = take(M * D * 2);
+    o.z2 = take(M * D * 2);
+    o.P = take(M * 4 * D * 4);
+    o.u = take(M * D * 4);
+    o.gv = take(M * 2 * F * 4);
+    o.da = take(M * F * 4);
+    o.dy_hi = take(M * D * 2);
+    o.dy_lo = take(M * D * 2);
+    o.dgv_hi = take(M * 2 * F * 2);
+    o.dgv_lo = take(M * 2 * F * 2);
+    o.a = take(M * F * 2);
+    o.wpart = take(wpart * 4);
+    o.dz2 = take(M * D * 4);
+    o.dz1 = take(M * D * 4);
+    o.partial = take(chunks * D * 4);
+    o.total = off;
+    return o;
+}
+
+BlockBwdLayout block_bwd_layout(void *ws, int B, int T, int D, int F)
+{
+    const BlockBwdOffsets o = block_bwd_offsets(B, T, D, F);
     char *p = static_cast<char *>(ws);
     BlockBwdLayout l;
-    l.err = reinterpret_cast<unsigned *>(p);
-    p += 256;
-    l.z1 = reinterpret_cast<__nv_bfloat16 *>(p);
-    p += al256(M * D * 2);
-    l.z2 = reinterpret_cast<__nv_bfloat16 *>(p);
-    p += al256(M * D * 2);
-    l.P = reinterpret_cast<float *>(p);
-    p += al256(M * 4 * D * 4);
-    l.u = reinterpret_cast<float *>(p);
-    p += al256(M * D * 4);
-    l.gv = reinterpret_cast<float *>(p);
-    p += al256(M * 2 * F * 4);
-    l.da = reinterpret_cast<float *>(p);
-    p += al256(M * F * 4);
-    l.dz2 = reinterpret_cast<float *>(p);
-    p += al256(M * D * 4);
-    l.dz1 = reinterpret_cast<float *>(p);
-    p += al256(M * D * 4);
-    l.partial = reinterpret_cast<float *>(p);
-    p += al256(chunks * D * 4);
-    l.cell_ws = p;
+    l.splits_down = o.splits_down;
+    l.splits_gu = o.splits_gu;
+    l.err = reinterpret_cast<unsigned *>(p + o.err);
+    l.z1 = reinterpret_cast<__nv_bfloat16 *>(p + o.z1);
+    l.z2 = reinterpret_cast<__nv_bfloat16 *>(p + o.z2);
+    l.P = reinterpret_cast<float *>(p + o.P);
+    l.u = reinterpret_cast<float *>(p + o.u);
+    l.gv = reinterpret_cast<float *>(p + o.gv);
+    l.da = reinterpret_cast<float *>(p + o.da);
+    l.dy_hi = reinterpret_cast<__nv_bfloat16 *>(p + o.dy_hi);
+    l.dy_lo = reinterpret_cast<__nv_bfloat16 *>(p + o.dy_lo);
+    l.dgv_hi = reinterpret_cast<__nv_bfloat16 *>(p + o.dgv_hi);
+    l.dgv_lo = reinterpret_cast<__nv_bfloat16 *>(p + o.dgv_lo);
+    l.a = reinterpret_cast<__nv_bfloat16 *>(p + o.a);
+    l.wpart = reinterpret_cast<float *>(p + o.wpart);
+    l.dz2 = reinterpret_cast<float *>(p + o.dz2);
+    l.dz1 = reinterpret_cast<float *>(p + o.dz1);
+    l.partial = reinterpret_cast<float *>(p + o.partial);
+    l.cell_ws = p + o.total;
     return l;
 }
 
@@ -232,34 +321,11 @@ cudaError_t colsum(const float *c, int M, int D, float *partial, float *out, cud
     return cudaGetLastError();
 }
 
-GemmDesc simt_desc(int M, int N, int K, const void *A, int adt, long long sam, long long sak, const void *Bm, int bdt,
-                   long long sbk, long long sbn, float *C)
-{
-    GemmDesc g;
-    g.M = M;
-    g.N = N;
-    g.K = K;
-    g.A = A;
-    g.a_dtype = adt;
-    g.sam = sam;
-    g.sak = sak;
-    g.B = Bm;
-    g.b_dtype = bdt;
-    g.sbk = sbk;
-    g.sbn = sbn;
-    g.bias = nullptr;
-    g.C = C;
-    return g;
-}
-
 }  // namespace
 
 size_t block_backward_workspace_bytes(int B, int T, int D, int F)
 {
-    const size_t M = (size_t)B * T;
-    const size_t chunks = (M + COLSUM_ROWS - 1) / COLSUM_ROWS;
-    return 256 + 2 * al256(M * D * 2) + al256(M * 4 * D * 4) + 3 * al256(M * D * 4) + al256(M * 2 * F * 4) +
-           al256(M * F * 4) + al256(chunks * D * 4) + backward_workspace_bytes(B, T, D, D);
+    return block_bwd_offsets(B, T, D, F).total + backward_workspace_bytes(B, T, D, D);
 }
 
 cudaError_t block_backward_launch(const float *x, const float *norm1_w, const void *Wx, const float *bias,
@@ -279,22 +345,38 @@ cudaError_t block_backward_launch(const float *x, const float *norm1_w, const vo
     if ((e = gemm_tc_bf16(l.z1, Wx, bias, l.P, M, 4 * D, D, l.err, st)) != cudaSuccess) return e;
     block_norm_kernel<true><<<rows, NORM_ROWS * 32, 0, st>>>(x, S, norm2_w, l.u, l.z2, M, D, eps);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // gate/up projections (interleaved columns) and dL/da = dY W_down
-    if ((e = gemm_simt(simt_desc(M, 2 * F, D, l.z2, SLSTM_BF16, D, 1, W_gu, SLSTM_BF16, 1, D, l.gv), st)) !=
+    // every GEMM below runs on the tcgen05 tensor cores; fp32 operands enter
+    // as a bf16 pair (hi + lo) on the A side
+    // gate/up projections (interleaved columns): gv = z2 W_gu^T
+    if ((e = gemm_tc_bf16(l.z2, W_gu, nullptr, l.gv, M, 2 * F, D, l.err, st)) != cudaSuccess) return e;
+    // dL/da = dY W_down (W_down (D, F) is an MN-major B operand)
+    const long long nmd = (long long)M * D;
+    split_pair_kernel<<<(unsigned)((nmd + 255) / 256), 256, 0, st>>>(dY, l.dy_hi, l.dy_lo, nmd);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = gemm_tc_bf16_ex(l.dy_hi, l.dy_lo, D, false, W_down, F, true, nullptr, l.da, M, F, D, 1, l.err, st)) !=
         cudaSuccess)
-        return e;
-    if ((e = gemm_simt(simt_desc(M, F, D, dY, SLSTM_F32, D, 1, W_down, SLSTM_BF16, F, 1, l.da), st)) != cudaSuccess)
         return e;
     const long long total = (long long)M * F;
-    swiglu_bwd_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(l.gv, l.da, total, F);
+    swiglu_bwd_pair_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(l.gv, l.da, l.dgv_hi, l.dgv_lo, l.a,
+                                                                             total, F);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // dW_down = dY^T a, dz2 = dgv W_gu, dW_gu = dgv^T z2
-    if ((e = gemm_simt(simt_desc(D, F, M, dY, SLSTM_F32, 1, D, l.da, SLSTM_F32, F, 1, dW_down), st)) != cudaSuccess)
+    // dW_down = dY^T a: A = the dY pair read MN-major (B*T, D), B = a (B*T, F)
+    // MN-major; split over B*T, partial sums added in order
+    if ((e = gemm_tc_bf16_ex(l.dy_hi, l.dy_lo, D, true, l.a, F, true, nullptr, l.wpart, D, F, M, l.splits_down,
+                             l.err, st)) != cudaSuccess)
         return e;
-    if ((e = gemm_simt(simt_desc(M, D, 2 * F, l.gv, SLSTM_F32, 2LL * F, 1, W_gu, SLSTM_BF16, D, 1, l.dz2), st)) !=
+    if ((e = sum_splits(l.wpart, dW_down, (long long)D * F, gemm_tc_splits(D, F, M, 2, l.splits_down), st)) !=
         cudaSuccess)
         return e;
-    if ((e = gemm_simt(simt_desc(2 * F, D, M, l.gv, SLSTM_F32, 1, 2LL * F, l.z2, SLSTM_BF16, D, 1, dW_gu), st)) !=
+    // dz2 = dgv W_gu: A = the dgv pair (B*T, 2F) K-major, W_gu (2F, D) MN-major
+    if ((e = gemm_tc_bf16_ex(l.dgv_hi, l.dgv_lo, 2 * F, false, W_gu, D, true, nullptr, l.dz2, M, D, 2 * F, 1, l.err,
+                             st)) != cudaSuccess)
+        return e;
+    // dW_gu = dgv^T z2: A = the dgv pair read MN-major, z2 (B*T, D) MN-major
+    if ((e = gemm_tc_bf16_ex(l.dgv_hi, l.dgv_lo, 2 * F, true, l.z2, D, true, nullptr, l.wpart, 2 * F, D, M,
+                             l.splits_gu, l.err, st)) != cudaSuccess)
+        return e;
+    if ((e = sum_splits(l.wpart, dW_gu, 2LL * F * D, gemm_tc_splits(2 * F, D, M, 2, l.splits_gu), st)) !=
         cudaSuccess)
         return e;
     // du = dY + RMSNorm2 backward (into dx), dnorm2_w

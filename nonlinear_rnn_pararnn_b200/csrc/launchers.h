@@ -22,7 +22,9 @@ struct NewtonSlot {
 struct NewtonCtrl {
     unsigned done;
     unsigned error;
-    unsigned pad[14];
+    unsigned init_raw;      // residual of the initial guess (float bits), recorded by the first iteration
+    unsigned init_scaled;
+    unsigned pad[12];
     NewtonSlot slot[2];
 };
 
@@ -52,9 +54,46 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
                            const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
                            int d, void *ws, cudaStream_t st, const Varlen *vl = nullptr);
 
+// The head-mixing solve's set-up in a Newton workspace (newton_workspace_bytes):
+// clears the control block and the stats record and, for SLSTM_INIT_DECOUPLED,
+// enqueues the decoupled guess into S (its residual is not tested).  *ctrl
+// receives the call's control block.
+cudaError_t newton_guess_prepare(const float *P, const float *s0, float *S, const slstm_newton_config &cfg,
+                                 slstm_newton_stats *stats, int B, int T, int d, void *ws, cudaStream_t st,
+                                 NewtonCtrl **ctrl);
+
+// Head mixing (head.cu): R_head (4, d / dh, dh, dh), 1 <= dh <= 32, dh | d.
+cudaError_t head_sequential_launch(const float *P, const float *Rh, const float *s0, float *S, int B, int T, int d,
+                                   int dh, int forget, cudaStream_t st);
+// Workspace: newton_workspace_bytes(B, T, d).
+cudaError_t head_newton_forward(const float *P, const float *Rh, const float *s0, float *S,
+                                const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T, int d,
+                                int dh, void *ws, cudaStream_t st);
+size_t head_backward_workspace_bytes(int B, int T, int d_in, int d, int dh);
+cudaError_t head_backward_launch(const void *x, const void *Wx, int dtype, const float *P, const float *Rh,
+                                 const float *s0, const float *S, const float *dH, float *dx, float *dWx, float *dRh,
+                                 float *db, float *ds0, int forget, int B, int T, int d_in, int d, int dh, void *ws,
+                                 cudaStream_t st);
+
+// Time context parallel (newton.cu): the phases of a solve split over time
+// slices; the caller exchanges the slice results between the phases.
+size_t cp_workspace_bytes(int B, int T, int d);
+cudaError_t cp_guess_run(const float *P, const float *R, const float *s_before, const float *S, bool sweep, int forget,
+                         float *run_out, int B, int T, int d, void *ws, cudaStream_t st);
+cudaError_t cp_guess_apply(const float *P, const float *R, const float *s0, const float *s_before,
+                           const float *runs, int rank, float *S, bool sweep, int forget, int B, int T, int d,
+                           void *ws, cudaStream_t st);
+cudaError_t cp_newton_map(const float *P, const float *R, const float *s_before, const float *S, int forget,
+                          float *map_out, int B, int T, int d, void *ws, cudaStream_t st);
+cudaError_t cp_newton_apply(const float *P, const float *R, const float *s_before, const float *maps, int rank,
+                            float *S, const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T, int d,
+                            void *ws, cudaStream_t st);
+
 size_t scan_workspace_bytes(int B, int T, int d);
+// debug_withhold: host-requested fault injection (one tile withholds its
+// carry; its successor's bounded wait expires and the outputs after it are NaN).
 cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, float *y, int B,
-                               int T, int d, bool reverse, void *ws, cudaStream_t st);
+                               int T, int d, bool reverse, void *ws, cudaStream_t st, bool debug_withhold = false);
 
 cudaError_t decode_launch(const void *x, const void *Wx, int dtype, const float *bias, const float *R,
                           const float *s_prev, float *s_next, int forget, int B, int d_in, int d, cudaStream_t st);
@@ -98,6 +137,8 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, 
                             cudaStream_t st);
 // The split count gemm_tc_bf16_ex will actually use for a request of `want`.
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want);
+// out[i] = sum over z in order of part[z * n + i] (split-K partial sums).
+cudaError_t sum_splits(const float *part, float *out, long long n, int splits, cudaStream_t st);
 
 // Input projection P = x Wx^T + bias (tcgen05 for bf16, CUDA cores for fp32).
 size_t preact_workspace_bytes(int B, int T, int d_in, int d_h, int dtype);

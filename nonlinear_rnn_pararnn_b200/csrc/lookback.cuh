@@ -21,7 +21,8 @@
 // for them, tile (chunk c, group g) has ticket c * n_groups + g, and a CTA
 // only waits on lower tickets, each held by a running CTA as its current
 // tile: every wait ends.  Waits are also bounded in time; on expiry the tile
-// records an error and continues with a zero carry.
+// records an error and continues with a NaN carry, so that the outputs that
+// depend on it are NaN rather than silently wrong.
 //
 // Two layouts of the per-warp maps are supported.  The plain one,
 // s_agg[w][20][32] (entry-major), is walked by warp 0 alone.  TileMaps stores
@@ -164,9 +165,11 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
         }
         if (++polls > 16) __nanosleep(64);
         if (globaltimer_ns() - t0 > ca.wait_ns) {
+            // gave up: the error word says so, and a NaN carry makes every
+            // output that depends on the missing prefix NaN
             atomicOr(ca.error, 1u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) carry[e] = 0.f;
+            for (int e = 0; e < 4; ++e) carry[e] = __int_as_float(0x7fc00000);
             return;
         }
     }
@@ -314,6 +317,16 @@ SLSTM_DEVINL void fold_p(AffP &agg, const Cell &J, const float r[4])
     } else {
         const float b[4] = {agg.b[0], agg.b[1], agg.b[2], agg.b[3]};
         jac_mul_add(J, b, r, agg.b);
+    }
+}
+
+SLSTM_DEVINL void affp_identity(AffP &x)
+{
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        x.a01[r] = make_float2(r == 0 ? 1.f : 0.f, r == 1 ? 1.f : 0.f);
+        x.a23[r] = make_float2(r == 2 ? 1.f : 0.f, r == 3 ? 1.f : 0.f);
+        x.b[r] = 0.f;
     }
 }
 
@@ -501,6 +514,11 @@ struct TileScanArgs {
     float *cin;                // [n_tiles][4][32] the carry entering each tile
     const unsigned *done;      // nonzero: the call has finished (or null)
     int n_groups, n_chunks, n_blk;
+    // the carry entering each group's first tile, (B, 4, d) with group g =
+    // (b, features 32 (g % gpr) ..), or null for zero (time slices after the
+    // first of a context-parallel solve)
+    const float *cin0 = nullptr;
+    int gpr = 1, d = 0;
 };
 
 // (group, block) per warp: the composition of the block's tile aggregates.
@@ -537,6 +555,13 @@ __global__ void __launch_bounds__(256) scan_block_carry(TileScanArgs s)
     const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (g >= s.n_groups) return;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (s.cin0) {
+        const int b = g / s.gpr, j = (g - b * s.gpr) * 32 + lane;
+        if (j < s.d) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = s.cin0[((size_t)b * 4 + e) * s.d + j];
+        }
+    }
     Aff x;
     for (int k = 0; k < s.n_blk; ++k) {
         const size_t w = (size_t)g * s.n_blk + k;

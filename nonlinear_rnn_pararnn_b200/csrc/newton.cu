@@ -32,6 +32,7 @@
 
 #include "launchers.h"
 #include "lookback.cuh"
+#include "stop_rule.cuh"
 #include "tma.cuh"
 
 namespace slstm {
@@ -54,6 +55,8 @@ struct Args {
     const float *P;
     const float *R;
     const float *s0;
+    const float *s0h;             // sweeps: the state whose h the gates of step 0 see (s0, or a time slice's
+                                  // previous guess just before it)
     float *S;
     NewtonCtrl *ctrl;
     unsigned *flags;              // [n_tiles] aggregate-published flags
@@ -72,9 +75,9 @@ struct Args {
     unsigned epoch;
     unsigned long long wait_ns;
     int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
-    int k0;             // launches before the first Newton iteration (the guess): 0 or 1
+    int k0;             // launches before the first Newton iteration (the guess and its sweeps)
     int resid_raw;      // stopping test on max|F| (else on the scaled residual)
-    int guess_tested;   // the guess launch evaluated and recorded its own residual
+    int guess_tested;   // the first iteration records the residual of the guess
     float tol;
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
@@ -115,6 +118,7 @@ constexpr uint64_t TMA_WAIT_NS = 1000000000ull;
 // (step, slot) rows for the tile loads, 32 x 16 rows for a warp's stores.
 struct NewtonMaps {
     CUtensorMap P, S, Sw;
+    CUtensorMap H;   // S as (d, 4, T, B): boxes of 32 features x 1 slot x 64 steps (the guess sweeps' h rows)
 };
 
 // TMA_THREAD only: start the loads of one tile into stage `st`: the P (and
@@ -249,53 +253,12 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo 
     }
 }
 
-// Last CTA of launch k: records the residual of Newton iteration n = k - k0
-// and decides whether the solve goes on.
+// Last CTA of launch k: records the residual of Newton iteration k - k0
+// and decides whether the solve goes on (stop_rule.cuh).
 __device__ void finalize(const Args &a, int k, bool resid)
 {
-    NewtonCtrl *c = a.ctrl;
-    slstm_newton_stats *st = a.stats;
-    NewtonSlot &s = c->slot[k & 1];
-    const float raw = __uint_as_float(atomicOr(&s.maxF_raw, 0u));
-    const float sc = __uint_as_float(atomicOr(&s.maxF_scaled, 0u));
-    const unsigned err = atomicOr(&c->error, 0u);
-    const int n = k - a.k0;
-    const bool last = (n + 1 == a.max_iters);
-    // the next iteration starts from a clean slot (its previous user,
-    // iteration k - 1, finished before this launch began)
-    NewtonSlot &nx = c->slot[(k + 1) & 1];
-    nx.ticket = 0u;
-    nx.finished = 0u;
-    nx.maxF_raw = 0u;
-    nx.maxF_scaled = 0u;
-    st->iters = n + 1;
-    st->max_abs_F[n % SLSTM_STATS_HISTORY] = resid ? raw : -1.0f;
-    st->max_scaled_F[n % SLSTM_STATS_HISTORY] = resid ? sc : -1.0f;
-    if (n == 0 && !a.guess_tested) {
-        st->init_max_abs_F = -1.0f;
-        st->init_max_scaled_F = -1.0f;
-    }
-    const float test = a.resid_raw ? raw : sc;
-    bool done = last;
-    if (err) {
-        st->error = SLSTM_ERR_TIMEOUT;
-        done = true;
-    } else if (resid) {
-        const bool bad = !(raw <= FLT_MAX) || !(sc <= FLT_MAX);
-        if (bad) {
-            st->diverged = 1;
-            st->error = SLSTM_ERR_DIVERGED;
-            done = true;
-        } else if (test <= a.tol && (!a.fixed || last)) {
-            st->converged = 1;
-            done = done || !a.fixed;
-        } else if (last && raw > 1.0f) {
-            st->diverged = 1;
-            st->error = SLSTM_ERR_DIVERGED;
-        }
-    }
-    __threadfence();
-    if (done) atomicExch(&c->done, 1u);
+    const StopRule r{a.ctrl, a.stats, a.k0, a.max_iters, a.fixed, a.resid_raw, a.guess_tested, a.tol};
+    finalize_iteration(r, k, resid);
 }
 
 // ---- the decoupled initial guess --------------------------------------------
@@ -365,32 +328,47 @@ SLSTM_DEVINL void guess_gates(float pz, float pf, float po, float &z, float &lf,
     }
 }
 
+// Runs of the tile in shared memory: [entry][feature][warp], the warp index
+// padded to 17 so that both the walk (lane = feature, one warp) and the scan
+// (lane = warp, two features per warp) touch 32 distinct banks.
+constexpr int SEG_LD = NW + 1;
+
 struct GuessSmem {
     float P[2][TT][4][32];   // stage s: rows (step, slot) of 32 features; TMA boxes land here
+    float Hs[2][TT][32];     // sweeps: h of the previous guess at every step of the tile
     float O[TT][4][32];      // TMA path: S of the tile, source of the warps' TMA stores
-    float R[2][4][32];       // TMA path: the tile's recurrent weights (gate-major)
-    float seg[NW][5][32];    // each warp's run: A, mu, u, v, o
-    float cin[NW][4][32];    // state (c, n, m, h) entering each warp
+    float seg[5][32][SEG_LD];   // each warp's run (A, mu, u, v, o), then the inclusive prefixes
+    float cin[4][32];        // state (c, n, m, h) entering the tile
+    float hb[2][32];         // sweeps: h of the previous guess just before the tile
     TileInfo info[3];
     uint64_t bar[2];
-    float red[2][NW];
     unsigned whead;
     int exit_flag;
 };
 constexpr size_t GUESS_SMEM_BYTES = sizeof(GuessSmem) + 1024;
 
+// Loads of one tile: P, and for a sweep the previous guess's h rows (TMA
+// box of slot 3) and the h just before the tile (the previous launch's
+// boundary buffer).
+template <bool SWEEP>
 SLSTM_DEVINL void guess_issue_load(const Args &a, const NewtonMaps &m, GuessSmem &sm, int st, const TileInfo &ti)
 {
     if (ti.ticket >= (unsigned)a.n_tiles) return;
-    const uint32_t rbytes = 4u * (uint32_t)min(32, a.d - ti.j0);   // a multiple of 16 (d % 4 == 0)
-    mbar_expect_tx(&sm.bar[st], (uint32_t)sizeof(sm.P[0]) + 4u * rbytes);
+    const bool bnd = SWEEP && ti.chunk > 0;
+    mbar_expect_tx(&sm.bar[st], (uint32_t)sizeof(sm.P[0]) + (SWEEP ? (uint32_t)sizeof(sm.Hs[0]) : 0u) +
+                                    (bnd ? 128u : 0u));
     tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, ti.chunk * TT * 4, ti.b);
-#pragma unroll
-    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    if (SWEEP) {
+        tma_load_4d(&sm.Hs[st][0][0], &m.H, &sm.bar[st], ti.j0, 3, ti.chunk * TT, ti.b);
+        if (bnd)
+            bulk_load(&sm.hb[st][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32 + 3 * 32, 128u,
+                      &sm.bar[st]);
+    }
 }
 
 // cp.async path: 4-byte copies, lane = feature; rows past T and features
 // past d arrive as zeros.
+template <bool SWEEP>
 SLSTM_DEVINL void guess_prefetch(const Args &a, GuessSmem &sm, int st, const TileInfo &ti)
 {
     if (ti.ticket >= (unsigned)a.n_tiles) return;
@@ -406,6 +384,56 @@ SLSTM_DEVINL void guess_prefetch(const Args &a, GuessSmem &sm, int st, const Til
         const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
         cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * roww : a.P, bytes);
     }
+    if (SWEEP) {
+        // h rows: warp w copies steps w, w + NW, ...
+        const float *hs = a.S + ti.off + 3 * (size_t)a.d + jl;
+#pragma unroll
+        for (int r = 0; r < L; ++r) {
+            const int step = r * NW + w;
+            const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+            cp_async4(&sm.Hs[st][step][jl], bytes ? hs + (size_t)step * 4 * a.d : a.S, bytes);
+        }
+        if (w == 0) {
+            const bool bnd = ti.chunk > 0;
+            const float *src = a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32 + 3 * 32 + jl;
+            cp_async4(&sm.hb[st][jl], bnd ? src : a.bnd_in, bnd ? 4 : 0);
+        }
+    }
+}
+
+SLSTM_DEVINL void seg_load(const GuessSmem &sm, int w, int f, Seg &x, bool head)
+{
+    x.A = sm.seg[0][f][w];
+    x.mu = sm.seg[1][f][w];
+    x.u = sm.seg[2][f][w];
+    x.v = sm.seg[3][f][w];
+    x.o = sm.seg[4][f][w];
+    x.head = head;
+}
+
+SLSTM_DEVINL void seg_store(GuessSmem &sm, int w, int f, const Seg &x)
+{
+    sm.seg[0][f][w] = x.A;
+    sm.seg[1][f][w] = x.mu;
+    sm.seg[2][f][w] = x.u;
+    sm.seg[3][f][w] = x.v;
+    sm.seg[4][f][w] = x.o;
+}
+
+// The state after the run x entered from v (c, n, m, h).
+SLSTM_DEVINL void seg_enter(const Seg &x, const float v[4], float out[4])
+{
+    if (x.head) {
+        out[0] = x.u;
+        out[1] = x.v;
+        out[2] = x.mu;
+    } else {
+        out[0] = v[0];
+        out[1] = v[1];
+        out[2] = v[2];
+        seg_apply(x.A, x.mu, x.u, x.v, out[2], out[0], out[1]);
+    }
+    out[3] = guess_h(x.o, out[0], out[1]);
 }
 
 // The guess's look-back when the predecessor's state is not published yet
@@ -436,12 +464,11 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
         const unsigned tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
         float w[4];
         if (__all_sync(0xffffffffu, read_inc_words(ca, tq, lane, w))) {
-            if (have) {
-                seg_apply(M.A, M.mu, M.u, M.v, w[2], w[0], w[1]);
-                w[3] = guess_h(M.o, w[0], w[1]);
-            }
+            if (have) seg_enter(M, w, v);
+            else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = w[e];
+                for (int e = 0; e < 4; ++e) v[e] = w[e];
+            }
             return;
         }
         const unsigned f = ld_acquire(a.flags + tq);
@@ -459,10 +486,7 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
             have = true;
             if (M.head) {
                 // a sequence starts inside: the state is the run's own end
-                v[0] = M.u;
-                v[1] = M.v;
-                v[2] = M.mu;
-                v[3] = guess_h(M.o, M.u, M.v);
+                seg_enter(M, v, v);
                 return;
             }
             --q;   // chunk 0 never publishes a run, so q stays >= 0
@@ -470,25 +494,39 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
         }
         if (++polls > 16) __nanosleep(64);
         if (globaltimer_ns() - t0 > a.wait_ns) {
+            // gave up: the error word says so, and a NaN state makes every
+            // output that depends on it NaN
             atomicOr(a.error, 1u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) v[e] = 0.f;
+            for (int e = 0; e < 4; ++e) v[e] = __int_as_float(0x7fc00000);
             return;
         }
     }
 }
 
-// The guess: one launch over every tile.  RESID: also evaluate the guess's
-// residual with the true R (tolerance mode), recorded as the initial
-// residual; a guess that meets the test ends the solve.
-template <int FORGET, bool RESID, bool TMA, bool VARLEN>
-__global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_constant__ NewtonMaps maps)
+// The decoupled guess (SWEEP false), or one refinement sweep of it (SWEEP
+// true: the gates of step t see r h_{t-1} of the previous guess, read from S
+// before this launch overwrites it and, at a tile's first step, from the
+// previous launch's boundary buffer).  One launch over every tile; launch k
+// of the solve (epoch k + 1, control slot k & 1).
+//   walk A  each thread folds its 4 steps into a run;
+//   scan    the 16 warp runs of each feature are scanned (inclusive) by a
+//           Kogge-Stone scan over 16 lanes, two features per warp, so that
+//           the tile's aggregate run and every warp's prefix are known
+//           without a serial walk;
+//   carry   warp 0 takes the state entering the tile (the predecessor's
+//           published state, or the look-back) and publishes the tile's
+//           state;
+//   walk B  each warp enters its steps through its prefix and replays them,
+//           writing S and the tile's last state for the next launch.
+template <int FORGET, bool SWEEP, bool TMA, bool VARLEN>
+__global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
     GuessSmem &sm = *reinterpret_cast<GuessSmem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    NewtonSlot &slot = a.ctrl->slot[0];
+    NewtonSlot &slot = a.ctrl->slot[k & 1];
 
     if (threadIdx.x == 0) {
         sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
@@ -508,14 +546,13 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
     const size_t d = (size_t)a.d;
     const int T = a.T;
     const unsigned G = (unsigned)a.n_groups;
-    float mx_raw = 0.f, mx_sc = 0.f;
     int ring = 0, st = 0;
     unsigned it = 0;
     bool tma_ok = true;
     if (TMA) {
-        if (threadIdx.x == 0) guess_issue_load(a, maps, sm, 0, sm.info[0]);
+        if (threadIdx.x == 0) guess_issue_load<SWEEP>(a, maps, sm, 0, sm.info[0]);
     } else {
-        guess_prefetch(a, sm, 0, sm.info[0]);
+        guess_prefetch<SWEEP>(a, sm, 0, sm.info[0]);
         cp_async_commit();
     }
 
@@ -526,14 +563,14 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
         unsigned after = 0;
         if (threadIdx.x == 0) after = atomicAdd(&slot.ticket, 1u);
         if (TMA) {
-            if (threadIdx.x == 32) guess_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
+            if (threadIdx.x == 32) guess_issue_load<SWEEP>(a, maps, sm, st ^ 1, sm.info[rn]);
             if (tma_ok && !mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS)) {
                 atomicOr(a.error, 2u);
                 (void)mbar_wait(&sm.bar[st], (it >> 1) & 1u, TMA_WAIT_NS);
                 tma_ok = false;
             }
         } else {
-            guess_prefetch(a, sm, st ^ 1, sm.info[rn]);
+            guess_prefetch<SWEEP>(a, sm, st ^ 1, sm.info[rn]);
             cp_async_commit();
             cp_async_wait_prev();
             __syncthreads();
@@ -545,17 +582,47 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
         const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
         const int t_seg = chunk * TT + warp * L;
 
+        // recurrent weights and the previous guess's h before this warp's
+        // first step (sweeps)
+        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f, hprev = 0.f;
+        if (SWEEP) {
+            if (jv) {
+                rz = __ldg(a.R + jj);
+                ri = __ldg(a.R + d + jj);
+                rf = __ldg(a.R + 2 * d + jj);
+                ro = __ldg(a.R + 3 * d + jj);
+            }
+            if (warp > 0) hprev = sm.Hs[st][warp * L - 1][lane];
+            else if (chunk > 0) hprev = sm.hb[st][lane];
+            else if (!VARLEN && a.s0h && jv) hprev = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
+        }
+
         // ---- walk A: this warp's run, lane = feature ----
         float gz[L], glf[L], go[L], gi[L];
-        Seg run;
         {
+            Seg run;
+            float hp = hprev;
 #pragma unroll
             for (int i = 0; i < L; ++i) {
                 const int sl = warp * L + i;
-                guess_gates<FORGET>(sm.P[st][sl][0][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], gz[i],
-                                    glf[i], go[i]);
-                gi[i] = sm.P[st][sl][1][lane];
                 const bool head = VARLEN && ((ti.mask >> sl) & 1ull);
+                if (SWEEP && head) {
+                    // a sequence starts here: its previous h is its own s0's
+                    float s0v[4];
+                    head_state(a, t_seg + i, jj, jv, s0v);
+                    hp = s0v[3];
+                }
+                float pz = sm.P[st][sl][0][lane], pi = sm.P[st][sl][1][lane], pf = sm.P[st][sl][2][lane],
+                      po = sm.P[st][sl][3][lane];
+                if (SWEEP) {
+                    pz = fmaf(rz, hp, pz);
+                    pi = fmaf(ri, hp, pi);
+                    pf = fmaf(rf, hp, pf);
+                    po = fmaf(ro, hp, po);
+                    hp = sm.Hs[st][sl][lane];
+                }
+                guess_gates<FORGET>(pz, pf, po, gz[i], glf[i], go[i]);
+                gi[i] = pi;
                 if (head) {
                     float s0v[4];
                     head_state(a, t_seg + i, jj, jv, s0v);
@@ -576,24 +643,46 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
                 }
                 run.o = go[i];
             }
-            sm.seg[warp][0][lane] = run.A;
-            sm.seg[warp][1][lane] = run.mu;
-            sm.seg[warp][2][lane] = run.u;
-            sm.seg[warp][3][lane] = run.v;
-            sm.seg[warp][4][lane] = run.o;
+            seg_store(sm, warp, lane, run);
         }
-        if (VARLEN && threadIdx.x == 0) {
+        if (threadIdx.x == 0) {
             unsigned wh = 0u;
+            if (VARLEN) {
 #pragma unroll
-            for (int w = 0; w < NW; ++w) wh |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
+                for (int w = 0; w < NW; ++w)
+                    wh |= (((ti.mask >> (w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
+            }
             sm.whead = wh;
         }
         __syncthreads();
 
-        // ---- carry: warp 0 walks the runs; warp w goes on once its state is stored ----
+        // ---- scan of the warp runs: lane (feature 2 warp + lane / 16, run lane % 16) ----
+        const unsigned whead = sm.whead;
+        {
+            const int f = 2 * warp + (lane >> 4), w = lane & 15;
+            Seg x;
+            seg_load(sm, w, f, x, ((whead >> w) & 1u) != 0u);
+#pragma unroll
+            for (int off = 1; off < NW; off *= 2) {
+                Seg y;
+                y.A = __shfl_up_sync(0xffffffffu, x.A, off, 16);
+                y.mu = __shfl_up_sync(0xffffffffu, x.mu, off, 16);
+                y.u = __shfl_up_sync(0xffffffffu, x.u, off, 16);
+                y.v = __shfl_up_sync(0xffffffffu, x.v, off, 16);
+                y.o = __shfl_up_sync(0xffffffffu, x.o, off, 16);
+                y.head = __shfl_up_sync(0xffffffffu, x.head ? 1 : 0, off, 16) != 0;
+                if (w >= off) seg_compose(x, y, x);
+            }
+            seg_store(sm, w, f, x);
+            // the inclusive prefix's head flag: any run up to w holds a head
+        }
+        __syncthreads();
+
+        // ---- carry: warp 0, lane = feature ----
         if (warp == 0) {
-            const unsigned whead = VARLEN ? sm.whead : 0u;
             float v[4] = {0.f, 0.f, 0.f, 0.f};
+            Seg tile;
+            seg_load(sm, NW - 1, lane, tile, whead != 0u);
             if (chunk == 0) {
                 if (!VARLEN && a.s0 && jv) {
 #pragma unroll
@@ -602,74 +691,46 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
             } else {
                 const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
                 const bool ok = read_inc_words(ca, ticket - G, lane, v);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    Seg tile;
-#pragma unroll 1
-                    for (int w = 0; w < NW; ++w) {
-                        Seg x;
-                        x.A = sm.seg[w][0][lane];
-                        x.mu = sm.seg[w][1][lane];
-                        x.u = sm.seg[w][2][lane];
-                        x.v = sm.seg[w][3][lane];
-                        x.o = sm.seg[w][4][lane];
-                        x.head = ((whead >> w) & 1u) != 0u;
-                        if (w == 0) tile = x;
-                        else seg_compose(x, tile, tile);
-                    }
+                if (!__all_sync(0xffffffffu, ok))
                     guess_lookback(a, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
-                }
             }
 #pragma unroll
-            for (int w = 0; w < NW; ++w) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sm.cin[w][e][lane] = v[e];
-                if (w > 0) named_bar_arrive(w, 2 * 32);
-                if ((whead >> w) & 1u) {
-                    v[0] = sm.seg[w][2][lane];
-                    v[1] = sm.seg[w][3][lane];
-                    v[2] = sm.seg[w][1][lane];
-                } else {
-                    seg_apply(sm.seg[w][0][lane], sm.seg[w][1][lane], sm.seg[w][2][lane], sm.seg[w][3][lane], v[2],
-                              v[0], v[1]);
-                }
-                v[3] = guess_h(sm.seg[w][4][lane], v[0], v[1]);
-            }
+            for (int e = 0; e < 4; ++e) sm.cin[e][lane] = v[e];
+            float vo[4];
+            seg_enter(tile, v, vo);
             unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, v[e]));
-        } else {
-            named_bar_sync(warp, 2 * 32);   // the state entering this warp is stored
+            for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
         }
+        __syncthreads();
 
-        // ---- walk B: replay the steps from the entering state ----
+        // ---- walk B: enter this warp's steps through the prefix before it ----
         if (TMA) {
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
         }
-        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-        if (RESID && jv) {
-            if (TMA) {
-                rz = sm.R[st][0][lane];
-                ri = sm.R[st][1][lane];
-                rf = sm.R[st][2][lane];
-                ro = sm.R[st][3][lane];
+        float sv[4];
+        {
+            float cv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cv[e] = sm.cin[e][lane];
+            if (warp == 0) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sv[e] = cv[e];
             } else {
-                rz = __ldg(a.R + jj);
-                ri = __ldg(a.R + d + jj);
-                rf = __ldg(a.R + 2 * d + jj);
-                ro = __ldg(a.R + 3 * d + jj);
+                // whether the prefix of runs 0 .. warp - 1 holds a sequence start
+                const bool ph = (whead & ((1u << warp) - 1u)) != 0u;
+                Seg x;
+                seg_load(sm, warp - 1, lane, x, ph);
+                seg_enter(x, cv, sv);
             }
         }
-        float sv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sv[e] = sm.cin[warp][e][lane];
         float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             const int sl = warp * L + i;
             const bool wr = jv && (t_seg + i < T);
             if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, sv);
-            const float prev[4] = {sv[0], sv[1], sv[2], sv[3]};
             seg_apply(glf[i], gi[i], gz[i], 1.0f, sv[2], sv[0], sv[1]);
             sv[3] = guess_h(go[i], sv[0], sv[1]);
             if (TMA) {
@@ -680,18 +741,6 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
                 for (int e = 0; e < 4; ++e)
                     if (wr) srow[(size_t)i * 4 * d + e * d] = sv[e];
             }
-            if (RESID) {
-                Cell f;
-                cell_eval<FORGET, false>(prev[0], prev[1], prev[2], prev[3], sm.P[st][sl][0][lane], gi[i],
-                                         sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri, rf, ro, f);
-                const float F[4] = {sv[0] - f.c, sv[1] - f.n, sv[2] - f.m, sv[3] - f.h};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float af = wr ? fabsf(F[e]) : 0.0f;
-                    mx_raw = fmax_nan(mx_raw, af);
-                    mx_sc = fmax_nan(mx_sc, __fdividef(af, 1.0f + fabsf(sv[e])));
-                }
-            }
         }
         if (TMA) {
             tma_store_fence();
@@ -701,7 +750,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
                 bulk_commit();
             }
         }
-        // state at the tile's last step, read by the first Newton iteration
+        // state at the tile's last step, read by the next launch
         if (warp == NW - 1 && t_seg + L - 1 < T) {
             float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
 #pragma unroll
@@ -718,42 +767,22 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, const __grid_
     } else {
         cp_async_wait_all();
     }
-    if (!RESID) return;
-    mx_raw = warp_max(mx_raw);
-    mx_sc = warp_max(mx_sc);
-    if (lane == 0) {
-        sm.red[0][warp] = mx_raw;
-        sm.red[1][warp] = mx_sc;
-    }
-    __syncthreads();
+    // the CTA that finishes the launch last clears the other control slot
+    // for launch k + 1; the guess itself (k = 0) also marks the guess's
+    // residual as not recorded (the first iteration records it)
     if (threadIdx.x == 0) {
-        float r0 = sm.red[0][0], r1 = sm.red[1][0];
-        for (int w = 1; w < NW; ++w) {
-            r0 = (__float_as_uint(sm.red[0][w]) > __float_as_uint(r0)) ? sm.red[0][w] : r0;
-            r1 = (__float_as_uint(sm.red[1][w]) > __float_as_uint(r1)) ? sm.red[1][w] : r1;
-        }
-        atomic_max_nonneg(&slot.maxF_raw, r0);
-        atomic_max_nonneg(&slot.maxF_scaled, r1);
         __threadfence();
-        const unsigned fin = atomicAdd(&slot.finished, 1u);
-        if (fin == gridDim.x - 1u) {
-            __threadfence();
-            const float raw = __uint_as_float(atomicOr(&slot.maxF_raw, 0u));
-            const float sc = __uint_as_float(atomicOr(&slot.maxF_scaled, 0u));
-            slstm_newton_stats *stt = a.stats;
-            stt->init_max_abs_F = raw;
-            stt->init_max_scaled_F = sc;
-            const unsigned err = atomicOr(a.error, 0u);
-            const float test = a.resid_raw ? raw : sc;
-            if (err) {
-                stt->error = SLSTM_ERR_TIMEOUT;
-                __threadfence();
-                atomicExch(&a.ctrl->done, 1u);
-            } else if (raw <= FLT_MAX && sc <= FLT_MAX && test <= a.tol) {
-                stt->converged = 1;
-                __threadfence();
-                atomicExch(&a.ctrl->done, 1u);
+        if (atomicAdd(&slot.finished, 1u) == gridDim.x - 1u) {
+            NewtonSlot &nx = a.ctrl->slot[(k + 1) & 1];
+            nx.ticket = 0u;
+            nx.finished = 0u;
+            nx.maxF_raw = 0u;
+            nx.maxF_scaled = 0u;
+            if (k == 0 && a.stats) {
+                a.stats->init_max_abs_F = -1.0f;
+                a.stats->init_max_scaled_F = -1.0f;
             }
+            __threadfence();
         }
     }
 }
@@ -782,7 +811,9 @@ __global__ void gather_boundaries(Args a)
 // and plain stores.
 // VARLEN: packed ragged sequences (B = 1); at a head step the previous state is
 // the sequence's s0 and the Jacobian is zero, which makes the scan segmented.
-template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE>
+// GRS: the first iteration from the decoupled guess also records the
+// guess's residual (tolerance mode).
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE, bool GRS>
 __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -813,6 +844,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     const size_t toff = prefetch_offset(a);
     const bool chain_warp = warp >= CHAIN0;
     float mx_raw = 0.f, mx_sc = 0.f;
+    // the first iteration from the decoupled guess records the guess's
+    // residual, which walk A forms anyway (r = f - S_old = -F)
+    constexpr bool grs = GRS && MODE != MODE_AGG && !FIRST;
+    float g_raw = 0.f, g_sc = 0.f;
 
     int ring = 0, st = 0;
     unsigned it = 0;       // tiles done by this CTA; stage it & 1, TMA phase (it >> 1) & 1
@@ -926,12 +961,30 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                                         rf, ro, Jc[i]);
                 if (head) cell_zero_jac(Jc[i]);
                 const float r[4] = {Jc[i].c - so[0], Jc[i].n - so[1], Jc[i].m - so[2], Jc[i].h - so[3]};
+                if (grs) {
+                    const bool valid = jv && (t_seg + i < T);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float af = valid ? fabsf(r[e]) : 0.0f;
+                        g_raw = fmax_nan(g_raw, af);
+                        g_sc = fmax_nan(g_sc, __fdividef(af, 1.0f + fabsf(so[e])));
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < 4; ++e) curS[e] = so[e];
                 // a head starts the warp's map afresh: select, never multiply
-                // what came before by its zero Jacobian
-                if (i == 0 || head) affp_from_cell<false>(agg, Jc[i], r);
-                else fold_p<false>(agg, Jc[i], r);
+                // what came before by its zero Jacobian; in the aggregate
+                // pass, steps past T (the last tile only) are left out, so
+                // that the tile's map is the map of its steps (a time
+                // slice's map composes it)
+                const bool valid = MODE != MODE_AGG || t_seg + i < T;
+                if (!valid) {
+                    if (i == 0) affp_identity(agg);
+                } else if (i == 0 || head) {
+                    affp_from_cell<false>(agg, Jc[i], r);
+                } else {
+                    fold_p<false>(agg, Jc[i], r);
+                }
             }
         }
         maps_store(sm.maps.m, warp, lane, agg);
@@ -1110,6 +1163,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             sm.red[1][warp] = mx_sc;
         }
     }
+    if (grs) {
+        g_raw = warp_max(g_raw);
+        g_sc = warp_max(g_sc);
+        if (lane == 0) {
+            atomic_max_nonneg(&a.ctrl->init_raw, g_raw);
+            atomic_max_nonneg(&a.ctrl->init_scaled, g_sc);
+        }
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         if (RESID) {
@@ -1130,10 +1191,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     }
 }
 
-template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE>
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE, bool GRS = false>
 cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = newton_iter<FORGET, FIRST, RESID, TMA, VARLEN, MODE>;
+    auto kern = newton_iter<FORGET, FIRST, RESID, TMA, VARLEN, MODE, GRS>;
     static int blocks_per_sm = 0;
     if (blocks_per_sm == 0) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -1153,14 +1214,16 @@ cudaError_t launch_pass(const Args &a, const NewtonMaps &m, int k, bool resid, i
     if (k == 0)
         return resid ? launch_one<FORGET, true, true, TMA, VARLEN, MODE>(a, m, k, sms, st)
                      : launch_one<FORGET, true, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
+    if (MODE != MODE_AGG && resid && a.guess_tested && k == a.k0)
+        return launch_one<FORGET, false, true, TMA, VARLEN, MODE, true>(a, m, k, sms, st);
     return resid ? launch_one<FORGET, false, true, TMA, VARLEN, MODE>(a, m, k, sms, st)
                  : launch_one<FORGET, false, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
 }
 
-template <int FORGET, bool RESID, bool TMA, bool VARLEN>
-cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int sms, cudaStream_t st)
+template <int FORGET, bool SWEEP, bool TMA, bool VARLEN>
+cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = guess_kernel<FORGET, RESID, TMA, VARLEN>;
+    auto kern = guess_kernel<FORGET, SWEEP, TMA, VARLEN>;
     static bool ready = false;
     if (!ready) {
         const cudaError_t e =
@@ -1168,23 +1231,41 @@ cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int sms, cudaStream
         if (e != cudaSuccess) return e;
         ready = true;
     }
-    kern<<<min(a.n_tiles, sms), NW * 32, GUESS_SMEM_BYTES, st>>>(a, m);
+    kern<<<min(a.n_tiles, sms), NW * 32, GUESS_SMEM_BYTES, st>>>(a, k, m);
     return cudaGetLastError();
 }
 
-// The launches of one solve: the initial guess as launch 0 (decoupled: the
-// guess kernel; given: the boundary gather), then Newton iterations
-// k = k0 .. k0 + max_iters - 1.  Launch k has epoch k + 1 and writes the
-// boundary buffer that launch k + 1 reads.
+// Launch k of a solve: epoch k + 1; it reads the boundary buffer launch
+// k - 1 wrote and writes the other one.
+inline Args launch_args(const Args &base, int k)
+{
+    Args a = base;
+    a.epoch = (unsigned)(k + 1);
+    a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
+    a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
+    return a;
+}
+
+// The decoupled guess (launch 0) and its refinement sweeps (launches
+// 1 .. sweeps).
+template <int FORGET, bool TMA, bool VARLEN>
+cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, int sms, cudaStream_t st)
+{
+    cudaError_t e = launch_guess<FORGET, false, TMA, VARLEN>(launch_args(base, 0), m, 0, sms, st);
+    for (int k = 1; k <= sweeps && e == cudaSuccess; ++k)
+        e = launch_guess<FORGET, true, TMA, VARLEN>(launch_args(base, k), m, k, sms, st);
+    return e;
+}
+
+// The launches of one solve: the initial guess (decoupled: the guess kernel
+// and its sweeps; given: the boundary gather) as launches 0 .. k0 - 1, then
+// Newton iterations k = k0 .. k0 + max_iters - 1.
 template <int FORGET, bool TMA, bool VARLEN>
 cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
                          int init, cudaStream_t st)
 {
     if (init == SLSTM_INIT_DECOUPLED) {
-        Args a = base;
-        a.epoch = 1u;
-        const cudaError_t e = fixed ? launch_guess<FORGET, false, TMA, VARLEN>(a, m, sms, st)
-                                    : launch_guess<FORGET, true, TMA, VARLEN>(a, m, sms, st);
+        const cudaError_t e = launch_guess_all<FORGET, TMA, VARLEN>(base, m, base.k0 - 1, sms, st);
         if (e != cudaSuccess) return e;
     } else if (init == SLSTM_INIT_GIVEN) {
         const long long n = (long long)base.n_tiles * 128;
@@ -1193,10 +1274,7 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         if (e != cudaSuccess) return e;
     }
     for (int k = base.k0; k < base.k0 + max_iters; ++k) {
-        Args a = base;
-        a.epoch = (unsigned)(k + 1);
-        a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
-        a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
+        const Args a = launch_args(base, k);
         const bool resid = !fixed || (k + 1 - base.k0 == max_iters);
         cudaError_t e;
         if (two_pass) {
@@ -1271,16 +1349,19 @@ cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, 
 
 size_t newton_workspace_bytes(int B, int T, int d) { return layout(B, T, d).total; }
 
-cudaError_t newton_forward(const float *P, const float *R, const float *s0, float *S,
-                           const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
-                           int d, void *ws, cudaStream_t st, const Varlen *vl)
+namespace {
+
+// Arguments, tensor maps and cleared control state of one call.
+cudaError_t prepare(const float *P, const float *R, const float *s0, float *S, const slstm_newton_config &cfg,
+                    slstm_newton_stats *stats, int B, int T, int d, void *ws, cudaStream_t st, const Varlen *vl,
+                    Args &a, NewtonMaps &m, bool &tma, bool &two_pass)
 {
     const Layout l = layout(B, T, d);
     char *base = static_cast<char *>(ws);
-    Args a;
     a.P = P;
     a.R = R;
     a.s0 = s0;
+    a.s0h = s0;
     a.S = S;
     a.ctrl = reinterpret_cast<NewtonCtrl *>(base + l.ctrl);
     a.flags = reinterpret_cast<unsigned *>(base + l.flags);
@@ -1307,7 +1388,7 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     a.max_iters = cfg.max_iters;
     a.fixed = cfg.fixed_iters ? 1 : 0;
     a.tol = cfg.tol;
-    a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : 1;
+    a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : (cfg.init == SLSTM_INIT_DECOUPLED ? 1 + cfg.guess_sweeps : 1);
     a.resid_raw = cfg.residual_mode == SLSTM_RESIDUAL_RAW ? 1 : 0;
     a.guess_tested = (cfg.init == SLSTM_INIT_DECOUPLED && !a.fixed) ? 1 : 0;
     a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(P) & 15) == 0 &&
@@ -1319,7 +1400,7 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     // control block, aggregate flags and the epoch tags of the inclusive
     // prefixes start cleared on every call
     cudaError_t e = cudaMemsetAsync(base + l.ctrl, 0, l.agg - l.ctrl, st);
-    if (e == cudaSuccess) e = cudaMemsetAsync(stats, 0, sizeof(slstm_newton_stats), st);
+    if (e == cudaSuccess && stats) e = cudaMemsetAsync(stats, 0, sizeof(slstm_newton_stats), st);
     if (e != cudaSuccess) return e;
     a.vmask = nullptr;
     a.vseq = nullptr;
@@ -1332,20 +1413,35 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     const int sms = sm_count();
     // TMA moves the tiles when the rows are 16-byte aligned and every row
     // coordinate fits a signed 32-bit box coordinate
-    NewtonMaps m;
     memset(&m, 0, sizeof(m));
     const uint64_t rows = 4 * (uint64_t)T, bstride = rows * (uint64_t)d;
-    const bool tma = a.vec16 && (reinterpret_cast<uintptr_t>(R) & 15) == 0 && rows < (1ull << 31) &&
-                     make_map_f32_3d(&m.P, P, d, rows, B, d, bstride, 32, TT * 4) &&
-                     make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
-                     make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4);
-    const bool v = vl != nullptr;
+    tma = a.vec16 && (reinterpret_cast<uintptr_t>(R) & 15) == 0 && rows < (1ull << 31) &&
+          make_map_f32_3d(&m.P, P, d, rows, B, d, bstride, 32, TT * 4) &&
+          make_map_f32_3d(&m.S, S, d, rows, B, d, bstride, 32, TT * 4) &&
+          make_map_f32_3d(&m.Sw, S, d, rows, B, d, bstride, 32, L * 4) &&
+          make_map_f32_4d(&m.H, S, d, 4, T, B, d, 4 * (uint64_t)d, bstride, 32, TT);
     // With few feature groups and a long time axis, most tiles of a fused
     // launch would wait for their predecessor: take the two passes instead.
     // Fault injection acts on the fused launch's publications.
-    const bool two_pass = cfg.carry_mode == SLSTM_CARRY_TWO_PASS ||
-                          (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 &&
-                           prefer_two_pass(l.n_groups, (long long)l.n_chunks * TT, sms));
+    two_pass = cfg.carry_mode == SLSTM_CARRY_TWO_PASS ||
+               (cfg.carry_mode == SLSTM_CARRY_AUTO && cfg.debug_fault == 0 &&
+                prefer_two_pass(l.n_groups, (long long)l.n_chunks * TT, sms));
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t newton_forward(const float *P, const float *R, const float *s0, float *S,
+                           const slstm_newton_config &cfg, slstm_newton_stats *stats, int B, int T,
+                           int d, void *ws, cudaStream_t st, const Varlen *vl)
+{
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    cudaError_t e = prepare(P, R, s0, S, cfg, stats, B, T, d, ws, st, vl, a, m, tma, two_pass);
+    if (e != cudaSuccess) return e;
+    const int sms = sm_count();
+    const bool v = vl != nullptr;
     const int init = cfg.init;
     if (cfg.forget == SLSTM_FORGET_EXP)
         return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
@@ -1354,6 +1450,401 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
                : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
                                                                st);
+}
+
+cudaError_t newton_guess_prepare(const float *P, const float *s0, float *S, const slstm_newton_config &cfg,
+                                 slstm_newton_stats *stats, int B, int T, int d, void *ws, cudaStream_t st,
+                                 NewtonCtrl **ctrl)
+{
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    cudaError_t e = prepare(P, nullptr, s0, S, cfg, stats, B, T, d, ws, st, nullptr, a, m, tma, two_pass);
+    if (e != cudaSuccess) return e;
+    *ctrl = a.ctrl;
+    if (cfg.init != SLSTM_INIT_DECOUPLED) return cudaSuccess;
+    const int sms = sm_count();
+    const Args a0 = launch_args(a, 0);
+    if (cfg.forget == SLSTM_FORGET_EXP)
+        return tma ? launch_guess<SLSTM_FORGET_EXP, false, true, false>(a0, m, 0, sms, st)
+                   : launch_guess<SLSTM_FORGET_EXP, false, false, false>(a0, m, 0, sms, st);
+    return tma ? launch_guess<SLSTM_FORGET_SIGMOID, false, true, false>(a0, m, 0, sms, st)
+               : launch_guess<SLSTM_FORGET_SIGMOID, false, false, false>(a0, m, 0, sms, st);
+}
+
+
+// ---------------------------------------------------------------------------
+// Time context parallel ("sLSTM in this library", section "Tensor parallel":
+// context parallel splits time).  Rank r of n holds the steps
+// [t_r, t_r + T_r) of every sequence.  Every scan of the solve becomes: each
+// rank composes its slice into one map (a run of the guess's monoid, or the
+// affine map of a Newton iteration's linear solve), the maps are exchanged
+// (all-gather, by the caller), and each rank enters its slice through the
+// composition of the maps of the ranks before it.
+// ---------------------------------------------------------------------------
+namespace {
+
+// The run of one tile of a guess (SWEEP: of a sweep, the gates seeing the
+// previous guess's h), one CTA per tile, warp w folding steps 4w .. 4w + 3
+// (steps past T are left out); warp 0 composes the 16 warp runs into
+// agg[tile] rows 0..4 and flags[tile] bit 0 (the tile is empty: never).
+template <int FORGET, bool SWEEP>
+__global__ void __launch_bounds__(NW * 32) cp_tile_run_kernel(Args a)
+{
+    __shared__ float runs[NW][5][32];
+    __shared__ int nonempty[NW];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned ticket = blockIdx.x;
+    TileInfo ti;
+    decode_tile(a, ticket, ti);
+    const size_t d = (size_t)a.d;
+    const bool jv = ti.j0 + lane < a.d;
+    const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
+    const int t_seg = ti.chunk * TT + warp * L;
+    float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f, hp = 0.f;
+    if (SWEEP && jv) {
+        rz = __ldg(a.R + jj);
+        ri = __ldg(a.R + d + jj);
+        rf = __ldg(a.R + 2 * d + jj);
+        ro = __ldg(a.R + 3 * d + jj);
+        const int tp = t_seg - 1;
+        if (tp >= 0 && tp < a.T) hp = __ldg(a.S + (((size_t)ti.b * a.T + tp) * 4 + 3) * d + jj);
+        else if (tp < 0 && a.s0h) hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
+    }
+    Seg run;
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+        const int t = t_seg + i;
+        if (t >= a.T) break;
+        const size_t row = ((size_t)ti.b * a.T + t) * 4;
+        float p[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) p[g] = jv ? __ldg(a.P + (row + g) * d + jj) : 0.0f;
+        if (SWEEP) {
+            p[0] = fmaf(rz, hp, p[0]);
+            p[1] = fmaf(ri, hp, p[1]);
+            p[2] = fmaf(rf, hp, p[2]);
+            p[3] = fmaf(ro, hp, p[3]);
+            hp = jv ? __ldg(a.S + (row + 3) * d + jj) : 0.0f;
+        }
+        float z, lf, o;
+        guess_gates<FORGET>(p[0], p[2], p[3], z, lf, o);
+        if (n == 0) {
+            run.A = lf;
+            run.mu = p[1];
+            run.u = z;
+            run.v = 1.0f;
+        } else {
+            seg_apply(lf, p[1], z, 1.0f, run.mu, run.u, run.v);
+            run.A += lf;
+        }
+        run.o = o;
+        ++n;
+    }
+    runs[warp][0][lane] = run.A;
+    runs[warp][1][lane] = run.mu;
+    runs[warp][2][lane] = run.u;
+    runs[warp][3][lane] = run.v;
+    runs[warp][4][lane] = run.o;
+    if (lane == 0) nonempty[warp] = n > 0;
+    __syncthreads();
+    if (warp == 0) {
+        Seg tile;
+        tile.head = false;
+        for (int w = 0; w < NW; ++w) {
+            if (!nonempty[w]) break;
+            Seg x;
+            x.A = runs[w][0][lane];
+            x.mu = runs[w][1][lane];
+            x.u = runs[w][2][lane];
+            x.v = runs[w][3][lane];
+            x.o = runs[w][4][lane];
+            x.head = false;
+            if (w == 0) tile = x;
+            else seg_compose(x, tile, tile);
+        }
+        float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
+        dst[0] = tile.A;
+        dst[32] = tile.mu;
+        dst[64] = tile.u;
+        dst[96] = tile.v;
+        dst[128] = tile.o;
+    }
+}
+
+// One warp per feature group: the tiles' runs composed in time order into
+// the slice's run, out (B, 5, d) with entries (A, mu, u, v, o).
+__global__ void __launch_bounds__(256) cp_slice_run_kernel(Args a, int n_chunks, float *out)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (g >= a.n_groups) return;
+    const int b = g / a.groups_per_row, j = (g - b * a.groups_per_row) * 32 + lane;
+    Seg acc;
+    for (int c = 0; c < n_chunks; ++c) {
+        const float *src = a.agg + ((size_t)c * a.n_groups + g) * 20 * 32 + lane;
+        Seg x;
+        x.A = src[0];
+        x.mu = src[32];
+        x.u = src[64];
+        x.v = src[96];
+        x.o = src[128];
+        x.head = false;
+        if (c == 0) acc = x;
+        else seg_compose(x, acc, acc);
+    }
+    if (j < a.d) {
+        const float e5[5] = {acc.A, acc.mu, acc.u, acc.v, acc.o};
+#pragma unroll
+        for (int e = 0; e < 5; ++e) out[((size_t)b * 5 + e) * a.d + j] = e5[e];
+    }
+}
+
+// Thread per (b, j): the state entering rank `rank`'s slice, s0 (or zero)
+// carried through the runs (n, B, 5, d) of ranks 0 .. rank - 1.
+__global__ void __launch_bounds__(256) cp_enter_runs_kernel(const float *runs, int rank, const float *s0, int B, int d,
+                                                            float *out)
+{
+    const long long q = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (q >= (long long)B * d) return;
+    const int b = (int)(q / d), j = (int)(q - (long long)b * d);
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = s0 ? s0[((size_t)b * 4 + e) * d + j] : 0.0f;
+    for (int r = 0; r < rank; ++r) {
+        const float *x = runs + (((size_t)r * B + b) * 5) * d + j;
+        Seg s;
+        s.A = x[0];
+        s.mu = x[d];
+        s.u = x[2 * d];
+        s.v = x[3 * d];
+        s.o = x[4 * d];
+        s.head = false;
+        seg_enter(s, v, v);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) out[((size_t)b * 4 + e) * d + j] = v[e];
+}
+
+// One warp per feature group: the block aggregates of the two-pass scan
+// (scan_block_agg) composed in time order into the slice's affine map, out
+// (B, 20, d): A row-major (16), then the offset (4).
+__global__ void __launch_bounds__(256) cp_slice_map_kernel(const float *blk_agg, int n_groups, int n_blk, int gpr, int d,
+                                                           float *out)
+{
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (g >= n_groups) return;
+    const int b = g / gpr, j = (g - b * gpr) * 32 + lane;
+    Aff acc, x;
+    load_agg(blk_agg + (size_t)g * n_blk * 640, lane, acc);
+    for (int k = 1; k < n_blk; ++k) {
+        load_agg(blk_agg + ((size_t)g * n_blk + k) * 640, lane, x);
+        aff_compose(x, acc, acc);
+    }
+    if (j < d) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) out[((size_t)b * 20 + e) * d + j] = acc.a[e];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) out[((size_t)b * 20 + 16 + e) * d + j] = acc.b[e];
+    }
+}
+
+// Thread per (b, j): the Newton correction entering rank `rank`'s slice, 0
+// carried through the maps (n, B, 20, d) of ranks 0 .. rank - 1.
+__global__ void __launch_bounds__(256) cp_enter_maps_kernel(const float *maps, int rank, int B, int d, float *out)
+{
+    const long long q = (long long)blockIdx.x * 256 + threadIdx.x;
+    if (q >= (long long)B * d) return;
+    const int b = (int)(q / d), j = (int)(q - (long long)b * d);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int r = 0; r < rank; ++r) {
+        const float *x = maps + (((size_t)r * B + b) * 20) * d + j;
+        Aff m;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) m.a[e] = x[(size_t)e * d];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m.b[e] = x[(size_t)(16 + e) * d];
+        aff_apply(m, v, v);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) out[((size_t)b * 4 + e) * d + j] = v[e];
+}
+
+struct CpLayout {
+    size_t newton, enter, total;
+};
+
+CpLayout cp_layout(int B, int T, int d)
+{
+    CpLayout c;
+    c.newton = 0;
+    c.enter = (newton_workspace_bytes(B, T, d) + 255) & ~(size_t)255;
+    c.total = c.enter + (((size_t)B * 4 * d * 4 + 255) & ~(size_t)255);
+    return c;
+}
+
+slstm_newton_config cp_config(int forget, const slstm_newton_config *cfg)
+{
+    slstm_newton_config c;
+    memset(&c, 0, sizeof(c));
+    if (cfg) c = *cfg;
+    c.forget = forget;
+    c.max_iters = 1;
+    c.fixed_iters = 0;
+    c.init = SLSTM_INIT_GIVEN;
+    c.guess_sweeps = 0;
+    c.carry_mode = SLSTM_CARRY_TWO_PASS;
+    c.debug_fault = 0;
+    return c;
+}
+
+template <int FORGET>
+cudaError_t cp_run_launch(const Args &a, bool sweep, cudaStream_t st)
+{
+    if (sweep) cp_tile_run_kernel<FORGET, true><<<a.n_tiles, NW * 32, 0, st>>>(a);
+    else cp_tile_run_kernel<FORGET, false><<<a.n_tiles, NW * 32, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t cp_workspace_bytes(int B, int T, int d) { return cp_layout(B, T, d).total; }
+
+cudaError_t cp_guess_run(const float *P, const float *R, const float *s_before, const float *S, bool sweep, int forget,
+                         float *run_out, int B, int T, int d, void *ws, cudaStream_t st)
+{
+    const slstm_newton_config cfg = cp_config(forget, nullptr);
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    cudaError_t e = prepare(P, R, nullptr, const_cast<float *>(S), cfg, nullptr, B, T, d, ws, st, nullptr, a, m,
+                            tma, two_pass);
+    if (e != cudaSuccess) return e;
+    a.s0h = s_before;
+    e = forget == SLSTM_FORGET_EXP ? cp_run_launch<SLSTM_FORGET_EXP>(a, sweep, st)
+                                   : cp_run_launch<SLSTM_FORGET_SIGMOID>(a, sweep, st);
+    if (e != cudaSuccess) return e;
+    const int n_chunks = a.n_tiles / a.n_groups;
+    cp_slice_run_kernel<<<(a.n_groups + 7) / 8, 256, 0, st>>>(a, n_chunks, run_out);
+    return cudaGetLastError();
+}
+
+cudaError_t cp_guess_apply(const float *P, const float *R, const float *s0, const float *s_before,
+                           const float *runs, int rank, float *S, bool sweep, int forget, int B, int T, int d,
+                           void *ws, cudaStream_t st)
+{
+    const CpLayout cl = cp_layout(B, T, d);
+    float *enter = reinterpret_cast<float *>(static_cast<char *>(ws) + cl.enter);
+    const long long nbd = (long long)B * d;
+    cp_enter_runs_kernel<<<(unsigned)((nbd + 255) / 256), 256, 0, st>>>(runs, rank, s0, B, d, enter);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    slstm_newton_config cfg = cp_config(forget, nullptr);
+    cfg.init = SLSTM_INIT_DECOUPLED;
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    if ((e = prepare(P, R, enter, S, cfg, nullptr, B, T, d, ws, st, nullptr, a, m, tma, two_pass)) != cudaSuccess)
+        return e;
+    a.s0h = s_before;
+    const int sms = sm_count();
+    if (!sweep) {
+        const Args a0 = launch_args(a, 0);
+        if (forget == SLSTM_FORGET_EXP)
+            return tma ? launch_guess<SLSTM_FORGET_EXP, false, true, false>(a0, m, 0, sms, st)
+                       : launch_guess<SLSTM_FORGET_EXP, false, false, false>(a0, m, 0, sms, st);
+        return tma ? launch_guess<SLSTM_FORGET_SIGMOID, false, true, false>(a0, m, 0, sms, st)
+                   : launch_guess<SLSTM_FORGET_SIGMOID, false, false, false>(a0, m, 0, sms, st);
+    }
+    // a sweep reads the previous guess's h at every tile's first step from
+    // the boundary buffer: gather it from S first (launch 0), then sweep as
+    // launch 1
+    const long long n = (long long)a.n_tiles * 128;
+    gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(launch_args(a, 0));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const Args a1 = launch_args(a, 1);
+    if (forget == SLSTM_FORGET_EXP)
+        return tma ? launch_guess<SLSTM_FORGET_EXP, true, true, false>(a1, m, 1, sms, st)
+                   : launch_guess<SLSTM_FORGET_EXP, true, false, false>(a1, m, 1, sms, st);
+    return tma ? launch_guess<SLSTM_FORGET_SIGMOID, true, true, false>(a1, m, 1, sms, st)
+               : launch_guess<SLSTM_FORGET_SIGMOID, true, false, false>(a1, m, 1, sms, st);
+}
+
+cudaError_t cp_newton_map(const float *P, const float *R, const float *s_before, const float *S, int forget,
+                          float *map_out, int B, int T, int d, void *ws, cudaStream_t st)
+{
+    const slstm_newton_config cfg = cp_config(forget, nullptr);
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    slstm_newton_stats *no_stats = nullptr;
+    cudaError_t e = prepare(P, R, s_before, const_cast<float *>(S), cfg, no_stats, B, T, d, ws, st, nullptr, a, m,
+                            tma, two_pass);
+    if (e != cudaSuccess) return e;
+    // the iterate's state at every tile's last step (launch 0), then the
+    // aggregate pass of iteration 1 and the block aggregates
+    const long long n = (long long)a.n_tiles * 128;
+    gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(launch_args(a, 0));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int sms = sm_count();
+    const Args a1 = launch_args(a, 1);
+    if (forget == SLSTM_FORGET_EXP)
+        e = tma ? launch_one<SLSTM_FORGET_EXP, false, false, true, false, MODE_AGG>(a1, m, 1, sms, st)
+                : launch_one<SLSTM_FORGET_EXP, false, false, false, false, MODE_AGG>(a1, m, 1, sms, st);
+    else
+        e = tma ? launch_one<SLSTM_FORGET_SIGMOID, false, false, true, false, MODE_AGG>(a1, m, 1, sms, st)
+                : launch_one<SLSTM_FORGET_SIGMOID, false, false, false, false, MODE_AGG>(a1, m, 1, sms, st);
+    if (e != cudaSuccess) return e;
+    const int n_chunks = a.n_tiles / a.n_groups;
+    TileScanArgs sa{a1.agg, a1.flags, a1.blk_agg, a1.blk_head, a1.blk_cin, a1.cin_buf, nullptr,
+                    a.n_groups, n_chunks, scan_blocks(n_chunks)};
+    const long long nw = (long long)sa.n_groups * sa.n_blk;
+    scan_block_agg<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cp_slice_map_kernel<<<(a.n_groups + 7) / 8, 256, 0, st>>>(a.blk_agg, a.n_groups, sa.n_blk, a.groups_per_row, d,
+                                                              map_out);
+    return cudaGetLastError();
+}
+
+cudaError_t cp_newton_apply(const float *P, const float *R, const float *s_before, const float *maps, int rank,
+                            float *S, const slstm_newton_config &user, slstm_newton_stats *stats, int B, int T, int d,
+                            void *ws, cudaStream_t st)
+{
+    const CpLayout cl = cp_layout(B, T, d);
+    float *enter = reinterpret_cast<float *>(static_cast<char *>(ws) + cl.enter);
+    const long long nbd = (long long)B * d;
+    cp_enter_maps_kernel<<<(unsigned)((nbd + 255) / 256), 256, 0, st>>>(maps, rank, B, d, enter);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const slstm_newton_config cfg = cp_config(user.forget, &user);
+    Args a;
+    NewtonMaps m;
+    bool tma = false, two_pass = false;
+    if ((e = prepare(P, R, s_before, S, cfg, stats, B, T, d, ws, st, nullptr, a, m, tma, two_pass)) != cudaSuccess)
+        return e;
+    // the tile aggregates, block aggregates and boundary states of
+    // cp_newton_map are still in the workspace; the carries start from the
+    // correction entering the slice
+    const int n_chunks = a.n_tiles / a.n_groups;
+    const Args a1 = launch_args(a, 1);
+    TileScanArgs sa{a1.agg, a1.flags, a1.blk_agg, a1.blk_head, a1.blk_cin, a1.cin_buf, &a1.ctrl->done,
+                    a.n_groups, n_chunks, scan_blocks(n_chunks)};
+    sa.cin0 = enter;
+    sa.gpr = a.groups_per_row;
+    sa.d = d;
+    scan_block_carry<<<(sa.n_groups + 7) / 8, 256, 0, st>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long nw = (long long)sa.n_groups * sa.n_blk;
+    scan_tile_carry<<<(unsigned)((nw + 7) / 8), 256, 0, st>>>(sa);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int sms = sm_count();
+    if (user.forget == SLSTM_FORGET_EXP)
+        return tma ? launch_one<SLSTM_FORGET_EXP, false, true, true, false, MODE_APPLY>(a1, m, 1, sms, st)
+                   : launch_one<SLSTM_FORGET_EXP, false, true, false, false, MODE_APPLY>(a1, m, 1, sms, st);
+    return tma ? launch_one<SLSTM_FORGET_SIGMOID, false, true, true, false, MODE_APPLY>(a1, m, 1, sms, st)
+               : launch_one<SLSTM_FORGET_SIGMOID, false, true, false, false, MODE_APPLY>(a1, m, 1, sms, st);
 }
 
 }  // namespace slstm

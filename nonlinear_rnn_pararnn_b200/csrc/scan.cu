@@ -36,6 +36,7 @@ struct ScanArgs {
     unsigned *ticket;
     CarryArgs ca;
     int T, d, groups_per_row, n_tiles, vec16;
+    int fault_ticket;   // this tile publishes nothing (host-requested fault injection), or -1
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
@@ -196,13 +197,15 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
             }
         }
         const bool fast = __syncthreads_and(ok);
+        const bool withhold = (int)ticket == a.fault_ticket;
         if (chain_warp) {
             if (fast) {
                 c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, 0u, CHAIN0);
-                st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+                if (!withhold) st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
                 named_bar_sync(CHAIN_BAR, 4 * 32);
             } else {
-                if (warp == CHAIN0) tile_carry_fallback<NW>(a.ca, sm.maps.m, sm.maps.cin, ticket, chunk, grp, false);
+                if (warp == CHAIN0)
+                    tile_carry_fallback<NW>(a.ca, sm.maps.m, sm.maps.cin, ticket, chunk, grp, withhold);
                 named_bar_sync(CHAIN_BAR, 4 * 32);
 #pragma unroll 1
                 for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
@@ -296,7 +299,7 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t st)
 size_t scan_workspace_bytes(int B, int T, int d) { return layout(B, T, d).total; }
 
 cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, float *y, int B,
-                               int T, int d, bool reverse, void *ws, cudaStream_t st)
+                               int T, int d, bool reverse, void *ws, cudaStream_t st, bool debug_withhold)
 {
     const Layout l = layout(B, T, d);
     char *base = static_cast<char *>(ws);
@@ -311,7 +314,10 @@ cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, 
     a.ca.incw = reinterpret_cast<unsigned long long *>(base + l.incw);
     a.ca.error = a.ticket + 1;
     a.ca.epoch = 1;
-    a.ca.wait_ns = 2000000000ull;
+    // fault injection: the first tile of chunk 1 publishes nothing, so the
+    // first tile of chunk 2 gives up after a short wait
+    a.fault_ticket = (debug_withhold && l.n_chunks >= 3) ? l.n_groups : -1;
+    a.ca.wait_ns = a.fault_ticket >= 0 ? 20000000ull : 2000000000ull;
     a.ca.n_groups = l.n_groups;
     a.T = T;
     a.d = d;

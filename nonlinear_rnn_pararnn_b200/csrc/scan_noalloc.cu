@@ -15,6 +15,8 @@
 // race on it and must be serialised by the caller.  The scan's ticket
 // counter and flag words are cleared on the stream at the start of every
 // call; the rest is overwritten before it is read.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -27,24 +29,53 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void *g_scratch_ptr[kMaxDevices] = {};
+// Per device: the context the address was looked up in, and the address.
+// A device reset ends that context; the next call runs in a new one and
+// looks the address up again.
+struct ScratchEntry {
+    CUcontext ctx;
+    void *ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of g_scan_scratch on the current device, looked up once per
-// device (the host-side name of the array is only a stand-in for it).
+PFN_cuCtxGetCurrent_v4000 ctx_getter()
+{
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    }
+    return fn;
+}
+
+// Device address of g_scan_scratch in the current device's current context,
+// looked up once per device and context (the host-side name of the array is
+// only a stand-in for it).
 cudaError_t scratch_on_current_device(void **out)
 {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    auto get_ctx = ctx_getter();
+    if (get_ctx == nullptr) return cudaErrorInitializationError;
+    // null before the runtime has made this device's context current here
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorInitializationError;
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_scratch_ptr[dev] == nullptr) {
+    ScratchEntry &s = g_scratch[dev];
+    if (ctx == nullptr || s.ptr == nullptr || s.ctx != ctx) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_scan_scratch);
+        e = cudaGetSymbolAddress(&p, g_scan_scratch);   // also initialises the context when needed
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+        if (ctx == nullptr && (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)) return cudaErrorInitializationError;
+        s.ctx = ctx;
+        s.ptr = p;
     }
-    *out = g_scratch_ptr[dev];
+    *out = s.ptr;
     return cudaSuccess;
 }
 

@@ -45,12 +45,21 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? SLSTM_OK : SLSTM_ERR_
 // The Newton configuration fields every forward entry point checks.
 bool config_ok(const slstm_newton_config &c)
 {
-    if (c.max_iters < 1 || c.max_iters > SLSTM_MAX_ITERS) return false;
+    if (c.max_iters < (c.init == SLSTM_INIT_DECOUPLED ? 0 : 1) || c.max_iters > SLSTM_MAX_ITERS) return false;
+    if (c.guess_sweeps < 0 || c.guess_sweeps > SLSTM_MAX_GUESS_SWEEPS) return false;
     if (c.forget != SLSTM_FORGET_SIGMOID && c.forget != SLSTM_FORGET_EXP) return false;
     if (!(c.tol >= 0.0f) || c.wait_limit_us < 0) return false;
     if (c.init < SLSTM_INIT_DECOUPLED || c.init > SLSTM_INIT_GIVEN) return false;
     if (c.residual_mode != SLSTM_RESIDUAL_SCALED && c.residual_mode != SLSTM_RESIDUAL_RAW) return false;
     return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
+}
+
+// Head mixing: whole heads of 1..SLSTM_MAX_HEAD_DIM features, one warp per
+// (batch row, head) on a one-dimensional grid.
+bool head_ok(int d_h, int d_head, int B)
+{
+    if (d_head < 1 || d_head > SLSTM_MAX_HEAD_DIM || d_h % d_head != 0) return false;
+    return (long long)B * (d_h / d_head) <= (1LL << 30);
 }
 
 // The trunk layer: K-major bf16 GEMMs over d_model (rows of 16 bytes) and a
@@ -102,6 +111,12 @@ size_t slstm_workspace_size(int op, int B, int T, int d_in, int d_h)
     case SLSTM_OP_NEWTON_BACKWARD_VARLEN:
         if (!varlen_sizes_ok(B, T, d_in, d_h)) return 0;
         return varlen_table_bytes(T) + backward_workspace_bytes(1, T, d_in, d_h);
+    case SLSTM_OP_CONTEXT_PARALLEL:
+        if (!sizes_ok(B, T, d_h, d_h)) return 0;
+        return cp_workspace_bytes(B, T, d_h);
+    case SLSTM_OP_NEWTON_BACKWARD_HEAD:
+        if (!sizes_ok(B, T, d_in, d_h)) return 0;
+        return head_backward_workspace_bytes(B, T, d_in, d_h, SLSTM_MAX_HEAD_DIM);
     default: return 0;
     }
 }
@@ -135,13 +150,109 @@ int slstm_newton_forward(const float *P, const float *R, const float *s0, float 
 int scan_block4(const float *A, const float *b, const float *y0, float *y, int B, int T, int d,
                 int flags, void *ws, size_t ws_bytes, slstm_stream_t stream)
 {
-    if ((flags & ~SLSTM_SCAN_REVERSE_T) != 0) return SLSTM_ERR_INVALID_ARG;
+    if ((flags & ~(SLSTM_SCAN_REVERSE_T | SLSTM_SCAN_DEBUG_WITHHOLD)) != 0) return SLSTM_ERR_INVALID_ARG;
     if (!sizes_ok(B, T, d, d)) return SLSTM_ERR_INVALID_ARG;
     if (!aligned16(A) || !aligned16(b) || !aligned16_or_null(y0) || !aligned16(y)) return SLSTM_ERR_INVALID_ARG;
     if (y == A || y == b) return SLSTM_ERR_INVALID_ARG;
     if (!ws_ok(ws, ws_bytes, scan_workspace_bytes(B, T, d))) return SLSTM_ERR_INVALID_ARG;
     return cuda_status(scan_block4_launch(A, b, y0, y, B, T, d, (flags & SLSTM_SCAN_REVERSE_T) != 0, ws,
-                                          static_cast<cudaStream_t>(stream)));
+                                          static_cast<cudaStream_t>(stream),
+                                          (flags & SLSTM_SCAN_DEBUG_WITHHOLD) != 0));
+}
+
+int slstm_cp_guess_run(const float *P, const float *R, const float *s_before, const float *S, int sweep, int forget,
+                       float *run, int B, int T, int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (sweep != 0 && sweep != 1) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16(run)) return SLSTM_ERR_INVALID_ARG;
+    if (sweep && (!aligned16(S) || !aligned16_or_null(s_before))) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, cp_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(cp_guess_run(P, R, s_before, S, sweep != 0, forget, run, B, T, d_h, ws,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_cp_guess_apply(const float *P, const float *R, const float *s0, const float *s_before, const float *runs,
+                         int rank, float *S, int sweep, int forget, int B, int T, int d_h, void *ws, size_t ws_bytes,
+                         slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (sweep != 0 && sweep != 1) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h) || rank < 0 || rank > 65535) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s0) || !aligned16_or_null(s_before) || !aligned16(S))
+        return SLSTM_ERR_INVALID_ARG;
+    if (rank > 0 && !aligned16(runs)) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, cp_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(cp_guess_apply(P, R, s0, s_before, runs, rank, S, sweep != 0, forget, B, T, d_h, ws,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_cp_newton_map(const float *P, const float *R, const float *s_before, const float *S, int forget, float *map,
+                        int B, int T, int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s_before) || !aligned16(S) || !aligned16(map))
+        return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, cp_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(cp_newton_map(P, R, s_before, S, forget, map, B, T, d_h, ws, static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_cp_newton_apply(const float *P, const float *R, const float *s_before, const float *maps, int rank,
+                          float *S, const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T, int d_h,
+                          void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (cfg == nullptr || !config_ok(*cfg)) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h) || rank < 0 || rank > 65535) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R) || !aligned16_or_null(s_before) || !aligned16(S) || !aligned16(stats))
+        return SLSTM_ERR_INVALID_ARG;
+    if (rank > 0 && !aligned16(maps)) return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, cp_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(cp_newton_apply(P, R, s_before, maps, rank, S, *cfg, stats, B, T, d_h, ws,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_sequential_step_head(const float *P, const float *R_head, const float *s0, float *S, int B, int T_steps,
+                               int d_h, int d_head, int forget, slstm_stream_t stream)
+{
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T_steps, d_h, d_h) || !head_ok(d_h, d_head, B)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R_head) || !aligned16_or_null(s0) || !aligned16(S)) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(head_sequential_launch(P, R_head, s0, S, B, T_steps, d_h, d_head, forget,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_newton_forward_head(const float *P, const float *R_head, const float *s0, float *S,
+                              const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T, int d_h,
+                              int d_head, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (cfg == nullptr || !config_ok(*cfg) || cfg->debug_fault != 0 || cfg->guess_sweeps != 0)
+        return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_h, d_h) || !head_ok(d_h, d_head, B)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(P) || !aligned16(R_head) || !aligned16_or_null(s0) || !aligned16(S) || !aligned16(stats))
+        return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, newton_workspace_bytes(B, T, d_h))) return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(head_newton_forward(P, R_head, s0, S, *cfg, stats, B, T, d_h, d_head, ws,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int slstm_newton_backward_head(const void *x, const void *Wx, int dtype, const float *P, const float *R_head,
+                               const float *s0, const float *S, const float *dH, float *dx, float *dWx,
+                               float *dR_head, float *db, float *ds0, int forget, int B, int T, int d_in, int d_h,
+                               int d_head, void *ws, size_t ws_bytes, slstm_stream_t stream)
+{
+    if (dtype != SLSTM_F32 && dtype != SLSTM_BF16) return SLSTM_ERR_INVALID_ARG;
+    if (forget != SLSTM_FORGET_SIGMOID && forget != SLSTM_FORGET_EXP) return SLSTM_ERR_INVALID_ARG;
+    if (!sizes_ok(B, T, d_in, d_h) || !head_ok(d_h, d_head, B)) return SLSTM_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(Wx) || !aligned16(P) || !aligned16(R_head) || !aligned16_or_null(s0) ||
+        !aligned16(S) || !aligned16(dH) || !aligned16(dx) || !aligned16(dWx) || !aligned16(dR_head) ||
+        !aligned16(db) || !aligned16_or_null(ds0))
+        return SLSTM_ERR_INVALID_ARG;
+    if (!ws_ok(ws, ws_bytes, head_backward_workspace_bytes(B, T, d_in, d_h, SLSTM_MAX_HEAD_DIM)))
+        return SLSTM_ERR_INVALID_ARG;
+    return cuda_status(head_backward_launch(x, Wx, dtype, P, R_head, s0, S, dH, dx, dWx, dR_head, db, ds0, forget,
+                                            B, T, d_in, d_h, d_head, ws, static_cast<cudaStream_t>(stream)));
 }
 
 int slstm_sequential_step(const float *P, const float *R, const float *s0, float *S, int B,

@@ -71,6 +71,15 @@ SLSTM_DEVINL void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, 
         : "memory");
 }
 
+SLSTM_DEVINL void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2, int c3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
 // Contiguous bulk copy global -> shared; size, src and dst multiples of 16 bytes.
 SLSTM_DEVINL void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
 {
@@ -123,5 +132,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // when the driver refuses (alignment: base and strides multiples of 16 bytes).
 bool make_map_f32_3d(CUtensorMap *map, const void *base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t ld1,
                      uint64_t ld2, uint32_t b0, uint32_t b1);
+
+// Host: fp32 tensor of dims (n0 contiguous, n1, n2, n3) with row strides ld1,
+// ld2, ld3 elements, box (b0, 1, b2, 1), no swizzle, zero fill out of bounds.
+bool make_map_f32_4d(CUtensorMap *map, const void *base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t n3,
+                     uint64_t ld1, uint64_t ld2, uint64_t ld3, uint32_t b0, uint32_t b2);
 
 }  // namespace slstm

@@ -65,7 +65,7 @@ def test_workspace_sizes():
 
 def _cfg(**kw):
     base = dict(max_iters=4, fixed_iters=0, tol=1e-5, forget=0, debug_fault=0, wait_limit_us=0, carry_mode=0,
-                init=0, residual_mode=0)
+                init=0, residual_mode=0, guess_sweeps=0)
     base.update(kw)
     return _lib.NewtonConfig(**base)
 
@@ -87,7 +87,7 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(S=FAKE_MIS) == E
     assert call(s0=FAKE_MIS) == E
     assert call(stats=NULL) == E
-    assert call(cfg=_cfg(max_iters=0)) == E
+    assert call(cfg=_cfg(max_iters=-1)) == E
     assert call(cfg=_cfg(max_iters=65537)) == E
     assert call(cfg=_cfg(forget=2)) == E
     assert call(cfg=_cfg(tol=float("nan"))) == E
@@ -96,6 +96,9 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(cfg=_cfg(init=3)) == E
     assert call(cfg=_cfg(init=-1)) == E
     assert call(cfg=_cfg(residual_mode=2)) == E
+    assert call(cfg=_cfg(guess_sweeps=-1)) == E
+    assert call(cfg=_cfg(guess_sweeps=65)) == E
+    assert call(cfg=_cfg(max_iters=0, init=1)) == E      # only the decoupled guess allows 0 iterations
     assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
     assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
     assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E
@@ -142,7 +145,7 @@ def test_varlen_entry_points_reject_bad_arguments():
     assert fwd(n=65, total=64) == E                   # more sequences than steps
     assert fwd(total=0) == E
     assert fwd(S=FAKE_MIS) == E
-    assert fwd(cfg=_cfg(max_iters=0)) == E
+    assert fwd(cfg=_cfg(max_iters=-1)) == E
     assert fwd(wb=ctypes.c_size_t(64)) == E
     assert lib.slstm_newton_forward_varlen(FAKE, FAKE, NULL, cu, 3, FAKE, None, FAKE, 64, 8, FAKE, big, NULL) == E
     # (x, Wx, dtype, P, R, s0, cu, n_seq, S, dH, dx, dWx, dR, db, ds0, forget, total_T, d_in, d_h, ws, bytes, stream)
@@ -187,7 +190,7 @@ def test_block_entry_point_rejects_bad_arguments():
     assert fwd(B=0) == E and fwd(T=0) == E
     assert fwd(eps=-1.0) == E and fwd(eps=float("nan")) == E
     assert fwd(x=FAKE_MIS) == E
-    assert fwd(cfg=_cfg(max_iters=0)) == E
+    assert fwd(cfg=_cfg(max_iters=-1)) == E
     assert fwd(wb=ctypes.c_size_t(64)) == E     # workspace too small
     assert fwd(S=ctypes.c_void_p(0x10000 + 256)) == E   # y and S overlap
     assert lib.slstm_block_workspace_size(2, 16, 60, 256) == 0

@@ -104,8 +104,9 @@ def _setup(w):
 def test_fullsize_forward_sampled(name, cuda_device):
     """Every step of the sampled lanes: the sequential stepping, the Newton
     iterate after the fixed K of the workload (against the fp64 iterate after
-    the same K from the same decoupled guess), and the converged tolerance
-    run (against the sequential trajectory)."""
+    the same K from the same guess: the decoupled trajectory and its default
+    refinement sweeps), and the converged tolerance run (against the
+    sequential trajectory)."""
     w = WORKLOADS[name]
     inp, P, R, s0, lanes, Pl, Rl, s0l = _setup(w)
     Sseq = api.sequential_step(P, R, s0, forget=w.forget)
@@ -123,14 +124,14 @@ def test_fullsize_forward_sampled(name, cuda_device):
     Snt, st = api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, fixed=True, tol=w.tol)
     stats = api.read_stats(st)
     assert stats["iters"] == K and stats["error"] == 0, stats
-    SK, _ = oracle.newton(Pl, Rl, s0l, w.forget, max_iters=K, fixed=True, tol=w.tol)
+    SK, _ = oracle.newton(Pl, Rl, s0l, w.forget, max_iters=K, fixed=True, tol=w.tol, sweeps=api.DEFAULT_GUESS_SWEEPS)
     e_fix = _serr(_gather(Snt, lanes), SK)
     assert e_fix <= tol, e_fix
     del Snt
 
     Sc, stc = api.newton_forward(P, R, s0, forget=w.forget, max_iters=w.max_iters, fixed=False, tol=w.tol)
     cst = api.read_stats(stc)
-    _, ost = oracle.newton(Pl, Rl, s0l, w.forget, max_iters=w.max_iters, tol=w.tol)
+    _, ost = oracle.newton(Pl, Rl, s0l, w.forget, max_iters=w.max_iters, tol=w.tol, sweeps=api.DEFAULT_GUESS_SWEEPS)
     print(f"{name}: P err {perr:.2e}, sequential h err {e_seq:.2e}, K={K} iterate err {e_fix:.2e}; "
           f"tolerance run: GPU {cst['iters']} iterations (all lanes) scaled residuals {cst['max_scaled_F']}, "
           f"fp64 {ost['iters']} iterations (sampled lanes) {list(ost['max_scaled_F'])}")

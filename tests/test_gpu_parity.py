@@ -20,6 +20,8 @@ pytestmark = pytest.mark.gpu
 
 TOL_F32 = 1e-4
 TOL_BF16 = 5e-3
+# refinement sweeps of the decoupled guess that the library's Python calls use by default
+SW = api.DEFAULT_GUESS_SWEEPS
 
 
 def _dev(t):
@@ -128,7 +130,8 @@ def test_newton_tiny_converges_to_sequential(cuda_device):
     w = WORKLOADS["tiny_f32"]
     inp, S, st, Pref = _newton_case(w)
     ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
-    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol,
+                                sweeps=SW)
     print("gpu stats", st, "oracle iters", ost["iters"])
     assert st["error"] == 0 and not st["diverged"]
     assert st["converged"]
@@ -160,7 +163,7 @@ def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, init, cud
     w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
     inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode, init=init)
     _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol,
-                                init=init)
+                                init=init, sweeps=SW)
     converged = _check_status_against_oracle(st, ost)
     if init == "decoupled":
         assert converged, (st, ost["iters"])
@@ -174,15 +177,16 @@ def _s_err(S_gpu, S_ref):
     return float((np.abs(S_gpu - S_ref) / (1 + np.abs(S_ref))).max())
 
 
-@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+@pytest.mark.parametrize("sweeps", [0, 2])
 @pytest.mark.parametrize("forget", ["sigmoid", "exp"])
 @pytest.mark.parametrize("B,T,d,s0_random", [(2, 50, 40, True), (1, 1, 1, False), (3, 64, 70, True),
                                               (1, 3000, 36, True), (2, 4100, 64, False)])
-def test_newton_decoupled_guess_matches_oracle(forget, B, T, d, s0_random, carry_mode, cuda_device):
-    """The guess launch alone (its test passes at any tolerance): every slot of
-    the decoupled trajectory against the oracle's, across many tiles and the
-    look-back over up to 65 chunks of 64 steps."""
-    w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 17, 1e30, 4)
+def test_newton_decoupled_guess_matches_oracle(forget, B, T, d, s0_random, sweeps, cuda_device):
+    """The guess launches alone (max_iters = 0 returns the guess): every slot
+    of the decoupled trajectory, and of its refinement sweeps, against the
+    oracle's, across many tiles and the look-back over up to 65 chunks of 64
+    steps (the TMA path for d % 4 == 0, the cp.async path otherwise)."""
+    w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 17, 1e-6, 4)
     inp = make_inputs(w, with_dH=False)
     s0 = inp["s0"]
     if s0_random:
@@ -190,15 +194,18 @@ def test_newton_decoupled_guess_matches_oracle(forget, B, T, d, s0_random, carry
         s0 = torch.stack([torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) + 0.5,
                           torch.randn(B, d, generator=g), torch.rand(B, d, generator=g) - 0.5], dim=1)
     Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
-    S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(s0), forget=forget, max_iters=4, fixed=False, tol=1e30,
-                               carry_mode=carry_mode)
+    S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(s0), forget=forget, max_iters=0, guess_sweeps=sweeps)
     s = api.read_stats(st)
-    assert s["iters"] == 0 and s["converged"] and s["error"] == 0, s
+    assert s["iters"] == 0 and not s["converged"] and s["error"] == 0 and s["init_max_abs_F"] == -1.0, s
     Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
-    Sg, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(s0), forget, 4, False, 1e30)
+    Sg, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(s0), forget, 0, False, 1e-6, sweeps=sweeps)
     assert ost["iters"] == 0
     assert _s_err(as_f64(S.cpu()), Sg) <= TOL_F32
-    g, o = s["init_max_scaled_F"], ost["init_max_scaled_F"]
+    # the first iteration records the guess's residual
+    _, st1 = api.newton_forward(Pt, _dev(inp["R"]), _dev(s0), forget=forget, max_iters=1, tol=1e-30,
+                                guess_sweeps=sweeps)
+    _, ost1 = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(s0), forget, 1, False, 1e-30, sweeps=sweeps)
+    g, o = api.read_stats(st1)["init_max_scaled_F"], ost1["init_max_scaled_F"]
     assert abs(g - o) <= 1e-3 * (1 + o), (g, o)
 
 
@@ -210,7 +217,8 @@ def test_newton_converges_where_zero_guess_diverges(forget, T, carry_mode, cuda_
     iterations as the fp64 run."""
     w = Workload("t", 2, T, 16, 40, "f32", forget, 0.5, 23, 1e-5, 16)
     inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode)
-    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol)
+    _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol,
+                                sweeps=SW)
     print("gpu", st["iters"], st["max_scaled_F"], "oracle", ost["iters"], list(ost["max_scaled_F"]))
     assert st["converged"] and st["error"] == 0, st
     assert ost["converged"] and abs(st["iters"] - ost["iters"]) <= 1
@@ -226,7 +234,7 @@ def test_newton_raw_residual_mode(cuda_device):
     w = scaled(WORKLOADS["tiny_f32"], tol=1e-4)
     inp, S, st, Pref = _newton_case(w, residual_mode="raw")
     _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol,
-                                residual_mode="raw")
+                                residual_mode="raw", sweeps=SW)
     print("gpu", st, "oracle", ost)
     assert st["converged"] and ost["converged"]
     assert st["max_abs_F"][-1] <= w.tol
@@ -345,3 +353,41 @@ def test_backward_matches_oracle_bptt(forget, B, T, d_in, d, dtype, cuda_device)
         got = as_f64(out[k].cpu())
         err = np.abs(got - ref[k]).max() / (1 + np.abs(ref[k]).max())
         assert err <= 1e-4, (k, err)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_scan_block4_bounded_wait_poisons_outputs(reverse, cuda_device):
+    """Fault injection on the host's request: a tile withholds its carry; the
+    successor's bounded wait expires and, instead of using a made-up carry,
+    it makes every output that depends on the missing one NaN.  Nothing is
+    silently wrong: every finite output equals the oracle's (tiles that a
+    stalled CTA held back may have given up too, and are NaN as well), the
+    steps before the withheld carry are finite, and the context stays
+    usable."""
+    B, T, d = 2, 200, 64
+    g = torch.Generator().manual_seed(77)
+    A = (torch.rand(B, T, 4, 4, d, generator=g) * 0.6 - 0.3)
+    b = torch.randn(B, T, 4, d, generator=g)
+    flags = api._lib.SLSTM_SCAN_DEBUG_WITHHOLD | (api._lib.SLSTM_SCAN_REVERSE_T if reverse else 0)
+    Ad, bd = _dev(A), _dev(b)
+    y = torch.empty_like(bd)
+    ws = api.workspace(api._lib.SLSTM_OP_SCAN_BLOCK4, B, T, 0, d, bd.device)
+    rc = api.load().scan_block4(api._ptr(Ad), api._ptr(bd), None, api._ptr(y), B, T, d, flags, api._ptr(ws),
+                                ws.numel(), api._stream())
+    assert rc == 0
+    torch.cuda.synchronize()
+    got = y.cpu()
+    Al = np.transpose(as_f64(A), (0, 4, 1, 2, 3)).reshape(B * d, T, 4, 4)
+    bl = np.transpose(as_f64(b), (0, 3, 1, 2)).reshape(B * d, T, 4)
+    ref = np.transpose(oracle.affine_solve(Al, bl, None, reverse=reverse).reshape(B, d, T, 4), (0, 2, 3, 1))
+    late = slice(0, T - 64) if reverse else slice(64, T)
+    early = slice(T - 64, T) if reverse else slice(0, 64)
+    assert torch.isnan(got[0, late, :, :32]).all()
+    fin = np.isfinite(as_f64(got))
+    err = np.abs(as_f64(got)[fin] - ref[fin]).max() / (1 + np.abs(ref).max())
+    assert err < 1e-5, err
+    assert np.isfinite(as_f64(got[0, early])).all()
+    # a normal call afterwards is unaffected
+    y2 = api.scan_block4(Ad, bd, None, reverse=reverse)
+    torch.cuda.synchronize()
+    assert np.abs(as_f64(y2.cpu()) - ref).max() / (1 + np.abs(ref).max()) < 1e-5

@@ -72,7 +72,8 @@ def test_varlen_fixed_k_matches_oracle(lengths, d, forget, carry_mode, cuda_devi
     assert api.read_stats(st)["iters"] == K
     # The whole iterate after K iterations from the decoupled guess of every
     # sequence, against the fp64 iterate of each sequence on its own.
-    ref = oracle.newton_varlen_fixed(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy(), forget, K)
+    ref = oracle.newton_varlen_fixed(Pref, as_f64(c["R"]), as_f64(c["s0"]), c["cu"].numpy(), forget, K,
+                                     sweeps=api.DEFAULT_GUESS_SWEEPS)
     assert float((np.abs(got - ref) / (1 + np.abs(ref))).max()) <= TOL_F32
     # Newton's prefix exactness, per sequence: after K iterations the first K
     # steps of every sequence are the sequential trajectory; a carry leaking

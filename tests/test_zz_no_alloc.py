@@ -6,15 +6,20 @@ or they are plugins handed only input and output pointers), so it brings
 its scratch from a fixed block of device memory inside the library.  This
 test calls it through the C ABI twice in a row, on different problems and
 directions, and checks each result against the workspace-taking scan_block4
-within the scan tests' tolerance; it also checks the size limit is reported
-before any work is enqueued.  The file is named to run last.
+within the scan tests' tolerance; it runs the largest problem the block
+holds, in both directions, against the fp64 oracle, and checks that the size
+limit is reported before any work is enqueued.  The file is named to run
+last.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from nonlinear_rnn_pararnn_b200 import _lib, api
+from nonlinear_rnn_pararnn_b200.workloads import as_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +53,27 @@ def test_noalloc_matches_scan_block4_twice(cuda_device):
         torch.cuda.synchronize()
         err = ((y - ref).abs().max() / (1 + ref.abs().max())).item()
         assert err < 1e-5, (B, T, d, err)
+
+
+@pytest.mark.parametrize("reverse", [False, True])
+def test_noalloc_largest_accepted_problem_matches_oracle(reverse, cuda_device):
+    """The largest problem the fixed block holds (2337 tiles of 32 steps x 32
+    features, within a few KB of the block's end), against the fp64
+    sequential solve of the oracle over the full length."""
+    B, T, d = 1, 2337 * 32, 32
+    lib = _lib.load()
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_SCAN_BLOCK4, B, T, 0, d) <= _lib.SLSTM_NOALLOC_SCRATCH_BYTES
+    assert lib.slstm_workspace_size(_lib.SLSTM_OP_SCAN_BLOCK4, B, T + 32, 0, d) > _lib.SLSTM_NOALLOC_SCRATCH_BYTES
+    A, b, y0 = _problem(B, T, d, 23, True)
+    y = torch.full_like(b, float("nan"))
+    assert _noalloc(A, b, y0, y, reverse) == _lib.SLSTM_OK
+    torch.cuda.synchronize()
+    Al = np.transpose(as_f64(A.cpu()), (0, 4, 1, 2, 3)).reshape(B * d, T, 4, 4)
+    bl = np.transpose(as_f64(b.cpu()), (0, 3, 1, 2)).reshape(B * d, T, 4)
+    y0l = np.transpose(as_f64(y0.cpu()), (0, 2, 1)).reshape(B * d, 4)
+    ref = np.transpose(oracle.affine_solve(Al, bl, y0l, reverse=reverse).reshape(B, d, T, 4), (0, 2, 3, 1))
+    err = np.abs(as_f64(y.cpu()) - ref).max() / (1 + np.abs(ref).max())
+    assert err < 1e-5, err
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_device):
