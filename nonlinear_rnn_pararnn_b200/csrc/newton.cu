@@ -39,6 +39,10 @@ namespace slstm {
 namespace {
 
 constexpr int NW = 16;   // warps per tile (time segments)
+// Guess stages (the decoupled guess and its sweeps) that one launch runs per
+// tile; each has its own look-back state (flags, runs in the aggregate
+// buffer, published states).
+constexpr int GUESS_STAGES = 4;
 // How a launch gets the carry entering each tile.  FUSED: from the tile
 // before it in the same launch (decoupled look-back).  With few feature
 // groups most tiles would wait on their predecessors, so an iteration can
@@ -76,6 +80,7 @@ struct Args {
     unsigned long long wait_ns;
     int B, T, d, groups_per_row, n_groups, n_tiles, max_iters, fixed, fault_ticket, vec16;
     int k0;             // launches before the first Newton iteration (the guess and its sweeps)
+    int guess_sweeps;   // refinement sweeps of the decoupled guess
     int resid_raw;      // stopping test on max|F| (else on the scaled residual)
     int guess_tested;   // the first iteration records the residual of the guess
     float tol;
@@ -339,6 +344,7 @@ struct GuessSmem {
     float O[TT][4][32];      // TMA path: S of the tile, source of the warps' TMA stores
     float seg[5][32][SEG_LD];   // each warp's run (A, mu, u, v, o), then the inclusive prefixes
     float cin[4][32];        // state (c, n, m, h) entering the tile
+    float hlast[NW][32];     // in-tile sweeps: the stage before's h at each warp's last step
     float hb[2][32];         // sweeps: h of the previous guess just before the tile
     TileInfo info[3];
     uint64_t bar[2];
@@ -436,15 +442,30 @@ SLSTM_DEVINL void seg_enter(const Seg &x, const float v[4], float out[4])
     out[3] = guess_h(x.o, out[0], out[1]);
 }
 
+// One guess stage's look-back state: per tile a flag word, the tile's run
+// (5 x 32 floats: A, mu, u, v, o) and its published state (4 x 32 words).
+struct GuessChain {
+    unsigned *flags;
+    float *runs;
+    unsigned long long *incw;
+};
+
+SLSTM_DEVINL GuessChain guess_chain(const Args &a, int stage)
+{
+    const size_t n = (size_t)a.n_tiles;
+    return GuessChain{a.flags + stage * n, a.agg + stage * n * 160, a.incw + stage * n * 128};
+}
+
 // The guess's look-back when the predecessor's state is not published yet
 // (warp 0, lane = feature, chunk > 0): publishes this tile's run, then
 // composes the runs of unfinished predecessors until it meets a published
 // state.  Returns the state (c, n, m, h) entering the tile in v.
-SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket, int chunk, int grp, float v[4])
+SLSTM_DEVINL void guess_lookback(const Args &a, const GuessChain &gc, const Seg &tile, unsigned ticket, int chunk,
+                                 int grp, float v[4])
 {
     const int lane = threadIdx.x & 31;
     {
-        float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
+        float *dst = gc.runs + (size_t)ticket * 160 + lane;
         dst[0] = tile.A;
         dst[32] = tile.mu;
         dst[64] = tile.u;
@@ -452,14 +473,14 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
         dst[128] = tile.o;
         __threadfence();
         __syncwarp();
-        if (lane == 0) st_release(a.flags + ticket, (a.epoch << 2) | FLAG_AGG | (tile.head ? FLAG_HEAD : 0u));
+        if (lane == 0) st_release(gc.flags + ticket, (a.epoch << 2) | FLAG_AGG | (tile.head ? FLAG_HEAD : 0u));
     }
     Seg M;            // composition of the runs met so far (latest last)
     bool have = false;
     int q = chunk - 1;
     const uint64_t t0 = globaltimer_ns();
     unsigned polls = 0;
-    const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+    const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
     for (;;) {
         const unsigned tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
         float w[4];
@@ -471,9 +492,9 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
             }
             return;
         }
-        const unsigned f = ld_acquire(a.flags + tq);
+        const unsigned f = ld_acquire(gc.flags + tq);
         if ((f >> 2) == a.epoch && (f & FLAG_AGG)) {
-            const float *src = a.agg + (size_t)tq * 20 * 32 + lane;
+            const float *src = gc.runs + (size_t)tq * 160 + lane;
             Seg x;
             x.A = __ldcg(src);
             x.mu = __ldcg(src + 32);
@@ -504,22 +525,27 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const Seg &tile, unsigned ticket
     }
 }
 
-// The decoupled guess (SWEEP false), or one refinement sweep of it (SWEEP
-// true: the gates of step t see r h_{t-1} of the previous guess, read from S
-// before this launch overwrites it and, at a tile's first step, from the
-// previous launch's boundary buffer).  One launch over every tile; launch k
-// of the solve (epoch k + 1, control slot k & 1).
+// The decoupled guess and its refinement sweeps, NS stages per tile in one
+// launch.  Stage 0 is the decoupled guess (SWEEP false) or a sweep of the
+// guess that S holds (SWEEP true: the gates see r h_{t-1} of S, read before
+// this launch overwrites it and, at a tile's first step, from the previous
+// launch's boundary buffer); every later stage is a sweep of the stage before
+// it, whose h never leaves the CTA.  Stage s of a tile takes its entering
+// state from stage s of the tile before (its own flags, runs and published
+// states), so the stages pipeline across tiles like one scan each.  One
+// launch over every tile; launch k of the solve (epoch k + 1, control slot
+// k & 1).  Per stage:
 //   walk A  each thread folds its 4 steps into a run;
 //   scan    the 16 warp runs of each feature are scanned (inclusive) by a
 //           Kogge-Stone scan over 16 lanes, two features per warp, so that
-//           the tile's aggregate run and every warp's prefix are known
-//           without a serial walk;
+//           the tile's run and every warp's prefix are known without a
+//           serial walk;
 //   carry   warp 0 takes the state entering the tile (the predecessor's
-//           published state, or the look-back) and publishes the tile's
-//           state;
-//   walk B  each warp enters its steps through its prefix and replays them,
-//           writing S and the tile's last state for the next launch.
-template <int FORGET, bool SWEEP, bool TMA, bool VARLEN>
+//           published state, or the look-back) and publishes the tile's;
+//   walk B  each warp enters its steps through its prefix and replays them;
+//           the last stage writes S and the tile's last state for the next
+//           launch.
+template <int FORGET, int NS, bool SWEEP, bool TMA, bool VARLEN>
 __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const __grid_constant__ NewtonMaps maps)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -527,6 +553,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     NewtonSlot &slot = a.ctrl->slot[k & 1];
+    constexpr bool ANY_SWEEP = SWEEP || NS > 1;
 
     if (threadIdx.x == 0) {
         sm.exit_flag = (int)*(volatile unsigned *)&a.ctrl->done;
@@ -582,68 +609,12 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
         const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
         const int t_seg = chunk * TT + warp * L;
 
-        // recurrent weights and the previous guess's h before this warp's
-        // first step (sweeps)
-        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f, hprev = 0.f;
-        if (SWEEP) {
-            if (jv) {
-                rz = __ldg(a.R + jj);
-                ri = __ldg(a.R + d + jj);
-                rf = __ldg(a.R + 2 * d + jj);
-                ro = __ldg(a.R + 3 * d + jj);
-            }
-            if (warp > 0) hprev = sm.Hs[st][warp * L - 1][lane];
-            else if (chunk > 0) hprev = sm.hb[st][lane];
-            else if (!VARLEN && a.s0h && jv) hprev = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
-        }
-
-        // ---- walk A: this warp's run, lane = feature ----
-        float gz[L], glf[L], go[L], gi[L];
-        {
-            Seg run;
-            float hp = hprev;
-#pragma unroll
-            for (int i = 0; i < L; ++i) {
-                const int sl = warp * L + i;
-                const bool head = VARLEN && ((ti.mask >> sl) & 1ull);
-                if (SWEEP && head) {
-                    // a sequence starts here: its previous h is its own s0's
-                    float s0v[4];
-                    head_state(a, t_seg + i, jj, jv, s0v);
-                    hp = s0v[3];
-                }
-                float pz = sm.P[st][sl][0][lane], pi = sm.P[st][sl][1][lane], pf = sm.P[st][sl][2][lane],
-                      po = sm.P[st][sl][3][lane];
-                if (SWEEP) {
-                    pz = fmaf(rz, hp, pz);
-                    pi = fmaf(ri, hp, pi);
-                    pf = fmaf(rf, hp, pf);
-                    po = fmaf(ro, hp, po);
-                    hp = sm.Hs[st][sl][lane];
-                }
-                guess_gates<FORGET>(pz, pf, po, gz[i], glf[i], go[i]);
-                gi[i] = pi;
-                if (head) {
-                    float s0v[4];
-                    head_state(a, t_seg + i, jj, jv, s0v);
-                    run.mu = s0v[2];
-                    run.u = s0v[0];
-                    run.v = s0v[1];
-                    seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
-                    run.head = true;
-                } else if (i == 0) {
-                    run.A = glf[i];
-                    run.mu = gi[i];
-                    run.u = gz[i];
-                    run.v = 1.0f;
-                    run.head = false;
-                } else {
-                    seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
-                    run.A += glf[i];
-                }
-                run.o = go[i];
-            }
-            seg_store(sm, warp, lane, run);
+        float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
+        if (ANY_SWEEP && jv) {
+            rz = __ldg(a.R + jj);
+            ri = __ldg(a.R + d + jj);
+            rf = __ldg(a.R + 2 * d + jj);
+            ro = __ldg(a.R + 3 * d + jj);
         }
         if (threadIdx.x == 0) {
             unsigned wh = 0u;
@@ -654,92 +625,170 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
             }
             sm.whead = wh;
         }
-        __syncthreads();
 
-        // ---- scan of the warp runs: lane (feature 2 warp + lane / 16, run lane % 16) ----
-        const unsigned whead = sm.whead;
-        {
-            const int f = 2 * warp + (lane >> 4), w = lane & 15;
-            Seg x;
-            seg_load(sm, w, f, x, ((whead >> w) & 1u) != 0u);
+        float hs[L];   // h of this thread's steps in the stage before (sweeps)
+        float sv[4];   // the state after this thread's last step in the current stage
 #pragma unroll
-            for (int off = 1; off < NW; off *= 2) {
-                Seg y;
-                y.A = __shfl_up_sync(0xffffffffu, x.A, off, 16);
-                y.mu = __shfl_up_sync(0xffffffffu, x.mu, off, 16);
-                y.u = __shfl_up_sync(0xffffffffu, x.u, off, 16);
-                y.v = __shfl_up_sync(0xffffffffu, x.v, off, 16);
-                y.o = __shfl_up_sync(0xffffffffu, x.o, off, 16);
-                y.head = __shfl_up_sync(0xffffffffu, x.head ? 1 : 0, off, 16) != 0;
-                if (w >= off) seg_compose(x, y, x);
-            }
-            seg_store(sm, w, f, x);
-            // the inclusive prefix's head flag: any run up to w holds a head
-        }
-        __syncthreads();
+        for (int i = 0; i < L; ++i) hs[i] = 0.f;
 
-        // ---- carry: warp 0, lane = feature ----
-        if (warp == 0) {
-            float v[4] = {0.f, 0.f, 0.f, 0.f};
-            Seg tile;
-            seg_load(sm, NW - 1, lane, tile, whead != 0u);
-            if (chunk == 0) {
-                if (!VARLEN && a.s0 && jv) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
+#pragma unroll 1
+        for (int stage = 0; stage < NS; ++stage) {
+            const bool sweep = stage > 0 || SWEEP;
+            const GuessChain gc = guess_chain(a, stage);
+            // the gates' h before this warp's first step: the stage before's
+            // state at step t_seg - 1
+            float hp = 0.f;
+            if (sweep) {
+                if (stage == 0) {
+                    if (warp > 0) hp = sm.Hs[st][warp * L - 1][lane];
+                    else if (chunk > 0) hp = sm.hb[st][lane];
+                    else if (!VARLEN && a.s0h && jv) hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
+                } else {
+                    hp = warp > 0 ? sm.hlast[warp - 1][lane] : sm.cin[3][lane];
                 }
-            } else {
-                const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-                const bool ok = read_inc_words(ca, ticket - G, lane, v);
-                if (!__all_sync(0xffffffffu, ok))
-                    guess_lookback(a, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
             }
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sm.cin[e][lane] = v[e];
-            float vo[4];
-            seg_enter(tile, v, vo);
-            unsigned long long *dst = a.incw + (size_t)ticket * 4 * 32 + lane;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
-        }
-        __syncthreads();
 
-        // ---- walk B: enter this warp's steps through the prefix before it ----
-        if (TMA) {
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
-        }
-        float sv[4];
-        {
-            float cv[4];
+            // ---- walk A: this warp's run, lane = feature ----
+            float gz[L], glf[L], go[L], gi[L];
+            {
+                Seg run;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) cv[e] = sm.cin[e][lane];
-            if (warp == 0) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sv[e] = cv[e];
-            } else {
-                // whether the prefix of runs 0 .. warp - 1 holds a sequence start
-                const bool ph = (whead & ((1u << warp) - 1u)) != 0u;
-                Seg x;
-                seg_load(sm, warp - 1, lane, x, ph);
-                seg_enter(x, cv, sv);
+                for (int i = 0; i < L; ++i) {
+                    const int sl = warp * L + i;
+                    const bool head = VARLEN && ((ti.mask >> sl) & 1ull);
+                    if (sweep && head) {
+                        // a sequence starts here: its previous h is its own s0's
+                        float s0v[4];
+                        head_state(a, t_seg + i, jj, jv, s0v);
+                        hp = s0v[3];
+                    }
+                    float pz = sm.P[st][sl][0][lane], pi = sm.P[st][sl][1][lane], pf = sm.P[st][sl][2][lane],
+                          po = sm.P[st][sl][3][lane];
+                    if (sweep) {
+                        pz = fmaf(rz, hp, pz);
+                        pi = fmaf(ri, hp, pi);
+                        pf = fmaf(rf, hp, pf);
+                        po = fmaf(ro, hp, po);
+                        hp = stage == 0 ? sm.Hs[st][sl][lane] : hs[i];
+                    }
+                    guess_gates<FORGET>(pz, pf, po, gz[i], glf[i], go[i]);
+                    gi[i] = pi;
+                    if (head) {
+                        float s0v[4];
+                        head_state(a, t_seg + i, jj, jv, s0v);
+                        run.mu = s0v[2];
+                        run.u = s0v[0];
+                        run.v = s0v[1];
+                        seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
+                        run.head = true;
+                    } else if (i == 0) {
+                        run.A = glf[i];
+                        run.mu = gi[i];
+                        run.u = gz[i];
+                        run.v = 1.0f;
+                        run.head = false;
+                    } else {
+                        seg_apply(glf[i], gi[i], gz[i], 1.0f, run.mu, run.u, run.v);
+                        run.A += glf[i];
+                    }
+                    run.o = go[i];
+                }
+                seg_store(sm, warp, lane, run);
             }
-        }
-        float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
+            __syncthreads();
+
+            // ---- scan of the warp runs: lane (feature 2 warp + lane / 16, run lane % 16) ----
+            const unsigned whead = sm.whead;
+            {
+                const int f = 2 * warp + (lane >> 4), w = lane & 15;
+                Seg x;
+                seg_load(sm, w, f, x, ((whead >> w) & 1u) != 0u);
 #pragma unroll
-        for (int i = 0; i < L; ++i) {
-            const int sl = warp * L + i;
-            const bool wr = jv && (t_seg + i < T);
-            if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, sv);
-            seg_apply(glf[i], gi[i], gz[i], 1.0f, sv[2], sv[0], sv[1]);
-            sv[3] = guess_h(go[i], sv[0], sv[1]);
-            if (TMA) {
+                for (int off = 1; off < NW; off *= 2) {
+                    Seg y;
+                    y.A = __shfl_up_sync(0xffffffffu, x.A, off, 16);
+                    y.mu = __shfl_up_sync(0xffffffffu, x.mu, off, 16);
+                    y.u = __shfl_up_sync(0xffffffffu, x.u, off, 16);
+                    y.v = __shfl_up_sync(0xffffffffu, x.v, off, 16);
+                    y.o = __shfl_up_sync(0xffffffffu, x.o, off, 16);
+                    y.head = __shfl_up_sync(0xffffffffu, x.head ? 1 : 0, off, 16) != 0;
+                    if (w >= off) seg_compose(x, y, x);
+                }
+                seg_store(sm, w, f, x);
+            }
+            __syncthreads();
+
+            // ---- carry: warp 0, lane = feature ----
+            if (warp == 0) {
+                float v[4] = {0.f, 0.f, 0.f, 0.f};
+                Seg tile;
+                seg_load(sm, NW - 1, lane, tile, whead != 0u);
+                if (chunk == 0) {
+                    if (!VARLEN && a.s0 && jv) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sv[e];
-            } else {
+                        for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
+                    }
+                } else {
+                    const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                    const bool ok = read_inc_words(ca, ticket - G, lane, v);
+                    if (!__all_sync(0xffffffffu, ok))
+                        guess_lookback(a, gc, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
+                }
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (wr) srow[(size_t)i * 4 * d + e * d] = sv[e];
+                for (int e = 0; e < 4; ++e) sm.cin[e][lane] = v[e];
+                float vo[4];
+                seg_enter(tile, v, vo);
+                unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + lane;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
+            }
+            __syncthreads();
+
+            // ---- walk B: enter this warp's steps through the prefix before it ----
+            {
+                float cv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cv[e] = sm.cin[e][lane];
+                if (warp == 0) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sv[e] = cv[e];
+                } else {
+                    // whether the prefix of runs 0 .. warp - 1 holds a sequence start
+                    const bool ph = (whead & ((1u << warp) - 1u)) != 0u;
+                    Seg x;
+                    seg_load(sm, warp - 1, lane, x, ph);
+                    seg_enter(x, cv, sv);
+                }
+            }
+            const bool last = stage == NS - 1;
+            if (last && TMA) {
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+            }
+            float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                const int sl = warp * L + i;
+                if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, sv);
+                seg_apply(glf[i], gi[i], gz[i], 1.0f, sv[2], sv[0], sv[1]);
+                sv[3] = guess_h(go[i], sv[0], sv[1]);
+                hs[i] = sv[3];
+                if (last) {
+                    const bool wr = jv && (t_seg + i < T);
+                    if (TMA) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sv[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (wr) srow[(size_t)i * 4 * d + e * d] = sv[e];
+                    }
+                }
+            }
+            if (!last) {
+                // the stage's h at this warp's last step, for the next warp's first gates
+                sm.hlast[warp][lane] = sv[3];
+                __syncthreads();
             }
         }
         if (TMA) {
@@ -1220,10 +1269,10 @@ cudaError_t launch_pass(const Args &a, const NewtonMaps &m, int k, bool resid, i
                  : launch_one<FORGET, false, false, TMA, VARLEN, MODE>(a, m, k, sms, st);
 }
 
-template <int FORGET, bool SWEEP, bool TMA, bool VARLEN>
-cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
+template <int FORGET, int NS, bool SWEEP, bool TMA, bool VARLEN>
+cudaError_t launch_guess_ns(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
-    auto kern = guess_kernel<FORGET, SWEEP, TMA, VARLEN>;
+    auto kern = guess_kernel<FORGET, NS, SWEEP, TMA, VARLEN>;
     static bool ready = false;
     if (!ready) {
         const cudaError_t e =
@@ -1233,6 +1282,13 @@ cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int k, int sms, cud
     }
     kern<<<min(a.n_tiles, sms), NW * 32, GUESS_SMEM_BYTES, st>>>(a, k, m);
     return cudaGetLastError();
+}
+
+// One guess launch of a single stage (the decoupled guess, or a sweep of S).
+template <int FORGET, bool SWEEP, bool TMA, bool VARLEN>
+cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
+{
+    return launch_guess_ns<FORGET, 1, SWEEP, TMA, VARLEN>(a, m, k, sms, st);
 }
 
 // Launch k of a solve: epoch k + 1; it reads the boundary buffer launch
@@ -1246,13 +1302,25 @@ inline Args launch_args(const Args &base, int k)
     return a;
 }
 
-// The decoupled guess (launch 0) and its refinement sweeps (launches
-// 1 .. sweeps).
+// Guess launches of a solve with `sweeps` refinement sweeps: launch 0 runs
+// the decoupled guess and the first GUESS_STAGES - 1 sweeps tile by tile;
+// any further sweep is a launch of its own (1, 2, ...).
+inline int guess_launches(int sweeps) { return 1 + (sweeps > GUESS_STAGES - 1 ? sweeps - (GUESS_STAGES - 1) : 0); }
+
 template <int FORGET, bool TMA, bool VARLEN>
 cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, int sms, cudaStream_t st)
 {
-    cudaError_t e = launch_guess<FORGET, false, TMA, VARLEN>(launch_args(base, 0), m, 0, sms, st);
-    for (int k = 1; k <= sweeps && e == cudaSuccess; ++k)
+    const int fused = 1 + (sweeps < GUESS_STAGES - 1 ? sweeps : GUESS_STAGES - 1);
+    const Args a0 = launch_args(base, 0);
+    cudaError_t e;
+    switch (fused) {
+    case 1: e = launch_guess_ns<FORGET, 1, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
+    case 2: e = launch_guess_ns<FORGET, 2, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
+    case 3: e = launch_guess_ns<FORGET, 3, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
+    default: e = launch_guess_ns<FORGET, 4, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
+    }
+    const int n = guess_launches(sweeps);
+    for (int k = 1; k < n && e == cudaSuccess; ++k)
         e = launch_guess<FORGET, true, TMA, VARLEN>(launch_args(base, k), m, k, sms, st);
     return e;
 }
@@ -1265,7 +1333,7 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
                          int init, cudaStream_t st)
 {
     if (init == SLSTM_INIT_DECOUPLED) {
-        const cudaError_t e = launch_guess_all<FORGET, TMA, VARLEN>(base, m, base.k0 - 1, sms, st);
+        const cudaError_t e = launch_guess_all<FORGET, TMA, VARLEN>(base, m, base.guess_sweeps, sms, st);
         if (e != cudaSuccess) return e;
     } else if (init == SLSTM_INIT_GIVEN) {
         const long long n = (long long)base.n_tiles * 128;
@@ -1311,8 +1379,8 @@ Layout layout(int B, int T, int d)
         return at;
     };
     l.ctrl = take(sizeof(NewtonCtrl));
-    l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles);
-    l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles);
+    l.flags = take(sizeof(unsigned) * (size_t)l.n_tiles * GUESS_STAGES);
+    l.incw = take(sizeof(unsigned long long) * 4 * 32 * (size_t)l.n_tiles * GUESS_STAGES);
     l.agg = take(sizeof(float) * 20 * 32 * (size_t)l.n_tiles);
     l.bnd0 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
     l.bnd1 = take(sizeof(float) * 4 * 32 * (size_t)l.n_tiles);
@@ -1388,7 +1456,8 @@ cudaError_t prepare(const float *P, const float *R, const float *s0, float *S, c
     a.max_iters = cfg.max_iters;
     a.fixed = cfg.fixed_iters ? 1 : 0;
     a.tol = cfg.tol;
-    a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : (cfg.init == SLSTM_INIT_DECOUPLED ? 1 + cfg.guess_sweeps : 1);
+    a.guess_sweeps = cfg.guess_sweeps;
+    a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : (cfg.init == SLSTM_INIT_DECOUPLED ? guess_launches(cfg.guess_sweeps) : 1);
     a.resid_raw = cfg.residual_mode == SLSTM_RESIDUAL_RAW ? 1 : 0;
     a.guess_tested = (cfg.init == SLSTM_INIT_DECOUPLED && !a.fixed) ? 1 : 0;
     a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(P) & 15) == 0 &&
