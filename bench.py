@@ -468,21 +468,24 @@ def run_gpu(args, w):
     fwd_ms = (ms_gemm + ms_newton) / args.steps
 
     hbm, peak_kind = _peaks()
-    # The Newton solve is one C call: the guess launch (reads P, writes S: 32
-    # algorithmic B/elem), its refinement sweeps (read P and h, write S: 36
-    # B/elem each) and n iterations (read P and the old S, write S: 48 B/elem
-    # each); in tolerance mode the launches after convergence return at once.
-    # Its CUDA-event time over the timed region against those bytes.
+    # The Newton solve is one C call: the guess launch, which runs the decoupled
+    # guess and up to GUESS_FUSED_SWEEPS refinement sweeps tile by tile (reads
+    # P, writes S: 32 algorithmic B/elem), one launch per further sweep (reads
+    # P and h, writes S: 36 B/elem each) and n iterations (read P and the old
+    # S, write S: 48 B/elem each); in tolerance mode the launches after
+    # convergence return at once.  Its CUDA-event time over the timed region
+    # against those bytes.
     n_it = st["iters"]
     sw = args.guess_sweeps
     newton_ms = ms_newton / args.steps
     newton_bytes = elems * solve_bytes_per_elem(n_it, sw)
     achieved = newton_bytes / (newton_ms / 1e3) / 1e9
     traffic = args.traffic_bytes if args.traffic_bytes else newton_traffic_bytes(elems, n_it, sw)
-    roofline = {"kernel": "newton solve (guess_kernel x (1 + sweeps) + newton_iter x iters)", "bound": "hbm",
+    n_launch = guess_launches(sw) + n_it
+    roofline = {"kernel": "newton solve (guess_kernel x guess launches + newton_iter x iters)", "bound": "hbm",
                 "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                 "traffic": traffic, "algorithmic_bytes_per_solve": newton_bytes,
-                "working_launches_per_solve": 1 + sw + n_it, "avg_launch_ms": newton_ms / (1 + sw + n_it),
+                "working_launches_per_solve": n_launch, "avg_launch_ms": newton_ms / n_launch,
                 "solve_ms": newton_ms}
 
     cpu = None
@@ -908,12 +911,21 @@ def newton_sources_sha256() -> str:
     return h.hexdigest()
 
 
+# Refinement sweeps that the guess launch runs itself, tile by tile, after the
+# decoupled guess; each further sweep is a launch of its own.
+GUESS_FUSED_SWEEPS = 3
+
+
+def guess_launches(sweeps: int) -> int:
+    return 1 + max(0, sweeps - GUESS_FUSED_SWEEPS)
+
+
 def solve_bytes_per_elem(iters: int, sweeps: int) -> int:
     """Algorithmic bytes per element of B*T*d_h of one Newton solve: the
-    decoupled guess reads P and writes S (32), a refinement sweep also reads
-    the previous guess's h (36), an iteration reads P and the old S and writes
-    S (48)."""
-    return 32 + 36 * sweeps + 48 * iters
+    guess launch reads P and writes S (32) whatever number of sweeps it fuses,
+    a sweep launch also reads the previous guess's h (36), an iteration reads
+    P and the old S and writes S (48)."""
+    return 32 + 36 * (guess_launches(sweeps) - 1) + 48 * iters
 
 
 def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
@@ -922,7 +934,7 @@ def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
     t = NEWTON_TRAFFIC
     if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
         return None
-    return (t["guess"] + t["sweep"] * sweeps + t["iter"] * iters) * elems
+    return (t["guess"] + t["sweep"] * (guess_launches(sweeps) - 1) + t["iter"] * iters) * elems
 
 
 def main(argv=None):

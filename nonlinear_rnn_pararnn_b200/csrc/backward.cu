@@ -3,11 +3,15 @@
 // packed cell VJP for the gradients of R and W_x).
 //
 // Fused adjoint + VJP kernel, tiles in reverse time order:
-//   lambda_t = e_h dH_t + J_{t+1}^T lambda_{t+1}   (J recomputed from S_t, P_{t+1})
-//   dP_t     = G_t^T lambda_t,  G_t = d s_t / d a_t (recomputed from S_{t-1}, P_t)
+//   lambda_t = e_h dH_t + J_{t+1}^T lambda_{t+1}
+//   dP_t     = G_t^T lambda_t,  G_t = d s_t / d a_t
 //   dR      += dP_t * h_{t-1},  db += dP_t   (per-tile partials, reduced after)
 //   ds0      = J_0^T lambda_0
-// then dx = dP W_x and dW_x = dP^T x.
+// then dx = dP W_x and dW_x = dP^T x.  The scan runs on kappa_{t-1} =
+// J_t^T lambda_t (so lambda_t = kappa_t + e_h dH_t), whose step map needs
+// only the cell of step t itself; each step's cell (J_t and G_t, recomputed
+// from S_{t-1} and P_t) is evaluated once, and the second walk forms G_t^T
+// lambda_t and J_t^T lambda_t from eight of its numbers (CellB).
 #include <cuda_bf16.h>
 #include <string.h>
 
@@ -57,11 +61,11 @@ struct BwdInfo {
     unsigned long long hmask;   // packed sequences: bit r set when step t_lo + r (r <= 32) starts a sequence
 };
 
-// Shared memory of one CTA.  A tile needs S at t_lo-1 .. t_hi, P at
-// t_lo .. t_hi+1 and dH at t_lo .. t_hi (t_hi = t_lo + 31).
+// Shared memory of one CTA.  A tile needs S at t_lo-1 .. t_hi, P and dH at
+// t_lo .. t_hi (t_hi = t_lo + 31).
 struct BwdSmem {
     float S[2][TT + 1][4][32];   // row r <-> t = t_lo - 1 + r
-    float P[2][TT + 1][4][32];   // row r <-> t = t_lo + r
+    float P[2][TT][4][32];       // row r <-> t = t_lo + r
     float dH[2][TT][32];         // row r <-> t = t_lo + r
     float R[2][4][32];           // TMA path: the tile's recurrent weights
     union {
@@ -79,8 +83,8 @@ constexpr size_t BWD_SMEM_BYTES = sizeof(BwdSmem) + 1024;
 constexpr int BWD_TMA_THREAD = (NW - 1) * 32;
 constexpr uint64_t BWD_TMA_WAIT_NS = 1000000000ull;
 
-// Tensor maps: S and P as (d, 4T, B) with boxes of 32 features x 132 (step,
-// slot) rows, dH as (d, T, B) with boxes of 32 x 32.
+// Tensor maps: S and P as (d, 4T, B) with boxes of 32 features x 132 (S) or
+// 128 (P) (step, slot) rows, dH as (d, T, B) with boxes of 32 x 32.
 struct BwdMaps {
     CUtensorMap S, P, H;
 };
@@ -121,7 +125,7 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdI
     const size_t d = (size_t)a.d;
     const size_t row0 = (size_t)ti.b * a.T;
     const int T = a.T;
-    constexpr int RS = (TT + 1) * 4;           // (row, slot) pairs of S and of P
+    constexpr int RS = (TT + 1) * 4;           // (row, slot) pairs of S; P has TT * 4
     if (a.vec16) {
         // thread (q, c) copies 16-byte chunk c of (row, slot) pairs q, q+32, ...
         const int c = threadIdx.x & 7, q = threadIdx.x >> 3;
@@ -134,9 +138,11 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdI
                 const int r = rs >> 2, slot = rs & 3;
                 const int tS = t_lo - 1 + r, tP = t_lo + r;
                 const int bS = (tS >= 0 && tS < T) ? fbytes : 0;
-                const int bP = (tP >= 0 && tP < T) ? fbytes : 0;
                 cp_async16(&sm.S[st][r][slot][4 * c], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
-                cp_async16(&sm.P[st][r][slot][4 * c], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+                if (r < TT) {
+                    const int bP = (tP >= 0 && tP < T) ? fbytes : 0;
+                    cp_async16(&sm.P[st][r][slot][4 * c], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+                }
             }
         }
         const int t = t_lo + q;   // dH row q
@@ -151,9 +157,11 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdI
             const int r = rs >> 2, slot = rs & 3;
             const int tS = t_lo - 1 + r, tP = t_lo + r;
             const int bS = (fj && tS >= 0 && tS < T) ? 4 : 0;
-            const int bP = (fj && tP >= 0 && tP < T) ? 4 : 0;
             cp_async4(&sm.S[st][r][slot][jl], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
-            cp_async4(&sm.P[st][r][slot][jl], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+            if (r < TT) {
+                const int bP = (fj && tP >= 0 && tP < T) ? 4 : 0;
+                cp_async4(&sm.P[st][r][slot][jl], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
+            }
         }
         for (int r = w; r < TT; r += NW) {
             const int t = t_lo + r;
@@ -267,36 +275,52 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
 
-        // ---- walk A: fold lambda -> J_{t+1}^T lambda + e_h dH_t, t descending ----
-        // Rows past T or before 0 are zero-filled: J_T (the step past the
-        // end) is finite and only ever meets the zero carry entering the
-        // sequence's last step; steps before 0 come last in this order and
-        // reach nothing that is stored.
-        Cell Jn[L];   // J_{t+1} of each step
+        // ---- walk A: fold kappa -> J_t^T (kappa + e_h dH_t), t descending ----
+        // Each step's cell is evaluated here, once: J_t for the fold, the
+        // factors of G_t and J_t (CellB) and h_{t-1} for walk B.  A sequence's
+        // first step takes its s0 as the state before it; its J is the true
+        // one (walk B forms ds0 from it), but what leaves it towards the
+        // previous sequence is zero.  Rows before t = 0 (the last chunk only)
+        // are zero-filled and come last in this order: nothing they reach is
+        // stored.
+        CellB cb[L];
+        float hp[L];   // h_{t-1} of each step
         AffP agg;
 #pragma unroll
         for (int i = 0; i < L; ++i) {
             if (i == L / 2 && look) w2 = ld_relaxed_u64(predw);
             const int rl = TT - 1 - (warp * L + i);   // t - t_lo
-            cell_eval<FORGET, true>(sm.S[st][rl + 1][0][lane], sm.S[st][rl + 1][1][lane], sm.S[st][rl + 1][2][lane],
-                                    sm.S[st][rl + 1][3][lane], sm.P[st][rl + 1][0][lane], sm.P[st][rl + 1][1][lane],
-                                    sm.P[st][rl + 1][2][lane], sm.P[st][rl + 1][3][lane], rz, ri, rf, ro, Jn[i]);
-            // step t + 1 starts a sequence: lambda_t does not depend on lambda_{t+1}
-            const bool reset = VARLEN && ((ti.hmask >> (rl + 1)) & 1ull);
-            if (reset) cell_zero_jac(Jn[i]);
-            const float r[4] = {0.f, 0.f, 0.f, sm.dH[st][rl][lane]};
-            if (i == 0 || reset) affp_from_cell<true>(agg, Jn[i], r);
-            else fold_p<true>(agg, Jn[i], r);
+            const int t = t_lo + rl;
+            float prev[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
+            const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
+            if (head) {
+                const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
+            }
+            Cell J;
+            cell_eval<FORGET, true, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
+                                                 sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane],
+                                                 rz, ri, rf, ro, J, nullptr, &cb[i]);
+            hp[i] = prev[3];
+            const bool reset = VARLEN && head;
+            if (reset) cell_zero_jac(J);
+            const float dh = sm.dH[st][rl][lane];
+            const float r[4] = {J.jhc * dh, J.jhn * dh, J.jhm * dh, J.jhh * dh};   // J^T e_h dH_t
+            if (i == 0 || reset) affp_from_cell<true>(agg, J, r);
+            else fold_p<true>(agg, J, r);
         }
         maps_store(sm.u.m, warp, lane, agg);
         if (threadIdx.x == 0) bwd_decode(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
 
-        // warps whose steps contain such a reset (bits rl + 1 of their steps)
+        // warps whose steps contain a sequence start (bits rl of their steps)
         unsigned whead = 0u;
         if (VARLEN) {
 #pragma unroll
             for (int w = 0; w < NW; ++w)
-                whead |= (((ti.hmask >> (TT - L - w * L + 1)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
+                whead |= (((ti.hmask >> (TT - L - w * L)) & ((1ull << L) - 1ull)) != 0ull) ? (1u << w) : 0u;
         }
         if constexpr (MODE == BWD_AGG) {
             if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
@@ -357,64 +381,54 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             }
             __syncthreads();   // the maps are dead from here on; the dP staging takes their place
 
-            // ---- walk B: lambda_t, then dP_t = G_t^T lambda_t ----
-            float lam[4];
+            // ---- walk B: lambda_t = kappa_t + e_h dH_t, dP_t = G_t^T lambda_t,
+            // kappa_{t-1} = J_t^T lambda_t ----
+            float kap[4];
     #pragma unroll
-            for (int e = 0; e < 4; ++e) lam[e] = sm.cin[warp][e][sw(e, lane)];
+            for (int e = 0; e < 4; ++e) kap[e] = sm.cin[warp][e][sw(e, lane)];
             float dr[4] = {0.f, 0.f, 0.f, 0.f}, dbs[4] = {0.f, 0.f, 0.f, 0.f};
             float dv[L][4];   // dP of the thread's steps (gate order z, i, f, o)
     #pragma unroll
             for (int i = 0; i < L; ++i) {
                 const int rl = TT - 1 - (warp * L + i);
                 const int t = t_lo + rl;
-                if (VARLEN && ((ti.hmask >> (rl + 1)) & 1ull)) {
-    #pragma unroll
-                    for (int e = 0; e < 4; ++e) lam[e] = 0.0f;
-                }
-                jacT_mul(Jn[i], lam[0], lam[1], lam[2], lam[3]);
-                lam[3] += sm.dH[st][rl][lane];
-                float prev[4];
-    #pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
-                Cell cc;
-                CellG g;
+                const CellB &q = cb[i];
+                const float lc = kap[0], ln = kap[1], lm = kap[2];
+                const float lh = kap[3] + sm.dH[st][rl][lane];
+                const float muc = fmaf(q.on, lh, lc);
+                const float mun = fmaf(-q.ony, lh, ln);
+                const float X = fmaf(q.gci, muc, q.gni * mun);
+                const bool fb = __float_as_int(q.dlfs) >= 0;
+                const float jtm = fb ? lm - X : -X;
+                const float g[4] = {q.gcz * muc, fb ? X : lm + X, fabsf(q.dlfs) * jtm, q.gho * lh};
+                kap[0] = q.fp * muc;
+                kap[1] = q.fp * mun;
+                kap[2] = jtm;
+                kap[3] = fmaf(rz, g[0], fmaf(ri, g[1], fmaf(rf, g[2], ro * g[3])));
                 const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
                 if (head) {
-                    // the state before the sequence is its s0; ds0 = J^T lambda at its first step
-                    const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
-    #pragma unroll
-                    for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
-                    cell_eval<FORGET, true, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
-                                                  sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
-                                                  ri, rf, ro, cc, &g);
+                    // ds0 = J^T lambda at the sequence's first step; nothing
+                    // enters the step before it (another sequence, or none)
                     if (a.ds0 && jv) {
-                        float v0 = lam[0], v1 = lam[1], v2 = lam[2], v3 = lam[3];
-                        jacT_mul(cc, v0, v1, v2, v3);
-                        float *q = a.ds0 + sq * 4 * d + jj;
-                        q[0] = v0;
-                        q[d] = v1;
-                        q[2 * d] = v2;
-                        q[3 * d] = v3;
+                        const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
+                        float *qd = a.ds0 + sq * 4 * d + jj;
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) qd[e * d] = kap[e];
                     }
-                } else {
-                    cell_eval<FORGET, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
-                                                   sm.P[st][rl][1][lane], sm.P[st][rl][2][lane], sm.P[st][rl][3][lane], rz,
-                                                   ri, rf, ro, cc, &g);
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) kap[e] = 0.0f;
                 }
                 const bool tv = t >= 0;   // steps before 0 (last chunk only) contribute nothing
-                dv[i][0] = tv ? fmaf(g.gcz, lam[0], g.ghz * lam[3]) : 0.f;
-                dv[i][1] = tv ? fmaf(g.gci, lam[0], fmaf(g.gni, lam[1], fmaf(g.gmi, lam[2], g.ghi * lam[3]))) : 0.f;
-                dv[i][2] = tv ? fmaf(g.gcf, lam[0], fmaf(g.gnf, lam[1], fmaf(g.gmf, lam[2], g.ghf * lam[3]))) : 0.f;
-                dv[i][3] = tv ? g.gho * lam[3] : 0.f;
+    #pragma unroll
+                for (int e = 0; e < 4; ++e) dv[i][e] = tv ? g[e] : 0.f;
                 if (!BF16OUT && jv && tv) {
                     float *pd = a.dP + (row0 + t) * 4 * d + jj;
     #pragma unroll
                     for (int e = 0; e < 4; ++e) pd[e * d] = dv[i][e];
                 }
-                const float hp = prev[3];
     #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    dr[e] = fmaf(dv[i][e], hp, dr[e]);
+                    dr[e] = fmaf(dv[i][e], hp[i], dr[e]);
                     dbs[e] += dv[i][e];
                 }
             }
@@ -741,7 +755,7 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     const uint64_t rows = 4 * (uint64_t)T;
     const bool tma = a.vec16 && (reinterpret_cast<uintptr_t>(R) & 15) == 0 && rows < (1ull << 31) &&
                      make_map_f32_3d(&m.S, S, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
-                     make_map_f32_3d(&m.P, P, d_h, rows, B, d_h, rows * d_h, 32, (TT + 1) * 4) &&
+                     make_map_f32_3d(&m.P, P, d_h, rows, B, d_h, rows * d_h, 32, TT * 4) &&
                      make_map_f32_3d(&m.H, dH, d_h, T, B, d_h, (uint64_t)T * d_h, 32, TT);
     // few feature groups and a long time axis: two passes with a scan of the
     // tile aggregates in between instead of waiting for predecessors

@@ -51,6 +51,20 @@ struct CellG {
     float gcz, gci, gcf, gni, gnf, gmi, gmf, ghz, ghi, ghf, gho;
 };
 
+// The factors of G that the adjoint keeps for its second walk.  The gates see
+// h_{t-1} only through the diagonal r (a_t = P_t + r h_{t-1}), so the h
+// column of J is G r, and with
+//   mu_c = lam_c + on lam_h,   mu_n = lam_n - ony lam_h,   X = gci mu_c + gni mu_n
+// both products follow from eight numbers:
+//   G^T lam = (gcz mu_c,  X + (1 - fb) lam_m,  dlf (fb lam_m - X),  gho lam_h)
+//   J^T lam = (fp mu_c,   fp mu_n,             fb lam_m - X,        r . G^T lam)
+// where on = o / n, ony = o c / n^2, dlf = d log f / d a_f, fb = 1 on the forget
+// branch of the stabiliser's max and 0 on the input branch, and
+// dlfs = fb ? dlf : -dlf carries fb in its sign bit.
+struct CellB {
+    float fp, gci, gni, on, ony, gcz, dlfs, gho;
+};
+
 // Transcendentals on the MUFU pipe through CUDA's fast intrinsics (__expf,
 // __logf, __fdividef), combined by the identities
 //   sigmoid(x) = 1 / (1 + e^{-x}),   tanh(x) = 1 - 2 / (1 + e^{2x}).
@@ -60,10 +74,10 @@ SLSTM_DEVINL float tanh_fast(float x) { return 1.0f - __fdividef(2.0f, 1.0f + __
 
 // forget: SLSTM_FORGET_SIGMOID or SLSTM_FORGET_EXP.  WANT_J: fill the
 // Jacobian fields.  WANT_G: fill *g.
-template <int FORGET, bool WANT_J, bool WANT_G = false>
+template <int FORGET, bool WANT_J, bool WANT_G = false, bool WANT_B = false>
 SLSTM_DEVINL void cell_eval(float c0, float n0, float m0, float h0, float pz, float pi, float pf,
                             float po, float rz, float ri, float rf, float ro, Cell &o,
-                            CellG *g = nullptr)
+                            CellG *g = nullptr, CellB *bq = nullptr)
 {
     const float az = fmaf(rz, h0, pz);
     const float ai = fmaf(ri, h0, pi);
@@ -97,9 +111,19 @@ SLSTM_DEVINL void cell_eval(float c0, float n0, float m0, float h0, float pz, fl
     o.n = n;
     o.m = m;
     o.h = og * y;
-    if (WANT_J || WANT_G) {
+    if (WANT_J || WANT_G || WANT_B) {
         const float on = og * inv_n;
         const float dz = 1.0f - z * z;
+        if (WANT_B) {
+            bq->fp = fp;
+            bq->gci = fb ? ip * z : -fp * c0;
+            bq->gni = fb ? ip : -fp * n0;
+            bq->on = on;
+            bq->ony = on * y;
+            bq->gcz = ip * dz;
+            bq->dlfs = fb ? dlf : -dlf;
+            bq->gho = y * og * (1.0f - og);
+        }
         if (WANT_J) {
             // d(log f') / d h0 - d(log i') / d h0 = dlf * rf - ri; only one of
             // the two is nonzero, selected by the branch of the max.

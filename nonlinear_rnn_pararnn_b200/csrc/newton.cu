@@ -648,6 +648,18 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                 }
             }
 
+            // the predecessor's published state of this stage, read now so
+            // that the load's latency hides behind walk A and the scan: lane
+            // 15 of each half-warp, for the feature it carries below
+            const int fc = 2 * warp + (lane >> 4);
+            const bool carry_lane = (lane & 15) == 15;
+            unsigned long long pw[4] = {0ull, 0ull, 0ull, 0ull};
+            if (carry_lane && chunk > 0) {
+                const unsigned long long *src = gc.incw + (size_t)(ticket - G) * 4 * 32 + fc;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pw[e] = ld_relaxed_u64(src + e * 32);
+            }
+
             // ---- walk A: this warp's run, lane = feature ----
             float gz[L], glf[L], go[L], gi[L];
             {
@@ -699,8 +711,10 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
 
             // ---- scan of the warp runs: lane (feature 2 warp + lane / 16, run lane % 16) ----
             const unsigned whead = sm.whead;
+            bool ok = true;   // this lane's carry found the predecessor's state
+            float vo[4];      // carry lanes: the state after the tile
             {
-                const int f = 2 * warp + (lane >> 4), w = lane & 15;
+                const int f = fc, w = lane & 15;
                 Seg x;
                 seg_load(sm, w, f, x, ((whead >> w) & 1u) != 0u);
 #pragma unroll
@@ -715,34 +729,63 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                     if (w >= off) seg_compose(x, y, x);
                 }
                 seg_store(sm, w, f, x);
-            }
-            __syncthreads();
-
-            // ---- carry: warp 0, lane = feature ----
-            if (warp == 0) {
-                float v[4] = {0.f, 0.f, 0.f, 0.f};
-                Seg tile;
-                seg_load(sm, NW - 1, lane, tile, whead != 0u);
-                if (chunk == 0) {
-                    if (!VARLEN && a.s0 && jv) {
+                // ---- carry (fast path): the last run lane holds the tile's
+                // run; entered from the predecessor's state read above ----
+                if (carry_lane) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    if (chunk == 0) {
+                        if (!VARLEN && a.s0 && ti.j0 + f < a.d) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
+                            for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + ti.j0 + f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            ok = ok && ((unsigned)(pw[e] >> 32) == a.epoch);
+                            v[e] = __uint_as_float((unsigned)pw[e]);
+                        }
                     }
-                } else {
-                    const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
-                    const bool ok = read_inc_words(ca, ticket - G, lane, v);
-                    if (!__all_sync(0xffffffffu, ok))
-                        guess_lookback(a, gc, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sm.cin[e][f] = v[e];
+                    seg_enter(x, v, vo);
                 }
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sm.cin[e][lane] = v[e];
-                float vo[4];
-                seg_enter(tile, v, vo);
-                unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + lane;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
             }
-            __syncthreads();
+            static_assert(NW == 16, "the carry lanes are the last of 16 run lanes");
+            if (__syncthreads_and(ok)) {
+                // every feature found its predecessor's state: publish
+                if (carry_lane) {
+                    unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + fc;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
+                }
+            } else {
+                // ---- carry (look-back): warp 0, lane = feature; nothing was
+                // published above, and cin is written again for every feature ----
+                if (warp == 0) {
+                    float v[4] = {0.f, 0.f, 0.f, 0.f};
+                    Seg tile;
+                    seg_load(sm, NW - 1, lane, tile, whead != 0u);
+                    if (chunk == 0) {
+                        if (!VARLEN && a.s0 && jv) {
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
+                        }
+                    } else {
+                        const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                        const bool got = read_inc_words(ca, ticket - G, lane, v);
+                        if (!__all_sync(0xffffffffu, got))
+                            guess_lookback(a, gc, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) sm.cin[e][lane] = v[e];
+                    float vt[4];
+                    seg_enter(tile, v, vt);
+                    unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + lane;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vt[e]));
+                }
+                __syncthreads();
+            }
 
             // ---- walk B: enter this warp's steps through the prefix before it ----
             {
