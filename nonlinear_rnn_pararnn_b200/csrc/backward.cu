@@ -80,7 +80,12 @@ struct BwdSmem {
     uint64_t bar[2];
 };
 constexpr size_t BWD_SMEM_BYTES = sizeof(BwdSmem) + 1024;
-constexpr int BWD_TMA_THREAD = (NW - 1) * 32;
+// Warps CHAIN0 .. NW-1 walk the carry through the warp maps (chain lanes);
+// warp w < CHAIN0 starts walk B as soon as the carry entering it is stored
+// (named barrier 1 + w), the chain warps themselves after CHAIN_BAR.
+constexpr int CHAIN0 = NW - 4;
+constexpr int CHAIN_BAR = CHAIN0 + 1;
+constexpr int BWD_TMA_THREAD = (CHAIN0 - 1) * 32;   // a warp with no chain lane
 constexpr uint64_t BWD_TMA_WAIT_NS = 1000000000ull;
 
 // Tensor maps: S and P as (d, 4T, B) with boxes of 32 features x 132 (S) or
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
     const unsigned G = (unsigned)a.ca.n_groups;
     const int T = a.T;
     const size_t d = (size_t)a.d;
-    const bool chain_warp = warp < 4;
+    const bool chain_warp = warp >= CHAIN0;
 
     if (threadIdx.x == 0) {
         // BWD_AGG tiles are independent: a static order needs no counter
@@ -370,16 +375,22 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             }
             const bool fast = __syncthreads_and(ok);
             if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
-            if (fast) {
-                if (chain_warp) {
-                    c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead);
+            if (chain_warp) {
+                if (fast) {
+                    c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead, CHAIN0);
                     if (MODE == BWD_FUSED) st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+                    named_bar_sync(CHAIN_BAR, 4 * 32);
+                } else {
+                    if (warp == CHAIN0)
+                        tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G),
+                                                false, whead);
+                    named_bar_sync(CHAIN_BAR, 4 * 32);
+    #pragma unroll 1
+                    for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
                 }
-            } else if (warp == 0) {
-                tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false,
-                                        whead);
+            } else {
+                named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
             }
-            __syncthreads();   // the maps are dead from here on; the dP staging takes their place
 
             // ---- walk B: lambda_t = kappa_t + e_h dH_t, dP_t = G_t^T lambda_t,
             // kappa_{t-1} = J_t^T lambda_t ----
@@ -432,6 +443,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                     dbs[e] += dv[i][e];
                 }
             }
+            __syncthreads();   // the maps are dead from here on; the dP staging takes their place
     #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 sm.u.o.part[warp][e][lane] = jv ? dr[e] : 0.f;

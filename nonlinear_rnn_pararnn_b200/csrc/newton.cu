@@ -710,7 +710,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
             __syncthreads();
 
             // ---- scan of the warp runs: lane (feature 2 warp + lane / 16, run lane % 16) ----
-            const unsigned whead = sm.whead;
+            const unsigned whead = VARLEN ? sm.whead : 0u;   // dense sequences: no run holds a start
             bool ok = true;   // this lane's carry found the predecessor's state
             float vo[4];      // carry lanes: the state after the tile
             {
