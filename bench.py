@@ -15,10 +15,16 @@ rank runs its own replica of the workload (independent batches, no data-path
 collective): `value` is the sum over ranks of elements divided by the slowest
 rank's device time.
 
+`roofline` is for the step's dominant kernel, newton_iter (the Newton
+iteration: 48 algorithmic bytes per element per launch), over the average
+duration of its working launches, taken from CUDA events that the library
+records on its stream around each of its launches inside the timed steps; the
+guess launch and the whole solve are reported beside it.
+
 With no flags the line also carries, measured in the same run on rank 0: the
 long-sequence workload's forward (B=4, T=65536, d=2048: input projection and
-the converged Newton solve, and the fixed K=4 solve) with the Newton solve's
-HBM roofline fraction, and the scan_block4 sweep at B=4, d=2048 over
+the converged Newton solve, and the fixed K=4 solve) with newton_iter's HBM
+roofline fraction, and the scan_block4 sweep at B=4, d=2048 over
 T = 4096, 16384, 65536.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
@@ -39,7 +45,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from nonlinear_rnn_pararnn_b200.workloads import ORDER, WORKLOADS, as_f64, make_inputs, scaled  # noqa: E402
+from nonlinear_rnn_pararnn_b200.workloads import (ORDER, WORKLOADS, as_f64, make_head_R, make_inputs,  # noqa: E402
+                                                   scaled)
 
 METRIC = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd+bwd)"
 METRIC_FWD = "sLSTM Newton solve elems/s (B*T*d_h/s, fwd)"
@@ -342,7 +349,9 @@ def run_gpu(args, w):
 
     dev_main = {"x": x, "Wx": Wx, "R": R, "bias": bias, "s0": s0, "dH": dH}
 
-    def step(ev=None, dv=None, gr=None):
+    n_launch = guess_launches(args.guess_sweeps) + K   # launches of work of one Newton call
+
+    def step(ev=None, dv=None, gr=None, lev=None):
         dv = dev_main if dv is None else dv
         gr = grads if gr is None else gr
         if ev is not None:
@@ -351,7 +360,7 @@ def run_gpu(args, w):
         if ev is not None:
             ev[1].record()
         api.newton_forward(P, dv["R"], dv["s0"], forget=w.forget, max_iters=K, fixed=not tol_mode, tol=w.tol, S=S,
-                           stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps)
+                           stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps, events=lev)
         if ev is not None:
             ev[2].record()
         if not forward_only:
@@ -368,13 +377,20 @@ def run_gpu(args, w):
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # the library records these around each of its Newton launches (guess,
+    # then one per iteration) inside the timed steps
+    levs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_launch + 1)] for _ in range(args.steps)]
+    for lv in levs:
+        for e in lv:
+            e.record()
+    torch.cuda.synchronize()
     sampler = ClockSampler(dev.index)
     time.sleep(0.25)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record()
     for s_ in range(args.steps):
-        step(evs[s_])
+        step(evs[s_], lev=levs[s_])
     end.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -479,14 +495,35 @@ def run_gpu(args, w):
     sw = args.guess_sweeps
     newton_ms = ms_newton / args.steps
     newton_bytes = elems * solve_bytes_per_elem(n_it, sw)
-    achieved = newton_bytes / (newton_ms / 1e3) / 1e9
-    traffic = args.traffic_bytes if args.traffic_bytes else newton_traffic_bytes(elems, n_it, sw)
-    n_launch = guess_launches(sw) + n_it
-    roofline = {"kernel": "newton solve (guess_kernel x guess launches + newton_iter x iters)", "bound": "hbm",
-                "achieved": achieved, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic, "algorithmic_bytes_per_solve": newton_bytes,
-                "working_launches_per_solve": n_launch, "avg_launch_ms": newton_ms / n_launch,
-                "solve_ms": newton_ms}
+    solve_gbs = newton_bytes / (newton_ms / 1e3) / 1e9
+    # Per launch, from the library's events: the guess launch(es), then the
+    # iterations that did work (the later launches of a converged call return
+    # at once and are listed apart).
+    g = guess_launches(sw)
+    per_it = [float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs])) for i in range(n_it)]
+    guess_ms = [lv[0].elapsed_time(lv[g]) for lv in levs]
+    idle_ms = [lv[g + n_it].elapsed_time(lv[n_launch]) for lv in levs]
+    per_it = max_over_ranks(per_it, device=dev) if per_it else []
+    it_ms = float(np.mean(per_it)) if per_it else 0.0
+    guess_ms, idle_ms = max_over_ranks([float(np.mean(guess_ms)), float(np.mean(idle_ms))], device=dev)
+    # the dominant kernel of the step (largest share of the ncu launch list):
+    # newton_iter, 48 algorithmic bytes per element per launch
+    achieved = 48.0 * elems / (it_ms / 1e3) / 1e9 if it_ms > 0 else 0.0
+    traffic = args.traffic_bytes if args.traffic_bytes else newton_iter_traffic_bytes(elems)
+    guess_bytes = 32.0 * elems
+    roofline = {"kernel": "newton_iter", "bound": "hbm", "achieved": achieved, "peak": hbm, "peak_kind": peak_kind,
+                "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
+                "algorithmic_bytes_per_launch": 48 * elems, "avg_launch_ms": it_ms,
+                "launches_per_step": n_it, "launch_ms": per_it,
+                "timing": "CUDA events the library records on its stream around each launch, over the timed steps",
+                "guess_kernel": {"launches_per_step": g, "ms": guess_ms, "algorithmic_bytes": guess_bytes,
+                                 "achieved": guess_bytes / (guess_ms / 1e3) / 1e9,
+                                 "frac": guess_bytes / (guess_ms / 1e3) / 1e9 / hbm,
+                                 "stages_per_tile": 1 + min(sw, GUESS_FUSED_SWEEPS),
+                                 "note": "one scan per stage over each tile; issue-bound"},
+                "converged_launches": {"per_step": n_launch - g - n_it, "ms": idle_ms},
+                "solve": {"ms": newton_ms, "algorithmic_bytes": newton_bytes, "achieved": solve_gbs,
+                          "frac": solve_gbs / hbm}}
 
     cpu = None
     if pool is not None:
@@ -514,7 +551,8 @@ def run_gpu(args, w):
     # launches (in tolerance mode those after convergence exit at once),
     # backward: adjoint 1 + dR/db reduction 1 + 2 GEMMs (+ the split-K sum of
     # the tensor-core path)
-    launches_per_step = 1 + 1 + args.guess_sweeps + K + (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0))
+    launches_per_step = (1 + guess_launches(args.guess_sweeps) + K +
+                         (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0)))
     line = {
         "metric": METRIC_FWD if forward_only else METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup,
@@ -597,21 +635,23 @@ def long_forward(args, dev, hbm, peak_kind):
     stats = api.new_stats(dev)
     ws_n = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
     out = {"workload": w.name, "B": w.B, "T": w.T, "d_h": w.d_h, "forget": w.forget, "tol": w.tol}
+    g = guess_launches(args.guess_sweeps)
     for mode, K in (("tol", w.max_iters), ("fixed", (w.fixed_iters or (4,))[0])):
-        def step(ev):
+        def step(ev, lev=None):
             ev[0].record()
             api.preact_gemm(x, Wx, bias, P=P)
             ev[1].record()
             api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, fixed=(mode == "fixed"), tol=w.tol, S=S,
-                               stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps)
+                               stats=stats, ws=ws_n, guess_sweeps=args.guess_sweeps, events=lev)
             ev[2].record()
         n = 5
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.warmup + n)]
+        levs = [[torch.cuda.Event(enable_timing=True) for _ in range(g + K + 1)] for _ in range(n)]
         for i in range(args.warmup):
             step(evs[i])
         torch.cuda.synchronize()
         for i in range(n):
-            step(evs[args.warmup + i])
+            step(evs[args.warmup + i], levs[i])
         torch.cuda.synchronize()
         timed = evs[args.warmup:]
         gemm_ms = sum(e[0].elapsed_time(e[1]) for e in timed) / n
@@ -620,16 +660,20 @@ def long_forward(args, dev, hbm, peak_kind):
         it = st["iters"]
         nbytes = w.elems * solve_bytes_per_elem(it, args.guess_sweeps)
         gbs = nbytes / (newton_ms / 1e3) / 1e9
+        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs for i in range(it)]))
+        guess_ms = float(np.mean([lv[0].elapsed_time(lv[g]) for lv in levs]))
+        it_gbs = 48.0 * w.elems / (it_ms / 1e3) / 1e9
         out[mode] = {"newton_mode": mode, "max_iters": K, "iters": it, "guess_sweeps": args.guess_sweeps,
                      "converged": st["converged"],
                      "error": st["error"], "max_scaled_F": st["max_scaled_F"],
                      "S_finite": bool(torch.isfinite(S).all().item()),
                      "fwd_elems_per_s": w.elems / ((gemm_ms + newton_ms) / 1e3), "ms_preact_gemm": gemm_ms,
                      "ms_newton": newton_ms, "steps": n,
-                     "roofline": {"kernel": "newton solve (guess_kernel x (1 + sweeps) + newton_iter x iters)",
-                                  "bound": "hbm",
-                                  "achieved": gbs, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                                  "frac": gbs / hbm, "algorithmic_bytes_per_solve": nbytes}}
+                     "roofline": {"kernel": "newton_iter", "bound": "hbm", "achieved": it_gbs, "peak": hbm,
+                                  "peak_kind": peak_kind, "unit": "GB/s", "frac": it_gbs / hbm,
+                                  "avg_launch_ms": it_ms, "algorithmic_bytes_per_launch": 48 * w.elems,
+                                  "guess_kernel_ms": guess_ms,
+                                  "solve": {"achieved": gbs, "frac": gbs / hbm, "algorithmic_bytes": nbytes}}}
     del x, Wx, R, bias, s0, P, S, ws_n
     torch.cuda.empty_cache()
     return out
@@ -722,11 +766,92 @@ def run_varlen(args, w):
                        "d_in": w.d_in, "d_h": w.d_h, "x_dtype": w.dtype, "forget": w.forget, "newton_max_iters": K,
                        "newton_mode": args.newton_mode, "guess_sweeps": args.guess_sweeps,
                        "l2": "inputs larger than L2"},
-            "roofline": {"kernel": "newton solve, packed (guess_kernel x (1 + sweeps) + newton_iter x iters)",
+            "roofline": {"kernel": "newton solve, packed (guess_kernel x guess launches + newton_iter x iters)",
                          "bound": "hbm",
                          "achieved": gbs, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm,
                          "traffic": None, "solve_ms": newton_ms},
             "newton_stats": {"iters": st["iters"], "converged": st["converged"], "error": st["error"]}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_head(args, w):
+    """Head mixing: the workload with block-diagonal R of d_head x d_head blocks (--head-dim, R
+    drawn U(-r, r) / sqrt(d_head)) in place of the diagonal R.  A step is the input-projection GEMM,
+    the head-mixing Newton solve from the decoupled guess (to the workload's tolerance, or K fixed)
+    and its backward.  The head solve applies its linear solve step by step (one warp per batch row
+    and head walks the sequence), so it is bound by that walk's latency, not by HBM; the roofline
+    object still states the solve's algorithmic bytes against the copy bandwidth."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+    _, rank, _ = _dist()
+    dev = torch.device("cuda", 0)
+    tol_mode = args.newton_mode == "tol"
+    K = w.max_iters if tol_mode else args.newton_iters
+    dh = args.head_dim
+    inp = make_inputs(w)
+    x, Wx, bias = inp["x"].to(dev), inp["Wx"].to(dev), inp["bias"].to(dev)
+    Rh = make_head_R(w, dh).to(dev)
+    s0, dH = inp["s0"].to(dev), inp["dH"].to(dev)
+    P = torch.empty(w.B, w.T, 4, w.d_h, device=dev)
+    S = torch.empty_like(P)
+    stats = api.new_stats(dev)
+    ws_f = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
+    ws_b = api.workspace(_lib.SLSTM_OP_NEWTON_BACKWARD_HEAD, w.B, w.T, w.d_in, w.d_h, dev)
+    grads = {"dx": torch.empty(w.B, w.T, w.d_in, device=dev), "dWx": torch.empty(4 * w.d_h, w.d_in, device=dev),
+             "dR_head": torch.empty_like(Rh), "db": torch.empty(4, w.d_h, device=dev),
+             "ds0": torch.empty(w.B, 4, w.d_h, device=dev)}
+
+    def step(ev=None):
+        api.preact_gemm(x, Wx, bias, P=P)
+        if ev is not None:
+            ev[0].record()
+        api.newton_forward_head(P, Rh, s0, forget=w.forget, max_iters=K, fixed=not tol_mode, tol=w.tol, S=S,
+                                stats=stats, ws=ws_f)
+        if ev is not None:
+            ev[1].record()
+        api.newton_backward_head(x, Wx, P, Rh, s0, S, dH, forget=w.forget, out=grads, ws=ws_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    e0.record()
+    for i in range(args.steps):
+        step(evs[i])
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    newton_ms = sum(a.elapsed_time(b) for a, b in evs) / args.steps
+    hbm, peak_kind = _peaks()
+    st = api.read_stats(stats)
+    elems = w.B * w.T * w.d_h
+    # the guess (reads P, writes S: 32 B/elem) and each iteration (reads P and
+    # the old S, writes S: 48 B/elem)
+    nbytes = elems * (32 + 48 * st["iters"])
+    gbs = nbytes / (newton_ms / 1e3) / 1e9
+    line = {"metric": METRIC + ", head mixing", "value": elems / (ms / 1e3), "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "operand_dtype": f"{w.dtype} x/W_x, fp32 state", "data": "synthetic",
+            "config": {"workload": f"{w.name}_head{dh}", "B": w.B, "T": w.T, "d_in": w.d_in, "d_h": w.d_h,
+                       "d_head": dh, "n_heads": w.d_h // dh, "x_dtype": w.dtype, "forget": w.forget,
+                       "R_head": f"U(-{w.r_scale}, {w.r_scale}) / sqrt({dh}), seed {w.seed + 1}",
+                       "newton_mode": args.newton_mode, "newton_max_iters": K, "newton_init": "decoupled",
+                       "l2": "inputs larger than L2"},
+            "breakdown_ms_per_step": {"preact_gemm_and_newton_forward": newton_ms, "backward": ms - newton_ms},
+            "roofline": {"kernel": "head newton solve (guess_kernel + head_newton_kernel x iters)", "bound": "latency",
+                         "achieved": gbs, "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": None, "solve_ms": newton_ms,
+                         "note": "one warp per (batch row, head) walks the sequence: bound by the walk's latency"},
+            "newton_stats": {"iters": st["iters"], "converged": st["converged"], "diverged": st["diverged"],
+                             "error": st["error"], "max_scaled_F": st["max_scaled_F"],
+                             "S_finite": bool(torch.isfinite(S).all().item())},
+            "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -937,6 +1062,15 @@ def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
     return (t["guess"] + t["sweep"] * (guess_launches(sweeps) - 1) + t["iter"] * iters) * elems
 
 
+def newton_iter_traffic_bytes(elems: int):
+    """Measured DRAM bytes of one newton_iter launch, or None when the
+    counters are not for this build."""
+    t = NEWTON_TRAFFIC
+    if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
+        return None
+    return t["iter"] * elems
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -954,11 +1088,14 @@ def main(argv=None):
     ap.add_argument("--cpu-lanes", type=int, default=16)
     ap.add_argument("--ref-lanes", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="train", choices=["train", "forward", "scan", "varlen", "decode", "block"],
+    ap.add_argument("--mode", default="train",
+                    choices=["train", "forward", "scan", "varlen", "decode", "block", "head"],
                     help="train: GEMM + Newton + backward (default); forward: GEMM + Newton; "
                          "scan: scan_block4 alone over T in --scan-T at B=4, d=2048; "
                          "varlen: the workload repacked into ragged sequences (cu_seqlens); "
-                         "decode: T = 1 steps under a CUDA graph; block: the trunk layer's forward")
+                         "decode: T = 1 steps under a CUDA graph; block: the trunk layer's forward; "
+                         "head: head mixing (block-diagonal R, --head-dim) forward + backward")
+    ap.add_argument("--head-dim", type=int, default=32, help="d_head of --mode head (1 .. 32, dividing d_h)")
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
@@ -986,6 +1123,8 @@ def main(argv=None):
         return run_decode(args, w)
     if args.mode == "block":
         return run_block(args, w)
+    if args.mode == "head":
+        return run_head(args, w)
     return run_gpu(args, w)
 
 

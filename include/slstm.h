@@ -133,10 +133,12 @@ typedef enum {
  *               SLSTM_INIT_DECOUPLED (0): the trajectory of the cell with
  *               its gates blind to h_{t-1} (R taken as 0: z, o, log i, log f
  *               from P alone, c, n, m recurring exactly), computed by an
- *               associative scan in one launch that reads P and writes S,
- *               then refined by guess_sweeps fixed-point sweeps (each a
- *               launch of the same scan whose gates see R h_{t-1} of the
- *               previous guess; it reads P and h, writes S).  From this
+ *               associative scan that reads P and writes S, then refined
+ *               by guess_sweeps fixed-point sweeps (the same scan with the
+ *               gates seeing R h_{t-1} of the previous guess).  The guess
+ *               and its first three sweeps run tile by tile in one launch
+ *               (P read once, S written once); each further sweep is a
+ *               launch of its own that reads P and h and writes S.  From this
  *               guess the solve converges in a few iterations on long
  *               sequences where the zero guess overflows.  In tolerance mode
  *               the first iteration records the guess's residual
@@ -150,12 +152,38 @@ typedef enum {
  *   residual_mode  the stopping test: SLSTM_RESIDUAL_SCALED (0),
  *               max |F| / (1 + |s|) <= tol; SLSTM_RESIDUAL_RAW, max|F| <= tol
  *               (the pages' own norm).  Both maxima are recorded either way.
+ *   history     what an iteration records of its residual (tolerance mode):
+ *               SLSTM_HISTORY_BOUND (0): once any part of the new iterate
+ *               fails the test the solve goes on whatever the rest is, so the
+ *               rest of that iteration only checks that its states are
+ *               finite; the recorded maxima of such an iteration are then
+ *               lower bounds of its residual (still above tol).  The
+ *               iteration that stops the solve, the last allowed one and
+ *               every fixed-K run record exact maxima, and the decisions
+ *               (converged, diverged, non-finite) are those of the exact
+ *               residual;  SLSTM_HISTORY_EXACT: every iteration evaluates and
+ *               records its whole residual.  (Packed sequences and rows that
+ *               are not 16-byte aligned always take the exact history.)
+ *   n_events, events  optional per-launch timing (0 / NULL: none): events
+ *               holds n_events CUDA events (cudaEvent_t handles, created by
+ *               the caller); events[i] is recorded on the stream just before
+ *               the call's i-th launch of work and events[n] just after its
+ *               last, for the indices below n_events.  The launches in order:
+ *               the guess launches (one with up to three sweeps, plus one per
+ *               further sweep; none for SLSTM_INIT_ZERO, a small copy kernel
+ *               for SLSTM_INIT_GIVEN), then one per iteration up to max_iters
+ *               (with the two-pass carry an iteration's three kernels count as
+ *               one); launches after the stop return at once but are still
+ *               bracketed.  Timing only: results do not depend on them.
+ *               slstm_newton_forward and slstm_newton_forward_varlen only.
  */
 typedef enum { SLSTM_CARRY_AUTO = 0, SLSTM_CARRY_FUSED = 1, SLSTM_CARRY_TWO_PASS = 2 } slstm_carry_mode;
 
 typedef enum { SLSTM_INIT_DECOUPLED = 0, SLSTM_INIT_ZERO = 1, SLSTM_INIT_GIVEN = 2 } slstm_init;
 
 typedef enum { SLSTM_RESIDUAL_SCALED = 0, SLSTM_RESIDUAL_RAW = 1 } slstm_residual_mode;
+
+typedef enum { SLSTM_HISTORY_BOUND = 0, SLSTM_HISTORY_EXACT = 1 } slstm_history;
 
 typedef struct {
     int max_iters;
@@ -168,6 +196,9 @@ typedef struct {
     int init;
     int residual_mode;
     int guess_sweeps;
+    int history;
+    int n_events;
+    void *const *events;
 } slstm_newton_config;
 
 /*
@@ -507,9 +538,10 @@ int slstm_block_forward(const float *x, const float *norm1_w, const void *Wx, co
  * rounding of z1, z2 and the SwiGLU product is piecewise constant): the
  * recomputed z1 and z2 are the forward's bf16 values, every gradient is
  * formed in fp32.  The cell's part is slstm_newton_backward's (dH = dL/du,
- * zero initial state, its tensor-core GEMMs); the SwiGLU and norm gradients
- * use CUDA-core fp32 GEMMs.  Sizes as slstm_block_forward and B * T <=
- * 8 388 480 (65535 row tiles of 128 for those GEMMs); workspace:
+ * zero initial state, its tensor-core GEMMs); the FFN gradient GEMMs run on
+ * the tensor cores with the fp32 upstream gradients as bf16 hi + lo pairs.
+ * Sizes as slstm_block_forward and B * T <= 16 776 960 (65535 chunks of 256
+ * rows for the norm weights' column sums); workspace:
  * slstm_block_backward_workspace_size(B, T, d_model, d_ff) bytes, 256-byte
  * aligned.  Returns SLSTM_ERR_INVALID_ARG before touching the GPU for bad
  * sizes, forget mode, eps, alignment or workspace.

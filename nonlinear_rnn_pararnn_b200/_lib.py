@@ -41,6 +41,8 @@ SLSTM_INIT_ZERO = 1
 SLSTM_INIT_GIVEN = 2
 SLSTM_RESIDUAL_SCALED = 0
 SLSTM_RESIDUAL_RAW = 1
+SLSTM_HISTORY_BOUND = 0
+SLSTM_HISTORY_EXACT = 1
 SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -48,7 +50,8 @@ class NewtonConfig(ctypes.Structure):
     _fields_ = [("max_iters", ctypes.c_int), ("fixed_iters", ctypes.c_int), ("tol", ctypes.c_float),
                 ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int),
                 ("carry_mode", ctypes.c_int), ("init", ctypes.c_int), ("residual_mode", ctypes.c_int),
-                ("guess_sweeps", ctypes.c_int)]
+                ("guess_sweeps", ctypes.c_int), ("history", ctypes.c_int), ("n_events", ctypes.c_int),
+                ("events", ctypes.c_void_p)]
 
 
 STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY + 2 * 4

@@ -80,14 +80,30 @@ DEFAULT_GUESS_SWEEPS = 2
 
 def newton_config(max_iters: int, fixed: bool, tol: float, forget, debug_fault: int = 0, wait_limit_us: int = 0,
                   carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                  guess_sweeps: int = DEFAULT_GUESS_SWEEPS) -> NewtonConfig:
+                  guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False) -> NewtonConfig:
     """The C ABI's slstm_newton_config.  init: "decoupled" (default; with
     guess_sweeps refinement sweeps), "zero" or "given" (S holds the guess on
-    entry); residual_mode: "scaled" or "raw"."""
-    return NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
-                        int(wait_limit_us), int(carry_mode), _INIT[init] if isinstance(init, str) else int(init),
-                        _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode),
-                        int(guess_sweeps))
+    entry); residual_mode: "scaled" or "raw"; events: optional list of
+    torch.cuda.Event (timing enabled) recorded before each launch of work and
+    after the last (see slstm.h); exact_history: every iteration records its
+    exact residual (else an iteration that fails the test may record a lower
+    bound)."""
+    cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
+                       int(wait_limit_us), int(carry_mode), _INIT[init] if isinstance(init, str) else int(init),
+                       _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode),
+                       int(guess_sweeps), _lib.SLSTM_HISTORY_EXACT if exact_history else _lib.SLSTM_HISTORY_BOUND,
+                       0, None)
+    if events:
+        handles = []
+        for ev in events:
+            if ev.cuda_event == 0:
+                ev.record()   # torch creates the CUDA event on its first record
+            handles.append(ev.cuda_event)
+        arr = (ctypes.c_void_p * len(handles))(*handles)
+        cfg.n_events = len(handles)
+        cfg.events = ctypes.cast(arr, ctypes.c_void_p)
+        cfg._keep = arr   # the array lives as long as the config
+    return cfg
 
 
 def new_stats(device=None) -> torch.Tensor:
@@ -113,9 +129,11 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
                    max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
                    stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
                    wait_limit_us: int = 0, carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS):
+                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False):
     """Newton solve; returns (S, stats) with stats a device record (see read_stats).
-    With init="given", S must be passed and holds the initial guess."""
+    With init="given", S must be passed and holds the initial guess.  events:
+    optional torch.cuda.Event list bracketing the launches; exact_history:
+    see newton_config."""
     B, T, four, d_h = P.shape
     _need(P, "P", (B, T, 4, d_h))
     _need(R, "R", (4, d_h))
@@ -131,7 +149,7 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
     cfg = newton_config(max_iters, fixed, tol, forget, debug_fault, wait_limit_us, carry_mode, init, residual_mode,
-                        guess_sweeps)
+                        guess_sweeps, events, exact_history)
     check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
                                                               ctypes.byref(cfg), _ptr(stats), B, T, d_h,
                                                               _ptr(ws), ws.numel(), _stream()))
@@ -250,9 +268,10 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
                           forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
                           S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None,
                           carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                          guess_sweeps: int = DEFAULT_GUESS_SWEEPS):
+                          guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False):
     """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
-    cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats)."""
+    cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats).
+    events, exact_history: as newton_forward."""
     total_T, four, d_h = P.shape
     n_seq = cu_seqlens.numel() - 1
     _need(P, "P", (total_T, 4, d_h))
@@ -267,7 +286,8 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
         stats = new_stats(P.device)
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
-    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode, guess_sweeps)
+    cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode, guess_sweeps, events,
+                        exact_history)
     check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
         _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
         _ptr(ws), ws.numel(), _stream()))

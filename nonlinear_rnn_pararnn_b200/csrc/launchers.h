@@ -16,6 +16,7 @@ struct NewtonSlot {
     unsigned finished;
     unsigned maxF_raw;     // float bits of a non-negative max
     unsigned maxF_scaled;
+    unsigned failed;       // nonzero once a residual of this iteration failed the stopping test
 };
 
 // Device-side control block of one slstm_newton_forward call.

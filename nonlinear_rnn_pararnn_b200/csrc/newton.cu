@@ -30,6 +30,8 @@
 #include <float.h>
 #include <string.h>
 
+#include <type_traits>
+
 #include "launchers.h"
 #include "lookback.cuh"
 #include "stop_rule.cuh"
@@ -82,6 +84,7 @@ struct Args {
     int k0;             // launches before the first Newton iteration (the guess and its sweeps)
     int guess_sweeps;   // refinement sweeps of the decoupled guess
     int resid_raw;      // stopping test on max|F| (else on the scaled residual)
+    int exact_hist;     // every iteration evaluates its whole residual (else a failed test ends that work)
     int guess_tested;   // the first iteration records the residual of the guess
     float tol;
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
@@ -108,6 +111,7 @@ struct Smem {
     uint64_t bar[2];    // TMA completion, one per stage
     float red[2][NW];
     int exit_flag;
+    int resid_skip;     // this tile: the iteration's test has already failed elsewhere
 };
 constexpr size_t SMEM_BYTES = sizeof(Smem) + 1024;   // + room to align the stages to 1 KB
 // Warps CHAIN0 .. NW-1 walk the carry through the warp maps (chain lanes);
@@ -870,6 +874,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
             nx.finished = 0u;
             nx.maxF_raw = 0u;
             nx.maxF_scaled = 0u;
+            nx.failed = 0u;
             if (k == 0 && a.stats) {
                 a.stats->init_max_abs_F = -1.0f;
                 a.stats->init_max_scaled_F = -1.0f;
@@ -940,6 +945,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     // residual, which walk A forms anyway (r = f - S_old = -F)
     constexpr bool grs = GRS && MODE != MODE_AGG && !FIRST;
     float g_raw = 0.f, g_sc = 0.f;
+    // Once a residual of this iteration fails the stopping test the solve
+    // goes on whatever the others are: later tiles then only check that their
+    // new states are finite (so that a non-finite iterate still stops the
+    // solve at once).  The last allowed iteration, and every one with the
+    // exact history, evaluates its whole residual; so do the cp.async path
+    // (rows that are not 16-byte aligned) and packed sequences, whose
+    // registers have no room for the second copy of walk B.
+    const bool may_skip = TMA && !VARLEN && RESID && !a.exact_hist && (k + 1 - a.k0 < a.max_iters);
 
     int ring = 0, st = 0;
     unsigned it = 0;       // tiles done by this CTA; stage it & 1, TMA phase (it >> 1) & 1
@@ -958,8 +971,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // tickets run two tiles ahead: fetch the one after the next now,
         // decode it into the ring at the end of this tile
         unsigned after = 0;
-        if (threadIdx.x == 0)
+        if (threadIdx.x == 0) {
             after = MODE == MODE_AGG ? blockIdx.x + (it + 2u) * gridDim.x : atomicAdd(&slot.ticket, 1u);
+            if (may_skip) sm.resid_skip = (int)*(volatile unsigned *)&slot.failed;
+        }
         if (TMA) {
             // the other stage is free (every warp passed the barrier that
             // ends the previous tile): start the next tile's loads a whole
@@ -1169,52 +1184,68 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             // row pointer of this lane's first step; lanes past d and steps past T
             // write nothing
             float *srow = a.S + ti.off + (size_t)warp * L * 4 * d + lane;
+            // the steps, with (FULL) or without the residual of the new iterate
+            auto walk_b = [&](auto full_tag) {
+                constexpr bool FULL = decltype(full_tag)::value;
     #pragma unroll
-            for (int i = 0; i < L; ++i) {
-                const int sl = warp * L + i;
-                const bool wr = jv && (t_seg + i < T);
-                if (VARLEN && ((ti.mask >> sl) & 1ull)) {
-                    // a sequence starts here: nothing from before enters it
+                for (int i = 0; i < L; ++i) {
+                    const int sl = warp * L + i;
+                    const bool wr = jv && (t_seg + i < T);
+                    if (VARLEN && ((ti.mask >> sl) & 1ull)) {
+                        // a sequence starts here: nothing from before enters it
     #pragma unroll
-                    for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
-                }
-                // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
-                const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
-                float sn[4];
-                jac_mul_add(Jc[i], dl, f4, sn);
-    #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
-                    dl[e] = sn[e] - so;
-                }
-                if (TMA) {
-                    // rows past T and features past d fall outside the tensor and
-                    // are not stored
-    #pragma unroll
-                    for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sn[e];
-                } else {
-    #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
-                }
-                if (RESID) {
-                    if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
-                    Cell f;
-                    cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
-                                             sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane], rz, ri,
-                                             rf, ro, f);
-                    const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+                        for (int e = 0; e < 4; ++e) dl[e] = 0.0f;
+                    }
+                    // S_new_t = f_t + J_t delta_{t-1};  delta_t = S_new_t - S_old_t
+                    const float f4[4] = {Jc[i].c, Jc[i].n, Jc[i].m, Jc[i].h};
+                    float sn[4];
+                    jac_mul_add(Jc[i], dl, f4, sn);
     #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float af = wr ? fabsf(F[e]) : 0.0f;
-                        const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
-                        mx_raw = fmax_nan(mx_raw, af);
-                        mx_sc = fmax_nan(mx_sc, sc);
+                        const float so = FIRST ? 0.f : sm.S[st][sl][e][lane];
+                        dl[e] = sn[e] - so;
                     }
-                }
+                    if (TMA) {
+                        // rows past T and features past d fall outside the tensor and
+                        // are not stored
     #pragma unroll
-                for (int e = 0; e < 4; ++e) snp[e] = sn[e];
-            }
+                        for (int e = 0; e < 4; ++e) sm.O[sl][e][lane] = sn[e];
+                    } else {
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+                    }
+                    if (FULL) {
+                        if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
+                        Cell f;
+                        cell_eval<FORGET, false>(snp[0], snp[1], snp[2], snp[3], sm.P[st][sl][0][lane],
+                                                 sm.P[st][sl][1][lane], sm.P[st][sl][2][lane], sm.P[st][sl][3][lane],
+                                                 rz, ri, rf, ro, f);
+                        const float F[4] = {sn[0] - f.c, sn[1] - f.n, sn[2] - f.m, sn[3] - f.h};
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float af = wr ? fabsf(F[e]) : 0.0f;
+                            const float sc = __fdividef(af, 1.0f + fabsf(sn[e]));
+                            mx_raw = fmax_nan(mx_raw, af);
+                            mx_sc = fmax_nan(mx_sc, sc);
+                        }
+                    } else if (RESID && i == L - 1) {
+                        // only whether the new states are finite: a non-finite
+                        // value travels down the lane to the thread's last
+                        // step (dense sequences: nothing resets the lane)
+                        const bool fin = (fabsf(sn[0]) <= FLT_MAX) && (fabsf(sn[1]) <= FLT_MAX) &&
+                                         (fabsf(sn[2]) <= FLT_MAX) && (fabsf(sn[3]) <= FLT_MAX);
+                        if (jv && !fin) {
+                            mx_raw = __int_as_float(0x7fc00000);
+                            mx_sc = mx_raw;
+                        }
+                    }
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) snp[e] = sn[e];
+                }
+            };
+            if (RESID && (!may_skip || !sm.resid_skip)) walk_b(std::true_type{});
+            else walk_b(std::false_type{});
             if (TMA) {
                 tma_store_fence();
                 __syncwarp();
@@ -1229,6 +1260,11 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     #pragma unroll
                 for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
             }
+            // a failure of the test is announced to the tiles after it (until
+            // this CTA has seen the announcement)
+            if (may_skip && !sm.resid_skip &&
+                __any_sync(0xffffffffu, (a.resid_raw ? mx_raw : mx_sc) > a.tol) && lane == 0)
+                atomicExch(&slot.failed, 1u);
 
         }
         // the tile after the next one (read two tiles from now), decoded where
@@ -1348,14 +1384,30 @@ inline Args launch_args(const Args &base, int k)
 // Guess launches of a solve with `sweeps` refinement sweeps: launch 0 runs
 // the decoupled guess and the first GUESS_STAGES - 1 sweeps tile by tile;
 // any further sweep is a launch of its own (1, 2, ...).
+// The caller's optional timing events (slstm_newton_config.events): the next
+// one is recorded before each launch of work and after the last.
+struct LaunchEvents {
+    int n;
+    void *const *ev;
+    int next;
+    cudaError_t record(cudaStream_t st)
+    {
+        const int i = next++;
+        if (i >= n || ev[i] == nullptr) return cudaSuccess;
+        return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
+    }
+};
+
 inline int guess_launches(int sweeps) { return 1 + (sweeps > GUESS_STAGES - 1 ? sweeps - (GUESS_STAGES - 1) : 0); }
 
 template <int FORGET, bool TMA, bool VARLEN>
-cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, int sms, cudaStream_t st)
+cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, int sms, LaunchEvents &le,
+                             cudaStream_t st)
 {
     const int fused = 1 + (sweeps < GUESS_STAGES - 1 ? sweeps : GUESS_STAGES - 1);
     const Args a0 = launch_args(base, 0);
-    cudaError_t e;
+    cudaError_t e = le.record(st);
+    if (e != cudaSuccess) return e;
     switch (fused) {
     case 1: e = launch_guess_ns<FORGET, 1, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
     case 2: e = launch_guess_ns<FORGET, 2, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
@@ -1363,8 +1415,10 @@ cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, 
     default: e = launch_guess_ns<FORGET, 4, false, TMA, VARLEN>(a0, m, 0, sms, st); break;
     }
     const int n = guess_launches(sweeps);
-    for (int k = 1; k < n && e == cudaSuccess; ++k)
+    for (int k = 1; k < n && e == cudaSuccess; ++k) {
+        if ((e = le.record(st)) != cudaSuccess) return e;
         e = launch_guess<FORGET, true, TMA, VARLEN>(launch_args(base, k), m, k, sms, st);
+    }
     return e;
 }
 
@@ -1373,21 +1427,23 @@ cudaError_t launch_guess_all(const Args &base, const NewtonMaps &m, int sweeps, 
 // Newton iterations k = k0 .. k0 + max_iters - 1.
 template <int FORGET, bool TMA, bool VARLEN>
 cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
-                         int init, cudaStream_t st)
+                         int init, LaunchEvents &le, cudaStream_t st)
 {
     if (init == SLSTM_INIT_DECOUPLED) {
-        const cudaError_t e = launch_guess_all<FORGET, TMA, VARLEN>(base, m, base.guess_sweeps, sms, st);
+        const cudaError_t e = launch_guess_all<FORGET, TMA, VARLEN>(base, m, base.guess_sweeps, sms, le, st);
         if (e != cudaSuccess) return e;
     } else if (init == SLSTM_INIT_GIVEN) {
         const long long n = (long long)base.n_tiles * 128;
-        gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(base);
-        const cudaError_t e = cudaGetLastError();
+        cudaError_t e = le.record(st);
         if (e != cudaSuccess) return e;
+        gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(base);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     for (int k = base.k0; k < base.k0 + max_iters; ++k) {
         const Args a = launch_args(base, k);
         const bool resid = !fixed || (k + 1 - base.k0 == max_iters);
-        cudaError_t e;
+        cudaError_t e = le.record(st);
+        if (e != cudaSuccess) return e;
         if (two_pass) {
             if ((e = launch_pass<FORGET, TMA, VARLEN, MODE_AGG>(a, m, k, false, sms, st)) != cudaSuccess) return e;
             const int n_chunks = a.n_tiles / a.n_groups;
@@ -1400,7 +1456,7 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         }
         if (e != cudaSuccess) return e;
     }
-    return cudaSuccess;
+    return le.record(st);
 }
 
 struct Layout {
@@ -1450,10 +1506,10 @@ int sm_count()
 
 template <int FORGET, bool TMA>
 cudaError_t launch_iters_any(const Args &a, const NewtonMaps &m, int max_iters, bool fixed, bool two_pass, int sms,
-                             bool varlen, int init, cudaStream_t st)
+                             bool varlen, int init, LaunchEvents &le, cudaStream_t st)
 {
-    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, two_pass, sms, init, st)
-                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, two_pass, sms, init, st);
+    return varlen ? launch_iters<FORGET, TMA, true>(a, m, max_iters, fixed, two_pass, sms, init, le, st)
+                  : launch_iters<FORGET, TMA, false>(a, m, max_iters, fixed, two_pass, sms, init, le, st);
 }
 
 }  // namespace
@@ -1502,6 +1558,7 @@ cudaError_t prepare(const float *P, const float *R, const float *s0, float *S, c
     a.guess_sweeps = cfg.guess_sweeps;
     a.k0 = cfg.init == SLSTM_INIT_ZERO ? 0 : (cfg.init == SLSTM_INIT_DECOUPLED ? guess_launches(cfg.guess_sweeps) : 1);
     a.resid_raw = cfg.residual_mode == SLSTM_RESIDUAL_RAW ? 1 : 0;
+    a.exact_hist = cfg.history == SLSTM_HISTORY_EXACT ? 1 : 0;
     a.guess_tested = (cfg.init == SLSTM_INIT_DECOUPLED && !a.fixed) ? 1 : 0;
     a.vec16 = ((d & 3) == 0 && (reinterpret_cast<uintptr_t>(P) & 15) == 0 &&
                (reinterpret_cast<uintptr_t>(S) & 15) == 0) ? 1 : 0;
@@ -1555,13 +1612,16 @@ cudaError_t newton_forward(const float *P, const float *R, const float *s0, floa
     const int sms = sm_count();
     const bool v = vl != nullptr;
     const int init = cfg.init;
+    LaunchEvents le{cfg.n_events, cfg.events, 0};
     if (cfg.forget == SLSTM_FORGET_EXP)
-        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
+        return tma ? launch_iters_any<SLSTM_FORGET_EXP, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, le,
+                                                              st)
                    : launch_iters_any<SLSTM_FORGET_EXP, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
-                                                               st);
-    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init, st)
+                                                               le, st);
+    return tma ? launch_iters_any<SLSTM_FORGET_SIGMOID, true>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
+                                                              le, st)
                : launch_iters_any<SLSTM_FORGET_SIGMOID, false>(a, m, cfg.max_iters, a.fixed, two_pass, sms, v, init,
-                                                               st);
+                                                               le, st);
 }
 
 cudaError_t newton_guess_prepare(const float *P, const float *s0, float *S, const slstm_newton_config &cfg,
@@ -1809,6 +1869,8 @@ slstm_newton_config cp_config(int forget, const slstm_newton_config *cfg)
     c.guess_sweeps = 0;
     c.carry_mode = SLSTM_CARRY_TWO_PASS;
     c.debug_fault = 0;
+    c.n_events = 0;
+    c.events = nullptr;
     return c;
 }
 

@@ -51,6 +51,8 @@ bool config_ok(const slstm_newton_config &c)
     if (!(c.tol >= 0.0f) || c.wait_limit_us < 0) return false;
     if (c.init < SLSTM_INIT_DECOUPLED || c.init > SLSTM_INIT_GIVEN) return false;
     if (c.residual_mode != SLSTM_RESIDUAL_SCALED && c.residual_mode != SLSTM_RESIDUAL_RAW) return false;
+    if (c.n_events < 0 || (c.n_events > 0 && c.events == nullptr)) return false;
+    if (c.history != SLSTM_HISTORY_BOUND && c.history != SLSTM_HISTORY_EXACT) return false;
     return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
 }
 
@@ -69,9 +71,9 @@ bool block_sizes_ok(int B, int T, int D, int F)
     return sizes_ok(B, T, D, F) && D % 8 == 0 && F % 32 == 0;
 }
 
-// The trunk backward's CUDA-core GEMMs tile the B*T rows 128 at a time on the
-// grid's y axis (at most 65535 tiles).
-constexpr long long kBlockBwdMaxRows = 65535LL * 128;
+// The trunk backward's column sums (weight gradients of the norms) take the
+// B*T rows 256 at a time on the grid's y axis (at most 65535 chunks).
+constexpr long long kBlockBwdMaxRows = 65535LL * 256;
 
 }  // namespace
 

@@ -40,6 +40,7 @@ __device__ inline void finalize_iteration(const StopRule &a, int k, bool resid)
     nx.finished = 0u;
     nx.maxF_raw = 0u;
     nx.maxF_scaled = 0u;
+    nx.failed = 0u;
     st->iters = n + 1;
     st->max_abs_F[n % SLSTM_STATS_HISTORY] = resid ? raw : -1.0f;
     st->max_scaled_F[n % SLSTM_STATS_HISTORY] = resid ? sc : -1.0f;

@@ -91,6 +91,18 @@ def make_inputs(w: Workload, with_dH: bool = True) -> dict:
     return {"x": x, "Wx": Wx, "R": R, "bias": bias, "s0": s0, "dH": dH}
 
 
+def make_head_R(w: Workload, d_head: int, seed: int = None) -> torch.Tensor:
+    """Block-diagonal recurrent weights (4, d_h / d_head, d_head, d_head) for
+    head mixing: entries U(-r, r) with r = the workload's R scale / sqrt(d_head),
+    so that a head's recurrent input has the diagonal workloads' magnitude."""
+    if w.d_h % d_head:
+        raise ValueError(f"d_head={d_head} does not divide d_h={w.d_h}")
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 1 if seed is None else seed)
+    H = w.d_h // d_head
+    return (torch.rand(4, H, d_head, d_head, generator=g, dtype=torch.float32) * 2.0 - 1.0) * (w.r_scale / d_head ** 0.5)
+
+
 def as_f64(t: torch.Tensor):
     """Exact widening of an fp32/bf16 tensor to a float64 numpy array."""
     return t.detach().to("cpu").to(torch.float64).numpy()

@@ -99,6 +99,8 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(cfg=_cfg(guess_sweeps=-1)) == E
     assert call(cfg=_cfg(guess_sweeps=65)) == E
     assert call(cfg=_cfg(max_iters=0, init=1)) == E      # only the decoupled guess allows 0 iterations
+    assert call(cfg=_cfg(n_events=-1)) == E
+    assert call(cfg=_cfg(n_events=3)) == E               # timing events announced, array missing
     assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
     assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
     assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E
@@ -210,7 +212,7 @@ def test_block_backward_entry_point_rejects_bad_arguments():
 
     assert bwd(forget=5) == E
     assert bwd(D=60) == E and bwd(F=100) == E and bwd(B=0) == E
-    assert bwd(B=2, T=65535 * 64 + 1) == E            # more row tiles than the grid's y axis
+    assert bwd(B=2, T=65535 * 128 + 1) == E           # more column-sum chunks than the grid's y axis
     assert bwd(eps=-1.0) == E
     assert bwd(x=FAKE_MIS) == E
     assert bwd(wb=ctypes.c_size_t(64)) == E

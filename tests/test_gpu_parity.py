@@ -94,13 +94,14 @@ def test_preact_gemm_matches_oracle(dtype, B, T, d_in, d_h, cuda_device):
 CARRY_MODES = [1, 2]
 
 
-def _newton_case(w: Workload, fixed_k=None, carry_mode=0, init="decoupled", residual_mode="scaled"):
+def _newton_case(w: Workload, fixed_k=None, carry_mode=0, init="decoupled", residual_mode="scaled",
+                 exact_history=False):
     inp = make_inputs(w, with_dH=False)
     Pt = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
     if fixed_k is None:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
                                    max_iters=w.max_iters, fixed=False, tol=w.tol, carry_mode=carry_mode,
-                                   init=init, residual_mode=residual_mode)
+                                   init=init, residual_mode=residual_mode, exact_history=exact_history)
     else:
         S, st = api.newton_forward(Pt, _dev(inp["R"]), _dev(inp["s0"]), forget=w.forget,
                                    max_iters=fixed_k, fixed=True, tol=w.tol, carry_mode=carry_mode, init=init,
@@ -126,9 +127,43 @@ def _check_status_against_oracle(st, ost):
     return False
 
 
+@pytest.mark.parametrize("sweeps,carry_mode", [(2, 1), (5, 1), (2, 2)])
+def test_newton_launch_events_bracket_every_launch(sweeps, carry_mode, cuda_device):
+    """The optional timing events: one before each launch of work (the guess
+    launches, then one per iteration) and one after the last; the solution
+    is that of the same call without them (up to the rounding order of the
+    decoupled look-back, which depends on timing: a tile's carry comes from
+    its predecessor's published state or from composing earlier runs)."""
+    w = scaled(WORKLOADS["slstm_f32_b8_t1024_d256"], B=2, T=300, d_in=64, d_h=64)
+    inp = make_inputs(w, with_dH=False)
+    P = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    R, s0 = _dev(inp["R"]), _dev(inp["s0"])
+    K = 6
+    kw = dict(forget=w.forget, max_iters=K, fixed=False, tol=w.tol, carry_mode=carry_mode, guess_sweeps=sweeps)
+    S_ref, st_ref = api.newton_forward(P, R, s0, **kw)
+    g = 1 + max(0, sweeps - 3)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(g + K + 1)]
+    S, st = api.newton_forward(P, R, s0, events=evs, **kw)
+    torch.cuda.synchronize()
+
+    def close(a, b):
+        return ((a - b).abs() / (1 + b.abs())).max().item() <= 1e-5
+
+    assert close(S, S_ref)
+    a, b = api.read_stats(st), api.read_stats(st_ref)
+    assert a["iters"] == b["iters"] and a["converged"] and b["converged"]
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(evs) - 1)]
+    assert all(t >= 0.0 for t in times), times
+    # fewer events than launches: only the first ones are recorded
+    few = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    S2, _ = api.newton_forward(P, R, s0, events=few, **kw)
+    torch.cuda.synchronize()
+    assert close(S2, S_ref) and few[0].elapsed_time(few[1]) >= 0.0
+
+
 def test_newton_tiny_converges_to_sequential(cuda_device):
     w = WORKLOADS["tiny_f32"]
-    inp, S, st, Pref = _newton_case(w)
+    inp, S, st, Pref = _newton_case(w, exact_history=True)
     ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget)
     _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), w.forget, w.max_iters, False, w.tol,
                                 sweeps=SW)
@@ -161,7 +196,9 @@ def test_newton_converges_to_sequential_sigmoid(B, T, d, carry_mode, cuda_device
 @pytest.mark.parametrize("B,T,d", [(2, 16, 40), (2, 32, 40), (1, 100, 33), (2, 128, 64), (8, 64, 256), (1, 300, 36), (2, 200, 40)])
 def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, init, cuda_device):
     w = Workload("t", B, T, 16, d, "f32", forget, 0.5, 11, 1e-6, 64)
-    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode, init=init)
+    # exact history: the iteration at which a diverging run stops is compared
+    # with the fp64 run's residual there
+    inp, S, st, Pref = _newton_case(w, carry_mode=carry_mode, init=init, exact_history=True)
     _, ost = oracle.newton_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget, w.max_iters, False, w.tol,
                                 init=init, sweeps=SW)
     converged = _check_status_against_oracle(st, ost)
@@ -170,6 +207,32 @@ def test_newton_status_agrees_with_oracle(forget, B, T, d, carry_mode, init, cud
     if converged:
         ref = oracle.sequential_btgd(Pref, as_f64(inp["R"]), as_f64(inp["s0"]), forget)
         assert _h_err(S, ref) <= TOL_F32
+
+
+@pytest.mark.parametrize("carry_mode", CARRY_MODES)
+@pytest.mark.parametrize("B,T,d,sweeps", [(2, 1000, 64, 0), (4, 2000, 96, 1), (8, 1024, 256, 2), (1, 300, 33, 0)])
+def test_newton_bound_history_keeps_the_decisions(B, T, d, sweeps, carry_mode, cuda_device):
+    """The default history (an iteration whose test already failed somewhere
+    stops evaluating the rest of its residual) takes the same decisions as the
+    exact one: the same iterations, converged, the same final residual; the
+    earlier entries are lower bounds above the tolerance."""
+    w = Workload("t", B, T, 16, d, "f32", "sigmoid", 0.5, 21, 1e-6, 32)
+    inp = make_inputs(w, with_dH=False)
+    P = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
+    kw = dict(forget=w.forget, max_iters=w.max_iters, fixed=False, tol=w.tol, carry_mode=carry_mode,
+              guess_sweeps=sweeps)
+    Sb, stb = api.newton_forward(P, _dev(inp["R"]), _dev(inp["s0"]), **kw)
+    Se, ste = api.newton_forward(P, _dev(inp["R"]), _dev(inp["s0"]), exact_history=True, **kw)
+    b, e = api.read_stats(stb), api.read_stats(ste)
+    print("bound", b["iters"], b["max_scaled_F"], "exact", e["iters"], e["max_scaled_F"])
+    assert b["converged"] and e["converged"] and b["iters"] == e["iters"] and b["error"] == 0
+    # the last entry is at the fp32 rounding floor of the iterate, which the
+    # look-back's timing-dependent rounding order moves between runs
+    assert b["max_scaled_F"][-1] <= w.tol and e["max_scaled_F"][-1] <= w.tol
+    assert abs(b["max_scaled_F"][-1] - e["max_scaled_F"][-1]) <= 1e-3 * e["max_scaled_F"][-1] + 5e-7
+    for x, y in zip(b["max_scaled_F"][:-1], e["max_scaled_F"][:-1]):
+        assert w.tol < x <= y * (1 + 1e-3), (x, y)
+    assert ((Sb - Se).abs() / (1 + Se.abs())).max().item() <= 1e-5
 
 
 def _s_err(S_gpu, S_ref):
