@@ -1020,10 +1020,12 @@ def run_block(args, w):
 
 # DRAM bytes (read + write) per element of B*T*d_h of the Newton solve's kernels, from one ncu
 # capture of the training workload shortened to T = 2048 (summarised under profiles/): the guess
-# launch, a refinement sweep and a Newton iteration that evaluates its residual.  The counters describe the kernel
-# sources with this SHA-256; any other build reports traffic null.  Traffic per element does not
-# depend on T (every tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": None, "guess": None, "sweep": None, "iter": None}
+# launch (the guess and two sweeps fused), a separate sweep launch (not captured: None) and a Newton
+# iteration that evaluates its whole residual.  The counters describe the kernel sources with this
+# SHA-256; any other build reports traffic null.  Traffic per element does not depend on T (every
+# tile moves the same bytes), so it scales to a full launch by the element count.
+NEWTON_TRAFFIC = {"sources_sha256": "d8ca6e5c40b3016b044fcdaf0b1713c0989975461c1f1ec72d322c322b4462bc",
+                  "guess": 30.9, "sweep": None, "iter": 46.4}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
@@ -1059,7 +1061,9 @@ def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
     t = NEWTON_TRAFFIC
     if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
         return None
-    return (t["guess"] + t["sweep"] * (guess_launches(sweeps) - 1) + t["iter"] * iters) * elems
+    if guess_launches(sweeps) > 1 and t["sweep"] is None:
+        return None
+    return (t["guess"] + (t["sweep"] or 0.0) * (guess_launches(sweeps) - 1) + t["iter"] * iters) * elems
 
 
 def newton_iter_traffic_bytes(elems: int):

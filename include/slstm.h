@@ -115,7 +115,11 @@ typedef enum {
  *   debug_fault 0 in normal use.  1 makes one tile of the first iteration
  *               withhold its scan carry, so that its successor's bounded
  *               wait expires (the run then reports SLSTM_ERR_TIMEOUT in
- *               stats.error; results are not meaningful).
+ *               stats.error; results are not meaningful).  2: in the
+ *               bounds-checked build, each iteration checks its last tile
+ *               boundary store against an extent one element short (the
+ *               store is skipped and reported; a self-test of the checks);
+ *               ignored in the normal build.
  *   wait_limit_us  upper bound of one bounded wait, in microseconds
  *               (0 = the default of 2 seconds).
  *   carry_mode  how a tile gets the scan carry entering it (same results up
@@ -230,6 +234,29 @@ typedef struct {
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *slstm_status_string(int status);
+
+/*
+ * Bounds-checked build.  The library can also be built with SLSTM_CHECKED
+ * defined (a separate diagnostic library, libslstm_checked.so): there every
+ * guarded global-memory access of the kernels tests its element index
+ * against the extent of its buffer, skips the access when it is outside,
+ * counts it and records the first one.  Nothing traps; the kernels run on.
+ *   slstm_check_enabled  1 in the checked build, 0 in the normal one.
+ *   slstm_check_status   waits for the device, then writes out[0] = the
+ *                        number of out-of-bounds accesses since the last
+ *                        clear and, for the first of them (0 when none),
+ *                        out[1] = its site (file id * 100000 + source line;
+ *                        slstm_check_site_file names the file), out[2] = the
+ *                        element index, out[3] = the extent.  All zero in the
+ *                        normal build.  SLSTM_ERR_INVALID_ARG for a null out,
+ *                        SLSTM_ERR_CUDA when the device cannot be read.
+ *   slstm_check_clear    zeroes the records (waits for the device).
+ *   slstm_check_site_file  the source file of a site's file id, or NULL.
+ */
+int slstm_check_enabled(void);
+int slstm_check_status(long long *out);
+int slstm_check_clear(void);
+const char *slstm_check_site_file(int file_id);
 
 /*
  * Bytes of workspace an operation needs for the given sizes (0 when it needs

@@ -63,6 +63,10 @@ _Z = ctypes.c_size_t
 # name -> (restype, argtypes); every function of include/slstm.h
 SIGNATURES = {
     "slstm_status_string": (ctypes.c_char_p, [_I]),
+    "slstm_check_enabled": (_I, []),
+    "slstm_check_status": (_I, [ctypes.POINTER(ctypes.c_longlong)]),
+    "slstm_check_clear": (_I, []),
+    "slstm_check_site_file": (ctypes.c_char_p, [_I]),
     "slstm_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "slstm_preact_gemm": (_I, [_V, _V, _I, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
     "slstm_newton_forward": (_I, [_V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _V, _Z, _V]),
@@ -100,20 +104,50 @@ def lib_path() -> str:
     return _build.LIB
 
 
+def _open(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(f"the library was not built at {path}")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def load() -> ctypes.CDLL:
-    """Load libslstm.so (building it first when it is missing or stale)."""
+    """The active library: libslstm.so (built first when missing or stale),
+    or the bounds-checked one inside `checked_library()`."""
     global _lib
     if _lib is None:
-        path = _build.build()
-        if not os.path.exists(path):
-            raise RuntimeError(f"libslstm.so was not built at {path}")
-        lib = ctypes.CDLL(path)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(lib, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = lib
+        _lib = _open(_build.build())
     return _lib
+
+
+_checked = None
+
+
+def load_checked() -> ctypes.CDLL:
+    """The bounds-checked diagnostic library, libslstm_checked.so."""
+    global _checked
+    if _checked is None:
+        _checked = _open(_build.build(checked=True))
+    return _checked
+
+
+class checked_library:
+    """Within this context every api call goes to the bounds-checked library."""
+
+    def __enter__(self):
+        global _lib
+        self._saved = load()
+        _lib = load_checked()
+        return _lib
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self._saved
+        return False
 
 
 class SlstmError(RuntimeError):

@@ -1,9 +1,11 @@
 """Build libslstm.so in-tree with nvcc for sm_100a.
 
-    python -m nonlinear_rnn_pararnn_b200.build [--verbose-ptxas]
+    python -m nonlinear_rnn_pararnn_b200.build [--verbose-ptxas] [--checked]
 
 The library is written next to this file (``libslstm.so``) so that it ships
 with the source tree; it is rebuilt when any source or header is newer.
+``--checked`` builds the bounds-checked diagnostic library
+(``libslstm_checked.so``, the sources compiled with SLSTM_CHECKED).
 """
 from __future__ import annotations
 
@@ -18,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libslstm.so")
+LIB_CHECKED = os.path.join(PKG, "libslstm_checked.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -43,21 +46,23 @@ def _inputs() -> list:
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+def build(force: bool = False, verbose_ptxas: bool = False, checked: bool = False) -> str:
     """Compile every source to an object in parallel (one nvcc per file),
-    then link the shared library; objects live in a temporary folder."""
-    if not force and not verbose_ptxas and up_to_date():
-        return LIB
+    then link the shared library; objects live in a temporary folder.
+    checked: the bounds-checked diagnostic library instead."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not verbose_ptxas and up_to_date(lib):
+        return lib
     import concurrent.futures
     import tempfile
-    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"] + (["-DSLSTM_CHECKED"] if checked else [])
     with tempfile.TemporaryDirectory(prefix="slstm_build_") as tmpdir:
         def compile_one(src):
             obj = os.path.join(tmpdir, os.path.basename(src) + ".o")
@@ -70,13 +75,12 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         workers = max(1, min(len(srcs), os.cpu_count() or 1))
         with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
             objs = list(pool.map(compile_one, srcs))
-        tmp = LIB + f".tmp{os.getpid()}"
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call([_nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-Xcompiler",
                                "-fPIC", "-o", tmp, *objs])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv)
-    print(LIB)
+    print(build(force=True, verbose_ptxas="--verbose-ptxas" in sys.argv, checked="--checked" in sys.argv))

@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 #include <string.h>
 
+#define SLSTM_FILE_ID 2
 #include "launchers.h"
 #include "lookback.cuh"
 #include "tma.cuh"
@@ -46,6 +47,7 @@ struct BwdArgs {
     const unsigned *vmask;   // packed sequences: head-flag words (one per 32 steps), else null
     const int *vseq;         // packed sequences: sequence index at each head step
     int T, d, groups_per_row, n_tiles, vec16, dpt_vec8;
+    long long n_ps, n_s0, n_dpt;   // elements of S and P (and dP), of s0 (and ds0), of each half of the pair
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
@@ -80,12 +82,7 @@ struct BwdSmem {
     uint64_t bar[2];
 };
 constexpr size_t BWD_SMEM_BYTES = sizeof(BwdSmem) + 1024;
-// Warps CHAIN0 .. NW-1 walk the carry through the warp maps (chain lanes);
-// warp w < CHAIN0 starts walk B as soon as the carry entering it is stored
-// (named barrier 1 + w), the chain warps themselves after CHAIN_BAR.
-constexpr int CHAIN0 = NW - 4;
-constexpr int CHAIN_BAR = CHAIN0 + 1;
-constexpr int BWD_TMA_THREAD = (CHAIN0 - 1) * 32;   // a warp with no chain lane
+constexpr int BWD_TMA_THREAD = (NW - 1) * 32;
 constexpr uint64_t BWD_TMA_WAIT_NS = 1000000000ull;
 
 // Tensor maps: S and P as (d, 4T, B) with boxes of 32 features x 132 (S) or
@@ -142,16 +139,18 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdI
             if (rs < RS) {
                 const int r = rs >> 2, slot = rs & 3;
                 const int tS = t_lo - 1 + r, tP = t_lo + r;
-                const int bS = (tS >= 0 && tS < T) ? fbytes : 0;
+                const int bS = (tS >= 0 && tS < T && SLSTM_IN(((row0 + tS) * 4 + slot) * d + jj + fbytes / 4 - 1, a.n_ps))
+                                   ? fbytes : 0;
                 cp_async16(&sm.S[st][r][slot][4 * c], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
                 if (r < TT) {
-                    const int bP = (tP >= 0 && tP < T) ? fbytes : 0;
+                    const int bP = (tP >= 0 && tP < T && SLSTM_IN(((row0 + tP) * 4 + slot) * d + jj + fbytes / 4 - 1,
+                                                                  a.n_ps)) ? fbytes : 0;
                     cp_async16(&sm.P[st][r][slot][4 * c], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
                 }
             }
         }
         const int t = t_lo + q;   // dH row q
-        const int bH = (t >= 0 && t < T) ? fbytes : 0;
+        const int bH = (t >= 0 && t < T && SLSTM_IN((row0 + t) * d + jj + fbytes / 4 - 1, a.n_ps / 4)) ? fbytes : 0;
         cp_async16(&sm.dH[st][q][4 * c], bH ? a.dH + (row0 + t) * d + jj : a.dH, bH);
     } else {
         // 4-byte copies, lane = feature, warp w takes every 8th row
@@ -161,16 +160,16 @@ SLSTM_DEVINL void bwd_prefetch(const BwdArgs &a, BwdSmem &sm, int st, const BwdI
         for (int rs = w; rs < RS; rs += NW) {
             const int r = rs >> 2, slot = rs & 3;
             const int tS = t_lo - 1 + r, tP = t_lo + r;
-            const int bS = (fj && tS >= 0 && tS < T) ? 4 : 0;
+            const int bS = (fj && tS >= 0 && tS < T && SLSTM_IN(((row0 + tS) * 4 + slot) * d + jj, a.n_ps)) ? 4 : 0;
             cp_async4(&sm.S[st][r][slot][jl], bS ? a.S + ((row0 + tS) * 4 + slot) * d + jj : a.S, bS);
             if (r < TT) {
-                const int bP = (fj && tP >= 0 && tP < T) ? 4 : 0;
+                const int bP = (fj && tP >= 0 && tP < T && SLSTM_IN(((row0 + tP) * 4 + slot) * d + jj, a.n_ps)) ? 4 : 0;
                 cp_async4(&sm.P[st][r][slot][jl], bP ? a.P + ((row0 + tP) * 4 + slot) * d + jj : a.P, bP);
             }
         }
         for (int r = w; r < TT; r += NW) {
             const int t = t_lo + r;
-            const int bH = (fj && t >= 0 && t < T) ? 4 : 0;
+            const int bH = (fj && t >= 0 && t < T && SLSTM_IN((row0 + t) * d + jj, a.n_ps / 4)) ? 4 : 0;
             cp_async4(&sm.dH[st][r][jl], bH ? a.dH + (row0 + t) * d + jj : a.dH, bH);
         }
     }
@@ -187,7 +186,9 @@ SLSTM_DEVINL void bwd_issue_load(const BwdArgs &a, const BwdMaps &m, BwdSmem &sm
     tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, ti.t_lo * 4, ti.b);
     tma_load_3d(&sm.dH[st][0][0], &m.H, &sm.bar[st], ti.j0, ti.t_lo, ti.b);
 #pragma unroll
-    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    for (int g = 0; g < 4; ++g)
+        if (SLSTM_IN((size_t)g * a.d + ti.j0 + rbytes / 4 - 1, 4LL * a.d))
+            bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
 }
 
 // TMA: tiles arrive by TMA (BWD_TMA_THREAD, mbarrier per stage); otherwise by
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
     const unsigned G = (unsigned)a.ca.n_groups;
     const int T = a.T;
     const size_t d = (size_t)a.d;
-    const bool chain_warp = warp >= CHAIN0;
+    const bool chain_warp = warp < 4;
 
     if (threadIdx.x == 0) {
         // BWD_AGG tiles are independent: a static order needs no counter
@@ -267,7 +268,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 rf = sm.R[st][2][lane];
                 ro = sm.R[st][3][lane];
             }
-        } else if (jv) {
+        } else if (jv && SLSTM_IN(3 * d + jj, 4 * d)) {
             rz = __ldg(a.R + jj);
             ri = __ldg(a.R + d + jj);
             rf = __ldg(a.R + 2 * d + jj);
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
         }
 
         // looks at the predecessor's (later-in-time) inclusive prefix
-        const bool look = MODE == BWD_FUSED && chain_warp && chunk > 0;
+        const bool look = MODE == BWD_FUSED && chain_warp && chunk > 0 && SLSTM_IN(ticket - G, a.n_tiles);
         const unsigned long long *predw = a.ca.incw + chain_word(ticket - G, warp, lane);
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
@@ -301,9 +302,11 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             for (int e = 0; e < 4; ++e) prev[e] = sm.S[st][rl][e][lane];
             const bool head = VARLEN ? (((ti.hmask >> rl) & 1ull) != 0ull) : (t == 0);
             if (head) {
-                const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
+                const size_t sq = VARLEN ? (SLSTM_IN(t, T) ? (size_t)a.vseq[t] : 0) : (size_t)ti.b;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) prev[e] = (a.s0 && jv) ? __ldg(a.s0 + (sq * 4 + e) * d + jj) : 0.f;
+                for (int e = 0; e < 4; ++e)
+                    prev[e] = (a.s0 && jv && SLSTM_IN((sq * 4 + e) * d + jj, a.n_s0)) ? __ldg(a.s0 + (sq * 4 + e) * d + jj)
+                                                                                      : 0.f;
             }
             Cell J;
             cell_eval<FORGET, true, false, true>(prev[0], prev[1], prev[2], prev[3], sm.P[st][rl][0][lane],
@@ -353,18 +356,21 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 Aff x;
                 maps_load(sm.u.m, NW - 1, lane, x);
                 float *dst = a.ca.agg + (size_t)ticket * 20 * 32 + lane;
+                if (SLSTM_IN(ticket, a.n_tiles)) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
+                    for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
-                if (lane == 0) a.ca.flags[ticket] = whead ? 1u : 0u;
+                    for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
+                    if (lane == 0) a.ca.flags[ticket] = whead ? 1u : 0u;
+                }
             }
         } else {
 
             // ---- carry ----
             float c = 0.f;   // chunk 0: nothing enters after the sequence's last step
             bool ok = true;
-            if (MODE == BWD_APPLY && chain_warp) c = a.cin_buf[chain_word(ticket, warp, lane)];
+            if (MODE == BWD_APPLY && chain_warp && SLSTM_IN(chain_word(ticket, warp, lane), (long long)a.n_tiles * 128))
+                c = a.cin_buf[chain_word(ticket, warp, lane)];
             if (look) {
                 if ((unsigned)(w1 >> 32) == a.ca.epoch) {
                     c = __uint_as_float((unsigned)w1);
@@ -375,22 +381,17 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
             }
             const bool fast = __syncthreads_and(ok);
             if (TMA && threadIdx.x == BWD_TMA_THREAD) bwd_issue_load(a, maps, sm, st ^ 1, sm.info[rn]);
-            if (chain_warp) {
-                if (fast) {
-                    c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead, CHAIN0);
-                    if (MODE == BWD_FUSED) st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
-                    named_bar_sync(CHAIN_BAR, 4 * 32);
-                } else {
-                    if (warp == CHAIN0)
-                        tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G),
-                                                false, whead);
-                    named_bar_sync(CHAIN_BAR, 4 * 32);
-    #pragma unroll 1
-                    for (int w = 0; w < CHAIN0; ++w) named_bar_arrive(1 + w, 5 * 32);
+            if (fast) {
+                if (chain_warp) {
+                    c = carry_chain4<NW>(sm.u.m, sm.cin, c, warp, lane, whead);
+                    if (MODE == BWD_FUSED && SLSTM_IN(chain_word(ticket, warp, lane), (long long)a.n_tiles * 128))
+                        st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
                 }
-            } else {
-                named_bar_sync(1 + warp, 5 * 32);   // the carry entering this warp is stored
+            } else if (warp == 0) {
+                tile_carry_fallback<NW>(a.ca, sm.u.m, sm.cin, ticket, chunk, (int)(ticket - (unsigned)chunk * G), false,
+                                        whead);
             }
+            __syncthreads();   // every warp's carry is stored; the maps are dead from here on
 
             // ---- walk B: lambda_t = kappa_t + e_h dH_t, dP_t = G_t^T lambda_t,
             // kappa_{t-1} = J_t^T lambda_t ----
@@ -420,8 +421,8 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 if (head) {
                     // ds0 = J^T lambda at the sequence's first step; nothing
                     // enters the step before it (another sequence, or none)
-                    if (a.ds0 && jv) {
-                        const size_t sq = VARLEN ? (size_t)a.vseq[t] : (size_t)ti.b;
+                    const size_t sq = VARLEN ? (SLSTM_IN(t, T) ? (size_t)a.vseq[t] : 0) : (size_t)ti.b;
+                    if (a.ds0 && jv && SLSTM_IN(sq * 4 * d + 3 * d + jj, a.n_s0)) {
                         float *qd = a.ds0 + sq * 4 * d + jj;
     #pragma unroll
                         for (int e = 0; e < 4; ++e) qd[e * d] = kap[e];
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 const bool tv = t >= 0;   // steps before 0 (last chunk only) contribute nothing
     #pragma unroll
                 for (int e = 0; e < 4; ++e) dv[i][e] = tv ? g[e] : 0.f;
-                if (!BF16OUT && jv && tv) {
+                if (!BF16OUT && jv && tv && SLSTM_IN((row0 + t) * 4 * d + 3 * d + jj, a.n_ps)) {
                     float *pd = a.dP + (row0 + t) * 4 * d + jj;
     #pragma unroll
                     for (int e = 0; e < 4; ++e) pd[e * d] = dv[i][e];
@@ -443,7 +444,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                     dbs[e] += dv[i][e];
                 }
             }
-            __syncthreads();   // the maps are dead from here on; the dP staging takes their place
+            // the dP staging takes the dead maps' place
     #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 sm.u.o.part[warp][e][lane] = jv ? dr[e] : 0.f;
@@ -475,7 +476,7 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                 float acc = 0.f;
     #pragma unroll
                 for (int w = 0; w < NW; ++w) acc += sm.u.o.part[w][e][lane];
-                a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
+                if (SLSTM_IN(ticket, a.n_tiles)) a.partial[((size_t)ticket * 8 + e) * 32 + lane] = acc;
             }
             if (BF16OUT) {
                 // rows (part, gate, feature) of the transposed pair, 32 steps each;
@@ -494,8 +495,9 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                             __nv_bfloat16 *dst = (part ? a.dpt_lo : a.dpt_hi) + base;
     #pragma unroll
                             for (int gi = 0; gi < 4; ++gi)
-                                *reinterpret_cast<uint2 *>(dst + gi * gstride) =
-                                    *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
+                                if (SLSTM_IN(base + gi * gstride + 3, a.n_dpt))
+                                    *reinterpret_cast<uint2 *>(dst + gi * gstride) =
+                                        *reinterpret_cast<const uint2 *>(&sm.u.o.dpt[part][gi][jl][4 * q]);
                         }
                     }
                 } else {
@@ -503,7 +505,8 @@ __global__ void __launch_bounds__(NW * 32, 2) adjoint_vjp_kernel(BwdArgs a, cons
                     const int t = t_lo + tl;
                     for (int r = warp; r < 2 * 4 * 32; r += NW) {
                         const int part = r >> 7, gi = (r >> 5) & 3, jl = r & 31;
-                        if (t >= 0 && ti.j0 + jl < a.d) {
+                        if (t >= 0 && ti.j0 + jl < a.d &&
+                            SLSTM_IN(((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t, a.n_dpt)) {
                             __nv_bfloat16 *dst = part ? a.dpt_lo : a.dpt_hi;
                             dst[((size_t)gi * d + ti.j0 + jl) * a.ldT + row0 + t] = sm.u.o.dpt[part][gi][jl][tl];
                         }
@@ -557,7 +560,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float *__res
     for (int q = warp; q < terms; q += 8) {
         const int c = q / B, b = q % B;
         const size_t ticket = (size_t)c * G + (size_t)b * groups_per_row + jb;
-        acc += partial[(ticket * 8 + e) * 32 + lane];
+        if (SLSTM_IN(ticket, (long long)n_chunks * G)) acc += partial[(ticket * 8 + e) * 32 + lane];
     }
     s_sum[warp][lane] = acc;
     __syncthreads();
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(256) reduce_partials_kernel(const float *__res
 #pragma unroll
         for (int w = 0; w < 8; ++w) t += s_sum[w][lane];
         const int j = jb * 32 + lane;
-        if (j < d) {
+        if (j < d && SLSTM_IN((size_t)(e & 3) * d + j, 4LL * d)) {
             if (e < 4)
                 dR[(size_t)e * d + j] = (float)t;
             else
@@ -727,6 +730,9 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.dpt_hi = reinterpret_cast<__nv_bfloat16 *>(base + l.dpt);
     a.dpt_lo = a.dpt_hi + 4LL * d_h * l.ldT;
     a.ldT = l.ldT;
+    a.n_ps = l.n;
+    a.n_dpt = 4LL * d_h * l.ldT;
+    a.n_s0 = (long long)(vl ? vl->n_seq : B) * 4 * d_h;
     a.partial = reinterpret_cast<float *>(base + l.partial);
     a.ds0 = ds0;
     a.ticket = reinterpret_cast<unsigned *>(base + l.ticket);
@@ -737,6 +743,7 @@ cudaError_t backward_launch(const void *x, const void *Wx, int dtype, const floa
     a.ca.epoch = 1;
     a.ca.wait_ns = 2000000000ull;
     a.ca.n_groups = l.n_groups;
+    a.ca.n_tiles = l.n_tiles;
     a.T = T;
     a.d = d_h;
     a.groups_per_row = l.groups_per_row;

@@ -15,6 +15,8 @@
 // same lane.
 #include <cuda_bf16.h>
 
+#define SLSTM_FILE_ID 6
+#include "checked.cuh"
 #include "common.cuh"
 #include "launchers.h"
 
@@ -75,10 +77,15 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const T *__restr
         for (int k = (q * 32 + lane) * VEC; k < d_in; k += DEC_WPF * 32 * VEC) {
             float w[4][VEC];
 #pragma unroll
-            for (int g = 0; g < 4; ++g) load_vec(Wx + ((size_t)g * dd + j) * d_in + k, w[g]);
+            for (int g = 0; g < 4; ++g) {
+                if (SLSTM_IN(((size_t)g * dd + j) * d_in + k + VEC - 1, 4LL * d * d_in))
+                    load_vec(Wx + ((size_t)g * dd + j) * d_in + k, w[g]);
+                else
+                    for (int i = 0; i < VEC; ++i) w[g][i] = 0.0f;
+            }
 #pragma unroll
             for (int b = 0; b < BM; ++b) {
-                if (b < B) {
+                if (b < B && SLSTM_IN((size_t)b * d_in + k + VEC - 1, (long long)B * d_in)) {
                     float xv[VEC];
                     load_vec(x + (size_t)b * d_in + k, xv);
 #pragma unroll
@@ -113,7 +120,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const T *__restr
         p[g] = t + __ldg(bias + g * dd + j);
     }
     float s[4] = {0.f, 0.f, 0.f, 0.f};
-    if (s_prev) {
+    if (s_prev && SLSTM_IN(((size_t)lane * 4 + 3) * dd + j, (long long)B * 4 * d)) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[e] = s_prev[((size_t)lane * 4 + e) * dd + j];
     }
@@ -121,6 +128,7 @@ __global__ void __launch_bounds__(DEC_WARPS * 32) decode_kernel(const T *__restr
     cell_eval<FORGET, false>(s[0], s[1], s[2], s[3], p[0], p[1], p[2], p[3], __ldg(R + j), __ldg(R + dd + j),
                              __ldg(R + 2 * dd + j), __ldg(R + 3 * dd + j), o);
     float *qo = s_next + (size_t)lane * 4 * dd + j;
+    if (!SLSTM_PIN(qo + 3 * dd, s_next, (long long)B * 4 * d)) return;
     qo[0] = o.c;
     qo[dd] = o.n;
     qo[2 * dd] = o.m;

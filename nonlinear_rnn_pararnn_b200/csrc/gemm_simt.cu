@@ -6,6 +6,8 @@
 // memory in slices of 16.
 #include <cuda_bf16.h>
 
+#define SLSTM_FILE_ID 9
+#include "checked.cuh"
 #include "common.cuh"
 #include "launchers.h"
 
@@ -37,6 +39,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g)
 
     const bool a_m_contig = (g.sam == 1);
     const bool b_n_contig = (g.sbn == 1);
+    // extents the strides span (checked build)
+    [[maybe_unused]] const long long n_a = (long long)(g.M - 1) * g.sam + (long long)(g.K - 1) * g.sak + 1;
+    [[maybe_unused]] const long long n_b = (long long)(g.K - 1) * g.sbk + (long long)(g.N - 1) * g.sbn + 1;
     for (int k0 = 0; k0 < g.K; k0 += BK) {
         // A tile: BM x BK = 2048 elements, 8 per thread; walk the contiguous
         // dimension across consecutive threads.
@@ -53,7 +58,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g)
             }
             const int m = m0 + mm, k = k0 + kk;
             float v = 0.f;
-            if (m < g.M && k < g.K) v = load_elem(g.A, g.a_dtype, (long long)m * g.sam + (long long)k * g.sak);
+            if (m < g.M && k < g.K && SLSTM_IN((long long)m * g.sam + (long long)k * g.sak, n_a))
+                v = load_elem(g.A, g.a_dtype, (long long)m * g.sam + (long long)k * g.sak);
             As[kk][mm] = v;
         }
 #pragma unroll
@@ -69,7 +75,8 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g)
             }
             const int n = n0 + nn, k = k0 + kk;
             float v = 0.f;
-            if (n < g.N && k < g.K) v = load_elem(g.B, g.b_dtype, (long long)k * g.sbk + (long long)n * g.sbn);
+            if (n < g.N && k < g.K && SLSTM_IN((long long)k * g.sbk + (long long)n * g.sbn, n_b))
+                v = load_elem(g.B, g.b_dtype, (long long)k * g.sbk + (long long)n * g.sbn);
             Bs[kk][nn] = v;
         }
         __syncthreads();
@@ -97,7 +104,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmDesc g)
             if (n >= g.N) continue;
             float v = acc[i][jn];
             if (g.bias) v += g.bias[n];
-            g.C[(size_t)m * g.N + n] = v;
+            if (SLSTM_IN((size_t)m * g.N + n, (long long)g.M * g.N)) g.C[(size_t)m * g.N + n] = v;
         }
     }
 }

@@ -32,6 +32,7 @@
 // product per map and lane instead of a 4x4 matrix-vector product.
 #pragma once
 
+#include "checked.cuh"
 #include "common.cuh"
 
 namespace slstm {
@@ -44,6 +45,7 @@ struct CarryArgs {
     unsigned epoch;               // nonzero, unique per launch since the tags were cleared
     unsigned long long wait_ns;   // bound of one wait
     int n_groups;                 // feature groups (tiles per chunk)
+    int n_tiles;                  // tiles of the launch (extent of the per-tile words; checked build)
 };
 
 SLSTM_DEVINL unsigned long long ld_relaxed_u64(const unsigned long long *p)
@@ -67,6 +69,11 @@ SLSTM_DEVINL unsigned long long inc_word(unsigned epoch, float v)
 // if published in this launch.
 SLSTM_DEVINL bool read_inc_words(const CarryArgs &ca, unsigned tq, int lane, float v[4])
 {
+    if (!SLSTM_IN(tq, ca.n_tiles)) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = 0.0f;
+        return false;
+    }
     const unsigned long long *src = ca.incw + (size_t)tq * 4 * 32 + lane;
     bool ok = true;
 #pragma unroll
@@ -121,7 +128,7 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
         if ((whead >> w) & 1u) tile = x;
         else aff_compose(x, tile, tile);
     }
-    if (!withhold) {
+    if (!withhold && SLSTM_IN(ticket, ca.n_tiles)) {
         float *dst = ca.agg + (size_t)ticket * 20 * 32;
 #pragma unroll
         for (int e = 0; e < 16; ++e) dst[e * 32 + lane] = tile.a[e];
@@ -146,7 +153,7 @@ SLSTM_DEVINL void tile_lookback(const CarryArgs &ca, LoadMap load, unsigned tick
             aff_apply(M, v, carry);
             return;
         }
-        const unsigned f = ld_acquire(ca.flags + tq);
+        const unsigned f = SLSTM_IN(tq, ca.n_tiles) ? ld_acquire(ca.flags + tq) : 0u;
         if ((f >> 2) == ca.epoch && (f & FLAG_AGG)) {
             Aff x;
             const float *src = ca.agg + (size_t)tq * 20 * 32;
@@ -201,7 +208,7 @@ SLSTM_DEVINL void carry_serial(const CarryArgs &ca, LoadMap load, PutCarry put, 
         }
         if (w + 1 < NW) x = xn;
     }
-    if (!withhold) {
+    if (!withhold && SLSTM_IN(ticket, ca.n_tiles)) {
         unsigned long long *dst = ca.incw + (size_t)ticket * 4 * 32 + lane;
 #pragma unroll
         for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(ca.epoch, v[e]));

@@ -32,6 +32,7 @@
 
 #include <type_traits>
 
+#define SLSTM_FILE_ID 1
 #include "launchers.h"
 #include "lookback.cuh"
 #include "stop_rule.cuh"
@@ -86,9 +87,17 @@ struct Args {
     int resid_raw;      // stopping test on max|F| (else on the scaled residual)
     int exact_hist;     // every iteration evaluates its whole residual (else a failed test ends that work)
     int guess_tested;   // the first iteration records the residual of the guess
+    int check_plant;    // checked build: one bounds check made to fail on purpose (a self-test)
     float tol;
+    long long n_s0;     // elements of s0 (and of s0h)
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
+
+// Element counts of the buffers that Args names, for the guards of the
+// checked build.
+[[maybe_unused]] SLSTM_DEVINL long long ext_ps(const Args &a) { return (long long)a.B * a.T * 4 * a.d; }
+[[maybe_unused]] SLSTM_DEVINL long long ext_tiles(const Args &a) { return (long long)a.n_tiles * 128; }
+#define SLSTM_RANGE(p, base, n, cnt) (SLSTM_PIN(p, base, n) && SLSTM_PIN((p) + (cnt) - 1, base, n))
 
 // A ticket decoded once (by thread 0) for the whole CTA.
 struct TileInfo {
@@ -144,8 +153,10 @@ SLSTM_DEVINL void issue_tile_load(const Args &a, const NewtonMaps &m, Smem &sm, 
     tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, row, ti.b);
     if (with_s) tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, row, ti.b);
 #pragma unroll
-    for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
-    if (bnd)
+    for (int g = 0; g < 4; ++g)
+        if (SLSTM_RANGE(a.R + (size_t)g * a.d + ti.j0, a.R, 4LL * a.d, rbytes / 4))
+            bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    if (bnd && SLSTM_RANGE(a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32, a.bnd_in, ext_tiles(a), 128))
         bulk_load(&sm.bnd[st][0][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32,
                   (uint32_t)sizeof(sm.bnd[0]), &sm.bar[st]);
 }
@@ -169,8 +180,11 @@ SLSTM_DEVINL void issue_tile_load_part(const Args &a, const NewtonMaps &m, Smem 
         if (with_s) tma_load_3d(&sm.S[st][0][0][0], &m.S, &sm.bar[st], ti.j0, row, ti.b);
     } else if (part == 2) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
-    } else if (bnd) {
+        for (int g = 0; g < 4; ++g)
+            if (SLSTM_RANGE(a.R + (size_t)g * a.d + ti.j0, a.R, 4LL * a.d, rbytes / 4))
+                bulk_load(&sm.R[st][g][0], a.R + (size_t)g * a.d + ti.j0, rbytes, &sm.bar[st]);
+    } else if (bnd && SLSTM_RANGE(a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32, a.bnd_in,
+                                  ext_tiles(a), 128)) {
         bulk_load(&sm.bnd[st][0][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32,
                   (uint32_t)sizeof(sm.bnd[0]), &sm.bar[st]);
     }
@@ -208,9 +222,11 @@ SLSTM_DEVINL void decode_tile(const Args &a, unsigned ticket, TileInfo &ti)
 // Packed sequences: the initial state of the sequence that starts at step t.
 SLSTM_DEVINL void head_state(const Args &a, int t, size_t jj, bool jv, float s[4])
 {
-    const size_t k = (size_t)a.vseq[t];
+    const size_t k = SLSTM_IN(t, a.T) ? (size_t)a.vseq[t] : 0;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) s[e] = (a.s0 && jv) ? __ldg(a.s0 + (k * 4 + e) * (size_t)a.d + jj) : 0.0f;
+    for (int e = 0; e < 4; ++e)
+        s[e] = (a.s0 && jv && SLSTM_IN((k * 4 + e) * (size_t)a.d + jj, a.n_s0))
+                   ? __ldg(a.s0 + (k * 4 + e) * (size_t)a.d + jj) : 0.0f;
 }
 
 // Per-thread part of the copy offsets (see prefetch_tile).
@@ -241,7 +257,7 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo 
 #pragma unroll
         for (int r = 0; r < L; ++r) {
             const int step = r * NW + w;
-            const int bytes = (t0 + step < a.T) ? fbytes : 0;
+            const int bytes = (t0 + step < a.T && SLSTM_RANGE(p + r * stepw, a.P, ext_ps(a), fbytes / 4)) ? fbytes : 0;
             cp_async16(&sm.P[st][step][slot][4 * c], bytes ? p + r * stepw : a.P, bytes);
             if (with_s) cp_async16(&sm.S[st][step][slot][4 * c], bytes ? s + r * stepw : a.S, bytes);
         }
@@ -255,7 +271,7 @@ SLSTM_DEVINL void prefetch_tile(const Args &a, Smem &sm, int st, const TileInfo 
         for (int r = 0; r < 4 * L; ++r) {
             const int rs = r * NW + w;
             const int step = rs >> 2, slot = rs & 3;
-            const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+            const int bytes = (fj && t0 + step < a.T && SLSTM_PIN(p + r * roww, a.P, ext_ps(a))) ? 4 : 0;
             cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * roww : a.P, bytes);
             if (with_s) cp_async4(&sm.S[st][step][slot][jl], bytes ? s + r * roww : a.S, bytes);
         }
@@ -370,7 +386,8 @@ SLSTM_DEVINL void guess_issue_load(const Args &a, const NewtonMaps &m, GuessSmem
     tma_load_3d(&sm.P[st][0][0][0], &m.P, &sm.bar[st], ti.j0, ti.chunk * TT * 4, ti.b);
     if (SWEEP) {
         tma_load_4d(&sm.Hs[st][0][0], &m.H, &sm.bar[st], ti.j0, 3, ti.chunk * TT, ti.b);
-        if (bnd)
+        if (bnd && SLSTM_RANGE(a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32 + 3 * 32, a.bnd_in,
+                               ext_tiles(a), 32))
             bulk_load(&sm.hb[st][0], a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32 + 3 * 32, 128u,
                       &sm.bar[st]);
     }
@@ -391,7 +408,7 @@ SLSTM_DEVINL void guess_prefetch(const Args &a, GuessSmem &sm, int st, const Til
     for (int r = 0; r < 4 * L; ++r) {
         const int rs = r * NW + w;
         const int step = rs >> 2, slot = rs & 3;
-        const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+        const int bytes = (fj && t0 + step < a.T && SLSTM_PIN(p + r * roww, a.P, ext_ps(a))) ? 4 : 0;
         cp_async4(&sm.P[st][step][slot][jl], bytes ? p + r * roww : a.P, bytes);
     }
     if (SWEEP) {
@@ -400,12 +417,12 @@ SLSTM_DEVINL void guess_prefetch(const Args &a, GuessSmem &sm, int st, const Til
 #pragma unroll
         for (int r = 0; r < L; ++r) {
             const int step = r * NW + w;
-            const int bytes = (fj && t0 + step < a.T) ? 4 : 0;
+            const int bytes = (fj && t0 + step < a.T && SLSTM_PIN(hs + (size_t)step * 4 * a.d, a.S, ext_ps(a))) ? 4 : 0;
             cp_async4(&sm.Hs[st][step][jl], bytes ? hs + (size_t)step * 4 * a.d : a.S, bytes);
         }
         if (w == 0) {
-            const bool bnd = ti.chunk > 0;
             const float *src = a.bnd_in + (size_t)(ti.ticket - (unsigned)a.n_groups) * 4 * 32 + 3 * 32 + jl;
+            const bool bnd = ti.chunk > 0 && SLSTM_PIN(src, a.bnd_in, ext_tiles(a));
             cp_async4(&sm.hb[st][jl], bnd ? src : a.bnd_in, bnd ? 4 : 0);
         }
     }
@@ -468,7 +485,7 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const GuessChain &gc, const Seg 
                                  int grp, float v[4])
 {
     const int lane = threadIdx.x & 31;
-    {
+    if (SLSTM_IN(ticket, a.n_tiles)) {
         float *dst = gc.runs + (size_t)ticket * 160 + lane;
         dst[0] = tile.A;
         dst[32] = tile.mu;
@@ -484,7 +501,7 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const GuessChain &gc, const Seg 
     int q = chunk - 1;
     const uint64_t t0 = globaltimer_ns();
     unsigned polls = 0;
-    const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+    const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups, a.n_tiles};
     for (;;) {
         const unsigned tq = (unsigned)q * (unsigned)a.n_groups + (unsigned)grp;
         float w[4];
@@ -496,7 +513,7 @@ SLSTM_DEVINL void guess_lookback(const Args &a, const GuessChain &gc, const Seg 
             }
             return;
         }
-        const unsigned f = ld_acquire(gc.flags + tq);
+        const unsigned f = SLSTM_IN(tq, a.n_tiles) ? ld_acquire(gc.flags + tq) : 0u;
         if ((f >> 2) == a.epoch && (f & FLAG_AGG)) {
             const float *src = gc.runs + (size_t)tq * 160 + lane;
             Seg x;
@@ -614,7 +631,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
         const int t_seg = chunk * TT + warp * L;
 
         float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f;
-        if (ANY_SWEEP && jv) {
+        if (ANY_SWEEP && jv && SLSTM_IN(3 * d + jj, 4 * d)) {
             rz = __ldg(a.R + jj);
             ri = __ldg(a.R + d + jj);
             rf = __ldg(a.R + 2 * d + jj);
@@ -646,7 +663,8 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                 if (stage == 0) {
                     if (warp > 0) hp = sm.Hs[st][warp * L - 1][lane];
                     else if (chunk > 0) hp = sm.hb[st][lane];
-                    else if (!VARLEN && a.s0h && jv) hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
+                    else if (!VARLEN && a.s0h && jv && SLSTM_IN(((size_t)ti.b * 4 + 3) * d + jj, a.n_s0))
+                        hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
                 } else {
                     hp = warp > 0 ? sm.hlast[warp - 1][lane] : sm.cin[3][lane];
                 }
@@ -658,7 +676,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
             const int fc = 2 * warp + (lane >> 4);
             const bool carry_lane = (lane & 15) == 15;
             unsigned long long pw[4] = {0ull, 0ull, 0ull, 0ull};
-            if (carry_lane && chunk > 0) {
+            if (carry_lane && chunk > 0 && SLSTM_IN(ticket - G, a.n_tiles)) {
                 const unsigned long long *src = gc.incw + (size_t)(ticket - G) * 4 * 32 + fc;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) pw[e] = ld_relaxed_u64(src + e * 32);
@@ -738,7 +756,8 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                 if (carry_lane) {
                     float v[4] = {0.f, 0.f, 0.f, 0.f};
                     if (chunk == 0) {
-                        if (!VARLEN && a.s0 && ti.j0 + f < a.d) {
+                        if (!VARLEN && a.s0 && ti.j0 + f < a.d &&
+                            SLSTM_IN(((size_t)ti.b * 4 + 3) * d + ti.j0 + f, a.n_s0)) {
 #pragma unroll
                             for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + ti.j0 + f);
                         }
@@ -757,7 +776,7 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
             static_assert(NW == 16, "the carry lanes are the last of 16 run lanes");
             if (__syncthreads_and(ok)) {
                 // every feature found its predecessor's state: publish
-                if (carry_lane) {
+                if (carry_lane && SLSTM_IN(ticket, a.n_tiles)) {
                     unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + fc;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vo[e]));
@@ -770,12 +789,12 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                     Seg tile;
                     seg_load(sm, NW - 1, lane, tile, whead != 0u);
                     if (chunk == 0) {
-                        if (!VARLEN && a.s0 && jv) {
+                        if (!VARLEN && a.s0 && jv && SLSTM_IN(((size_t)ti.b * 4 + 3) * d + jj, a.n_s0)) {
 #pragma unroll
                             for (int e = 0; e < 4; ++e) v[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
                         }
                     } else {
-                        const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                        const CarryArgs ca{gc.flags, nullptr, gc.incw, a.error, a.epoch, a.wait_ns, a.n_groups, a.n_tiles};
                         const bool got = read_inc_words(ca, ticket - G, lane, v);
                         if (!__all_sync(0xffffffffu, got))
                             guess_lookback(a, gc, tile, ticket, chunk, (int)(ticket - (unsigned)chunk * G), v);
@@ -785,8 +804,10 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                     float vt[4];
                     seg_enter(tile, v, vt);
                     unsigned long long *dst = gc.incw + (size_t)ticket * 4 * 32 + lane;
+                    if (SLSTM_IN(ticket, a.n_tiles)) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vt[e]));
+                        for (int e = 0; e < 4; ++e) st_relaxed_u64(dst + e * 32, inc_word(a.epoch, vt[e]));
+                    }
                 }
                 __syncthreads();
             }
@@ -828,7 +849,8 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                     } else {
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            if (wr) srow[(size_t)i * 4 * d + e * d] = sv[e];
+                            if (wr && SLSTM_PIN(srow + (size_t)i * 4 * d + e * d, a.S, ext_ps(a)))
+                                srow[(size_t)i * 4 * d + e * d] = sv[e];
                     }
                 }
             }
@@ -850,7 +872,8 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
         if (warp == NW - 1 && t_seg + L - 1 < T) {
             float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = sv[e];
+            for (int e = 0; e < 4; ++e)
+                if (SLSTM_PIN(dst + e * 32 + lane, a.bnd_out, ext_tiles(a))) dst[e * 32 + lane] = sv[e];
         }
         if (threadIdx.x == 0) decode_tile(a, after, sm.info[rn == 2 ? 0 : rn + 1]);
         __syncthreads();   // this stage is free for the loads of the tile after next
@@ -899,8 +922,9 @@ __global__ void gather_boundaries(Args a)
     const int j = (int)(grp - b * (unsigned)a.groups_per_row) * 32 + lane;
     const long long t = (long long)chunk * TT + TT - 1;
     float v = 0.0f;
-    if (t < a.T && j < a.d) v = a.S[(((size_t)b * a.T + (size_t)t) * 4 + e) * (size_t)a.d + j];
-    a.bnd_out[idx] = v;
+    const size_t src = (((size_t)b * a.T + (size_t)t) * 4 + e) * (size_t)a.d + j;
+    if (t < a.T && j < a.d && SLSTM_IN(src, ext_ps(a))) v = a.S[src];
+    if (SLSTM_IN(idx, ext_tiles(a))) a.bnd_out[idx] = v;
 }
 
 // TMA: tiles move by TMA (loads by TMA_THREAD into an mbarrier-guarded
@@ -1007,7 +1031,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                 rf = sm.R[st][2][lane];
                 ro = sm.R[st][3][lane];
             }
-        } else if (jv) {
+        } else if (jv && SLSTM_IN(3 * d + jj, 4 * d)) {
             rz = __ldg(a.R + jj);
             ri = __ldg(a.R + d + jj);
             rf = __ldg(a.R + 2 * d + jj);
@@ -1016,7 +1040,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // old state just before this warp's segment
         float sp[4] = {0.f, 0.f, 0.f, 0.f};
         if (t_seg == 0) {
-            if (!VARLEN && a.s0 && jv) {
+            if (!VARLEN && a.s0 && jv && SLSTM_IN(((size_t)ti.b * 4 + 3) * d + jj, a.n_s0)) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sp[e] = __ldg(a.s0 + ((size_t)ti.b * 4 + e) * d + jj);
             }
@@ -1027,8 +1051,10 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                     for (int e = 0; e < 4; ++e) sp[e] = sm.bnd[st][e][lane];
                 } else {
                     const float *src = a.bnd_in + (size_t)(ticket - G) * 4 * 32;
+                    if (SLSTM_RANGE(src, a.bnd_in, ext_tiles(a), 128)) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
+                        for (int e = 0; e < 4; ++e) sp[e] = src[e * 32 + lane];
+                    }
                 }
             } else {
 #pragma unroll
@@ -1039,7 +1065,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // looks at the predecessor's inclusive prefix (chain lanes): before
         // and halfway through walk A, so that both loads' latency is hidden;
         // the second is read only when the first found nothing
-        const bool look = MODE == MODE_FUSED && chain_warp && chunk > 0;
+        const bool look = MODE == MODE_FUSED && chain_warp && chunk > 0 && SLSTM_IN(ticket - G, a.n_tiles);
         const unsigned long long *predw = a.incw + chain_word(ticket - G, warp, lane);
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
@@ -1127,18 +1153,21 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                 Aff x;
                 maps_load(sm.maps.m, NW - 1, lane, x);
                 float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
+                if (SLSTM_IN(ticket, a.n_tiles)) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
+                    for (int e = 0; e < 16; ++e) dst[e * 32] = x.a[e];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
-                if (lane == 0) a.flags[ticket] = whead ? 1u : 0u;
+                    for (int e = 0; e < 4; ++e) dst[(16 + e) * 32] = x.b[e];
+                    if (lane == 0) a.flags[ticket] = whead ? 1u : 0u;
+                }
             }
         } else {
 
             // ---- carry ----
             float c = 0.f;   // chunk 0: the iterate before t = 0 is fixed, no correction enters
             bool ok = true;
-            if (MODE == MODE_APPLY && chain_warp) c = a.cin_buf[chain_word(ticket, warp, lane)];
+            if (MODE == MODE_APPLY && chain_warp && SLSTM_IN(chain_word(ticket, warp, lane), ext_tiles(a)))
+                c = a.cin_buf[chain_word(ticket, warp, lane)];
             if (look) {
                 if ((unsigned)(w1 >> 32) == a.epoch) {
                     c = __uint_as_float((unsigned)w1);
@@ -1152,12 +1181,12 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             if (chain_warp) {
                 if (fast) {
                     c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, whead, CHAIN0);
-                    if (MODE == MODE_FUSED && !withhold)
+                    if (MODE == MODE_FUSED && !withhold && SLSTM_IN(chain_word(ticket, warp, lane), ext_tiles(a)))
                         st_relaxed_u64(a.incw + chain_word(ticket, warp, lane), inc_word(a.epoch, c));
                     named_bar_sync(CHAIN_BAR, 4 * 32);
                 } else {
                     if (warp == CHAIN0) {
-                        const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups};
+                        const CarryArgs ca{a.flags, a.agg, a.incw, a.error, a.epoch, a.wait_ns, a.n_groups, a.n_tiles};
                         tile_carry_fallback<NW>(ca, sm.maps.m, sm.maps.cin, ticket, chunk,
                                                 (int)(ticket - (unsigned)chunk * G), withhold, whead);
                     }
@@ -1213,7 +1242,8 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
                     } else {
     #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            if (wr) srow[(size_t)i * 4 * d + e * d] = sn[e];
+                            if (wr && SLSTM_PIN(srow + (size_t)i * 4 * d + e * d, a.S, ext_ps(a)))
+                                srow[(size_t)i * 4 * d + e * d] = sn[e];
                     }
                     if (FULL) {
                         if (VARLEN && ((ti.mask >> sl) & 1ull)) head_state(a, t_seg + i, jj, jv, snp);
@@ -1257,8 +1287,11 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             // state at the tile's last step, for the next launch's successor tile
             if (warp == NW - 1 && t_seg + L - 1 < T) {
                 float *dst = a.bnd_out + (size_t)ticket * 4 * 32;
+                // (a self-test of the checked build can shorten the extent by one)
     #pragma unroll
-                for (int e = 0; e < 4; ++e) dst[e * 32 + lane] = snp[e];
+                for (int e = 0; e < 4; ++e)
+                    if (SLSTM_PIN(dst + e * 32 + lane, a.bnd_out, ext_tiles(a) - a.check_plant))
+                        dst[e * 32 + lane] = snp[e];
             }
             // a failure of the test is announced to the tiles after it (until
             // this CTA has seen the announcement)
@@ -1565,6 +1598,8 @@ cudaError_t prepare(const float *P, const float *R, const float *s0, float *S, c
     // fault injection: the first tile of chunk 1 withholds its publications,
     // so the first tile of chunk 2 has nothing to wait for
     a.fault_ticket = (cfg.debug_fault == 1 && l.n_chunks >= 3) ? l.n_groups : -1;
+    a.check_plant = cfg.debug_fault == 2 ? 1 : 0;
+    a.n_s0 = (long long)(vl ? vl->n_seq : B) * 4 * d;
 
     // control block, aggregate flags and the epoch tags of the inclusive
     // prefixes start cleared on every call
@@ -1674,14 +1709,16 @@ __global__ void __launch_bounds__(NW * 32) cp_tile_run_kernel(Args a)
     const size_t jj = jv ? (size_t)(ti.j0 + lane) : 0;
     const int t_seg = ti.chunk * TT + warp * L;
     float rz = 0.f, ri = 0.f, rf = 0.f, ro = 0.f, hp = 0.f;
-    if (SWEEP && jv) {
+    if (SWEEP && jv && SLSTM_IN(3 * d + jj, 4 * d)) {
         rz = __ldg(a.R + jj);
         ri = __ldg(a.R + d + jj);
         rf = __ldg(a.R + 2 * d + jj);
         ro = __ldg(a.R + 3 * d + jj);
         const int tp = t_seg - 1;
-        if (tp >= 0 && tp < a.T) hp = __ldg(a.S + (((size_t)ti.b * a.T + tp) * 4 + 3) * d + jj);
-        else if (tp < 0 && a.s0h) hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
+        if (tp >= 0 && tp < a.T && SLSTM_IN((((size_t)ti.b * a.T + tp) * 4 + 3) * d + jj, ext_ps(a)))
+            hp = __ldg(a.S + (((size_t)ti.b * a.T + tp) * 4 + 3) * d + jj);
+        else if (tp < 0 && a.s0h && SLSTM_IN(((size_t)ti.b * 4 + 3) * d + jj, a.n_s0))
+            hp = __ldg(a.s0h + ((size_t)ti.b * 4 + 3) * d + jj);
     }
     Seg run;
     int n = 0;
@@ -1692,13 +1729,13 @@ __global__ void __launch_bounds__(NW * 32) cp_tile_run_kernel(Args a)
         const size_t row = ((size_t)ti.b * a.T + t) * 4;
         float p[4];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) p[g] = jv ? __ldg(a.P + (row + g) * d + jj) : 0.0f;
+        for (int g = 0; g < 4; ++g) p[g] = (jv && SLSTM_IN((row + g) * d + jj, ext_ps(a))) ? __ldg(a.P + (row + g) * d + jj) : 0.0f;
         if (SWEEP) {
             p[0] = fmaf(rz, hp, p[0]);
             p[1] = fmaf(ri, hp, p[1]);
             p[2] = fmaf(rf, hp, p[2]);
             p[3] = fmaf(ro, hp, p[3]);
-            hp = jv ? __ldg(a.S + (row + 3) * d + jj) : 0.0f;
+            hp = (jv && SLSTM_IN((row + 3) * d + jj, ext_ps(a))) ? __ldg(a.S + (row + 3) * d + jj) : 0.0f;
         }
         float z, lf, o;
         guess_gates<FORGET>(p[0], p[2], p[3], z, lf, o);
@@ -1737,11 +1774,13 @@ __global__ void __launch_bounds__(NW * 32) cp_tile_run_kernel(Args a)
             else seg_compose(x, tile, tile);
         }
         float *dst = a.agg + (size_t)ticket * 20 * 32 + lane;
-        dst[0] = tile.A;
-        dst[32] = tile.mu;
-        dst[64] = tile.u;
-        dst[96] = tile.v;
-        dst[128] = tile.o;
+        if (SLSTM_IN(ticket, a.n_tiles)) {
+            dst[0] = tile.A;
+            dst[32] = tile.mu;
+            dst[64] = tile.u;
+            dst[96] = tile.v;
+            dst[128] = tile.o;
+        }
     }
 }
 

@@ -16,6 +16,7 @@
 //            it through the warp maps, one (feature, slot) pair per lane,
 //            releasing each other warp as soon as its carry is stored;
 //   walk B   each thread applies its maps from its carry and writes y.
+#define SLSTM_FILE_ID 3
 #include "launchers.h"
 #include "lookback.cuh"
 
@@ -37,6 +38,7 @@ struct ScanArgs {
     CarryArgs ca;
     int T, d, groups_per_row, n_tiles, vec16;
     int fault_ticket;   // this tile publishes nothing (host-requested fault injection), or -1
+    long long n_b;      // elements of b and y (A has 4 n_b)
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
 
@@ -73,7 +75,10 @@ SLSTM_DEVINL void scan_prefetch(const ScanArgs &a, ScanSmem &sm, int st, unsigne
         const int c = threadIdx.x & 7, q = threadIdx.x >> 3;
         const int jj = j0 + 4 * c;
         const int t = step_time<REVERSE>(T, chunk, q);
-        const int bytes = (jj < a.d && t >= 0 && t < T) ? 4 * min(4, a.d - jj) : 0;
+        const int nb = 4 * min(4, a.d - jj);
+        const int bytes = (jj < a.d && t >= 0 && t < T &&
+                           SLSTM_IN((row0 + t) * 16 * d + jj + 15 * d + nb / 4 - 1, 4 * a.n_b) &&
+                           SLSTM_IN((row0 + t) * 4 * d + jj + 3 * d + nb / 4 - 1, a.n_b)) ? nb : 0;
         const float *pa = bytes ? a.A + (row0 + t) * 16 * d + jj : a.A;
         const float *pb = bytes ? a.b + (row0 + t) * 4 * d + jj : a.b;
 #pragma unroll
@@ -86,7 +91,8 @@ SLSTM_DEVINL void scan_prefetch(const ScanArgs &a, ScanSmem &sm, int st, unsigne
         const bool fj = j0 + jl < a.d;
         for (int q = w; q < TT; q += NW) {
             const int t = step_time<REVERSE>(T, chunk, q);
-            const int bytes = (fj && t >= 0 && t < T) ? 4 : 0;
+            const int bytes = (fj && t >= 0 && t < T && SLSTM_IN((row0 + t) * 16 * d + j0 + jl + 15 * d, 4 * a.n_b) &&
+                               SLSTM_IN((row0 + t) * 4 * d + j0 + jl + 3 * d, a.n_b)) ? 4 : 0;
             const float *pa = bytes ? a.A + (row0 + t) * 16 * d + j0 + jl : a.A;
             const float *pb = bytes ? a.b + (row0 + t) * 4 * d + j0 + jl : a.b;
 #pragma unroll
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
 
         // the predecessor's inclusive prefix (chain lanes), looked at before
         // and halfway through walk A
-        const bool look = chain_warp && chunk > 0;
+        const bool look = chain_warp && chunk > 0 && SLSTM_IN(ticket - (unsigned)G, a.n_tiles);
         const unsigned long long *predw = a.ca.incw + chain_word(ticket - (unsigned)G, warp, lane);
         unsigned long long w1 = 0ull, w2 = 0ull;
         if (look) w1 = ld_relaxed_u64(predw);
@@ -186,7 +192,8 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
         if (chain_warp && chunk == 0 && a.y0) {
             // chunk 0: y0 enters (chain lane (row, feature))
             const int jf = (grp - bb * a.groups_per_row) * 32 + chain_feature(warp, lane);
-            if (jf < a.d) c = __ldg(a.y0 + ((size_t)bb * 4 + chain_row(lane)) * d + jf);
+            if (jf < a.d && SLSTM_IN(((size_t)bb * 4 + chain_row(lane)) * d + jf, a.n_b / T))
+                c = __ldg(a.y0 + ((size_t)bb * 4 + chain_row(lane)) * d + jf);
         }
         if (look) {
             if ((unsigned)(w1 >> 32) == a.ca.epoch) {
@@ -201,7 +208,8 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
         if (chain_warp) {
             if (fast) {
                 c = carry_chain4<NW>(sm.maps.m, sm.maps.cin, c, warp, lane, 0u, CHAIN0);
-                if (!withhold) st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
+                if (!withhold && SLSTM_IN(chain_word(ticket, warp, lane), (long long)a.n_tiles * 128))
+                    st_relaxed_u64(a.ca.incw + chain_word(ticket, warp, lane), inc_word(a.ca.epoch, c));
                 named_bar_sync(CHAIN_BAR, 4 * 32);
             } else {
                 if (warp == CHAIN0)
@@ -227,7 +235,7 @@ __global__ void __launch_bounds__(NW * 32, 1) scan_kernel(ScanArgs a)
                 float *py = a.y + (row0 + t) * 4 * d + jj;
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    if (jv) py[e * d] = v[e];
+                    if (jv && SLSTM_PIN(py + e * d, a.y, a.n_b)) py[e * d] = v[e];
             }
         }
         if (threadIdx.x == 0) sm.tick[0] = after;
@@ -319,6 +327,8 @@ cudaError_t scan_block4_launch(const float *A, const float *b, const float *y0, 
     a.fault_ticket = (debug_withhold && l.n_chunks >= 3) ? l.n_groups : -1;
     a.ca.wait_ns = a.fault_ticket >= 0 ? 20000000ull : 2000000000ull;
     a.ca.n_groups = l.n_groups;
+    a.ca.n_tiles = l.n_tiles;
+    a.n_b = (long long)B * T * 4 * d;
     a.T = T;
     a.d = d;
     a.groups_per_row = l.groups_per_row;

@@ -2,6 +2,8 @@
 // thread per (batch row, feature) walking time ("sLSTM in this library",
 // section "API notes": evaluation runs the sequential step; at T = 1 it is
 // one recurrent-step launch while W_x stays a GEMM).
+#define SLSTM_FILE_ID 4
+#include "checked.cuh"
 #include "common.cuh"
 #include "launchers.h"
 
@@ -18,9 +20,13 @@ __global__ void __launch_bounds__(128) sequential_kernel(const float *__restrict
     const int b = blockIdx.y;
     if (j >= d) return;
     const size_t dd = (size_t)d;
+    // extents (checked build): P and S (B, T, 4, d), s0 (B, 4, d), R (4, d)
+    [[maybe_unused]] const long long n_ps = (long long)gridDim.y * T * 4 * d;
+    [[maybe_unused]] const long long n_s0 = (long long)gridDim.y * 4 * d;
+    if (!SLSTM_IN(3 * dd + j, 4LL * d)) return;
     const float rz = R[j], ri = R[dd + j], rf = R[2 * dd + j], ro = R[3 * dd + j];
     float c = 0.f, n = 0.f, m = 0.f, h = 0.f;
-    if (s0) {
+    if (s0 && SLSTM_IN((size_t)b * 4 * dd + 3 * dd + j, n_s0)) {
         const float *p = s0 + (size_t)b * 4 * dd + j;
         c = p[0];
         n = p[dd];
@@ -30,10 +36,16 @@ __global__ void __launch_bounds__(128) sequential_kernel(const float *__restrict
     const float *pp = P + (size_t)b * T * 4 * dd + j;
     float *ps = S + (size_t)b * T * 4 * dd + j;
     // one step ahead prefetch of P keeps a load in flight while the step computes
-    float nz = __ldg(pp), ni = __ldg(pp + dd), nf = __ldg(pp + 2 * dd), no = __ldg(pp + 3 * dd);
+    float nz = 0.f, ni = 0.f, nf = 0.f, no = 0.f;
+    if (SLSTM_PIN(pp + 3 * dd, P, n_ps)) {
+        nz = __ldg(pp);
+        ni = __ldg(pp + dd);
+        nf = __ldg(pp + 2 * dd);
+        no = __ldg(pp + 3 * dd);
+    }
     for (int t = 0; t < T; ++t) {
         const float pz = nz, pi = ni, pf = nf, po = no;
-        if (t + 1 < T) {
+        if (t + 1 < T && SLSTM_PIN(pp + (size_t)(t + 1) * 4 * dd + 3 * dd, P, n_ps)) {
             const float *q = pp + (size_t)(t + 1) * 4 * dd;
             nz = __ldg(q);
             ni = __ldg(q + dd);
@@ -47,6 +59,7 @@ __global__ void __launch_bounds__(128) sequential_kernel(const float *__restrict
         m = o.m;
         h = o.h;
         float *q = ps + (size_t)t * 4 * dd;
+        if (!SLSTM_PIN(q + 3 * dd, S, n_ps)) continue;
         q[0] = c;
         q[dd] = n;
         q[2 * dd] = m;

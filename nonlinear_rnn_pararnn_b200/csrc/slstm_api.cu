@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include "block.h"
+#include "checked.cuh"
 #include "launchers.h"
 
 using namespace slstm;
@@ -53,6 +54,7 @@ bool config_ok(const slstm_newton_config &c)
     if (c.residual_mode != SLSTM_RESIDUAL_SCALED && c.residual_mode != SLSTM_RESIDUAL_RAW) return false;
     if (c.n_events < 0 || (c.n_events > 0 && c.events == nullptr)) return false;
     if (c.history != SLSTM_HISTORY_BOUND && c.history != SLSTM_HISTORY_EXACT) return false;
+    if (c.debug_fault < 0 || c.debug_fault > 2) return false;
     return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
 }
 
@@ -77,7 +79,70 @@ constexpr long long kBlockBwdMaxRows = 65535LL * 256;
 
 }  // namespace
 
+namespace slstm {
+
+namespace {
+struct CheckUnit {
+    CheckReader read;
+    CheckClearer clear;
+};
+CheckUnit g_units[32];
+int g_n_units = 0;
+}  // namespace
+
+int check_register(CheckReader r, CheckClearer c)
+{
+    if (g_n_units < 32) g_units[g_n_units++] = CheckUnit{r, c};
+    return g_n_units;
+}
+
+}  // namespace slstm
+
 extern "C" {
+
+int slstm_check_enabled(void)
+{
+#ifdef SLSTM_CHECKED
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int slstm_check_status(long long *out)
+{
+    if (out == nullptr) return SLSTM_ERR_INVALID_ARG;
+    for (int i = 0; i < 4; ++i) out[i] = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SLSTM_ERR_CUDA;
+    for (int u = 0; u < g_n_units; ++u) {
+        CheckRecord r;
+        if (g_units[u].read(&r) != cudaSuccess) return SLSTM_ERR_CUDA;
+        if (r.count != 0ull && out[0] == 0) {
+            out[1] = r.site;
+            out[2] = r.index;
+            out[3] = r.extent;
+        }
+        out[0] += (long long)r.count;
+    }
+    return SLSTM_OK;
+}
+
+int slstm_check_clear(void)
+{
+    if (cudaDeviceSynchronize() != cudaSuccess) return SLSTM_ERR_CUDA;
+    for (int u = 0; u < g_n_units; ++u)
+        if (g_units[u].clear() != cudaSuccess) return SLSTM_ERR_CUDA;
+    return SLSTM_OK;
+}
+
+const char *slstm_check_site_file(int file_id)
+{
+    static const char *const names[] = {nullptr,         "newton.cu", "backward.cu", "scan.cu",  "sequential.cu",
+                                        "varlen.cu",     "decode.cu", "head.cu",     "block.cu", "gemm_simt.cu",
+                                        "scan_noalloc.cu"};
+    if (file_id < 1 || file_id >= (int)(sizeof(names) / sizeof(names[0]))) return nullptr;
+    return names[file_id];
+}
 
 const char *slstm_status_string(int status)
 {

@@ -5,6 +5,8 @@
 // steps, the tile height of the Newton and adjoint kernels) and records the
 // sequence index there.  Offsets are clamped into [0, total_T], so malformed
 // input can never lead to an out-of-range access; it is reported instead.
+#define SLSTM_FILE_ID 5
+#include "checked.cuh"
 #include "launchers.h"
 
 namespace slstm {
@@ -16,7 +18,7 @@ __global__ void varlen_table_kernel(const int *__restrict__ cu, int n_seq, int t
                                     unsigned *err, slstm_newton_stats *stats, unsigned *done)
 {
     const int k = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= n_seq) return;
+    if (k >= n_seq || !SLSTM_IN(k + 1, n_seq + 1)) return;
     int a = cu[k], b = cu[k + 1];
     const bool bad = a < 0 || b < a || b > total_T || (k == 0 && a != 0) || (k == n_seq - 1 && b != total_T);
     if (bad) {
@@ -26,7 +28,7 @@ __global__ void varlen_table_kernel(const int *__restrict__ cu, int n_seq, int t
     }
     a = min(max(a, 0), total_T);
     b = min(max(b, 0), total_T);
-    if (b > a) {
+    if (b > a && SLSTM_IN(a >> 5, (total_T + 31) / 32) && SLSTM_IN(a, total_T)) {
         atomicOr(&mask[a >> 5], 1u << (a & 31));
         seq[a] = k;
     }

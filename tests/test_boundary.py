@@ -70,6 +70,16 @@ def _cfg(**kw):
     return _lib.NewtonConfig(**base)
 
 
+def test_checked_build_entry_points_in_the_normal_library():
+    """The normal library exports the bounds-check calls too: checks off,
+    nothing recorded, a null output rejected (no device access)."""
+    lib = _lib.load()
+    assert lib.slstm_check_enabled() == 0
+    assert lib.slstm_check_status(None) == _lib.SLSTM_ERR_INVALID_ARG
+    assert lib.slstm_check_site_file(1) == b"newton.cu"
+    assert lib.slstm_check_site_file(0) is None and lib.slstm_check_site_file(99) is None
+
+
 def test_newton_forward_rejects_bad_arguments():
     lib = _lib.load()
     E = _lib.SLSTM_ERR_INVALID_ARG
@@ -101,6 +111,8 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(cfg=_cfg(max_iters=0, init=1)) == E      # only the decoupled guess allows 0 iterations
     assert call(cfg=_cfg(n_events=-1)) == E
     assert call(cfg=_cfg(n_events=3)) == E               # timing events announced, array missing
+    assert call(cfg=_cfg(history=2)) == E
+    assert call(cfg=_cfg(debug_fault=3)) == E
     assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
     assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
     assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E
