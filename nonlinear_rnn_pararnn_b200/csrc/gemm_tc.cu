@@ -12,9 +12,9 @@
 //                      of two 256-column fp32 accumulators in TMEM, so that a
 //                      tile's epilogue overlaps the next tile's main loop;
 //   warps 2-5          epilogue: tcgen05.ld of their TMEM lane quarter, + bias,
-//                      32-column slices staged in shared memory and written
-//                      by TMA stores (plain stores when C rows are not
-//                      16-byte aligned).
+//                      16-column slices staged in shared memory (four
+//                      buffers) and written by TMA stores (plain stores when C
+//                      rows are not 16-byte aligned).
 // No multicast and no clusters.  Every mbarrier wait is bounded in time; on
 // expiry the CTA records an error, waits (bounded) for the loads and MMAs it
 // issued, frees its TMEM and returns.
@@ -33,9 +33,11 @@ constexpr uint32_t A_STAGE = BM * BK * 2;   // 16 KB
 constexpr uint32_t B_STAGE = BN * BK * 2;   // 32 KB
 constexpr uint32_t STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr uint32_t TMEM_COLS = 2 * BN;      // two accumulators: one tile's epilogue overlaps the next one's MMAs
-constexpr int EPI_COLS = 32;                // columns per epilogue store box (128 bytes of fp32)
-constexpr uint32_t EPI_BYTES = BM * EPI_COLS * 4;   // 16 KB, two of them
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * EPI_BYTES + 1024 + 256;
+constexpr int EPI_COLS = 32;                // columns per TMEM load of the epilogue
+constexpr int STORE_COLS = 16;              // columns per store box (64 bytes of fp32, 64-byte swizzle)
+constexpr uint32_t STORE_BYTES = BM * STORE_COLS * 4;   // 8 KB
+constexpr int STORE_BUFS = 4;               // staging buffers: up to three stores still reading
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BUFS * STORE_BYTES + 1024 + 256;
 constexpr int THREADS = 192;                // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint64_t WAIT_NS = 1000000000ull;   // 1 s bound on any single wait
 
@@ -158,8 +160,8 @@ SLSTM_DEVINL void tmem_ld32(uint32_t taddr, float (&v)[32])
 //                      [256 (i & 1), 256 (i & 1) + 256), handed to the
 //                      epilogue by tcgen05.commit and back by an mbarrier;
 //   warps 2-5          epilogue: TMEM lane quarter (warp & 3), + bias, then
-//                      32-column slices staged in shared memory (128-byte
-//                      swizzle) and written by TMA stores, two staging buffers.
+//                      16-column slices staged in shared memory (64-byte
+//                      swizzle) and written by TMA stores, four staging buffers.
 template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tma2,
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * A_STAGE;
     uint8_t *sE = smem + STAGES * STAGE_BYTES;   // 1024-aligned: the swizzle pattern is address based
-    uint64_t *full = reinterpret_cast<uint64_t *>(sE + 2 * EPI_BYTES);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sE + STORE_BUFS * STORE_BYTES);
     uint64_t *empty = full + STAGES;
     uint64_t *tfull = empty + STAGES;    // [2] accumulator ready
     uint64_t *tempty = tfull + 2;        // [2] accumulator drained (4 epilogue warps)
@@ -373,21 +375,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int i = 0; i < 32; ++i) v[i] += (col0 + i < g.N) ? __ldg(g.bias + col0 + i) : 0.0f;
                 }
                 if (g.tma_out) {
-                    uint8_t *buf_e = sE + (chunk & 1) * EPI_BYTES;
-                    // the store that last read this staging buffer is done with it
-                    if (et == 0) bulk_wait_read_1();
-                    bar_named(1, 128);
-                    // row `row`, 16-byte piece j at piece j ^ (row & 7): the
-                    // tensor map's 128-byte swizzle
+                    // two boxes of 16 columns, each staged in the next of four
+                    // buffers (row `row`, 16-byte piece j at piece j ^ ((row >> 1)
+                    // & 3): the tensor map's 64-byte swizzle) once the store that
+                    // last read that buffer is done with it
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4 *>(buf_e + row * 128 + ((j ^ (row & 7)) << 4)) =
-                            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-                    tma_store_fence();
-                    bar_named(1, 128);
-                    if (et == 0) {
-                        tma_store_3d(&tmc, buf_e, col0, m0, z);
-                        bulk_commit();
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint8_t *buf_e = sE + ((2 * chunk + hf) % STORE_BUFS) * STORE_BYTES;
+                        if (et == 0) bulk_wait_read_3();
+                        bar_named(1, 128);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<float4 *>(buf_e + row * 64 + ((j ^ ((row >> 1) & 3)) << 4)) =
+                                make_float4(v[16 * hf + 4 * j], v[16 * hf + 4 * j + 1], v[16 * hf + 4 * j + 2],
+                                            v[16 * hf + 4 * j + 3]);
+                        tma_store_fence();
+                        bar_named(1, 128);
+                        if (et == 0) {
+                            tma_store_3d(&tmc, buf_e, col0 + STORE_COLS * hf, m0, z);
+                            bulk_commit();
+                        }
                     }
                 } else {
                     const int grow = m0 + row;
@@ -449,10 +456,10 @@ bool make_c_map(CUtensorMap *map, float *C, int M, int N, int splits)
     if (fn == nullptr) return false;
     cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)splits};
     cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
-    cuuint32_t box[3] = {(cuuint32_t)EPI_COLS, (cuuint32_t)BM, 1u};
+    cuuint32_t box[3] = {(cuuint32_t)STORE_COLS, (cuuint32_t)BM, 1u};
     cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, C, dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
