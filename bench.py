@@ -24,8 +24,8 @@ guess launch and the whole solve are reported beside it.
 With no flags the line also carries, measured in the same run on rank 0: the
 long-sequence workload's forward (B=4, T=65536, d=2048: input projection and
 the converged Newton solve, and the fixed K=4 solve) with newton_iter's HBM
-roofline fraction, and the scan_block4 sweep at B=4, d=2048 over
-T = 4096, 16384, 65536.
+roofline fraction, the same solve at T = 4096 and 16384 (newton_sweep), and
+the scan_block4 sweep at B=4, d=2048 over T = 4096, 16384, 65536.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of lanes of the same workload.
@@ -545,6 +545,8 @@ def run_gpu(args, w):
         torch.cuda.empty_cache()
         extra["long_forward"] = long_forward(args, dev, hbm, peak_kind)
         torch.cuda.empty_cache()
+        extra["newton_sweep"] = newton_sweep(args, dev, hbm, peak_kind)
+        torch.cuda.empty_cache()
         extra["scan_block4_sweep"] = scan_sweep(args, dev, hbm, peak_kind)
 
     # kernels launched per step: preact GEMM 1, Newton: the guess + K iteration
@@ -676,6 +678,49 @@ def long_forward(args, dev, hbm, peak_kind):
                                   "solve": {"achieved": gbs, "frac": gbs / hbm, "algorithmic_bytes": nbytes}}}
     del x, Wx, R, bias, s0, P, S, ws_n
     torch.cuda.empty_cache()
+    return out
+
+
+def newton_sweep(args, dev, hbm, peak_kind, T_list=(4096, 16384)):
+    """The long-sequence workload's Newton solve (B=4, d=2048, bf16 x/W_x) at shorter T, to the
+    workload's tolerance from the decoupled guess: iterations, solve time and newton_iter's HBM
+    fraction per T (T = 65536 is the long_forward entry)."""
+    import torch
+    from nonlinear_rnn_pararnn_b200 import _lib, api
+    base = WORKLOADS["slstm_bf16_long_b4_t65536_d2048"]
+    out = []
+    g = guess_launches(args.guess_sweeps)
+    for T in T_list:
+        w = scaled(base, T=T, name=f"{base.name}_T{T}")
+        inp = make_inputs(w, with_dH=False)
+        x, Wx, R, bias, s0 = (inp[k].to(dev) for k in ("x", "Wx", "R", "bias", "s0"))
+        P = api.preact_gemm(x, Wx, bias)
+        del x
+        S = torch.empty_like(P)
+        stats = api.new_stats(dev)
+        ws_n = api.workspace(_lib.SLSTM_OP_NEWTON_FORWARD, w.B, w.T, 0, w.d_h, dev)
+        K = w.max_iters
+        n = 10
+        levs = [[torch.cuda.Event(enable_timing=True) for _ in range(g + K + 1)] for _ in range(n)]
+        for _ in range(args.warmup):
+            api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, tol=w.tol, S=S, stats=stats, ws=ws_n,
+                               guess_sweeps=args.guess_sweeps)
+        torch.cuda.synchronize()
+        for i in range(n):
+            api.newton_forward(P, R, s0, forget=w.forget, max_iters=K, tol=w.tol, S=S, stats=stats, ws=ws_n,
+                               guess_sweeps=args.guess_sweeps, events=levs[i])
+        torch.cuda.synchronize()
+        st = api.read_stats(stats)
+        it = st["iters"]
+        solve_ms = float(np.median([lv[0].elapsed_time(lv[-1]) for lv in levs]))
+        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs for i in range(it)]))
+        gbs = 48.0 * w.elems / (it_ms / 1e3) / 1e9
+        out.append({"workload": w.name, "T": T, "iters": it, "converged": st["converged"],
+                    "solve_ms": solve_ms, "solve_elems_per_s": w.elems / (solve_ms / 1e3),
+                    "newton_iter_ms": it_ms, "newton_iter_achieved_GBs": gbs, "peak": hbm, "peak_kind": peak_kind,
+                    "newton_iter_frac": gbs / hbm, "steps": n})
+        del P, S, ws_n
+        torch.cuda.empty_cache()
     return out
 
 

@@ -51,8 +51,12 @@
  *     bounded waits.  A wait that expires (it should never happen; it means
  *     a tile was not scheduled within the limit) makes the carry it waited
  *     for NaN, so every output that depends on it is NaN instead of silently
- *     wrong, and sets a nonzero error word in the workspace.
- *     slstm_newton_forward also reports it as SLSTM_ERR_TIMEOUT in its stats.
+ *     wrong, and sets a nonzero error word in the workspace: the 32-bit word
+ *     at byte offset 4 for scan_block4 and slstm_newton_backward(_varlen)
+ *     (cleared by every call), the same word of the library's own block for
+ *     scan_block4_noalloc (not readable by the caller; the NaN outputs show
+ *     it).  slstm_newton_forward also reports it as SLSTM_ERR_TIMEOUT in its
+ *     stats.
  *   - Sizes: 1 <= B <= 65535, 1 <= T, 1 <= d_in, d_h, d <= 2^20, B*T < 2^31
  *     and B * ceil(T/32) * ceil(max(d_in, d_h)/32) < 2^31.
  */

@@ -441,6 +441,8 @@ def test_scan_block4_bounded_wait_poisons_outputs(reverse, cuda_device):
                                 ws.numel(), api._stream())
     assert rc == 0
     torch.cuda.synchronize()
+    # the expired wait is reported in the workspace's error word (bytes 4..7)
+    assert ws[4:8].view(torch.int32).item() != 0
     got = y.cpu()
     Al = np.transpose(as_f64(A), (0, 4, 1, 2, 3)).reshape(B * d, T, 4, 4)
     bl = np.transpose(as_f64(b), (0, 3, 1, 2)).reshape(B * d, T, 4)
@@ -453,6 +455,7 @@ def test_scan_block4_bounded_wait_poisons_outputs(reverse, cuda_device):
     assert err < 1e-5, err
     assert np.isfinite(as_f64(got[0, early])).all()
     # a normal call afterwards is unaffected
-    y2 = api.scan_block4(Ad, bd, None, reverse=reverse)
+    y2 = api.scan_block4(Ad, bd, None, reverse=reverse, ws=ws)
     torch.cuda.synchronize()
     assert np.abs(as_f64(y2.cpu()) - ref).max() / (1 + np.abs(ref).max()) < 1e-5
+    assert ws[4:8].view(torch.int32).item() == 0
