@@ -1069,8 +1069,8 @@ def run_block(args, w):
 # iteration that evaluates its whole residual.  The counters describe the kernel sources with this
 # SHA-256; any other build reports traffic null.  Traffic per element does not depend on T (every
 # tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "2a8ded3ac5129afc25e8751a55a999d4e1b76a52310a8571b133d59838643b53",
-                  "guess": 30.9, "sweep": None, "iter": 46.3}
+NEWTON_TRAFFIC = {"sources_sha256": "508a94120148295a0ce844634e0af7a141dc1a2ac4bccf8e358f883df1c4429c",
+                  "guess": 30.9, "sweep": None, "iter": 46.5}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 

@@ -18,6 +18,8 @@
 // zero state (d_in = d_h = D).
 #include <cuda_bf16.h>
 
+#define SLSTM_FILE_ID 8
+#include "checked.cuh"
 #include "common.cuh"
 #include "block.h"
 #include "launchers.h"
@@ -41,6 +43,9 @@ __global__ void __launch_bounds__(NORM_ROWS * 32) block_norm_kernel(const float 
     const int lane = threadIdx.x & 31;
     if (r >= M) return;
     const int n4 = D >> 2;
+    // the row's last element in x, u, z and (RESID) h's slot of S
+    if (!SLSTM_IN((size_t)r * D + 4 * n4 - 1, (long long)M * D)) return;
+    if (RESID && !SLSTM_IN(((size_t)r * 4 + 3) * D + 4 * n4 - 1, 4LL * M * D)) return;
     const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)r * D);
     float4 *ur = RESID ? reinterpret_cast<float4 *>(u + (size_t)r * D) : nullptr;
     const float4 *hr = RESID ? reinterpret_cast<const float4 *>(S + ((size_t)r * 4 + 3) * D) : nullptr;
@@ -108,6 +113,7 @@ __global__ void __launch_bounds__(NORM_ROWS * 32) norm_bwd_kernel(const float *v
     const int lane = threadIdx.x & 31;
     if (r >= M) return;
     const int n4 = D >> 2;
+    if (!SLSTM_IN((size_t)r * D + 4 * n4 - 1, (long long)M * D)) return;   // the row's last element
     const float4 *vr = reinterpret_cast<const float4 *>(v + (size_t)r * D);
     float4 *dr = reinterpret_cast<float4 *>(dz_c + (size_t)r * D);
     const float4 *br = reinterpret_cast<const float4 *>(base + (size_t)r * D);
@@ -163,6 +169,7 @@ __global__ void __launch_bounds__(256) swiglu_bwd_pair_kernel(const float *__res
     const long long m = q / F;
     const int f = (int)(q - m * F);
     const long long cg = m * 2 * F + (f >> 5) * 64 + (f & 31);
+    if (!SLSTM_IN(cg + 32, 2 * total)) return;   // the up column of the pair (F a multiple of 32)
     const float g = gv[cg], u = gv[cg + 32], d = da[q];
     const float sg = __fdividef(1.0f, 1.0f + __expf(-g));
     const float silu = g * sg;
@@ -186,8 +193,10 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const float *__rest
     const int r0 = blockIdx.y * rows_per_chunk;
     const int r1 = min(M, r0 + rows_per_chunk);
     float acc = 0.0f;
-    for (int r = r0; r < r1; ++r) acc += c[(size_t)r * D + i];
-    partial[(size_t)blockIdx.y * D + i] = acc;
+    for (int r = r0; r < r1; ++r)
+        if (SLSTM_IN((size_t)r * D + i, (long long)M * D)) acc += c[(size_t)r * D + i];
+    if (SLSTM_IN((size_t)blockIdx.y * D + i, ((long long)(M + rows_per_chunk - 1) / rows_per_chunk) * D))
+        partial[(size_t)blockIdx.y * D + i] = acc;
 }
 
 __global__ void __launch_bounds__(256) colsum_final_kernel(const float *__restrict__ partial, int n_chunks, int D,

@@ -19,6 +19,8 @@
 #include <cuda_bf16.h>
 #include <string.h>
 
+#define SLSTM_FILE_ID 7
+#include "checked.cuh"
 #include "common.cuh"
 #include "launchers.h"
 #include "stop_rule.cuh"
@@ -35,6 +37,7 @@ struct HeadArgs {
     const float *s0;    // (B, 4, d) or null
     float *S;           // (B, T, 4, d)
     int B, T, d, dh, H;
+    long long n_ps, n_s0;   // elements of P (and S), of s0 (checked build)
     StopRule rule;
 };
 
@@ -45,7 +48,8 @@ SLSTM_DEVINL void load_rows(const float *Rh, int H, int dh, int hd, int lane, fl
     for (int g = 0; g < 4; ++g)
 #pragma unroll
         for (int k = 0; k < MAXDH; ++k)
-            r[g][k] = (lane < dh && k < dh) ? __ldg(Rh + (((size_t)g * H + hd) * dh + lane) * dh + k) : 0.0f;
+            r[g][k] = (lane < dh && k < dh && SLSTM_IN((((size_t)g * H + hd) * dh + lane) * dh + k, 4LL * H * dh * dh))
+                          ? __ldg(Rh + (((size_t)g * H + hd) * dh + lane) * dh + k) : 0.0f;
 }
 
 // This lane's R columns: c[g][i] = Rh[g][hd][i][lane], zero past d_head.
@@ -55,7 +59,8 @@ SLSTM_DEVINL void load_cols(const float *Rh, int H, int dh, int hd, int lane, fl
     for (int g = 0; g < 4; ++g)
 #pragma unroll
         for (int i = 0; i < MAXDH; ++i)
-            c[g][i] = (lane < dh && i < dh) ? __ldg(Rh + (((size_t)g * H + hd) * dh + i) * dh + lane) : 0.0f;
+            c[g][i] = (lane < dh && i < dh && SLSTM_IN((((size_t)g * H + hd) * dh + i) * dh + lane, 4LL * H * dh * dh))
+                          ? __ldg(Rh + (((size_t)g * H + hd) * dh + i) * dh + lane) : 0.0f;
 }
 
 // out[g] = sum_k r[g][k] v_k, v_k = lane k's v (lanes past d_head hold 0).
@@ -94,15 +99,18 @@ SLSTM_DEVINL void gT_mul(const CellG &g, const float l[4], float out[4])
     out[3] = g.gho * l[3];
 }
 
-SLSTM_DEVINL void load4(const float *p, size_t stride, bool ok, float v[4])
+// base, n: the buffer p points into and its element count (checked build).
+SLSTM_DEVINL void load4(const float *p, size_t stride, bool ok, float v[4], const float *base, long long n)
 {
+    ok = ok && SLSTM_PIN(p + 3 * stride, base, n);
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e] = ok ? __ldg(p + e * stride) : 0.0f;
 }
 
 // The same through the coherent path, for an array this kernel also writes.
-SLSTM_DEVINL void load4_rw(const float *p, size_t stride, bool ok, float v[4])
+SLSTM_DEVINL void load4_rw(const float *p, size_t stride, bool ok, float v[4], const float *base, long long n)
 {
+    ok = ok && SLSTM_PIN(p + 3 * stride, base, n);
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e] = ok ? p[e * stride] : 0.0f;
 }
@@ -121,14 +129,14 @@ __global__ void __launch_bounds__(HW * 32) head_seq_kernel(HeadArgs a)
     float r[4][MAXDH];
     load_rows(a.Rh, a.H, a.dh, hd, lane, r);
     float s[4];
-    load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, s);
+    load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, s, a.s0, a.n_s0);
     const float *pp = a.P + (size_t)b * a.T * 4 * d + j;
     float *sp = a.S + (size_t)b * a.T * 4 * d + j;
     float p[4];
-    load4(pp, d, jv, p);
+    load4(pp, d, jv, p, a.P, a.n_ps);
     for (int t = 0; t < a.T; ++t) {
         float pn[4];
-        load4(pp + (size_t)(t + 1) * 4 * d, d, jv && t + 1 < a.T, pn);   // next step's inputs, ahead
+        load4(pp + (size_t)(t + 1) * 4 * d, d, jv && t + 1 < a.T, pn, a.P, a.n_ps);   // next step's inputs, ahead
         float m4[4];
         mix(r, jv ? s[3] : 0.0f, m4);
         Cell c;
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(HW * 32) head_seq_kernel(HeadArgs a)
         s[1] = c.n;
         s[2] = c.m;
         s[3] = c.h;
-        if (jv) {
+        if (jv && SLSTM_PIN(sp + (size_t)t * 4 * d + 3 * d, a.S, a.n_ps)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) sp[(size_t)t * 4 * d + e * d] = s[e];
         }
@@ -168,19 +176,19 @@ __global__ void __launch_bounds__(HW * 32) head_newton_kernel(HeadArgs a, int k)
         float r[4][MAXDH];
         load_rows(a.Rh, a.H, a.dh, hd, lane, r);
         float so_p[4], sn_p[4], dl[4] = {0.f, 0.f, 0.f, 0.f};
-        load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, so_p);
+        load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, so_p, a.s0, a.n_s0);
 #pragma unroll
         for (int e = 0; e < 4; ++e) sn_p[e] = so_p[e];
         const float *pp = a.P + (size_t)b * a.T * 4 * d + j;
         float *sp = a.S + (size_t)b * a.T * 4 * d + j;
         float p[4], so[4];
-        load4(pp, d, jv, p);
-        load4_rw(sp, d, jv && !FIRST, so);
+        load4(pp, d, jv, p, a.P, a.n_ps);
+        load4_rw(sp, d, jv && !FIRST, so, a.S, a.n_ps);
         for (int t = 0; t < a.T; ++t) {
             // next step's inputs, ahead (S at t + 1 is not written before it is read here)
             float pn[4], son[4];
-            load4(pp + (size_t)(t + 1) * 4 * d, d, jv && t + 1 < a.T, pn);
-            load4_rw(sp + (size_t)(t + 1) * 4 * d, d, jv && !FIRST && t + 1 < a.T, son);
+            load4(pp + (size_t)(t + 1) * 4 * d, d, jv && t + 1 < a.T, pn, a.P, a.n_ps);
+            load4_rw(sp + (size_t)(t + 1) * 4 * d, d, jv && !FIRST && t + 1 < a.T, son, a.S, a.n_ps);
             // f, Jl and G at the old iterate
             float mo[4];
             mix(r, jv ? so_p[3] : 0.0f, mo);
@@ -197,7 +205,7 @@ __global__ void __launch_bounds__(HW * 32) head_newton_kernel(HeadArgs a, int k)
             jac_mul_add(c, dl, f4, sn);
 #pragma unroll
             for (int e = 0; e < 4; ++e) dl[e] = sn[e] - so[e];
-            if (jv) {
+            if (jv && SLSTM_PIN(sp + (size_t)t * 4 * d + 3 * d, a.S, a.n_ps)) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sp[(size_t)t * 4 * d + e * d] = sn[e];
             }
@@ -275,11 +283,13 @@ __global__ void __launch_bounds__(HW * 32) head_preact_kernel(HeadArgs a, float 
     const size_t row0 = (size_t)b * a.T;
     for (int t = t0; t < t1; ++t) {
         float hp;
-        if (t == 0) hp = (a.s0 && jv) ? __ldg(a.s0 + ((size_t)b * 4 + 3) * d + j) : 0.0f;
-        else hp = jv ? __ldg(a.S + ((row0 + t - 1) * 4 + 3) * d + j) : 0.0f;
+        if (t == 0) hp = (a.s0 && jv && SLSTM_IN(((size_t)b * 4 + 3) * d + j, a.n_s0))
+                             ? __ldg(a.s0 + ((size_t)b * 4 + 3) * d + j) : 0.0f;
+        else hp = (jv && SLSTM_IN(((row0 + t - 1) * 4 + 3) * d + j, a.n_ps))
+                      ? __ldg(a.S + ((row0 + t - 1) * 4 + 3) * d + j) : 0.0f;
         float m4[4];
         mix(r, hp, m4);
-        if (jv) {
+        if (jv && SLSTM_IN(((row0 + t) * 4 + 3) * d + j, a.n_ps)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) A[((row0 + t) * 4 + e) * d + j] = __ldg(a.P + ((row0 + t) * 4 + e) * d + j) + m4[e];
         }
@@ -319,11 +329,11 @@ __global__ void __launch_bounds__(HW * 32) head_adjoint_kernel(HeadArgs a, const
             for (int g = 0; g < 4; ++g) rt = fmaf(rc[g][i], __shfl_sync(0xffffffffu, dp1[g], i), rt);
         }
         jacT_mul(j1, lam[0], lam[1], lam[2], lam[3]);
-        lam[3] += rt + (jv ? __ldg(dH + (row0 + t) * d + j) : 0.0f);
+        lam[3] += rt + ((jv && SLSTM_IN((row0 + t) * d + j, a.n_ps / 4)) ? __ldg(dH + (row0 + t) * d + j) : 0.0f);
         float sp[4], av[4];
-        if (t == 0) load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, sp);
-        else load4(a.S + (row0 + t - 1) * 4 * d + j, d, jv, sp);
-        load4(A + (row0 + t) * 4 * d + j, d, jv, av);
+        if (t == 0) load4(a.s0 + (size_t)b * 4 * d + j, d, a.s0 && jv, sp, a.s0, a.n_s0);
+        else load4(a.S + (row0 + t - 1) * 4 * d + j, d, jv, sp, a.S, a.n_ps);
+        load4(A + (row0 + t) * 4 * d + j, d, jv, av, A, a.n_ps);
         Cell c;
         CellG gg;
         cell_eval<FORGET, true, true>(sp[0], sp[1], sp[2], sp[3], av[0], av[1], av[2], av[3], 0.f, 0.f, 0.f, 0.f, c,
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(HW * 32) head_adjoint_kernel(HeadArgs a, const
 #pragma unroll
             for (int e = 0; e < 4; ++e) dp[e] = 0.0f;
         }
-        if (jv) {
+        if (jv && SLSTM_IN((row0 + t) * 4 * d + 3 * d + j, a.n_ps)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) dP[(row0 + t) * 4 * d + e * d + j] = dp[e];
         }
@@ -351,7 +361,7 @@ __global__ void __launch_bounds__(HW * 32) head_adjoint_kernel(HeadArgs a, const
         }
         jacT_mul(j1, lam[0], lam[1], lam[2], lam[3]);
         lam[3] += rt;
-        if (jv) {
+        if (jv && SLSTM_IN(((size_t)b * 4 + 3) * d + j, a.n_s0)) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) ds0[((size_t)b * 4 + e) * d + j] = lam[e];
         }
@@ -392,11 +402,13 @@ __global__ void __launch_bounds__(256) head_dr_partial_kernel(HeadArgs a, const 
             if (row < r1 && i < dh) {
                 const size_t jj = (size_t)hd * dh + i;
                 if (e < 4) {
-                    v = __ldg(dP + ((size_t)row * 4 + e) * d + jj);
+                    if (SLSTM_IN(((size_t)row * 4 + e) * d + jj, a.n_ps)) v = __ldg(dP + ((size_t)row * 4 + e) * d + jj);
                 } else {
                     const long long b = row / a.T, t = row - b * a.T;
-                    if (t > 0) v = __ldg(a.S + (((size_t)row - 1) * 4 + 3) * d + jj);
-                    else if (a.s0) v = __ldg(a.s0 + ((size_t)b * 4 + 3) * d + jj);
+                    if (t > 0 && SLSTM_IN((((size_t)row - 1) * 4 + 3) * d + jj, a.n_ps))
+                        v = __ldg(a.S + (((size_t)row - 1) * 4 + 3) * d + jj);
+                    else if (t == 0 && a.s0 && SLSTM_IN(((size_t)b * 4 + 3) * d + jj, a.n_s0))
+                        v = __ldg(a.s0 + ((size_t)b * 4 + 3) * d + jj);
                 }
             }
             if (e < 4) s_dp[rr][e][i] = v;
@@ -475,6 +487,8 @@ HeadArgs head_args(const float *P, const float *Rh, const float *s0, float *S, i
     a.d = d;
     a.dh = dh;
     a.H = d / dh;
+    a.n_ps = (long long)B * T * 4 * d;
+    a.n_s0 = (long long)B * 4 * d;
     return a;
 }
 

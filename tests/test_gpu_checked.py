@@ -94,6 +94,44 @@ def test_checked_build_runs_clean_packed(cuda_device):
         assert st[0] == 0, _describe(lib, st)
 
 
+@pytest.mark.parametrize("B,T,d,dh", [(2, 70, 36, 12), (1, 33, 64, 32), (3, 5, 8, 1)])
+def test_checked_build_runs_clean_head(B, T, d, dh, cuda_device):
+    with _lib.checked_library() as lib:
+        assert lib.slstm_check_clear() == _lib.SLSTM_OK
+        w, dev = _dense_case(B, T, 16, d, "f32", "sigmoid", 11)
+        g = torch.Generator().manual_seed(12)
+        Rh = ((torch.rand(4, d // dh, dh, dh, generator=g) * 2 - 1) * (0.5 / dh ** 0.5)).cuda()
+        P = api.preact_gemm(dev["x"], dev["Wx"], dev["bias"])
+        api.sequential_step_head(P, Rh, dev["s0"])
+        S, _ = api.newton_forward_head(P, Rh, dev["s0"], max_iters=16, tol=1e-5)
+        api.newton_forward_head(P, Rh, None, max_iters=3, fixed=True, init="zero")
+        api.newton_backward_head(dev["x"], dev["Wx"], P, Rh, dev["s0"], S, dev["dH"])
+        st = _status(lib)
+        assert st[0] == 0, _describe(lib, st)
+
+
+@pytest.mark.parametrize("B,T,D,F", [(2, 40, 64, 256), (1, 33, 96, 384)])
+def test_checked_build_runs_clean_block(B, T, D, F, cuda_device):
+    with _lib.checked_library() as lib:
+        assert lib.slstm_check_clear() == _lib.SLSTM_OK
+        g = torch.Generator().manual_seed(21)
+        x = torch.randn(B, T, D, generator=g).cuda()
+        w1 = (torch.rand(D, generator=g) + 0.5).cuda()
+        w2 = (torch.rand(D, generator=g) + 0.5).cuda()
+        Wx = (torch.randn(4 * D, D, generator=g) * D ** -0.5).to(torch.bfloat16).cuda()
+        bias = torch.zeros(4, D).cuda()
+        R = ((torch.rand(4, D, generator=g) * 2 - 1) * 0.5).cuda()
+        Wg = (torch.randn(F, D, generator=g) * D ** -0.5).to(torch.bfloat16)
+        Wu = (torch.randn(F, D, generator=g) * D ** -0.5).to(torch.bfloat16)
+        W_gu = api.interleave_gate_up(Wg, Wu).contiguous().cuda()
+        Wd = (torch.randn(D, F, generator=g) * F ** -0.5).to(torch.bfloat16).cuda()
+        y, S, _ = api.block_forward(x, w1, Wx, bias, R, w2, W_gu, Wd, max_iters=32, tol=1e-6)
+        dY = torch.randn(B, T, D, generator=g).cuda()
+        api.block_backward(x, w1, Wx, bias, R, w2, W_gu, Wd, S, dY)
+        st = _status(lib)
+        assert st[0] == 0, _describe(lib, st)
+
+
 def test_checked_build_reports_a_planted_violation(cuda_device):
     """debug_fault = 2: the checked build checks each iteration's last tile
     boundary store against an extent one element short, so every iteration

@@ -113,3 +113,29 @@ def test_head_backward_matches_oracle(B, T, d, dh, forget, dtype, cuda_device):
         got = as_f64(out[k].cpu())
         err = np.abs(got - ref[rk]).max() / (1 + np.abs(ref[rk]).max())
         assert err <= tol, (k, err)
+
+
+@pytest.mark.parametrize("forget,dtype", [("sigmoid", "bf16"), ("exp", "f32")])
+def test_head_newton_long_sequence_sampled_heads(forget, dtype, cuda_device):
+    """A long sequence (T = 4096, 8 heads of 32): the converged GPU solve
+    against the oracle's sequential trajectory of two sampled heads over every
+    step (the heads are independent, so the oracle runs each alone)."""
+    B, T, d, dh = 2, 4096, 256, 32
+    w = Workload("head_long", B, T, 64, d, dtype, forget, 0.5, 17, 1e-5, 16)
+    inp = make_inputs(w, with_dH=False)
+    g = torch.Generator().manual_seed(18)
+    H = d // dh
+    Rh = (torch.rand(4, H, dh, dh, generator=g) * 2 - 1) * (0.5 / dh ** 0.5)
+    P = api.preact_gemm(inp["x"].cuda(), inp["Wx"].cuda(), inp["bias"].cuda())
+    S, st = api.newton_forward_head(P, Rh.cuda(), inp["s0"].cuda(), forget=forget, max_iters=16, tol=1e-5)
+    s = api.read_stats(st)
+    print("gpu", s["iters"], s["max_scaled_F"])
+    assert s["converged"] and not s["diverged"] and s["error"] == 0, s
+    Pref = oracle.preact(as_f64(inp["x"]), as_f64(inp["Wx"]), as_f64(inp["bias"]))
+    S_gpu = as_f64(S.cpu())
+    tol = 5e-3 if dtype == "bf16" else 1e-4
+    for hd in (1, H - 1):
+        cols = slice(hd * dh, (hd + 1) * dh)
+        ref = oracle.sequential_head(Pref[:, :, :, cols], as_f64(Rh[:, hd:hd + 1]), as_f64(inp["s0"])[:, :, cols],
+                                     forget)
+        assert _h_err(S_gpu[:, :, :, cols], ref) <= tol, (hd, _h_err(S_gpu[:, :, :, cols], ref))
