@@ -562,7 +562,7 @@ def run_gpu(args, w):
         "dtype": "f32", "operand_dtype": "bf16 x/W_x, fp32 state and scans" if w.dtype == "bf16" else "f32",
         "data": "synthetic",
         "config": dict(w.describe(), newton_mode=args.newton_mode, newton_max_iters=K, newton_init="decoupled",
-                       guess_sweeps=args.guess_sweeps,
+                       guess_sweeps=args.guess_sweeps, gemm_tiles=args.gemm_tiles,
                        l2="inputs larger than L2 (P and S are %.2f GB each)" % (elems * 16 / 1e9),
                        parallelism=f"replicas x{ws}"),
         "fwd": {"value": aggregate(elems, ws, fwd_ms), "unit": UNIT, "ms_per_step": fwd_ms},
@@ -1048,6 +1048,7 @@ def run_block(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "operand_dtype": "bf16 GEMM operands, fp32 accumulation, state and residual stream", "data": "synthetic",
             "config": {"workload": f"{w.name}_block", "B": B, "T": T, "d_model": D, "d_ff": F, "forget": w.forget,
+                       "gemm_tiles": args.gemm_tiles,
                        "newton_max_iters": K, "newton_mode": args.newton_mode, "newton_iters": st["iters"],
                        "converged": st["converged"], "error": st["error"],
                        "l2": "inputs larger than L2"},
@@ -1148,6 +1149,9 @@ def main(argv=None):
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="ncu dram read+write bytes per Newton launch, when captured for this build")
+    ap.add_argument("--gemm-tiles", default="auto", choices=["auto", "pair", "single"],
+                    help="tile shape of the tensor-core GEMMs: auto (the library default: SM pairs for the gradient GEMMs), "
+                         "256 x 256 on SM pairs, or 128 x 256 per SM")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="run the workload with T shortened to this length (small cases for ncu "
                          "captures; the bench line then names the shortened workload)")
@@ -1164,6 +1168,9 @@ def main(argv=None):
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={ws}")
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.gemm_tiles != "auto":
+        from nonlinear_rnn_pararnn_b200 import api
+        api.set_gemm_tiles(args.gemm_tiles)
     if args.mode == "scan":
         return run_scan(args)
     if args.mode == "varlen":

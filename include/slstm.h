@@ -284,6 +284,28 @@ int slstm_preact_gemm(const void *x, const void *Wx, int dtype, const float *bia
                       slstm_stream_t stream);
 
 /*
+ * Tile shape of every tensor-core (bf16) GEMM of the library: the input
+ * projection, the gradient GEMMs and the trunk layer's GEMMs.
+ *   SLSTM_GEMM_TILES_PAIR: 256 x 256 tiles of C on a pair of SMs (a cluster
+ *     of two CTAs, tcgen05 cta_group::2); each SM stages its own 128 rows of
+ *     A and 128 rows of B, and the pair's tensor cores read both.
+ *   SLSTM_GEMM_TILES_SINGLE: 128 x 256 tiles, one CTA per SM.
+ *   SLSTM_GEMM_TILES_AUTO (the default): SM pairs for the products whose
+ *     work items span at least 4096 of K and only store C (the gradient
+ *     GEMMs), single SMs for the others, whose output stream the pair's
+ *     shared accumulator hand-off slows (the input projection, the trunk
+ *     layer's forward GEMMs).
+ * Where clusters of two cannot run, single-SM tiles are used.  Process-wide
+ * setting (not synchronised with calls in flight on other host threads).
+ * Both shapes compute the same fp32-accumulated products; the input
+ * projection is identical bit for bit, while the gradient GEMMs may round
+ * differently (their split-K counts follow the tile shape).  Returns the
+ * previous setting, or -1 (and changes nothing) for another value.
+ */
+typedef enum { SLSTM_GEMM_TILES_AUTO = 0, SLSTM_GEMM_TILES_PAIR = 1, SLSTM_GEMM_TILES_SINGLE = 2 } slstm_gemm_tiles;
+int slstm_set_gemm_tiles(int tiles);
+
+/*
  * Newton solve of the whole trajectory ("sLSTM in this library", "Cell";
  * "pararnn-torch structure", "Current surface"):
  *   initial guess as cfg->init selects; s0 enters as the step before t = 0;

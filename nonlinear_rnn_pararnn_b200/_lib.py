@@ -43,6 +43,9 @@ SLSTM_RESIDUAL_SCALED = 0
 SLSTM_RESIDUAL_RAW = 1
 SLSTM_HISTORY_BOUND = 0
 SLSTM_HISTORY_EXACT = 1
+SLSTM_GEMM_TILES_AUTO = 0
+SLSTM_GEMM_TILES_PAIR = 1
+SLSTM_GEMM_TILES_SINGLE = 2
 SLSTM_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -69,6 +72,7 @@ SIGNATURES = {
     "slstm_check_site_file": (ctypes.c_char_p, [_I]),
     "slstm_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "slstm_preact_gemm": (_I, [_V, _V, _I, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
+    "slstm_set_gemm_tiles": (_I, [_I]),
     "slstm_newton_forward": (_I, [_V, _V, _V, _V, ctypes.POINTER(NewtonConfig), _V, _I, _I, _I, _V, _Z, _V]),
     "scan_block4": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V, _Z, _V]),
     "scan_block4_noalloc": (_I, [_V, _V, _V, _V, _I, _I, _I, _I, _V]),

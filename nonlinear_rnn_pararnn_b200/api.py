@@ -78,6 +78,21 @@ _RESIDUAL = {"scaled": _lib.SLSTM_RESIDUAL_SCALED, "raw": _lib.SLSTM_RESIDUAL_RA
 DEFAULT_GUESS_SWEEPS = 2
 
 
+def set_gemm_tiles(tiles: str) -> str:
+    """Tile shape of the tensor-core GEMMs: "auto" (the default: SM pairs for
+    the gradient GEMMs, whose work items span K >= 4096, single SMs for the
+    others), "pair"
+    (256 x 256 tiles on a pair of SMs) or "single" (128 x 256 per SM); returns
+    the previous one.  The shapes agree to fp32 rounding (the input projection
+    bit for bit)."""
+    codes = {"auto": _lib.SLSTM_GEMM_TILES_AUTO, "pair": _lib.SLSTM_GEMM_TILES_PAIR,
+             "single": _lib.SLSTM_GEMM_TILES_SINGLE}
+    if tiles not in codes:
+        raise ValueError(f"tiles must be 'auto', 'pair' or 'single', got {tiles!r}")
+    prev = load().slstm_set_gemm_tiles(codes[tiles])
+    return {v: k for k, v in codes.items()}[prev]
+
+
 def newton_config(max_iters: int, fixed: bool, tol: float, forget, debug_fault: int = 0, wait_limit_us: int = 0,
                   carry_mode: int = 0, init="decoupled", residual_mode="scaled",
                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False) -> NewtonConfig:

@@ -650,12 +650,14 @@ struct Layout {
 long long round8(long long v) { return (v + 7) & ~7LL; }
 
 // split-K count of the W_x-gradient GEMM: the count (up to 16) whose work
-// items fill whole waves of the persistent CTAs best; a larger count only
+// items fill whole waves of the persistent CTAs (or CTA pairs) best; a larger count only
 // when it fills them at least 2% better (each split adds an M x N partial).
 int wgrad_splits(int B, int T, int d_in, int d_h)
 {
-    const long long tiles = ((4LL * d_h + 127) / 128) * ((d_in + 255) / 256);
-    const long long sms = sm_count_bwd();
+    int rows = 128, units = 148;
+    gemm_tc_waves(&rows, &units);
+    const long long tiles = ((4LL * d_h + rows - 1) / rows) * ((d_in + 255) / 256);
+    const long long sms = units;
     int best = 1;
     double best_eff = 0.0;
     for (int want = 1; want <= 16; ++want) {

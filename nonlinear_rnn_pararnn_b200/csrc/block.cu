@@ -230,14 +230,12 @@ struct BlockBwdLayout {
 
 // split-K count of a weight-gradient GEMM (M x N output, K = B*T rows, two A
 // parts): the count (up to 16) whose work items fill whole waves of the
-// persistent CTAs (128 x 256 output tiles) best.
+// persistent CTAs or CTA pairs (128 x 256 or 256 x 256 output tiles) best.
 int block_wgrad_splits(int M, int N, int K)
 {
-    const long long tiles = ((long long)(M + 127) / 128) * ((N + 255) / 256);
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
-                                                   cudaSuccess || sms < 1)
-        sms = 148;
+    int rows = 128, sms = 148;
+    gemm_tc_waves(&rows, &sms);
+    const long long tiles = ((long long)(M + rows - 1) / rows) * ((N + 255) / 256);
     int best = 1;
     double best_eff = 0.0;
     for (int want = 1; want <= 16; ++want) {

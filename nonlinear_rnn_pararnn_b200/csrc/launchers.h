@@ -138,6 +138,13 @@ cudaError_t gemm_tc_bf16_ex(const void *A0, const void *A1, int lda, bool a_mn, 
                             cudaStream_t st);
 // The split count gemm_tc_bf16_ex will actually use for a request of `want`.
 int gemm_tc_splits(int M, int N, int K, int a_parts, int want);
+// The tile shape of the tensor-core GEMMs (SLSTM_GEMM_TILES_*); returns the
+// previous one, or -1 for an unknown value.
+int gemm_tc_set_tiles(int tiles);
+// Rows of C per work item of a split-K product (256 on SM pairs, 128 on
+// single SMs; 256 columns either way) and the work items that run at once
+// (clusters, or SMs).
+void gemm_tc_waves(int *tile_rows, int *units);
 // out[i] = sum over z in order of part[z * n + i] (split-K partial sums).
 cudaError_t sum_splits(const float *part, float *out, long long n, int splits, cudaStream_t st);
 

@@ -200,6 +200,8 @@ int slstm_preact_gemm(const void *x, const void *Wx, int dtype, const float *bia
                                      static_cast<cudaStream_t>(stream)));
 }
 
+int slstm_set_gemm_tiles(int tiles) { return gemm_tc_set_tiles(tiles); }
+
 int slstm_newton_forward(const float *P, const float *R, const float *s0, float *S,
                          const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
                          int d_h, void *ws, size_t ws_bytes, slstm_stream_t stream)

@@ -8,7 +8,7 @@ import re
 
 import pytest
 
-from nonlinear_rnn_pararnn_b200 import _lib
+from nonlinear_rnn_pararnn_b200 import _lib, api
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER_DIR = os.path.join(ROOT, "include")
@@ -247,3 +247,21 @@ def test_interleave_gate_up_layout():
         assert torch.equal(W[64 * k + 32:64 * k + 64], Wu[32 * k:32 * k + 32])
     with pytest.raises(ValueError):
         api.interleave_gate_up(Wg[:40], Wu[:40])
+
+
+def test_gemm_tile_shape_switch():
+    """slstm_set_gemm_tiles takes the three settings, returns the previous one
+    and refuses anything else without changing the setting (no GPU work)."""
+    lib = _lib.load()
+    prev = lib.slstm_set_gemm_tiles(_lib.SLSTM_GEMM_TILES_SINGLE)
+    assert prev in (_lib.SLSTM_GEMM_TILES_AUTO, _lib.SLSTM_GEMM_TILES_PAIR, _lib.SLSTM_GEMM_TILES_SINGLE)
+    assert lib.slstm_set_gemm_tiles(7) == -1
+    assert lib.slstm_set_gemm_tiles(-1) == -1
+    assert lib.slstm_set_gemm_tiles(_lib.SLSTM_GEMM_TILES_PAIR) == _lib.SLSTM_GEMM_TILES_SINGLE
+    assert lib.slstm_set_gemm_tiles(_lib.SLSTM_GEMM_TILES_AUTO) == _lib.SLSTM_GEMM_TILES_PAIR
+    assert api.set_gemm_tiles("single") == "auto"
+    assert api.set_gemm_tiles("pair") == "single"
+    assert api.set_gemm_tiles("auto") == "pair"
+    with pytest.raises(ValueError):
+        api.set_gemm_tiles("quad")
+    lib.slstm_set_gemm_tiles(prev)
