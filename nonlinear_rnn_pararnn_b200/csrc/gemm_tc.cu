@@ -476,11 +476,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 //              remotely) once accumulator b is drained.
 // No TMA load names another CTA's memory or another GPU's; no multicast.
 // ---------------------------------------------------------------------------
-constexpr int STAGES2 = 5;
+constexpr int STAGES2 = 6;
 constexpr int BNH = BN / 2;                               // rows of B per CTA
 constexpr uint32_t B_HALF = BNH * BK * 2;                 // 16 KB
 constexpr uint32_t STAGE2_BYTES = A_STAGE + B_HALF;       // 32 KB per CTA and stage
-constexpr int STORE_BUFS2 = 8;                            // staging buffers: up to seven stores still reading
+constexpr int STORE_BUFS2 = 4;                            // staging buffers: up to three stores still reading
 constexpr int SMEM2_BYTES = STAGES2 * STAGE2_BYTES + STORE_BUFS2 * STORE_BYTES + 1024 + 256;
 static_assert(SMEM2_BYTES <= 227 * 1024, "pair-tile shared memory");
 
