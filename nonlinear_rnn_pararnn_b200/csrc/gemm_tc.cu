@@ -59,6 +59,13 @@ struct TcArgs {
     const float *res;       // GEMM_EPI_RESIDUAL: C = acc + res, res [M][N] (may be C)
 };
 
+// At most N of this thread's bulk store groups still read shared memory.
+template <int N>
+SLSTM_DEVINL void bulk_wait_read_n()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
 // Named barrier with an OR reduction over `n` threads: every participant
 // gets the same answer.
 SLSTM_DEVINL bool bar_or(int id, int n, bool v)

@@ -118,12 +118,6 @@ SLSTM_DEVINL void tma_store_2d(const CUtensorMap *map, const void *src, int c0, 
 SLSTM_DEVINL void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // At most three of this thread's bulk store groups still read shared memory.
 SLSTM_DEVINL void bulk_wait_read_3() { asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); }
-// At most N of this thread's bulk store groups still read shared memory.
-template <int N>
-SLSTM_DEVINL void bulk_wait_read_n()
-{
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
 
 SLSTM_DEVINL void tma_store_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 SLSTM_DEVINL void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
