@@ -741,13 +741,16 @@ __global__ void __launch_bounds__(NW * 32, 1) guess_kernel(Args a, int k, const 
                 seg_load(sm, w, f, x, ((whead >> w) & 1u) != 0u);
 #pragma unroll
                 for (int off = 1; off < NW; off *= 2) {
+                    // the composition keeps the later run's output gate, so
+                    // the earlier run's is not moved; dense sequences hold no
+                    // start, so no head flag is either
                     Seg y;
                     y.A = __shfl_up_sync(0xffffffffu, x.A, off, 16);
                     y.mu = __shfl_up_sync(0xffffffffu, x.mu, off, 16);
                     y.u = __shfl_up_sync(0xffffffffu, x.u, off, 16);
                     y.v = __shfl_up_sync(0xffffffffu, x.v, off, 16);
-                    y.o = __shfl_up_sync(0xffffffffu, x.o, off, 16);
-                    y.head = __shfl_up_sync(0xffffffffu, x.head ? 1 : 0, off, 16) != 0;
+                    y.o = 0.0f;
+                    y.head = VARLEN && __shfl_up_sync(0xffffffffu, x.head ? 1 : 0, off, 16) != 0;
                     if (w >= off) seg_compose(x, y, x);
                 }
                 seg_store(sm, w, f, x);
