@@ -455,7 +455,9 @@ SLSTM_DEVINL float carry_chain4(const MapArr *m, CinArr *cin, float c, int warp,
         const float v1 = __shfl_sync(0xffffffffu, c, 8 + i8);
         const float v2 = __shfl_sync(0xffffffffu, c, 16 + i8);
         const float v3 = __shfl_sync(0xffffffffu, c, 24 + i8);
-        const float nc = fmaf(a[3], v3, fmaf(a[2], v2, fmaf(a[1], v1, fmaf(a[0], v0, a[4]))));
+        // two FMA chains of depth two joined by an add: one level less on
+        // the chain's critical path than a single chain of four
+        const float nc = fmaf(a[1], v1, fmaf(a[0], v0, a[4])) + fmaf(a[3], v3, a[2] * v2);
         c = ((whead >> w) & 1u) ? a[4] : nc;
     }
     return c;
