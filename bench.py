@@ -1071,7 +1071,7 @@ def run_block(args, w):
 # SHA-256; any other build reports traffic null.  Traffic per element does not depend on T (every
 # tile moves the same bytes), so it scales to a full launch by the element count.
 NEWTON_TRAFFIC = {"sources_sha256": "6049c6905d4f1fb894f77be44de5ac782a5c6031f35fb1ac5de701415a587d24",
-                  "guess": 30.9, "sweep": None, "iter": 46.5}
+                  "guess": 31.1, "sweep": None, "iter": 46.4}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
