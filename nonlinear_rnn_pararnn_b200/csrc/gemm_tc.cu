@@ -471,8 +471,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 // B (the two halves of the tile's N range) into its shared memory, the pair's
 // tensor cores read both, and each CTA's TMEM holds the accumulator of its
 // 128 rows x 256 columns.  Per CTA and k-block the ring holds 32 KB instead
-// of 48 (the other half of B sits in the peer), which leaves room for a
-// deeper ring and more epilogue staging buffers than the single-SM kernel.
+// of 48 (the other half of B sits in the peer), so it is six stages deep
+// (the single-SM kernel's is four) beside the same four staging buffers.
 // Synchronisation, all through mbarriers:
 //   full[s]    leader's: both CTAs' loads of stage s complete their bytes on
 //              it (the leader arms it with both CTAs' byte counts);
