@@ -1103,7 +1103,7 @@ def solve_bytes_per_elem(iters: int, sweeps: int) -> int:
 
 def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
     """Measured DRAM bytes of one Newton solve (the guess, its sweeps and
-    `iters` iterations), or None when the counters are not for this build."""
+    `iters` iterations), or None when the counters were taken on other kernel sources."""
     t = NEWTON_TRAFFIC
     if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
         return None
@@ -1114,7 +1114,7 @@ def newton_traffic_bytes(elems: int, iters: int, sweeps: int):
 
 def newton_iter_traffic_bytes(elems: int):
     """Measured DRAM bytes of one newton_iter launch, or None when the
-    counters are not for this build."""
+    counters were taken on other kernel sources."""
     t = NEWTON_TRAFFIC
     if t["sources_sha256"] is None or newton_sources_sha256() != t["sources_sha256"]:
         return None
@@ -1148,7 +1148,7 @@ def main(argv=None):
     ap.add_argument("--head-dim", type=int, default=32, help="d_head of --mode head (1 .. 32, dividing d_h)")
     ap.add_argument("--scan-T", default="4096,16384,65536")
     ap.add_argument("--traffic-bytes", type=float, default=None,
-                    help="ncu dram read+write bytes per Newton launch, when captured for this build")
+                    help="ncu dram read+write bytes per Newton launch, when captured for the current kernel sources")
     ap.add_argument("--gemm-tiles", default="auto", choices=["auto", "pair", "single"],
                     help="tile shape of the tensor-core GEMMs: auto (the library default: SM pairs for the gradient GEMMs), "
                          "256 x 256 on SM pairs, or 128 x 256 per SM")

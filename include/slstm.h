@@ -77,7 +77,7 @@ typedef enum {
     SLSTM_ERR_CUDA = 2,
     SLSTM_ERR_DIVERGED = 3,    /* stats.error only: max|F| > 1 or non-finite */
     SLSTM_ERR_TIMEOUT = 4,     /* stats.error only: a bounded wait ran out   */
-    SLSTM_ERR_UNSUPPORTED = 5  /* valid request this build cannot run        */
+    SLSTM_ERR_UNSUPPORTED = 5  /* valid request the library cannot run       */
 } slstm_status;
 
 typedef enum { SLSTM_F32 = 0, SLSTM_BF16 = 1 } slstm_dtype;
