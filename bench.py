@@ -1068,7 +1068,7 @@ def run_block(args, w):
 # capture of the training workload shortened to T = 2048 (summarised under profiles/): the guess
 # launch (the guess and two sweeps fused), a separate sweep launch (not captured: None) and a Newton
 # iteration that evaluates its whole residual.  The counters describe the kernel sources with this
-# SHA-256; any other build reports traffic null.  Traffic per element does not depend on T (every
+# SHA-256; other sources report traffic null.  Traffic per element does not depend on T (every
 # tile moves the same bytes), so it scales to a full launch by the element count.
 NEWTON_TRAFFIC = {"sources_sha256": "6049c6905d4f1fb894f77be44de5ac782a5c6031f35fb1ac5de701415a587d24",
                   "guess": 31.1, "sweep": None, "iter": 46.4}
