@@ -349,7 +349,7 @@ def run_gpu(args, w):
 
     dev_main = {"x": x, "Wx": Wx, "R": R, "bias": bias, "s0": s0, "dH": dH}
 
-    n_launch = guess_launches(args.guess_sweeps) + K   # launches of work of one Newton call
+    n_launch = newton_launches(args.guess_sweeps, K, tol_mode)   # launches of work of one Newton call
 
     def step(ev=None, dv=None, gr=None, lev=None):
         dv = dev_main if dv is None else dv
@@ -497,12 +497,14 @@ def run_gpu(args, w):
     newton_bytes = elems * solve_bytes_per_elem(n_it, sw)
     solve_gbs = newton_bytes / (newton_ms / 1e3) / 1e9
     # Per launch, from the library's events: the guess launch(es), then the
-    # iterations that did work (the later launches of a converged call return
-    # at once and are listed apart).
+    # iterations launched one by one (in tolerance mode the first LOOP_FROM;
+    # the rest of the cap is one launch that loops on the device and ends with
+    # the solve, listed apart with whatever iterations it ran).
     g = guess_launches(sw)
-    per_it = [float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs])) for i in range(n_it)]
+    n_sep = separate_iterations(n_it, tol_mode)
+    per_it = [float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs])) for i in range(n_sep)]
     guess_ms = [lv[0].elapsed_time(lv[g]) for lv in levs]
-    idle_ms = [lv[g + n_it].elapsed_time(lv[n_launch]) for lv in levs]
+    idle_ms = [lv[g + n_sep].elapsed_time(lv[-1]) for lv in levs]
     per_it = max_over_ranks(per_it, device=dev) if per_it else []
     it_ms = float(np.mean(per_it)) if per_it else 0.0
     guess_ms, idle_ms = max_over_ranks([float(np.mean(guess_ms)), float(np.mean(idle_ms))], device=dev)
@@ -514,14 +516,15 @@ def run_gpu(args, w):
     roofline = {"kernel": "newton_iter", "bound": "hbm", "achieved": achieved, "peak": hbm, "peak_kind": peak_kind,
                 "unit": "GB/s", "frac": achieved / hbm, "traffic": traffic,
                 "algorithmic_bytes_per_launch": 48 * elems, "avg_launch_ms": it_ms,
-                "launches_per_step": n_it, "launch_ms": per_it,
+                "launches_per_step": n_sep, "launch_ms": per_it,
                 "timing": "CUDA events the library records on its stream around each launch, over the timed steps",
                 "guess_kernel": {"launches_per_step": g, "ms": guess_ms, "algorithmic_bytes": guess_bytes,
                                  "achieved": guess_bytes / (guess_ms / 1e3) / 1e9,
                                  "frac": guess_bytes / (guess_ms / 1e3) / 1e9 / hbm,
                                  "stages_per_tile": 1 + min(sw, GUESS_FUSED_SWEEPS),
                                  "note": "one scan per stage over each tile; issue-bound"},
-                "converged_launches": {"per_step": n_launch - g - n_it, "ms": idle_ms},
+                "device_loop": {"launches_per_step": n_launch - g - n_sep, "iterations_inside": n_it - n_sep,
+                                "ms": idle_ms, "note": "the rest of the iteration cap, one launch looping on the device"},
                 "solve": {"ms": newton_ms, "algorithmic_bytes": newton_bytes, "achieved": solve_gbs,
                           "frac": solve_gbs / hbm}}
 
@@ -549,12 +552,11 @@ def run_gpu(args, w):
         torch.cuda.empty_cache()
         extra["scan_block4_sweep"] = scan_sweep(args, dev, hbm, peak_kind)
 
-    # kernels launched per step: preact GEMM 1, Newton: the guess + K iteration
-    # launches (in tolerance mode those after convergence exit at once),
-    # backward: adjoint 1 + dR/db reduction 1 + 2 GEMMs (+ the split-K sum of
-    # the tensor-core path)
-    launches_per_step = (1 + guess_launches(args.guess_sweeps) + K +
-                         (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0)))
+    # kernels launched per step: preact GEMM 1, Newton: the guess, the
+    # iterations launched one by one and (tolerance mode) the device loop over
+    # the rest of the cap, backward: adjoint 1 + dR/db reduction 1 + 2 GEMMs
+    # (+ the split-K sum of the tensor-core path)
+    launches_per_step = (1 + n_launch + (0 if forward_only else 4 + (1 if w.dtype == "bf16" else 0)))
     line = {
         "metric": METRIC_FWD if forward_only else METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup,
@@ -662,7 +664,8 @@ def long_forward(args, dev, hbm, peak_kind):
         it = st["iters"]
         nbytes = w.elems * solve_bytes_per_elem(it, args.guess_sweeps)
         gbs = nbytes / (newton_ms / 1e3) / 1e9
-        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs for i in range(it)]))
+        n_sep = separate_iterations(it, mode == "tol")
+        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs for i in range(n_sep)]))
         guess_ms = float(np.mean([lv[0].elapsed_time(lv[g]) for lv in levs]))
         it_gbs = 48.0 * w.elems / (it_ms / 1e3) / 1e9
         out[mode] = {"newton_mode": mode, "max_iters": K, "iters": it, "guess_sweeps": args.guess_sweeps,
@@ -713,7 +716,8 @@ def newton_sweep(args, dev, hbm, peak_kind, T_list=(4096, 16384)):
         st = api.read_stats(stats)
         it = st["iters"]
         solve_ms = float(np.median([lv[0].elapsed_time(lv[-1]) for lv in levs]))
-        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs for i in range(it)]))
+        it_ms = float(np.mean([lv[g + i].elapsed_time(lv[g + i + 1]) for lv in levs
+                               for i in range(separate_iterations(it, True))]))
         gbs = 48.0 * w.elems / (it_ms / 1e3) / 1e9
         out.append({"workload": w.name, "T": T, "iters": it, "converged": st["converged"],
                     "solve_ms": solve_ms, "solve_elems_per_s": w.elems / (solve_ms / 1e3),
@@ -1058,7 +1062,7 @@ def run_block(args, w):
                          "tensor_peak_tflops": tflops, "tensor_peak_kind": tkind, "hbm_gbs": hbm,
                          "hbm_peak_kind": peak_kind, "algorithmic_bytes_per_step": nbytes},
             "clocks": clocks,
-            "gpu_launches": (6 + K + 20) * args.steps}
+            "gpu_launches": (5 + newton_launches(args.guess_sweeps, K, tol_mode) + 20) * args.steps}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
@@ -1091,6 +1095,22 @@ GUESS_FUSED_SWEEPS = 3
 
 def guess_launches(sweeps: int) -> int:
     return 1 + max(0, sweeps - GUESS_FUSED_SWEEPS)
+
+
+# Tolerance mode with the fused carry: the library launches the first
+# LOOP_FROM iterations one by one (slstm_newton_config.loop_from, its default)
+# and the rest of the cap as one launch that loops on the device.
+LOOP_FROM = 2
+
+
+def newton_launches(sweeps: int, K: int, tol_mode: bool) -> int:
+    """Launches of work of one Newton call (fused carry)."""
+    return guess_launches(sweeps) + (LOOP_FROM + 1 if tol_mode and K > LOOP_FROM else K)
+
+
+def separate_iterations(iters: int, tol_mode: bool) -> int:
+    """How many of a call's iterations ran as launches of their own."""
+    return min(iters, LOOP_FROM) if tol_mode else iters
 
 
 def solve_bytes_per_elem(iters: int, sweeps: int) -> int:

@@ -56,7 +56,8 @@
  *     (cleared by every call), the same word of the library's own block for
  *     scan_block4_noalloc (not readable by the caller; the NaN outputs show
  *     it).  slstm_newton_forward also reports it as SLSTM_ERR_TIMEOUT in its
- *     stats.
+ *     stats (with the bit 4 of the same word at byte offset 4 of its
+ *     workspace when the wait was a grid barrier of its device loop).
  *   - Sizes: 1 <= B <= 65535, 1 <= T, 1 <= d_in, d_h, d <= 2^20, B*T < 2^31
  *     and B * ceil(T/32) * ceil(max(d_in, d_h)/32) < 2^31.
  */
@@ -123,7 +124,10 @@ typedef enum {
  *               bounds-checked build, each iteration checks its last tile
  *               boundary store against an extent one element short (the
  *               store is skipped and reported; a self-test of the checks);
- *               ignored in the normal build.
+ *               ignored in the normal build.  3: the device loop (loop_from)
+ *               loses one CTA before its first grid barrier, whose wait then
+ *               expires in the others (SLSTM_ERR_TIMEOUT in stats.error; a
+ *               self-test of the bounded barrier).
  *   wait_limit_us  upper bound of one bounded wait, in microseconds
  *               (0 = the default of 2 seconds).
  *   carry_mode  how a tile gets the scan carry entering it (same results up
@@ -181,10 +185,25 @@ typedef enum {
  *               further sweep; none for SLSTM_INIT_ZERO, a small copy kernel
  *               for SLSTM_INIT_GIVEN), then one per iteration up to max_iters
  *               (with the two-pass carry an iteration's three kernels count as
- *               one); launches after the stop return at once but are still
- *               bracketed.  Timing only: results do not depend on them.
+ *               one; the device loop below counts as one launch); launches
+ *               after the stop return at once but are still bracketed.  The
+ *               events past the last launch's are all recorded after it, so
+ *               events[n_events - 1] marks the end of the call whatever the
+ *               number of launches.  Timing only: results do not depend on
+ *               them.
  *               slstm_newton_forward and slstm_newton_forward_varlen only.
+ *   loop_from   tolerance mode with the fused carry: the iterations from
+ *               this one on (counting from 0) run inside one cooperative
+ *               launch that loops on the device, a grid-wide barrier between
+ *               two iterations, and ends as soon as the stopping rule does,
+ *               so a converged solve does not pay for the rest of its cap.
+ *               0: SLSTM_DEFAULT_LOOP_FROM; negative: never (one launch per
+ *               iteration).  The earlier iterations, the fixed mode, the
+ *               two-pass carry and calls on a stream being captured into a
+ *               graph keep one launch per iteration.  Results do not depend
+ *               on it.
  */
+#define SLSTM_DEFAULT_LOOP_FROM 2
 typedef enum { SLSTM_CARRY_AUTO = 0, SLSTM_CARRY_FUSED = 1, SLSTM_CARRY_TWO_PASS = 2 } slstm_carry_mode;
 
 typedef enum { SLSTM_INIT_DECOUPLED = 0, SLSTM_INIT_ZERO = 1, SLSTM_INIT_GIVEN = 2 } slstm_init;
@@ -207,6 +226,7 @@ typedef struct {
     int history;
     int n_events;
     void *const *events;
+    int loop_from;
 } slstm_newton_config;
 
 /*

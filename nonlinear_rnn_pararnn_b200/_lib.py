@@ -43,6 +43,7 @@ SLSTM_RESIDUAL_SCALED = 0
 SLSTM_RESIDUAL_RAW = 1
 SLSTM_HISTORY_BOUND = 0
 SLSTM_HISTORY_EXACT = 1
+SLSTM_DEFAULT_LOOP_FROM = 2
 SLSTM_GEMM_TILES_AUTO = 0
 SLSTM_GEMM_TILES_PAIR = 1
 SLSTM_GEMM_TILES_SINGLE = 2
@@ -54,7 +55,7 @@ class NewtonConfig(ctypes.Structure):
                 ("forget", ctypes.c_int), ("debug_fault", ctypes.c_int), ("wait_limit_us", ctypes.c_int),
                 ("carry_mode", ctypes.c_int), ("init", ctypes.c_int), ("residual_mode", ctypes.c_int),
                 ("guess_sweeps", ctypes.c_int), ("history", ctypes.c_int), ("n_events", ctypes.c_int),
-                ("events", ctypes.c_void_p)]
+                ("events", ctypes.c_void_p), ("loop_from", ctypes.c_int)]
 
 
 STATS_BYTES = 4 * 4 + 2 * 4 * SLSTM_STATS_HISTORY + 2 * 4

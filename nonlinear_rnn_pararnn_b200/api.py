@@ -95,19 +95,22 @@ def set_gemm_tiles(tiles: str) -> str:
 
 def newton_config(max_iters: int, fixed: bool, tol: float, forget, debug_fault: int = 0, wait_limit_us: int = 0,
                   carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                  guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False) -> NewtonConfig:
+                  guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False,
+                  loop_from: int = 0) -> NewtonConfig:
     """The C ABI's slstm_newton_config.  init: "decoupled" (default; with
     guess_sweeps refinement sweeps), "zero" or "given" (S holds the guess on
     entry); residual_mode: "scaled" or "raw"; events: optional list of
     torch.cuda.Event (timing enabled) recorded before each launch of work and
     after the last (see slstm.h); exact_history: every iteration records its
     exact residual (else an iteration that fails the test may record a lower
-    bound)."""
+    bound); loop_from: in tolerance mode, the iterations from this one on run
+    in one launch that loops on the device (0: the library default, negative:
+    never)."""
     cfg = NewtonConfig(int(max_iters), 1 if fixed else 0, float(tol), forget_code(forget), int(debug_fault),
                        int(wait_limit_us), int(carry_mode), _INIT[init] if isinstance(init, str) else int(init),
                        _RESIDUAL[residual_mode] if isinstance(residual_mode, str) else int(residual_mode),
                        int(guess_sweeps), _lib.SLSTM_HISTORY_EXACT if exact_history else _lib.SLSTM_HISTORY_BOUND,
-                       0, None)
+                       0, None, int(loop_from))
     if events:
         handles = []
         for ev in events:
@@ -144,11 +147,12 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
                    max_iters: int = 8, fixed: bool = False, tol: float = 1e-5, S: torch.Tensor = None,
                    stats: torch.Tensor = None, ws: torch.Tensor = None, debug_fault: int = 0,
                    wait_limit_us: int = 0, carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False):
+                   guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False,
+                   loop_from: int = 0):
     """Newton solve; returns (S, stats) with stats a device record (see read_stats).
     With init="given", S must be passed and holds the initial guess.  events:
-    optional torch.cuda.Event list bracketing the launches; exact_history:
-    see newton_config."""
+    optional torch.cuda.Event list bracketing the launches; exact_history,
+    loop_from: see newton_config."""
     B, T, four, d_h = P.shape
     _need(P, "P", (B, T, 4, d_h))
     _need(R, "R", (4, d_h))
@@ -164,7 +168,7 @@ def newton_forward(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor = None, *,
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD, B, T, 0, d_h, P.device)
     cfg = newton_config(max_iters, fixed, tol, forget, debug_fault, wait_limit_us, carry_mode, init, residual_mode,
-                        guess_sweeps, events, exact_history)
+                        guess_sweeps, events, exact_history, loop_from)
     check("slstm_newton_forward", load().slstm_newton_forward(_ptr(P), _ptr(R), _ptr(s0), _ptr(S),
                                                               ctypes.byref(cfg), _ptr(stats), B, T, d_h,
                                                               _ptr(ws), ws.numel(), _stream()))
@@ -283,10 +287,11 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
                           forget="sigmoid", max_iters: int = 8, fixed: bool = False, tol: float = 1e-5,
                           S: torch.Tensor = None, stats: torch.Tensor = None, ws: torch.Tensor = None,
                           carry_mode: int = 0, init="decoupled", residual_mode="scaled",
-                          guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False):
+                          guess_sweeps: int = DEFAULT_GUESS_SWEEPS, events=None, exact_history: bool = False,
+                          loop_from: int = 0):
     """Newton solve of packed sequences: P (total_T, 4, d_h), s0 (n_seq, 4, d_h) or None,
     cu_seqlens int32 (n_seq + 1,) exclusive-prefix offsets; returns (S, stats).
-    events, exact_history: as newton_forward."""
+    events, exact_history, loop_from: as newton_forward."""
     total_T, four, d_h = P.shape
     n_seq = cu_seqlens.numel() - 1
     _need(P, "P", (total_T, 4, d_h))
@@ -302,7 +307,7 @@ def newton_forward_varlen(P: torch.Tensor, R: torch.Tensor, s0: torch.Tensor, cu
     if ws is None:
         ws = workspace(_lib.SLSTM_OP_NEWTON_FORWARD_VARLEN, n_seq, total_T, 0, d_h, P.device)
     cfg = newton_config(max_iters, fixed, tol, forget, 0, 0, carry_mode, init, residual_mode, guess_sweeps, events,
-                        exact_history)
+                        exact_history, loop_from)
     check("slstm_newton_forward_varlen", load().slstm_newton_forward_varlen(
         _ptr(P), _ptr(R), _ptr(s0), _ptr(cu_seqlens), n_seq, _ptr(S), ctypes.byref(cfg), _ptr(stats), total_T, d_h,
         _ptr(ws), ws.numel(), _stream()))

@@ -25,7 +25,8 @@ struct NewtonCtrl {
     unsigned error;
     unsigned init_raw;      // residual of the initial guess (float bits), recorded by the first iteration
     unsigned init_scaled;
-    unsigned pad[12];
+    unsigned gbar;          // grid-barrier arrivals of the device loop over iterations
+    unsigned pad[11];
     NewtonSlot slot[2];
 };
 

@@ -88,10 +88,24 @@ struct Args {
     int exact_hist;     // every iteration evaluates its whole residual (else a failed test ends that work)
     int guess_tested;   // the first iteration records the residual of the guess
     int check_plant;    // checked build: one bounds check made to fail on purpose (a self-test)
+    int loop_from;      // tolerance mode, fused carry: iterations from this one on loop on the device (0: never)
+    int loop_fault;     // self-test: CTA 0 of the device loop leaves before its first grid barrier
     float tol;
     long long n_s0;     // elements of s0 (and of s0h)
     FastDiv div_groups, div_gpr;   // by n_groups and by groups_per_row
 };
+
+// Launch k of a solve: epoch k + 1; it reads the boundary buffer launch
+// k - 1 wrote and writes the other one.  (On the device: the iterations of
+// newton_iter_loop.)
+__host__ __device__ inline Args launch_args(const Args &base, int k)
+{
+    Args a = base;
+    a.epoch = (unsigned)(k + 1);
+    a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
+    a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
+    return a;
+}
 
 // Element counts of the buffers that Args names, for the guards of the
 // checked build.
@@ -937,8 +951,15 @@ __global__ void gather_boundaries(Args a)
 // the sequence's s0 and the Jacobian is zero, which makes the scan segmented.
 // GRS: the first iteration from the decoupled guess also records the
 // guess's residual (tolerance mode).
+// One iteration (launch k of the solve) over every tile; newton_iter runs one
+// per launch, newton_iter_loop several in one launch.  The TMA stages'
+// mbarriers are initialised once per launch (bars_ready false: this body does
+// it) and never again, since re-initialising a live mbarrier is not allowed;
+// tiles_done, the tiles this CTA has taken in earlier bodies of the launch,
+// carries their phases from one body to the next.
 template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE, bool GRS>
-__global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
+SLSTM_DEVINL void newton_iter_body(const Args &a, int k, const NewtonMaps &maps, unsigned &tiles_done,
+                                   bool &bars_ready)
 {
     extern __shared__ unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
@@ -954,11 +975,12 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
             decode_tile(a, MODE == MODE_AGG ? blockIdx.x + gridDim.x : atomicAdd(&slot.ticket, 1u), sm.info[1]);
         }
     }
-    if (TMA && threadIdx.x == TMA_THREAD) {
+    if (TMA && !bars_ready && threadIdx.x == TMA_THREAD) {
         mbar_init(&sm.bar[0], 1);
         mbar_init(&sm.bar[1], 1);
         mbar_init_fence();
     }
+    bars_ready = true;
     __syncthreads();
     if (sm.exit_flag) return;
 
@@ -981,13 +1003,14 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     // registers have no room for the second copy of walk B.
     const bool may_skip = TMA && !VARLEN && RESID && !a.exact_hist && (k + 1 - a.k0 < a.max_iters);
 
-    int ring = 0, st = 0;
-    unsigned it = 0;       // tiles done by this CTA; stage it & 1, TMA phase (it >> 1) & 1
+    unsigned it = tiles_done;   // tiles done by this CTA in the launch; stage it & 1, TMA phase (it >> 1) & 1
+    const unsigned it0 = it;
+    int ring = 0, st = (int)(it & 1u);
     bool tma_ok = true;    // false after a TMA wait expired: no further waits
     if (TMA) {
-        if (threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, 0, sm.info[0], !FIRST);
+        if (threadIdx.x == TMA_THREAD) issue_tile_load(a, maps, sm, st, sm.info[0], !FIRST);
     } else {
-        prefetch_tile(a, sm, 0, sm.info[0], toff, !FIRST);
+        prefetch_tile(a, sm, st, sm.info[0], toff, !FIRST);
         cp_async_commit();
     }
 
@@ -999,7 +1022,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
         // decode it into the ring at the end of this tile
         unsigned after = 0;
         if (threadIdx.x == 0) {
-            after = MODE == MODE_AGG ? blockIdx.x + (it + 2u) * gridDim.x : atomicAdd(&slot.ticket, 1u);
+            after = MODE == MODE_AGG ? blockIdx.x + (it - it0 + 2u) * gridDim.x : atomicAdd(&slot.ticket, 1u);
             if (may_skip) sm.resid_skip = (int)*(volatile unsigned *)&slot.failed;
         }
         if (TMA) {
@@ -1317,6 +1340,7 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     } else {
         cp_async_wait_all();
     }
+    tiles_done = it;
     if constexpr (MODE == MODE_AGG) return;   // the iteration itself is the APPLY launch
 
     if (RESID) {
@@ -1355,6 +1379,72 @@ __global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, c
     }
 }
 
+template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE, bool GRS>
+__global__ void __launch_bounds__(NW * 32, 16 / NW) newton_iter(Args a, int k, const __grid_constant__ NewtonMaps maps)
+{
+    unsigned tiles = 0;
+    bool bars = false;
+    newton_iter_body<FORGET, FIRST, RESID, TMA, VARLEN, MODE, GRS>(a, k, maps, tiles, bars);
+}
+
+// Every CTA of the launch arrives at the counter, which then reaches `target`
+// (arrivals accumulate over the launch's barriers); true once it has, false
+// when the wait ran out (bit 4 of the error word, the stats record's error set
+// to SLSTM_ERR_TIMEOUT and the solve marked done).  The launch must be
+// cooperative, so that every CTA is resident.
+SLSTM_DEVINL bool grid_barrier(const Args &a, unsigned target)
+{
+    bool ok = true;
+    // this CTA's TMA stores of S (async proxy, waited for) ordered before the
+    // arrival, and the TMA loads of the next iteration after the barrier
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();   // this CTA's writes of the iteration (and the finaliser's) before the arrival
+        atomicAdd(&a.ctrl->gbar, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        unsigned polls = 0;
+        while (ld_acquire(&a.ctrl->gbar) < target) {
+            if (++polls > 8) __nanosleep(128);
+            if (globaltimer_ns() - t0 > a.wait_ns) {
+                atomicOr(a.error, 4u);
+                if (a.stats) atomicExch(&a.stats->error, (int)SLSTM_ERR_TIMEOUT);
+                atomicExch(&a.ctrl->done, 1u);
+                ok = false;
+                break;
+            }
+        }
+    }
+    const bool all = !__syncthreads_or(!ok);
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return all;
+}
+
+// Launches k_begin .. k_end - 1 of a tolerance-mode solve with the fused
+// carry, in one cooperative launch: each iteration is newton_iter_body, and a
+// grid-wide barrier between two iterations stands in for the launch
+// boundary (the iteration's finaliser has reset the next control slot and
+// decided whether the solve is done).  The loop ends as soon as the
+// stopping rule has, so a converged solve costs one short launch for the
+// rest of its iteration cap.  debug_fault 3: CTA 0 leaves before the first
+// barrier, whose wait then runs out in every other CTA.
+template <int FORGET, bool TMA, bool VARLEN>
+__global__ void __launch_bounds__(NW * 32, 16 / NW)
+    newton_iter_loop(Args base, int k_begin, int k_end, const __grid_constant__ NewtonMaps maps)
+{
+    unsigned tiles = 0;   // this CTA's tiles so far: the TMA stages' phases
+    bool bars = false;
+    for (int k = k_begin; k < k_end; ++k) {
+        if (k > k_begin) {
+            if (base.loop_fault && blockIdx.x == 0) return;
+            if (!grid_barrier(base, (unsigned)(k - k_begin) * gridDim.x)) return;
+            if (*(volatile unsigned *)&base.ctrl->done) return;
+        }
+        newton_iter_body<FORGET, false, true, TMA, VARLEN, MODE_FUSED, false>(launch_args(base, k), k, maps, tiles,
+                                                                              bars);
+    }
+}
+
 template <int FORGET, bool FIRST, bool RESID, bool TMA, bool VARLEN, int MODE, bool GRS = false>
 cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaStream_t st)
 {
@@ -1370,6 +1460,59 @@ cudaError_t launch_one(const Args &a, const NewtonMaps &m, int k, int sms, cudaS
     const int grid = min(a.n_tiles, sms * blocks_per_sm);
     kern<<<grid, NW * 32, SMEM_BYTES, st>>>(a, k, m);
     return cudaGetLastError();
+}
+
+// Launches k_begin .. k_end - 1 as one cooperative newton_iter_loop launch
+// (every CTA resident, which its grid barriers need).
+template <int FORGET, bool TMA, bool VARLEN>
+cudaError_t launch_loop(const Args &a, const NewtonMaps &m, int k_begin, int k_end, int sms, cudaStream_t st)
+{
+    auto kern = newton_iter_loop<FORGET, TMA, VARLEN>;
+    static int blocks_per_sm = 0;
+    if (blocks_per_sm == 0) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        int b = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, NW * 32, SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        if (b < 1) return cudaErrorInvalidConfiguration;
+        blocks_per_sm = b;
+    }
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.gridDim = dim3((unsigned)min(a.n_tiles, sms * blocks_per_sm), 1, 1);
+    cfg.blockDim = dim3(NW * 32, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, k_begin, k_end, m);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Whether newton_iter_loop can run on `st`: the device takes cooperative
+// launches and the stream is not being captured into a graph (a captured
+// call keeps one launch per iteration).
+bool device_loop_ok(cudaStream_t st)
+{
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    if (cs != cudaStreamCaptureStatusNone) return false;
+    static int coop = -1;
+    if (coop < 0) {
+        int dev = 0, v = 0;
+        coop = (cudaGetDevice(&dev) == cudaSuccess &&
+                cudaDeviceGetAttribute(&v, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && v != 0)
+                   ? 1
+                   : 0;
+    }
+    return coop == 1;
 }
 
 template <int FORGET, bool TMA, bool VARLEN, int MODE>
@@ -1406,16 +1549,6 @@ cudaError_t launch_guess(const Args &a, const NewtonMaps &m, int k, int sms, cud
     return launch_guess_ns<FORGET, 1, SWEEP, TMA, VARLEN>(a, m, k, sms, st);
 }
 
-// Launch k of a solve: epoch k + 1; it reads the boundary buffer launch
-// k - 1 wrote and writes the other one.
-inline Args launch_args(const Args &base, int k)
-{
-    Args a = base;
-    a.epoch = (unsigned)(k + 1);
-    a.bnd_in = (k & 1) ? base.bnd_out : base.bnd_in;
-    a.bnd_out = (k & 1) ? base.bnd_in : base.bnd_out;
-    return a;
-}
 
 // Guess launches of a solve with `sweeps` refinement sweeps: launch 0 runs
 // the decoupled guess and the first GUESS_STAGES - 1 sweeps tile by tile;
@@ -1431,6 +1564,13 @@ struct LaunchEvents {
         const int i = next++;
         if (i >= n || ev[i] == nullptr) return cudaSuccess;
         return cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), st);
+    }
+    // after the last launch: this and every remaining event mark the end
+    cudaError_t finish(cudaStream_t st)
+    {
+        cudaError_t e = cudaSuccess;
+        while (e == cudaSuccess && next < n) e = record(st);
+        return e == cudaSuccess ? record(st) : e;
     }
 };
 
@@ -1475,7 +1615,13 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         gather_boundaries<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(base);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    for (int k = base.k0; k < base.k0 + max_iters; ++k) {
+    // in tolerance mode with the fused carry, the iterations from loop_from
+    // on run inside one cooperative launch that stops with the solve
+    const int k_end = base.k0 + max_iters;
+    const int loop_at = (!fixed && !two_pass && base.loop_from > 0 && base.loop_from < max_iters && device_loop_ok(st))
+                            ? base.k0 + base.loop_from
+                            : k_end;
+    for (int k = base.k0; k < loop_at; ++k) {
         const Args a = launch_args(base, k);
         const bool resid = !fixed || (k + 1 - base.k0 == max_iters);
         cudaError_t e = le.record(st);
@@ -1492,7 +1638,12 @@ cudaError_t launch_iters(const Args &base, const NewtonMaps &m, int max_iters, b
         }
         if (e != cudaSuccess) return e;
     }
-    return le.record(st);
+    if (loop_at < k_end) {
+        cudaError_t e = le.record(st);
+        if (e != cudaSuccess) return e;
+        if ((e = launch_loop<FORGET, TMA, VARLEN>(base, m, loop_at, k_end, sms, st)) != cudaSuccess) return e;
+    }
+    return le.finish(st);
 }
 
 struct Layout {
@@ -1602,6 +1753,8 @@ cudaError_t prepare(const float *P, const float *R, const float *s0, float *S, c
     // so the first tile of chunk 2 has nothing to wait for
     a.fault_ticket = (cfg.debug_fault == 1 && l.n_chunks >= 3) ? l.n_groups : -1;
     a.check_plant = cfg.debug_fault == 2 ? 1 : 0;
+    a.loop_fault = cfg.debug_fault == 3 ? 1 : 0;
+    a.loop_from = cfg.loop_from < 0 ? 0 : (cfg.loop_from == 0 ? SLSTM_DEFAULT_LOOP_FROM : cfg.loop_from);
     a.n_s0 = (long long)(vl ? vl->n_seq : B) * 4 * d;
 
     // control block, aggregate flags and the epoch tags of the inclusive

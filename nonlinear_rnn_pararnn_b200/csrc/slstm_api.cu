@@ -54,7 +54,7 @@ bool config_ok(const slstm_newton_config &c)
     if (c.residual_mode != SLSTM_RESIDUAL_SCALED && c.residual_mode != SLSTM_RESIDUAL_RAW) return false;
     if (c.n_events < 0 || (c.n_events > 0 && c.events == nullptr)) return false;
     if (c.history != SLSTM_HISTORY_BOUND && c.history != SLSTM_HISTORY_EXACT) return false;
-    if (c.debug_fault < 0 || c.debug_fault > 2) return false;
+    if (c.debug_fault < 0 || c.debug_fault > 3) return false;
     return c.carry_mode >= SLSTM_CARRY_AUTO && c.carry_mode <= SLSTM_CARRY_TWO_PASS;
 }
 

@@ -112,7 +112,7 @@ def test_newton_forward_rejects_bad_arguments():
     assert call(cfg=_cfg(n_events=-1)) == E
     assert call(cfg=_cfg(n_events=3)) == E               # timing events announced, array missing
     assert call(cfg=_cfg(history=2)) == E
-    assert call(cfg=_cfg(debug_fault=3)) == E
+    assert call(cfg=_cfg(debug_fault=4)) == E
     assert call(wb=ctypes.c_size_t(16)) == E          # workspace too small
     assert call(w=ctypes.c_void_p(0x10010)) == E      # workspace not 256-aligned
     assert lib.slstm_newton_forward(FAKE, FAKE, NULL, FAKE, None, FAKE, 2, 64, 8, ws, big, NULL) == E

@@ -127,19 +127,22 @@ def _check_status_against_oracle(st, ost):
     return False
 
 
-@pytest.mark.parametrize("sweeps,carry_mode", [(2, 1), (5, 1), (2, 2)])
-def test_newton_launch_events_bracket_every_launch(sweeps, carry_mode, cuda_device):
+@pytest.mark.parametrize("sweeps,carry_mode,loop_from", [(2, 1, -1), (5, 1, -1), (2, 2, -1), (2, 1, 0), (5, 1, 3)])
+def test_newton_launch_events_bracket_every_launch(sweeps, carry_mode, loop_from, cuda_device):
     """The optional timing events: one before each launch of work (the guess
-    launches, then one per iteration) and one after the last; the solution
-    is that of the same call without them (up to the rounding order of the
-    decoupled look-back, which depends on timing: a tile's carry comes from
-    its predecessor's published state or from composing earlier runs)."""
+    launches, then one per iteration, or the device loop over the rest of
+    the cap as one launch) and one after the last, the events past it
+    recorded there too; the solution is that of the same call without them
+    (up to the rounding order of the decoupled look-back, which depends on
+    timing: a tile's carry comes from its predecessor's published state or
+    from composing earlier runs)."""
     w = scaled(WORKLOADS["slstm_f32_b8_t1024_d256"], B=2, T=300, d_in=64, d_h=64)
     inp = make_inputs(w, with_dH=False)
     P = api.preact_gemm(_dev(inp["x"]), _dev(inp["Wx"]), _dev(inp["bias"]))
     R, s0 = _dev(inp["R"]), _dev(inp["s0"])
     K = 6
-    kw = dict(forget=w.forget, max_iters=K, fixed=False, tol=w.tol, carry_mode=carry_mode, guess_sweeps=sweeps)
+    kw = dict(forget=w.forget, max_iters=K, fixed=False, tol=w.tol, carry_mode=carry_mode, guess_sweeps=sweeps,
+              loop_from=loop_from)
     S_ref, st_ref = api.newton_forward(P, R, s0, **kw)
     g = 1 + max(0, sweeps - 3)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(g + K + 1)]
@@ -154,6 +157,10 @@ def test_newton_launch_events_bracket_every_launch(sweeps, carry_mode, cuda_devi
     assert a["iters"] == b["iters"] and a["converged"] and b["converged"]
     times = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(evs) - 1)]
     assert all(t >= 0.0 for t in times), times
+    loops = carry_mode == 1 and loop_from != -1
+    n_launch = g + ((loop_from or 2) + 1 if loops else K)
+    # the events past the last launch's mark the end of the call with it
+    assert all(t <= 0.05 for t in times[n_launch:]), times
     # fewer events than launches: only the first ones are recorded
     few = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     S2, _ = api.newton_forward(P, R, s0, events=few, **kw)
