@@ -1074,7 +1074,7 @@ def run_block(args, w):
 # iteration that evaluates its whole residual.  The counters describe the kernel sources with this
 # SHA-256; other sources report traffic null.  Traffic per element does not depend on T (every
 # tile moves the same bytes), so it scales to a full launch by the element count.
-NEWTON_TRAFFIC = {"sources_sha256": "6049c6905d4f1fb894f77be44de5ac782a5c6031f35fb1ac5de701415a587d24",
+NEWTON_TRAFFIC = {"sources_sha256": "60725403a102fc65e60d077642cfd653092b1f5b85ccd2a3c71016a8c77cb7f7",
                   "guess": 31.1, "sweep": None, "iter": 46.4}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
