@@ -1075,7 +1075,7 @@ def run_block(args, w):
 # SHA-256; other sources report traffic null.  Traffic per element does not depend on T (every
 # tile moves the same bytes), so it scales to a full launch by the element count.
 NEWTON_TRAFFIC = {"sources_sha256": "60725403a102fc65e60d077642cfd653092b1f5b85ccd2a3c71016a8c77cb7f7",
-                  "guess": 31.1, "sweep": None, "iter": 46.4}
+                  "guess": 30.9, "sweep": None, "iter": 46.3}
 NEWTON_SOURCES = ("newton.cu", "lookback.cuh", "common.cuh", "tma.cuh", "launchers.h")
 
 
