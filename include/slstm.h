@@ -339,9 +339,13 @@ int slstm_set_gemm_tiles(int tiles);
  *   S     (B, T, 4, d_h) fp32 output (the last iterate; h is slot 3)
  *   cfg   host pointer, read during the call
  *   stats device pointer to one slstm_newton_stats, written on the stream
- * The call enqueues max_iters iterations; iterations after convergence (or
- * after a timeout or non-finite residual) return immediately on the device,
- * so the call never synchronises with the host.
+ * The call enqueues up to max_iters iterations without synchronising with the
+ * host: in tolerance mode the first cfg->loop_from of them as launches of
+ * their own and the rest as one launch that loops on the device and ends
+ * with the solve (see loop_from); iterations after convergence (or after a
+ * timeout or non-finite residual) do no work.  Two calls may run on one
+ * workspace only in stream order; the device loop needs every CTA of its
+ * cooperative launch resident, which the library's grid size ensures.
  */
 int slstm_newton_forward(const float *P, const float *R, const float *s0, float *S,
                          const slstm_newton_config *cfg, slstm_newton_stats *stats, int B, int T,
